@@ -1,0 +1,157 @@
+"""Pins of the oracle's indexer: exact score, ranking keys, Top-k, block-max
+pool, Full/Reindex/Reuse selection and the needle closed form (no GPU)."""
+import numpy as np
+import pytest
+
+import synth
+from tests._exact import exact_score
+
+
+def _rand_rows(rng, n, width, smin=120, smax=134):
+    codes = rng.integers(0, 256, (n, width // 2), dtype=np.uint8)
+    scales = rng.integers(smin, smax + 1, (n, width // 32), dtype=np.uint8)
+    return codes, scales
+
+
+def _rand_query(rng, smin=120, smax=134):
+    qc = rng.integers(0, 256, (4, 64), dtype=np.uint8)
+    qs = rng.integers(smin, smax + 1, (4, 4), dtype=np.uint8)
+    w = (0.5 + rng.random(4)).astype(np.float32)
+    return qc, qs, w
+
+
+def test_score_equals_exact_rational(orc):
+    rng = np.random.default_rng(10)
+    for trial in range(6):
+        smin, smax = [(120, 134), (100, 140), (125, 127)][trial % 3]
+        kc, ks = _rand_rows(rng, 24, 128, smin, smax)
+        qc, qs, w = _rand_query(rng, smin, smax)
+        got = orc.index_scores(kc, ks, np.arange(24), qc, qs, w)
+        for t in range(24):
+            want = exact_score(kc[t], ks[t], qc, qs, w)
+            assert got[t].tobytes() == want.tobytes(), (trial, t, got[t], want)
+
+
+def test_score_one_hot_weight_is_rounded_dot(orc):
+    """w = (1,0,0,0) leaves exactly d_0 = fp32(q_0 . k)."""
+    rng = np.random.default_rng(11)
+    kc, ks = _rand_rows(rng, 16, 128)
+    qc, qs, _ = _rand_query(rng)
+    w = np.array([1, 0, 0, 0], np.float32)
+    got = orc.index_scores(kc, ks, np.arange(16), qc, qs, w)
+    dk = orc.mxfp4_decode(kc, ks)
+    dq = orc.mxfp4_decode(qc, qs)
+    ref = (dk @ dq[0]).astype(np.float32)       # exact in fp64 for these scales
+    assert np.array_equal(got, ref)
+
+
+def test_rank_key_order(orc):
+    rng = np.random.default_rng(12)
+    vals = np.concatenate([rng.standard_normal(300).astype(np.float32),
+                           np.array([0.0, -0.0, 1e-45, -1e-45, np.inf, -np.inf, 3.4e38, -3.4e38], np.float32)])
+    keys = np.array([orc.rank_key(v) for v in vals], np.uint64)
+    assert orc.rank_key(-0.0) == orc.rank_key(0.0)
+    for i in range(len(vals)):
+        for j in range(0, len(vals), 7):
+            if vals[i] < vals[j]:
+                assert keys[i] < keys[j]
+            elif vals[i] == vals[j]:
+                assert keys[i] == keys[j]
+
+
+def test_topk_matches_full_sort(orc):
+    rng = np.random.default_rng(13)
+    for n, k, levels in [(1000, 64, 5), (5000, 512, 50), (300, 512, 3), (0, 8, 1), (700, 700, 2)]:
+        keys = rng.integers(0, levels, n).astype(np.uint32) * 1000 + 7
+        ids = rng.permutation(n).astype(np.int64)
+        got = orc.topk(keys, ids, k)
+        order = sorted(range(n), key=lambda i: (-int(keys[i]), int(ids[i])))[:k]
+        want = sorted(int(ids[i]) for i in order)
+        want += [-1] * (k - len(want))
+        assert got.tolist() == want
+
+
+def test_topk_all_equal_picks_lowest_positions(orc):
+    keys = np.full(4096, 12345, np.uint32)
+    got = orc.topk(keys, np.arange(4096), 512)
+    assert got.tolist() == list(range(512))
+
+
+def _brute_full(orc, kc, ks, qc, qs, w, L, P, k):
+    s = orc.index_scores(kc, ks, np.arange(L), qc, qs, w)
+    key = [orc.rank_key(v) for v in s]
+    nb = (L + 7) // 8
+    bkey = [max(key[8 * b:min(L, 8 * b + 8)]) for b in range(nb)]
+    pool = sorted(sorted(range(nb), key=lambda b: (-bkey[b], b))[:P])
+    top = sorted(sorted(range(L), key=lambda t: (-key[t], t))[:k])
+    return pool + [-1] * (P - len(pool)), top + [-1] * (k - len(top)), s
+
+
+@pytest.mark.parametrize("L,P,k", [(203, 8, 16), (64, 16, 16), (5, 4, 8), (0, 4, 4), (1000, 16, 100)])
+def test_index_full_bruteforce(orc, L, P, k):
+    rng = np.random.default_rng(L + P)
+    cap = max(L, 1) + 16
+    kc, ks = _rand_rows(rng, cap, 128, 125, 127)
+    kc[8:40] = kc[0]                                   # runs of equal scores (ties)
+    ks[8:40] = ks[0]
+    qc, qs, w = _rand_query(rng, 125, 127)
+    off = np.array([8], np.int64)
+    pool, top, sc = orc.index_full(kc, ks, qc[None], qs[None], w[None], off, np.array([L]), P, k, want_scores=True)
+    bp, bt, bs = _brute_full(orc, kc[8:], ks[8:], qc, qs, w, L, P, k)
+    assert pool[0].tolist() == bp
+    assert top[0].tolist() == bt
+    assert np.array_equal(sc[0, :L], bs)
+
+
+def test_pool_contains_full_topk_when_P_ge_k(orc):
+    """Containment: every Full Top-k position's block is in the pool when P >= k."""
+    rng = np.random.default_rng(14)
+    B, L, P, k = 3, 4096, 64, 64
+    kc, ks = _rand_rows(rng, B * L, 128, 124, 128)
+    # heavy ties: repeat a few rows everywhere
+    kc[::5] = kc[0]
+    ks[::5] = ks[0]
+    qc, qs, w = _rand_query(rng, 124, 128)
+    off = np.arange(B, dtype=np.int64) * L
+    lens = np.array([L, L - 3, 777], np.int32)
+    pool, top, _ = orc.index_full(kc, ks, np.repeat(qc[None], B, 0), np.repeat(qs[None], B, 0),
+                                  np.repeat(w[None], B, 0), off, lens, P, k)
+    for b in range(B):
+        blocks = set(pool[b][pool[b] >= 0].tolist())
+        assert all((t // 8) in blocks for t in top[b] if t >= 0)
+
+
+def test_reindex_with_full_pool_equals_full_topk(orc):
+    rng = np.random.default_rng(15)
+    L, P, k = 2000, 256, 128
+    kc, ks = _rand_rows(rng, L, 128)
+    qc, qs, w = _rand_query(rng)
+    off, lens = np.array([0], np.int64), np.array([L], np.int32)
+    pool, top, _ = orc.index_full(kc, ks, qc[None], qs[None], w[None], off, lens, P, k)
+    assert (pool[0] >= 0).sum() == 250                # all ceil(2000/8) blocks
+    re = orc.index_reindex(kc, ks, qc[None], qs[None], w[None], off, lens, pool, k)
+    assert np.array_equal(re, top)
+    # a Reindex layer with another query over a partial pool = brute force
+    qc2, qs2, w2 = _rand_query(rng)
+    part = np.full((1, P), -1, np.int32)
+    part[0, :40] = np.sort(rng.choice(250, 40, replace=False))
+    re2 = orc.index_reindex(kc, ks, qc2[None], qs2[None], w2[None], off, lens, part, k)
+    pos = [8 * b + j for b in part[0, :40] for j in range(8)]
+    s = orc.index_scores(kc, ks, np.array(pos), qc2, qs2, w2)
+    key = [orc.rank_key(v) for v in s]
+    best = sorted(sorted(range(len(pos)), key=lambda i: (-key[i], pos[i]))[:k])
+    assert re2[0].tolist() == sorted(pos[i] for i in best)
+
+
+def test_needles_always_selected(orc):
+    """Closed form: needle keys (head-0 query codes, scales +2) are in the Top-512."""
+    seed, L = 7, 8192
+    qc = synth.mxfp4_rows(seed, synth.T_QIDX_CODES, synth.T_QIDX_SCALES, 0, 0, 0, 4, 128)
+    w = synth.head_weights(seed, 0, 0)
+    kc, ks = synth.mxfp4_rows(seed, synth.T_IDXK_CODES, synth.T_IDXK_SCALES, 0, 0, 0, L, 128)
+    pos = synth.needle_positions(seed, 0, 0, L, 8)
+    nc, ns = synth.needle_rows(qc[0][0], qc[1][0], len(pos))
+    kc[pos], ks[pos] = nc, ns
+    pool, top, _ = orc.index_full(kc, ks, qc[0][None], qc[1][None], w[None], np.array([0]), np.array([L]), 256, 512)
+    assert set(pos.tolist()) <= set(top[0].tolist())
+    assert set((pos // 8).tolist()) <= set(pool[0].tolist())

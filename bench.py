@@ -1,0 +1,422 @@
+"""Benchmark of the CSA2 decode step (default: batch 64, L = 2^20, layers F R R U).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-cpu-baseline]
+
+One step = the whole hot path for one decode token per sequence: the Full
+layer's full-context FP4 scan + block-max pool + Top-512, two Reindex layers,
+one Reuse layer, and four sparse attentions (MXFP4 selection + FP8 window).
+Inputs are synthetic and already resident in HBM; the scan alone streams
+4.56 GB per step, more than L2, so no extra L2 flush is needed.  Under
+torchrun each rank runs its own batch of 64 different sequences (weak scaling,
+no data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode queries/sec at L=1M batch 64; achieved HBM GB/s as % of B200 peak"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="long_decode_b64_l1m")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def algorithmic_bytes(wl):
+    """Per step, from the method's own reads (no scratch traffic):
+    Full scan L*68 B; each pool-scored layer min(16384, 8*ceil(L/8))*68 B
+    (the Full layer re-scores its pool for its own Top-512, each Reindex layer
+    scores the pool); each attention 512*272 + 128*512 B."""
+    L = wl.lengths.astype(np.int64)
+    pooled = np.minimum(wl.P * 8, (L + 7) // 8 * 8)
+    n_scan = sum(1 for _, m in enumerate(wl.pattern) if m == "F")
+    n_pool = sum(1 for m in wl.pattern if m in "FR")
+    scan = int((L * 68).sum()) * 1  # only the first Full layer scans (default plan)
+    pool = int((pooled * 68).sum()) * n_pool
+    attn = wl.B * (wl.k * 272 + 128 * 512) * len(wl.pattern)
+    return dict(scan=scan, pool=pool, attn=attn, total=scan + pool + attn, n_full=n_scan)
+
+
+class ClockSampler:
+    """nvidia-smi clocks during the timed region (median SM MHz, reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = tempfile.mktemp(suffix=".csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# oracle timing (CPU baseline and the reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_sample_inputs(wl, layers, caches_dev, seqs):
+    """Host copies of the sampled sequences' cache rows and per-layer inputs."""
+    import torch
+
+    off = wl.row_offsets()[0]
+    out = []
+    for b in seqs:
+        o, L = int(off[b]), int(wl.lengths[b])
+        ch = [dict(idx_codes=c["idx_codes"][o:o + L].cpu().numpy(), idx_scales=c["idx_scales"][o:o + L].cpu().numpy(),
+                   main_codes=c["main_codes"][o:o + L].cpu().numpy(),
+                   main_scales=c["main_scales"][o:o + L].cpu().numpy()) for c in caches_dev]
+        lb = [{k: v[b:b + 1] for k, v in Ld.items()} for Ld in layers]
+        out.append((ch, L, lb))
+    torch.cuda.synchronize()
+    return out
+
+
+def time_oracle(wl, samples, nthreads):
+    """Runs the oracle's decode step on every sampled sequence, one thread
+    per sequence (threads in parallel); returns (seconds, sequences)."""
+    import threading
+
+    import oracle
+
+    def one(s):
+        ch, L, lb = s
+        oracle.decode_step(wl.pattern, ch, np.array([0]), np.array([L], np.int32), lb, wl.P, wl.k,
+                           1 / math.sqrt(512), nthreads=1)
+
+    t0 = time.perf_counter()
+    for i in range(0, len(samples), nthreads):
+        th = [threading.Thread(target=one, args=(s,)) for s in samples[i:i + nthreads]]
+        for t in th:
+            t.start()
+        for t in th:
+            t.join()
+    return time.perf_counter() - t0, len(samples)
+
+
+# ----------------------------------------------------------------------------
+
+def build_workload(wl, rank, device):
+    import torch
+
+    import synth.workloads as W
+    from long_context_decode_csa2_b200 import csa2 as C
+    from long_context_decode_csa2_b200.decode import FullCache
+
+    if rank:
+        wl = W.DecodeWorkload(wl.name, wl.lengths, wl.pattern, wl.P, wl.k, wl.needles, wl.lognormal,
+                              seed=wl.seed + 1000 * rank)
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    caches_dev = [W.full_cache_device(wl, f, layers[f]["q_codes"], layers[f]["q_scales"], device)
+                  for f in wl.full_layers()]
+    caches = [FullCache(C.cache(c["idx_codes"], c["idx_scales"]), C.cache(c["main_codes"], c["main_scales"]))
+              for c in caches_dev]
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+        return torch.from_numpy(a).to(device)
+
+    keys = ("q", "q_codes", "q_scales", "w", "win", "win_scale", "win_len")
+    layers_dev = [{k: to_dev(L[k]) for k in keys} for L in layers]
+    off = caches_dev[0]["seq_row_off"]
+    return wl, layers, caches_dev, caches, layers_dev, to_dev(off), to_dev(wl.lengths.astype(np.int32))
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import synth.workloads as W
+    from long_context_decode_csa2_b200 import csa2 as C
+    from long_context_decode_csa2_b200.decode import DecodeStep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
+
+    wl = W.decode_workloads()[args.workload]
+    wl, layers, caches_dev, caches, layers_dev, off_d, len_d = build_workload(wl, rank, device)
+    C.lib()
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
+    stream = torch.cuda.current_stream()
+
+    # events around every csa2_index_full call of the timed region (the
+    # dominant call: full-context scan, block max, pool, Top-512)
+    n_layers = len(wl.pattern)
+    ev_full = []
+    recording = [False]
+
+    def hook(name, phase):
+        if not recording[0] or name != "csa2_index_full":
+            return
+        if phase == "begin":
+            ev_full.append([torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)])
+            ev_full[-1][0].record(stream)
+        else:
+            ev_full[-1][1].record(stream)
+
+    step.hook = hook
+
+    def run_step(record=False):
+        recording[0] = record
+        step.run(caches, off_d, len_d, layers_dev)
+        recording[0] = False
+
+    for _ in range(args.warmup):
+        run_step()
+    torch.cuda.synchronize()
+    if step.device_flags():
+        raise RuntimeError("device status flags set during warm-up")
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            run_step(record=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    full_ms = [a.elapsed_time(b) for a, b in ev_full]
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end to end: host (pinned) query inputs -> device, step, outputs -> host
+    keys_in = ("q", "q_codes", "q_scales", "w")
+    host_in = [{k: torch.from_numpy(np.ascontiguousarray(
+        L[k].view(np.int16) if L[k].dtype == np.uint16 else L[k])).pin_memory() for k in keys_in} for L in layers]
+    h2d = sum(t.numel() * t.element_size() for L in host_in for t in L.values())
+    out_host = torch.empty(step.out.shape, dtype=torch.float32).pin_memory()
+    top_host = torch.empty((n_layers, wl.B, wl.k), dtype=torch.int32).pin_memory()
+    d2h = out_host.numel() * 4 + top_host.numel() * 4
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for l in range(n_layers):
+            for k in keys_in:
+                dst = layers_dev[l][k]
+                src = host_in[l][k]
+                (dst.view(torch.int16) if dst.dtype == torch.bfloat16 else dst).copy_(src, non_blocking=True)
+        step.run(caches, off_d, len_d, layers_dev)
+        out_host.copy_(step.out, non_blocking=True)
+        for l in range(n_layers):
+            top_host[l].copy_(step.topk[l], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    flags = step.device_flags()
+
+    ab = algorithmic_bytes(wl)
+    peak, peak_kind = measured_peaks()
+    full_avg = sum(full_ms) / len(full_ms)
+    full_bytes = ab["scan"] + ab["pool"] // max(1, sum(1 for m in wl.pattern if m in "FR"))
+    achieved = full_bytes / (full_avg * 1e-3) / 1e9
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "index_full_traffic.json")
+    if os.path.exists(prof):
+        try:
+            traffic = json.load(open(prof)).get(wl.name)
+        except Exception:
+            traffic = None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nthreads = min(os.cpu_count() or 1, 8)
+        seqs = list(range(0, wl.B, max(1, wl.B // nthreads)))[:nthreads]
+        samples = oracle_sample_inputs(wl, layers, caches_dev, seqs)
+        secs, nseq = time_oracle(wl, samples, nthreads)
+        cpu = {"value": nseq / secs, "unit": "queries/s", "cores": min(nthreads, len(samples)), "kind": "oracle",
+               "sample": f"{nseq} of {wl.B} sequences (L={wl.max_len}), one full {wl.pattern} step each, "
+                         f"one thread per sequence; {secs:.1f} s"}
+
+    if rank == 0:
+        launches_per_step = 0
+        for _, m in enumerate(step.plan):
+            act = m[3]
+            launches_per_step += {"scan": 5, "reindex": 3, "reuse": 0}[act] + 3
+        res = {
+            "metric": METRIC,
+            "value": world * wl.B / (ms * 1e-3),
+            "unit": "queries/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "int32+f64 indexer / f32 attention",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len, "layers": wl.pattern,
+                       "pool_blocks": wl.P, "topk": wl.k, "window": 128,
+                       "l2": "no flush: inputs larger than L2 (%.2f GB read per step)" % (ab["total"] / 1e9)},
+            "tokens_per_s": world * wl.B / (ms * 1e-3),
+            "hbm_algorithmic_gbs": ab["total"] / (ms * 1e-3) / 1e9,
+            "hbm_frac_of_8tbs": ab["total"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+            "roofline": {"kernel": "csa2_index_full (scan + block max + pool + Top-512)", "bound": "hbm",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind, "traffic": traffic, "algorithmic_bytes": full_bytes,
+                         "avg_ms": full_avg},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * wl.B / (e2e_ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "device_flags": flags,
+        }
+        print(json.dumps(res))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as the reference arm: K timed steps, each one oracle decode
+    step over a bounded sample of the workload's sequences on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    import synth.workloads as W
+
+    wl = W.decode_workloads()[args.workload]
+    nthreads = min(os.cpu_count() or 1, 8)
+    if torch.cuda.is_available():
+        # inputs from the device generator (same bytes as the NumPy generator)
+        wl2, layers, caches_dev, _, _, _, _ = build_workload(wl, 0, torch.device("cuda", 0))
+        seqs = list(range(nthreads))
+        samples = oracle_sample_inputs(wl2, layers, caches_dev, seqs)
+        del caches_dev
+    else:
+        small = W.DecodeWorkload(wl.name, np.full(nthreads, min(wl.max_len, 65536)), wl.pattern, wl.P, wl.k,
+                                 wl.needles, wl.lognormal)
+        layers = [W.layer_inputs_host(small, l) for l in range(len(small.pattern))]
+        caches = [W.full_cache_host(small, f, layers[f]["q_codes"], layers[f]["q_scales"])
+                  for f in small.full_layers()]
+        samples = []
+        off = small.row_offsets()[0]
+        for b in range(nthreads):
+            o, L = int(off[b]), int(small.lengths[b])
+            ch = [{k: c[k][o:o + L] for k in ("idx_codes", "idx_scales", "main_codes", "main_scales")} for c in caches]
+            samples.append((ch, L, [{k: v[b:b + 1] for k, v in Ld.items()} for Ld in layers]))
+    for _ in range(args.warmup):
+        time_oracle(wl, samples[:1], 1)
+    secs = 0.0
+    nseq = 0
+    for _ in range(args.steps):
+        s, n = time_oracle(wl, samples, nthreads)
+        secs += s
+        nseq += n
+    value = nseq / secs
+    res = {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64 (CPU oracle)",
+           "data": "synthetic", "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len,
+                                            "layers": wl.pattern, "pool_blocks": wl.P, "topk": wl.k},
+           "cpu_baseline": {"value": value, "unit": "queries/s", "cores": nthreads, "kind": "oracle",
+                            "sample": f"{len(samples)} sequences per step, one thread each"},
+           "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

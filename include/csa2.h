@@ -1,0 +1,236 @@
+/*
+ * csa2.h -- C ABI of the CSA2 compressed-sparse-attention library (sm_100a).
+ *
+ * The operations follow the CSA2 step described on the page
+ * [V41] "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression"
+ * (fupanwang summary), sections "后 20 层干脆共用一份 KV" and
+ * "三个方向一起压小缓存", with the mode semantics corroborated by
+ * [NOTES] "DeepSeek-V4.1" (dreamax reading notes).  In short:
+ *   - Full layers compute their own main KV and indexer K; the first Full
+ *     layer scans the whole visible context, reduces every 8 positions to
+ *     their maximum score and keeps the best <= 2048 blocks as the candidate
+ *     pool (<= 16384 positions); every layer finally reads 512 entries;
+ *   - Reindex layers reuse the nearest Full layer's main KV and indexer K and
+ *     select again, only inside the pool;
+ *   - Reuse layers take the most recent Top-512 unchanged (no call here);
+ *   - main KV is OCP MXFP4, the indexer q/k are FP4, the 128-token sliding
+ *     window stays FP8; every m tokens (m = 2 in the encoder, 1 in the
+ *     decoder) become one cache entry with no overlap between entries.
+ *
+ * Conventions for every call
+ *   - All array arguments are DEVICE pointers into caller-owned memory unless
+ *     a comment says "host".  The library never allocates, never frees and
+ *     never synchronises (except csa2_device_status).  Every launch goes to
+ *     `stream` (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *   - Fixed dimensions: main latent D = 512, query heads Hq = 16, indexer
+ *     heads Hi = 4, indexer dim Di = 128, block S = 8, window W = 128.
+ *   - MXFP4 row of n elements: n/2 bytes of packed E2M1 codes (element 2j in
+ *     the low nibble of byte j, sign in bit 3 of the nibble) in the `codes`
+ *     plane, and n/32 E8M0 block-scale bytes (scale = 2^(byte-127)) in the
+ *     `scales` plane.  Row r starts at codes + r*n/2 and scales + r*n/32.
+ *   - Sequence b of a cache occupies rows seq_row_off[b] .. +seq_len[b]-1;
+ *     seq_row_off[b] must be a multiple of 8 (one indexer block) and the
+ *     cache's `rows` (its capacity) a multiple of 8.
+ *   - Scores are ranked by (score descending, position ascending); outputs
+ *     holding positions or block ids are sorted ascending and padded with -1.
+ *   - workspace: device scratch of at least the size the matching
+ *     *_workspace_bytes() function returns, 256-byte aligned, ZERO-FILLED
+ *     before its first use.  Its first 256 bytes hold a device status word
+ *     that kernels OR flags into (see CSA2_DEV_*); read and clear it with
+ *     csa2_device_status().  One workspace must not be used by two calls that
+ *     may run concurrently.
+ *   - Return value: CSA2_OK, or a negative error; on an error nothing was
+ *     launched, except CSA2_ERR_CUDA (a launch failed; see csa2_last_error()).
+ *     Arguments are validated on the host before the first launch.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSA2_MAIN_DIM 512
+#define CSA2_Q_HEADS 16
+#define CSA2_IDX_HEADS 4
+#define CSA2_IDX_DIM 128
+#define CSA2_BLOCK 8
+#define CSA2_WINDOW 128
+#define CSA2_MAX_POOL_BLOCKS 2048
+#define CSA2_MAX_TOPK 2048
+
+typedef int csa2_status;
+#define CSA2_OK 0
+#define CSA2_ERR_INVALID_ARG (-1)  /* null pointer, bad size, misaligned pointer */
+#define CSA2_ERR_UNSUPPORTED (-2)  /* valid but outside what the kernels handle */
+#define CSA2_ERR_WORKSPACE (-3)    /* workspace smaller than *_workspace_bytes() */
+#define CSA2_ERR_CUDA (-4)         /* a CUDA launch or runtime call failed */
+#define CSA2_ERR_DEVICE_CHECK (-5) /* returned by csa2_device_status() only */
+
+/* Flags of the device status word (OR-ed by kernels, never cleared by them). */
+#define CSA2_DEV_INDEX_RANGE 1u    /* a selected index was >= the visible length; it was skipped */
+#define CSA2_DEV_ROW_LAYOUT 2u     /* seq_row_off not a multiple of 8, or rows past the capacity; sequence skipped */
+#define CSA2_DEV_FP16_RANGE 4u     /* an attention operand lies outside the fp16-exact range; output invalid */
+#define CSA2_DEV_LENGTH 8u         /* a device length exceeded the host bound (max_len / n_entries); clamped */
+
+/* One MXFP4 cache (main KV: n = 512, indexer K: n = 128).  `rows` is the
+ * capacity in rows (multiple of 8).  Pointers must be 16-byte aligned. */
+typedef struct {
+  uint8_t* codes;  /* [rows][n/2]  */
+  uint8_t* scales; /* [rows][n/32] */
+  int64_t rows;
+} csa2_mxfp4_cache;
+
+/* ---------------------------------------------------------------------------
+ * csa2_index_full -- Full-mode decode indexer, one query token per sequence.
+ * Source: [V41] section "三个方向一起压小缓存", the hierarchical sparse indexer
+ * (the first Full layer scores everything, ranks 8-position blocks by their
+ * best score and keeps at most 2048 of them as the pool) and its figure.
+ * Scores every visible position t < seq_len[b] of sequence b:
+ *   s_t = sum_h w_h * (q_h . k_t), computed exactly from the FP4 codes (each
+ *   32-block dot product is an exact integer times a power of two; per head the
+ *   four block terms are summed in double and rounded once to float; the heads
+ *   are combined as s = w0*d0, then fmaf(w_h, d_h, s)); -0 counts as +0.
+ * Block maxima over positions [8j, 8j+8) form the ranking of blocks; the pool
+ * is the best `pool_blocks` blocks; topk_out is the layer's own Top-k over ALL
+ * visible positions.
+ *   idx_k       indexer-K cache (n = 128), read only
+ *   q_codes     [B][4][64] E2M1 codes of the indexer query (4 heads x 128)
+ *   q_scales    [B][4][4]  E8M0 scales of the indexer query
+ *   w           [B][4]     fp32 head weights
+ *   seq_row_off [B] int64, seq_len [B] int32 (0 <= seq_len <= max_len)
+ *   max_len     host: upper bound of seq_len (grid sizing, scores_out stride)
+ *   pool_blocks host: P, 1..2048;   k  host: 1..2048
+ *   pool_out    [B][P] int32: pool block ids (block j = positions 8j..8j+7)
+ *   topk_out    [B][k] int32: selected positions
+ *   scores_out  [B][max_len] fp32 or NULL: every visible score
+ * ------------------------------------------------------------------------- */
+size_t csa2_index_full_workspace_bytes(int B, int max_len, int pool_blocks, int k);
+csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                            const float* w, const int64_t* seq_row_off, const int32_t* seq_len, int B,
+                            int max_len, int pool_blocks, int k, int32_t* pool_out, int32_t* topk_out,
+                            float* scores_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * csa2_index_reindex -- Reindex-mode selection inside the pool.
+ * Source: [V41] section "三个方向一起压小缓存" (later layers score only inside
+ * the pool) and [NOTES] on the modes (Reindex keeps the main KV and selects
+ * again).  Scores the positions 8*pool[b][i] + j (j < 8, only
+ * those < seq_len[b]; pool entries < 0 are skipped) with THIS layer's indexer
+ * query against the nearest Full layer's indexer K, and returns their Top-k.
+ * Same score definition and tie rule as csa2_index_full.
+ *   pool        [B][P] int32: strictly ascending block ids, then -1 padding,
+ *               as csa2_index_full writes them (ties resolve in this order)
+ *   topk_out    [B][k] int32
+ * ------------------------------------------------------------------------- */
+size_t csa2_index_reindex_workspace_bytes(int B, int pool_blocks, int k);
+csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                               const float* w, const int64_t* seq_row_off, const int32_t* seq_len,
+                               const int32_t* pool, int B, int pool_blocks, int k, int32_t* topk_out,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * csa2_sparse_attn_decode -- MXFP4 + FP8 sparse attention, one softmax.
+ * Source: [V41] sections "三个方向一起压小缓存" (each layer reads 512 entries;
+ * MXFP4 main KV; FP8 window) and "后 20 层干脆共用一份 KV" (128-token window
+ * per layer); [NOTES] on the sliding-window branch.  For each sequence b and head h: one softmax over the
+ * keys  {dequantised main row seq_row_off[b] + topk[b][j] : topk[b][j] >= 0}
+ * followed by the first win_len[b] rows of the FP8 window, each E4M3 value
+ * times win_scale[b].  Keys are also the values (shared latent).
+ *   logit = sm_scale * (q_h . key);  out = softmax-weighted sum of keys;
+ *   lse = log(sum(exp(logit))) (= -inf and out = 0 when there is no key).
+ *   q          [B][16][512] bf16 (uint16 bit patterns)
+ *   main_kv    main-KV cache (n = 512), read only
+ *   topk       [B][k] int32 (-1 = empty slot); k host, 1..2048
+ *   win        [B][128][512] E4M3 bytes;  win_scale [B] fp32;  win_len [B] int32 (0..128)
+ *   out        [B][16][512] fp32;  lse [B][16] fp32 or NULL
+ * Accuracy: max-abs error <= 2e-3 and relative-L2 error <= 1e-3 against exact
+ * arithmetic for inputs whose dequantised values are exact in fp16.
+ * ------------------------------------------------------------------------- */
+size_t csa2_sparse_attn_decode_workspace_bytes(int B, int k);
+csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv, const int64_t* seq_row_off,
+                                    const int32_t* seq_len, const int32_t* topk, int k, const uint8_t* win,
+                                    const float* win_scale, const int32_t* win_len, float sm_scale, float* out,
+                                    float* lse, int B, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * csa2_compress_append -- pair compression + MXFP4 quantisation of new entries.
+ * Source: [V41] architecture figure caption (ratio 2 in the encoder, 1 in the
+ * decoder), section "三个方向一起压小缓存" (entries have disjoint sources and no
+ * absolute position encoding; the indexer K is a projection of the main KV;
+ * quantisation comes after positional encoding) and section
+ * "后 20 层干脆共用一份 KV" (each layer also projects compression weights).
+ * Sequence b contributes raw tokens tok_off[b] .. tok_off[b+1]-1 and appends
+ * n_b = (tok_off[b+1]-tok_off[b]) / ratio entries (an odd trailing token of a
+ * ratio-2 append is not emitted; resend it with the next call) at cache rows
+ * seq_row_off[b] + seq_len_in[b] + j.  seq_len_out[b] = seq_len_in[b] + n_b.
+ *   ratio 1: c = x.   ratio 2: entry j merges tokens 2j, 2j+1 with weights
+ *     w = softmax(z_2j, z_2j+1) in double (an exp of this library's own), and
+ *     c_i = float(fma(w0, x0_i, w1 * x1_i)) in double.
+ *   indexer row: w_idx != NULL -> r_o = float(sum_i c_i * w_idx[i][o]) by a
+ *     double fma chain in order i = 0..511; else idx_raw merged like x.
+ *   Both rows are MXFP4-encoded per OCP MX v1.0: X = floor(log2 amax) - 2,
+ *   nearest E2M1 with ties to even, saturating at 6, sign kept.
+ *   raw        [n_tok][512] bf16;  logits [n_tok] fp32 (ratio 2; may be NULL for ratio 1)
+ *   w_idx      [512][128] fp32 or NULL;  idx_raw [n_tok][128] bf16 or NULL (exactly one given)
+ *   tok_off    [B+1] int64;  seq_row_off [B] int64;  seq_len_in [B], seq_len_out [B] int32
+ *   n_tok      host: tok_off[B];  max_new host: upper bound of n_b (grid sizing)
+ * ------------------------------------------------------------------------- */
+size_t csa2_compress_append_workspace_bytes(int B);
+csa2_status csa2_compress_append(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k, const uint16_t* raw,
+                                 const float* logits, const float* w_idx, const uint16_t* idx_raw,
+                                 const int64_t* tok_off, const int64_t* seq_row_off, const int32_t* seq_len_in,
+                                 int32_t* seq_len_out, int B, int ratio, int64_t n_tok, int64_t max_new,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * csa2_index_prefill -- causal Full-mode indexer for a prefill chunk.
+ * Source: [V41] hierarchical indexer (as csa2_index_full), applied to every
+ * query of a causal prefill chunk.
+ * Query i sits at raw position q_pos[i]; it sees the entries j with
+ * (j+1)*ratio - 1 <= q_pos[i] (entry j covers raw tokens ratio*j ..
+ * ratio*j+ratio-1), at most n_entries, of the single sequence stored at cache
+ * rows row0 .. row0+n_entries-1.  Per query: the same score, block pool and
+ * Top-k over all visible entries as csa2_index_full.
+ *   q_codes [T][4][64], q_scales [T][4][4], w [T][4], q_pos [T] int32 (>= 0)
+ *   row0, n_entries host; ratio 1 or 2; pool_out [T][P]; topk_out [T][k]
+ * ------------------------------------------------------------------------- */
+size_t csa2_index_prefill_workspace_bytes(int T, int64_t n_entries, int pool_blocks, int k);
+csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                               const float* w, const int32_t* q_pos, int T, int64_t row0, int64_t n_entries,
+                               int ratio, int pool_blocks, int k, int32_t* pool_out, int32_t* topk_out,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * csa2_sparse_attn_prefill -- causal sparse attention of a prefill chunk.
+ * Query i attends its selected entries (topk[i][j] >= 0, each < the visible
+ * count of csa2_index_prefill) and the raw FP8 window rows
+ * max(0, q_pos[i]-127) .. q_pos[i] of raw_win (one fp32 scale), in one
+ * softmax; otherwise as csa2_sparse_attn_decode.
+ *   q [T][16][512] bf16; topk [T][k]; raw_win [n_raw][512] E4M3 (q_pos < n_raw)
+ *   out [T][16][512] fp32; lse [T][16] fp32 or NULL
+ * ------------------------------------------------------------------------- */
+size_t csa2_sparse_attn_prefill_workspace_bytes(int T, int k);
+csa2_status csa2_sparse_attn_prefill(const uint16_t* q, const int32_t* q_pos, int T, csa2_mxfp4_cache main_kv,
+                                     int64_t row0, int64_t n_entries, int ratio, const int32_t* topk, int k,
+                                     const uint8_t* raw_win, int64_t n_raw, float win_scale, float sm_scale,
+                                     float* out, float* lse, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/* Synchronises `stream`, returns the status word of `workspace` in *flags
+ * (CSA2_DEV_* bits) and clears it.  Returns CSA2_ERR_DEVICE_CHECK when any
+ * flag was set, CSA2_OK otherwise.  Test and debugging helper. */
+csa2_status csa2_device_status(void* workspace, void* stream, uint32_t* flags);
+
+/* Static text of a status code, and the message of the last CSA2_ERR_* of the
+ * calling host thread ("" if none). */
+const char* csa2_status_string(csa2_status s);
+const char* csa2_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H */

@@ -1,0 +1,391 @@
+// C ABI entry points of the CSA2 library: host-side validation, workspace
+// carving, and the launch sequence of each call (all on the caller's stream).
+#include <cstdio>
+#include <string>
+
+#include "internal.cuh"
+
+namespace csa2 {
+
+namespace {
+thread_local std::string g_last_error;
+}
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+csa2_status fail(csa2_status code, const std::string& msg) {
+  set_error(msg);
+  return code;
+}
+
+csa2_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(CSA2_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return CSA2_OK;
+}
+
+// Sequential carving of a workspace into 256-byte aligned pieces.
+struct Carve {
+  char* base;
+  size_t used;
+  explicit Carve(void* ws) : base(static_cast<char*>(ws)), used(0) {}
+  template <class T>
+  T* take(size_t count) {
+    T* p = reinterpret_cast<T*>(base ? base + used : nullptr);
+    used = round_up(used + count * sizeof(T), 256);
+    return p;
+  }
+};
+
+bool cache_ok(const csa2_mxfp4_cache& c) {
+  return c.codes && c.scales && aligned16(c.codes) && aligned16(c.scales) && c.rows >= 0 && (c.rows % 8) == 0;
+}
+
+struct IndexFullWs {
+  uint32_t* status;
+  int32_t* seg_eff;
+  uint32_t* bkeys;
+  uint32_t* ckeys;
+  float* scores;
+  size_t bytes;
+};
+
+IndexFullWs index_full_ws(void* ws, int B, int max_len, int P, int k, bool need_scores) {
+  Carve c(ws);
+  IndexFullWs w;
+  w.status = c.take<uint32_t>(kStatusBytes / 4);
+  w.seg_eff = c.take<int32_t>(size_t(B));
+  const size_t nb = (size_t(max_len) + kBlk - 1) / kBlk;
+  w.bkeys = c.take<uint32_t>(size_t(B) * nb);
+  w.ckeys = (P >= k) ? c.take<uint32_t>(size_t(B) * P * kBlk) : nullptr;
+  w.scores = need_scores ? c.take<float>(size_t(B) * max_len) : nullptr;
+  w.bytes = c.used;
+  return w;
+}
+
+}  // namespace csa2
+
+using namespace csa2;
+
+extern "C" {
+
+const char* csa2_status_string(csa2_status s) {
+  switch (s) {
+    case CSA2_OK: return "ok";
+    case CSA2_ERR_INVALID_ARG: return "invalid argument";
+    case CSA2_ERR_UNSUPPORTED: return "unsupported";
+    case CSA2_ERR_WORKSPACE: return "workspace too small";
+    case CSA2_ERR_CUDA: return "CUDA error";
+    case CSA2_ERR_DEVICE_CHECK: return "device check failed";
+    default: return "unknown status";
+  }
+}
+
+const char* csa2_last_error(void) { return g_last_error.c_str(); }
+
+csa2_status csa2_device_status(void* workspace, void* stream, uint32_t* flags) {
+  if (!workspace || !flags) return fail(CSA2_ERR_INVALID_ARG, "csa2_device_status: null argument");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(h), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(CSA2_ERR_CUDA, std::string("csa2_device_status: ") + cudaGetErrorString(e));
+  *flags = h;
+  return h ? CSA2_ERR_DEVICE_CHECK : CSA2_OK;
+}
+
+// ---------------------------------------------------------------------------
+size_t csa2_index_full_workspace_bytes(int B, int max_len, int pool_blocks, int k) {
+  if (B < 0 || max_len < 0) return 0;
+  return index_full_ws(nullptr, B, max_len, pool_blocks, k, pool_blocks < k).bytes;
+}
+
+csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                            const int64_t* seq_row_off, const int32_t* seq_len, int B, int max_len,
+                            int pool_blocks, int k, int32_t* pool_out, int32_t* topk_out, float* scores_out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_full";
+  if (B < 0 || max_len < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
+  if (pool_blocks < 1 || pool_blocks > CSA2_MAX_POOL_BLOCKS || k < 1 || k > CSA2_MAX_TOPK)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": pool_blocks and k must be in 1..2048");
+  if (B == 0) return CSA2_OK;
+  if (!cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad indexer-K cache");
+  if (!q_codes || !q_scales || !w || !seq_row_off || !seq_len || !pool_out || !topk_out || !workspace)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (!aligned16(q_codes) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": q_codes must be 16-byte and workspace 256-byte aligned");
+  const bool need_scores = pool_blocks < k && scores_out == nullptr;
+  IndexFullWs ws = index_full_ws(workspace, B, max_len, pool_blocks, k, need_scores);
+  if (workspace_bytes < ws.bytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SegDesc sd{seq_row_off, 0, seq_len, max_len, idx_k.rows};
+  const int64_t nb = (int64_t(max_len) + kBlk - 1) / kBlk;
+  float* scores = scores_out ? scores_out : ws.scores;
+  launch_seg_check(sd, B, ws.seg_eff, ws.status, st);
+  launch_scan(idx_k.codes, idx_k.scales, sd, ws.seg_eff, B, q_codes, q_scales, w, ws.bkeys, nb, scores, max_len, st);
+  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, st);
+  if (pool_blocks >= k) {
+    // Every Top-k position's block ranks within the first k blocks, so the
+    // Top-k over the pool equals the Top-k over all positions.
+    launch_pool_score(idx_k.codes, idx_k.scales, sd, ws.seg_eff, B, q_codes, q_scales, w, pool_out, pool_blocks,
+                      ws.ckeys, ws.status, st);
+    launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.seg_eff, B, pool_blocks, pool_out, k,
+                  topk_out, st);
+  } else {
+    launch_select(kSelScores, scores, max_len, ws.seg_eff, B, 0, nullptr, k, topk_out, st);
+  }
+  return check_launch(fn);
+}
+
+// ---------------------------------------------------------------------------
+size_t csa2_index_reindex_workspace_bytes(int B, int pool_blocks, int k) {
+  (void)k;
+  Carve c(nullptr);
+  c.take<uint32_t>(kStatusBytes / 4);
+  c.take<int32_t>(size_t(B));
+  c.take<uint32_t>(size_t(B) * pool_blocks * kBlk);
+  return c.used;
+}
+
+csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                               const float* w, const int64_t* seq_row_off, const int32_t* seq_len,
+                               const int32_t* pool, int B, int pool_blocks, int k, int32_t* topk_out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_reindex";
+  if (B < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
+  if (pool_blocks < 1 || pool_blocks > CSA2_MAX_POOL_BLOCKS || k < 1 || k > CSA2_MAX_TOPK)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": pool_blocks and k must be in 1..2048");
+  if (B == 0) return CSA2_OK;
+  if (!cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad indexer-K cache");
+  if (!q_codes || !q_scales || !w || !seq_row_off || !seq_len || !pool || !topk_out || !workspace)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": workspace must be 256-byte aligned");
+  if (workspace_bytes < csa2_index_reindex_workspace_bytes(B, pool_blocks, k))
+    return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  Carve c(workspace);
+  uint32_t* status = c.take<uint32_t>(kStatusBytes / 4);
+  int32_t* seg_eff = c.take<int32_t>(size_t(B));
+  uint32_t* ckeys = c.take<uint32_t>(size_t(B) * pool_blocks * kBlk);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SegDesc sd{seq_row_off, 0, seq_len, INT32_MAX, idx_k.rows};
+  launch_seg_check(sd, B, seg_eff, status, st);
+  launch_pool_score(idx_k.codes, idx_k.scales, sd, seg_eff, B, q_codes, q_scales, w, pool, pool_blocks, ckeys,
+                    status, st);
+  launch_select(kSelPoolCand, ckeys, int64_t(pool_blocks) * kBlk, seg_eff, B, pool_blocks, pool, k, topk_out, st);
+  return check_launch(fn);
+}
+
+// ---------------------------------------------------------------------------
+size_t csa2_sparse_attn_decode_workspace_bytes(int B, int k) {
+  Carve c(nullptr);
+  c.take<uint32_t>(kStatusBytes / 4);
+  c.take<int32_t>(size_t(B));
+  c.take<char>(attn_partial_bytes(B, k));
+  return c.used;
+}
+
+csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv, const int64_t* seq_row_off,
+                                    const int32_t* seq_len, const int32_t* topk, int k, const uint8_t* win,
+                                    const float* win_scale, const int32_t* win_len, float sm_scale, float* out,
+                                    float* lse, int B, void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_sparse_attn_decode";
+  if (B < 0 || k < 1 || k > CSA2_MAX_TOPK) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad B or k");
+  if (B == 0) return CSA2_OK;
+  if (!cache_ok(main_kv)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad main-KV cache");
+  if (!q || !seq_row_off || !seq_len || !topk || !win || !win_scale || !win_len || !out || !workspace)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (!aligned16(win) || !aligned16(q) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": q/win must be 16-byte, workspace 256-byte aligned");
+  if (workspace_bytes < csa2_sparse_attn_decode_workspace_bytes(B, k))
+    return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  Carve c(workspace);
+  AttnArgs a{};
+  a.status = c.take<uint32_t>(kStatusBytes / 4);
+  int32_t* seg_eff = c.take<int32_t>(size_t(B));
+  a.partial = reinterpret_cast<float*>(c.take<char>(attn_partial_bytes(B, k)));
+  a.q = q;
+  a.mcodes = main_kv.codes;
+  a.mscales = main_kv.scales;
+  a.sd = SegDesc{seq_row_off, 0, seq_len, INT32_MAX, main_kv.rows};
+  a.seg_eff = seg_eff;
+  a.topk = topk;
+  a.k = k;
+  a.win = win;
+  a.win_scale = win_scale;
+  a.win_len = win_len;
+  a.sm_scale = sm_scale;
+  a.out = out;
+  a.lse = lse;
+  a.S = B;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  launch_seg_check(a.sd, B, seg_eff, a.status, st);
+  launch_attention(a, st);
+  return check_launch(fn);
+}
+
+// ---------------------------------------------------------------------------
+size_t csa2_compress_append_workspace_bytes(int B) {
+  (void)B;
+  return kStatusBytes;
+}
+
+csa2_status csa2_compress_append(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k, const uint16_t* raw,
+                                 const float* logits, const float* w_idx, const uint16_t* idx_raw,
+                                 const int64_t* tok_off, const int64_t* seq_row_off, const int32_t* seq_len_in,
+                                 int32_t* seq_len_out, int B, int ratio, int64_t n_tok, int64_t max_new,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_compress_append";
+  if (B < 0 || n_tok < 0 || max_new < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
+  if (ratio != 1 && ratio != 2) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": ratio must be 1 or 2");
+  if (B == 0) return CSA2_OK;
+  if (!cache_ok(main_kv) || !cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad cache");
+  if (!raw || !tok_off || !seq_row_off || !seq_len_in || !seq_len_out || !workspace)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (ratio == 2 && !logits) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": ratio 2 needs logits");
+  if ((w_idx == nullptr) == (idx_raw == nullptr))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": give exactly one of w_idx and idx_raw");
+  if (!aligned16(raw) || (idx_raw && (reinterpret_cast<uintptr_t>(idx_raw) & 7)))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": raw must be 16-byte and idx_raw 8-byte aligned");
+  if (workspace_bytes < kStatusBytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  CompressArgs a{};
+  a.mcodes = main_kv.codes;
+  a.mscales = main_kv.scales;
+  a.mrows = main_kv.rows;
+  a.icodes = idx_k.codes;
+  a.iscales = idx_k.scales;
+  a.irows = idx_k.rows;
+  a.raw = raw;
+  a.logits = logits;
+  a.w_idx = w_idx;
+  a.idx_raw = idx_raw;
+  a.tok_off = tok_off;
+  a.seq_row_off = seq_row_off;
+  a.seq_len_in = seq_len_in;
+  a.seq_len_out = seq_len_out;
+  a.B = B;
+  a.ratio = ratio;
+  a.max_new = max_new;
+  a.status = static_cast<uint32_t*>(workspace);
+  launch_compress(a, static_cast<cudaStream_t>(stream));
+  return check_launch(fn);
+}
+
+// ---------------------------------------------------------------------------
+namespace {
+struct PrefillWs {
+  uint32_t* status;
+  int32_t* vis;
+  uint32_t* bkeys;
+  uint32_t* ckeys;
+  float* scores;
+  size_t bytes;
+};
+PrefillWs prefill_ws(void* ws, int T, int64_t n_entries, int P, int k) {
+  Carve c(ws);
+  PrefillWs w;
+  w.status = c.take<uint32_t>(kStatusBytes / 4);
+  w.vis = c.take<int32_t>(size_t(T));
+  const size_t nb = (size_t(n_entries) + kBlk - 1) / kBlk;
+  w.bkeys = c.take<uint32_t>(size_t(T) * nb);
+  w.ckeys = c.take<uint32_t>(size_t(T) * P * kBlk);
+  w.scores = nullptr;
+  w.bytes = c.used;
+  return w;
+}
+}  // namespace
+
+size_t csa2_index_prefill_workspace_bytes(int T, int64_t n_entries, int pool_blocks, int k) {
+  if (T < 0 || n_entries < 0) return 0;
+  return prefill_ws(nullptr, T, n_entries, pool_blocks, k).bytes;
+}
+
+csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                               const float* w, const int32_t* q_pos, int T, int64_t row0, int64_t n_entries,
+                               int ratio, int pool_blocks, int k, int32_t* pool_out, int32_t* topk_out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_prefill";
+  if (T < 0 || n_entries < 0 || row0 < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
+  if (ratio != 1 && ratio != 2) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": ratio must be 1 or 2");
+  if (pool_blocks < 1 || pool_blocks > CSA2_MAX_POOL_BLOCKS || k < 1 || k > CSA2_MAX_TOPK)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": pool_blocks and k must be in 1..2048");
+  if (pool_blocks < k)
+    return fail(CSA2_ERR_UNSUPPORTED, std::string(fn) + ": prefill needs pool_blocks >= k");
+  if (T == 0) return CSA2_OK;
+  if (!cache_ok(idx_k) || (row0 % 8) != 0 || row0 + n_entries > idx_k.rows || n_entries > INT32_MAX)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad cache, row0 or n_entries");
+  if (!q_codes || !q_scales || !w || !q_pos || !pool_out || !topk_out || !workspace)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": workspace must be 256-byte aligned");
+  PrefillWs ws = prefill_ws(workspace, T, n_entries, pool_blocks, k);
+  if (workspace_bytes < ws.bytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t nb = (n_entries + kBlk - 1) / kBlk;
+  launch_prefill_vis(q_pos, T, ratio, n_entries, ws.vis, ws.status, st);
+  launch_prefill_scan(idx_k.codes, idx_k.scales, row0, ws.vis, T, n_entries, q_codes, q_scales, w, ws.bkeys, nb, st);
+  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, T, 0, nullptr, pool_blocks, pool_out, st);
+  SegDesc sd{nullptr, row0, ws.vis, n_entries, idx_k.rows};
+  launch_pool_score(idx_k.codes, idx_k.scales, sd, ws.vis, T, q_codes, q_scales, w, pool_out, pool_blocks, ws.ckeys,
+                    ws.status, st);
+  launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.vis, T, pool_blocks, pool_out, k, topk_out,
+                st);
+  return check_launch(fn);
+}
+
+// ---------------------------------------------------------------------------
+size_t csa2_sparse_attn_prefill_workspace_bytes(int T, int k) {
+  Carve c(nullptr);
+  c.take<uint32_t>(kStatusBytes / 4);
+  c.take<int32_t>(size_t(T));
+  c.take<char>(attn_partial_bytes(T, k));
+  return c.used;
+}
+
+csa2_status csa2_sparse_attn_prefill(const uint16_t* q, const int32_t* q_pos, int T, csa2_mxfp4_cache main_kv,
+                                     int64_t row0, int64_t n_entries, int ratio, const int32_t* topk, int k,
+                                     const uint8_t* raw_win, int64_t n_raw, float win_scale, float sm_scale,
+                                     float* out, float* lse, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  const char* fn = "csa2_sparse_attn_prefill";
+  if (T < 0 || k < 1 || k > CSA2_MAX_TOPK || n_entries < 0 || n_raw < 0 || row0 < 0)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad size");
+  if (ratio != 1 && ratio != 2) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": ratio must be 1 or 2");
+  if (T == 0) return CSA2_OK;
+  if (!cache_ok(main_kv) || row0 + n_entries > main_kv.rows || n_entries > INT32_MAX)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad cache, row0 or n_entries");
+  if (!q || !q_pos || !topk || !raw_win || !out || !workspace)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (!aligned16(q) || !aligned16(raw_win) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": q/raw_win must be 16-byte, workspace 256-byte aligned");
+  if (workspace_bytes < csa2_sparse_attn_prefill_workspace_bytes(T, k))
+    return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  Carve c(workspace);
+  AttnArgs a{};
+  a.status = c.take<uint32_t>(kStatusBytes / 4);
+  int32_t* vis = c.take<int32_t>(size_t(T));
+  a.partial = reinterpret_cast<float*>(c.take<char>(attn_partial_bytes(T, k)));
+  a.q = q;
+  a.mcodes = main_kv.codes;
+  a.mscales = main_kv.scales;
+  a.sd = SegDesc{nullptr, row0, vis, n_entries, main_kv.rows};
+  a.seg_eff = vis;
+  a.topk = topk;
+  a.k = k;
+  a.q_pos = q_pos;
+  a.raw_win = raw_win;
+  a.n_raw = n_raw;
+  a.raw_scale = win_scale;
+  a.sm_scale = sm_scale;
+  a.out = out;
+  a.lse = lse;
+  a.S = T;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  launch_prefill_vis(q_pos, T, ratio, n_entries, vis, a.status, st);
+  launch_attention(a, st);
+  return check_launch(fn);
+}
+
+}  // extern "C"

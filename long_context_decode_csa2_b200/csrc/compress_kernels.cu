@@ -1,0 +1,200 @@
+// Pair compression (ratio 2) / pass-through (ratio 1), optional indexer-K
+// projection, and OCP MXFP4 encoding of the new cache entries.
+//
+// "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression": the
+// architecture figure caption (ratio 2 in the encoder, 1 in the decoder),
+// section "三个方向一起压小缓存" (disjoint sources, no absolute position
+// encoding, indexer K projected from the main KV, MXFP4 after positional
+// encoding) and section "后 20 层干脆共用一份 KV" (per-layer compression
+// weights).  Every floating-point step is an explicit _rn intrinsic so that
+// nvcc cannot contract it; the exp is this library's own (Cody & Waite
+// reduction by ln 2, Taylor series of degree 14) so results are reproducible
+// bit for bit on any IEEE-754 implementation taking the same steps.
+#include "device_common.cuh"
+
+namespace csa2 {
+
+// ln 2 split into an exactly representable 24-bit head and a tail.
+__device__ __constant__ double kLn2Head = 0.6931471824645996;   // 11629080 * 2^-24
+__device__ __constant__ double kLn2Tail = -1.904654299957768e-09;
+__device__ __constant__ double kInvLn2 = 1.4426950408889634;
+
+__device__ double own_exp(double x) {
+  if (x < -745.0) return 0.0;
+  if (x > 709.0) return __longlong_as_double(0x7FF0000000000000LL);
+  const double k = rint(__dmul_rn(x, kInvLn2));  // nearest, ties to even
+  const double r = __dsub_rn(__dsub_rn(x, __dmul_rn(k, kLn2Head)), __dmul_rn(k, kLn2Tail));
+  // Taylor coefficients 1/n!, n = 14 .. 0 (Horner)
+  double p = 1.0 / 87178291200.0;
+  p = __fma_rn(p, r, 1.0 / 6227020800.0);
+  p = __fma_rn(p, r, 1.0 / 479001600.0);
+  p = __fma_rn(p, r, 1.0 / 39916800.0);
+  p = __fma_rn(p, r, 1.0 / 3628800.0);
+  p = __fma_rn(p, r, 1.0 / 362880.0);
+  p = __fma_rn(p, r, 1.0 / 40320.0);
+  p = __fma_rn(p, r, 1.0 / 5040.0);
+  p = __fma_rn(p, r, 1.0 / 720.0);
+  p = __fma_rn(p, r, 1.0 / 120.0);
+  p = __fma_rn(p, r, 1.0 / 24.0);
+  p = __fma_rn(p, r, 1.0 / 6.0);
+  p = __fma_rn(p, r, 1.0 / 2.0);
+  p = __fma_rn(p, r, 1.0);
+  p = __fma_rn(p, r, 1.0);
+  const int ki = static_cast<int>(k);
+  if (ki >= -1020) return __dmul_rn(p, pow2d(ki));
+  return __dmul_rn(__dmul_rn(p, pow2d(ki + 1000)), pow2d(-1000));  // one rounding
+}
+
+__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
+
+// OCP MXFP4 block exponent X = floor(log2 amax) - 2, clamped to [-127, 127];
+// amax == 0 gives -127.
+__device__ __forceinline__ int mx_block_exp(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  if (bits == 0u) return -127;
+  const int e = int((bits >> 23) & 255u);
+  int fl;
+  if (e == 0) fl = -149 + (31 - __clz(int(bits & 0x7FFFFFu)));
+  else fl = e - 127;
+  return max(-127, min(127, fl - 2));
+}
+
+// 2^-X as float (X in [-127, 127]).
+__device__ __forceinline__ float pow2f_neg(int X) {
+  const int e = -X;  // in [-127, 127]
+  return e >= -126 ? __uint_as_float(uint32_t(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// E2M1 code of x at block exponent X: nearest magnitude, ties to the even
+// mantissa, saturating at 6; the sign bit is x's sign bit.
+__device__ __forceinline__ uint32_t e2m1_code(float x, float inv_scale) {
+  const float a = fabsf(__fmul_rn(x, inv_scale));
+  const uint32_t idx = uint32_t(a > 0.25f) + uint32_t(a >= 0.75f) + uint32_t(a > 1.25f) + uint32_t(a >= 1.75f) +
+                       uint32_t(a > 2.5f) + uint32_t(a >= 3.5f) + uint32_t(a > 5.0f);
+  return idx | ((__float_as_uint(x) >> 28) & 8u);
+}
+
+constexpr int kCompWarps = 8;
+
+// grid = (ceil(max_new / 8), B), block = 256: one warp per new entry.
+__global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
+  __shared__ float cbuf[kCompWarps][kD];
+  __shared__ float rbuf[kCompWarps][kDi];
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tok0 = a.tok_off[b];
+  const int64_t ntok = a.tok_off[b + 1] - tok0;
+  const int64_t nnew = ntok > 0 ? ntok / a.ratio : 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.seq_len_out[b] = a.seq_len_in[b] + int32_t(nnew);
+  const int64_t j = int64_t(blockIdx.x) * kCompWarps + warp;
+  if (j >= nnew) return;
+  const int64_t row = a.seq_row_off[b] + a.seq_len_in[b] + j;
+  if (row < 0 || row >= a.mrows || row >= a.irows) {
+    if (lane == 0) set_status(a.status, CSA2_DEV_ROW_LAYOUT);
+    return;
+  }
+  const int64_t t0 = tok0 + a.ratio * j;  // first raw token of the entry
+
+  double w0 = 1.0, w1 = 0.0;
+  if (a.ratio == 2) {
+    const double z0 = a.logits[t0], z1 = a.logits[t0 + 1];
+    const double m = fmax(z0, z1);
+    const double e0 = own_exp(__dsub_rn(z0, m)), e1 = own_exp(__dsub_rn(z1, m));
+    const double s = __dadd_rn(e0, e1);
+    w0 = __ddiv_rn(e0, s);
+    w1 = __ddiv_rn(e1, s);
+  }
+
+  // ---- main row: lane holds elements 16*lane .. 16*lane+15 ----
+  float c[16];
+  {
+    const uint4* p0 = reinterpret_cast<const uint4*>(a.raw + t0 * kD + 16 * lane);
+    const uint4 u0 = __ldg(p0), u1 = __ldg(p0 + 1);
+    const uint32_t x0w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    if (a.ratio == 2) {
+      const uint4* p1 = reinterpret_cast<const uint4*>(a.raw + (t0 + 1) * kD + 16 * lane);
+      const uint4 v0 = __ldg(p1), v1 = __ldg(p1 + 1);
+      const uint32_t x1w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+        const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
+        c[i] = __double2float_rn(__fma_rn(w0, x0, __dmul_rn(w1, x1)));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) c[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+    }
+  }
+  {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(c[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    const int X = mx_block_exp(amax);
+    const float inv = pow2f_neg(X);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) lo |= e2m1_code(c[i], inv) << (4 * i);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hi |= e2m1_code(c[8 + i], inv) << (4 * i);
+    *reinterpret_cast<uint2*>(a.mcodes + row * kMainCodeBytes + 8 * lane) = make_uint2(lo, hi);
+    if ((lane & 1) == 0) a.mscales[row * kMainScaleBytes + lane / 2] = uint8_t(X + 127);
+  }
+
+  // ---- indexer row: 128 elements, lane holds 4*lane .. 4*lane+3 ----
+  float r[4];
+  if (a.w_idx) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cbuf[warp][16 * lane + i] = c[i];
+    __syncwarp();
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int i = 0; i < kD; ++i) {
+      const double ci = cbuf[warp][i];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[m] = __fma_rn(ci, double(__ldg(a.w_idx + i * kDi + lane + 32 * m)), acc[m]);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) rbuf[warp][lane + 32 * m] = __double2float_rn(acc[m]);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = rbuf[warp][4 * lane + i];
+  } else {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(a.idx_raw + t0 * kDi + 4 * lane));
+    const uint32_t x0w[2] = {u.x, u.y};
+    if (a.ratio == 2) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.idx_raw + (t0 + 1) * kDi + 4 * lane));
+      const uint32_t x1w[2] = {v.x, v.y};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+        const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
+        r[i] = __double2float_rn(__fma_rn(w0, x0, __dmul_rn(w1, x1)));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+    }
+  }
+  {
+    float amax = fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3])));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    const int X = mx_block_exp(amax);
+    const float inv = pow2f_neg(X);
+    uint32_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v |= e2m1_code(r[i], inv) << (4 * i);
+    *reinterpret_cast<uint16_t*>(a.icodes + row * kIdxCodeBytes + 2 * lane) = uint16_t(v);
+    if ((lane & 7) == 0) a.iscales[row * kIdxScaleBytes + lane / 8] = uint8_t(X + 127);
+  }
+}
+
+void launch_compress(const CompressArgs& a, cudaStream_t st) {
+  if (a.B == 0) return;
+  const int64_t gx = a.max_new > 0 ? (a.max_new + kCompWarps - 1) / kCompWarps : 1;
+  k_compress<<<dim3(static_cast<unsigned>(gx), a.B), kCompWarps * 32, 0, st>>>(a);
+}
+
+}  // namespace csa2

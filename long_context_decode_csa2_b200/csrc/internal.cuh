@@ -1,0 +1,138 @@
+// Internal declarations shared by the CSA2 CUDA sources (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "csa2.h"
+
+namespace csa2 {
+
+constexpr int kD = CSA2_MAIN_DIM;      // 512
+constexpr int kHq = CSA2_Q_HEADS;      // 16
+constexpr int kHi = CSA2_IDX_HEADS;    // 4
+constexpr int kDi = CSA2_IDX_DIM;      // 128
+constexpr int kBlk = CSA2_BLOCK;       // 8
+constexpr int kWin = CSA2_WINDOW;      // 128
+constexpr int kIdxCodeBytes = kDi / 2;        // 64
+constexpr int kIdxScaleBytes = kDi / 32;      // 4
+constexpr int kMainCodeBytes = kD / 2;        // 256
+constexpr int kMainScaleBytes = kD / 32;      // 16
+constexpr size_t kStatusBytes = 256;          // head of every workspace
+
+// ---------------------------------------------------------------------------
+// Host-side error plumbing (thread-local message, no other global state).
+// ---------------------------------------------------------------------------
+void set_error(const std::string& msg);
+csa2_status fail(csa2_status code, const std::string& msg);
+csa2_status check_launch(const char* what);
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------
+// Segments: a "segment" is one ranking problem (a decode sequence, or one
+// prefill query).  Segment s reads cache rows row_off(s) .. + len(s) - 1.
+// ---------------------------------------------------------------------------
+struct SegDesc {
+  const int64_t* row_off;  // [S] or null (then row0 for every segment)
+  int64_t row0;
+  const int32_t* len;      // [S]
+  int64_t max_len;         // host bound
+  int64_t cache_rows;      // capacity of the cache
+};
+
+// Prepared FP4 indexer query for CUDA-core scoring.
+struct IdxQueryPrep;
+
+// ---------------------------------------------------------------------------
+// Kernel launchers (each returns after enqueueing on `st`).
+// ---------------------------------------------------------------------------
+// Effective length per segment after layout checks -> seg_eff [S].
+void launch_seg_check(const SegDesc& sd, int S, int32_t* seg_eff, uint32_t* status, cudaStream_t st);
+
+// Decode scan over all visible positions: block keys [S][nb_stride] and
+// optional scores [S][max_len].
+void launch_scan(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
+                 int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w, uint32_t* bkeys,
+                 int64_t nb_stride, float* scores, int64_t score_stride, cudaStream_t st);
+
+// Scores of pool candidates 8*pool[s][i/8] + i%8 -> keys [S][P*8] (0 = absent).
+void launch_pool_score(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
+                       int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                       const int32_t* pool, int P, uint32_t* ckeys, uint32_t* status, cudaStream_t st);
+
+// Prefill scan: block keys [T][nb_stride] for every query against the visible
+// prefix of one sequence.
+void launch_prefill_scan(const uint8_t* kcodes, const uint8_t* kscales, int64_t row0, const int32_t* vis, int T,
+                         int64_t max_vis, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                         uint32_t* bkeys, int64_t nb_stride, cudaStream_t st);
+
+// Visible entry counts of prefill queries.
+void launch_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entries, int32_t* vis, uint32_t* status,
+                        cudaStream_t st);
+
+// Selection: per segment the k best of n keys (0 = absent) by (key desc,
+// index asc), written ascending.  Input kinds below.
+enum SelectKind : int {
+  kSelBlockKeys = 0,  // u32 keys, n = ceil(seg_eff/8), id = index
+  kSelScores = 1,     // fp32 scores, n = seg_eff, id = index
+  kSelPoolCand = 2,   // u32 keys, n = P*8, id = 8*pool[i/8] + i%8
+};
+void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P,
+                   const int32_t* pool, int k, int32_t* out, cudaStream_t st);
+
+// Attention partials + combine.
+struct AttnArgs {
+  const uint16_t* q;            // [S][16][512] bf16
+  const uint8_t* mcodes;
+  const uint8_t* mscales;
+  SegDesc sd;                   // rows of segment s (len = visible count)
+  const int32_t* seg_eff;       // checked visible count
+  const int32_t* topk;          // [S][k]
+  int k;
+  // decode window
+  const uint8_t* win;           // [S][128][512] or null
+  const float* win_scale;       // [S]
+  const int32_t* win_len;       // [S]
+  // prefill window
+  const int32_t* q_pos;         // [S] or null
+  const uint8_t* raw_win;       // [n_raw][512]
+  int64_t n_raw;
+  float raw_scale;
+  float sm_scale;
+  float* out;                   // [S][16][512]
+  float* lse;                   // [S][16] or null
+  float* partial;               // workspace
+  uint32_t* status;
+  int S;
+};
+int attn_num_chunks(int k);
+size_t attn_partial_bytes(int S, int k);
+void launch_attention(const AttnArgs& a, cudaStream_t st);
+
+// Compression + MXFP4 encode.
+struct CompressArgs {
+  uint8_t* mcodes;
+  uint8_t* mscales;
+  int64_t mrows;
+  uint8_t* icodes;
+  uint8_t* iscales;
+  int64_t irows;
+  const uint16_t* raw;
+  const float* logits;
+  const float* w_idx;
+  const uint16_t* idx_raw;
+  const int64_t* tok_off;
+  const int64_t* seq_row_off;
+  const int32_t* seq_len_in;
+  int32_t* seq_len_out;
+  int B;
+  int ratio;
+  int64_t max_new;
+  uint32_t* status;
+};
+void launch_compress(const CompressArgs& a, cudaStream_t st);
+
+}  // namespace csa2

@@ -252,3 +252,47 @@ def attn_prefill(q_bf16, q_pos, mcodes, mscales, row0, n_entries, ratio, topk_id
     if rc != 0:
         raise ValueError("oracle: a selected index lies outside the visible context")
     return out, lse
+
+
+# ----------------------------------------------------------------------------
+# a whole decode step through a layer pattern (F / R / U)
+# ----------------------------------------------------------------------------
+
+def decode_step(pattern, caches, seq_row_off, seq_len, layers, P, k, sm_scale, full_rescan=False, nthreads=0,
+                attention=True):
+    """Oracle decode step.  caches: per Full layer dict(idx_codes, idx_scales,
+    main_codes, main_scales); layers: per layer dict(q, q_codes, q_scales, w,
+    win, win_scale, win_len).  Modes per the pages: the first Full layer scans
+    and builds the pool; a later Full layer selects inside that pool with its
+    own caches (or rescans when full_rescan); Reindex selects inside the pool
+    with the nearest Full layer's indexer K; Reuse repeats the latest Top-k.
+    Returns dict(pools, topk, out, lse) with one entry per layer (pools: per
+    Full layer that scanned)."""
+    full_idx = -1
+    scanned = False
+    pool = None
+    last = None
+    res = dict(pools={}, topk=[], out=[], lse=[])
+    for layer, mode in enumerate(pattern):
+        L = layers[layer]
+        if mode == "F":
+            full_idx += 1
+        c = caches[full_idx]
+        if mode == "F" and (not scanned or full_rescan):
+            pool, top, _ = index_full(c["idx_codes"], c["idx_scales"], L["q_codes"], L["q_scales"], L["w"],
+                                      seq_row_off, seq_len, P, k, nthreads=nthreads)
+            res["pools"][layer] = pool
+            scanned = True
+            last = top
+        elif mode in ("F", "R"):
+            last = index_reindex(c["idx_codes"], c["idx_scales"], L["q_codes"], L["q_scales"], L["w"], seq_row_off,
+                                 seq_len, pool, k, nthreads=nthreads)
+        elif mode != "U":
+            raise ValueError(mode)
+        res["topk"].append(last)
+        if attention:
+            o, l = attn_decode(L["q"], c["main_codes"], c["main_scales"], seq_row_off, seq_len, last, L["win"],
+                               L["win_scale"], L["win_len"], sm_scale, nthreads=nthreads)
+            res["out"].append(o)
+            res["lse"].append(l)
+    return res

@@ -410,9 +410,10 @@ int orc_attn_decode(const uint16_t* q, const uint8_t* mcodes, const uint8_t* msc
   return bad ? -1 : 0;
 }
 
-// Compression + quantisation of new cache entries [V41] ("every m tokens
-// become one entry, no overlap, no absolute position encoding"; the weights
-// are a softmax over the pair's per-token logits, this build's reading).
+// Compression + quantisation of new cache entries [V41]: m tokens become one
+// entry, entries have disjoint sources and no absolute position encoding; the
+// weights are a softmax over the pair's per-token logits (this build's
+// reading of the garbled weighting formula).
 // ratio 1: c = x.  ratio 2: entry j merges raw rows 2j, 2j+1:
 //   m = max(z0, z1); a = exp(z0-m); b = exp(z1-m); w0 = a/(a+b); w1 = b/(a+b)
 //   c_i = fp32( fma(w0, x0_i, w1*x1_i) )   (fp64, own exp)

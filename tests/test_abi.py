@@ -1,0 +1,92 @@
+"""The C-ABI library loads, exports every function include/csa2.h declares,
+and rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes as Cc
+import os
+import re
+
+import pytest
+
+from long_context_decode_csa2_b200 import _build
+from long_context_decode_csa2_b200 import csa2 as C
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "csa2.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(csa2_\w+)\s*\(", text)))
+
+
+def test_library_builds_and_exports_every_declared_symbol():
+    path = _build.build()
+    lib = Cc.CDLL(path)
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    L = C.lib()
+    assert L.csa2_status_string(0) == b"ok"
+    assert L.csa2_status_string(-3) == b"workspace too small"
+
+
+FAKE = 0x10000  # an aligned non-null address; never dereferenced (rejected first)
+
+
+def _cache(rows=1024, codes=FAKE, scales=FAKE):
+    return C.MXFP4Cache(codes, scales, rows)
+
+
+def test_index_full_validation():
+    L = C.lib()
+    ws = L.csa2_index_full_workspace_bytes(2, 1000, 64, 64)
+    args = dict(q=FAKE, qs=FAKE, w=FAKE, off=FAKE, ln=FAKE, pool=FAKE, top=FAKE)
+
+    def call(cache=None, B=2, max_len=1000, P=64, k=64, ws_bytes=ws, wsp=FAKE, q=FAKE):
+        return L.csa2_index_full(cache or _cache(), q, FAKE, FAKE, FAKE, FAKE, B, max_len, P, k, FAKE, FAKE, None,
+                                 wsp, ws_bytes, None)
+
+    assert call(P=0) == -1 and call(k=4096) == -1 and call(B=-1) == -1
+    assert call(cache=_cache(rows=1001)) == -1                 # capacity not a multiple of 8
+    assert call(cache=_cache(codes=FAKE + 4)) == -1            # misaligned
+    assert call(q=0) == -1                                     # null pointer
+    assert call(wsp=FAKE + 64) == -1                           # workspace not 256-aligned
+    assert call(ws_bytes=ws - 1) == -3
+    assert call(B=0) == 0                                      # nothing to do
+    assert b"workspace" in L.csa2_last_error()
+
+
+def test_other_calls_validation():
+    L = C.lib()
+    assert L.csa2_index_reindex(_cache(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, 64, FAKE, FAKE, 1 << 20, None) == -1
+    assert L.csa2_sparse_attn_decode(FAKE, _cache(), FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, 0.1, FAKE, None, 2, FAKE,
+                                     1 << 30, None) == -1
+    assert L.csa2_sparse_attn_decode(FAKE, _cache(), FAKE, FAKE, FAKE, 512, FAKE, FAKE, FAKE, 0.1, FAKE, None, 2, FAKE,
+                                     16, None) == -3
+    # ratio 3, and ratio 2 without logits, and both / neither indexer sources
+    base = [_cache(), _cache(), FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, 1]
+    assert L.csa2_compress_append(*base, 3, 10, 5, FAKE, 256, None) == -1
+    b2 = list(base)
+    b2[3] = None
+    assert L.csa2_compress_append(*b2, 2, 10, 5, FAKE, 256, None) == -1
+    b3 = list(base)
+    b3[4] = FAKE
+    assert L.csa2_compress_append(*b3, 2, 10, 5, FAKE, 256, None) == -1
+    assert L.csa2_index_prefill(_cache(), FAKE, FAKE, FAKE, FAKE, 4, 0, 100, 2, 64, 512, FAKE, FAKE, FAKE, 1 << 30,
+                                None) == -2                    # pool smaller than k
+    assert L.csa2_index_prefill(_cache(rows=64), FAKE, FAKE, FAKE, FAKE, 4, 0, 100, 2, 64, 64, FAKE, FAKE, FAKE,
+                                1 << 30, None) == -1           # entries beyond the capacity
+    assert L.csa2_sparse_attn_prefill(FAKE, FAKE, 4, _cache(), 0, 100, 3, FAKE, 512, FAKE, 300, 0.1, 0.1, FAKE, None,
+                                      FAKE, 1 << 30, None) == -1
+
+
+def test_workspace_sizes_grow_with_the_problem():
+    L = C.lib()
+    a = L.csa2_index_full_workspace_bytes(4, 1 << 16, 2048, 512)
+    b = L.csa2_index_full_workspace_bytes(8, 1 << 16, 2048, 512)
+    assert 256 < a < b and a % 256 == 0
+    assert L.csa2_index_full_workspace_bytes(1, 8192, 256, 512) > L.csa2_index_full_workspace_bytes(1, 8192, 512, 512)
+    assert L.csa2_sparse_attn_decode_workspace_bytes(64, 512) >= 64 * 5 * (16 * 512 + 32) * 4

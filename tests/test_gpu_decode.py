@@ -1,0 +1,94 @@
+"""End-to-end decode steps (layer patterns F / FRRU / (FRURU)x) on the GPU
+against the oracle's own step: pools and Top-k bit-exact, attention within
+tolerance.  Includes the full-size configurations (sampled for the 1M one)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth.workloads as W
+from long_context_decode_csa2_b200 import csa2 as C
+from long_context_decode_csa2_b200.decode import DecodeStep, FullCache
+from tests._gpu import check_attention, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _device_layers(layers):
+    keys = ("q", "q_codes", "q_scales", "w", "win", "win_scale", "win_len")
+    return [{k: dev(L[k]) for k in keys} for L in layers]
+
+
+def _run_and_compare(wl, full_rescan=False, host_caches=True):
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    fulls = wl.full_layers()
+    caches_h = [W.full_cache_host(wl, f, layers[f]["q_codes"], layers[f]["q_scales"]) for f in fulls]
+    caches_d = [FullCache(C.cache(dev(c["idx_codes"]), dev(c["idx_scales"])),
+                          C.cache(dev(c["main_codes"]), dev(c["main_scales"]))) for c in caches_h]
+    off = caches_h[0]["seq_row_off"]
+    lens = wl.lengths.astype(np.int32)
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, full_rescan=full_rescan)
+    dl = _device_layers(layers)
+    off_d, len_d = dev(off), dev(lens)
+    step.run(caches_d, off_d, len_d, dl)
+    torch.cuda.synchronize()
+    assert step.device_flags() == 0
+    ref = oracle.decode_step(wl.pattern, caches_h, off, lens, layers, wl.P, wl.k, 1 / math.sqrt(512),
+                             full_rescan=full_rescan)
+    for layer in range(len(wl.pattern)):
+        assert np.array_equal(host(step.topk[layer]), ref["topk"][layer]), f"layer {layer} Top-k"
+        check_attention(host(step.out[layer]), ref["out"][layer], host(step.lse[layer]), ref["lse"][layer],
+                        what=f"layer {layer}")
+    first_full = wl.full_layers()[0]
+    assert np.array_equal(host(step.pool), ref["pools"][max(ref["pools"])])
+    return step, ref
+
+
+def test_decode_tiny_config():
+    _run_and_compare(W.decode_workloads()["tiny_decode_b1_l8192"])
+
+
+def test_decode_stack_reduced():
+    wl = W.DecodeWorkload("stack_small", np.array([131072, 50001, 9000, 333, 8]), "FRRU", needles=64)
+    _run_and_compare(wl)
+
+
+@pytest.mark.parametrize("rescan", [False, True])
+def test_decode_ragged_reduced(rescan):
+    wl = W.DecodeWorkload("ragged_small", np.array([4096, 65536, 7777, 20000, 4100, 33333]), "FRURU" * 2,
+                          needles=32, lognormal=True)
+    _run_and_compare(wl, full_rescan=rescan)
+
+
+def test_decode_stack_full_size():
+    _run_and_compare(W.decode_workloads()["stack_decode_b32_l128k"])
+
+
+def test_decode_long_full_size_sampled():
+    """B=64, L=2^20, F R R U: the whole batch runs on the GPU; three sequences
+    are recomputed by the oracle (their cache rows copied back from the device
+    generator, which equals the NumPy generator byte for byte)."""
+    wl = W.decode_workloads()["long_decode_b64_l1m"]
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    c = W.full_cache_device(wl, 0, layers[0]["q_codes"], layers[0]["q_scales"])
+    cache = FullCache(C.cache(c["idx_codes"], c["idx_scales"]), C.cache(c["main_codes"], c["main_scales"]))
+    off = c["seq_row_off"]
+    lens = wl.lengths.astype(np.int32)
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
+    step.run([cache], dev(off), dev(lens), _device_layers(layers))
+    torch.cuda.synchronize()
+    assert step.device_flags() == 0
+    for b in (0, 37, 63):
+        o, L = int(off[b]), int(lens[b])
+        ch = dict(idx_codes=host(c["idx_codes"][o:o + L]), idx_scales=host(c["idx_scales"][o:o + L]),
+                  main_codes=host(c["main_codes"][o:o + L]), main_scales=host(c["main_scales"][o:o + L]))
+        lb = [{k: (v[b:b + 1] if isinstance(v, np.ndarray) and v.ndim >= 1 and v.shape[0] == wl.B else v)
+               for k, v in L_.items()} for L_ in layers]
+        ref = oracle.decode_step(wl.pattern, [ch], np.array([0]), np.array([L], np.int32), lb, wl.P, wl.k,
+                                 1 / math.sqrt(512))
+        for layer in range(4):
+            assert np.array_equal(host(step.topk[layer][b:b + 1]), ref["topk"][layer]), (b, layer)
+            check_attention(host(step.out[layer][b:b + 1]), ref["out"][layer], what=f"seq {b} layer {layer}")
+        assert np.array_equal(host(step.pool[b:b + 1]), ref["pools"][0])

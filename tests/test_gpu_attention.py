@@ -88,7 +88,7 @@ def test_attention_prefill_window_matches_oracle():
     rng = np.random.default_rng(12)
     n_raw, ratio, k, T = 3000, 2, 512, 9
     n_ent = n_raw // ratio
-    mc, ms = synth.mxfp4_rows(4, synth.T_MAIN_CODES, synth.T_MAIN_SCALES, 0, 0, 0, n_ent, 512)
+    mc, ms = synth.mxfp4_rows(4, synth.T_MAIN_CODES, synth.T_MAIN_SCALES, 0, 0, 0, (n_ent + 7) // 8 * 8, 512)
     raw_win = synth.e4m3_rows(4, synth.T_RAWWIN, 0, 0, 0, n_raw)
     q_pos = np.array([0, 1, 2, 126, 127, 128, 255, 1500, 2999], np.int32)
     q = synth.normal_bf16(4, synth.T_Q, 0, 0, T * 8192).reshape(T, 16, 512)

@@ -220,6 +220,32 @@ csa2_status csa2_sparse_attn_prefill(const uint16_t* q, const int32_t* q_pos, in
                                      float* out, float* lse, void* workspace, size_t workspace_bytes,
                                      void* stream);
 
+/* ---------------------------------------------------------------------------
+ * csa2_sparse_attn_decode_noalloc -- csa2_sparse_attn_decode without a
+ * workspace, for callers that may not allocate device memory while they run
+ * (for example a plugin inside another inference runtime that owns all
+ * allocations, or a serving loop held to a fixed memory budget).  The pages
+ * have no counterpart of this call; it is a deployment convenience.
+ * Same arguments, results and accuracy as csa2_sparse_attn_decode, except:
+ *   - no workspace: the scratch is a fixed 10,527,232-byte array of device
+ *     memory inside this library, which every GPU that loads the library keeps
+ *     until the process exits; the call allocates nothing;
+ *   - limits: B <= 64 and k <= 512; larger problems return
+ *     CSA2_ERR_UNSUPPORTED with a message, and nothing is launched;
+ *   - flags_out: device uint32 that receives this call's CSA2_DEV_* flags, or
+ *     NULL;
+ *   - the first call on a device looks up the scratch's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture;
+ *   - all calls on a device share the one scratch array: calls that may run
+ *     at the same time on the GPU (different streams, or different host
+ *     threads) race and corrupt each other's results.  Serialise them.
+ * ------------------------------------------------------------------------- */
+csa2_status csa2_sparse_attn_decode_noalloc(const uint16_t* q, csa2_mxfp4_cache main_kv, const int64_t* seq_row_off,
+                                            const int32_t* seq_len, const int32_t* topk, int k, const uint8_t* win,
+                                            const float* win_scale, const int32_t* win_len, float sm_scale,
+                                            float* out, float* lse, uint32_t* flags_out, int B, void* stream);
+
 /* Synchronises `stream`, returns the status word of `workspace` in *flags
  * (CSA2_DEV_* bits) and clears it.  Returns CSA2_ERR_DEVICE_CHECK when any
  * flag was set, CSA2_OK otherwise.  Test and debugging helper. */

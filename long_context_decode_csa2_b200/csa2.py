@@ -56,6 +56,7 @@ def lib():
             "csa2_index_prefill": (I, [Cache, P, P, P, P, I, I64, I64, I, I, I, P, P, P, Z, P]),
             "csa2_sparse_attn_prefill_workspace_bytes": (Z, [I, I]),
             "csa2_sparse_attn_prefill": (I, [P, P, I, Cache, I64, I64, I, P, I, P, I64, F, F, P, P, P, Z, P]),
+            "csa2_sparse_attn_decode_noalloc": (I, [P, Cache, P, P, P, I, P, P, P, F, P, P, P, I, P]),
             "csa2_device_status": (I, [P, P, C.POINTER(C.c_uint32)]),
             "csa2_status_string": (C.c_char_p, [I]),
             "csa2_last_error": (C.c_char_p, []),
@@ -203,3 +204,16 @@ def csa2_sparse_attn_prefill(q, q_pos, main_kv, row0, n_entries, ratio, topk, ra
                                         _ptr(raw_win), raw_win.shape[0], float(win_scale), float(sm_scale), _ptr(out),
                                         _ptr(lse), wp, wn, _stream(stream))
     _check(rc, "csa2_sparse_attn_prefill")
+
+
+def csa2_sparse_attn_decode_noalloc(q, main_kv, seq_row_off, seq_len, topk, win, win_scale, win_len, sm_scale, out,
+                                    lse=None, flags_out=None, stream=None):
+    """csa2_sparse_attn_decode without a workspace (fixed library scratch; B <= 64, k <= 512).
+
+    For callers that may not allocate device memory while they run.  All calls
+    on one device share the scratch, so calls that overlap on the GPU race."""
+    B, k = topk.shape
+    rc = lib().csa2_sparse_attn_decode_noalloc(_ptr(q), main_kv, _ptr(seq_row_off), _ptr(seq_len), _ptr(topk), k,
+                                               _ptr(win), _ptr(win_scale), _ptr(win_len), float(sm_scale), _ptr(out),
+                                               _ptr(lse), _ptr(flags_out), B, _stream(stream))
+    _check(rc, "csa2_sparse_attn_decode_noalloc")

@@ -41,6 +41,7 @@ def parse():
     ap.add_argument("--workload", default="long_decode_b64_l1m")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling captures)")
     return ap.parse_args()
 
 
@@ -214,6 +215,9 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
 
     wl = W.decode_workloads()[args.workload]
+    if args.batch:
+        wl = W.DecodeWorkload(wl.name + f"_b{args.batch}", wl.lengths[:args.batch], wl.pattern, wl.P, wl.k,
+                              wl.needles, wl.lognormal, wl.seed)
     wl, layers, caches_dev, caches, layers_dev, off_d, len_d = build_workload(wl, rank, device)
     C.lib()
     step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)

@@ -75,6 +75,7 @@ typedef int csa2_status;
 #define CSA2_DEV_ROW_LAYOUT 2u     /* seq_row_off not a multiple of 8, or rows past the capacity; sequence skipped */
 #define CSA2_DEV_FP16_RANGE 4u     /* an attention operand lies outside the fp16-exact range; output invalid */
 #define CSA2_DEV_LENGTH 8u         /* a device length exceeded the host bound (max_len / n_entries); clamped */
+#define CSA2_DEV_TIMEOUT 16u       /* a pipeline wait inside a kernel gave up after its time limit; output invalid */
 
 /* One MXFP4 cache (main KV: n = 512, indexer K: n = 128).  `rows` is the
  * capacity in rows (multiple of 8).  Pointers must be 16-byte aligned. */

@@ -44,6 +44,7 @@ bool cache_ok(const csa2_mxfp4_cache& c) {
 struct IndexFullWs {
   uint32_t* status;
   int32_t* seg_eff;
+  int32_t* tile_start;
   uint32_t* bkeys;
   uint32_t* ckeys;
   float* scores;
@@ -55,6 +56,7 @@ IndexFullWs index_full_ws(void* ws, int B, int max_len, int P, int k, bool need_
   IndexFullWs w;
   w.status = c.take<uint32_t>(kStatusBytes / 4);
   w.seg_eff = c.take<int32_t>(size_t(B));
+  w.tile_start = c.take<int32_t>(scan_tc_prefix_ints(B));
   const size_t nb = (size_t(max_len) + kBlk - 1) / kBlk;
   w.bkeys = c.take<uint32_t>(size_t(B) * nb);
   w.ckeys = (P >= k) ? c.take<uint32_t>(size_t(B) * P * kBlk) : nullptr;
@@ -123,8 +125,9 @@ csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, cons
   SegDesc sd{seq_row_off, 0, seq_len, max_len, idx_k.rows};
   const int64_t nb = (int64_t(max_len) + kBlk - 1) / kBlk;
   float* scores = scores_out ? scores_out : ws.scores;
-  launch_seg_check(sd, B, ws.seg_eff, ws.status, st);
-  launch_scan(idx_k.codes, idx_k.scales, sd, ws.seg_eff, B, q_codes, q_scales, w, ws.bkeys, nb, scores, max_len, st);
+  const csa2_status rc = launch_scan_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, ws.tile_start, B, q_codes, q_scales,
+                                        w, ws.bkeys, nb, scores, max_len, ws.status, st);
+  if (rc != CSA2_OK) return rc;
   launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, st);
   if (pool_blocks >= k) {
     // Every Top-k position's block ranks within the first k blocks, so the

@@ -58,6 +58,14 @@ void launch_scan(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& s
                  int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w, uint32_t* bkeys,
                  int64_t nb_stride, float* scores, int64_t score_stride, cudaStream_t st);
 
+// Tensor-core scan (tcgen05 + TMA): segment checks, work-item prefix
+// (tile_start [S+1]), block keys and optional scores.
+size_t scan_tc_prefix_ints(int S);
+csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, int32_t* seg_eff,
+                           int32_t* tile_start, int S, const uint8_t* q_codes, const uint8_t* q_scales,
+                           const float* w, uint32_t* bkeys, int64_t nb_stride, float* scores, int64_t score_stride,
+                           uint32_t* status, cudaStream_t st);
+
 // Scores of pool candidates 8*pool[s][i/8] + i%8 -> keys [S][P*8] (0 = absent).
 void launch_pool_score(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
                        int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,

@@ -1,0 +1,452 @@
+// Full-context indexer scan on the 5th-generation tensor cores (sm_100a).
+//
+// Score definition: "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache
+// Compression", section "三个方向一起压小缓存" (FP4 indexer q/k, block maxima over
+// 8 positions); see csa2.h for the exact rounding rules.
+//
+// One persistent CTA per SM walks a contiguous range of work items; an item
+// is 256 consecutive positions of one sequence.  Per item:
+//   * warp 0 (producer) loads the 256 x 64-byte code rows with one TMA tile
+//     copy (64-byte swizzle), the 256 x 4-byte E8M0 scales with one bulk copy,
+//     and writes the item's B operand: the sequence's indexer query laid out
+//     "one 32-element block per output column" (column 4h+b holds head h's
+//     block b, zeros elsewhere), so that each output is a single block dot;
+//   * warp 1 issues four tcgen05.mma kind::mxf4 (M=128 positions, N=16,
+//     K=64) with every block scale = 1: each accumulator is D/4 for an exact
+//     integer |D| <= 4608, i.e. exact in fp32;
+//   * warps 2-5 read the 16 accumulators of each position from TMEM, apply
+//     the E8M0 scales exactly (fp32 when the block exponents are close, else
+//     the same fp64 sum as the definition), combine the heads with the fp32
+//     fma chain, turn scores into rank keys and reduce every 8 positions to
+//     their maximum.
+// Stages are recycled through mbarriers (smem ring of 8, TMEM ring of 4).
+// Every wait is time-bounded; on a timeout the kernel sets CSA2_DEV_TIMEOUT,
+// drains its own copies and MMAs, frees TMEM and returns.
+#include <mutex>
+
+#include "device_common.cuh"
+#include "sm100.cuh"
+
+namespace csa2 {
+
+namespace {
+
+constexpr int kTile = 256;             // positions per work item
+constexpr int kStages = 8;             // smem ring
+constexpr int kAcc = 4;                // TMEM accumulator ring (32 columns each)
+constexpr int kTmemCols = 256;         // 128 accumulator + 64 scale-factor columns used
+constexpr uint32_t kSfCol = 128;       // scale factors (all 0x7F = 2^0) live here
+constexpr int kThreads = 192;          // producer, MMA, 4 epilogue warps
+constexpr uint32_t kCodeBytes = kTile * kIdxCodeBytes;  // 16384
+
+struct __align__(1024) ScanSmem {
+  uint8_t a[kStages][kCodeBytes];      // code rows, 64-byte swizzled
+  uint8_t bop[kStages][1024];          // B operand: 16 rows x 64 bytes, swizzled
+  uint32_t sc[kStages][kTile];         // E8M0 scale words
+  int2 info[kStages];                  // (sequence, tile index)
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull[kAcc];
+  uint64_t tempty[kAcc];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct ScanParams {
+  const uint8_t* kscales;
+  const uint8_t* q_codes;
+  const uint8_t* q_scales;
+  const float* w;
+  const int64_t* row_off;
+  const int32_t* seg_eff;
+  const int32_t* tile_start;  // [S+1]
+  int S;
+  uint32_t* bkeys;
+  int64_t nb_stride;
+  float* scores;
+  int64_t score_stride;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ int find_seq(const int32_t* tile_start, int S, int item) {
+  int lo = 0, hi = S;  // tile_start[lo] <= item < tile_start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(tile_start + mid) <= item) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void abort_kernel(ScanSmem& sm, uint32_t* status) {
+  set_status(status, CSA2_DEV_TIMEOUT);
+  atomicExch(&sm.abort_flag, 1);
+}
+
+__device__ __forceinline__ bool aborted(ScanSmem& sm) {
+  return *reinterpret_cast<volatile int*>(&sm.abort_flag) != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_scan_tc(const __grid_constant__ CUtensorMap tmap, ScanParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  ScanSmem& sm = *reinterpret_cast<ScanSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int n_items = __ldg(p.tile_start + p.S);
+  const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
+  const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      sm100::mbar_init(&sm.full[s], 1);
+      sm100::mbar_init(&sm.empty[s], 1 + 4);
+    }
+    for (int a = 0; a < kAcc; ++a) {
+      sm100::mbar_init(&sm.tfull[a], 1);
+      sm100::mbar_init(&sm.tempty[a], 4);
+    }
+    sm100::mbar_init(&sm.done, 1);
+    sm.abort_flag = 0;
+    sm100::fence_mbar_init();
+    sm100::tma_prefetch_desc(&tmap);
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc(&sm.tmem_base, kTmemCols);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  // unit block scales for both operands: fill 64 scale-factor columns with 0x7F
+  if (warp >= 2) {
+    const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
+#pragma unroll
+    for (int c = 0; c < 64; c += 8) sm100::tmem_st8_same(tmem + lane_base + kSfCol + c, 0x7F7F7F7Fu);
+    sm100::tmem_st_wait();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int last_round[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) last_round[s] = -1;
+    if (i0 < i1) {
+      int b = find_seq(p.tile_start, p.S, i0);
+      int next_start = __ldg(p.tile_start + b + 1);
+      int qb = -1;
+      uint2 qreg = make_uint2(0, 0);
+      int built[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) built[s] = -1;
+      for (int it = i0; it < i1; ++it) {
+        const int t = it - i0, s = t % kStages, round = t / kStages;
+        while (it >= next_start) {
+          ++b;
+          next_start = __ldg(p.tile_start + b + 1);
+        }
+        const int j = it - __ldg(p.tile_start + b);
+        const bool ok = round == 0 || sm100::mbar_wait(&sm.empty[s], (round - 1) & 1);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) abort_kernel(sm, p.status);
+          break;
+        }
+        if (__any_sync(0xffffffffu, aborted(sm))) break;
+        if (built[s] != b) {
+          if (qb != b) {
+            qreg = __ldg(reinterpret_cast<const uint2*>(p.q_codes + int64_t(b) * kHi * 64) + lane);
+            qb = b;
+          }
+          // B operand image: row n = 4*head + block; its chunk `block` holds
+          // the head's 32 codes of that block, the other chunks are zero.
+          uint8_t* bo = sm.bop[s];
+          *reinterpret_cast<uint4*>(bo + lane * 32) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(bo + lane * 32 + 16) = make_uint4(0, 0, 0, 0);
+          __syncwarp();
+          const int head = lane >> 3, part = lane & 7, blk = part >> 1;
+          const int n = head * 4 + blk;
+          const int phys = n * 64 + ((blk ^ ((n >> 1) & 3)) << 4) + (part & 1) * 8;
+          *reinterpret_cast<uint2*>(bo + phys) = qreg;
+          built[s] = b;
+        }
+        sm100::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          sm.info[s] = make_int2(b, j);
+          const int64_t L = p.seg_eff[b];
+          const int64_t rem_rows = L - int64_t(j) * kTile;
+          const int rows_valid = rem_rows < kTile ? int(rem_rows) : kTile;
+          const uint32_t sbytes = uint32_t((rows_valid + 7) & ~7) * 4u;
+          const int64_t row0 = p.row_off[b] + int64_t(j) * kTile;
+          sm100::mbar_arrive_expect_tx(&sm.full[s], kCodeBytes + sbytes);
+          sm100::tma_load_2d(sm.a[s], &tmap, 0, int32_t(row0), &sm.full[s]);
+          sm100::bulk_load(sm.sc[s], p.kscales + row0 * 4, sbytes, &sm.full[s]);
+        }
+        last_round[s] = round;
+      }
+    }
+    // drain: every copy this warp issued has landed before the CTA exits
+    if (lane == 0)
+      for (int s = 0; s < kStages; ++s)
+        if (last_round[s] >= 0 && !sm100::mbar_wait(&sm.full[s], last_round[s] & 1, 200000000ull))
+          set_status(p.status, CSA2_DEV_TIMEOUT);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = sm100::idesc_mxf4(128, 16);
+      const uint32_t sfa = tmem + kSfCol, sfb = tmem + kSfCol + 32;
+      for (int it = i0; it < i1; ++it) {
+        const int t = it - i0, s = t % kStages, a = t % kAcc;
+        if (!sm100::mbar_wait(&sm.full[s], (t / kStages) & 1)) {
+          abort_kernel(sm, p.status);
+          break;
+        }
+        if (t >= kAcc && !sm100::mbar_wait(&sm.tempty[a], ((t / kAcc) - 1) & 1)) {
+          abort_kernel(sm, p.status);
+          break;
+        }
+        if (aborted(sm)) break;
+        sm100::tc_fence_after();
+        const uint32_t abase = sm100::smem_u32(sm.a[s]);
+        const uint32_t bbase = sm100::smem_u32(sm.bop[s]);
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            sm100::mma_mxf4(tmem + a * 32 + half * 16, sm100::smem_desc_k64b(abase + half * 8192 + kk * 32),
+                            sm100::smem_desc_k64b(bbase + kk * 32), idesc, uint32_t(kk), sfa, sfb);
+        sm100::mma_commit(&sm.empty[s]);
+        sm100::mma_commit(&sm.tfull[a]);
+      }
+      // all MMAs of this CTA complete before TMEM is released
+      sm100::mma_commit(&sm.done);
+      if (!sm100::mbar_wait(&sm.done, 0, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int g = warp & 3;  // TMEM lane quarter of this warp
+    const uint32_t lane_base = uint32_t(32 * g) << 16;
+    int cur = -1;
+    int64_t L = 0;
+    uint32_t qsh[kHi][4];
+    int qlo = 0, qhi = 0, qspread = 0;
+    float wv[kHi];
+    for (int it = i0; it < i1; ++it) {
+      const int t = it - i0, s = t % kStages, a = t % kAcc;
+      const bool ok = sm100::mbar_wait(&sm.full[s], (t / kStages) & 1) && sm100::mbar_wait(&sm.tfull[a], (t / kAcc) & 1);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) abort_kernel(sm, p.status);
+        break;
+      }
+      if (__any_sync(0xffffffffu, aborted(sm))) break;
+      sm100::tc_fence_after();
+      const int2 inf = sm.info[s];
+      if (inf.x != cur) {
+        cur = inf.x;
+        L = p.seg_eff[cur];
+        qlo = 255;
+        qhi = 0;
+        qspread = 0;
+#pragma unroll
+        for (int h = 0; h < kHi; ++h) {
+          int mn = 255, mx = 0;
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) {
+            const int q = p.q_scales[int64_t(cur) * 16 + h * 4 + bb];
+            qsh[h][bb] = uint32_t(q - 127) << 23;
+            mn = min(mn, q);
+            mx = max(mx, q);
+          }
+          qlo = min(qlo, mn);
+          qhi = max(qhi, mx);
+          qspread = max(qspread, mx - mn);
+          wv[h] = p.w[int64_t(cur) * kHi + h];
+        }
+      }
+      const uint32_t sw0 = sm.sc[s][32 * g + lane];
+      const uint32_t sw1 = sm.sc[s][128 + 32 * g + lane];
+      uint32_t v[2][16];
+      sm100::tmem_ld16(tmem + lane_base + a * 32, v[0]);
+      sm100::tmem_ld16(tmem + lane_base + a * 32 + 16, v[1]);
+      sm100::tmem_ld_wait();
+      sm100::tc_fence_before();
+      sm100::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        sm100::mbar_arrive(&sm.empty[s]);
+        sm100::mbar_arrive(&sm.tempty[a]);
+      }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int64_t pos = int64_t(inf.y) * kTile + half * 128 + 32 * g + lane;
+        const uint32_t sw = half ? sw1 : sw0;
+        float sc = 0.0f;
+        uint32_t key = 0;
+        if (pos < L) {
+          const int k0 = int(sw & 255u), k1 = int((sw >> 8) & 255u), k2 = int((sw >> 16) & 255u),
+                    k3 = int(sw >> 24);
+          const int kmin = min(min(k0, k1), min(k2, k3)), kmax = max(max(k0, k1), max(k2, k3));
+          const bool fast = (kmax - kmin + qspread <= 9) && (qlo + kmin - 254 >= -100) && (qhi + kmax - 254 <= 100);
+          const uint32_t ksh[4] = {uint32_t(k0) << 23, uint32_t(k1) << 23, uint32_t(k2) << 23, uint32_t(k3) << 23};
+          float d[kHi];
+          if (fast) {
+            // every term and partial sum is exact in fp32
+#pragma unroll
+            for (int h = 0; h < kHi; ++h) {
+              float acc = __fmul_rn(__uint_as_float(v[half][4 * h]), __uint_as_float(qsh[h][0] + ksh[0]));
+#pragma unroll
+              for (int bb = 1; bb < 4; ++bb)
+                acc = __fmaf_rn(__uint_as_float(v[half][4 * h + bb]), __uint_as_float(qsh[h][bb] + ksh[bb]), acc);
+              d[h] = acc;
+            }
+          } else {
+            const int kb[4] = {k0, k1, k2, k3};
+#pragma unroll
+            for (int h = 0; h < kHi; ++h) {
+              double acc = 0.0;
+#pragma unroll
+              for (int bb = 0; bb < 4; ++bb) {
+                const int e = int(int32_t(qsh[h][bb]) >> 23) + kb[bb] - 127;  // eq + ek
+                acc = __dadd_rn(acc, __dmul_rn(double(__uint_as_float(v[half][4 * h + bb])), pow2d(e)));
+              }
+              d[h] = __double2float_rn(acc);
+            }
+          }
+          sc = __fmul_rn(wv[0], d[0]);
+#pragma unroll
+          for (int h = 1; h < kHi; ++h) sc = __fmaf_rn(wv[h], d[h], sc);
+          if (sc == 0.0f) sc = 0.0f;
+          key = rank_key(sc);
+          if (p.scores) p.scores[int64_t(cur) * p.score_stride + pos] = sc;
+        }
+        key = group8_max(key);
+        if ((lane & 7) == 0 && pos < L) p.bkeys[int64_t(cur) * p.nb_stride + pos / kBlk] = key;
+      }
+    }
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Effective lengths and the exclusive prefix of work items per segment
+// (one CTA of 1024 threads, any S).
+__global__ void __launch_bounds__(1024) k_seg_prep(SegDesc sd, int S, int32_t* seg_eff, int32_t* tile_start,
+                                                    uint32_t* status) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int base = 0; base < S; base += 1024) {
+    const int s = base + threadIdx.x;
+    int32_t ntile = 0;
+    if (s < S) {
+      int64_t L = sd.len[s];
+      const int64_t off = sd.row_off ? sd.row_off[s] : sd.row0;
+      if (L < 0) L = 0;
+      if (L > sd.max_len) {
+        set_status(status, CSA2_DEV_LENGTH);
+        L = sd.max_len;
+      }
+      if ((off & 7) != 0 || off < 0 || off + L > sd.cache_rows) {
+        set_status(status, CSA2_DEV_ROW_LAYOUT);
+        L = 0;
+      }
+      seg_eff[s] = int32_t(L);
+      ntile = int32_t((L + kTile - 1) / kTile);
+    }
+    int32_t x = ntile;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      const int32_t ws = warp_sums[lane];
+      int32_t z = ws;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, z, o);
+        if (lane >= o) z += y;
+      }
+      warp_sums[lane] = z - ws;
+    }
+    __syncthreads();
+    const int32_t excl = carry + warp_sums[wid] + x - ntile;
+    if (s < S) tile_start[s] = excl;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry = excl + ntile;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) tile_start[S] = carry;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+}  // namespace
+
+size_t scan_tc_prefix_ints(int S) { return size_t(S) + 1; }
+
+csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, int32_t* seg_eff,
+                           int32_t* tile_start, int S, const uint8_t* q_codes, const uint8_t* q_scales,
+                           const float* w, uint32_t* bkeys, int64_t nb_stride, float* scores, int64_t score_stride,
+                           uint32_t* status, cudaStream_t st) {
+  if (S == 0) return CSA2_OK;
+  k_seg_prep<<<1, 1024, 0, st>>>(sd, S, seg_eff, tile_start, status);
+  if (sd.max_len == 0) return CSA2_OK;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {cuuint64_t(kIdxCodeBytes), cuuint64_t(sd.cache_rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(kIdxCodeBytes)};
+  const cuuint32_t box[2] = {cuuint32_t(kIdxCodeBytes), cuuint32_t(kTile)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(kcodes), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled failed for the indexer-K codes");
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t smem = sizeof(ScanSmem) + 1024;
+  cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  ScanParams p{kscales, q_codes, q_scales, w, sd.row_off, seg_eff, tile_start, S, bkeys, nb_stride, scores,
+               score_stride, status};
+  // the host cannot see the item count; cap the grid by an upper bound of it
+  const int64_t max_items = int64_t(S) * ((sd.max_len + kTile - 1) / kTile);
+  const int grid = int(std::min<int64_t>(sms, std::max<int64_t>(max_items, 1)));
+  k_scan_tc<<<grid, kThreads, smem, st>>>(map, p);
+  return CSA2_OK;
+}
+
+}  // namespace csa2

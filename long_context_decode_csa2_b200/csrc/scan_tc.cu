@@ -5,21 +5,22 @@
 // 8 positions); see csa2.h for the exact rounding rules.
 //
 // One persistent CTA per SM walks a contiguous range of work items; an item
-// is 256 consecutive positions of one sequence.  Per item:
-//   * warp 0 (producer) loads the 256 x 64-byte code rows with one TMA tile
-//     copy (64-byte swizzle), the 256 x 4-byte E8M0 scales with one bulk copy,
+// is 512 consecutive positions of one sequence.  Per item:
+//   * warp 0 (producer) loads the 512 x 64-byte code rows with two TMA tile
+//     copies (64-byte swizzle), the 512 x 4-byte E8M0 scales with one bulk copy,
 //     and writes the item's B operand: the sequence's indexer query laid out
 //     "one 32-element block per output column" (column 4h+b holds head h's
 //     block b, zeros elsewhere), so that each output is a single block dot;
-//   * warp 1 issues four tcgen05.mma kind::mxf4 (M=128 positions, N=16,
+//   * warp 1 issues eight tcgen05.mma kind::mxf4 (M=128 positions, N=16,
 //     K=64) with every block scale = 1: each accumulator is D/4 for an exact
 //     integer |D| <= 4608, i.e. exact in fp32;
-//   * warps 2-5 read the 16 accumulators of each position from TMEM, apply
+//   * two teams of four epilogue warps (alternate items) read the 16
+//     accumulators of each position from TMEM, apply
 //     the E8M0 scales exactly (fp32 when the block exponents are close, else
 //     the same fp64 sum as the definition), combine the heads with the fp32
 //     fma chain, turn scores into rank keys and reduce every 8 positions to
 //     their maximum.
-// Stages are recycled through mbarriers (smem ring of 8, TMEM ring of 4).
+// Stages are recycled through mbarriers (smem ring of 4, TMEM ring of 3).
 // Every wait is time-bounded; on a timeout the kernel sets CSA2_DEV_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <mutex>
@@ -31,13 +32,18 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kTile = 256;             // positions per work item
-constexpr int kStages = 8;             // smem ring
-constexpr int kAcc = 4;                // TMEM accumulator ring (32 columns each)
-constexpr int kTmemCols = 256;         // 128 accumulator + 64 scale-factor columns used
-constexpr uint32_t kSfCol = 128;       // scale factors (all 0x7F = 2^0) live here
-constexpr int kThreads = 192;          // producer, MMA, 4 epilogue warps
-constexpr uint32_t kCodeBytes = kTile * kIdxCodeBytes;  // 16384
+constexpr int kTile = 512;             // positions per work item
+constexpr int kMT = kTile / 128;       // 128-row MMA tiles per item
+constexpr int kStages = 4;             // smem ring
+constexpr int kAcc = 3;                // TMEM accumulator ring (16 columns per MMA tile)
+constexpr int kAccCols = 16 * kMT;
+constexpr int kTmemCols = 256;
+constexpr uint32_t kSfCol = 192;       // scale factors (all 0x7F = 2^0) live here
+constexpr int kEpiTeams = 2;           // epilogue teams of 4 warps, items round-robin
+constexpr int kThreads = 64 + 128 * kEpiTeams;  // producer, MMA, epilogue warps
+constexpr uint32_t kCodeBytes = kTile * kIdxCodeBytes;
+constexpr int kBoxRows = 256;          // TMA box height limit
+static_assert(kAcc * kAccCols <= int(kSfCol), "TMEM accumulators overlap the scale factors");
 
 struct __align__(1024) ScanSmem {
   uint8_t a[kStages][kCodeBytes];      // code rows, 64-byte swizzled
@@ -51,6 +57,7 @@ struct __align__(1024) ScanSmem {
   uint64_t done;
   uint32_t tmem_base;
   int abort_flag;
+  int built[kStages];                  // sequence whose B operand each stage holds
 };
 
 struct ScanParams {
@@ -123,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
 
   // unit block scales for both operands: fill 64 scale-factor columns with 0x7F
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 6) {
     const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
 #pragma unroll
     for (int c = 0; c < 64; c += 8) sm100::tmem_st8_same(tmem + lane_base + kSfCol + c, 0x7F7F7F7Fu);
@@ -135,31 +142,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    int last_round[kStages];
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) last_round[s] = -1;
+    int issued = 0;
+    if (lane < kStages) sm.built[lane] = -1;
+    __syncwarp();
     if (i0 < i1) {
+      // per-sequence values live in registers; global loads only when the
+      // sequence changes
       int b = find_seq(p.tile_start, p.S, i0);
-      int next_start = __ldg(p.tile_start + b + 1);
+      int seq_start = __ldg(p.tile_start + b), next_start = __ldg(p.tile_start + b + 1);
+      int64_t seq_off = p.row_off[b];
+      int64_t seq_len = p.seg_eff[b];
       int qb = -1;
       uint2 qreg = make_uint2(0, 0);
-      int built[kStages];
-#pragma unroll
-      for (int s = 0; s < kStages; ++s) built[s] = -1;
       for (int it = i0; it < i1; ++it) {
         const int t = it - i0, s = t % kStages, round = t / kStages;
         while (it >= next_start) {
           ++b;
+          seq_start = next_start;
           next_start = __ldg(p.tile_start + b + 1);
+          seq_off = p.row_off[b];
+          seq_len = p.seg_eff[b];
         }
-        const int j = it - __ldg(p.tile_start + b);
+        const int j = it - seq_start;
         const bool ok = round == 0 || sm100::mbar_wait(&sm.empty[s], (round - 1) & 1);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) abort_kernel(sm, p.status);
           break;
         }
         if (__any_sync(0xffffffffu, aborted(sm))) break;
-        if (built[s] != b) {
+        if (sm.built[s] != b) {
           if (qb != b) {
             qreg = __ldg(reinterpret_cast<const uint2*>(p.q_codes + int64_t(b) * kHi * 64) + lane);
             qb = b;
@@ -174,29 +185,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = head * 4 + blk;
           const int phys = n * 64 + ((blk ^ ((n >> 1) & 3)) << 4) + (part & 1) * 8;
           *reinterpret_cast<uint2*>(bo + phys) = qreg;
-          built[s] = b;
+          sm100::fence_proxy_async_smem();  // generic writes -> MMA (async proxy) reads
+          __syncwarp();
+          if (lane == 0) sm.built[s] = b;
         }
-        sm100::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           sm.info[s] = make_int2(b, j);
-          const int64_t L = p.seg_eff[b];
-          const int64_t rem_rows = L - int64_t(j) * kTile;
+          const int64_t rem_rows = seq_len - int64_t(j) * kTile;
           const int rows_valid = rem_rows < kTile ? int(rem_rows) : kTile;
           const uint32_t sbytes = uint32_t((rows_valid + 7) & ~7) * 4u;
-          const int64_t row0 = p.row_off[b] + int64_t(j) * kTile;
+          const int64_t row0 = seq_off + int64_t(j) * kTile;
           sm100::mbar_arrive_expect_tx(&sm.full[s], kCodeBytes + sbytes);
-          sm100::tma_load_2d(sm.a[s], &tmap, 0, int32_t(row0), &sm.full[s]);
+#pragma unroll
+          for (int bx = 0; bx < kTile / kBoxRows; ++bx)
+            sm100::tma_load_2d(sm.a[s] + bx * kBoxRows * kIdxCodeBytes, &tmap, 0, int32_t(row0 + bx * kBoxRows),
+                               &sm.full[s]);
           sm100::bulk_load(sm.sc[s], p.kscales + row0 * 4, sbytes, &sm.full[s]);
         }
-        last_round[s] = round;
+        ++issued;
       }
     }
     // drain: every copy this warp issued has landed before the CTA exits
     if (lane == 0)
-      for (int s = 0; s < kStages; ++s)
-        if (last_round[s] >= 0 && !sm100::mbar_wait(&sm.full[s], last_round[s] & 1, 200000000ull))
-          set_status(p.status, CSA2_DEV_TIMEOUT);
+      for (int s = 0; s < kStages && s < issued; ++s) {
+        const int last_round = (issued - 1 - s) / kStages;
+        if (!sm100::mbar_wait(&sm.full[s], last_round & 1, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
+      }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -217,10 +232,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t abase = sm100::smem_u32(sm.a[s]);
         const uint32_t bbase = sm100::smem_u32(sm.bop[s]);
 #pragma unroll
-        for (int half = 0; half < 2; ++half)
+        for (int half = 0; half < kMT; ++half)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            sm100::mma_mxf4(tmem + a * 32 + half * 16, sm100::smem_desc_k64b(abase + half * 8192 + kk * 32),
+            sm100::mma_mxf4(tmem + a * kAccCols + half * 16, sm100::smem_desc_k64b(abase + half * 8192 + kk * 32),
                             sm100::smem_desc_k64b(bbase + kk * 32), idesc, uint32_t(kk), sfa, sfb);
         sm100::mma_commit(&sm.empty[s]);
         sm100::mma_commit(&sm.tfull[a]);
@@ -233,13 +248,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int g = warp & 3;  // TMEM lane quarter of this warp
+    const int team = (warp - 2) >> 2;
     const uint32_t lane_base = uint32_t(32 * g) << 16;
     int cur = -1;
     int64_t L = 0;
     uint32_t qsh[kHi][4];
     int qlo = 0, qhi = 0, qspread = 0;
     float wv[kHi];
-    for (int it = i0; it < i1; ++it) {
+    for (int it = i0 + team; it < i1; it += kEpiTeams) {
       const int t = it - i0, s = t % kStages, a = t % kAcc;
       const bool ok = sm100::mbar_wait(&sm.full[s], (t / kStages) & 1) && sm100::mbar_wait(&sm.tfull[a], (t / kAcc) & 1);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -271,11 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           wv[h] = p.w[int64_t(cur) * kHi + h];
         }
       }
-      const uint32_t sw0 = sm.sc[s][32 * g + lane];
-      const uint32_t sw1 = sm.sc[s][128 + 32 * g + lane];
-      uint32_t v[2][16];
-      sm100::tmem_ld16(tmem + lane_base + a * 32, v[0]);
-      sm100::tmem_ld16(tmem + lane_base + a * 32 + 16, v[1]);
+      uint32_t swv[kMT];
+      uint32_t v[kMT][16];
+#pragma unroll
+      for (int half = 0; half < kMT; ++half) {
+        swv[half] = sm.sc[s][128 * half + 32 * g + lane];
+        sm100::tmem_ld16(tmem + lane_base + a * kAccCols + half * 16, v[half]);
+      }
       sm100::tmem_ld_wait();
       sm100::tc_fence_before();
       sm100::fence_proxy_async_smem();
@@ -285,9 +303,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm100::mbar_arrive(&sm.tempty[a]);
       }
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < kMT; ++half) {
         const int64_t pos = int64_t(inf.y) * kTile + half * 128 + 32 * g + lane;
-        const uint32_t sw = half ? sw1 : sw0;
+        const uint32_t sw = swv[half];
         float sc = 0.0f;
         uint32_t key = 0;
         if (pos < L) {
@@ -429,7 +447,7 @@ csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
   CUtensorMap map;
   const cuuint64_t dims[2] = {cuuint64_t(kIdxCodeBytes), cuuint64_t(sd.cache_rows)};
   const cuuint64_t strides[1] = {cuuint64_t(kIdxCodeBytes)};
-  const cuuint32_t box[2] = {cuuint32_t(kIdxCodeBytes), cuuint32_t(kTile)};
+  const cuuint32_t box[2] = {cuuint32_t(kIdxCodeBytes), cuuint32_t(kBoxRows)};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(kcodes), dims, strides, box,
                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,

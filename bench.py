@@ -340,7 +340,7 @@ def run_ours(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "int32+f64 indexer / f32 attention",
+            "dtype": "int32+f64 indexer, f16 tensor-core attention (f32 accumulate)",
             "data": "synthetic",
             "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len, "layers": wl.pattern,
                        "pool_blocks": wl.P, "topk": wl.k, "window": 128,

@@ -328,7 +328,9 @@ def run_ours(args):
         launches_per_step = 0
         for _, m in enumerate(step.plan):
             act = m[3]
-            launches_per_step += {"scan": 5, "reindex": 3, "reuse": 0}[act] + 3
+            # index_full: prep, scan, pool select, pool score, Top-k select;
+            # reindex: check, pool score, select; attention: check + one kernel
+            launches_per_step += {"scan": 5, "reindex": 3, "reuse": 0}[act] + 2
         res = {
             "metric": METRIC,
             "value": world * wl.B / (ms * 1e-3),

@@ -186,6 +186,7 @@ size_t csa2_sparse_attn_decode_workspace_bytes(int B, int k) {
   Carve c(nullptr);
   c.take<uint32_t>(kStatusBytes / 4);
   c.take<int32_t>(size_t(B));
+  c.take<int32_t>(size_t(B));
   c.take<char>(attn_partial_bytes(B, k));
   return c.used;
 }
@@ -208,6 +209,7 @@ csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv,
   AttnArgs a{};
   a.status = c.take<uint32_t>(kStatusBytes / 4);
   int32_t* seg_eff = c.take<int32_t>(size_t(B));
+  a.counters = c.take<int32_t>(size_t(B));
   a.partial = reinterpret_cast<float*>(c.take<char>(attn_partial_bytes(B, k)));
   a.q = q;
   a.mcodes = main_kv.codes;
@@ -343,6 +345,7 @@ size_t csa2_sparse_attn_prefill_workspace_bytes(int T, int k) {
   Carve c(nullptr);
   c.take<uint32_t>(kStatusBytes / 4);
   c.take<int32_t>(size_t(T));
+  c.take<int32_t>(size_t(T));
   c.take<char>(attn_partial_bytes(T, k));
   return c.used;
 }
@@ -369,6 +372,7 @@ csa2_status csa2_sparse_attn_prefill(const uint16_t* q, const int32_t* q_pos, in
   AttnArgs a{};
   a.status = c.take<uint32_t>(kStatusBytes / 4);
   int32_t* vis = c.take<int32_t>(size_t(T));
+  a.counters = c.take<int32_t>(size_t(T));
   a.partial = reinterpret_cast<float*>(c.take<char>(attn_partial_bytes(T, k)));
   a.q = q;
   a.mcodes = main_kv.codes;

@@ -11,7 +11,8 @@
 //   S = Q K^T  (16 heads x 128 keys),  P = exp(S*scale - max),  O = P V.
 // The window's fp32 scale multiplies its logits and its partial output in
 // fp32, never the fp16 values.  Each CTA writes an unnormalised partial
-// (O, max, sum) per head; a second kernel combines the chunks in a fixed order.
+// (O, max, sum) per head; the last CTA of each segment to finish combines the
+// chunks in a fixed order (deterministic) and resets the segment's counter.
 #include <cuda_fp16.h>
 
 #include "device_common.cuh"
@@ -36,30 +37,28 @@ struct AttnSmem {
   float red_max[8][kHq];
   float red_sum[8][kHq];
   int valid[kChunk];
+  float fac[CSA2_MAX_TOPK / kChunk + 1][kHq];
+  int last;
 };
 
-// fp16 bit patterns of the E2M1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}
-__device__ __forceinline__ uint32_t e2m1_half_bits(uint32_t code) {
-  const uint32_t lo = 0x3E003C00u, hi = 0x46004400u;  // 1.5|1, 6|4
-  const uint32_t mag = code & 7u;
-  uint32_t bits;
-  if (mag < 2) bits = mag ? 0x3800u : 0u;
-  else if (mag < 4) bits = (mag == 2) ? (lo & 0xFFFFu) : (lo >> 16);
-  else if (mag < 6) bits = (mag == 4) ? 0x4000u : 0x4200u;
-  else bits = (mag == 6) ? (hi & 0xFFFFu) : (hi >> 16);
-  return bits | ((code & 8u) << 12);
+// Two E2M1 codes (low nibble = lower element) -> f16x2, exact.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tmov.b16 {t, _}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "h"(uint16_t(byte)));
+  return r;
+}
+// Two E4M3 bytes (low byte = lower element) -> f16x2, exact.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(uint32_t two) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(uint16_t(two)));
+  return r;
 }
 
-// OCP E4M3 -> fp16 bits (exact: 3 mantissa bits, exponent -9 .. 8).
-__device__ __forceinline__ uint32_t e4m3_half_bits(uint32_t b) {
-  const uint32_t s = (b & 0x80u) << 8, e = (b >> 3) & 15u, m = b & 7u;
-  uint32_t bits;
-  if (e == 0) {
-    bits = m ? __half_as_ushort(__float2half_rn(float(m) * 0.001953125f)) : 0u;  // m * 2^-9, exact
-  } else {
-    bits = ((e + 8u) << 10) | (m << 7);  // exponent bias 7 -> 15
-  }
-  return bits | s;
+// Packed f16x2 multiply on raw 32-bit registers (round to nearest).
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t x, uint32_t y) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(y));
+  return r;
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
@@ -80,47 +79,11 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(kAttnThreads) k_attn_partial(AttnArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
-  const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
+__device__ __forceinline__ void attn_chunk(const AttnArgs& a, AttnSmem& sm, float* part, int s, int c, int nkeys,
+                                           bool is_win, float kscale, const uint8_t* win_base, int64_t eff,
+                                           int64_t off) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int nmain = (a.k + kChunk - 1) / kChunk;
-  const bool is_win = (c == nmain);
-  const int64_t eff = a.seg_eff[s];
-  const int64_t off = a.sd.row_off ? a.sd.row_off[s] : a.sd.row0;
-  float* part = a.partial + (int64_t(s) * gridDim.x + c) * kPartFloats;
-
-  int nkeys;
-  float kscale = 1.0f;
-  const uint8_t* win_base = nullptr;
-  if (!is_win) {
-    nkeys = min(kChunk, a.k - c * kChunk);
-  } else if (a.q_pos == nullptr) {
-    nkeys = max(0, min(kWin, a.win_len[s]));
-    kscale = a.win_scale[s];
-    win_base = a.win + int64_t(s) * kWin * kD;
-  } else {
-    int64_t p = a.q_pos[s];
-    if (p >= a.n_raw) {
-      set_status(a.status, CSA2_DEV_LENGTH);
-      p = a.n_raw - 1;
-    }
-    const int64_t lo = p - (kWin - 1) > 0 ? p - (kWin - 1) : 0;
-    nkeys = p >= 0 ? int(p - lo + 1) : 0;
-    kscale = a.raw_scale;
-    win_base = a.raw_win + lo * kD;
-  }
-  if (nkeys == 0) {
-    for (int i = tid; i < kHq * kD; i += kAttnThreads) part[i] = 0.0f;
-    if (tid < kHq) {
-      part[kHq * kD + tid] = -INFINITY;
-      part[kHq * kD + kHq + tid] = 0.0f;
-    }
-    return;
-  }
-
   // Q: bf16 -> fp16 (exact for |q| in [2^-14, 65504]; smaller values keep 2^-24 resolution)
   for (int i = tid; i < kHq * kD / 2; i += kAttnThreads) {
     const uint32_t w2 = reinterpret_cast<const uint32_t*>(a.q + int64_t(s) * kHq * kD)[i];
@@ -130,64 +93,86 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_partial(AttnArgs a) {
     *reinterpret_cast<__half2*>(&sm.q[h][d]) = __floats2half2_rn(lo, hi);
   }
   // keys: thread -> one row r (lanes on consecutive rows, which keeps the
-  // shared-memory stores conflict-free) and 8 of its 16 blocks
+  // shared-memory stores conflict-free) and blocks b = tid/128 + 2i; all of
+  // a thread's loads are issued before any conversion
   const int r = tid & (kChunk - 1);
+  constexpr int kBPT = 16 / (kAttnThreads / kChunk);  // blocks per thread (8)
   int64_t tpos = -1;
   if (!is_win && r < nkeys) {
     tpos = a.topk[int64_t(s) * a.k + c * kChunk + r];
     if (tpos >= eff) {
-      if (tid < kChunk) set_status(a.status, CSA2_DEV_INDEX_RANGE);
+      set_status(a.status, CSA2_DEV_INDEX_RANGE);
       tpos = -1;
     }
   }
   const bool row_ok = (r < nkeys) && (is_win || tpos >= 0);
   if (tid < kChunk) sm.valid[r] = row_ok;
-  for (int b = tid >> 7; b < 16; b += kAttnThreads / kChunk) {
-    const bool ok = row_ok;
-    uint4 out[4];
-    if (!is_win) {
-      if (ok) {
-        const int64_t row = off + tpos;
-        const uint4 cw = __ldg(reinterpret_cast<const uint4*>(a.mcodes + row * kMainCodeBytes) + b);
-        const uint32_t sb = a.mscales[row * kMainScaleBytes + b];
-        // fp16-exact iff the block exponent X = sb - 127 lies in [-23, 13]
-        if (sb < 104u || sb > 140u) set_status(a.status, CSA2_DEV_FP16_RANGE);
-        const int X = int(sb) - 127;
-        const __half2 sc2 = __half2half2(__ushort_as_half(
-            X >= -14 ? uint16_t((X + 15) << 10) : uint16_t(1u << (X + 24 > 0 ? X + 24 : 0))));
-        const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
-        uint32_t hv[16];
+  const int b0 = tid / kChunk;
+  if (!is_win) {
+    uint4 cw[kBPT];
+    uint32_t sbv[kBPT];
+    if (row_ok) {
+      const int64_t row = off + tpos;
+      const uint4* cp = reinterpret_cast<const uint4*>(a.mcodes + row * kMainCodeBytes);
+      const uint8_t* sp = a.mscales + row * kMainScaleBytes;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int n = 0; n < 4; ++n) {
-            const uint32_t c0 = (w4[q] >> (8 * n)) & 15u, c1 = (w4[q] >> (8 * n + 4)) & 15u;
-            const uint32_t pair = e2m1_half_bits(c0) | (e2m1_half_bits(c1) << 16);
-            const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&pair), sc2);
-            hv[4 * q + n] = *reinterpret_cast<const uint32_t*>(&v);
-          }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) out[q] = make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+      for (int i = 0; i < kBPT; ++i) {
+        cw[i] = __ldg(cp + b0 + 2 * i);
+        sbv[i] = __ldg(sp + b0 + 2 * i);
       }
-    } else if (ok) {
-      const uint4* src = reinterpret_cast<const uint4*>(win_base + int64_t(r) * kD + 32 * b);
-      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-      const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      uint32_t hv[16];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        hv[2 * q] = e4m3_half_bits(w8[q] & 255u) | (e4m3_half_bits((w8[q] >> 8) & 255u) << 16);
-        hv[2 * q + 1] = e4m3_half_bits((w8[q] >> 16) & 255u) | (e4m3_half_bits(w8[q] >> 24) << 16);
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) out[q] = make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
     }
-    if (!ok)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) out[q] = make_uint4(0, 0, 0, 0);
-    uint4* dst = reinterpret_cast<uint4*>(&sm.kv[r][32 * b]);
+    for (int i = 0; i < kBPT; ++i) {
+      const int b = b0 + 2 * i;
+      uint4* dst = reinterpret_cast<uint4*>(&sm.kv[r][32 * b]);
+      if (!row_ok) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = out[q];
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      // fp16-exact iff the block exponent X = byte - 127 lies in [-23, 13]
+      const uint32_t sb = sbv[i];
+      if (sb < 104u || sb > 140u) set_status(a.status, CSA2_DEV_FP16_RANGE);
+      const int X = int(sb) - 127;
+      const uint16_t xb = X >= -14 ? uint16_t((X + 15) << 10) : uint16_t(1u << (X + 24 > 0 ? X + 24 : 0));
+      const uint32_t sc2 = uint32_t(xb) | (uint32_t(xb) << 16);
+      const uint32_t w4[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t hv[4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          hv[n] = hmul2_u32(cvt_e2m1x2((w4[q] >> (8 * n)) & 255u), sc2);
+        }
+        dst[q] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      }
+    }
+  } else {
+    uint4 wv[kBPT][2];
+    if (row_ok) {
+      const uint4* src = reinterpret_cast<const uint4*>(win_base + int64_t(r) * kD);
+#pragma unroll
+      for (int i = 0; i < kBPT; ++i) {
+        wv[i][0] = __ldg(src + 2 * (b0 + 2 * i));
+        wv[i][1] = __ldg(src + 2 * (b0 + 2 * i) + 1);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kBPT; ++i) {
+      const int b = b0 + 2 * i;
+      uint4* dst = reinterpret_cast<uint4*>(&sm.kv[r][32 * b]);
+      if (!row_ok) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      const uint32_t w8[8] = {wv[i][0].x, wv[i][0].y, wv[i][0].z, wv[i][0].w,
+                              wv[i][1].x, wv[i][1].y, wv[i][1].z, wv[i][1].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dst[q] = make_uint4(cvt_e4m3x2(w8[2 * q] & 0xFFFFu), cvt_e4m3x2(w8[2 * q] >> 16),
+                            cvt_e4m3x2(w8[2 * q + 1] & 0xFFFFu), cvt_e4m3x2(w8[2 * q + 1] >> 16));
+    }
   }
   __syncthreads();
 
@@ -303,35 +288,90 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_partial(AttnArgs a) {
   }
 }
 
-// Combine the chunk partials of one segment in chunk order.  grid = S,
-// block = 512 (thread = output dim); per-head factors computed once in smem.
-__global__ void __launch_bounds__(512) k_attn_combine(AttnArgs a, int nchunks) {
-  constexpr int kMaxChunks = CSA2_MAX_TOPK / kChunk + 1;
-  __shared__ float fac[kMaxChunks][kHq];  // exp(m_c - M) / L per chunk and head
-  __shared__ float lse_s[kHq];
-  const int s = blockIdx.x, d = threadIdx.x;
+// Last-arriving CTA of a segment: combine the chunk partials in chunk order
+// (deterministic), write out / lse, and reset the segment's arrival counter.
+__device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm, int s) {
+  const int tid = threadIdx.x;
+  const int nchunks = gridDim.x;
+  __threadfence();  // this thread's partial is visible before the arrival below
+  __syncthreads();
+  if (tid == 0) sm.last = (atomicAdd(a.counters + s, 1) == nchunks - 1);
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
   const float* base = a.partial + int64_t(s) * nchunks * kPartFloats;
-  if (d < kHq) {
+  if (tid < kHq) {
     float M = -INFINITY;
-    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, base[c * kPartFloats + kHq * kD + d]);
+    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, __ldcg(base + c * kPartFloats + kHq * kD + tid));
     float L = 0.0f;
     for (int c = 0; c < nchunks; ++c) {
-      const float mc = base[c * kPartFloats + kHq * kD + d];
+      const float mc = __ldcg(base + c * kPartFloats + kHq * kD + tid);
       const float f = (mc == -INFINITY) ? 0.0f : __expf(mc - M);
-      fac[c][d] = f;
-      L += base[c * kPartFloats + kHq * kD + kHq + d] * f;
+      sm.fac[c][tid] = f;
+      L += __ldcg(base + c * kPartFloats + kHq * kD + kHq + tid) * f;
     }
-    for (int c = 0; c < nchunks; ++c) fac[c][d] = (M == -INFINITY) ? 0.0f : fac[c][d] / L;
-    lse_s[d] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+    for (int c = 0; c < nchunks; ++c) sm.fac[c][tid] = (M == -INFINITY) ? 0.0f : sm.fac[c][tid] / L;
+    if (a.lse) a.lse[int64_t(s) * kHq + tid] = (M == -INFINITY) ? -INFINITY : M + logf(L);
   }
   __syncthreads();
-#pragma unroll 4
-  for (int h = 0; h < kHq; ++h) {
-    float o = 0.0f;
-    for (int c = 0; c < nchunks; ++c) o = fmaf(base[c * kPartFloats + h * kD + d], fac[c][h], o);
-    a.out[(int64_t(s) * kHq + h) * kD + d] = o;
+  for (int i = tid; i < kHq * kD / 4; i += kAttnThreads) {
+    const int h = (4 * i) / kD;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < nchunks; ++c) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(base + c * kPartFloats) + i);
+      const float f = sm.fac[c][h];
+      o.x = fmaf(v.x, f, o.x);
+      o.y = fmaf(v.y, f, o.y);
+      o.z = fmaf(v.z, f, o.z);
+      o.w = fmaf(v.w, f, o.w);
+    }
+    reinterpret_cast<float4*>(a.out + int64_t(s) * kHq * kD)[i] = o;
   }
-  if (a.lse && d < kHq) a.lse[int64_t(s) * kHq + d] = lse_s[d];
+  if (tid == 0) a.counters[s] = 0;
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
+  const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int nmain = (a.k + kChunk - 1) / kChunk;
+  const bool is_win = (c == nmain);
+  const int64_t eff = a.seg_eff[s];
+  const int64_t off = a.sd.row_off ? a.sd.row_off[s] : a.sd.row0;
+  float* part = a.partial + (int64_t(s) * gridDim.x + c) * kPartFloats;
+
+  int nkeys;
+  float kscale = 1.0f;
+  const uint8_t* win_base = nullptr;
+  if (!is_win) {
+    nkeys = min(kChunk, a.k - c * kChunk);
+  } else if (a.q_pos == nullptr) {
+    nkeys = max(0, min(kWin, a.win_len[s]));
+    kscale = a.win_scale[s];
+    win_base = a.win + int64_t(s) * kWin * kD;
+  } else {
+    int64_t p = a.q_pos[s];
+    if (p >= a.n_raw) {
+      set_status(a.status, CSA2_DEV_LENGTH);
+      p = a.n_raw - 1;
+    }
+    const int64_t lo = p - (kWin - 1) > 0 ? p - (kWin - 1) : 0;
+    nkeys = p >= 0 ? int(p - lo + 1) : 0;
+    kscale = a.raw_scale;
+    win_base = a.raw_win + lo * kD;
+  }
+  if (nkeys == 0) {
+    for (int i = tid; i < kHq * kD; i += kAttnThreads) part[i] = 0.0f;
+    if (tid < kHq) {
+      part[kHq * kD + tid] = -INFINITY;
+      part[kHq * kD + kHq + tid] = 0.0f;
+    }
+  } else {
+    attn_chunk(a, sm, part, s, c, nkeys, is_win, kscale, win_base, eff, off);
+  }
+  combine_if_last(a, sm, s);
 }
 
 void launch_attention(const AttnArgs& a, cudaStream_t st) {
@@ -340,7 +380,6 @@ void launch_attention(const AttnArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(AttnSmem);
   cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   k_attn_partial<<<dim3(nchunks, a.S), kAttnThreads, smem, st>>>(a);
-  k_attn_combine<<<a.S, 512, 0, st>>>(a, nchunks);
 }
 
 }  // namespace csa2

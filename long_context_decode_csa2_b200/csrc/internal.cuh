@@ -113,6 +113,7 @@ struct AttnArgs {
   float* out;                   // [S][16][512]
   float* lse;                   // [S][16] or null
   float* partial;               // workspace
+  int32_t* counters;            // [S] arrival counters, zero between calls
   uint32_t* status;
   int S;
 };

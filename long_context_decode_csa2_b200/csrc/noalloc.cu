@@ -22,11 +22,13 @@ constexpr int kNoAllocMaxSeqs = 64;
 constexpr int kNoAllocMaxTopk = 512;
 constexpr size_t kNoAllocStatusBytes = 256;                       // device status word
 constexpr size_t kNoAllocSeqBytes = 256;                          // 64 visible counts
+constexpr size_t kNoAllocCounterBytes = 256;                      // 64 arrival counters (self-resetting)
 constexpr size_t kNoAllocPartialBytes =                           // split-KV partials
     size_t(kNoAllocMaxSeqs) * (kNoAllocMaxTopk / 128 + 1) * (kHq * kD + 2 * kHq) * sizeof(float);
-constexpr size_t kNoAllocScratchBytes = kNoAllocStatusBytes + kNoAllocSeqBytes + kNoAllocPartialBytes;
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocStatusBytes + kNoAllocSeqBytes + kNoAllocCounterBytes + kNoAllocPartialBytes;
 
-// The scratch: 10,527,232 bytes of device memory that every GPU which loads
+// The scratch: 10,527,488 bytes of device memory that every GPU which loads
 // this library keeps until the process exits.  All calls on a device share it
 // and it keeps whatever the last call left in it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -89,9 +91,11 @@ extern "C" csa2_status csa2_sparse_attn_decode_noalloc(const uint16_t* q, csa2_m
   AttnArgs a{};
   a.status = reinterpret_cast<uint32_t*>(p);
   int32_t* seg_eff = reinterpret_cast<int32_t*>(p + kNoAllocStatusBytes);
-  a.partial = reinterpret_cast<float*>(p + kNoAllocStatusBytes + kNoAllocSeqBytes);
-  // The status word must start at zero for this call; nothing else does
-  // (visible counts and partials are fully written before they are read).
+  a.counters = reinterpret_cast<int32_t*>(p + kNoAllocStatusBytes + kNoAllocSeqBytes);
+  a.partial = reinterpret_cast<float*>(p + kNoAllocStatusBytes + kNoAllocSeqBytes + kNoAllocCounterBytes);
+  // The status word must start at zero for this call.  The arrival counters
+  // are zero when the library loads and every call leaves them at zero; the
+  // visible counts and partials are fully written before they are read.
   cudaError_t e = cudaMemsetAsync(a.status, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return fail(CSA2_ERR_CUDA, std::string(fn) + ": " + cudaGetErrorString(e));
   a.q = q;

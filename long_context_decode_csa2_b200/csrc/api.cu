@@ -132,8 +132,9 @@ csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, cons
   if (pool_blocks >= k) {
     // Every Top-k position's block ranks within the first k blocks, so the
     // Top-k over the pool equals the Top-k over all positions.
-    launch_pool_score(idx_k.codes, idx_k.scales, sd, ws.seg_eff, B, q_codes, q_scales, w, pool_out, pool_blocks,
-                      ws.ckeys, ws.status, st);
+    const csa2_status rc2 = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, B, q_codes, q_scales, w,
+                                           pool_out, pool_blocks, ws.ckeys, ws.status, st);
+    if (rc2 != CSA2_OK) return rc2;
     launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.seg_eff, B, pool_blocks, pool_out, k,
                   topk_out, st);
   } else {
@@ -175,8 +176,9 @@ csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SegDesc sd{seq_row_off, 0, seq_len, INT32_MAX, idx_k.rows};
   launch_seg_check(sd, B, seg_eff, status, st);
-  launch_pool_score(idx_k.codes, idx_k.scales, sd, seg_eff, B, q_codes, q_scales, w, pool, pool_blocks, ckeys,
-                    status, st);
+  const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, seg_eff, B, q_codes, q_scales, w, pool,
+                                        pool_blocks, ckeys, status, st);
+  if (rc != CSA2_OK) return rc;
   launch_select(kSelPoolCand, ckeys, int64_t(pool_blocks) * kBlk, seg_eff, B, pool_blocks, pool, k, topk_out, st);
   return check_launch(fn);
 }
@@ -333,8 +335,9 @@ csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
   launch_prefill_scan(idx_k.codes, idx_k.scales, row0, ws.vis, T, n_entries, q_codes, q_scales, w, ws.bkeys, nb, st);
   launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, T, 0, nullptr, pool_blocks, pool_out, st);
   SegDesc sd{nullptr, row0, ws.vis, n_entries, idx_k.rows};
-  launch_pool_score(idx_k.codes, idx_k.scales, sd, ws.vis, T, q_codes, q_scales, w, pool_out, pool_blocks, ws.ckeys,
-                    ws.status, st);
+  const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.vis, T, q_codes, q_scales, w, pool_out,
+                                        pool_blocks, ws.ckeys, ws.status, st);
+  if (rc != CSA2_OK) return rc;
   launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.vis, T, pool_blocks, pool_out, k, topk_out,
                 st);
   return check_launch(fn);

@@ -43,20 +43,11 @@ struct SegDesc {
   int64_t cache_rows;      // capacity of the cache
 };
 
-// Prepared FP4 indexer query for CUDA-core scoring.
-struct IdxQueryPrep;
-
 // ---------------------------------------------------------------------------
 // Kernel launchers (each returns after enqueueing on `st`).
 // ---------------------------------------------------------------------------
 // Effective length per segment after layout checks -> seg_eff [S].
 void launch_seg_check(const SegDesc& sd, int S, int32_t* seg_eff, uint32_t* status, cudaStream_t st);
-
-// Decode scan over all visible positions: block keys [S][nb_stride] and
-// optional scores [S][max_len].
-void launch_scan(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
-                 int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w, uint32_t* bkeys,
-                 int64_t nb_stride, float* scores, int64_t score_stride, cudaStream_t st);
 
 // Tensor-core scan (tcgen05 + TMA): segment checks, work-item prefix
 // (tile_start [S+1]), block keys and optional scores.
@@ -66,10 +57,11 @@ csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
                            const float* w, uint32_t* bkeys, int64_t nb_stride, float* scores, int64_t score_stride,
                            uint32_t* status, cudaStream_t st);
 
-// Scores of pool candidates 8*pool[s][i/8] + i%8 -> keys [S][P*8] (0 = absent).
-void launch_pool_score(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
-                       int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
-                       const int32_t* pool, int P, uint32_t* ckeys, uint32_t* status, cudaStream_t st);
+// Scores of pool candidates 8*pool[s][i/8] + i%8 -> keys [S][P*8] (0 = absent),
+// on the tensor cores (gathered 8-row TMA boxes).
+csa2_status launch_pool_tc(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
+                           int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                           const int32_t* pool, int P, uint32_t* ckeys, uint32_t* status, cudaStream_t st);
 
 // Prefill scan: block keys [T][nb_stride] for every query against the visible
 // prefix of one sequence.

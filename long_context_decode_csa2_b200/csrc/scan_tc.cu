@@ -1,25 +1,30 @@
-// Full-context indexer scan on the 5th-generation tensor cores (sm_100a).
+// Indexer scoring on the 5th-generation tensor cores (sm_100a): the
+// full-context scan (block maxima) and the pool-candidate scoring (one key per
+// candidate) share one kernel.
 //
 // Score definition: "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache
 // Compression", section "三个方向一起压小缓存" (FP4 indexer q/k, block maxima over
-// 8 positions); see csa2.h for the exact rounding rules.
+// 8 positions, candidate pool of 2048 blocks x 8); see csa2.h for the exact
+// rounding rules.
 //
 // One persistent CTA per SM walks a contiguous range of work items; an item
-// is 512 consecutive positions of one sequence.  Per item:
-//   * warp 0 (producer) loads the 512 x 64-byte code rows with two TMA tile
-//     copies (64-byte swizzle), the 512 x 4-byte E8M0 scales with one bulk copy,
-//     and writes the item's B operand: the sequence's indexer query laid out
-//     "one 32-element block per output column" (column 4h+b holds head h's
-//     block b, zeros elsewhere), so that each output is a single block dot;
+// is 512 positions of one segment: 512 consecutive rows (scan) or the rows of
+// 64 pool blocks (pool scoring).  Per item:
+//   * warp 0 (producer) loads the 64-byte code rows with TMA tile copies
+//     (64-byte swizzle; two 256-row boxes for the scan, sixty-four 8-row boxes
+//     gathered by the 32 lanes for the pool), the 4-byte E8M0 scale words
+//     with bulk copies, and writes the item's B operand: the segment's
+//     indexer query laid out "one 32-element block per output column" (column
+//     4h+b holds head h's block b, zeros elsewhere);
 //   * warp 1 issues eight tcgen05.mma kind::mxf4 (M=128 positions, N=16,
 //     K=64) with every block scale = 1: each accumulator is D/4 for an exact
 //     integer |D| <= 4608, i.e. exact in fp32;
 //   * two teams of four epilogue warps (alternate items) read the 16
-//     accumulators of each position from TMEM, apply
-//     the E8M0 scales exactly (fp32 when the block exponents are close, else
-//     the same fp64 sum as the definition), combine the heads with the fp32
-//     fma chain, turn scores into rank keys and reduce every 8 positions to
-//     their maximum.
+//     accumulators of each position from TMEM, apply the E8M0 scales exactly
+//     (fp32 when the block exponents are close, else the same fp64 sum as the
+//     definition), combine the heads with the fp32 fma chain and emit rank
+//     keys: the maximum of every 8 positions (scan) or one key per candidate
+//     (pool; 0 for absent candidates).
 // Stages are recycled through mbarriers (smem ring of 4, TMEM ring of 3).
 // Every wait is time-bounded; on a timeout the kernel sets CSA2_DEV_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
@@ -42,14 +47,16 @@ constexpr uint32_t kSfCol = 192;       // scale factors (all 0x7F = 2^0) live he
 constexpr int kEpiTeams = 2;           // epilogue teams of 4 warps, items round-robin
 constexpr int kThreads = 64 + 128 * kEpiTeams;  // producer, MMA, epilogue warps
 constexpr uint32_t kCodeBytes = kTile * kIdxCodeBytes;
-constexpr int kBoxRows = 256;          // TMA box height limit
+constexpr int kBoxRows = 256;          // TMA box height (scan)
+constexpr int kPoolSlots = kTile / kBlk;  // pool blocks per item (64)
 static_assert(kAcc * kAccCols <= int(kSfCol), "TMEM accumulators overlap the scale factors");
 
 struct __align__(1024) ScanSmem {
   uint8_t a[kStages][kCodeBytes];      // code rows, 64-byte swizzled
   uint8_t bop[kStages][1024];          // B operand: 16 rows x 64 bytes, swizzled
   uint32_t sc[kStages][kTile];         // E8M0 scale words
-  int2 info[kStages];                  // (sequence, tile index)
+  int32_t blk[kStages][kPoolSlots];    // pool mode: block id of each 8-row slot
+  int2 info[kStages];                  // (segment, item index within the segment)
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t tfull[kAcc];
@@ -57,7 +64,7 @@ struct __align__(1024) ScanSmem {
   uint64_t done;
   uint32_t tmem_base;
   int abort_flag;
-  int built[kStages];                  // sequence whose B operand each stage holds
+  int built[kStages];                  // segment whose B operand each stage holds
 };
 
 struct ScanParams {
@@ -65,14 +72,21 @@ struct ScanParams {
   const uint8_t* q_codes;
   const uint8_t* q_scales;
   const float* w;
-  const int64_t* row_off;
+  const int64_t* row_off;     // [S] or null -> row0
+  int64_t row0;
   const int32_t* seg_eff;
-  const int32_t* tile_start;  // [S+1]
+  const int32_t* tile_start;  // scan: [S+1] item prefix
   int S;
+  // scan outputs
   uint32_t* bkeys;
   int64_t nb_stride;
   float* scores;
   int64_t score_stride;
+  // pool mode
+  const int32_t* pool;        // [S][P]
+  int P;
+  int items_per_seg;
+  uint32_t* ckeys;            // [S][P*8]
   uint32_t* status;
 };
 
@@ -95,14 +109,31 @@ __device__ __forceinline__ bool aborted(ScanSmem& sm) {
   return *reinterpret_cast<volatile int*>(&sm.abort_flag) != 0;
 }
 
+__device__ __forceinline__ int64_t seg_row_off(const ScanParams& p, int s) {
+  return p.row_off ? p.row_off[s] : p.row0;
+}
+
+// Writes the B operand image of a segment's query into `bo` (whole warp).
+__device__ __forceinline__ void build_b_operand(uint8_t* bo, uint2 qreg, int lane) {
+  *reinterpret_cast<uint4*>(bo + lane * 32) = make_uint4(0, 0, 0, 0);
+  *reinterpret_cast<uint4*>(bo + lane * 32 + 16) = make_uint4(0, 0, 0, 0);
+  __syncwarp();
+  const int head = lane >> 3, part = lane & 7, blk = part >> 1;
+  const int n = head * 4 + blk;
+  const int phys = n * 64 + ((blk ^ ((n >> 1) & 3)) << 4) + (part & 1) * 8;
+  *reinterpret_cast<uint2*>(bo + phys) = qreg;
+  sm100::fence_proxy_async_smem();  // generic writes -> MMA (async proxy) reads
+}
+
+template <bool kPool>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_scan_tc(const __grid_constant__ CUtensorMap tmap, ScanParams p) {
+    k_index_tc(const __grid_constant__ CUtensorMap tmap, ScanParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   ScanSmem& sm = *reinterpret_cast<ScanSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int n_items = __ldg(p.tile_start + p.S);
+  const int n_items = kPool ? p.S * p.items_per_seg : __ldg(p.tile_start + p.S);
   const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
   const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
 
@@ -146,24 +177,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane < kStages) sm.built[lane] = -1;
     __syncwarp();
     if (i0 < i1) {
-      // per-sequence values live in registers; global loads only when the
-      // sequence changes
-      int b = find_seq(p.tile_start, p.S, i0);
-      int seq_start = __ldg(p.tile_start + b), next_start = __ldg(p.tile_start + b + 1);
-      int64_t seq_off = p.row_off[b];
+      int b, seq_start = 0, next_start = 0;
+      if (kPool) {
+        b = i0 / p.items_per_seg;
+      } else {
+        b = find_seq(p.tile_start, p.S, i0);
+        seq_start = __ldg(p.tile_start + b);
+        next_start = __ldg(p.tile_start + b + 1);
+      }
+      int64_t seq_off = seg_row_off(p, b);
       int64_t seq_len = p.seg_eff[b];
       int qb = -1;
       uint2 qreg = make_uint2(0, 0);
       for (int it = i0; it < i1; ++it) {
         const int t = it - i0, s = t % kStages, round = t / kStages;
-        while (it >= next_start) {
-          ++b;
-          seq_start = next_start;
-          next_start = __ldg(p.tile_start + b + 1);
-          seq_off = p.row_off[b];
-          seq_len = p.seg_eff[b];
+        int j;
+        if (kPool) {
+          const int nb = it / p.items_per_seg;
+          if (nb != b) {
+            b = nb;
+            seq_off = seg_row_off(p, b);
+            seq_len = p.seg_eff[b];
+          }
+          j = it - b * p.items_per_seg;
+        } else {
+          while (it >= next_start) {
+            ++b;
+            seq_start = next_start;
+            next_start = __ldg(p.tile_start + b + 1);
+            seq_off = seg_row_off(p, b);
+            seq_len = p.seg_eff[b];
+          }
+          j = it - seq_start;
         }
-        const int j = it - seq_start;
         const bool ok = round == 0 || sm100::mbar_wait(&sm.empty[s], (round - 1) & 1);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) abort_kernel(sm, p.status);
@@ -175,22 +221,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             qreg = __ldg(reinterpret_cast<const uint2*>(p.q_codes + int64_t(b) * kHi * 64) + lane);
             qb = b;
           }
-          // B operand image: row n = 4*head + block; its chunk `block` holds
-          // the head's 32 codes of that block, the other chunks are zero.
-          uint8_t* bo = sm.bop[s];
-          *reinterpret_cast<uint4*>(bo + lane * 32) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(bo + lane * 32 + 16) = make_uint4(0, 0, 0, 0);
-          __syncwarp();
-          const int head = lane >> 3, part = lane & 7, blk = part >> 1;
-          const int n = head * 4 + blk;
-          const int phys = n * 64 + ((blk ^ ((n >> 1) & 3)) << 4) + (part & 1) * 8;
-          *reinterpret_cast<uint2*>(bo + phys) = qreg;
-          sm100::fence_proxy_async_smem();  // generic writes -> MMA (async proxy) reads
+          build_b_operand(sm.bop[s], qreg, lane);
           __syncwarp();
           if (lane == 0) sm.built[s] = b;
         }
         __syncwarp();
-        if (lane == 0) {
+        if (kPool) {
+          // gather: lane handles pool slots 64j + 2*lane + {0, 1}
+          int32_t blk2[2];
+          bool v2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int slot = j * kPoolSlots + 2 * lane + u;
+            blk2[u] = slot < p.P ? __ldg(p.pool + int64_t(b) * p.P + slot) : -1;
+            const bool in_range = blk2[u] >= 0 && int64_t(blk2[u]) * kBlk < seq_len;
+            if (blk2[u] >= 0 && !in_range) set_status(p.status, CSA2_DEV_INDEX_RANGE);
+            v2[u] = in_range;
+            sm.blk[s][2 * lane + u] = in_range ? blk2[u] : -1;
+          }
+          const uint32_t nvalid =
+              __popc(__ballot_sync(0xffffffffu, v2[0])) + __popc(__ballot_sync(0xffffffffu, v2[1]));
+          __syncwarp();  // every lane's slot ids are written before the arrive
+          if (lane == 0) {
+            sm.info[s] = make_int2(b, j);
+            sm100::mbar_arrive_expect_tx(&sm.full[s], nvalid * (kBlk * kIdxCodeBytes + kBlk * 4));
+          }
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+            if (v2[u]) {
+              const int sl = 2 * lane + u;
+              const int64_t row = seq_off + int64_t(blk2[u]) * kBlk;
+              sm100::tma_load_2d(sm.a[s] + sl * kBlk * kIdxCodeBytes, &tmap, 0, int32_t(row), &sm.full[s]);
+              sm100::bulk_load(&sm.sc[s][sl * kBlk], p.kscales + row * 4, kBlk * 4, &sm.full[s]);
+            }
+        } else if (lane == 0) {
           sm.info[s] = make_int2(b, j);
           const int64_t rem_rows = seq_len - int64_t(j) * kTile;
           const int rows_valid = rem_rows < kTile ? int(rem_rows) : kTile;
@@ -257,7 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float wv[kHi];
     for (int it = i0 + team; it < i1; it += kEpiTeams) {
       const int t = it - i0, s = t % kStages, a = t % kAcc;
-      const bool ok = sm100::mbar_wait(&sm.full[s], (t / kStages) & 1) && sm100::mbar_wait(&sm.tfull[a], (t / kAcc) & 1);
+      const bool ok =
+          sm100::mbar_wait(&sm.full[s], (t / kStages) & 1) && sm100::mbar_wait(&sm.tfull[a], (t / kAcc) & 1);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) abort_kernel(sm, p.status);
         break;
@@ -288,10 +354,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       uint32_t swv[kMT];
+      int64_t posv[kMT];
       uint32_t v[kMT][16];
 #pragma unroll
       for (int half = 0; half < kMT; ++half) {
-        swv[half] = sm.sc[s][128 * half + 32 * g + lane];
+        const int pl = 128 * half + 32 * g + lane;  // position within the item
+        swv[half] = sm.sc[s][pl];
+        if (kPool) {
+          const int32_t bk = sm.blk[s][pl >> 3];
+          posv[half] = bk >= 0 ? int64_t(bk) * kBlk + (pl & 7) : int64_t(-1);
+        } else {
+          posv[half] = int64_t(inf.y) * kTile + pl;
+        }
         sm100::tmem_ld16(tmem + lane_base + a * kAccCols + half * 16, v[half]);
       }
       sm100::tmem_ld_wait();
@@ -304,15 +378,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int half = 0; half < kMT; ++half) {
-        const int64_t pos = int64_t(inf.y) * kTile + half * 128 + 32 * g + lane;
+        const int64_t pos = posv[half];
         const uint32_t sw = swv[half];
         float sc = 0.0f;
         uint32_t key = 0;
-        if (pos < L) {
+        if (pos >= 0 && pos < L) {
           const int k0 = int(sw & 255u), k1 = int((sw >> 8) & 255u), k2 = int((sw >> 16) & 255u),
                     k3 = int(sw >> 24);
           const int kmin = min(min(k0, k1), min(k2, k3)), kmax = max(max(k0, k1), max(k2, k3));
-          const bool fast = (kmax - kmin + qspread <= 9) && (qlo + kmin - 254 >= -100) && (qhi + kmax - 254 <= 100);
+          const bool fast =
+              (kmax - kmin + qspread <= 9) && (qlo + kmin - 254 >= -100) && (qhi + kmax - 254 <= 100);
           const uint32_t ksh[4] = {uint32_t(k0) << 23, uint32_t(k1) << 23, uint32_t(k2) << 23, uint32_t(k3) << 23};
           float d[kHi];
           if (fast) {
@@ -343,10 +418,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int h = 1; h < kHi; ++h) sc = __fmaf_rn(wv[h], d[h], sc);
           if (sc == 0.0f) sc = 0.0f;
           key = rank_key(sc);
-          if (p.scores) p.scores[int64_t(cur) * p.score_stride + pos] = sc;
+          if (!kPool && p.scores) p.scores[int64_t(cur) * p.score_stride + pos] = sc;
         }
-        key = group8_max(key);
-        if ((lane & 7) == 0 && pos < L) p.bkeys[int64_t(cur) * p.nb_stride + pos / kBlk] = key;
+        if (kPool) {
+          const int64_t ci = int64_t(inf.y) * kTile + 128 * half + 32 * g + lane;  // candidate index
+          if (ci < int64_t(p.P) * kBlk) p.ckeys[int64_t(cur) * p.P * kBlk + ci] = key;
+        } else {
+          key = group8_max(key);
+          if ((lane & 7) == 0 && pos < L) p.bkeys[int64_t(cur) * p.nb_stride + pos / kBlk] = key;
+        }
       }
     }
   }
@@ -431,6 +511,37 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Tensor map over the indexer-K code plane: rows of 64 bytes, box of
+// `box_rows` rows, 64-byte swizzle, out-of-range rows read as zero.
+csa2_status code_map(CUtensorMap* map, const uint8_t* kcodes, int64_t rows, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {cuuint64_t(kIdxCodeBytes), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(kIdxCodeBytes)};
+  const cuuint32_t box[2] = {cuuint32_t(kIdxCodeBytes), cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(kcodes), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled failed for the indexer-K codes");
+  return CSA2_OK;
+}
+
+int num_sms() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <bool kPool>
+void launch_index_tc(const CUtensorMap& map, const ScanParams& p, int64_t max_items, cudaStream_t st) {
+  const size_t smem = sizeof(ScanSmem) + 1024;
+  cudaFuncSetAttribute(k_index_tc<kPool>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  const int grid = int(std::min<int64_t>(num_sms(), std::max<int64_t>(max_items, 1)));
+  k_index_tc<kPool><<<grid, kThreads, smem, st>>>(map, p);
+}
+
 }  // namespace
 
 size_t scan_tc_prefix_ints(int S) { return size_t(S) + 1; }
@@ -442,28 +553,51 @@ csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
   if (S == 0) return CSA2_OK;
   k_seg_prep<<<1, 1024, 0, st>>>(sd, S, seg_eff, tile_start, status);
   if (sd.max_len == 0) return CSA2_OK;
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   CUtensorMap map;
-  const cuuint64_t dims[2] = {cuuint64_t(kIdxCodeBytes), cuuint64_t(sd.cache_rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(kIdxCodeBytes)};
-  const cuuint32_t box[2] = {cuuint32_t(kIdxCodeBytes), cuuint32_t(kBoxRows)};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(kcodes), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled failed for the indexer-K codes");
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const size_t smem = sizeof(ScanSmem) + 1024;
-  cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  ScanParams p{kscales, q_codes, q_scales, w, sd.row_off, seg_eff, tile_start, S, bkeys, nb_stride, scores,
-               score_stride, status};
+  const csa2_status rc = code_map(&map, kcodes, sd.cache_rows, kBoxRows);
+  if (rc != CSA2_OK) return rc;
+  ScanParams p{};
+  p.kscales = kscales;
+  p.q_codes = q_codes;
+  p.q_scales = q_scales;
+  p.w = w;
+  p.row_off = sd.row_off;
+  p.row0 = sd.row0;
+  p.seg_eff = seg_eff;
+  p.tile_start = tile_start;
+  p.S = S;
+  p.bkeys = bkeys;
+  p.nb_stride = nb_stride;
+  p.scores = scores;
+  p.score_stride = score_stride;
+  p.status = status;
   // the host cannot see the item count; cap the grid by an upper bound of it
-  const int64_t max_items = int64_t(S) * ((sd.max_len + kTile - 1) / kTile);
-  const int grid = int(std::min<int64_t>(sms, std::max<int64_t>(max_items, 1)));
-  k_scan_tc<<<grid, kThreads, smem, st>>>(map, p);
+  launch_index_tc<false>(map, p, int64_t(S) * ((sd.max_len + kTile - 1) / kTile), st);
+  return CSA2_OK;
+}
+
+csa2_status launch_pool_tc(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
+                           int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                           const int32_t* pool, int P, uint32_t* ckeys, uint32_t* status, cudaStream_t st) {
+  if (S == 0) return CSA2_OK;
+  CUtensorMap map;
+  const csa2_status rc = code_map(&map, kcodes, sd.cache_rows, kBlk);
+  if (rc != CSA2_OK) return rc;
+  ScanParams p{};
+  p.kscales = kscales;
+  p.q_codes = q_codes;
+  p.q_scales = q_scales;
+  p.w = w;
+  p.row_off = sd.row_off;
+  p.row0 = sd.row0;
+  p.seg_eff = seg_eff;
+  p.S = S;
+  p.pool = pool;
+  p.P = P;
+  p.items_per_seg = (P * kBlk + kTile - 1) / kTile;
+  p.ckeys = ckeys;
+  p.status = status;
+  launch_index_tc<true>(map, p, int64_t(S) * p.items_per_seg, st);
   return CSA2_OK;
 }
 

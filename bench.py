@@ -223,20 +223,21 @@ def run_ours(args):
     step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
     stream = torch.cuda.current_stream()
 
-    # events around every csa2_index_full call of the timed region (the
-    # dominant call: full-context scan, block max, pool, Top-512)
+    # events around every C-ABI call of the timed region; csa2_index_full
+    # (full-context scan, block max, pool, Top-512) is the dominant call
     n_layers = len(wl.pattern)
-    ev_full = []
+    ev_calls = {}
     recording = [False]
 
     def hook(name, phase):
-        if not recording[0] or name != "csa2_index_full":
+        if not recording[0]:
             return
+        lst = ev_calls.setdefault(name, [])
         if phase == "begin":
-            ev_full.append([torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)])
-            ev_full[-1][0].record(stream)
+            lst.append([torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)])
+            lst[-1][0].record(stream)
         else:
-            ev_full[-1][1].record(stream)
+            lst[-1][1].record(stream)
 
     step.hook = hook
 
@@ -265,7 +266,8 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1) / args.steps
-    full_ms = [a.elapsed_time(b) for a, b in ev_full]
+    per_call = {name: sum(a.elapsed_time(b) for a, b in lst) / len(lst) for name, lst in ev_calls.items()}
+    full_ms = [a.elapsed_time(b) for a, b in ev_calls["csa2_index_full"]]
     if world > 1:
         t = torch.tensor([ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -358,6 +360,7 @@ def run_ours(args):
             "e2e": {"value": world * wl.B / (e2e_ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
+            "per_call_ms": per_call,
             "clocks": clk.summary(),
             "device_flags": flags,
         }

@@ -84,13 +84,29 @@ __device__ __forceinline__ void attn_chunk(const AttnArgs& a, AttnSmem& sm, floa
                                            int64_t off) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  // Q: bf16 -> fp16 (exact for |q| in [2^-14, 65504]; smaller values keep 2^-24 resolution)
-  for (int i = tid; i < kHq * kD / 2; i += kAttnThreads) {
-    const uint32_t w2 = reinterpret_cast<const uint32_t*>(a.q + int64_t(s) * kHq * kD)[i];
-    const float lo = __uint_as_float(w2 << 16), hi = __uint_as_float(w2 & 0xFFFF0000u);
-    if (fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f) set_status(a.status, CSA2_DEV_FP16_RANGE);
-    const int h = (2 * i) / kD, d = (2 * i) % kD;
-    *reinterpret_cast<__half2*>(&sm.q[h][d]) = __floats2half2_rn(lo, hi);
+  // Q: bf16 -> fp16 (exact for |q| in [2^-14, 65504]; smaller values keep
+  // 2^-24 resolution); 8 values per 16-byte load, both loads in flight
+  {
+    constexpr int kQV = kHq * kD / 8 / kAttnThreads;  // 16-byte vectors per thread (4)
+    uint4 qv[kQV];
+    const uint4* qsrc = reinterpret_cast<const uint4*>(a.q + int64_t(s) * kHq * kD);
+#pragma unroll
+    for (int m = 0; m < kQV; ++m) qv[m] = __ldg(qsrc + tid + m * kAttnThreads);
+#pragma unroll
+    for (int m = 0; m < kQV; ++m) {
+      const int e = 8 * (tid + m * kAttnThreads);
+      const int h = e / kD, d = e % kD;
+      const uint32_t w[4] = {qv[m].x, qv[m].y, qv[m].z, qv[m].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
+        if (fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f) set_status(a.status, CSA2_DEV_FP16_RANGE);
+        const __half2 h2 = __floats2half2_rn(lo, hi);
+        o[q] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      *reinterpret_cast<uint4*>(&sm.q[h][d]) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
   // keys: thread -> one row r (lanes on consecutive rows, which keeps the
   // shared-memory stores conflict-free) and blocks b = tid/128 + 2i; all of
@@ -314,19 +330,26 @@ __device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm,
     if (a.lse) a.lse[int64_t(s) * kHq + tid] = (M == -INFINITY) ? -INFINITY : M + logf(L);
   }
   __syncthreads();
-  for (int i = tid; i < kHq * kD / 4; i += kAttnThreads) {
-    const int h = (4 * i) / kD;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < nchunks; ++c) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(base + c * kPartFloats) + i);
-      const float f = sm.fac[c][h];
-      o.x = fmaf(v.x, f, o.x);
-      o.y = fmaf(v.y, f, o.y);
-      o.z = fmaf(v.z, f, o.z);
-      o.w = fmaf(v.w, f, o.w);
+  // 8 float4 per thread; per chunk all 8 loads are independent
+  constexpr int kOV = kHq * kD / 4 / kAttnThreads;
+  float4 o[kOV];
+#pragma unroll
+  for (int m = 0; m < kOV; ++m) o[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = 0; c < nchunks; ++c) {
+    float4 v[kOV];
+#pragma unroll
+    for (int m = 0; m < kOV; ++m) v[m] = __ldcg(reinterpret_cast<const float4*>(base + c * kPartFloats) + tid + m * kAttnThreads);
+#pragma unroll
+    for (int m = 0; m < kOV; ++m) {
+      const float f = sm.fac[c][(4 * (tid + m * kAttnThreads)) / kD];
+      o[m].x = fmaf(v[m].x, f, o[m].x);
+      o[m].y = fmaf(v[m].y, f, o[m].y);
+      o[m].z = fmaf(v[m].z, f, o[m].z);
+      o[m].w = fmaf(v[m].w, f, o[m].w);
     }
-    reinterpret_cast<float4*>(a.out + int64_t(s) * kHq * kD)[i] = o;
   }
+#pragma unroll
+  for (int m = 0; m < kOV; ++m) reinterpret_cast<float4*>(a.out + int64_t(s) * kHq * kD)[tid + m * kAttnThreads] = o[m];
   if (tid == 0) a.counters[s] = 0;
 }
 

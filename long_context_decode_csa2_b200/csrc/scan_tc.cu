@@ -25,7 +25,8 @@
 //     definition), combine the heads with the fp32 fma chain and emit rank
 //     keys: the maximum of every 8 positions (scan) or one key per candidate
 //     (pool; 0 for absent candidates).
-// Stages are recycled through mbarriers (smem ring of 4, TMEM ring of 3).
+// Stages are recycled through mbarriers (smem ring of 4 for the scan, 6 for
+// the pool gather; TMEM ring of 3).
 // Every wait is time-bounded; on a timeout the kernel sets CSA2_DEV_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <mutex>
@@ -39,7 +40,13 @@ namespace {
 
 constexpr int kTile = 512;             // positions per work item
 constexpr int kMT = kTile / 128;       // 128-row MMA tiles per item
-constexpr int kStages = 4;             // smem ring
+// smem ring: 4 stages stream the contiguous scan fastest; the pool gather
+// signals a stage only kGatherDepth items after issuing it, so it needs more
+template <bool kPool>
+struct Ring {
+  static constexpr int kStages = kPool ? 6 : 4;
+  static constexpr int kGatherDepth = 3;  // gathered items in flight before signalling
+};
 constexpr int kAcc = 3;                // TMEM accumulator ring (16 columns per MMA tile)
 constexpr int kAccCols = 16 * kMT;
 constexpr int kTmemCols = 256;
@@ -51,6 +58,7 @@ constexpr int kBoxRows = 256;          // TMA box height (scan)
 constexpr int kPoolSlots = kTile / kBlk;  // pool blocks per item (64)
 static_assert(kAcc * kAccCols <= int(kSfCol), "TMEM accumulators overlap the scale factors");
 
+template <int kStages>
 struct __align__(1024) ScanSmem {
   uint8_t a[kStages][kCodeBytes];      // code rows, 64-byte swizzled
   uint8_t bop[kStages][1024];          // B operand: 16 rows x 64 bytes, swizzled
@@ -65,9 +73,11 @@ struct __align__(1024) ScanSmem {
   uint32_t tmem_base;
   int abort_flag;
   int built[kStages];                  // segment whose B operand each stage holds
+  int32_t segpool[CSA2_MAX_POOL_BLOCKS]; // pool mode: the current segment's pool block ids
 };
 
 struct ScanParams {
+  const uint8_t* kcodes;      // code plane (pool gather)
   const uint8_t* kscales;
   const uint8_t* q_codes;
   const uint8_t* q_scales;
@@ -100,12 +110,14 @@ __device__ __forceinline__ int find_seq(const int32_t* tile_start, int S, int it
   return lo;
 }
 
-__device__ __forceinline__ void abort_kernel(ScanSmem& sm, uint32_t* status) {
+template <class Smem>
+__device__ __forceinline__ void abort_kernel(Smem& sm, uint32_t* status) {
   set_status(status, CSA2_DEV_TIMEOUT);
   atomicExch(&sm.abort_flag, 1);
 }
 
-__device__ __forceinline__ bool aborted(ScanSmem& sm) {
+template <class Smem>
+__device__ __forceinline__ bool aborted(Smem& sm) {
   return *reinterpret_cast<volatile int*>(&sm.abort_flag) != 0;
 }
 
@@ -128,8 +140,11 @@ __device__ __forceinline__ void build_b_operand(uint8_t* bo, uint2 qreg, int lan
 template <bool kPool>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_tc(const __grid_constant__ CUtensorMap tmap, ScanParams p) {
+  constexpr int kStages = Ring<kPool>::kStages;
+  constexpr int kGatherDepth = Ring<kPool>::kGatherDepth;
+  using Smem = ScanSmem<kStages>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  ScanSmem& sm = *reinterpret_cast<ScanSmem*>(
+  Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -189,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t seq_len = p.seg_eff[b];
       int qb = -1;
       uint2 qreg = make_uint2(0, 0);
+      int pool_seg = -1;  // segment whose pool ids are in sm.segpool
       for (int it = i0; it < i1; ++it) {
         const int t = it - i0, s = t % kStages, round = t / kStages;
         int j;
@@ -227,34 +243,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         if (kPool) {
-          // gather: lane handles pool slots 64j + 2*lane + {0, 1}
-          int32_t blk2[2];
-          bool v2[2];
+          if (pool_seg != b) {
+            // all of the segment's pool ids at once (one round trip per segment);
+            // every stage that still holds unsignalled copies keeps its own ids
+            const int32_t* src = p.pool + int64_t(b) * p.P;
+            int32_t v[CSA2_MAX_POOL_BLOCKS / 32];
+#pragma unroll
+            for (int m = 0; m < CSA2_MAX_POOL_BLOCKS / 32; ++m) {
+              const int i = lane + 32 * m;
+              v[m] = i < p.P ? __ldg(src + i) : -1;
+            }
+#pragma unroll
+            for (int m = 0; m < CSA2_MAX_POOL_BLOCKS / 32; ++m) sm.segpool[lane + 32 * m] = v[m];
+            __syncwarp();
+            pool_seg = b;
+          }
+          // gather: block ids of the item's 64 pool slots
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int slot = j * kPoolSlots + 2 * lane + u;
-            blk2[u] = slot < p.P ? __ldg(p.pool + int64_t(b) * p.P + slot) : -1;
-            const bool in_range = blk2[u] >= 0 && int64_t(blk2[u]) * kBlk < seq_len;
-            if (blk2[u] >= 0 && !in_range) set_status(p.status, CSA2_DEV_INDEX_RANGE);
-            v2[u] = in_range;
-            sm.blk[s][2 * lane + u] = in_range ? blk2[u] : -1;
+            const int32_t bk = slot < p.P ? sm.segpool[slot] : -1;
+            const bool in_range = bk >= 0 && int64_t(bk) * kBlk < seq_len;
+            if (bk >= 0 && !in_range) set_status(p.status, CSA2_DEV_INDEX_RANGE);
+            sm.blk[s][2 * lane + u] = in_range ? bk : -1;
           }
-          const uint32_t nvalid =
-              __popc(__ballot_sync(0xffffffffu, v2[0])) + __popc(__ballot_sync(0xffffffffu, v2[1]));
-          __syncwarp();  // every lane's slot ids are written before the arrive
-          if (lane == 0) {
-            sm.info[s] = make_int2(b, j);
-            sm100::mbar_arrive_expect_tx(&sm.full[s], nvalid * (kBlk * kIdxCodeBytes + kBlk * 4));
-          }
+          if (lane == 0) sm.info[s] = make_int2(b, j);
           __syncwarp();
+          // one warp instruction per 512-byte block: lane = (row l/4, chunk l%4),
+          // destination in the 64-byte swizzle the MMA descriptor expects
+          const int r8 = lane >> 2, ch = lane & 3;
+          const int phys = r8 * 64 + ((ch ^ ((r8 >> 1) & 3)) << 4);
+          for (int sl = 0; sl < kPoolSlots; ++sl) {
+            const int32_t bk = sm.blk[s][sl];
+            if (bk >= 0)
+              sm100::cp_async16(sm.a[s] + sl * kBlk * kIdxCodeBytes + phys,
+                                p.kcodes + (seq_off + int64_t(bk) * kBlk) * kIdxCodeBytes + lane * 16);
+          }
+          // scales: 32 bytes per block, two 16-byte chunks
 #pragma unroll
-          for (int u = 0; u < 2; ++u)
-            if (v2[u]) {
-              const int sl = 2 * lane + u;
-              const int64_t row = seq_off + int64_t(blk2[u]) * kBlk;
-              sm100::tma_load_2d(sm.a[s] + sl * kBlk * kIdxCodeBytes, &tmap, 0, int32_t(row), &sm.full[s]);
-              sm100::bulk_load(&sm.sc[s][sl * kBlk], p.kscales + row * 4, kBlk * 4, &sm.full[s]);
-            }
+          for (int m = 0; m < 4; ++m) {
+            const int chk = 32 * m + lane, sl = chk >> 1;
+            const int32_t bk = sm.blk[s][sl];
+            if (bk >= 0)
+              sm100::cp_async16(&sm.sc[s][sl * kBlk + 4 * (chk & 1)],
+                                p.kscales + (seq_off + int64_t(bk) * kBlk) * 4 + 16 * (chk & 1));
+          }
+          sm100::cp_async_commit();
+          // signal the item issued kGatherDepth items ago once its copies landed
+          if (t >= kGatherDepth) {
+            sm100::cp_async_wait<kGatherDepth>();
+            sm100::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&sm.full[(t - kGatherDepth) % kStages]);
+          }
         } else if (lane == 0) {
           sm.info[s] = make_int2(b, j);
           const int64_t rem_rows = seq_len - int64_t(j) * kTile;
@@ -270,9 +311,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++issued;
       }
+      if (kPool) {
+        sm100::cp_async_wait<0>();
+        sm100::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0)
+          for (int t = max(0, issued - kGatherDepth); t < issued; ++t) sm100::mbar_arrive(&sm.full[t % kStages]);
+      }
     }
     // drain: every copy this warp issued has landed before the CTA exits
-    if (lane == 0)
+    if (!kPool && lane == 0)
       for (int s = 0; s < kStages && s < issued; ++s) {
         const int last_round = (issued - 1 - s) / kStages;
         if (!sm100::mbar_wait(&sm.full[s], last_round & 1, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
@@ -536,7 +584,7 @@ int num_sms() {
 
 template <bool kPool>
 void launch_index_tc(const CUtensorMap& map, const ScanParams& p, int64_t max_items, cudaStream_t st) {
-  const size_t smem = sizeof(ScanSmem) + 1024;
+  const size_t smem = sizeof(ScanSmem<Ring<kPool>::kStages>) + 1024;
   cudaFuncSetAttribute(k_index_tc<kPool>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   const int grid = int(std::min<int64_t>(num_sms(), std::max<int64_t>(max_items, 1)));
   k_index_tc<kPool><<<grid, kThreads, smem, st>>>(map, p);
@@ -584,6 +632,7 @@ csa2_status launch_pool_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
   const csa2_status rc = code_map(&map, kcodes, sd.cache_rows, kBlk);
   if (rc != CSA2_OK) return rc;
   ScanParams p{};
+  p.kcodes = kcodes;
   p.kscales = kscales;
   p.q_codes = q_codes;
   p.q_scales = q_scales;

@@ -94,14 +94,18 @@ class DecodeStep:
                 self._hook("csa2_index_full", "end")
                 last = self.topk[layer]
             elif act == "reindex":
+                self._hook("csa2_index_reindex", "begin")
                 C.csa2_index_reindex(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len, self.pool,
                                      self.k, self.topk[layer], self.ws_re, stream=stream)
+                self._hook("csa2_index_reindex", "end")
                 last = self.topk[layer]
             else:
                 self.topk[layer] = last  # Reuse: the same tensor, no copy
+            self._hook("csa2_sparse_attn_decode", "begin")
             C.csa2_sparse_attn_decode(L["q"], cache.main, seq_row_off, seq_len, last, L["win"], L["win_scale"],
                                       L["win_len"], self.sm_scale, self.out[layer], self.ws_attn,
                                       lse=self.lse[layer], stream=stream)
+            self._hook("csa2_sparse_attn_decode", "end")
         return self.out
 
     def device_flags(self) -> int:

@@ -168,6 +168,34 @@ def time_oracle(wl, samples, nthreads):
 
 # ----------------------------------------------------------------------------
 
+def rank_workload(wl, rank):
+    """Weak scaling: rank r runs its own batch of the same shape, drawn with
+    seed + 1000 r, so no two ranks share a sequence and no data crosses ranks."""
+    import synth.workloads as W
+
+    if rank == 0:
+        return wl
+    return W.DecodeWorkload(wl.name, wl.lengths, wl.pattern, wl.P, wl.k, wl.needles, wl.lognormal,
+                            seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(x, device, world):
+    """The slowest rank's value (timings are reported as the max over ranks)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, batch_per_rank, ms_per_step):
+    """Whole-job queries/s: every rank decodes its batch once per step."""
+    return world * batch_per_rank / (ms_per_step * 1e-3)
+
+
 def build_workload(wl, rank, device):
     import torch
 
@@ -175,9 +203,7 @@ def build_workload(wl, rank, device):
     from long_context_decode_csa2_b200 import csa2 as C
     from long_context_decode_csa2_b200.decode import FullCache
 
-    if rank:
-        wl = W.DecodeWorkload(wl.name, wl.lengths, wl.pattern, wl.P, wl.k, wl.needles, wl.lognormal,
-                              seed=wl.seed + 1000 * rank)
+    wl = rank_workload(wl, rank)
     layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
     caches_dev = [W.full_cache_device(wl, f, layers[f]["q_codes"], layers[f]["q_scales"], device)
                   for f in wl.full_layers()]
@@ -268,10 +294,7 @@ def run_ours(args):
     ms = t0.elapsed_time(t1) / args.steps
     per_call = {name: sum(a.elapsed_time(b) for a, b in lst) / len(lst) for name, lst in ev_calls.items()}
     full_ms = [a.elapsed_time(b) for a, b in ev_calls["csa2_index_full"]]
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, device, world)
 
     # end to end: host (pinned) query inputs -> device, step, outputs -> host
     keys_in = ("q", "q_codes", "q_scales", "w")
@@ -297,10 +320,7 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, device, world)
     flags = step.device_flags()
 
     ab = algorithmic_bytes(wl)
@@ -335,7 +355,7 @@ def run_ours(args):
             launches_per_step += {"scan": 5, "reindex": 3, "reuse": 0}[act] + 2
         res = {
             "metric": METRIC,
-            "value": world * wl.B / (ms * 1e-3),
+            "value": job_throughput(world, wl.B, ms),
             "unit": "queries/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -349,7 +369,7 @@ def run_ours(args):
             "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len, "layers": wl.pattern,
                        "pool_blocks": wl.P, "topk": wl.k, "window": 128,
                        "l2": "no flush: inputs larger than L2 (%.2f GB read per step)" % (ab["total"] / 1e9)},
-            "tokens_per_s": world * wl.B / (ms * 1e-3),
+            "tokens_per_s": job_throughput(world, wl.B, ms),
             "hbm_algorithmic_gbs": ab["total"] / (ms * 1e-3) / 1e9,
             "hbm_frac_of_8tbs": ab["total"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
             "roofline": {"kernel": "csa2_index_full (scan + block max + pool + Top-512)", "bound": "hbm",
@@ -357,7 +377,7 @@ def run_ours(args):
                          "peak_kind": peak_kind, "traffic": traffic, "algorithmic_bytes": full_bytes,
                          "avg_ms": full_avg},
             "cpu_baseline": cpu,
-            "e2e": {"value": world * wl.B / (e2e_ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": job_throughput(world, wl.B, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "per_call_ms": per_call,

@@ -52,10 +52,17 @@ constexpr int kAccCols = 16 * kMT;
 constexpr int kTmemCols = 256;
 constexpr uint32_t kSfCol = 192;       // scale factors (all 0x7F = 2^0) live here
 constexpr int kEpiTeams = 2;           // epilogue teams of 4 warps, items round-robin
-constexpr int kThreads = 64 + 128 * kEpiTeams;  // producer, MMA, epilogue warps
+constexpr int kFirstExtra = 2 + 4 * kEpiTeams;  // first extra producer warp (pool mode)
+constexpr int kPoolProducers = 4;      // pool mode: warps sharing the gather of an item
+template <bool kPool>
+constexpr int threads_of() {           // producer, MMA, epilogue (+ extra producer) warps
+  return 32 * (kFirstExtra + (kPool ? kPoolProducers - 1 : 0));
+}
 constexpr uint32_t kCodeBytes = kTile * kIdxCodeBytes;
 constexpr int kBoxRows = 256;          // TMA box height (scan)
 constexpr int kPoolSlots = kTile / kBlk;  // pool blocks per item (64)
+constexpr int kSlotsPerWarp = kPoolSlots / kPoolProducers;
+static_assert(kSlotsPerWarp <= 32 && kPoolSlots % kPoolProducers == 0, "one pool slot per lane at most");
 static_assert(kAcc * kAccCols <= int(kSfCol), "TMEM accumulators overlap the scale factors");
 
 template <int kStages>
@@ -73,7 +80,9 @@ struct __align__(1024) ScanSmem {
   uint32_t tmem_base;
   int abort_flag;
   int built[kStages];                  // segment whose B operand each stage holds
-  int32_t segpool[CSA2_MAX_POOL_BLOCKS]; // pool mode: the current segment's pool block ids
+  // pool mode: each producer warp's share of the current segment's pool ids
+  // (slot i of item j of warp w is pool entry 64 j + kSlotsPerWarp w + i)
+  int32_t segpool[kPoolProducers][CSA2_MAX_POOL_BLOCKS / kPoolProducers];
 };
 
 struct ScanParams {
@@ -138,7 +147,7 @@ __device__ __forceinline__ void build_b_operand(uint8_t* bo, uint2 qreg, int lan
 }
 
 template <bool kPool>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_of<kPool>(), 1)
     k_index_tc(const __grid_constant__ CUtensorMap tmap, ScanParams p) {
   constexpr int kStages = Ring<kPool>::kStages;
   constexpr int kGatherDepth = Ring<kPool>::kGatherDepth;
@@ -154,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      sm100::mbar_init(&sm.full[s], 1);
+      sm100::mbar_init(&sm.full[s], kPool ? kPoolProducers : 1);
       sm100::mbar_init(&sm.empty[s], 1 + 4);
     }
     for (int a = 0; a < kAcc; ++a) {
@@ -186,10 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   sm100::tc_fence_after();
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp >= kFirstExtra) {
+    // ------------------------------------------------------------ producer(s)
+    // pool mode: warp 0 and the extra warps each gather kSlotsPerWarp blocks of
+    // every item; warp 0 alone writes the B operand and the item info
+    const int pw = warp == 0 ? 0 : warp - kFirstExtra + 1;
     int issued = 0;
-    if (lane < kStages) sm.built[lane] = -1;
+    if (warp == 0 && lane < kStages) sm.built[lane] = -1;
     __syncwarp();
     if (i0 < i1) {
       int b, seq_start = 0, next_start = 0;
@@ -232,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (__any_sync(0xffffffffu, aborted(sm))) break;
-        if (sm.built[s] != b) {
+        if (pw == 0 && sm.built[s] != b) {
           if (qb != b) {
             qreg = __ldg(reinterpret_cast<const uint2*>(p.q_codes + int64_t(b) * kHi * 64) + lane);
             qb = b;
@@ -244,49 +256,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (kPool) {
           if (pool_seg != b) {
-            // all of the segment's pool ids at once (one round trip per segment);
-            // every stage that still holds unsignalled copies keeps its own ids
+            // this warp's share of the segment's pool ids (one round trip per
+            // segment); copies already issued carry their own addresses
             const int32_t* src = p.pool + int64_t(b) * p.P;
-            int32_t v[CSA2_MAX_POOL_BLOCKS / 32];
+            constexpr int kPer = CSA2_MAX_POOL_BLOCKS / kPoolProducers / 32;
+            int32_t v[kPer];
 #pragma unroll
-            for (int m = 0; m < CSA2_MAX_POOL_BLOCKS / 32; ++m) {
-              const int i = lane + 32 * m;
-              v[m] = i < p.P ? __ldg(src + i) : -1;
+            for (int m = 0; m < kPer; ++m) {
+              const int e = lane + 32 * m;  // entry (item e / kSlotsPerWarp, slot e % kSlotsPerWarp)
+              const int slot = (e / kSlotsPerWarp) * kPoolSlots + pw * kSlotsPerWarp + e % kSlotsPerWarp;
+              v[m] = slot < p.P ? __ldg(src + slot) : -1;
             }
 #pragma unroll
-            for (int m = 0; m < CSA2_MAX_POOL_BLOCKS / 32; ++m) sm.segpool[lane + 32 * m] = v[m];
+            for (int m = 0; m < kPer; ++m) sm.segpool[pw][lane + 32 * m] = v[m];
             __syncwarp();
             pool_seg = b;
           }
-          // gather: block ids of the item's 64 pool slots
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int slot = j * kPoolSlots + 2 * lane + u;
-            const int32_t bk = slot < p.P ? sm.segpool[slot] : -1;
+          // lane i < kSlotsPerWarp owns slot pw * kSlotsPerWarp + i of the item
+          int32_t my = -1;
+          if (lane < kSlotsPerWarp) {
+            const int32_t bk = sm.segpool[pw][j * kSlotsPerWarp + lane];
             const bool in_range = bk >= 0 && int64_t(bk) * kBlk < seq_len;
             if (bk >= 0 && !in_range) set_status(p.status, CSA2_DEV_INDEX_RANGE);
-            sm.blk[s][2 * lane + u] = in_range ? bk : -1;
+            my = in_range ? bk : -1;
+            sm.blk[s][pw * kSlotsPerWarp + lane] = my;
           }
-          if (lane == 0) sm.info[s] = make_int2(b, j);
-          __syncwarp();
+          if (pw == 0 && lane == 0) sm.info[s] = make_int2(b, j);
           // one warp instruction per 512-byte block: lane = (row l/4, chunk l%4),
           // destination in the 64-byte swizzle the MMA descriptor expects
           const int r8 = lane >> 2, ch = lane & 3;
           const int phys = r8 * 64 + ((ch ^ ((r8 >> 1) & 3)) << 4);
-          for (int sl = 0; sl < kPoolSlots; ++sl) {
-            const int32_t bk = sm.blk[s][sl];
-            if (bk >= 0)
-              sm100::cp_async16(sm.a[s] + sl * kBlk * kIdxCodeBytes + phys,
-                                p.kcodes + (seq_off + int64_t(bk) * kBlk) * kIdxCodeBytes + lane * 16);
+          const uint8_t* kbase = p.kcodes + seq_off * kIdxCodeBytes + lane * 16;
+          uint8_t* abase = sm.a[s] + pw * kSlotsPerWarp * kBlk * kIdxCodeBytes + phys;
+#pragma unroll
+          for (int i = 0; i < kSlotsPerWarp; ++i) {
+            const int32_t bk = __shfl_sync(0xffffffffu, my, i);
+            if (bk >= 0) sm100::cp_async16(abase + i * kBlk * kIdxCodeBytes, kbase + int64_t(bk) * kBlk * kIdxCodeBytes);
           }
           // scales: 32 bytes per block, two 16-byte chunks
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int chk = 32 * m + lane, sl = chk >> 1;
-            const int32_t bk = sm.blk[s][sl];
-            if (bk >= 0)
-              sm100::cp_async16(&sm.sc[s][sl * kBlk + 4 * (chk & 1)],
-                                p.kscales + (seq_off + int64_t(bk) * kBlk) * 4 + 16 * (chk & 1));
+          for (int c0 = 0; c0 < 2 * kSlotsPerWarp; c0 += 32) {
+            const int c = c0 + lane, i = (c >> 1) & 31;
+            const int32_t bk = __shfl_sync(0xffffffffu, my, i);
+            if (c < 2 * kSlotsPerWarp && bk >= 0)
+              sm100::cp_async16(&sm.sc[s][(pw * kSlotsPerWarp + i) * kBlk + 4 * (c & 1)],
+                                p.kscales + (seq_off + int64_t(bk) * kBlk) * 4 + 16 * (c & 1));
           }
           sm100::cp_async_commit();
           // signal the item issued kGatherDepth items ago once its copies landed
@@ -587,7 +601,7 @@ void launch_index_tc(const CUtensorMap& map, const ScanParams& p, int64_t max_it
   const size_t smem = sizeof(ScanSmem<Ring<kPool>::kStages>) + 1024;
   cudaFuncSetAttribute(k_index_tc<kPool>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   const int grid = int(std::min<int64_t>(num_sms(), std::max<int64_t>(max_items, 1)));
-  k_index_tc<kPool><<<grid, kThreads, smem, st>>>(map, p);
+  k_index_tc<kPool><<<grid, threads_of<kPool>(), smem, st>>>(map, p);
 }
 
 }  // namespace

@@ -17,10 +17,9 @@
 //  [OCP]  OCP Microscaling Formats (MX) v1.0: E2M1, E8M0, MXFP4 block of 32.
 //
 // The pages give no formula for the indexer score, the compression weights or
-// the attention scale; the readings used here are the plainest ones and are
-// listed with their reasons in the design notes of this repository.  Every
-// function below is pinned by tests under tests/ (no function is "parity
-// unpinned").
+// the attention scale; the readings used here are the plainest ones, and each
+// function states the reading it takes.  Every function below is pinned by
+// tests under tests/ (no function is "parity unpinned").
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -151,7 +150,7 @@ double own_exp(double x) {
 }
 
 // ---------------------------------------------------------------------------
-// Indexer score  [V41] "FP4 indexer q/k"; the formula is this build's reading:
+// Indexer score  [V41] "FP4 indexer q/k"; the pages give no formula; the plainest reading is
 //   s_t = sum_h w_h * (q_h . k_t)   (no ReLU), one 128-d key per position
 // shared by the 4 indexer heads.  Exactness: per head h and 32-block b the
 // doubled-E2M1 integer dot D (|D| <= 4608) times 2^(eq+ek-2) is exact; the
@@ -412,8 +411,8 @@ int orc_attn_decode(const uint16_t* q, const uint8_t* mcodes, const uint8_t* msc
 
 // Compression + quantisation of new cache entries [V41]: m tokens become one
 // entry, entries have disjoint sources and no absolute position encoding; the
-// weights are a softmax over the pair's per-token logits (this build's
-// reading of the garbled weighting formula).
+// weights are a softmax over the pair's per-token logits (the plainest
+// reading of a weighting formula the page prints garbled).
 // ratio 1: c = x.  ratio 2: entry j merges raw rows 2j, 2j+1:
 //   m = max(z0, z1); a = exp(z0-m); b = exp(z1-m); w0 = a/(a+b); w1 = b/(a+b)
 //   c_i = fp32( fma(w0, x0_i, w1*x1_i) )   (fp64, own exp)

@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling captures)")
+    ap.add_argument("--context", type=int, default=0,
+                    help="override every sequence's length (small profiling captures of the attention)")
     return ap.parse_args()
 
 
@@ -244,26 +246,31 @@ def run_ours(args):
     if args.batch:
         wl = W.DecodeWorkload(wl.name + f"_b{args.batch}", wl.lengths[:args.batch], wl.pattern, wl.P, wl.k,
                               wl.needles, wl.lognormal, wl.seed)
+    if args.context:
+        wl = W.DecodeWorkload(wl.name + f"_l{args.context}", np.full(wl.B, args.context), wl.pattern, wl.P, wl.k,
+                              min(wl.needles, max(1, args.context // 1024)), wl.lognormal, wl.seed)
     wl, layers, caches_dev, caches, layers_dev, off_d, len_d = build_workload(wl, rank, device)
     C.lib()
     step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
     stream = torch.cuda.current_stream()
 
-    # events around every C-ABI call of the timed region; csa2_index_full
-    # (full-context scan, block max, pool, Top-512) is the dominant call
+    # events around every C-ABI call of the timed region, on the stream the
+    # call runs on; csa2_index_full (full-context scan, block max, pool,
+    # Top-512) is the dominant call and runs alone.  The other calls overlap
+    # one another on side streams, so their times include that sharing.
     n_layers = len(wl.pattern)
     ev_calls = {}
     recording = [False]
 
-    def hook(name, phase):
+    def hook(name, phase, on_stream):
         if not recording[0]:
             return
         lst = ev_calls.setdefault(name, [])
         if phase == "begin":
             lst.append([torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)])
-            lst[-1][0].record(stream)
+            lst[-1][0].record(on_stream)
         else:
-            lst[-1][1].record(stream)
+            lst[-1][1].record(on_stream)
 
     step.hook = hook
 
@@ -389,6 +396,119 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_prefill(args):
+    """Prefill workload: ratio-2 compression of n_raw tokens into a fresh
+    cache (with the W_idx projection), the causal indexer for T queries, and
+    their sparse attention; one step = those three calls.  Reports prefill
+    queries/s and per-call times (compressed tokens/s for the first call)."""
+    import torch
+
+    import synth
+    import synth.gpu as sg
+    import synth.workloads as W
+    from long_context_decode_csa2_b200 import csa2 as C
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
+    pw = W.prefill_workload()
+    seed = pw.seed + 1000 * rank
+    n_raw, T, ratio, P, k = pw.n_raw, pw.T, pw.ratio, pw.P, pw.k
+    n_ent = n_raw // ratio
+    rows = (n_ent + 7) // 8 * 8
+    raw = torch.empty((n_raw, 512), dtype=torch.bfloat16, device=device)
+    sg.normal_bf16_into(raw, seed, synth.T_RAW, 0, 0)
+    q = torch.empty((T, 16, 512), dtype=torch.bfloat16, device=device)
+    sg.normal_bf16_into(q, seed, synth.T_Q, 0, 0)
+    raw_win = torch.empty((n_raw, 512), dtype=torch.uint8, device=device)
+    sg.e4m3_rows_into(raw_win, seed, synth.T_RAWWIN, 0, 0, 0, n_raw)
+    logits = torch.from_numpy(synth.normal_f32(seed, synth.T_LOGITS, 0, 0, n_raw)).to(device)
+    w_idx = torch.from_numpy(synth.normal_f32(seed, synth.T_WIDX, 0, 0, 512 * 128, log2_div=13)).to(device)
+    qc, qs = synth.mxfp4_rows(seed, synth.T_QIDX_CODES, synth.T_QIDX_SCALES, 0, 0, 0, T * 4, 128)
+    q_codes = torch.from_numpy(np.ascontiguousarray(qc.reshape(T, 4, 64))).to(device)
+    q_scales = torch.from_numpy(np.ascontiguousarray(qs.reshape(T, 4, 4))).to(device)
+    w = torch.from_numpy(synth.head_weights(seed, 0, 0, T * 4).reshape(T, 4)).to(device)
+    win_scale = float(synth.window_scale(seed, 0, 0))
+    q_pos = torch.arange(n_raw - T, n_raw, dtype=torch.int32, device=device)
+    main = C.cache(torch.zeros((rows, 256), dtype=torch.uint8, device=device),
+                   torch.zeros((rows, 16), dtype=torch.uint8, device=device))
+    idx = C.cache(torch.zeros((rows, 64), dtype=torch.uint8, device=device),
+                  torch.zeros((rows, 4), dtype=torch.uint8, device=device))
+    tok_off = torch.tensor([0, n_raw], dtype=torch.int64, device=device)
+    row_off = torch.zeros(1, dtype=torch.int64, device=device)
+    len_in = torch.zeros(1, dtype=torch.int32, device=device)
+    len_out = torch.zeros(1, dtype=torch.int32, device=device)
+    pool = torch.empty((T, P), dtype=torch.int32, device=device)
+    top = torch.empty((T, k), dtype=torch.int32, device=device)
+    out = torch.empty((T, 16, 512), dtype=torch.float32, device=device)
+    lse = torch.empty((T, 16), dtype=torch.float32, device=device)
+    ws1 = C.workspace(C.csa2_compress_append_workspace_bytes(1), device)
+    ws2 = C.workspace(C.csa2_index_prefill_workspace_bytes(T, n_ent, P, k), device)
+    ws3 = C.workspace(C.csa2_sparse_attn_prefill_workspace_bytes(T, k), device)
+    stream = torch.cuda.current_stream()
+    names = ("csa2_compress_append", "csa2_index_prefill", "csa2_sparse_attn_prefill")
+    times = {n: [] for n in names}
+
+    def step(record):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
+        if record:
+            ev[0].record(stream)
+        C.csa2_compress_append(main, idx, raw, logits, tok_off, row_off, len_in, len_out, ratio, n_ent, ws1,
+                               w_idx=w_idx)
+        if record:
+            ev[1].record(stream)
+        C.csa2_index_prefill(idx, q_codes, q_scales, w, q_pos, 0, n_ent, ratio, P, k, pool, top, ws2)
+        if record:
+            ev[2].record(stream)
+        C.csa2_sparse_attn_prefill(q, q_pos, main, 0, n_ent, ratio, top, raw_win, win_scale, 1 / math.sqrt(512), out,
+                                   ws3, lse=lse)
+        if record:
+            ev[3].record(stream)
+            for i, n in enumerate(names):
+                times[n].append((ev[i], ev[i + 1]))
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    flags = C.device_status(ws1) | C.device_status(ws2) | C.device_status(ws3)
+    if flags:
+        raise RuntimeError(f"device status flags {flags} during warm-up")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.5)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, device, world)
+    per_call = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) for n, v in times.items()}
+    if rank == 0:
+        print(json.dumps({
+            "metric": "prefill queries/sec (ratio-2 compression of 262144 tokens, 4096-query causal chunk)",
+            "value": job_throughput(world, T, ms), "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int32+f64 indexer, f16 tensor-core attention (f32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": pw.name, "raw_tokens": n_raw, "entries": n_ent, "queries": T, "pool_blocks": P,
+                       "topk": k, "window": 128},
+            "compress_tokens_per_s": n_raw / (per_call["csa2_compress_append"] * 1e-3),
+            "per_call_ms": per_call, "clocks": clk.summary(), "device_flags": flags}))
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     """The oracle as the reference arm: K timed steps, each one oracle decode
     step over a bounded sample of the workload's sequences on the host cores."""
@@ -444,6 +564,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload.startswith("prefill"):
+        run_prefill(args)
     else:
         run_ours(args)
 

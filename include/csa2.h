@@ -38,7 +38,9 @@
  *     before its first use.  Its first 256 bytes hold a device status word
  *     that kernels OR flags into (see CSA2_DEV_*); read and clear it with
  *     csa2_device_status().  One workspace must not be used by two calls that
- *     may run concurrently.
+ *     may run concurrently.  Calls keep internal counters and histograms in
+ *     the workspace and leave them zero when they finish; after a call that
+ *     set a device flag, zero-fill the workspace again before reusing it.
  *   - Return value: CSA2_OK, or a negative error; on an error nothing was
  *     launched, except CSA2_ERR_CUDA (a launch failed; see csa2_last_error()).
  *     Arguments are validated on the host before the first launch.

@@ -48,6 +48,7 @@ struct IndexFullWs {
   uint32_t* bkeys;
   uint32_t* ckeys;
   float* scores;
+  uint32_t* hist;  // [B][kSelHistBins] (block keys, then candidates), zero between calls
   size_t bytes;
 };
 
@@ -57,10 +58,11 @@ IndexFullWs index_full_ws(void* ws, int B, int max_len, int P, int k, bool need_
   w.status = c.take<uint32_t>(kStatusBytes / 4);
   w.seg_eff = c.take<int32_t>(size_t(B));
   w.tile_start = c.take<int32_t>(scan_tc_prefix_ints(B));
-  const size_t nb = (size_t(max_len) + kBlk - 1) / kBlk;
+  const size_t nb = size_t(block_key_stride(max_len));
   w.bkeys = c.take<uint32_t>(size_t(B) * nb);
   w.ckeys = (P >= k) ? c.take<uint32_t>(size_t(B) * P * kBlk) : nullptr;
   w.scores = need_scores ? c.take<float>(size_t(B) * max_len) : nullptr;
+  w.hist = c.take<uint32_t>(size_t(B) * kSelHistBins);
   w.bytes = c.used;
   return w;
 }
@@ -123,22 +125,22 @@ csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, cons
   if (workspace_bytes < ws.bytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SegDesc sd{seq_row_off, 0, seq_len, max_len, idx_k.rows};
-  const int64_t nb = (int64_t(max_len) + kBlk - 1) / kBlk;
+  const int64_t nb = block_key_stride(max_len);
   float* scores = scores_out ? scores_out : ws.scores;
   const csa2_status rc = launch_scan_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, ws.tile_start, B, q_codes, q_scales,
-                                        w, ws.bkeys, nb, scores, max_len, ws.status, st);
+                                        w, ws.bkeys, nb, scores, max_len, ws.hist, ws.status, st);
   if (rc != CSA2_OK) return rc;
-  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, st);
+  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, ws.hist, st);
   if (pool_blocks >= k) {
     // Every Top-k position's block ranks within the first k blocks, so the
     // Top-k over the pool equals the Top-k over all positions.
     const csa2_status rc2 = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, B, q_codes, q_scales, w,
-                                           pool_out, pool_blocks, ws.ckeys, ws.status, st);
+                                           pool_out, pool_blocks, ws.ckeys, ws.hist, ws.status, st);
     if (rc2 != CSA2_OK) return rc2;
     launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.seg_eff, B, pool_blocks, pool_out, k,
-                  topk_out, st);
+                  topk_out, ws.hist, st);
   } else {
-    launch_select(kSelScores, scores, max_len, ws.seg_eff, B, 0, nullptr, k, topk_out, st);
+    launch_select(kSelScores, scores, max_len, ws.seg_eff, B, 0, nullptr, k, topk_out, nullptr, st);
   }
   return check_launch(fn);
 }
@@ -150,6 +152,7 @@ size_t csa2_index_reindex_workspace_bytes(int B, int pool_blocks, int k) {
   c.take<uint32_t>(kStatusBytes / 4);
   c.take<int32_t>(size_t(B));
   c.take<uint32_t>(size_t(B) * pool_blocks * kBlk);
+  c.take<uint32_t>(size_t(B) * kCandHistBins);
   return c.used;
 }
 
@@ -173,13 +176,15 @@ csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
   uint32_t* status = c.take<uint32_t>(kStatusBytes / 4);
   int32_t* seg_eff = c.take<int32_t>(size_t(B));
   uint32_t* ckeys = c.take<uint32_t>(size_t(B) * pool_blocks * kBlk);
+  uint32_t* hist = c.take<uint32_t>(size_t(B) * kCandHistBins);  // zero between calls
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SegDesc sd{seq_row_off, 0, seq_len, INT32_MAX, idx_k.rows};
   launch_seg_check(sd, B, seg_eff, status, st);
   const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, seg_eff, B, q_codes, q_scales, w, pool,
-                                        pool_blocks, ckeys, status, st);
+                                        pool_blocks, ckeys, hist, status, st);
   if (rc != CSA2_OK) return rc;
-  launch_select(kSelPoolCand, ckeys, int64_t(pool_blocks) * kBlk, seg_eff, B, pool_blocks, pool, k, topk_out, st);
+  launch_select(kSelPoolCand, ckeys, int64_t(pool_blocks) * kBlk, seg_eff, B, pool_blocks, pool, k, topk_out, hist,
+                st);
   return check_launch(fn);
 }
 
@@ -295,7 +300,7 @@ PrefillWs prefill_ws(void* ws, int T, int64_t n_entries, int P, int k) {
   PrefillWs w;
   w.status = c.take<uint32_t>(kStatusBytes / 4);
   w.vis = c.take<int32_t>(size_t(T));
-  const size_t nb = (size_t(n_entries) + kBlk - 1) / kBlk;
+  const size_t nb = size_t(block_key_stride(n_entries));
   w.bkeys = c.take<uint32_t>(size_t(T) * nb);
   w.ckeys = c.take<uint32_t>(size_t(T) * P * kBlk);
   w.scores = nullptr;
@@ -325,21 +330,23 @@ csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad cache, row0 or n_entries");
   if (!q_codes || !q_scales || !w || !q_pos || !pool_out || !topk_out || !workspace)
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
-  if (reinterpret_cast<uintptr_t>(workspace) & 255)
-    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": workspace must be 256-byte aligned");
+  if (!aligned16(q_codes) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": q_codes must be 16-byte and workspace 256-byte aligned");
   PrefillWs ws = prefill_ws(workspace, T, n_entries, pool_blocks, k);
   if (workspace_bytes < ws.bytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t nb = (n_entries + kBlk - 1) / kBlk;
+  const int64_t nb = block_key_stride(n_entries);
   launch_prefill_vis(q_pos, T, ratio, n_entries, ws.vis, ws.status, st);
-  launch_prefill_scan(idx_k.codes, idx_k.scales, row0, ws.vis, T, n_entries, q_codes, q_scales, w, ws.bkeys, nb, st);
-  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, T, 0, nullptr, pool_blocks, pool_out, st);
+  const csa2_status rc0 = launch_prefill_tc(idx_k.codes, idx_k.scales, row0, idx_k.rows, ws.vis, T, n_entries, q_codes,
+                                            q_scales, w, ws.bkeys, nb, ws.status, st);
+  if (rc0 != CSA2_OK) return rc0;
+  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, T, 0, nullptr, pool_blocks, pool_out, nullptr, st);
   SegDesc sd{nullptr, row0, ws.vis, n_entries, idx_k.rows};
   const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.vis, T, q_codes, q_scales, w, pool_out,
-                                        pool_blocks, ws.ckeys, ws.status, st);
+                                        pool_blocks, ws.ckeys, nullptr, ws.status, st);
   if (rc != CSA2_OK) return rc;
   launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.vis, T, pool_blocks, pool_out, k, topk_out,
-                st);
+                nullptr, st);
   return check_launch(fn);
 }
 

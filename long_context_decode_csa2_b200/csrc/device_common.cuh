@@ -1,4 +1,5 @@
-// Device helpers: FP4 indexer scoring on CUDA cores, ranking keys, status.
+// Device helpers: exact FP4 indexer scores from tensor-core accumulators,
+// ranking keys, block maxima, status flags.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -25,109 +26,77 @@ __device__ __forceinline__ double pow2d(int e) {
   return __longlong_as_double(static_cast<long long>(e + 1023) << 52);
 }
 
-// Doubled E2M1 value of a code: {0,1,2,3,4,6,8,12} with sign.
-__device__ __forceinline__ int e2m1_twice(uint32_t code) {
-  const uint32_t mag = (0xC8643210u >> (4 * (code & 7))) & 15u;  // nibbles 0,1,2,3,4,6,8,12
-  return (code & 8) ? -static_cast<int>(mag) : static_cast<int>(mag);
-}
-
-// One indexer query prepared for dp4a scoring:
-//   qp[h][m] packs the doubled values of elements 4m..4m+3 (signed bytes),
-//   qn[h][m] the same bytes negated; eq[h][b] = block-scale exponent (byte-127);
-//   w[h] the head weights.
-struct IdxQueryPrep {
-  uint32_t qp[kHi][32];
-  uint32_t qn[kHi][32];
-  int eq[kHi][4];
+// Scale context of one indexer query for the tensor-core epilogues:
+// qsh[h][b] = (E8M0 byte - 127) << 23 (an fp32 exponent-field offset), the
+// head weights, and the range of the query's block exponents.
+struct IdxQCtx {
+  uint32_t qsh[kHi][4];
   float w[kHi];
+  int qlo, qhi, qspread;
 };
 
-// Fill `qs` from the raw query (call with all threads of the block, then sync).
-__device__ __forceinline__ void prep_query(IdxQueryPrep& qs, const uint8_t* q_codes /*[4][64]*/,
-                                           const uint8_t* q_scales /*[4][4]*/, const float* w, int tid,
-                                           int nthreads) {
-  for (int i = tid; i < kHi * 32; i += nthreads) {
-    const int h = i / 32, m = i % 32;
-    const uint8_t b0 = q_codes[h * 64 + 2 * m], b1 = q_codes[h * 64 + 2 * m + 1];
-    const int v0 = e2m1_twice(b0 & 15), v1 = e2m1_twice(b0 >> 4);
-    const int v2 = e2m1_twice(b1 & 15), v3 = e2m1_twice(b1 >> 4);
-    qs.qp[h][m] = (uint32_t(v0) & 255u) | ((uint32_t(v1) & 255u) << 8) | ((uint32_t(v2) & 255u) << 16) |
-                  ((uint32_t(v3) & 255u) << 24);
-    qs.qn[h][m] = (uint32_t(-v0) & 255u) | ((uint32_t(-v1) & 255u) << 8) | ((uint32_t(-v2) & 255u) << 16) |
-                  ((uint32_t(-v3) & 255u) << 24);
-  }
-  for (int i = tid; i < kHi * 4; i += nthreads) qs.eq[i / 4][i % 4] = int(q_scales[i]) - 127;
-  for (int i = tid; i < kHi; i += nthreads) qs.w[i] = w[i];
-}
-
-// Exact block dot products D[h][b] (doubled-E2M1 integers) of one 128-element
-// key row (16 code words) with the prepared query.
-__device__ __forceinline__ void block_dots(const IdxQueryPrep& q, const uint32_t (&kw)[16], int (&D)[kHi][4]) {
-#pragma unroll
-  for (int h = 0; h < kHi; ++h)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) D[h][b] = 0;
-#pragma unroll
-  for (int wd = 0; wd < 16; ++wd) {
-    const uint32_t c = kw[wd];
-    const uint32_t lo = c & 0xFFFFu, hi = c >> 16;
-    const uint32_t mlo = __byte_perm(0x03020100u, 0x0C080604u, lo & 0x7777u);
-    const uint32_t mhi = __byte_perm(0x03020100u, 0x0C080604u, hi & 0x7777u);
-    const uint32_t slo = 0x3210u | ((lo & 0x8888u) >> 1);
-    const uint32_t shi = 0x3210u | ((hi & 0x8888u) >> 1);
-#pragma unroll
-    for (int h = 0; h < kHi; ++h) {
-      const uint32_t a0 = __byte_perm(q.qp[h][2 * wd], q.qn[h][2 * wd], slo);
-      const uint32_t a1 = __byte_perm(q.qp[h][2 * wd + 1], q.qn[h][2 * wd + 1], shi);
-      D[h][wd / 4] = __dp4a(int(a0), int(mlo), D[h][wd / 4]);
-      D[h][wd / 4] = __dp4a(int(a1), int(mhi), D[h][wd / 4]);
-    }
-  }
-}
-
-// Score from exact block dots: per head the four terms D*2^(eq+ek-2) are
-// summed in double in block order and rounded once to float; heads combine
-// with an fp32 fma chain.  Explicit _rn intrinsics keep nvcc from contracting.
-__device__ __forceinline__ float combine_score(const IdxQueryPrep& q, const int (&D)[kHi][4], uint32_t kscale_word) {
-  float d[kHi];
+__device__ __forceinline__ void make_qctx(IdxQCtx& c, const uint8_t* q_scales /*[4][4]*/, const float* w /*[4]*/) {
+  c.qlo = 255;
+  c.qhi = 0;
+  c.qspread = 0;
 #pragma unroll
   for (int h = 0; h < kHi; ++h) {
-    double acc = 0.0;
+    int mn = 255, mx = 0;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int ek = int((kscale_word >> (8 * b)) & 255u) - 127;
-      const double term = __dmul_rn(static_cast<double>(D[h][b]), pow2d(q.eq[h][b] + ek - 2));
-      acc = __dadd_rn(acc, term);
+    for (int bb = 0; bb < 4; ++bb) {
+      const int q = q_scales[h * 4 + bb];
+      c.qsh[h][bb] = uint32_t(q - 127) << 23;
+      mn = min(mn, q);
+      mx = max(mx, q);
     }
-    d[h] = __double2float_rn(acc);
-  }
-  float s = __fmul_rn(q.w[0], d[0]);
-#pragma unroll
-  for (int h = 1; h < kHi; ++h) s = __fmaf_rn(q.w[h], d[h], s);
-  if (s == 0.0f) s = 0.0f;
-  return s;
-}
-
-__device__ __forceinline__ void load_key_row(const uint8_t* kcodes, int64_t row, uint32_t (&kw)[16]) {
-  const uint4* p = reinterpret_cast<const uint4*>(kcodes + row * kIdxCodeBytes);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 v = __ldg(p + i);
-    kw[4 * i + 0] = v.x;
-    kw[4 * i + 1] = v.y;
-    kw[4 * i + 2] = v.z;
-    kw[4 * i + 3] = v.w;
+    c.qlo = min(c.qlo, mn);
+    c.qhi = max(c.qhi, mx);
+    c.qspread = max(c.qspread, mx - mn);
+    c.w[h] = w[h];
   }
 }
 
-__device__ __forceinline__ float score_row(const IdxQueryPrep& q, const uint8_t* kcodes, const uint8_t* kscales,
-                                           int64_t row) {
-  uint32_t kw[16];
-  load_key_row(kcodes, row, kw);
-  const uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(kscales) + row);
-  int D[kHi][4];
-  block_dots(q, kw, D);
-  return combine_score(q, D, sw);
+// Exact score of one position from its 16 tensor-core accumulators
+// v[4h+b] = D_{h,b}/4 (the block dot of doubled E2M1 values, exact in fp32)
+// and its key's E8M0 scale word sw (block b in byte b):
+//   d_h = fp32( sum_b D_{h,b} * 2^(eq+ek-2) )  (summed in order b = 0..3),
+//   s = w0*d0, then s = fma(w_h, d_h, s); -0 -> +0.
+// When the block exponents lie within 9 of each other (and away from the
+// fp32 range limits) every term and partial sum is exact in fp32, so the sum
+// is done there; otherwise in fp64 as the definition states.
+__device__ __forceinline__ float exact_score(const uint32_t (&v)[16], uint32_t sw, const IdxQCtx& q) {
+  const int k0 = int(sw & 255u), k1 = int((sw >> 8) & 255u), k2 = int((sw >> 16) & 255u), k3 = int(sw >> 24);
+  const int kmin = min(min(k0, k1), min(k2, k3)), kmax = max(max(k0, k1), max(k2, k3));
+  const bool fast = (kmax - kmin + q.qspread <= 9) && (q.qlo + kmin - 254 >= -100) && (q.qhi + kmax - 254 <= 100);
+  const uint32_t ksh[4] = {uint32_t(k0) << 23, uint32_t(k1) << 23, uint32_t(k2) << 23, uint32_t(k3) << 23};
+  float d[kHi];
+  if (fast) {
+#pragma unroll
+    for (int h = 0; h < kHi; ++h) {
+      float acc = __fmul_rn(__uint_as_float(v[4 * h]), __uint_as_float(q.qsh[h][0] + ksh[0]));
+#pragma unroll
+      for (int bb = 1; bb < 4; ++bb)
+        acc = __fmaf_rn(__uint_as_float(v[4 * h + bb]), __uint_as_float(q.qsh[h][bb] + ksh[bb]), acc);
+      d[h] = acc;
+    }
+  } else {
+    const int kb[4] = {k0, k1, k2, k3};
+#pragma unroll
+    for (int h = 0; h < kHi; ++h) {
+      double acc = 0.0;
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const int e = int(int32_t(q.qsh[h][bb]) >> 23) + kb[bb] - 127;  // eq + ek
+        acc = __dadd_rn(acc, __dmul_rn(double(__uint_as_float(v[4 * h + bb])), pow2d(e)));
+      }
+      d[h] = __double2float_rn(acc);
+    }
+  }
+  float sc = __fmul_rn(q.w[0], d[0]);
+#pragma unroll
+  for (int h = 1; h < kHi; ++h) sc = __fmaf_rn(q.w[h], d[h], sc);
+  if (sc == 0.0f) sc = 0.0f;
+  return sc;
 }
 
 // Max over aligned groups of 8 lanes; every lane of the group gets it.

@@ -1,7 +1,6 @@
-// Indexer kernels: segment checks, the multi-query causal prefill scan, and
-// deterministic radix selection (Top-k by key desc / index asc, output
-// ascending).  The decode scan and the pool scoring run on the tensor cores
-// (scan_tc.cu).
+// Indexer kernels: segment checks, prefill visibility, and deterministic radix
+// selection (Top-k by key desc / index asc, output ascending).  The scans and
+// the pool scoring run on the tensor cores (scan_tc.cu, prefill_tc.cu).
 //
 // Score definition and selection rule: "DeepSeek-V4.1-Flash: Pushing the
 // Limits of KV Cache Compression", section "三个方向一起压小缓存" (hierarchical
@@ -36,7 +35,8 @@ void launch_seg_check(const SegDesc& sd, int S, int32_t* seg_eff, uint32_t* stat
 }
 
 // ---------------------------------------------------------------------------
-// Prefill: visible entry counts, then the multi-query scan.
+// Prefill: visible entry counts (the scan itself runs on the tensor cores,
+// prefill_tc.cu).
 // ---------------------------------------------------------------------------
 __global__ void k_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entries, int32_t* vis,
                               uint32_t* status) {
@@ -58,90 +58,36 @@ void launch_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entrie
   k_prefill_vis<<<(T + 255) / 256, 256, 0, st>>>(q_pos, T, ratio, n_entries, vis, status);
 }
 
-// grid = (ceil(max_vis/256), ceil(T/kPQ)), block = 256.  Each thread unpacks
-// its key row once and scores it against kPQ queries.
-constexpr int kPQ = 16;
-__global__ void __launch_bounds__(256) k_prefill_scan(const uint8_t* __restrict__ kcodes,
-                                                      const uint8_t* __restrict__ kscales, int64_t row0,
-                                                      const int32_t* __restrict__ vis, int T,
-                                                      const uint8_t* __restrict__ q_codes,
-                                                      const uint8_t* __restrict__ q_scales,
-                                                      const float* __restrict__ w, uint32_t* __restrict__ bkeys,
-                                                      int64_t nb_stride) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  IdxQueryPrep* qs = reinterpret_cast<IdxQueryPrep*>(smem_raw);
-  const int i0 = blockIdx.y * kPQ;
-  const int nq = min(kPQ, T - i0);
-  const int64_t t0 = int64_t(blockIdx.x) * 256;
-  __shared__ int any_vis;
-  if (threadIdx.x == 0) {
-    int a = 0;
-    for (int j = 0; j < nq; ++j) a |= (vis[i0 + j] > t0);
-    any_vis = a;
-  }
-  __syncthreads();
-  if (!any_vis) return;
-  for (int j = 0; j < nq; ++j)
-    prep_query(qs[j], q_codes + int64_t(i0 + j) * kHi * 64, q_scales + int64_t(i0 + j) * kHi * 4,
-               w + int64_t(i0 + j) * kHi, threadIdx.x, 256);
-  __syncthreads();
-  const int64_t t = t0 + threadIdx.x;
-  uint32_t kw[16];
-  uint32_t sw = 0;
-  const int64_t row = row0 + t;
-  // rows beyond the longest visibility of this query tile are never used
-  int maxv = 0;
-  for (int j = 0; j < nq; ++j) maxv = max(maxv, vis[i0 + j]);
-  const bool live = t < maxv;
-  if (live) {
-    load_key_row(kcodes, row, kw);
-    sw = __ldg(reinterpret_cast<const uint32_t*>(kscales) + row);
-  } else {
-#pragma unroll
-    for (int m = 0; m < 16; ++m) kw[m] = 0;
-  }
-  for (int j = 0; j < nq; ++j) {
-    const int64_t v = vis[i0 + j];
-    uint32_t key = 0;
-    if (t < v) {
-      int D[kHi][4];
-      block_dots(qs[j], kw, D);
-      key = rank_key(combine_score(qs[j], D, sw));
-    }
-    key = group8_max(key);
-    if ((threadIdx.x & 7) == 0 && t < v) bkeys[int64_t(i0 + j) * nb_stride + t / kBlk] = key;
-  }
-}
-
-void launch_prefill_scan(const uint8_t* kcodes, const uint8_t* kscales, int64_t row0, const int32_t* vis, int T,
-                         int64_t max_vis, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
-                         uint32_t* bkeys, int64_t nb_stride, cudaStream_t st) {
-  if (T == 0 || max_vis == 0) return;
-  dim3 grid(static_cast<unsigned>((max_vis + 255) / 256), (T + kPQ - 1) / kPQ);
-  const size_t smem = sizeof(IdxQueryPrep) * kPQ;
-  cudaFuncSetAttribute(k_prefill_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  k_prefill_scan<<<grid, 256, smem, st>>>(kcodes, kscales, row0, vis, T, q_codes, q_scales, w, bkeys, nb_stride);
-}
-
 // ---------------------------------------------------------------------------
 // Selection: one CTA (1024 threads) per segment finds the k best of n keys
 // (key 0 = absent) by (key desc, index asc) and writes their ids ascending.
-//   * small n (<= 16384): the keys live in shared memory; radix passes of
-//     8 bits and the ordered output pass all read shared memory;
-//   * large n: one global pass builds a 15-bit histogram, a second collects
-//     the keys of the threshold bucket (<= 12288 of them; otherwise a global
-//     radix pass per remaining digit), the exact threshold comes from an
-//     in-smem radix over those candidates, and a last global pass writes the
-//     selection in index order.
+// Keys are read in chunks of 16384 (16 consecutive keys per thread, four
+// 16-byte loads), so every thread keeps 64 bytes in flight per chunk.
+//   * small n (<= 16384): one chunk; the keys stay in registers through 8-bit
+//     radix passes (shared-memory histograms) and the ordered output;
+//   * large n: pass A builds a 15-bit histogram and finds the threshold
+//     bucket; pass B collects, in index order, the ids of the keys above the
+//     bucket and the (low bits, id) of the keys inside it (<= 12288); the
+//     exact threshold comes from radix passes over those candidates in shared
+//     memory, and the two ordered lists are merged into the output without a
+//     third pass over the keys.  A bucket with more than 12288 keys falls
+//     back to global radix passes and an ordered output pass.
 // Output rule: key > T, or key == T among the first `rem` equal keys in
-// index order, goes to position (#greater before) + min(#equal before, rem).
+// index order; ids leave in ascending order.
 // ---------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
-constexpr int kSelSmallMax = 16384;
-constexpr int kHist1Bits = 15;
-constexpr int kHist1Bins = 1 << kHist1Bits;
+constexpr int kSelPer = 16;                          // keys per thread per chunk
+constexpr int kSelChunk = kSelThreads * kSelPer;     // 16384
+constexpr int kSelSmallMax = kSelChunk;
+constexpr int kHist1Bits = kSelHistBits;
+constexpr int kHist1Bins = kSelHistBins;
 constexpr int kLowBits = 32 - kHist1Bits;  // 17
+constexpr uint32_t kLowMask = (1u << kLowBits) - 1u;
 constexpr int kCandCap = 12288;
+constexpr int kSelMaxK = CSA2_MAX_TOPK;
+// large-path shared memory: the histogram, later reused for the lists
+constexpr int kSelLargeWords = kHist1Bins;
+static_assert(kSelMaxK + 2 * kCandCap + 512 + kSelMaxK <= kSelLargeWords, "selection lists exceed the histogram");
 
 template <int KIND>
 __device__ __forceinline__ uint32_t sel_key(const void* in, int64_t base, int64_t i, int64_t n) {
@@ -149,6 +95,41 @@ __device__ __forceinline__ uint32_t sel_key(const void* in, int64_t base, int64_
   if (KIND == kSelScores) return rank_key(static_cast<const float*>(in)[base + i]);
   return static_cast<const uint32_t*>(in)[base + i];
 }
+
+// Keys i0 .. i0+15 (0 beyond n); 16-byte loads when the run is whole and aligned.
+template <int KIND>
+__device__ __forceinline__ void load_keys(const void* in, int64_t base, int64_t i0, int64_t n,
+                                          uint32_t (&kk)[kSelPer]) {
+  if (i0 + kSelPer <= n && ((base + i0) & 3) == 0) {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint32_t*>(in) + base + i0);
+    uint4 v[kSelPer / 4];
+#pragma unroll
+    for (int j = 0; j < kSelPer / 4; ++j) v[j] = __ldg(p + j);
+#pragma unroll
+    for (int j = 0; j < kSelPer / 4; ++j) {
+      kk[4 * j] = v[j].x, kk[4 * j + 1] = v[j].y, kk[4 * j + 2] = v[j].z, kk[4 * j + 3] = v[j].w;
+      if (KIND == kSelScores) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kk[4 * j + e] = rank_key(__uint_as_float(kk[4 * j + e]));
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kSelPer; ++e) kk[e] = sel_key<KIND>(in, base, i0 + e, n);
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ int32_t sel_id(const int32_t* pool, int s, int P, int64_t i) {
+  if (KIND == kSelPoolCand) return pool[int64_t(s) * P + i / kBlk] * kBlk + int32_t(i % kBlk);
+  return static_cast<int32_t>(i);
+}
+
+struct SelShared {
+  uint32_t warp_sums[32];
+  uint32_t total;
+  uint32_t digit, rem;
+};
 
 // Block-wide exclusive scan of one uint32 per thread; returns the exclusive
 // prefix and writes the total to *total.
@@ -179,17 +160,14 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   return r;
 }
 
-struct SelShared {
-  uint32_t warp_sums[32];
-  uint32_t total;
-  uint32_t digit, rem, found;
-  uint32_t ncand;
-};
-
-// Finds, among `cnt` bins of `hist` scanned from the top, the bin where the
+// Finds, among `nbins` bins of `hist` scanned from the top, the bin where the
 // running count reaches `need`; returns it in sh.digit with the count still
 // needed from it in sh.rem.  (Whole block; `hist` in shared memory.)
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32_t need, SelShared& sh) {
+  if (threadIdx.x == 0) {  // defined result even for an inconsistent histogram
+    sh.digit = 0;
+    sh.rem = need;
+  }
   const int per = (nbins + kSelThreads - 1) / kSelThreads;
   // thread j owns bins [nbins - per*(j+1), nbins - per*j) (top bins first)
   const int hi = nbins - per * int(threadIdx.x);
@@ -211,17 +189,87 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32
   __syncthreads();
 }
 
-template <int KIND, bool SMALL>
-__device__ __forceinline__ uint32_t get_key(const uint32_t* ks, const void* in, int64_t base, int64_t i, int64_t n) {
-  if (SMALL) return i < n ? ks[i] : 0u;
-  return sel_key<KIND>(in, base, i, n);
+// Adds one to hist[bin] for an active lane.  (Aggregating equal bins across
+// the warp with match.any first was measured slower than the plain atomics.)
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  if (active) atomicAdd(&hist[bin], 1u);
+}
+
+// Copies a segment's histogram row (written by the kernel that produced the
+// keys) into shared memory and zeroes the row for the next call; returns this
+// thread's share of the key count.
+template <int NB>
+__device__ __forceinline__ uint32_t take_hist(uint32_t* __restrict__ gh, uint32_t* __restrict__ hist) {
+  constexpr int kVec = NB / 4 / kSelThreads;  // uint4 per thread
+  static_assert(kVec >= 1 && NB % (4 * kSelThreads) == 0, "histogram rows are whole uint4 per thread");
+  uint4 v[kVec];
+  uint4* g4 = reinterpret_cast<uint4*>(gh);
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) v[j] = __ldcg(g4 + threadIdx.x + j * kSelThreads);
+  uint32_t sum = 0;
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) {
+    reinterpret_cast<uint4*>(hist)[threadIdx.x + j * kSelThreads] = v[j];
+    sum += v[j].x + v[j].y + v[j].z + v[j].w;
+    if ((v[j].x | v[j].y | v[j].z | v[j].w) != 0u) g4[threadIdx.x + j * kSelThreads] = make_uint4(0, 0, 0, 0);
+  }
+  return sum;
+}
+
+// Position of the first element >= x in the ascending list a[0..n).
+__device__ __forceinline__ uint32_t lower_bound_u32(const uint32_t* a, uint32_t n, uint32_t x) {
+  uint32_t lo = 0, hi = n;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi) >> 1;
+    if (a[mid] < x) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// Ordered output pass over the keys in global memory (fallback of the large path).
+template <int KIND>
+__device__ void ordered_output_global(const void* in, int64_t base, int64_t n, uint32_t T, uint32_t rem,
+                                      const int32_t* pool, int s, int P, int32_t* o, int k, SelShared& sh) {
+  const int tid = threadIdx.x;
+  uint32_t run_gt = 0, run_eq = 0;
+  for (int64_t c0 = 0; c0 < n; c0 += kSelChunk) {
+    uint32_t kk[kSelPer];
+    const int64_t i0 = c0 + int64_t(tid) * kSelPer;
+    load_keys<KIND>(in, base, i0, n, kk);
+    uint32_t gt = 0, eq = 0;
+#pragma unroll
+    for (int e = 0; e < kSelPer; ++e) {
+      gt += (kk[e] > T);
+      eq += (kk[e] == T && kk[e] != 0u);
+    }
+    const uint32_t ex = block_exclusive_scan((gt << 16) | eq, sh.warp_sums, &sh.total);
+    const uint32_t tot = sh.total;
+    uint32_t g = run_gt + (ex >> 16), q = run_eq + (ex & 0xFFFFu);
+#pragma unroll
+    for (int e = 0; e < kSelPer; ++e) {
+      const uint32_t key = kk[e];
+      if (key > T) {
+        const uint32_t at = g + min(q, rem);
+        if (at < uint32_t(k)) o[at] = sel_id<KIND>(pool, s, P, i0 + e);
+        ++g;
+      } else if (key == T && key != 0u) {
+        if (q < rem && g + q < uint32_t(k)) o[g + q] = sel_id<KIND>(pool, s, P, i0 + e);
+        ++q;
+      }
+    }
+    run_gt += tot >> 16;
+    run_eq += tot & 0xFFFFu;
+  }
+  const uint32_t nsel = run_gt + min(run_eq, rem);
+  for (int j = int(nsel) + tid; j < k; j += kSelThreads) o[j] = -1;
 }
 
 template <int KIND, bool SMALL>
 __global__ void __launch_bounds__(kSelThreads) k_select(const void* __restrict__ in, int64_t in_stride,
                                                         const int32_t* __restrict__ seg_eff, int P,
                                                         const int32_t* __restrict__ pool, int k,
-                                                        int32_t* __restrict__ out) {
+                                                        int32_t* __restrict__ out, uint32_t* __restrict__ ghist) {
   extern __shared__ __align__(16) uint32_t dsm[];
   __shared__ SelShared sh;
   const int s = blockIdx.x;
@@ -232,29 +280,60 @@ __global__ void __launch_bounds__(kSelThreads) k_select(const void* __restrict__
   else n = int64_t(P) * kBlk;
   const int64_t base = int64_t(s) * in_stride;
   int32_t* o = out + int64_t(s) * k;
-  uint32_t* ks = dsm;  // small: the keys; large: unused
 
-  uint32_t T = 0, rem = 0, total;
   if (SMALL) {
-    // ---- keys into shared memory, present count ----
+    // ---- one chunk: this thread's 16 keys stay in registers ----
+    uint32_t kk[kSelPer];
+    const int64_t i0 = int64_t(tid) * kSelPer;
+    load_keys<KIND>(in, base, i0, n, kk);
     uint32_t present = 0;
-    for (int64_t i = tid; i < n; i += kSelThreads) {
-      const uint32_t key = sel_key<KIND>(in, base, i, n);
-      ks[i] = key;
-      present += (key != 0u);
-    }
+#pragma unroll
+    for (int e = 0; e < kSelPer; ++e) present += (kk[e] != 0u);
     block_exclusive_scan(present, sh.warp_sums, &sh.total);
-    total = sh.total;
-    if (total > uint32_t(k)) {
-      uint32_t* hist = dsm + kSelSmallMax;
+    const uint32_t total = sh.total;
+    uint32_t T = 0, rem = 0;
+    if (ghist) {
+      // the top HB bits from the producer's histogram; the low bits by radix
+      // digits of up to 8 bits over the keys of the threshold bucket only
+      constexpr int HB = (KIND == kSelPoolCand) ? kCandHistBits : kHist1Bits;
+      constexpr int NB = 1 << HB;
+      uint32_t* hist = dsm;       // NB
+      uint32_t* h2 = dsm + NB;    // 256
+      take_hist<NB>(ghist + int64_t(s) * NB, hist);
+      __syncthreads();
+      if (total > uint32_t(k)) {
+        find_bin(hist, NB, uint32_t(k), sh);
+        uint32_t prefix = sh.digit << (32 - HB), pmask = ~((1u << (32 - HB)) - 1u);
+        rem = sh.rem;
+        for (int hi = 31 - HB; hi >= 0; hi -= 8) {
+          const int width = min(8, hi + 1), shift = hi - width + 1;
+          const uint32_t dm = (1u << width) - 1u;
+          if (tid < 256) h2[tid] = 0;
+          __syncthreads();
+#pragma unroll
+          for (int e = 0; e < kSelPer; ++e) {
+            const uint32_t key = kk[e];
+            hist_add(h2, (key >> shift) & dm, key != 0u && (key & pmask) == prefix);
+          }
+          __syncthreads();
+          find_bin(h2, 1 << width, rem, sh);
+          prefix |= sh.digit << shift;
+          pmask |= dm << shift;
+          rem = sh.rem;
+        }
+        T = prefix;
+      }
+    } else if (total > uint32_t(k)) {
+      uint32_t* hist = dsm;  // 256 bins
       uint32_t prefix = 0, pmask = 0;
       rem = uint32_t(k);
       for (int shift = 24; shift >= 0; shift -= 8) {
         if (tid < 256) hist[tid] = 0;
         __syncthreads();
-        for (int64_t i = tid; i < n; i += kSelThreads) {
-          const uint32_t key = ks[i];
-          if (key != 0u && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+#pragma unroll
+        for (int e = 0; e < kSelPer; ++e) {
+          const uint32_t key = kk[e];
+          hist_add(hist, (key >> shift) & 255u, key != 0u && (key & pmask) == prefix);
         }
         __syncthreads();
         find_bin(hist, 256, rem, sh);
@@ -264,165 +343,240 @@ __global__ void __launch_bounds__(kSelThreads) k_select(const void* __restrict__
       }
       T = prefix;
     }
-  } else {
-    // ---- pass A: 15-bit histogram of the present keys ----
-    uint32_t* hist = dsm;                        // kHist1Bins
-    uint32_t* cand = dsm + kHist1Bins;           // kCandCap low parts
-    for (int i = tid; i < kHist1Bins; i += kSelThreads) hist[i] = 0;
-    __syncthreads();
-    uint32_t present = 0;
-    for (int64_t i0 = int64_t(tid) * 4; i0 < n; i0 += int64_t(kSelThreads) * 4) {
-      uint32_t kk[4];
-      if (KIND == kSelBlockKeys && i0 + 3 < n && ((base + i0) & 3) == 0) {
-        const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const uint32_t*>(in) + base + i0);
-        kk[0] = v.x, kk[1] = v.y, kk[2] = v.z, kk[3] = v.w;
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) kk[j] = sel_key<KIND>(in, base, i0 + j, n);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (kk[j] != 0u) {
-          ++present;
-          atomicAdd(&hist[kk[j] >> kLowBits], 1u);
-        }
-    }
-    block_exclusive_scan(present, sh.warp_sums, &sh.total);
-    total = sh.total;
-    if (total > uint32_t(k)) {
-      find_bin(hist, kHist1Bins, uint32_t(k), sh);
-      const uint32_t b1 = sh.digit, need = sh.rem, cnt = hist[b1];
-      __syncthreads();
-      if (cnt <= uint32_t(kCandCap)) {
-        // ---- pass B: collect the low bits of the threshold bucket's keys ----
-        if (tid == 0) sh.ncand = 0;
-        __syncthreads();
-        for (int64_t i = tid; i < n; i += kSelThreads) {
-          const uint32_t key = sel_key<KIND>(in, base, i, n);
-          if (key != 0u && (key >> kLowBits) == b1) cand[atomicAdd(&sh.ncand, 1u)] = key & ((1u << kLowBits) - 1u);
-        }
-        __syncthreads();
-        const uint32_t nc = sh.ncand;
-        // exact threshold among the candidates: digits of 9 and 8 bits
-        uint32_t prefix = 0, pmask = 0, r = need;
-        uint32_t* h2 = hist;  // reuse (first 512 bins)
-        const int shifts[2] = {8, 0};
-        const int widths[2] = {9, 8};
-        for (int d = 0; d < 2; ++d) {
-          const int nb = 1 << widths[d];
-          for (int i = tid; i < nb; i += kSelThreads) h2[i] = 0;
-          __syncthreads();
-          const uint32_t dm = uint32_t(nb - 1);
-          for (uint32_t i = tid; i < nc; i += kSelThreads) {
-            const uint32_t low = cand[i];
-            if ((low & pmask) == prefix) atomicAdd(&h2[(low >> shifts[d]) & dm], 1u);
-          }
-          __syncthreads();
-          find_bin(h2, nb, r, sh);
-          prefix |= sh.digit << shifts[d];
-          pmask |= dm << shifts[d];
-          r = sh.rem;
-        }
-        T = (b1 << kLowBits) | prefix;
-        rem = r;
-      } else {
-        // more than kCandCap keys share the threshold bucket: finish with
-        // global radix passes over the low 17 bits (9 + 8)
-        uint32_t prefix = b1 << kLowBits, pmask = ~((1u << kLowBits) - 1u), r = need;
-        uint32_t* h2 = hist;
-        const int shifts[2] = {8, 0};
-        const int widths[2] = {9, 8};
-        for (int d = 0; d < 2; ++d) {
-          const int nb = 1 << widths[d];
-          for (int i = tid; i < nb; i += kSelThreads) h2[i] = 0;
-          __syncthreads();
-          const uint32_t dm = uint32_t(nb - 1);
-          for (int64_t i = tid; i < n; i += kSelThreads) {
-            const uint32_t key = sel_key<KIND>(in, base, i, n);
-            if (key != 0u && (key & pmask) == prefix) atomicAdd(&h2[(key >> shifts[d]) & dm], 1u);
-          }
-          __syncthreads();
-          find_bin(h2, nb, r, sh);
-          prefix |= sh.digit << shifts[d];
-          pmask |= dm << shifts[d];
-          r = sh.rem;
-        }
-        T = prefix;
-        rem = r;
-      }
-    }
-  }
-  if (total <= uint32_t(k)) {
-    T = 0;
-    rem = 0;
-  }
-
-  // ---- ordered output pass ----
-  uint32_t run_gt = 0, run_eq = 0;
-  for (int64_t t0 = 0; t0 < n; t0 += 4 * kSelThreads) {
-    uint32_t kk[4];
+    // ---- ordered output ----
     uint32_t gt = 0, eq = 0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      kk[j] = get_key<KIND, SMALL>(ks, in, base, t0 + 4 * tid + j, n);
-      gt += (kk[j] > T);
-      eq += (kk[j] == T && kk[j] != 0u);
+    for (int e = 0; e < kSelPer; ++e) {
+      gt += (kk[e] > T);
+      eq += (kk[e] == T && kk[e] != 0u);
     }
-    const uint32_t packed = (gt << 16) | eq;
-    const uint32_t ex = block_exclusive_scan(packed, sh.warp_sums, &sh.total);
+    const uint32_t ex = block_exclusive_scan((gt << 16) | eq, sh.warp_sums, &sh.total);
     const uint32_t tot = sh.total;
-    uint32_t g = run_gt + (ex >> 16), e = run_eq + (ex & 0xFFFFu);
+    uint32_t g = ex >> 16, q = ex & 0xFFFFu;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t i = t0 + 4 * tid + j;
-      const uint32_t key = kk[j];
-      if (key > T || (key == T && key != 0u)) {
-        int64_t id;
-        if (KIND == kSelPoolCand) id = int64_t(pool[int64_t(s) * P + i / kBlk]) * kBlk + (i % kBlk);
-        else id = i;
-        if (key > T) {
-          o[g + min(e, rem)] = static_cast<int32_t>(id);
-          ++g;
-        } else {
-          if (e < rem) o[g + e] = static_cast<int32_t>(id);
-          ++e;
-        }
+    for (int e = 0; e < kSelPer; ++e) {
+      const uint32_t key = kk[e];
+      if (key > T) {
+        const uint32_t at = g + min(q, rem);
+        if (at < uint32_t(k)) o[at] = sel_id<KIND>(pool, s, P, i0 + e);
+        ++g;
+      } else if (key == T && key != 0u) {
+        if (q < rem && g + q < uint32_t(k)) o[g + q] = sel_id<KIND>(pool, s, P, i0 + e);
+        ++q;
       }
     }
-    run_gt += tot >> 16;
-    run_eq += tot & 0xFFFFu;
+    const uint32_t nsel = (tot >> 16) + min(tot & 0xFFFFu, rem);
+    for (int j = int(nsel) + tid; j < k; j += kSelThreads) o[j] = -1;
+    return;
   }
-  const uint32_t nsel = run_gt + min(run_eq, rem);
-  for (int j = int(nsel) + tid; j < k; j += kSelThreads) o[j] = -1;
+
+  // ---- large n, pass A: 15-bit histogram of the present keys ----
+  uint32_t* hist = dsm;
+  uint32_t present = 0;
+  if (ghist) {
+    present = take_hist<kHist1Bins>(ghist + int64_t(s) * kHist1Bins, hist);
+  } else {
+    for (int i = tid; i < kHist1Bins; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    uint32_t kk[kSelPer], nx[kSelPer];
+    load_keys<KIND>(in, base, int64_t(tid) * kSelPer, n, kk);
+    for (int64_t c0 = 0; c0 < n; c0 += kSelChunk) {
+      if (c0 + kSelChunk < n) load_keys<KIND>(in, base, c0 + kSelChunk + int64_t(tid) * kSelPer, n, nx);
+#pragma unroll
+      for (int e = 0; e < kSelPer; ++e) {
+        present += (kk[e] != 0u);
+        hist_add(hist, kk[e] >> kLowBits, kk[e] != 0u);
+      }
+#pragma unroll
+      for (int e = 0; e < kSelPer; ++e) kk[e] = nx[e];
+    }
+  }
+  __syncthreads();
+  block_exclusive_scan(present, sh.warp_sums, &sh.total);
+  const uint32_t total = sh.total;
+  const bool all = total <= uint32_t(k);
+  uint32_t b1 = 0, need = 0, cnt = 0;
+  if (!all) {
+    find_bin(hist, kHist1Bins, uint32_t(k), sh);
+    b1 = sh.digit;
+    need = sh.rem;
+    cnt = hist[b1];
+  }
+  __syncthreads();  // the histogram's memory is reused below
+
+  if (!all && cnt > uint32_t(kCandCap)) {
+    // more than kCandCap keys share the threshold bucket: global radix passes
+    // over the low 17 bits (9 + 8), then an ordered pass over the keys
+    uint32_t prefix = b1 << kLowBits, pmask = ~kLowMask, r = need;
+    uint32_t* h2 = dsm;
+    const int shifts[2] = {8, 0};
+    const int widths[2] = {9, 8};
+    for (int d = 0; d < 2; ++d) {
+      const int nb = 1 << widths[d];
+      for (int i = tid; i < nb; i += kSelThreads) h2[i] = 0;
+      __syncthreads();
+      const uint32_t dm = uint32_t(nb - 1);
+      for (int64_t c0 = 0; c0 < n; c0 += kSelChunk) {
+        uint32_t kk[kSelPer];
+        load_keys<KIND>(in, base, c0 + int64_t(tid) * kSelPer, n, kk);
+#pragma unroll
+        for (int e = 0; e < kSelPer; ++e)
+          hist_add(h2, (kk[e] >> shifts[d]) & dm, kk[e] != 0u && (kk[e] & pmask) == prefix);
+      }
+      __syncthreads();
+      find_bin(h2, nb, r, sh);
+      prefix |= sh.digit << shifts[d];
+      pmask |= dm << shifts[d];
+      r = sh.rem;
+    }
+    ordered_output_global<KIND>(in, base, n, prefix, r, pool, s, P, o, k, sh);
+    return;
+  }
+
+  // ---- pass B: ordered lists of the keys above the bucket and inside it ----
+  uint32_t* A = dsm;                     // [kSelMaxK] ids above the bucket (all present ids if `all`)
+  uint32_t* Clow = A + kSelMaxK;         // [kCandCap] low bits of the bucket's keys
+  uint32_t* Cidx = Clow + kCandCap;      // [kCandCap] their ids
+  uint32_t* h2 = Cidx + kCandCap;        // [512]
+  uint32_t* Csel = h2 + 512;             // [kSelMaxK] selected bucket ids
+  uint32_t run_a = 0, run_c = 0;
+  {
+    uint32_t kk[kSelPer], nx[kSelPer];
+    load_keys<KIND>(in, base, int64_t(tid) * kSelPer, n, kk);
+    for (int64_t c0 = 0; c0 < n; c0 += kSelChunk) {
+      if (c0 + kSelChunk < n) load_keys<KIND>(in, base, c0 + kSelChunk + int64_t(tid) * kSelPer, n, nx);
+      uint32_t na = 0, nc = 0;
+#pragma unroll
+      for (int e = 0; e < kSelPer; ++e) {
+        const uint32_t key = kk[e], hi = key >> kLowBits;
+        if (key != 0u) {
+          if (all || hi > b1) ++na;
+          else if (hi == b1) ++nc;
+        }
+      }
+      const uint32_t ex = block_exclusive_scan((na << 16) | nc, sh.warp_sums, &sh.total);
+      const uint32_t tot = sh.total;
+      uint32_t a = run_a + (ex >> 16), c = run_c + (ex & 0xFFFFu);
+      const uint32_t i0 = uint32_t(c0) + uint32_t(tid) * kSelPer;
+#pragma unroll
+      for (int e = 0; e < kSelPer; ++e) {
+        const uint32_t key = kk[e], hi = key >> kLowBits;
+        if (key != 0u) {
+          if (all || hi > b1) {
+            if (a < uint32_t(kSelMaxK)) A[a] = i0 + e;
+            ++a;
+          } else if (hi == b1) {
+            if (c < uint32_t(kCandCap)) {
+              Clow[c] = key & kLowMask;
+              Cidx[c] = i0 + e;
+            }
+            ++c;
+          }
+        }
+      }
+      run_a += tot >> 16;
+      run_c += tot & 0xFFFFu;
+#pragma unroll
+      for (int e = 0; e < kSelPer; ++e) kk[e] = nx[e];
+    }
+  }
+  __syncthreads();
+  // (the list lengths only exceed their capacities if the histogram and the
+  // keys disagree, i.e. after a producer failure that already set a flag)
+  run_a = min(run_a, uint32_t(kSelMaxK));
+  if (all) {
+    for (uint32_t i = tid; i < run_a; i += kSelThreads)
+      if (i < uint32_t(k)) o[i] = sel_id<KIND>(pool, s, P, A[i]);
+    for (int j = int(run_a) + tid; j < k; j += kSelThreads) o[j] = -1;
+    return;
+  }
+  // exact threshold inside the bucket: digits of 9 and 8 bits over the candidates
+  const uint32_t nc = min(run_c, uint32_t(kCandCap));
+  uint32_t prefix = 0, pmask = 0, r = need;
+  {
+    const int shifts[2] = {8, 0};
+    const int widths[2] = {9, 8};
+    for (int d = 0; d < 2; ++d) {
+      const int nb = 1 << widths[d];
+      for (int i = tid; i < nb; i += kSelThreads) h2[i] = 0;
+      __syncthreads();
+      const uint32_t dm = uint32_t(nb - 1);
+      for (uint32_t i0 = 0; i0 < nc; i0 += kSelThreads) {
+        const uint32_t i = i0 + tid;
+        const uint32_t low = i < nc ? Clow[i] : 0u;
+        hist_add(h2, (low >> shifts[d]) & dm, i < nc && (low & pmask) == prefix);
+      }
+      __syncthreads();
+      find_bin(h2, nb, r, sh);
+      prefix |= sh.digit << shifts[d];
+      pmask |= dm << shifts[d];
+      r = sh.rem;
+    }
+  }
+  // the bucket's selected ids in index order: low > prefix, or == prefix among the first r
+  {
+    const uint32_t per = (nc + kSelThreads - 1) / kSelThreads;
+    const uint32_t lo = min(nc, per * tid), hi = min(nc, lo + per);
+    uint32_t gt = 0, eq = 0;
+    for (uint32_t i = lo; i < hi; ++i) {
+      gt += (Clow[i] > prefix);
+      eq += (Clow[i] == prefix);
+    }
+    const uint32_t ex = block_exclusive_scan((gt << 16) | eq, sh.warp_sums, &sh.total);
+    uint32_t g = ex >> 16, q = ex & 0xFFFFu;
+    for (uint32_t i = lo; i < hi; ++i) {
+      if (Clow[i] > prefix) {
+        const uint32_t at = g + min(q, r);
+        if (at < need) Csel[at] = Cidx[i];
+        ++g;
+      } else if (Clow[i] == prefix) {
+        if (q < r && g + q < need) Csel[g + q] = Cidx[i];
+        ++q;
+      }
+    }
+  }
+  __syncthreads();
+  // merge the two ascending lists: k - need ids above the bucket, need from it
+  const uint32_t na = run_a;
+  for (uint32_t i = tid; i < na; i += kSelThreads) {
+    const uint32_t at = i + lower_bound_u32(Csel, need, A[i]);
+    if (at < uint32_t(k)) o[at] = sel_id<KIND>(pool, s, P, A[i]);
+  }
+  for (uint32_t j = tid; j < need; j += kSelThreads) {
+    const uint32_t at = j + lower_bound_u32(A, na, Csel[j]);
+    if (at < uint32_t(k)) o[at] = sel_id<KIND>(pool, s, P, Csel[j]);
+  }
 }
 
 template <int KIND>
 void launch_select_kind(const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P, const int32_t* pool,
-                        int k, int32_t* out, int64_t n_bound, cudaStream_t st) {
+                        int k, int32_t* out, uint32_t* hist, int64_t n_bound, cudaStream_t st) {
   if (n_bound <= kSelSmallMax) {
-    const size_t smem = (kSelSmallMax + 256) * sizeof(uint32_t);
-    cudaFuncSetAttribute(k_select<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out);
+    constexpr int NB = (KIND == kSelPoolCand) ? kCandHistBins : kHist1Bins;
+    const size_t smem = (hist ? NB + 256 : 256) * sizeof(uint32_t);
+    cudaFuncSetAttribute(k_select<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         int((NB + 256) * sizeof(uint32_t)));
+    k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist);
   } else {
-    const size_t smem = (kHist1Bins + kCandCap) * sizeof(uint32_t);
+    const size_t smem = kSelLargeWords * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    k_select<KIND, false><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out);
+    k_select<KIND, false><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist);
   }
 }
 
 void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P,
-                   const int32_t* pool, int k, int32_t* out, cudaStream_t st) {
+                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st) {
   if (S == 0) return;
   // n per segment is at most the row stride of the input
   switch (kind) {
     case kSelBlockKeys:
-      launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, in_stride, st);
+      launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
       break;
     case kSelScores:
-      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, in_stride, st);
+      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
       break;
     case kSelPoolCand:
-      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, in_stride, st);
+      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
       break;
   }
 }

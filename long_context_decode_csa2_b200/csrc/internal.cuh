@@ -30,6 +30,9 @@ csa2_status fail(csa2_status code, const std::string& msg);
 csa2_status check_launch(const char* what);
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+// Row stride (in keys) of the per-block key arrays: whole 16-byte groups, so
+// every row starts 16-byte aligned for vector loads.
+inline int64_t block_key_stride(int64_t len) { return int64_t(round_up(size_t((len + 7) / 8), 4)); }
 
 // ---------------------------------------------------------------------------
 // Segments: a "segment" is one ranking problem (a decode sequence, or one
@@ -43,6 +46,17 @@ struct SegDesc {
   int64_t cache_rows;      // capacity of the cache
 };
 
+// Selection histograms: one row per segment in the workspace over the top
+// bits of the rank keys (15 bits for block keys, 12 bits for the 16384 pool
+// candidates, whose row must stay small next to the keys themselves).  The
+// kernel that writes the keys adds each present key to its bin; the
+// selection reads the row and leaves it zeroed for the next call (the
+// workspace starts zero-filled).
+constexpr int kSelHistBits = 15;
+constexpr int kSelHistBins = 1 << kSelHistBits;
+constexpr int kCandHistBits = 12;
+constexpr int kCandHistBins = 1 << kCandHistBits;
+
 // ---------------------------------------------------------------------------
 // Kernel launchers (each returns after enqueueing on `st`).
 // ---------------------------------------------------------------------------
@@ -55,19 +69,21 @@ size_t scan_tc_prefix_ints(int S);
 csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, int32_t* seg_eff,
                            int32_t* tile_start, int S, const uint8_t* q_codes, const uint8_t* q_scales,
                            const float* w, uint32_t* bkeys, int64_t nb_stride, float* scores, int64_t score_stride,
-                           uint32_t* status, cudaStream_t st);
+                           uint32_t* hist, uint32_t* status, cudaStream_t st);
 
 // Scores of pool candidates 8*pool[s][i/8] + i%8 -> keys [S][P*8] (0 = absent),
 // on the tensor cores (gathered 8-row TMA boxes).
 csa2_status launch_pool_tc(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
                            int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
-                           const int32_t* pool, int P, uint32_t* ckeys, uint32_t* status, cudaStream_t st);
+                           const int32_t* pool, int P, uint32_t* ckeys, uint32_t* hist, uint32_t* status,
+                           cudaStream_t st);
 
-// Prefill scan: block keys [T][nb_stride] for every query against the visible
-// prefix of one sequence.
-void launch_prefill_scan(const uint8_t* kcodes, const uint8_t* kscales, int64_t row0, const int32_t* vis, int T,
-                         int64_t max_vis, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
-                         uint32_t* bkeys, int64_t nb_stride, cudaStream_t st);
+// Prefill scan on the tensor cores: block keys [T][nb_stride] of every query
+// against the visible prefix (vis[i] entries from row0) of one sequence.
+csa2_status launch_prefill_tc(const uint8_t* kcodes, const uint8_t* kscales, int64_t row0, int64_t cache_rows,
+                              const int32_t* vis, int T, int64_t max_vis, const uint8_t* q_codes,
+                              const uint8_t* q_scales, const float* w, uint32_t* bkeys, int64_t nb_stride,
+                              uint32_t* status, cudaStream_t st);
 
 // Visible entry counts of prefill queries.
 void launch_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entries, int32_t* vis, uint32_t* status,
@@ -80,8 +96,10 @@ enum SelectKind : int {
   kSelScores = 1,     // fp32 scores, n = seg_eff, id = index
   kSelPoolCand = 2,   // u32 keys, n = P*8, id = 8*pool[i/8] + i%8
 };
+// `hist` (or null): the keys' histogram rows, zeroed on return: [S][kSelHistBins]
+// for block keys, [S][kCandHistBins] for pool candidates.
 void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P,
-                   const int32_t* pool, int k, int32_t* out, cudaStream_t st);
+                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st);
 
 // Attention partials + combine.
 struct AttnArgs {

@@ -1,0 +1,355 @@
+// Causal multi-query indexer scan for prefill on the 5th-generation tensor
+// cores (sm_100a): the block-scaled FP4 GEMM of T indexer queries (4 heads x
+// 128) against the visible indexer-K rows of one sequence, reduced to block
+// maxima per query.
+//
+// Source: "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression",
+// section "三个方向一起压小缓存" (FP4 indexer q/k; every 8 positions reduced to
+// their best score; pool of at most 2048 blocks), with the causal visibility
+// of compressed entries to raw query positions (section "后 20 层干脆共用一份
+// KV": m raw tokens per entry).
+//
+// Work item = (group of 8 consecutive queries, tile of 128 positions); items
+// run group-major, so a persistent CTA keeps one group's B operand for many
+// key tiles.  Per item:
+//   * warp 0 loads the tile's 128 code rows with one TMA tile copy (64-byte
+//     swizzle) and its 128 scale words with a bulk copy; when the group
+//     changes it also writes the group's B operand, 128 rows of which row
+//     16j + 4h + b holds block b of head h of query j (zeros elsewhere), and
+//     the queries' scale contexts;
+//   * warp 1 issues two tcgen05.mma kind::mxf4 (M = 128 positions, N = 128,
+//     K = 64) with every block scale = 1, so each accumulator is an exact
+//     block dot D/4;
+//   * two teams of four epilogue warps read each position's 16 accumulators
+//     per query, form the exact score (the same rounding as the decode scan),
+//     mask positions the query cannot see, and write the maximum of every 8
+//     positions as one rank key.
+// Items past the visibility of every query of a group are skipped by all
+// roles alike.  Every wait is time-bounded (CSA2_DEV_TIMEOUT on expiry).
+#include <algorithm>
+
+#include "device_common.cuh"
+#include "sm100.cuh"
+
+namespace csa2 {
+
+namespace {
+
+constexpr int kQG = 8;                   // queries per group
+constexpr int kN = 16 * kQG;             // MMA N: 4 heads x 4 blocks per query
+constexpr int kPT = 128;                 // positions per item (MMA M)
+constexpr int kSt = 6;                   // smem ring
+constexpr int kAc = 3;                   // TMEM accumulator ring, kN columns each
+constexpr int kTmemCols = 512;
+constexpr uint32_t kSf = 448;            // scale-factor columns (all 2^0)
+constexpr int kTeams = 2;                // epilogue teams of 4 warps
+constexpr int kThr = 64 + 128 * kTeams;  // producer, MMA, epilogue warps
+constexpr uint32_t kTileBytes = kPT * kIdxCodeBytes;
+static_assert(kAc * kN <= int(kSf), "TMEM accumulators overlap the scale factors");
+
+struct QCtxS {
+  IdxQCtx c;
+  int vis;  // visible entries of this query (0 past the end of the batch)
+};
+
+struct __align__(1024) PfSmem {
+  uint8_t a[kSt][kTileBytes];           // code rows, 64-byte swizzled
+  uint8_t bop[kSt][kN * kIdxCodeBytes]; // B operand of the stage's group
+  uint32_t sc[kSt][kPT];                // E8M0 scale words of the rows
+  int2 info[kSt];                       // (group, tile)
+  QCtxS qctx[kSt][kQG];
+  uint64_t full[kSt];
+  uint64_t empty[kSt];
+  uint64_t tfull[kAc];
+  uint64_t tempty[kAc];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort_flag;
+  int built[kSt];                       // group whose B operand each stage holds
+};
+
+struct PfParams {
+  const uint8_t* kscales;
+  const uint8_t* q_codes;   // [T][4][64]
+  const uint8_t* q_scales;  // [T][4][4]
+  const float* w;           // [T][4]
+  const int32_t* vis;       // [T]
+  int T;
+  int64_t row0;
+  int64_t cache_rows;
+  int n_groups;
+  int n_tiles;
+  uint32_t* bkeys;          // [T][nb_stride]
+  int64_t nb_stride;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ void pf_abort(PfSmem& sm, uint32_t* status) {
+  set_status(status, CSA2_DEV_TIMEOUT);
+  atomicExch(&sm.abort_flag, 1);
+}
+__device__ __forceinline__ bool pf_aborted(PfSmem& sm) {
+  return *reinterpret_cast<volatile int*>(&sm.abort_flag) != 0;
+}
+
+// Largest visibility among the group's queries.
+__device__ __forceinline__ int group_vis(const PfParams& p, int g) {
+  int m = 0;
+  for (int j = 0; j < kQG; ++j) {
+    const int qi = g * kQG + j;
+    if (qi < p.T) m = max(m, __ldg(p.vis + qi));
+  }
+  return m;
+}
+
+// Writes group g's B operand and scale contexts into stage s (whole warp).
+__device__ __forceinline__ void build_group(PfSmem& sm, int s, const PfParams& p, int g, int lane) {
+  uint8_t* bo = sm.bop[s];
+#pragma unroll
+  for (int m = 0; m < kN * kIdxCodeBytes / 16 / 32; ++m)
+    *reinterpret_cast<uint4*>(bo + 16 * (lane + 32 * m)) = make_uint4(0, 0, 0, 0);
+  __syncwarp();
+  // 128 chunks of 16 bytes: chunk c = (query j, head h, block b), 4 per lane
+#pragma unroll
+  for (int m = 0; m < kN / 32; ++m) {
+    const int c = lane + 32 * m;
+    const int j = c >> 4, h = (c >> 2) & 3, b = c & 3;
+    const int qi = g * kQG + j;
+    if (qi < p.T) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.q_codes + int64_t(qi) * kHi * 64 + h * 64 + b * 16));
+      const int n = 16 * j + 4 * h + b;
+      *reinterpret_cast<uint4*>(bo + n * 64 + ((b ^ ((n >> 1) & 3)) << 4)) = v;
+    }
+  }
+  if (lane < kQG) {
+    const int qi = g * kQG + lane;
+    QCtxS& q = sm.qctx[s][lane];
+    if (qi < p.T) {
+      make_qctx(q.c, p.q_scales + int64_t(qi) * 16, p.w + int64_t(qi) * kHi);
+      q.vis = __ldg(p.vis + qi);
+    } else {
+      const uint8_t unit[16] = {127, 127, 127, 127, 127, 127, 127, 127, 127, 127, 127, 127, 127, 127, 127, 127};
+      const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+      make_qctx(q.c, unit, zero);
+      q.vis = 0;
+    }
+  }
+  sm100::fence_proxy_async_smem();  // generic writes -> MMA (async proxy) reads
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ CUtensorMap tmap, PfParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  PfSmem& sm = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = p.n_groups * p.n_tiles;
+  const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
+  const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSt; ++s) {
+      sm100::mbar_init(&sm.full[s], 1);
+      sm100::mbar_init(&sm.empty[s], 1 + 4);
+    }
+    for (int a = 0; a < kAc; ++a) {
+      sm100::mbar_init(&sm.tfull[a], 1);
+      sm100::mbar_init(&sm.tempty[a], 4);
+    }
+    sm100::mbar_init(&sm.done, 1);
+    sm.abort_flag = 0;
+    sm100::fence_mbar_init();
+    sm100::tma_prefetch_desc(&tmap);
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc(&sm.tmem_base, kTmemCols);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (warp >= 2 && warp < 6) {  // unit block scales in columns kSf .. kSf+63
+    const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
+#pragma unroll
+    for (int c = 0; c < 64; c += 8) sm100::tmem_st8_same(tmem + lane_base + kSf + c, 0x7F7F7F7Fu);
+    sm100::tmem_st_wait();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane < kSt) sm.built[lane] = -1;
+    __syncwarp();
+    int issued = 0, cg = -1, gmax = 0;
+    for (int it = i0; it < i1; ++it) {
+      const int g = it / p.n_tiles, tile = it - g * p.n_tiles;
+      if (g != cg) {
+        cg = g;
+        gmax = group_vis(p, g);
+      }
+      if (int64_t(tile) * kPT >= gmax) continue;
+      const int t = issued, s = t % kSt, round = t / kSt;
+      const bool ok = round == 0 || sm100::mbar_wait(&sm.empty[s], (round - 1) & 1);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) pf_abort(sm, p.status);
+        break;
+      }
+      if (__any_sync(0xffffffffu, pf_aborted(sm))) break;
+      if (sm.built[s] != g) {
+        build_group(sm, s, p, g, lane);
+        if (lane == 0) sm.built[s] = g;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        sm.info[s] = make_int2(g, tile);
+        const int64_t row = p.row0 + int64_t(tile) * kPT;
+        const int64_t left = p.cache_rows - row;  // > 0 and a multiple of 8
+        const uint32_t sbytes = uint32_t(left < kPT ? left : kPT) * 4u;
+        sm100::mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sbytes);
+        sm100::tma_load_2d(sm.a[s], &tmap, 0, int32_t(row), &sm.full[s]);
+        sm100::bulk_load(sm.sc[s], p.kscales + row * 4, sbytes, &sm.full[s]);
+      }
+      ++issued;
+    }
+    // every copy this warp issued has landed before the CTA exits
+    if (lane == 0)
+      for (int s = 0; s < kSt && s < issued; ++s) {
+        const int last_round = (issued - 1 - s) / kSt;
+        if (!sm100::mbar_wait(&sm.full[s], last_round & 1, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
+      }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = sm100::idesc_mxf4(kPT, kN);
+      const uint32_t sfa = tmem + kSf, sfb = tmem + kSf + 32;
+      int t = 0, cg = -1, gmax = 0;
+      for (int it = i0; it < i1; ++it) {
+        const int g = it / p.n_tiles, tile = it - g * p.n_tiles;
+        if (g != cg) {
+          cg = g;
+          gmax = group_vis(p, g);
+        }
+        if (int64_t(tile) * kPT >= gmax) continue;
+        const int s = t % kSt, a = t % kAc;
+        if (!sm100::mbar_wait(&sm.full[s], (t / kSt) & 1)) {
+          pf_abort(sm, p.status);
+          break;
+        }
+        if (t >= kAc && !sm100::mbar_wait(&sm.tempty[a], ((t / kAc) - 1) & 1)) {
+          pf_abort(sm, p.status);
+          break;
+        }
+        if (pf_aborted(sm)) break;
+        sm100::tc_fence_after();
+        const uint32_t abase = sm100::smem_u32(sm.a[s]);
+        const uint32_t bbase = sm100::smem_u32(sm.bop[s]);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          sm100::mma_mxf4(tmem + a * kN, sm100::smem_desc_k64b(abase + kk * 32), sm100::smem_desc_k64b(bbase + kk * 32),
+                          idesc, uint32_t(kk), sfa, sfb);
+        sm100::mma_commit(&sm.empty[s]);
+        sm100::mma_commit(&sm.tfull[a]);
+        ++t;
+      }
+      sm100::mma_commit(&sm.done);  // all MMAs complete before TMEM is released
+      if (!sm100::mbar_wait(&sm.done, 0, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp & 3;  // TMEM lane quarter of this warp
+    const int team = (warp - 2) >> 2;
+    const uint32_t lane_base = uint32_t(32 * q4) << 16;
+    int t = -1, cg = -1, gmax = 0;
+    for (int it = i0; it < i1; ++it) {
+      const int g = it / p.n_tiles, tile = it - g * p.n_tiles;
+      if (g != cg) {
+        cg = g;
+        gmax = group_vis(p, g);
+      }
+      if (int64_t(tile) * kPT >= gmax) continue;
+      ++t;
+      if (t % kTeams != team) continue;
+      const int s = t % kSt, a = t % kAc;
+      const bool ok = sm100::mbar_wait(&sm.full[s], (t / kSt) & 1) && sm100::mbar_wait(&sm.tfull[a], (t / kAc) & 1);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) pf_abort(sm, p.status);
+        break;
+      }
+      if (__any_sync(0xffffffffu, pf_aborted(sm))) break;
+      sm100::tc_fence_after();
+      const int pl = 32 * q4 + lane;
+      const int64_t pos = int64_t(tile) * kPT + pl;
+      const uint32_t sw = sm.sc[s][pl];
+      const uint32_t tcol = tmem + lane_base + uint32_t(a * kN);
+      uint32_t va[16], vb[16];
+      sm100::tmem_ld16(tcol, va);
+      sm100::tmem_ld_wait(va);
+#pragma unroll
+      for (int j = 0; j < kQG; ++j) {
+        uint32_t(&cur)[16] = (j & 1) ? vb : va;
+        uint32_t(&nxt)[16] = (j & 1) ? va : vb;
+        if (j + 1 < kQG) sm100::tmem_ld16(tcol + 16 * (j + 1), nxt);
+        const QCtxS& q = sm.qctx[s][j];
+        uint32_t key = 0;
+        if (pos < q.vis) key = rank_key(exact_score(cur, sw, q.c));
+        key = group8_max(key);
+        if ((lane & 7) == 0 && pos < q.vis)
+          p.bkeys[int64_t(g * kQG + j) * p.nb_stride + pos / kBlk] = key;
+        if (j + 1 < kQG) sm100::tmem_ld_wait(nxt);
+      }
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        sm100::mbar_arrive(&sm.empty[s]);
+        sm100::mbar_arrive(&sm.tempty[a]);
+      }
+    }
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+csa2_status launch_prefill_tc(const uint8_t* kcodes, const uint8_t* kscales, int64_t row0, int64_t cache_rows,
+                              const int32_t* vis, int T, int64_t max_vis, const uint8_t* q_codes,
+                              const uint8_t* q_scales, const float* w, uint32_t* bkeys, int64_t nb_stride,
+                              uint32_t* status, cudaStream_t st) {
+  if (T == 0 || max_vis == 0) return CSA2_OK;
+  CUtensorMap map;
+  const csa2_status rc = code_map(&map, kcodes, cache_rows, kPT);
+  if (rc != CSA2_OK) return rc;
+  PfParams p{};
+  p.kscales = kscales;
+  p.q_codes = q_codes;
+  p.q_scales = q_scales;
+  p.w = w;
+  p.vis = vis;
+  p.T = T;
+  p.row0 = row0;
+  p.cache_rows = cache_rows;
+  p.n_groups = (T + kQG - 1) / kQG;
+  p.n_tiles = int((max_vis + kPT - 1) / kPT);
+  p.bkeys = bkeys;
+  p.nb_stride = nb_stride;
+  p.status = status;
+  const int64_t n_items = int64_t(p.n_groups) * p.n_tiles;
+  if (n_items > INT32_MAX) return fail(CSA2_ERR_UNSUPPORTED, "csa2_index_prefill: too many query tiles");
+  // more than half of the SM's shared memory, so that one CTA (and one
+  // 512-column TMEM allocation) runs per SM
+  const size_t smem = std::max<size_t>(sizeof(PfSmem) + 1024, 120 * 1024);
+  cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  const int grid = int(std::min<int64_t>(num_sms(), n_items));
+  k_prefill_tc<<<grid, kThr, smem, st>>>(map, p);
+  return CSA2_OK;
+}
+
+}  // namespace csa2

@@ -106,6 +106,8 @@ struct ScanParams {
   int P;
   int items_per_seg;
   uint32_t* ckeys;            // [S][P*8]
+  uint32_t* hist;             // histogram rows of the emitted keys, or null:
+                              // [S][kSelHistBins] (scan), [S][kCandHistBins] (pool)
   uint32_t* status;
 };
 
@@ -379,9 +381,7 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
     const uint32_t lane_base = uint32_t(32 * g) << 16;
     int cur = -1;
     int64_t L = 0;
-    uint32_t qsh[kHi][4];
-    int qlo = 0, qhi = 0, qspread = 0;
-    float wv[kHi];
+    IdxQCtx qc;
     for (int it = i0 + team; it < i1; it += kEpiTeams) {
       const int t = it - i0, s = t % kStages, a = t % kAcc;
       const bool ok =
@@ -396,24 +396,7 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
       if (inf.x != cur) {
         cur = inf.x;
         L = p.seg_eff[cur];
-        qlo = 255;
-        qhi = 0;
-        qspread = 0;
-#pragma unroll
-        for (int h = 0; h < kHi; ++h) {
-          int mn = 255, mx = 0;
-#pragma unroll
-          for (int bb = 0; bb < 4; ++bb) {
-            const int q = p.q_scales[int64_t(cur) * 16 + h * 4 + bb];
-            qsh[h][bb] = uint32_t(q - 127) << 23;
-            mn = min(mn, q);
-            mx = max(mx, q);
-          }
-          qlo = min(qlo, mn);
-          qhi = max(qhi, mx);
-          qspread = max(qspread, mx - mn);
-          wv[h] = p.w[int64_t(cur) * kHi + h];
-        }
+        make_qctx(qc, p.q_scales + int64_t(cur) * 16, p.w + int64_t(cur) * kHi);
       }
       uint32_t swv[kMT];
       int64_t posv[kMT];
@@ -445,49 +428,23 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
         float sc = 0.0f;
         uint32_t key = 0;
         if (pos >= 0 && pos < L) {
-          const int k0 = int(sw & 255u), k1 = int((sw >> 8) & 255u), k2 = int((sw >> 16) & 255u),
-                    k3 = int(sw >> 24);
-          const int kmin = min(min(k0, k1), min(k2, k3)), kmax = max(max(k0, k1), max(k2, k3));
-          const bool fast =
-              (kmax - kmin + qspread <= 9) && (qlo + kmin - 254 >= -100) && (qhi + kmax - 254 <= 100);
-          const uint32_t ksh[4] = {uint32_t(k0) << 23, uint32_t(k1) << 23, uint32_t(k2) << 23, uint32_t(k3) << 23};
-          float d[kHi];
-          if (fast) {
-            // every term and partial sum is exact in fp32
-#pragma unroll
-            for (int h = 0; h < kHi; ++h) {
-              float acc = __fmul_rn(__uint_as_float(v[half][4 * h]), __uint_as_float(qsh[h][0] + ksh[0]));
-#pragma unroll
-              for (int bb = 1; bb < 4; ++bb)
-                acc = __fmaf_rn(__uint_as_float(v[half][4 * h + bb]), __uint_as_float(qsh[h][bb] + ksh[bb]), acc);
-              d[h] = acc;
-            }
-          } else {
-            const int kb[4] = {k0, k1, k2, k3};
-#pragma unroll
-            for (int h = 0; h < kHi; ++h) {
-              double acc = 0.0;
-#pragma unroll
-              for (int bb = 0; bb < 4; ++bb) {
-                const int e = int(int32_t(qsh[h][bb]) >> 23) + kb[bb] - 127;  // eq + ek
-                acc = __dadd_rn(acc, __dmul_rn(double(__uint_as_float(v[half][4 * h + bb])), pow2d(e)));
-              }
-              d[h] = __double2float_rn(acc);
-            }
-          }
-          sc = __fmul_rn(wv[0], d[0]);
-#pragma unroll
-          for (int h = 1; h < kHi; ++h) sc = __fmaf_rn(wv[h], d[h], sc);
-          if (sc == 0.0f) sc = 0.0f;
+          sc = exact_score(v[half], sw, qc);
           key = rank_key(sc);
           if (!kPool && p.scores) p.scores[int64_t(cur) * p.score_stride + pos] = sc;
         }
         if (kPool) {
           const int64_t ci = int64_t(inf.y) * kTile + 128 * half + 32 * g + lane;  // candidate index
-          if (ci < int64_t(p.P) * kBlk) p.ckeys[int64_t(cur) * p.P * kBlk + ci] = key;
+          if (ci < int64_t(p.P) * kBlk) {
+            p.ckeys[int64_t(cur) * p.P * kBlk + ci] = key;
+            if (p.hist && key != 0u)
+              atomicAdd(p.hist + int64_t(cur) * kCandHistBins + (key >> (32 - kCandHistBits)), 1u);
+          }
         } else {
           key = group8_max(key);
-          if ((lane & 7) == 0 && pos < L) p.bkeys[int64_t(cur) * p.nb_stride + pos / kBlk] = key;
+          if ((lane & 7) == 0 && pos < L) {
+            p.bkeys[int64_t(cur) * p.nb_stride + pos / kBlk] = key;
+            if (p.hist && key != 0u) atomicAdd(p.hist + int64_t(cur) * kSelHistBins + (key >> (32 - kSelHistBits)), 1u);
+          }
         }
       }
     }
@@ -556,11 +513,13 @@ __global__ void __launch_bounds__(1024) k_seg_prep(SegDesc sd, int S, int32_t* s
   if (threadIdx.x == 0) tile_start[S] = carry;
 }
 
+}  // namespace
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
+static EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -596,6 +555,8 @@ int num_sms() {
   return sms;
 }
 
+namespace {
+
 template <bool kPool>
 void launch_index_tc(const CUtensorMap& map, const ScanParams& p, int64_t max_items, cudaStream_t st) {
   const size_t smem = sizeof(ScanSmem<Ring<kPool>::kStages>) + 1024;
@@ -611,7 +572,7 @@ size_t scan_tc_prefix_ints(int S) { return size_t(S) + 1; }
 csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, int32_t* seg_eff,
                            int32_t* tile_start, int S, const uint8_t* q_codes, const uint8_t* q_scales,
                            const float* w, uint32_t* bkeys, int64_t nb_stride, float* scores, int64_t score_stride,
-                           uint32_t* status, cudaStream_t st) {
+                           uint32_t* hist, uint32_t* status, cudaStream_t st) {
   if (S == 0) return CSA2_OK;
   k_seg_prep<<<1, 1024, 0, st>>>(sd, S, seg_eff, tile_start, status);
   if (sd.max_len == 0) return CSA2_OK;
@@ -632,6 +593,7 @@ csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
   p.nb_stride = nb_stride;
   p.scores = scores;
   p.score_stride = score_stride;
+  p.hist = hist;
   p.status = status;
   // the host cannot see the item count; cap the grid by an upper bound of it
   launch_index_tc<false>(map, p, int64_t(S) * ((sd.max_len + kTile - 1) / kTile), st);
@@ -640,7 +602,8 @@ csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
 
 csa2_status launch_pool_tc(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
                            int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
-                           const int32_t* pool, int P, uint32_t* ckeys, uint32_t* status, cudaStream_t st) {
+                           const int32_t* pool, int P, uint32_t* ckeys, uint32_t* hist, uint32_t* status,
+                           cudaStream_t st) {
   if (S == 0) return CSA2_OK;
   CUtensorMap map;
   const csa2_status rc = code_map(&map, kcodes, sd.cache_rows, kBlk);
@@ -659,6 +622,7 @@ csa2_status launch_pool_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
   p.P = P;
   p.items_per_seg = (P * kBlk + kTile - 1) / kTile;
   p.ckeys = ckeys;
+  p.hist = hist;
   p.status = status;
   launch_index_tc<true>(map, p, int64_t(S) * p.items_per_seg, st);
   return CSA2_OK;

@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "csa2.h"
+
 namespace csa2 {
 namespace sm100 {
 
@@ -155,6 +157,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Same wait, tied to the registers of an earlier tmem_ld16 so that no use of
+// them can be scheduled before it.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
 
 // 32 lanes x 32 bits, 8 consecutive columns per thread, same value.
 __device__ __forceinline__ void tmem_st8_same(uint32_t taddr, uint32_t v) {
@@ -184,4 +195,11 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
 }
 
 }  // namespace sm100
+
+// Host helpers of the tensor-core kernels (defined in scan_tc.cu).
+// Tensor map over an indexer-K code plane: rows of 64 bytes, boxes of
+// `box_rows` rows, 64-byte swizzle, rows past `rows` read as zero.
+csa2_status code_map(CUtensorMap* map, const uint8_t* kcodes, int64_t rows, int box_rows);
+int num_sms();
+
 }  // namespace csa2

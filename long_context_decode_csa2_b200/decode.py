@@ -56,57 +56,116 @@ def layer_plan(pattern: str, full_rescan: bool = False):
 
 
 class DecodeStep:
-    """Owns the workspaces and outputs of one decode step; ``run`` enqueues it."""
+    """Owns the workspaces and outputs of one decode step; ``run`` enqueues it.
+
+    With ``concurrent=True`` (default) the calls that do not depend on each
+    other run on side streams: every Reindex layer waits only for the pool,
+    every attention only for its layer's Top-k, so the latency-bound tail of
+    the step (pool scoring, Top-k selection, attention) overlaps across
+    layers.  Each such call then gets its own workspace.  The caller's stream
+    waits for all of them before ``run`` returns, and the scans stay on the
+    caller's stream in layer order."""
 
     def __init__(self, pattern: str, B: int, max_len: int, P: int = 2048, k: int = 512, full_rescan: bool = False,
-                 device="cuda", sm_scale: float | None = None):
+                 device="cuda", sm_scale: float | None = None, concurrent: bool = True, side_streams: int = 3):
         self.pattern, self.B, self.max_len, self.P, self.k = pattern, B, max_len, P, k
         self.plan = layer_plan(pattern, full_rescan)
         self.sm_scale = sm_scale if sm_scale is not None else 1.0 / math.sqrt(C.MAIN_DIM)
+        self.concurrent = concurrent
         dev = torch.device(device)
-        self.ws_full = C.workspace(C.csa2_index_full_workspace_bytes(B, max_len, P, k), dev)
-        self.ws_re = C.workspace(C.csa2_index_reindex_workspace_bytes(B, P, k), dev)
-        self.ws_attn = C.workspace(C.csa2_sparse_attn_decode_workspace_bytes(B, k), dev)
-        self.pool = torch.full((B, P), -1, dtype=torch.int32, device=dev)
         nL = len(pattern)
+        self.ws_full = C.workspace(C.csa2_index_full_workspace_bytes(B, max_len, P, k), dev)
+        re_bytes = C.csa2_index_reindex_workspace_bytes(B, P, k)
+        attn_bytes = C.csa2_sparse_attn_decode_workspace_bytes(B, k)
+        if concurrent:
+            self.ws_re = [C.workspace(re_bytes, dev) if act == "reindex" else None for _, _, _, act in self.plan]
+            self.ws_attn = [C.workspace(attn_bytes, dev) for _ in range(nL)]
+            self.streams = [torch.cuda.Stream(device=dev) for _ in range(max(1, side_streams))]
+            self.ev_start = torch.cuda.Event()
+            self.ev_idx = [torch.cuda.Event() for _ in range(nL)]
+            self.ev_done = [torch.cuda.Event() for _ in range(nL)]
+        else:
+            ws_re, ws_attn = C.workspace(re_bytes, dev), C.workspace(attn_bytes, dev)
+            self.ws_re = [ws_re] * nL
+            self.ws_attn = [ws_attn] * nL
+        # one pool per scanning layer (a rescan must not overwrite a pool that
+        # an earlier Reindex layer may still be reading)
+        self.pools = {layer: torch.full((B, P), -1, dtype=torch.int32, device=dev)
+                      for layer, _, _, act in self.plan if act == "scan"}
         self.topk = [torch.full((B, k), -1, dtype=torch.int32, device=dev) for _ in range(nL)]
         self.out = torch.zeros((nL, B, C.Q_HEADS, C.MAIN_DIM), dtype=torch.float32, device=dev)
         self.lse = torch.zeros((nL, B, C.Q_HEADS), dtype=torch.float32, device=dev)
         self.scores = None
-        # optional callable(call_name, "begin" | "end"), e.g. to record events
+        # optional callable(call_name, "begin" | "end", stream), e.g. to record events
         self.hook = None
 
-    def _hook(self, name, phase):
+    @property
+    def pool(self):
+        """The pool of the last scanning Full layer."""
+        return self.pools[max(self.pools)]
+
+    def _hook(self, name, phase, stream):
         if self.hook is not None:
-            self.hook(name, phase)
+            self.hook(name, phase, stream)
 
     def run(self, caches, seq_row_off, seq_len, layers, stream=None):
         """caches: [FullCache] per Full layer; layers: per layer dict of device
         tensors q, q_codes, q_scales, w, win, win_scale, win_len."""
-        last = None
+        main = stream if stream is not None else torch.cuda.current_stream()
+        if self.concurrent:
+            self.ev_start.record(main)
+        pool, pool_ev = None, None
+        last, last_ev = None, None
+        side = 0
         for layer, mode, f, act in self.plan:
             L = layers[layer]
             cache = caches[f]
             if act == "scan":
-                self._hook("csa2_index_full", "begin")
+                pool = self.pools[layer]
+                self._hook("csa2_index_full", "begin", main)
                 C.csa2_index_full(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len, self.max_len,
-                                  self.P, self.k, self.pool, self.topk[layer], self.ws_full, stream=stream)
-                self._hook("csa2_index_full", "end")
+                                  self.P, self.k, pool, self.topk[layer], self.ws_full, stream=main)
+                self._hook("csa2_index_full", "end", main)
                 last = self.topk[layer]
-            elif act == "reindex":
-                self._hook("csa2_index_reindex", "begin")
-                C.csa2_index_reindex(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len, self.pool,
-                                     self.k, self.topk[layer], self.ws_re, stream=stream)
-                self._hook("csa2_index_reindex", "end")
-                last = self.topk[layer]
+                if self.concurrent:
+                    self.ev_idx[layer].record(main)
+                    pool_ev = last_ev = self.ev_idx[layer]
+            if self.concurrent:
+                s = self.streams[side % len(self.streams)]
+                side += 1
             else:
+                s = main
+            if act == "reindex":
+                if self.concurrent:
+                    s.wait_event(pool_ev)
+                self._hook("csa2_index_reindex", "begin", s)
+                C.csa2_index_reindex(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len, pool,
+                                     self.k, self.topk[layer], self.ws_re[layer], stream=s)
+                self._hook("csa2_index_reindex", "end", s)
+                last = self.topk[layer]
+                if self.concurrent:
+                    self.ev_idx[layer].record(s)
+                    last_ev = self.ev_idx[layer]
+            elif act == "reuse":
                 self.topk[layer] = last  # Reuse: the same tensor, no copy
-            self._hook("csa2_sparse_attn_decode", "begin")
+                if self.concurrent:
+                    s.wait_event(last_ev)
+            elif self.concurrent:  # scan: the attention runs beside the next layers
+                s.wait_event(last_ev)
+            self._hook("csa2_sparse_attn_decode", "begin", s)
             C.csa2_sparse_attn_decode(L["q"], cache.main, seq_row_off, seq_len, last, L["win"], L["win_scale"],
-                                      L["win_len"], self.sm_scale, self.out[layer], self.ws_attn,
-                                      lse=self.lse[layer], stream=stream)
-            self._hook("csa2_sparse_attn_decode", "end")
+                                      L["win_len"], self.sm_scale, self.out[layer], self.ws_attn[layer],
+                                      lse=self.lse[layer], stream=s)
+            self._hook("csa2_sparse_attn_decode", "end", s)
+            if self.concurrent:
+                self.ev_done[layer].record(s)
+        if self.concurrent:
+            for ev in self.ev_done:
+                main.wait_event(ev)
         return self.out
 
     def device_flags(self) -> int:
-        return C.device_status(self.ws_full) | C.device_status(self.ws_re) | C.device_status(self.ws_attn)
+        flags = C.device_status(self.ws_full)
+        for ws in {id(w): w for w in self.ws_re + self.ws_attn if w is not None}.values():
+            flags |= C.device_status(ws)
+        return flags

@@ -21,7 +21,7 @@ def _device_layers(layers):
     return [{k: dev(L[k]) for k in keys} for L in layers]
 
 
-def _run_and_compare(wl, full_rescan=False, host_caches=True):
+def _run_and_compare(wl, full_rescan=False, host_caches=True, concurrent=True):
     layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
     fulls = wl.full_layers()
     caches_h = [W.full_cache_host(wl, f, layers[f]["q_codes"], layers[f]["q_scales"]) for f in fulls]
@@ -29,10 +29,11 @@ def _run_and_compare(wl, full_rescan=False, host_caches=True):
                           C.cache(dev(c["main_codes"]), dev(c["main_scales"]))) for c in caches_h]
     off = caches_h[0]["seq_row_off"]
     lens = wl.lengths.astype(np.int32)
-    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, full_rescan=full_rescan)
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, full_rescan=full_rescan, concurrent=concurrent)
     dl = _device_layers(layers)
     off_d, len_d = dev(off), dev(lens)
-    step.run(caches_d, off_d, len_d, dl)
+    for _ in range(2):  # the second step reuses the workspaces (counters and histograms back at zero)
+        step.run(caches_d, off_d, len_d, dl)
     torch.cuda.synchronize()
     assert step.device_flags() == 0
     ref = oracle.decode_step(wl.pattern, caches_h, off, lens, layers, wl.P, wl.k, 1 / math.sqrt(512),
@@ -50,9 +51,10 @@ def test_decode_tiny_config():
     _run_and_compare(W.decode_workloads()["tiny_decode_b1_l8192"])
 
 
-def test_decode_stack_reduced():
+@pytest.mark.parametrize("concurrent", [True, False])
+def test_decode_stack_reduced(concurrent):
     wl = W.DecodeWorkload("stack_small", np.array([131072, 50001, 9000, 333, 8]), "FRRU", needles=64)
-    _run_and_compare(wl)
+    _run_and_compare(wl, concurrent=concurrent)
 
 
 @pytest.mark.parametrize("rescan", [False, True])

@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling captures)")
+    ap.add_argument("--sequential", action="store_true",
+                    help="issue every call on one stream (isolated per-call times) instead of the concurrent tail")
     ap.add_argument("--context", type=int, default=0,
                     help="override every sequence's length (small profiling captures of the attention)")
     return ap.parse_args()
@@ -251,7 +253,7 @@ def run_ours(args):
                               min(wl.needles, max(1, args.context // 1024)), wl.lognormal, wl.seed)
     wl, layers, caches_dev, caches, layers_dev, off_d, len_d = build_workload(wl, rank, device)
     C.lib()
-    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, concurrent=not args.sequential)
     stream = torch.cuda.current_stream()
 
     # events around every C-ABI call of the timed region, on the stream the
@@ -375,7 +377,8 @@ def run_ours(args):
             "data": "synthetic",
             "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len, "layers": wl.pattern,
                        "pool_blocks": wl.P, "topk": wl.k, "window": 128,
-                       "l2": "no flush: inputs larger than L2 (%.2f GB read per step)" % (ab["total"] / 1e9)},
+                       "l2": "no flush: inputs larger than L2 (%.2f GB read per step)" % (ab["total"] / 1e9),
+                       "schedule": "sequential" if args.sequential else "concurrent tail (side streams)"},
             "tokens_per_s": job_throughput(world, wl.B, ms),
             "hbm_algorithmic_gbs": ab["total"] / (ms * 1e-3) / 1e9,
             "hbm_frac_of_8tbs": ab["total"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,

@@ -4,18 +4,25 @@
 // MXFP4 main KV, FP8 window; section "后 20 层干脆共用一份 KV": 128-token window).
 //
 // Work split: ceil(k/128) chunks of selected rows plus one window chunk per
-// segment.  A CTA gathers its <= 128 key rows, dequantises them exactly into
-// fp16 in shared memory (E2M1 x 2^X and raw E4M3 are exact in fp16 inside the
-// range checked below), and runs both products on the tensor cores with
-// warp-level mma (fp16 inputs, fp32 accumulation):
+// segment, walked by a persistent grid (one CTA per SM, consecutive chunks
+// per CTA).  While a CTA computes one chunk, cp.async brings the next
+// chunk's raw rows (272-byte MXFP4 rows or 512-byte E4M3 rows) into a staging
+// buffer; the chunk's Top-k ids are loaded one chunk earlier still.  Each
+// chunk's rows are dequantised exactly into fp16 in shared memory (E2M1 x 2^X
+// and raw E4M3 are exact in fp16 inside the range checked below), and both
+// products run on the tensor cores with warp-level mma (fp16 inputs, fp32
+// accumulation):
 //   S = Q K^T  (16 heads x 128 keys),  P = exp(S*scale - max),  O = P V.
 // The window's fp32 scale multiplies its logits and its partial output in
-// fp32, never the fp16 values.  Each CTA writes an unnormalised partial
-// (O, max, sum) per head; the last CTA of each segment to finish combines the
-// chunks in a fixed order (deterministic) and resets the segment's counter.
+// fp32, never the fp16 values.  Each chunk leaves an unnormalised partial
+// (O, max, sum) per head; the last CTA to finish a segment's chunks combines
+// them in a fixed order (deterministic) and resets the segment's counter.
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "device_common.cuh"
+#include "sm100.cuh"
 
 namespace csa2 {
 
@@ -30,16 +37,101 @@ size_t attn_partial_bytes(int S, int k) {
   return size_t(S) * attn_num_chunks(k) * kPartFloats * sizeof(float);
 }
 
+constexpr int kRawMain = kMainCodeBytes + kMainScaleBytes + 0;  // 272: codes then scales (row stride
+                                                                 // 68 words: conflict-free 16-byte reads)
+constexpr int kRawWin = kD + 16;                                 // 528: one E4M3 row + pad
+
 struct AttnSmem {
   __half q[kHq][kQS];
   __half kv[kChunk][kQS];
   __half p[kHq][kPS];
+  union {
+    uint8_t main[kChunk][kRawMain];
+    uint8_t win[kChunk][kRawWin];
+  } raw;                                 // staged raw rows of the next chunk
   float red_max[8][kHq];
   float red_sum[8][kHq];
   int valid[kChunk];
   float fac[CSA2_MAX_TOPK / kChunk + 1][kHq];
   int last;
 };
+
+// Rows of chunk c of segment s: how many, where from, and the window scale.
+struct ChunkSrc {
+  int nkeys;
+  bool is_win;
+  float kscale;
+  const uint8_t* win_base;  // window rows (contiguous), or null
+};
+
+__device__ __forceinline__ ChunkSrc chunk_src(const AttnArgs& a, int s, int c) {
+  ChunkSrc r;
+  const int nmain = (a.k + kChunk - 1) / kChunk;
+  r.is_win = (c == nmain);
+  r.kscale = 1.0f;
+  r.win_base = nullptr;
+  if (!r.is_win) {
+    r.nkeys = min(kChunk, a.k - c * kChunk);
+  } else if (a.q_pos == nullptr) {
+    r.nkeys = max(0, min(kWin, a.win_len[s]));
+    r.kscale = a.win_scale[s];
+    r.win_base = a.win + int64_t(s) * kWin * kD;
+  } else {
+    int64_t p = a.q_pos[s];
+    if (p >= a.n_raw) {
+      set_status(a.status, CSA2_DEV_LENGTH);
+      p = a.n_raw - 1;
+    }
+    const int64_t lo = p - (kWin - 1) > 0 ? p - (kWin - 1) : 0;
+    r.nkeys = p >= 0 ? int(p - lo + 1) : 0;
+    r.kscale = a.raw_scale;
+    r.win_base = a.raw_win + lo * kD;
+  }
+  return r;
+}
+
+// Top-k id of this thread's row of chunk c (or -1 when the row is not a
+// selected main row).  Issued one chunk ahead of its use.
+__device__ __forceinline__ int32_t chunk_tpos(const AttnArgs& a, int s, int c, int r) {
+  const int nmain = (a.k + kChunk - 1) / kChunk;
+  if (c >= nmain) return -1;
+  const int idx = c * kChunk + r;
+  return idx < a.k ? __ldg(a.topk + int64_t(s) * a.k + idx) : -1;
+}
+
+// Issues the cp.async copies of chunk c's rows into sm.raw (this thread: row
+// r = tid % 128, half tid / 128 of it) and returns whether row r is present.
+__device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, int s, int c, int32_t tpos) {
+  const int tid = threadIdx.x, r = tid & (kChunk - 1), half = tid / kChunk;
+  const ChunkSrc src = chunk_src(a, s, c);
+  bool ok = r < src.nkeys;
+  if (!src.is_win && ok) {
+    const int64_t eff = a.seg_eff[s];
+    if (tpos >= eff) {
+      if (half == 0) set_status(a.status, CSA2_DEV_INDEX_RANGE);
+      ok = false;
+    } else if (tpos < 0) {
+      ok = false;
+    }
+  }
+  if (ok) {
+    if (!src.is_win) {
+      const int64_t off = a.sd.row_off ? a.sd.row_off[s] : a.sd.row0;
+      const int64_t row = off + tpos;
+      const uint8_t* cs = a.mcodes + row * kMainCodeBytes + half * (kMainCodeBytes / 2);
+      uint8_t* dst = sm.raw.main[r] + half * (kMainCodeBytes / 2);
+#pragma unroll
+      for (int i = 0; i < kMainCodeBytes / 2 / 16; ++i) sm100::cp_async16(dst + 16 * i, cs + 16 * i);
+      if (half == 0) sm100::cp_async16(sm.raw.main[r] + kMainCodeBytes, a.mscales + row * kMainScaleBytes);
+    } else {
+      const uint8_t* ws = src.win_base + int64_t(r) * kD + half * (kD / 2);
+      uint8_t* dst = sm.raw.win[r] + half * (kD / 2);
+#pragma unroll
+      for (int i = 0; i < kD / 2 / 16; ++i) sm100::cp_async16(dst + 16 * i, ws + 16 * i);
+    }
+  }
+  return ok;
+}
 
 // Two E2M1 codes (low nibble = lower element) -> f16x2, exact.
 __device__ __forceinline__ uint32_t cvt_e2m1x2(uint32_t byte) {
@@ -79,119 +171,82 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void attn_chunk(const AttnArgs& a, AttnSmem& sm, float* part, int s, int c, int nkeys,
-                                           bool is_win, float kscale, const uint8_t* win_base, int64_t eff,
-                                           int64_t off) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  // Q: bf16 -> fp16 (exact for |q| in [2^-14, 65504]; smaller values keep
-  // 2^-24 resolution); 8 values per 16-byte load, both loads in flight
-  {
-    constexpr int kQV = kHq * kD / 8 / kAttnThreads;  // 16-byte vectors per thread (4)
-    uint4 qv[kQV];
-    const uint4* qsrc = reinterpret_cast<const uint4*>(a.q + int64_t(s) * kHq * kD);
+// Q of segment s: bf16 -> fp16 into sm.q (exact for |q| in [2^-14, 65504];
+// smaller values keep 2^-24 resolution).
+__device__ __forceinline__ void load_q(const AttnArgs& a, AttnSmem& sm, int s) {
+  const int tid = threadIdx.x;
+  constexpr int kQV = kHq * kD / 8 / kAttnThreads;  // 16-byte vectors per thread (4)
+  uint4 qv[kQV];
+  const uint4* qsrc = reinterpret_cast<const uint4*>(a.q + int64_t(s) * kHq * kD);
 #pragma unroll
-    for (int m = 0; m < kQV; ++m) qv[m] = __ldg(qsrc + tid + m * kAttnThreads);
+  for (int m = 0; m < kQV; ++m) qv[m] = __ldg(qsrc + tid + m * kAttnThreads);
 #pragma unroll
-    for (int m = 0; m < kQV; ++m) {
-      const int e = 8 * (tid + m * kAttnThreads);
-      const int h = e / kD, d = e % kD;
-      const uint32_t w[4] = {qv[m].x, qv[m].y, qv[m].z, qv[m].w};
-      uint32_t o[4];
+  for (int m = 0; m < kQV; ++m) {
+    const int e = 8 * (tid + m * kAttnThreads);
+    const int h = e / kD, d = e % kD;
+    const uint32_t w[4] = {qv[m].x, qv[m].y, qv[m].z, qv[m].w};
+    uint32_t o[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
-        if (fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f) set_status(a.status, CSA2_DEV_FP16_RANGE);
-        const __half2 h2 = __floats2half2_rn(lo, hi);
-        o[q] = *reinterpret_cast<const uint32_t*>(&h2);
-      }
-      *reinterpret_cast<uint4*>(&sm.q[h][d]) = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int q = 0; q < 4; ++q) {
+      const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
+      if (fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f) set_status(a.status, CSA2_DEV_FP16_RANGE);
+      const __half2 h2 = __floats2half2_rn(lo, hi);
+      o[q] = *reinterpret_cast<const uint32_t*>(&h2);
     }
+    *reinterpret_cast<uint4*>(&sm.q[h][d]) = make_uint4(o[0], o[1], o[2], o[3]);
   }
-  // keys: thread -> one row r (lanes on consecutive rows, which keeps the
-  // shared-memory stores conflict-free) and blocks b = tid/128 + 2i; all of
-  // a thread's loads are issued before any conversion
+}
+
+// Staged raw rows -> fp16 keys in sm.kv (absent rows as zeros) and the
+// row-valid flags.  Thread: row r = tid % 128, blocks tid/128 + 2i.
+__device__ __forceinline__ void dequant_chunk(const AttnArgs& a, AttnSmem& sm, bool is_win, bool row_ok) {
+  const int tid = threadIdx.x;
   const int r = tid & (kChunk - 1);
   constexpr int kBPT = 16 / (kAttnThreads / kChunk);  // blocks per thread (8)
-  int64_t tpos = -1;
-  if (!is_win && r < nkeys) {
-    tpos = a.topk[int64_t(s) * a.k + c * kChunk + r];
-    if (tpos >= eff) {
-      set_status(a.status, CSA2_DEV_INDEX_RANGE);
-      tpos = -1;
-    }
-  }
-  const bool row_ok = (r < nkeys) && (is_win || tpos >= 0);
-  if (tid < kChunk) sm.valid[r] = row_ok;
   const int b0 = tid / kChunk;
-  if (!is_win) {
-    uint4 cw[kBPT];
-    uint32_t sbv[kBPT];
-    if (row_ok) {
-      const int64_t row = off + tpos;
-      const uint4* cp = reinterpret_cast<const uint4*>(a.mcodes + row * kMainCodeBytes);
-      const uint8_t* sp = a.mscales + row * kMainScaleBytes;
+  if (b0 == 0) sm.valid[r] = row_ok;
 #pragma unroll
-      for (int i = 0; i < kBPT; ++i) {
-        cw[i] = __ldg(cp + b0 + 2 * i);
-        sbv[i] = __ldg(sp + b0 + 2 * i);
-      }
+  for (int i = 0; i < kBPT; ++i) {
+    const int b = b0 + 2 * i;
+    uint4* dst = reinterpret_cast<uint4*>(&sm.kv[r][32 * b]);
+    if (!row_ok) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
+      continue;
     }
-#pragma unroll
-    for (int i = 0; i < kBPT; ++i) {
-      const int b = b0 + 2 * i;
-      uint4* dst = reinterpret_cast<uint4*>(&sm.kv[r][32 * b]);
-      if (!row_ok) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
-        continue;
-      }
+    if (!is_win) {
       // fp16-exact iff the block exponent X = byte - 127 lies in [-23, 13]
-      const uint32_t sb = sbv[i];
+      const uint4 cw = *reinterpret_cast<const uint4*>(sm.raw.main[r] + 16 * b);
+      const uint32_t sb = sm.raw.main[r][kMainCodeBytes + b];
       if (sb < 104u || sb > 140u) set_status(a.status, CSA2_DEV_FP16_RANGE);
       const int X = int(sb) - 127;
       const uint16_t xb = X >= -14 ? uint16_t((X + 15) << 10) : uint16_t(1u << (X + 24 > 0 ? X + 24 : 0));
       const uint32_t sc2 = uint32_t(xb) | (uint32_t(xb) << 16);
-      const uint32_t w4[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
+      const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t hv[4];
 #pragma unroll
-        for (int n = 0; n < 4; ++n) {
-          hv[n] = hmul2_u32(cvt_e2m1x2((w4[q] >> (8 * n)) & 255u), sc2);
-        }
+        for (int n = 0; n < 4; ++n) hv[n] = hmul2_u32(cvt_e2m1x2((w4[q] >> (8 * n)) & 255u), sc2);
         dst[q] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
       }
-    }
-  } else {
-    uint4 wv[kBPT][2];
-    if (row_ok) {
-      const uint4* src = reinterpret_cast<const uint4*>(win_base + int64_t(r) * kD);
-#pragma unroll
-      for (int i = 0; i < kBPT; ++i) {
-        wv[i][0] = __ldg(src + 2 * (b0 + 2 * i));
-        wv[i][1] = __ldg(src + 2 * (b0 + 2 * i) + 1);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kBPT; ++i) {
-      const int b = b0 + 2 * i;
-      uint4* dst = reinterpret_cast<uint4*>(&sm.kv[r][32 * b]);
-      if (!row_ok) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
-        continue;
-      }
-      const uint32_t w8[8] = {wv[i][0].x, wv[i][0].y, wv[i][0].z, wv[i][0].w,
-                              wv[i][1].x, wv[i][1].y, wv[i][1].z, wv[i][1].w};
+    } else {
+      const uint4 v0 = *reinterpret_cast<const uint4*>(sm.raw.win[r] + 32 * b);
+      const uint4 v1 = *reinterpret_cast<const uint4*>(sm.raw.win[r] + 32 * b + 16);
+      const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         dst[q] = make_uint4(cvt_e4m3x2(w8[2 * q] & 0xFFFFu), cvt_e4m3x2(w8[2 * q] >> 16),
                             cvt_e4m3x2(w8[2 * q + 1] & 0xFFFFu), cvt_e4m3x2(w8[2 * q + 1] >> 16));
     }
   }
-  __syncthreads();
+}
 
+// S = Q K^T, softmax, O = P V over the chunk in sm.kv; writes the partial.
+__device__ __forceinline__ void attn_compute(const AttnArgs& a, AttnSmem& sm, float* part, int nkeys,
+                                             float kscale) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
   // ---- S = Q K^T: warp w owns keys 16w .. 16w+15 (two n-tiles of 8) ----
   float sacc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
   {
@@ -306,9 +361,8 @@ __device__ __forceinline__ void attn_chunk(const AttnArgs& a, AttnSmem& sm, floa
 
 // Last-arriving CTA of a segment: combine the chunk partials in chunk order
 // (deterministic), write out / lse, and reset the segment's arrival counter.
-__device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm, int s) {
+__device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm, int s, int nchunks) {
   const int tid = threadIdx.x;
-  const int nchunks = gridDim.x;
   __threadfence();  // this thread's partial is visible before the arrival below
   __syncthreads();
   if (tid == 0) sm.last = (atomicAdd(a.counters + s, 1) == nchunks - 1);
@@ -353,48 +407,48 @@ __device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm,
   if (tid == 0) a.counters[s] = 0;
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnArgs a) {
+__global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnArgs a, int nchunks) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
-  const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  const int nmain = (a.k + kChunk - 1) / kChunk;
-  const bool is_win = (c == nmain);
-  const int64_t eff = a.seg_eff[s];
-  const int64_t off = a.sd.row_off ? a.sd.row_off[s] : a.sd.row0;
-  float* part = a.partial + (int64_t(s) * gridDim.x + c) * kPartFloats;
-
-  int nkeys;
-  float kscale = 1.0f;
-  const uint8_t* win_base = nullptr;
-  if (!is_win) {
-    nkeys = min(kChunk, a.k - c * kChunk);
-  } else if (a.q_pos == nullptr) {
-    nkeys = max(0, min(kWin, a.win_len[s]));
-    kscale = a.win_scale[s];
-    win_base = a.win + int64_t(s) * kWin * kD;
-  } else {
-    int64_t p = a.q_pos[s];
-    if (p >= a.n_raw) {
-      set_status(a.status, CSA2_DEV_LENGTH);
-      p = a.n_raw - 1;
+  const int tid = threadIdx.x, r = tid & (kChunk - 1);
+  const int n_items = a.S * nchunks;
+  const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
+  const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
+  if (i0 >= i1) return;
+  // prologue: the first chunk's rows in flight, the second chunk's ids loaded
+  bool ok = issue_gather(a, sm, i0 / nchunks, i0 % nchunks, chunk_tpos(a, i0 / nchunks, i0 % nchunks, r));
+  sm100::cp_async_commit();
+  int32_t tnext = (i0 + 1 < i1) ? chunk_tpos(a, (i0 + 1) / nchunks, (i0 + 1) % nchunks, r) : -1;
+  int qseg = -1;
+  for (int it = i0; it < i1; ++it) {
+    const int s = it / nchunks, c = it - s * nchunks;
+    const ChunkSrc src = chunk_src(a, s, c);
+    if (s != qseg) {  // the previous chunk's products are done (barrier at its end)
+      load_q(a, sm, s);
+      qseg = s;
     }
-    const int64_t lo = p - (kWin - 1) > 0 ? p - (kWin - 1) : 0;
-    nkeys = p >= 0 ? int(p - lo + 1) : 0;
-    kscale = a.raw_scale;
-    win_base = a.raw_win + lo * kD;
-  }
-  if (nkeys == 0) {
-    for (int i = tid; i < kHq * kD; i += kAttnThreads) part[i] = 0.0f;
-    if (tid < kHq) {
-      part[kHq * kD + tid] = -INFINITY;
-      part[kHq * kD + kHq + tid] = 0.0f;
+    sm100::cp_async_wait<0>();
+    __syncthreads();  // this chunk's rows (and Q) are in shared memory
+    dequant_chunk(a, sm, src.is_win, ok);
+    __syncthreads();  // keys ready; the staging buffer is free
+    if (it + 1 < i1) {
+      ok = issue_gather(a, sm, (it + 1) / nchunks, (it + 1) % nchunks, tnext);
+      sm100::cp_async_commit();
+      tnext = (it + 2 < i1) ? chunk_tpos(a, (it + 2) / nchunks, (it + 2) % nchunks, r) : -1;
     }
-  } else {
-    attn_chunk(a, sm, part, s, c, nkeys, is_win, kscale, win_base, eff, off);
+    float* part = a.partial + (int64_t(s) * nchunks + c) * kPartFloats;
+    if (src.nkeys == 0) {
+      for (int i = tid; i < kHq * kD; i += kAttnThreads) part[i] = 0.0f;
+      if (tid < kHq) {
+        part[kHq * kD + tid] = -INFINITY;
+        part[kHq * kD + kHq + tid] = 0.0f;
+      }
+    } else {
+      attn_compute(a, sm, part, src.nkeys, src.kscale);
+    }
+    combine_if_last(a, sm, s, nchunks);
   }
-  combine_if_last(a, sm, s);
+  sm100::cp_async_wait<0>();
 }
 
 void launch_attention(const AttnArgs& a, cudaStream_t st) {
@@ -402,7 +456,9 @@ void launch_attention(const AttnArgs& a, cudaStream_t st) {
   const int nchunks = attn_num_chunks(a.k);
   const size_t smem = sizeof(AttnSmem);
   cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  k_attn_partial<<<dim3(nchunks, a.S), kAttnThreads, smem, st>>>(a);
+  const int64_t n_items = int64_t(a.S) * nchunks;
+  const int grid = int(std::min<int64_t>(num_sms(), n_items));
+  k_attn_partial<<<grid, kAttnThreads, smem, st>>>(a, nchunks);
 }
 
 }  // namespace csa2

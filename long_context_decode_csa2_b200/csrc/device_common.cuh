@@ -64,29 +64,44 @@ __device__ __forceinline__ void make_qctx(IdxQCtx& c, const uint8_t* q_scales /*
 // When the block exponents lie within 9 of each other (and away from the
 // fp32 range limits) every term and partial sum is exact in fp32, so the sum
 // is done there; otherwise in fp64 as the definition states.
-__device__ __forceinline__ float exact_score(const uint32_t (&v)[16], uint32_t sw, const IdxQCtx& q) {
-  const int k0 = int(sw & 255u), k1 = int((sw >> 8) & 255u), k2 = int((sw >> 16) & 255u), k3 = int(sw >> 24);
-  const int kmin = min(min(k0, k1), min(k2, k3)), kmax = max(max(k0, k1), max(k2, k3));
-  const bool fast = (kmax - kmin + q.qspread <= 9) && (q.qlo + kmin - 254 >= -100) && (q.qhi + kmax - 254 <= 100);
-  const uint32_t ksh[4] = {uint32_t(k0) << 23, uint32_t(k1) << 23, uint32_t(k2) << 23, uint32_t(k3) << 23};
+// Key side of the score: the four block exponents of one indexer-K row.
+struct KeyScale {
+  int kb[4];
+  int kmin, kmax;
+};
+
+__device__ __forceinline__ KeyScale key_scale(uint32_t sw) {
+  KeyScale k;
+  k.kb[0] = int(sw & 255u);
+  k.kb[1] = int((sw >> 8) & 255u);
+  k.kb[2] = int((sw >> 16) & 255u);
+  k.kb[3] = int(sw >> 24);
+  k.kmin = min(min(k.kb[0], k.kb[1]), min(k.kb[2], k.kb[3]));
+  k.kmax = max(max(k.kb[0], k.kb[1]), max(k.kb[2], k.kb[3]));
+  return k;
+}
+
+__device__ __forceinline__ float exact_score(const uint32_t (&v)[16], const KeyScale& ks, const IdxQCtx& q) {
+  const bool fast = (ks.kmax - ks.kmin + q.qspread <= 9) && (q.qlo + ks.kmin - 254 >= -100) &&
+                    (q.qhi + ks.kmax - 254 <= 100);
   float d[kHi];
   if (fast) {
 #pragma unroll
     for (int h = 0; h < kHi; ++h) {
-      float acc = __fmul_rn(__uint_as_float(v[4 * h]), __uint_as_float(q.qsh[h][0] + ksh[0]));
+      float acc = __fmul_rn(__uint_as_float(v[4 * h]), __uint_as_float(q.qsh[h][0] + (uint32_t(ks.kb[0]) << 23)));
 #pragma unroll
       for (int bb = 1; bb < 4; ++bb)
-        acc = __fmaf_rn(__uint_as_float(v[4 * h + bb]), __uint_as_float(q.qsh[h][bb] + ksh[bb]), acc);
+        acc = __fmaf_rn(__uint_as_float(v[4 * h + bb]), __uint_as_float(q.qsh[h][bb] + (uint32_t(ks.kb[bb]) << 23)),
+                        acc);
       d[h] = acc;
     }
   } else {
-    const int kb[4] = {k0, k1, k2, k3};
 #pragma unroll
     for (int h = 0; h < kHi; ++h) {
       double acc = 0.0;
 #pragma unroll
       for (int bb = 0; bb < 4; ++bb) {
-        const int e = int(int32_t(q.qsh[h][bb]) >> 23) + kb[bb] - 127;  // eq + ek
+        const int e = int(int32_t(q.qsh[h][bb]) >> 23) + ks.kb[bb] - 127;  // eq + ek
         acc = __dadd_rn(acc, __dmul_rn(double(__uint_as_float(v[4 * h + bb])), pow2d(e)));
       }
       d[h] = __double2float_rn(acc);
@@ -97,6 +112,10 @@ __device__ __forceinline__ float exact_score(const uint32_t (&v)[16], uint32_t s
   for (int h = 1; h < kHi; ++h) sc = __fmaf_rn(q.w[h], d[h], sc);
   if (sc == 0.0f) sc = 0.0f;
   return sc;
+}
+
+__device__ __forceinline__ float exact_score(const uint32_t (&v)[16], uint32_t sw, const IdxQCtx& q) {
+  return exact_score(v, key_scale(sw), q);
 }
 
 // Max over aligned groups of 8 lanes; every lane of the group gets it.

@@ -47,10 +47,21 @@ constexpr int kThr = 64 + 128 * kTeams;  // producer, MMA, epilogue warps
 constexpr uint32_t kTileBytes = kPT * kIdxCodeBytes;
 static_assert(kAc * kN <= int(kSf), "TMEM accumulators overlap the scale factors");
 
-struct QCtxS {
+struct __align__(16) QCtxS {
   IdxQCtx c;
   int vis;  // visible entries of this query (0 past the end of the batch)
 };
+static_assert(sizeof(QCtxS) == 96, "QCtxS is read as six 16-byte words");
+
+// One query's context from shared memory in six 16-byte loads.
+__device__ __forceinline__ QCtxS load_qctx(const QCtxS& src) {
+  QCtxS q;
+  const uint4* s4 = reinterpret_cast<const uint4*>(&src);
+  uint4* d4 = reinterpret_cast<uint4*>(&q);
+#pragma unroll
+  for (int i = 0; i < 6; ++i) d4[i] = s4[i];
+  return q;
+}
 
 struct __align__(1024) PfSmem {
   uint8_t a[kSt][kTileBytes];           // code rows, 64-byte swizzled
@@ -282,7 +293,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       sm100::tc_fence_after();
       const int pl = 32 * q4 + lane;
       const int64_t pos = int64_t(tile) * kPT + pl;
-      const uint32_t sw = sm.sc[s][pl];
+      const KeyScale ks = key_scale(sm.sc[s][pl]);
       const uint32_t tcol = tmem + lane_base + uint32_t(a * kN);
       uint32_t va[16], vb[16];
       sm100::tmem_ld16(tcol, va);
@@ -292,9 +303,9 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
         uint32_t(&cur)[16] = (j & 1) ? vb : va;
         uint32_t(&nxt)[16] = (j & 1) ? va : vb;
         if (j + 1 < kQG) sm100::tmem_ld16(tcol + 16 * (j + 1), nxt);
-        const QCtxS& q = sm.qctx[s][j];
+        const QCtxS q = load_qctx(sm.qctx[s][j]);
         uint32_t key = 0;
-        if (pos < q.vis) key = rank_key(exact_score(cur, sw, q.c));
+        if (pos < q.vis) key = rank_key(exact_score(cur, ks, q.c));
         key = group8_max(key);
         if ((lane & 7) == 0 && pos < q.vis)
           p.bkeys[int64_t(g * kQG + j) * p.nb_stride + pos / kBlk] = key;

@@ -363,43 +363,65 @@ __device__ __forceinline__ void attn_compute(const AttnArgs& a, AttnSmem& sm, fl
 // (deterministic), write out / lse, and reset the segment's arrival counter.
 __device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm, int s, int nchunks) {
   const int tid = threadIdx.x;
-  __threadfence();  // this thread's partial is visible before the arrival below
+  // The barrier orders every thread's partial stores before thread 0's
+  // release-acquire arrival (gpu scope); the last arrival therefore sees all
+  // chunks' partials.
   __syncthreads();
-  if (tid == 0) sm.last = (atomicAdd(a.counters + s, 1) == nchunks - 1);
+  if (tid == 0) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(a.counters + s) : "memory");
+    sm.last = (old == nchunks - 1);
+  }
   __syncthreads();
   if (!sm.last) return;
-  __threadfence();
   const float* base = a.partial + int64_t(s) * nchunks * kPartFloats;
   if (tid < kHq) {
+    constexpr int kMaxC = CSA2_MAX_TOPK / kChunk + 1;
+    float mc[kMaxC], lc[kMaxC];
     float M = -INFINITY;
-    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, __ldcg(base + c * kPartFloats + kHq * kD + tid));
+#pragma unroll
+    for (int c = 0; c < kMaxC; ++c) {  // all loads first
+      mc[c] = c < nchunks ? __ldcg(base + c * kPartFloats + kHq * kD + tid) : -INFINITY;
+      lc[c] = c < nchunks ? __ldcg(base + c * kPartFloats + kHq * kD + kHq + tid) : 0.0f;
+    }
+#pragma unroll
+    for (int c = 0; c < kMaxC; ++c) M = fmaxf(M, mc[c]);
     float L = 0.0f;
-    for (int c = 0; c < nchunks; ++c) {
-      const float mc = __ldcg(base + c * kPartFloats + kHq * kD + tid);
-      const float f = (mc == -INFINITY) ? 0.0f : __expf(mc - M);
-      sm.fac[c][tid] = f;
-      L += __ldcg(base + c * kPartFloats + kHq * kD + kHq + tid) * f;
+#pragma unroll
+    for (int c = 0; c < kMaxC; ++c) {
+      const float f = (mc[c] == -INFINITY) ? 0.0f : __expf(mc[c] - M);
+      if (c < nchunks) sm.fac[c][tid] = f;
+      L += lc[c] * f;
     }
     for (int c = 0; c < nchunks; ++c) sm.fac[c][tid] = (M == -INFINITY) ? 0.0f : sm.fac[c][tid] / L;
     if (a.lse) a.lse[int64_t(s) * kHq + tid] = (M == -INFINITY) ? -INFINITY : M + logf(L);
   }
   __syncthreads();
-  // 8 float4 per thread; per chunk all 8 loads are independent
+  // 8 float4 per thread; two chunks' loads in flight at a time
   constexpr int kOV = kHq * kD / 4 / kAttnThreads;
   float4 o[kOV];
 #pragma unroll
   for (int m = 0; m < kOV; ++m) o[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c = 0; c < nchunks; ++c) {
-    float4 v[kOV];
+  for (int c0 = 0; c0 < nchunks; c0 += 2) {
+    float4 v[2][kOV];
 #pragma unroll
-    for (int m = 0; m < kOV; ++m) v[m] = __ldcg(reinterpret_cast<const float4*>(base + c * kPartFloats) + tid + m * kAttnThreads);
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-    for (int m = 0; m < kOV; ++m) {
-      const float f = sm.fac[c][(4 * (tid + m * kAttnThreads)) / kD];
-      o[m].x = fmaf(v[m].x, f, o[m].x);
-      o[m].y = fmaf(v[m].y, f, o[m].y);
-      o[m].z = fmaf(v[m].z, f, o[m].z);
-      o[m].w = fmaf(v[m].w, f, o[m].w);
+      for (int m = 0; m < kOV; ++m)
+        v[u][m] = (c0 + u < nchunks)
+                      ? __ldcg(reinterpret_cast<const float4*>(base + (c0 + u) * kPartFloats) + tid + m * kAttnThreads)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (c0 + u >= nchunks) break;
+#pragma unroll
+      for (int m = 0; m < kOV; ++m) {
+        const float f = sm.fac[c0 + u][(4 * (tid + m * kAttnThreads)) / kD];
+        o[m].x = fmaf(v[u][m].x, f, o[m].x);
+        o[m].y = fmaf(v[u][m].y, f, o[m].y);
+        o[m].z = fmaf(v[u][m].z, f, o[m].z);
+        o[m].w = fmaf(v[u][m].w, f, o[m].w);
+      }
     }
   }
 #pragma unroll
@@ -456,8 +478,12 @@ void launch_attention(const AttnArgs& a, cudaStream_t st) {
   const int nchunks = attn_num_chunks(a.k);
   const size_t smem = sizeof(AttnSmem);
   cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  // one chunk per CTA while there are few chunks (the first gather of a
+  // persistent CTA would not be hidden); a persistent grid with prefetching
+  // beyond four chunks per SM
   const int64_t n_items = int64_t(a.S) * nchunks;
-  const int grid = int(std::min<int64_t>(num_sms(), n_items));
+  const int sms = num_sms();
+  const int grid = int(n_items <= 4 * int64_t(sms) ? n_items : int64_t(sms));
   k_attn_partial<<<grid, kAttnThreads, smem, st>>>(a, nchunks);
 }
 

@@ -20,10 +20,10 @@
 //   * warp 1 issues two tcgen05.mma kind::mxf4 (M = 128 positions, N = 128,
 //     K = 64) with every block scale = 1, so each accumulator is an exact
 //     block dot D/4;
-//   * two teams of four epilogue warps read each position's 16 accumulators
-//     per query, form the exact score (the same rounding as the decode scan),
-//     mask positions the query cannot see, and write the maximum of every 8
-//     positions as one rank key.
+//   * four teams of four epilogue warps (two of the eight queries each) read
+//     each position's 16 accumulators per query, form the exact score (the
+//     same rounding as the decode scan), mask positions the query cannot see,
+//     and write the maximum of every 8 positions as one rank key.
 // Items past the visibility of every query of a group are skipped by all
 // roles alike.  Every wait is time-bounded (CSA2_DEV_TIMEOUT on expiry).
 #include <algorithm>
@@ -42,8 +42,10 @@ constexpr int kSt = 6;                   // smem ring
 constexpr int kAc = 3;                   // TMEM accumulator ring, kN columns each
 constexpr int kTmemCols = 512;
 constexpr uint32_t kSf = 448;            // scale-factor columns (all 2^0)
-constexpr int kTeams = 2;                // epilogue teams of 4 warps
-constexpr int kThr = 64 + 128 * kTeams;  // producer, MMA, epilogue warps
+constexpr int kTeams = 4;                // epilogue teams of 4 warps, all on every item
+constexpr int kQPT = kQG / kTeams;       // queries per team and item
+constexpr int kEpiWarps = 4 * kTeams;
+constexpr int kThr = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
 constexpr uint32_t kTileBytes = kPT * kIdxCodeBytes;
 static_assert(kAc * kN <= int(kSf), "TMEM accumulators overlap the scale factors");
 
@@ -160,11 +162,11 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSt; ++s) {
       sm100::mbar_init(&sm.full[s], 1);
-      sm100::mbar_init(&sm.empty[s], 1 + 4);
+      sm100::mbar_init(&sm.empty[s], 1 + kEpiWarps);
     }
     for (int a = 0; a < kAc; ++a) {
       sm100::mbar_init(&sm.tfull[a], 1);
-      sm100::mbar_init(&sm.tempty[a], 4);
+      sm100::mbar_init(&sm.tempty[a], kEpiWarps);
     }
     sm100::mbar_init(&sm.done, 1);
     sm.abort_flag = 0;
@@ -272,6 +274,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
     // ------------------------------------------------------------ epilogue
     const int q4 = warp & 3;  // TMEM lane quarter of this warp
     const int team = (warp - 2) >> 2;
+    const int j0 = team * kQPT;  // this team's queries of the group
     const uint32_t lane_base = uint32_t(32 * q4) << 16;
     int t = -1, cg = -1, gmax = 0;
     for (int it = i0; it < i1; ++it) {
@@ -282,7 +285,6 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       }
       if (int64_t(tile) * kPT >= gmax) continue;
       ++t;
-      if (t % kTeams != team) continue;
       const int s = t % kSt, a = t % kAc;
       const bool ok = sm100::mbar_wait(&sm.full[s], (t / kSt) & 1) && sm100::mbar_wait(&sm.tfull[a], (t / kAc) & 1);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -295,21 +297,20 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       const int64_t pos = int64_t(tile) * kPT + pl;
       const KeyScale ks = key_scale(sm.sc[s][pl]);
       const uint32_t tcol = tmem + lane_base + uint32_t(a * kN);
-      uint32_t va[16], vb[16];
-      sm100::tmem_ld16(tcol, va);
-      sm100::tmem_ld_wait(va);
+      uint32_t v[kQPT][16];
 #pragma unroll
-      for (int j = 0; j < kQG; ++j) {
-        uint32_t(&cur)[16] = (j & 1) ? vb : va;
-        uint32_t(&nxt)[16] = (j & 1) ? va : vb;
-        if (j + 1 < kQG) sm100::tmem_ld16(tcol + 16 * (j + 1), nxt);
+      for (int jj = 0; jj < kQPT; ++jj) sm100::tmem_ld16(tcol + 16 * (j0 + jj), v[jj]);
+#pragma unroll
+      for (int jj = 0; jj < kQPT; ++jj) sm100::tmem_ld_wait(v[jj]);
+#pragma unroll
+      for (int jj = 0; jj < kQPT; ++jj) {
+        const int j = j0 + jj;
         const QCtxS q = load_qctx(sm.qctx[s][j]);
         uint32_t key = 0;
-        if (pos < q.vis) key = rank_key(exact_score(cur, ks, q.c));
+        if (pos < q.vis) key = rank_key(exact_score(v[jj], ks, q.c));
         key = group8_max(key);
         if ((lane & 7) == 0 && pos < q.vis)
           p.bkeys[int64_t(g * kQG + j) * p.nb_stride + pos / kBlk] = key;
-        if (j + 1 < kQG) sm100::tmem_ld_wait(nxt);
       }
       sm100::tc_fence_before();
       __syncwarp();

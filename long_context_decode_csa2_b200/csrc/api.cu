@@ -179,11 +179,11 @@ csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
   uint32_t* hist = c.take<uint32_t>(size_t(B) * kCandHistBins);  // zero between calls
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SegDesc sd{seq_row_off, 0, seq_len, INT32_MAX, idx_k.rows};
-  launch_seg_check(sd, B, seg_eff, status, st);
-  const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, seg_eff, B, q_codes, q_scales, w, pool,
+  (void)seg_eff;  // lengths are checked inside the kernels
+  const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, nullptr, B, q_codes, q_scales, w, pool,
                                         pool_blocks, ckeys, hist, status, st);
   if (rc != CSA2_OK) return rc;
-  launch_select(kSelPoolCand, ckeys, int64_t(pool_blocks) * kBlk, seg_eff, B, pool_blocks, pool, k, topk_out, hist,
+  launch_select(kSelPoolCand, ckeys, int64_t(pool_blocks) * kBlk, nullptr, B, pool_blocks, pool, k, topk_out, hist,
                 st);
   return check_launch(fn);
 }
@@ -222,7 +222,8 @@ csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv,
   a.mcodes = main_kv.codes;
   a.mscales = main_kv.scales;
   a.sd = SegDesc{seq_row_off, 0, seq_len, INT32_MAX, main_kv.rows};
-  a.seg_eff = seg_eff;
+  a.seg_eff = nullptr;  // checked per segment inside the kernel
+  (void)seg_eff;
   a.topk = topk;
   a.k = k;
   a.win = win;
@@ -233,7 +234,6 @@ csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv,
   a.lse = lse;
   a.S = B;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  launch_seg_check(a.sd, B, seg_eff, a.status, st);
   launch_attention(a, st);
   return check_launch(fn);
 }

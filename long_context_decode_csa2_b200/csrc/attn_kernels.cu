@@ -106,7 +106,7 @@ __device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, in
   const ChunkSrc src = chunk_src(a, s, c);
   bool ok = r < src.nkeys;
   if (!src.is_win && ok) {
-    const int64_t eff = a.seg_eff[s];
+    const int64_t eff = a.seg_eff ? int64_t(a.seg_eff[s]) : seg_len_checked(a.sd, s, a.status);
     if (tpos >= eff) {
       if (half == 0) set_status(a.status, CSA2_DEV_INDEX_RANGE);
       ok = false;

@@ -13,6 +13,24 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t flag) {
   if (status) atomicOr(status, flag);
 }
 
+// Checked visible length of segment s: negative lengths count as 0, lengths
+// above the host bound are clamped (CSA2_DEV_LENGTH), and a misaligned or
+// out-of-capacity row range makes the segment empty (CSA2_DEV_ROW_LAYOUT).
+__device__ __forceinline__ int64_t seg_len_checked(const SegDesc& sd, int s, uint32_t* status) {
+  int64_t L = sd.len[s];
+  const int64_t off = sd.row_off ? sd.row_off[s] : sd.row0;
+  if (L < 0) L = 0;
+  if (L > sd.max_len) {
+    set_status(status, CSA2_DEV_LENGTH);
+    L = sd.max_len;
+  }
+  if ((off & 7) != 0 || off < 0 || off + L > sd.cache_rows) {
+    set_status(status, CSA2_DEV_ROW_LAYOUT);
+    L = 0;
+  }
+  return L;
+}
+
 // Order-preserving map of an fp32 score to a uint32 key; -0 ranks as +0.
 // Key 0 is reserved for "absent" (only a negative NaN would map there).
 __device__ __forceinline__ uint32_t rank_key(float s) {

@@ -1,4 +1,4 @@
-// Indexer kernels: segment checks, prefill visibility, and deterministic radix
+// Indexer kernels: prefill visibility and deterministic radix
 // selection (Top-k by key desc / index asc, output ascending).  The scans and
 // the pool scoring run on the tensor cores (scan_tc.cu, prefill_tc.cu).
 //
@@ -9,30 +9,6 @@
 #include "device_common.cuh"
 
 namespace csa2 {
-
-// ---------------------------------------------------------------------------
-// Segment checks: effective visible length (0 for a bad layout).
-// ---------------------------------------------------------------------------
-__global__ void k_seg_check(SegDesc sd, int S, int32_t* seg_eff, uint32_t* status) {
-  const int s = blockIdx.x * blockDim.x + threadIdx.x;
-  if (s >= S) return;
-  int64_t L = sd.len[s];
-  const int64_t off = sd.row_off ? sd.row_off[s] : sd.row0;
-  if (L < 0) L = 0;
-  if (L > sd.max_len) {
-    set_status(status, CSA2_DEV_LENGTH);
-    L = sd.max_len;
-  }
-  if ((off & 7) != 0 || off < 0 || off + L > sd.cache_rows) {
-    set_status(status, CSA2_DEV_ROW_LAYOUT);
-    L = 0;
-  }
-  seg_eff[s] = static_cast<int32_t>(L);
-}
-
-void launch_seg_check(const SegDesc& sd, int S, int32_t* seg_eff, uint32_t* status, cudaStream_t st) {
-  k_seg_check<<<(S + 255) / 256, 256, 0, st>>>(sd, S, seg_eff, status);
-}
 
 // ---------------------------------------------------------------------------
 // Prefill: visible entry counts (the scan itself runs on the tensor cores,

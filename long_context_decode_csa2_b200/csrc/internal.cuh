@@ -60,9 +60,6 @@ constexpr int kCandHistBins = 1 << kCandHistBits;
 // ---------------------------------------------------------------------------
 // Kernel launchers (each returns after enqueueing on `st`).
 // ---------------------------------------------------------------------------
-// Effective length per segment after layout checks -> seg_eff [S].
-void launch_seg_check(const SegDesc& sd, int S, int32_t* seg_eff, uint32_t* status, cudaStream_t st);
-
 // Tensor-core scan (tcgen05 + TMA): segment checks, work-item prefix
 // (tile_start [S+1]), block keys and optional scores.
 size_t scan_tc_prefix_ints(int S);
@@ -72,7 +69,8 @@ csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
                            uint32_t* hist, uint32_t* status, cudaStream_t st);
 
 // Scores of pool candidates 8*pool[s][i/8] + i%8 -> keys [S][P*8] (0 = absent),
-// on the tensor cores (gathered 8-row TMA boxes).
+// on the tensor cores (gathered with cp.async).  seg_eff may be null: the
+// kernel then checks each segment's length from sd itself.
 csa2_status launch_pool_tc(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const int32_t* seg_eff,
                            int S, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
                            const int32_t* pool, int P, uint32_t* ckeys, uint32_t* hist, uint32_t* status,
@@ -107,7 +105,7 @@ struct AttnArgs {
   const uint8_t* mcodes;
   const uint8_t* mscales;
   SegDesc sd;                   // rows of segment s (len = visible count)
-  const int32_t* seg_eff;       // checked visible count
+  const int32_t* seg_eff;       // checked visible count, or null: checked from sd in the kernel
   const int32_t* topk;          // [S][k]
   int k;
   // decode window

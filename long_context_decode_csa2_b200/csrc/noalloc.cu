@@ -102,7 +102,8 @@ extern "C" csa2_status csa2_sparse_attn_decode_noalloc(const uint16_t* q, csa2_m
   a.mcodes = main_kv.codes;
   a.mscales = main_kv.scales;
   a.sd = SegDesc{seq_row_off, 0, seq_len, INT32_MAX, main_kv.rows};
-  a.seg_eff = seg_eff;
+  a.seg_eff = nullptr;  // checked per segment inside the kernel
+  (void)seg_eff;
   a.topk = topk;
   a.k = k;
   a.win = win;
@@ -112,7 +113,6 @@ extern "C" csa2_status csa2_sparse_attn_decode_noalloc(const uint16_t* q, csa2_m
   a.out = out;
   a.lse = lse;
   a.S = B;
-  launch_seg_check(a.sd, B, seg_eff, a.status, st);
   launch_attention(a, st);
   if (flags_out) {
     e = cudaMemcpyAsync(flags_out, a.status, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st);

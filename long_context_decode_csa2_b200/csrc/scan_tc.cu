@@ -93,7 +93,8 @@ struct ScanParams {
   const float* w;
   const int64_t* row_off;     // [S] or null -> row0
   int64_t row0;
-  const int32_t* seg_eff;
+  const int32_t* seg_eff;     // checked lengths, or null: computed from sd
+  SegDesc sd;
   const int32_t* tile_start;  // scan: [S+1] item prefix
   int S;
   // scan outputs
@@ -134,6 +135,10 @@ __device__ __forceinline__ bool aborted(Smem& sm) {
 
 __device__ __forceinline__ int64_t seg_row_off(const ScanParams& p, int s) {
   return p.row_off ? p.row_off[s] : p.row0;
+}
+
+__device__ __forceinline__ int64_t seg_len(const ScanParams& p, int s) {
+  return p.seg_eff ? int64_t(p.seg_eff[s]) : seg_len_checked(p.sd, s, p.status);
 }
 
 // Writes the B operand image of a segment's query into `bo` (whole warp).
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
         next_start = __ldg(p.tile_start + b + 1);
       }
       int64_t seq_off = seg_row_off(p, b);
-      int64_t seq_len = p.seg_eff[b];
+      int64_t seq_len = seg_len(p, b);
       int qb = -1;
       uint2 qreg = make_uint2(0, 0);
       int pool_seg = -1;  // segment whose pool ids are in sm.segpool
@@ -227,7 +232,7 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
           if (nb != b) {
             b = nb;
             seq_off = seg_row_off(p, b);
-            seq_len = p.seg_eff[b];
+            seq_len = seg_len(p, b);
           }
           j = it - b * p.items_per_seg;
         } else {
@@ -236,7 +241,7 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
             seq_start = next_start;
             next_start = __ldg(p.tile_start + b + 1);
             seq_off = seg_row_off(p, b);
-            seq_len = p.seg_eff[b];
+            seq_len = seg_len(p, b);
           }
           j = it - seq_start;
         }
@@ -395,7 +400,7 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
       const int2 inf = sm.info[s];
       if (inf.x != cur) {
         cur = inf.x;
-        L = p.seg_eff[cur];
+        L = seg_len(p, cur);
         make_qctx(qc, p.q_scales + int64_t(cur) * 16, p.w + int64_t(cur) * kHi);
       }
       uint32_t swv[kMT];
@@ -587,6 +592,7 @@ csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
   p.row_off = sd.row_off;
   p.row0 = sd.row0;
   p.seg_eff = seg_eff;
+  p.sd = sd;
   p.tile_start = tile_start;
   p.S = S;
   p.bkeys = bkeys;
@@ -617,6 +623,7 @@ csa2_status launch_pool_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
   p.row_off = sd.row_off;
   p.row0 = sd.row0;
   p.seg_eff = seg_eff;
+  p.sd = sd;
   p.S = S;
   p.pool = pool;
   p.P = P;

@@ -81,7 +81,6 @@ class DecodeStep:
             self.ws_re = [C.workspace(re_bytes, dev) if act == "reindex" else None for _, _, _, act in self.plan]
             self.ws_attn = [C.workspace(attn_bytes, dev) for _ in range(nL)]
             self.streams = [torch.cuda.Stream(device=dev) for _ in range(max(1, side_streams))]
-            self.ev_start = torch.cuda.Event()
             self.ev_idx = [torch.cuda.Event() for _ in range(nL)]
             self.ev_done = [torch.cuda.Event() for _ in range(nL)]
         else:
@@ -108,19 +107,26 @@ class DecodeStep:
         if self.hook is not None:
             self.hook(name, phase, stream)
 
-    def run(self, caches, seq_row_off, seq_len, layers, stream=None):
+    def run(self, caches, seq_row_off, seq_len, layers, stream=None, ready=None, on_layer_done=None):
         """caches: [FullCache] per Full layer; layers: per layer dict of device
-        tensors q, q_codes, q_scales, w, win, win_scale, win_len."""
+        tensors q, q_codes, q_scales, w, win, win_scale, win_len.
+
+        ready: optional per-layer CUDA events; a layer's calls wait for its
+        event (e.g. its inputs arriving on a copy stream).  on_layer_done:
+        optional callable(layer, event), called once the layer's attention is
+        enqueued, with an event that completes after it (e.g. to copy the
+        layer's output out while later layers run)."""
         main = stream if stream is not None else torch.cuda.current_stream()
-        if self.concurrent:
-            self.ev_start.record(main)
         pool, pool_ev = None, None
         last, last_ev = None, None
         side = 0
         for layer, mode, f, act in self.plan:
             L = layers[layer]
             cache = caches[f]
+            ev_ready = ready[layer] if ready is not None else None
             if act == "scan":
+                if ev_ready is not None:
+                    main.wait_event(ev_ready)
                 pool = self.pools[layer]
                 self._hook("csa2_index_full", "begin", main)
                 C.csa2_index_full(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len, self.max_len,
@@ -135,6 +141,8 @@ class DecodeStep:
                 side += 1
             else:
                 s = main
+            if ev_ready is not None and act != "scan":
+                s.wait_event(ev_ready)
             if act == "reindex":
                 if self.concurrent:
                     s.wait_event(pool_ev)
@@ -159,6 +167,13 @@ class DecodeStep:
             self._hook("csa2_sparse_attn_decode", "end", s)
             if self.concurrent:
                 self.ev_done[layer].record(s)
+            if on_layer_done is not None:
+                if self.concurrent:
+                    on_layer_done(layer, self.ev_done[layer])
+                else:
+                    ev = torch.cuda.Event()
+                    ev.record(s)
+                    on_layer_done(layer, ev)
         if self.concurrent:
             for ev in self.ev_done:
                 main.wait_event(ev)

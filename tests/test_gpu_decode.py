@@ -94,3 +94,45 @@ def test_decode_long_full_size_sampled():
             assert np.array_equal(host(step.topk[layer][b:b + 1]), ref["topk"][layer]), (b, layer)
             check_attention(host(step.out[layer][b:b + 1]), ref["out"][layer], what=f"seq {b} layer {layer}")
         assert np.array_equal(host(step.pool[b:b + 1]), ref["pools"][0])
+
+
+def test_decode_with_input_events_and_layer_callbacks():
+    """Inputs arriving on a copy stream (per-layer events) and outputs copied
+    out per layer give the same results as the plain step."""
+    wl = W.DecodeWorkload("stack_tiny", np.array([20000, 777, 4096]), "FRRU", needles=8)
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    caches_h = [W.full_cache_host(wl, f, layers[f]["q_codes"], layers[f]["q_scales"]) for f in wl.full_layers()]
+    caches_d = [FullCache(C.cache(dev(c["idx_codes"]), dev(c["idx_scales"])),
+                          C.cache(dev(c["main_codes"]), dev(c["main_scales"]))) for c in caches_h]
+    off_d, len_d = dev(caches_h[0]["seq_row_off"]), dev(wl.lengths.astype(np.int32))
+    plain = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
+    plain.run(caches_d, off_d, len_d, _device_layers(layers))
+    torch.cuda.synchronize()
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
+    keys = ("q", "q_codes", "q_scales", "w", "win", "win_scale", "win_len")
+    dl = [{k: torch.empty_like(dev(L[k])) for k in keys} for L in layers]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = [torch.cuda.Event() for _ in layers]
+    with torch.cuda.stream(h2d):
+        for l, L in enumerate(layers):
+            for k in keys:
+                dl[l][k].copy_(torch.from_numpy(np.ascontiguousarray(
+                    L[k].view(np.int16) if L[k].dtype == np.uint16 else L[k])).pin_memory().view(dl[l][k].dtype),
+                    non_blocking=True)
+            ev[l].record(h2d)
+    outs = torch.empty((len(layers),) + tuple(step.out.shape[1:]), dtype=torch.float32).pin_memory()
+    done = []
+
+    def copy_out(layer, e):
+        done.append(layer)
+        d2h.wait_event(e)
+        with torch.cuda.stream(d2h):
+            outs[layer].copy_(step.out[layer], non_blocking=True)
+
+    step.run(caches_d, off_d, len_d, dl, ready=ev, on_layer_done=copy_out)
+    torch.cuda.synchronize()
+    assert done == list(range(len(layers)))
+    assert step.device_flags() == 0 and plain.device_flags() == 0
+    for layer in range(len(layers)):
+        assert np.array_equal(host(step.topk[layer]), host(plain.topk[layer]))
+        assert np.array_equal(outs[layer].numpy(), host(plain.out[layer]))

@@ -175,9 +175,37 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool acti
 // keys) into shared memory and zeroes the row for the next call; returns this
 // thread's share of the key count.
 template <int NB>
-__device__ __forceinline__ uint32_t take_hist(uint32_t* __restrict__ gh, uint32_t* __restrict__ hist) {
-  constexpr int kVec = NB / 4 / kSelThreads;  // uint4 per thread
+struct HistPart {
+  static constexpr int kVec = NB / 4 / kSelThreads;  // uint4 per thread
   static_assert(kVec >= 1 && NB % (4 * kSelThreads) == 0, "histogram rows are whole uint4 per thread");
+  uint4 v[kVec];
+};
+
+// First half of take_hist: this thread's share of the row, loaded (kept in
+// registers so the loads overlap other work).
+template <int NB>
+__device__ __forceinline__ void load_hist(const uint32_t* __restrict__ gh, HistPart<NB>& hp) {
+#pragma unroll
+  for (int j = 0; j < HistPart<NB>::kVec; ++j)
+    hp.v[j] = __ldcg(reinterpret_cast<const uint4*>(gh) + threadIdx.x + j * kSelThreads);
+}
+
+// Second half: into shared memory, and the global row zeroed where non-zero.
+template <int NB>
+__device__ __forceinline__ void store_hist(uint32_t* __restrict__ gh, uint32_t* __restrict__ hist,
+                                           const HistPart<NB>& hp) {
+  uint4* g4 = reinterpret_cast<uint4*>(gh);
+#pragma unroll
+  for (int j = 0; j < HistPart<NB>::kVec; ++j) {
+    const uint4 v = hp.v[j];
+    reinterpret_cast<uint4*>(hist)[threadIdx.x + j * kSelThreads] = v;
+    if ((v.x | v.y | v.z | v.w) != 0u) g4[threadIdx.x + j * kSelThreads] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+template <int NB>
+__device__ __forceinline__ uint32_t take_hist(uint32_t* __restrict__ gh, uint32_t* __restrict__ hist) {
+  constexpr int kVec = HistPart<NB>::kVec;
   uint4 v[kVec];
   uint4* g4 = reinterpret_cast<uint4*>(gh);
 #pragma unroll
@@ -242,7 +270,7 @@ __device__ void ordered_output_global(const void* in, int64_t base, int64_t n, u
 }
 
 template <int KIND, bool SMALL>
-__global__ void __launch_bounds__(kSelThreads) k_select(const void* __restrict__ in, int64_t in_stride,
+__global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restrict__ in, int64_t in_stride,
                                                         const int32_t* __restrict__ seg_eff, int P,
                                                         const int32_t* __restrict__ pool, int k,
                                                         int32_t* __restrict__ out, uint32_t* __restrict__ ghist) {
@@ -259,8 +287,12 @@ __global__ void __launch_bounds__(kSelThreads) k_select(const void* __restrict__
 
   if (SMALL) {
     // ---- one chunk: this thread's 16 keys stay in registers ----
+    constexpr int HB = (KIND == kSelPoolCand) ? kCandHistBits : kHist1Bits;
+    constexpr int NB = 1 << HB;
     uint32_t kk[kSelPer];
     const int64_t i0 = int64_t(tid) * kSelPer;
+    HistPart<NB> hp;
+    if (ghist) load_hist<NB>(ghist + int64_t(s) * NB, hp);  // in flight with the keys
     load_keys<KIND>(in, base, i0, n, kk);
     uint32_t present = 0;
 #pragma unroll
@@ -271,11 +303,9 @@ __global__ void __launch_bounds__(kSelThreads) k_select(const void* __restrict__
     if (ghist) {
       // the top HB bits from the producer's histogram; the low bits by radix
       // digits of up to 8 bits over the keys of the threshold bucket only
-      constexpr int HB = (KIND == kSelPoolCand) ? kCandHistBits : kHist1Bits;
-      constexpr int NB = 1 << HB;
       uint32_t* hist = dsm;       // NB
       uint32_t* h2 = dsm + NB;    // 256
-      take_hist<NB>(ghist + int64_t(s) * NB, hist);
+      store_hist<NB>(ghist + int64_t(s) * NB, hist, hp);
       __syncthreads();
       if (total > uint32_t(k)) {
         find_bin(hist, NB, uint32_t(k), sh);
@@ -421,13 +451,20 @@ __global__ void __launch_bounds__(kSelThreads) k_select(const void* __restrict__
     load_keys<KIND>(in, base, int64_t(tid) * kSelPer, n, kk);
     for (int64_t c0 = 0; c0 < n; c0 += kSelChunk) {
       if (c0 + kSelChunk < n) load_keys<KIND>(in, base, c0 + kSelChunk + int64_t(tid) * kSelPer, n, nx);
-      uint32_t na = 0, nc = 0;
+      // most threads hold no key at or above the bucket: one max decides
+      uint32_t mx = 0;
 #pragma unroll
-      for (int e = 0; e < kSelPer; ++e) {
-        const uint32_t key = kk[e], hi = key >> kLowBits;
-        if (key != 0u) {
-          if (all || hi > b1) ++na;
-          else if (hi == b1) ++nc;
+      for (int e = 0; e < kSelPer; ++e) mx = max(mx, kk[e]);
+      const bool hot = mx != 0u && (all || (mx >> kLowBits) >= b1);
+      uint32_t na = 0, nc = 0;
+      if (hot) {
+#pragma unroll
+        for (int e = 0; e < kSelPer; ++e) {
+          const uint32_t key = kk[e], hi = key >> kLowBits;
+          if (key != 0u) {
+            if (all || hi > b1) ++na;
+            else if (hi == b1) ++nc;
+          }
         }
       }
       const uint32_t ex = block_exclusive_scan((na << 16) | nc, sh.warp_sums, &sh.total);
@@ -435,7 +472,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select(const void* __restrict__
       uint32_t a = run_a + (ex >> 16), c = run_c + (ex & 0xFFFFu);
       const uint32_t i0 = uint32_t(c0) + uint32_t(tid) * kSelPer;
 #pragma unroll
-      for (int e = 0; e < kSelPer; ++e) {
+      for (int e = 0; e < kSelPer && hot; ++e) {
         const uint32_t key = kk[e], hi = key >> kLowBits;
         if (key != 0u) {
           if (all || hi > b1) {

@@ -21,7 +21,7 @@ namespace {
 constexpr int kNoAllocMaxSeqs = 64;
 constexpr int kNoAllocMaxTopk = 512;
 constexpr size_t kNoAllocStatusBytes = 256;                       // device status word
-constexpr size_t kNoAllocSeqBytes = 256;                          // 64 visible counts
+constexpr size_t kNoAllocSeqBytes = 256;                          // reserved (layout unchanged)
 constexpr size_t kNoAllocCounterBytes = 256;                      // 64 arrival counters (self-resetting)
 constexpr size_t kNoAllocPartialBytes =                           // split-KV partials
     size_t(kNoAllocMaxSeqs) * (kNoAllocMaxTopk / 128 + 1) * (kHq * kD + 2 * kHq) * sizeof(float);
@@ -90,7 +90,6 @@ extern "C" csa2_status csa2_sparse_attn_decode_noalloc(const uint16_t* q, csa2_m
   char* p = static_cast<char*>(base);
   AttnArgs a{};
   a.status = reinterpret_cast<uint32_t*>(p);
-  int32_t* seg_eff = reinterpret_cast<int32_t*>(p + kNoAllocStatusBytes);
   a.counters = reinterpret_cast<int32_t*>(p + kNoAllocStatusBytes + kNoAllocSeqBytes);
   a.partial = reinterpret_cast<float*>(p + kNoAllocStatusBytes + kNoAllocSeqBytes + kNoAllocCounterBytes);
   // The status word must start at zero for this call.  The arrival counters
@@ -102,8 +101,7 @@ extern "C" csa2_status csa2_sparse_attn_decode_noalloc(const uint16_t* q, csa2_m
   a.mcodes = main_kv.codes;
   a.mscales = main_kv.scales;
   a.sd = SegDesc{seq_row_off, 0, seq_len, INT32_MAX, main_kv.rows};
-  a.seg_eff = nullptr;  // checked per segment inside the kernel
-  (void)seg_eff;
+  a.seg_eff = nullptr;  // lengths are checked per segment inside the kernel
   a.topk = topk;
   a.k = k;
   a.win = win;

@@ -3,20 +3,24 @@
 // KV Cache Compression", section "三个方向一起压小缓存": 512 entries per layer,
 // MXFP4 main KV, FP8 window; section "后 20 层干脆共用一份 KV": 128-token window).
 //
-// Work split: ceil(k/128) chunks of selected rows plus one window chunk per
-// segment, walked by a persistent grid (one CTA per SM, consecutive chunks
-// per CTA).  While a CTA computes one chunk, cp.async brings the next
-// chunk's raw rows (272-byte MXFP4 rows or 512-byte E4M3 rows) into a staging
-// buffer; the chunk's Top-k ids are loaded one chunk earlier still.  Each
-// chunk's rows are dequantised exactly into fp16 in shared memory (E2M1 x 2^X
-// and raw E4M3 are exact in fp16 inside the range checked below), and both
+// Work split: a segment's keys are chunks of 64 rows (ceil(k/64) chunks of
+// selected rows, then two window chunks), and R CTAs share a segment, each
+// walking a contiguous run of its chunks (R = SMs / segments, at most 4, so
+// that small batches still fill the GPU in one wave).  A CTA loads Q once,
+// keeps an online softmax (running max, sum and output per head) across its
+// chunks, and while it computes one chunk, cp.async brings the next chunk's
+// raw rows (272-byte MXFP4 rows or 512-byte E4M3 rows) into a staging
+// buffer; the Top-k ids are loaded one chunk earlier still.  Each chunk's
+// rows are dequantised exactly into fp16 in shared memory (E2M1 x 2^X and
+// raw E4M3 are exact in fp16 inside the range checked below), and both
 // products run on the tensor cores with warp-level mma (fp16 inputs, fp32
 // accumulation):
-//   S = Q K^T  (16 heads x 128 keys),  P = exp(S*scale - max),  O = P V.
-// The window's fp32 scale multiplies its logits and its partial output in
-// fp32, never the fp16 values.  Each chunk leaves an unnormalised partial
-// (O, max, sum) per head; the last CTA to finish a segment's chunks combines
-// them in a fixed order (deterministic) and resets the segment's counter.
+//   S = Q K^T  (16 heads x 64 keys),  P = exp(S*scale - max),  O = P V.
+// The window's fp32 scale multiplies its logits and its output in fp32, never
+// the fp16 values, so a CTA keeps the window chunks in a partial of their
+// own.  Each CTA writes its partials (O, max, sum per head); the last CTA of
+// a segment to finish combines them in a fixed order (deterministic) and
+// resets the segment's arrival counter.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -26,20 +30,32 @@
 
 namespace csa2 {
 
-constexpr int kChunk = 128;
-constexpr int kAttnThreads = 256;                 // 8 warps
-constexpr int kPartFloats = kHq * kD + 2 * kHq;  // O, then m, then l
-constexpr int kQS = kD + 8;                       // smem row stride (halves) of Q and K
-constexpr int kPS = kChunk + 8;                   // smem row stride (halves) of P
+constexpr int kChunk = 64;                         // keys per chunk
+constexpr int kAttnThreads = 256;                  // 8 warps
+constexpr int kPartFloats = kHq * kD + 2 * kHq;    // O, then m, then l
+constexpr int kQS = kD + 8;                        // smem row stride (halves) of Q and K
+constexpr int kPS = kChunk + 8;                    // smem row stride (halves) of P
+constexpr int kWinChunks = kWin / kChunk;          // 2
+constexpr int kMaxSplits = 4;                      // CTAs per segment at most
+constexpr int kMaxSlots = 2 * kMaxSplits;          // partials per segment (main + window per CTA)
+constexpr int kRawMain = kMainCodeBytes + kMainScaleBytes;  // 272: codes then scales (row stride 68
+                                                            // words: conflict-free 16-byte reads)
+constexpr int kRawWin = kD + 16;                   // 528: one E4M3 row + pad
 
-int attn_num_chunks(int k) { return (k + kChunk - 1) / kChunk + 1; }
-size_t attn_partial_bytes(int S, int k) {
-  return size_t(S) * attn_num_chunks(k) * kPartFloats * sizeof(float);
+__host__ __device__ inline int attn_main_chunks(int k) { return (k + kChunk - 1) / kChunk; }
+
+int attn_num_chunks(int k) { return attn_main_chunks(k) + kWinChunks; }
+
+int attn_splits(int S, int k) {
+  const int sms = num_sms();
+  int r = S > 0 ? sms / S : 1;
+  r = std::min(r, std::min(kMaxSplits, attn_num_chunks(k)));
+  return std::max(r, 1);
 }
 
-constexpr int kRawMain = kMainCodeBytes + kMainScaleBytes + 0;  // 272: codes then scales (row stride
-                                                                 // 68 words: conflict-free 16-byte reads)
-constexpr int kRawWin = kD + 16;                                 // 528: one E4M3 row + pad
+size_t attn_partial_bytes(int S, int k) {
+  return size_t(S) * 2 * attn_splits(S, k) * kPartFloats * sizeof(float);
+}
 
 struct AttnSmem {
   __half q[kHq][kQS];
@@ -51,8 +67,10 @@ struct AttnSmem {
   } raw;                                 // staged raw rows of the next chunk
   float red_max[8][kHq];
   float red_sum[8][kHq];
+  float m_run[kHq];                      // online softmax state of the current part
+  float l_run[kHq];
   int valid[kChunk];
-  float fac[CSA2_MAX_TOPK / kChunk + 1][kHq];
+  float fac[kMaxSlots][kHq];
   int last;
 };
 
@@ -66,16 +84,21 @@ struct ChunkSrc {
 
 __device__ __forceinline__ ChunkSrc chunk_src(const AttnArgs& a, int s, int c) {
   ChunkSrc r;
-  const int nmain = (a.k + kChunk - 1) / kChunk;
-  r.is_win = (c == nmain);
+  const int nmain = attn_main_chunks(a.k);
+  r.is_win = (c >= nmain);
   r.kscale = 1.0f;
   r.win_base = nullptr;
   if (!r.is_win) {
     r.nkeys = min(kChunk, a.k - c * kChunk);
-  } else if (a.q_pos == nullptr) {
-    r.nkeys = max(0, min(kWin, a.win_len[s]));
+    return r;
+  }
+  const int wc = c - nmain;  // window chunk 0 or 1
+  int nwin;
+  const uint8_t* base;
+  if (a.q_pos == nullptr) {
+    nwin = max(0, min(kWin, a.win_len[s]));
     r.kscale = a.win_scale[s];
-    r.win_base = a.win + int64_t(s) * kWin * kD;
+    base = a.win + int64_t(s) * kWin * kD;
   } else {
     int64_t p = a.q_pos[s];
     if (p >= a.n_raw) {
@@ -83,32 +106,33 @@ __device__ __forceinline__ ChunkSrc chunk_src(const AttnArgs& a, int s, int c) {
       p = a.n_raw - 1;
     }
     const int64_t lo = p - (kWin - 1) > 0 ? p - (kWin - 1) : 0;
-    r.nkeys = p >= 0 ? int(p - lo + 1) : 0;
+    nwin = p >= 0 ? int(p - lo + 1) : 0;
     r.kscale = a.raw_scale;
-    r.win_base = a.raw_win + lo * kD;
+    base = a.raw_win + lo * kD;
   }
+  r.nkeys = max(0, min(kChunk, nwin - wc * kChunk));
+  r.win_base = base + int64_t(wc) * kChunk * kD;
   return r;
 }
 
 // Top-k id of this thread's row of chunk c (or -1 when the row is not a
 // selected main row).  Issued one chunk ahead of its use.
 __device__ __forceinline__ int32_t chunk_tpos(const AttnArgs& a, int s, int c, int r) {
-  const int nmain = (a.k + kChunk - 1) / kChunk;
-  if (c >= nmain) return -1;
+  if (c >= attn_main_chunks(a.k)) return -1;
   const int idx = c * kChunk + r;
   return idx < a.k ? __ldg(a.topk + int64_t(s) * a.k + idx) : -1;
 }
 
 // Issues the cp.async copies of chunk c's rows into sm.raw (this thread: row
-// r = tid % 128, half tid / 128 of it) and returns whether row r is present.
+// r = tid % 64, quarter tid / 64 of it) and returns whether row r is present.
 __device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, int s, int c, int32_t tpos) {
-  const int tid = threadIdx.x, r = tid & (kChunk - 1), half = tid / kChunk;
+  const int tid = threadIdx.x, r = tid & (kChunk - 1), qt = tid / kChunk;
   const ChunkSrc src = chunk_src(a, s, c);
   bool ok = r < src.nkeys;
   if (!src.is_win && ok) {
     const int64_t eff = a.seg_eff ? int64_t(a.seg_eff[s]) : seg_len_checked(a.sd, s, a.status);
     if (tpos >= eff) {
-      if (half == 0) set_status(a.status, CSA2_DEV_INDEX_RANGE);
+      if (qt == 0) set_status(a.status, CSA2_DEV_INDEX_RANGE);
       ok = false;
     } else if (tpos < 0) {
       ok = false;
@@ -118,16 +142,16 @@ __device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, in
     if (!src.is_win) {
       const int64_t off = a.sd.row_off ? a.sd.row_off[s] : a.sd.row0;
       const int64_t row = off + tpos;
-      const uint8_t* cs = a.mcodes + row * kMainCodeBytes + half * (kMainCodeBytes / 2);
-      uint8_t* dst = sm.raw.main[r] + half * (kMainCodeBytes / 2);
+      const uint8_t* cs = a.mcodes + row * kMainCodeBytes + qt * (kMainCodeBytes / 4);
+      uint8_t* dst = sm.raw.main[r] + qt * (kMainCodeBytes / 4);
 #pragma unroll
-      for (int i = 0; i < kMainCodeBytes / 2 / 16; ++i) sm100::cp_async16(dst + 16 * i, cs + 16 * i);
-      if (half == 0) sm100::cp_async16(sm.raw.main[r] + kMainCodeBytes, a.mscales + row * kMainScaleBytes);
+      for (int i = 0; i < kMainCodeBytes / 4 / 16; ++i) sm100::cp_async16(dst + 16 * i, cs + 16 * i);
+      if (qt == 0) sm100::cp_async16(sm.raw.main[r] + kMainCodeBytes, a.mscales + row * kMainScaleBytes);
     } else {
-      const uint8_t* ws = src.win_base + int64_t(r) * kD + half * (kD / 2);
-      uint8_t* dst = sm.raw.win[r] + half * (kD / 2);
+      const uint8_t* ws = src.win_base + int64_t(r) * kD + qt * (kD / 4);
+      uint8_t* dst = sm.raw.win[r] + qt * (kD / 4);
 #pragma unroll
-      for (int i = 0; i < kD / 2 / 16; ++i) sm100::cp_async16(dst + 16 * i, ws + 16 * i);
+      for (int i = 0; i < kD / 4 / 16; ++i) sm100::cp_async16(dst + 16 * i, ws + 16 * i);
     }
   }
   return ok;
@@ -198,16 +222,16 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, AttnSmem& sm, int s) {
 }
 
 // Staged raw rows -> fp16 keys in sm.kv (absent rows as zeros) and the
-// row-valid flags.  Thread: row r = tid % 128, blocks tid/128 + 2i.
+// row-valid flags.  Thread: row r = tid % 64, blocks tid/64 + 4i.
 __device__ __forceinline__ void dequant_chunk(const AttnArgs& a, AttnSmem& sm, bool is_win, bool row_ok) {
   const int tid = threadIdx.x;
   const int r = tid & (kChunk - 1);
-  constexpr int kBPT = 16 / (kAttnThreads / kChunk);  // blocks per thread (8)
+  constexpr int kBPT = 16 / (kAttnThreads / kChunk);  // blocks per thread (4)
   const int b0 = tid / kChunk;
   if (b0 == 0) sm.valid[r] = row_ok;
 #pragma unroll
   for (int i = 0; i < kBPT; ++i) {
-    const int b = b0 + 2 * i;
+    const int b = b0 + 4 * i;
     uint4* dst = reinterpret_cast<uint4*>(&sm.kv[r][32 * b]);
     if (!row_ok) {
 #pragma unroll
@@ -242,39 +266,48 @@ __device__ __forceinline__ void dequant_chunk(const AttnArgs& a, AttnSmem& sm, b
   }
 }
 
-// S = Q K^T, softmax, O = P V over the chunk in sm.kv; writes the partial.
-__device__ __forceinline__ void attn_compute(const AttnArgs& a, AttnSmem& sm, float* part, int nkeys,
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+}
+
+// One chunk (keys in sm.kv) into the running softmax state: S = Q K^T for the
+// chunk's keys, the running max / sum per head (sm.m_run, sm.l_run) and the
+// output accumulator oacc (warp w: dims 64w .. 64w+63, rows g and g+8).
+__device__ __forceinline__ void chunk_update(const AttnArgs& a, AttnSmem& sm, float (&oacc)[8][4], int nkeys,
                                              float kscale) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  // ---- S = Q K^T: warp w owns keys 16w .. 16w+15 (two n-tiles of 8) ----
-  float sacc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+  // ---- S: warp w owns keys 8w .. 8w+7; two accumulators over alternate k-steps ----
+  float sa[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
   {
-    const int kr = 16 * warp + (lane & 7) + 8 * (lane >> 4);  // key row for the B matrices
+    const int kr = 8 * warp + (lane & 7);
     const int kc = 8 * ((lane >> 3) & 1);
-    const int qr = (lane & 7) + 8 * ((lane >> 3) & 1);        // head row for the A matrices
+    const int qr = (lane & 7) + 8 * ((lane >> 3) & 1);
     const int qc = 8 * (lane >> 4);
 #pragma unroll 4
-    for (int k0 = 0; k0 < kD; k0 += 16) {
-      uint32_t af[4], bf[4];
+    for (int k0 = 0; k0 < kD; k0 += 32) {
+      uint32_t af[4], bf[2], af2[4], bf2[2];
       ldsm_x4(af, &sm.q[qr][k0 + qc]);
-      ldsm_x4(bf, &sm.kv[kr][k0 + kc]);
-      mma16816(sacc[0], af, bf[0], bf[1]);
-      mma16816(sacc[1], af, bf[2], bf[3]);
+      ldsm_x2(bf, &sm.kv[kr][k0 + kc]);
+      ldsm_x4(af2, &sm.q[qr][k0 + 16 + qc]);
+      ldsm_x2(bf2, &sm.kv[kr][k0 + 16 + kc]);
+      mma16816(sa, af, bf[0], bf[1]);
+      mma16816(sb, af2, bf2[0], bf2[1]);
     }
   }
-  // ---- softmax over the chunk's keys (per head) ----
+  // ---- logits, chunk maxima (per head) ----
   const float lscale = a.sm_scale * kscale;
+  float sv[4];
   float mx[2] = {-INFINITY, -INFINITY};  // heads g, g+8
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int key = 16 * warp + 8 * nt + 2 * t + (j & 1);
-      const float v = sm.valid[key] ? sacc[nt][j] * lscale : -INFINITY;
-      sacc[nt][j] = v;
-      mx[j >> 1] = fmaxf(mx[j >> 1], v);
-    }
+  for (int j = 0; j < 4; ++j) {
+    const int key = 8 * warp + 2 * t + (j & 1);
+    const float v = (key < nkeys && sm.valid[key]) ? (sa[j] + sb[j]) * lscale : -INFINITY;
+    sv[j] = v;
+    mx[j >> 1] = fmaxf(mx[j >> 1], v);
+  }
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
@@ -285,26 +318,28 @@ __device__ __forceinline__ void attn_compute(const AttnArgs& a, AttnSmem& sm, fl
     sm.red_max[warp][g + 8] = mx[1];
   }
   __syncthreads();
-  float m[2], sum[2] = {0.0f, 0.0f};
+  // ---- new running max, rescale factor, fp16 weights ----
+  float mnew[2], alpha[2], sum[2] = {0.0f, 0.0f};
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
-    float v = -INFINITY;
+    const int h = g + 8 * hh;
+    float cm = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v = fmaxf(v, sm.red_max[w][g + 8 * hh]);
-    m[hh] = v;
+    for (int w = 0; w < 8; ++w) cm = fmaxf(cm, sm.red_max[w][h]);
+    const float mold = sm.m_run[h];
+    mnew[hh] = fmaxf(mold, cm);
+    alpha[hh] = (mold == -INFINITY) ? 0.0f : __expf(mold - mnew[hh]);
   }
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int j = 0; j < 4; j += 2) {
-      const int hh = j >> 1;
-      const float p0 = (m[hh] == -INFINITY) ? 0.0f : __expf(sacc[nt][j] - m[hh]);
-      const float p1 = (m[hh] == -INFINITY) ? 0.0f : __expf(sacc[nt][j + 1] - m[hh]);
-      const __half2 ph = __floats2half2_rn(p0, p1);
-      const float2 pr = __half22float2(ph);  // the sum uses the rounded fp16 weights
-      sum[hh] += pr.x + pr.y;
-      *reinterpret_cast<__half2*>(&sm.p[g + 8 * hh][16 * warp + 8 * nt + 2 * t]) = ph;
-    }
+  for (int j = 0; j < 4; j += 2) {
+    const int hh = j >> 1;
+    const float p0 = (mnew[hh] == -INFINITY) ? 0.0f : __expf(sv[j] - mnew[hh]);
+    const float p1 = (mnew[hh] == -INFINITY) ? 0.0f : __expf(sv[j + 1] - mnew[hh]);
+    const __half2 ph = __floats2half2_rn(p0, p1);
+    const float2 pr = __half22float2(ph);  // the sum uses the rounded fp16 weights
+    sum[hh] += pr.x + pr.y;
+    *reinterpret_cast<__half2*>(&sm.p[g + 8 * hh][8 * warp + 2 * t]) = ph;
+  }
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     sum[hh] += __shfl_xor_sync(0xffffffffu, sum[hh], 1);
@@ -315,13 +350,27 @@ __device__ __forceinline__ void attn_compute(const AttnArgs& a, AttnSmem& sm, fl
     sm.red_sum[warp][g + 8] = sum[1];
   }
   __syncthreads();
-
-  // ---- O = P V: warp w owns dims 64w .. 64w+63 (eight n-tiles of 8) ----
-  float oacc[8][4];
+  if (tid < kHq) {  // running state (read again only after the next chunk's barriers)
+    float l = 0.0f;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
+    for (int w = 0; w < 8; ++w) l += sm.red_sum[w][tid];
+    float cm = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) oacc[nt][j] = 0.0f;
+    for (int w = 0; w < 8; ++w) cm = fmaxf(cm, sm.red_max[w][tid]);
+    const float mold = sm.m_run[tid];
+    const float mn = fmaxf(mold, cm);
+    const float al = (mold == -INFINITY) ? 0.0f : __expf(mold - mn);
+    sm.l_run[tid] = sm.l_run[tid] * al + l;
+    sm.m_run[tid] = mn;
+  }
+  // ---- O = alpha O + P V over the chunk's keys ----
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) {
+    oacc[nt][0] *= alpha[0];
+    oacc[nt][1] *= alpha[0];
+    oacc[nt][2] *= alpha[1];
+    oacc[nt][3] *= alpha[1];
+  }
   {
     const int pr_ = (lane & 7) + 8 * ((lane >> 3) & 1);
     const int pc = 8 * (lane >> 4);
@@ -340,88 +389,100 @@ __device__ __forceinline__ void attn_compute(const AttnArgs& a, AttnSmem& sm, fl
       }
     }
   }
-  // ---- partial out (window values carry their fp32 scale) ----
+}
+
+// Writes the running part (O x kscale, max, sum) to partial slot `slot` and
+// resets the state.
+__device__ __forceinline__ void flush_part(const AttnArgs& a, AttnSmem& sm, float (&oacc)[8][4], int s, int nslots,
+                                           int slot, float kscale) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  float* part = a.partial + (int64_t(s) * nslots + slot) * kPartFloats;
+  __syncthreads();  // the running max / sum of the last chunk are written
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) {
     const int d = 64 * warp + 8 * nt + 2 * t;
     *reinterpret_cast<float2*>(&part[g * kD + d]) = make_float2(oacc[nt][0] * kscale, oacc[nt][1] * kscale);
     *reinterpret_cast<float2*>(&part[(g + 8) * kD + d]) = make_float2(oacc[nt][2] * kscale, oacc[nt][3] * kscale);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) oacc[nt][j] = 0.0f;
   }
+  __syncthreads();
   if (tid < kHq) {
-    float l = 0.0f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) l += sm.red_sum[w][tid];
-    float mm = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) mm = fmaxf(mm, sm.red_max[w][tid]);
-    part[kHq * kD + tid] = mm;
-    part[kHq * kD + kHq + tid] = l;
+    part[kHq * kD + tid] = sm.m_run[tid];
+    part[kHq * kD + kHq + tid] = sm.l_run[tid];
+    sm.m_run[tid] = -INFINITY;
+    sm.l_run[tid] = 0.0f;
   }
 }
 
-// Last-arriving CTA of a segment: combine the chunk partials in chunk order
+// An empty partial: max -inf, sum 0 (its O is never read).
+__device__ __forceinline__ void empty_part(const AttnArgs& a, int s, int nslots, int slot) {
+  float* part = a.partial + (int64_t(s) * nslots + slot) * kPartFloats;
+  if (threadIdx.x < kHq) {
+    part[kHq * kD + threadIdx.x] = -INFINITY;
+    part[kHq * kD + kHq + threadIdx.x] = 0.0f;
+  }
+}
+
+// Last-arriving CTA of a segment: combine the partials in slot order
 // (deterministic), write out / lse, and reset the segment's arrival counter.
-__device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm, int s, int nchunks) {
+__device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm, int s, int nctas, int nslots) {
   const int tid = threadIdx.x;
   // The barrier orders every thread's partial stores before thread 0's
   // release-acquire arrival (gpu scope); the last arrival therefore sees all
-  // chunks' partials.
+  // of the segment's partials.
   __syncthreads();
   if (tid == 0) {
     int old;
     asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(a.counters + s) : "memory");
-    sm.last = (old == nchunks - 1);
+    sm.last = (old == nctas - 1);
   }
   __syncthreads();
   if (!sm.last) return;
-  const float* base = a.partial + int64_t(s) * nchunks * kPartFloats;
+  const float* base = a.partial + int64_t(s) * nslots * kPartFloats;
   if (tid < kHq) {
-    constexpr int kMaxC = CSA2_MAX_TOPK / kChunk + 1;
-    float mc[kMaxC], lc[kMaxC];
+    float mc[kMaxSlots], lc[kMaxSlots];
     float M = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < kMaxC; ++c) {  // all loads first
-      mc[c] = c < nchunks ? __ldcg(base + c * kPartFloats + kHq * kD + tid) : -INFINITY;
-      lc[c] = c < nchunks ? __ldcg(base + c * kPartFloats + kHq * kD + kHq + tid) : 0.0f;
+    for (int c = 0; c < kMaxSlots; ++c) {  // all loads first
+      mc[c] = c < nslots ? __ldcg(base + c * kPartFloats + kHq * kD + tid) : -INFINITY;
+      lc[c] = c < nslots ? __ldcg(base + c * kPartFloats + kHq * kD + kHq + tid) : 0.0f;
     }
 #pragma unroll
-    for (int c = 0; c < kMaxC; ++c) M = fmaxf(M, mc[c]);
+    for (int c = 0; c < kMaxSlots; ++c) M = fmaxf(M, mc[c]);
     float L = 0.0f;
 #pragma unroll
-    for (int c = 0; c < kMaxC; ++c) {
+    for (int c = 0; c < kMaxSlots; ++c) {
       const float f = (mc[c] == -INFINITY) ? 0.0f : __expf(mc[c] - M);
-      if (c < nchunks) sm.fac[c][tid] = f;
+      if (c < nslots) sm.fac[c][tid] = f;
       L += lc[c] * f;
     }
-    for (int c = 0; c < nchunks; ++c) sm.fac[c][tid] = (M == -INFINITY) ? 0.0f : sm.fac[c][tid] / L;
+    for (int c = 0; c < nslots; ++c) sm.fac[c][tid] = (M == -INFINITY) ? 0.0f : sm.fac[c][tid] / L;
     if (a.lse) a.lse[int64_t(s) * kHq + tid] = (M == -INFINITY) ? -INFINITY : M + logf(L);
   }
   __syncthreads();
-  // 8 float4 per thread; two chunks' loads in flight at a time
+  // 8 float4 per thread; slots whose factor is 0 (empty or negligible) are
+  // skipped, so an empty slot's O is never read
   constexpr int kOV = kHq * kD / 4 / kAttnThreads;
   float4 o[kOV];
 #pragma unroll
   for (int m = 0; m < kOV; ++m) o[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c0 = 0; c0 < nchunks; c0 += 2) {
-    float4 v[2][kOV];
+  for (int c = 0; c < nslots; ++c) {
+    float4 v[kOV];
+    float f[kOV];
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
+    for (int m = 0; m < kOV; ++m) {
+      f[m] = sm.fac[c][(4 * (tid + m * kAttnThreads)) / kD];
+      v[m] = f[m] != 0.0f ? __ldcg(reinterpret_cast<const float4*>(base + c * kPartFloats) + tid + m * kAttnThreads)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
-      for (int m = 0; m < kOV; ++m)
-        v[u][m] = (c0 + u < nchunks)
-                      ? __ldcg(reinterpret_cast<const float4*>(base + (c0 + u) * kPartFloats) + tid + m * kAttnThreads)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      if (c0 + u >= nchunks) break;
-#pragma unroll
-      for (int m = 0; m < kOV; ++m) {
-        const float f = sm.fac[c0 + u][(4 * (tid + m * kAttnThreads)) / kD];
-        o[m].x = fmaf(v[u][m].x, f, o[m].x);
-        o[m].y = fmaf(v[u][m].y, f, o[m].y);
-        o[m].z = fmaf(v[u][m].z, f, o[m].z);
-        o[m].w = fmaf(v[u][m].w, f, o[m].w);
-      }
+    for (int m = 0; m < kOV; ++m) {
+      o[m].x = fmaf(v[m].x, f[m], o[m].x);
+      o[m].y = fmaf(v[m].y, f[m], o[m].y);
+      o[m].z = fmaf(v[m].z, f[m], o[m].z);
+      o[m].w = fmaf(v[m].w, f[m], o[m].w);
     }
   }
 #pragma unroll
@@ -429,62 +490,72 @@ __device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm,
   if (tid == 0) a.counters[s] = 0;
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnArgs a, int nchunks) {
+// grid = (R, S): CTA (r, s) takes chunks [r n / R, (r + 1) n / R) of segment s.
+__global__ void __launch_bounds__(kAttnThreads, 1) k_attn(AttnArgs a, int R) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
-  const int tid = threadIdx.x, r = tid & (kChunk - 1);
-  const int n_items = a.S * nchunks;
-  const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
-  const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
-  if (i0 >= i1) return;
-  // prologue: the first chunk's rows in flight, the second chunk's ids loaded
-  bool ok = issue_gather(a, sm, i0 / nchunks, i0 % nchunks, chunk_tpos(a, i0 / nchunks, i0 % nchunks, r));
-  sm100::cp_async_commit();
-  int32_t tnext = (i0 + 1 < i1) ? chunk_tpos(a, (i0 + 1) / nchunks, (i0 + 1) % nchunks, r) : -1;
-  int qseg = -1;
-  for (int it = i0; it < i1; ++it) {
-    const int s = it / nchunks, c = it - s * nchunks;
+  const int s = blockIdx.y, r = blockIdx.x, tid = threadIdx.x, row = tid & (kChunk - 1);
+  const int n = attn_main_chunks(a.k) + kWinChunks;
+  const int c0 = int(int64_t(n) * r / R), c1 = int(int64_t(n) * (r + 1) / R);
+  const int nslots = 2 * R;
+  float oacc[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) oacc[nt][j] = 0.0f;
+  if (tid < kHq) {
+    sm.m_run[tid] = -INFINITY;
+    sm.l_run[tid] = 0.0f;
+  }
+  bool ok = false;
+  int32_t tnext = -1;
+  if (c0 < c1) {
+    ok = issue_gather(a, sm, s, c0, chunk_tpos(a, s, c0, row));
+    sm100::cp_async_commit();
+    tnext = (c0 + 1 < c1) ? chunk_tpos(a, s, c0 + 1, row) : -1;
+  }
+  load_q(a, sm, s);  // overlaps the first gather
+  bool in_win = false, wrote_main = false;
+  float win_scale = 1.0f;
+  for (int c = c0; c < c1; ++c) {
     const ChunkSrc src = chunk_src(a, s, c);
-    if (s != qseg) {  // the previous chunk's products are done (barrier at its end)
-      load_q(a, sm, s);
-      qseg = s;
+    if (src.is_win && !in_win) {
+      if (c > c0) {  // this CTA's selected rows are done: their partial
+        flush_part(a, sm, oacc, s, nslots, 2 * r, 1.0f);
+        wrote_main = true;
+      }
+      in_win = true;
+      win_scale = src.kscale;
     }
     sm100::cp_async_wait<0>();
     __syncthreads();  // this chunk's rows (and Q) are in shared memory
     dequant_chunk(a, sm, src.is_win, ok);
     __syncthreads();  // keys ready; the staging buffer is free
-    if (it + 1 < i1) {
-      ok = issue_gather(a, sm, (it + 1) / nchunks, (it + 1) % nchunks, tnext);
+    if (c + 1 < c1) {
+      ok = issue_gather(a, sm, s, c + 1, tnext);
       sm100::cp_async_commit();
-      tnext = (it + 2 < i1) ? chunk_tpos(a, (it + 2) / nchunks, (it + 2) % nchunks, r) : -1;
+      tnext = (c + 2 < c1) ? chunk_tpos(a, s, c + 2, row) : -1;
     }
-    float* part = a.partial + (int64_t(s) * nchunks + c) * kPartFloats;
-    if (src.nkeys == 0) {
-      for (int i = tid; i < kHq * kD; i += kAttnThreads) part[i] = 0.0f;
-      if (tid < kHq) {
-        part[kHq * kD + tid] = -INFINITY;
-        part[kHq * kD + kHq + tid] = 0.0f;
-      }
-    } else {
-      attn_compute(a, sm, part, src.nkeys, src.kscale);
-    }
-    combine_if_last(a, sm, s, nchunks);
+    chunk_update(a, sm, oacc, src.nkeys, src.kscale);
   }
+  if (in_win) {
+    flush_part(a, sm, oacc, s, nslots, 2 * r + 1, win_scale);
+  } else if (c0 < c1) {
+    flush_part(a, sm, oacc, s, nslots, 2 * r, 1.0f);
+    wrote_main = true;
+  }
+  if (!wrote_main) empty_part(a, s, nslots, 2 * r);
+  if (!in_win) empty_part(a, s, nslots, 2 * r + 1);
   sm100::cp_async_wait<0>();
+  combine_if_last(a, sm, s, R, nslots);
 }
 
 void launch_attention(const AttnArgs& a, cudaStream_t st) {
   if (a.S == 0) return;
-  const int nchunks = attn_num_chunks(a.k);
+  const int R = attn_splits(a.S, a.k);
   const size_t smem = sizeof(AttnSmem);
-  cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  // one chunk per CTA while there are few chunks (the first gather of a
-  // persistent CTA would not be hidden); a persistent grid with prefetching
-  // beyond four chunks per SM
-  const int64_t n_items = int64_t(a.S) * nchunks;
-  const int sms = num_sms();
-  const int grid = int(n_items <= 4 * int64_t(sms) ? n_items : int64_t(sms));
-  k_attn_partial<<<grid, kAttnThreads, smem, st>>>(a, nchunks);
+  cudaFuncSetAttribute(k_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  k_attn<<<dim3(R, a.S), kAttnThreads, smem, st>>>(a, R);
 }
 
 }  // namespace csa2

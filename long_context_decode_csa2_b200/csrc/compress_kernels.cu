@@ -75,125 +75,170 @@ __device__ __forceinline__ uint32_t e2m1_code(float x, float inv_scale) {
 }
 
 constexpr int kCompWarps = 8;
+constexpr int kCompEntries = 16;                       // entries per CTA (two per warp)
+constexpr int kCompGroups = kCompWarps * 32 / kDi;     // projection: entry groups of the CTA (2)
+constexpr int kCompPerThread = kCompEntries / kCompGroups;  // entries per projecting thread (8)
 
-// grid = (ceil(max_new / 8), B), block = 256: one warp per new entry.
+// Writes one MXFP4 row of 32*V elements held V per lane (lane: elements
+// V*lane .. V*lane+V-1), blocks of 32 = 32/V lanes.
+template <int V>
+__device__ __forceinline__ void encode_row(const float (&x)[V], uint8_t* codes, uint8_t* scales, int lane) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+  for (int o = 1; o < 32 / V; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const int X = mx_block_exp(amax);
+  const float inv = pow2f_neg(X);
+  if constexpr (V == 16) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) lo |= e2m1_code(x[i], inv) << (4 * i);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hi |= e2m1_code(x[8 + i], inv) << (4 * i);
+    *reinterpret_cast<uint2*>(codes + 8 * lane) = make_uint2(lo, hi);
+  } else {
+    uint32_t v = 0;
+#pragma unroll
+    for (int i = 0; i < V; ++i) v |= e2m1_code(x[i], inv) << (4 * i);
+    *reinterpret_cast<uint16_t*>(codes + 2 * lane) = uint16_t(v);
+  }
+  if ((lane % (32 / V)) == 0) scales[lane / (32 / V)] = uint8_t(X + 127);
+}
+
+// grid = (ceil(max_new / 16), B), block = 256.  Each warp merges and encodes
+// two entries' main rows; the optional W_idx projection is shared by the CTA
+// (thread t: column t % 128 for eight entries, so every W_idx element read
+// feeds eight fma chains), and each warp then encodes its two indexer rows.
 __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
-  __shared__ float cbuf[kCompWarps][kD];
-  __shared__ float rbuf[kCompWarps][kDi];
+  __shared__ float cbuf[kCompEntries][kD];
+  __shared__ float rbuf[kCompEntries][kDi];
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t tok0 = a.tok_off[b];
   const int64_t ntok = a.tok_off[b + 1] - tok0;
   const int64_t nnew = ntok > 0 ? ntok / a.ratio : 0;
   if (blockIdx.x == 0 && threadIdx.x == 0) a.seq_len_out[b] = a.seq_len_in[b] + int32_t(nnew);
-  const int64_t j = int64_t(blockIdx.x) * kCompWarps + warp;
-  if (j >= nnew) return;
-  const int64_t row = a.seq_row_off[b] + a.seq_len_in[b] + j;
-  if (row < 0 || row >= a.mrows || row >= a.irows) {
-    if (lane == 0) set_status(a.status, CSA2_DEV_ROW_LAYOUT);
-    return;
-  }
-  const int64_t t0 = tok0 + a.ratio * j;  // first raw token of the entry
+  const int64_t j0 = int64_t(blockIdx.x) * kCompEntries;
+  if (j0 >= nnew) return;  // uniform for the whole CTA
 
-  double w0 = 1.0, w1 = 0.0;
-  if (a.ratio == 2) {
-    const double z0 = a.logits[t0], z1 = a.logits[t0 + 1];
-    const double m = fmax(z0, z1);
-    const double e0 = own_exp(__dsub_rn(z0, m)), e1 = own_exp(__dsub_rn(z1, m));
-    const double s = __dadd_rn(e0, e1);
-    w0 = __ddiv_rn(e0, s);
-    w1 = __ddiv_rn(e1, s);
-  }
-
-  // ---- main row: lane holds elements 16*lane .. 16*lane+15 ----
-  float c[16];
-  {
-    const uint4* p0 = reinterpret_cast<const uint4*>(a.raw + t0 * kD + 16 * lane);
-    const uint4 u0 = __ldg(p0), u1 = __ldg(p0 + 1);
-    const uint32_t x0w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    if (a.ratio == 2) {
-      const uint4* p1 = reinterpret_cast<const uint4*>(a.raw + (t0 + 1) * kD + 16 * lane);
-      const uint4 v0 = __ldg(p1), v1 = __ldg(p1 + 1);
-      const uint32_t x1w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  // ---- phase 1: merge + encode the main rows (entries warp, warp + 8) ----
+  bool ok[2];
+  int64_t rows[2], toks[2];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
-        const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
-        c[i] = __double2float_rn(__fma_rn(w0, x0, __dmul_rn(w1, x1)));
+  for (int u = 0; u < 2; ++u) {
+    const int e = warp + kCompWarps * u;
+    const int64_t j = j0 + e;
+    const int64_t row = a.seq_row_off[b] + a.seq_len_in[b] + j;
+    ok[u] = j < nnew;
+    if (ok[u] && (row < 0 || row >= a.mrows || row >= a.irows)) {
+      if (lane == 0) set_status(a.status, CSA2_DEV_ROW_LAYOUT);
+      ok[u] = false;
+    }
+    rows[u] = row;
+    toks[u] = tok0 + a.ratio * j;  // first raw token of the entry
+    float c[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) c[i] = 0.0f;
+    if (ok[u]) {
+      const int64_t t0 = toks[u];
+      double w0 = 1.0, w1 = 0.0;
+      if (a.ratio == 2) {
+        const double z0 = a.logits[t0], z1 = a.logits[t0 + 1];
+        const double m = fmax(z0, z1);
+        const double e0 = own_exp(__dsub_rn(z0, m)), e1 = own_exp(__dsub_rn(z1, m));
+        const double sum = __dadd_rn(e0, e1);
+        w0 = __ddiv_rn(e0, sum);
+        w1 = __ddiv_rn(e1, sum);
       }
-    } else {
+      // lane holds elements 16*lane .. 16*lane+15
+      const uint4* p0 = reinterpret_cast<const uint4*>(a.raw + t0 * kD + 16 * lane);
+      const uint4 u0 = __ldg(p0), u1 = __ldg(p0 + 1);
+      const uint32_t x0w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      if (a.ratio == 2) {
+        const uint4* p1 = reinterpret_cast<const uint4*>(a.raw + (t0 + 1) * kD + 16 * lane);
+        const uint4 v0 = __ldg(p1), v1 = __ldg(p1 + 1);
+        const uint32_t x1w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-      for (int i = 0; i < 16; ++i) c[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+        for (int i = 0; i < 16; ++i) {
+          const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+          const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
+          c[i] = __double2float_rn(__fma_rn(w0, x0, __dmul_rn(w1, x1)));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) c[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+      }
+      encode_row<16>(c, a.mcodes + row * kMainCodeBytes, a.mscales + row * kMainScaleBytes, lane);
+    }
+    if (a.w_idx) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) cbuf[e][16 * lane + i] = c[i];
     }
   }
-  {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(c[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    const int X = mx_block_exp(amax);
-    const float inv = pow2f_neg(X);
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) lo |= e2m1_code(c[i], inv) << (4 * i);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) hi |= e2m1_code(c[8 + i], inv) << (4 * i);
-    *reinterpret_cast<uint2*>(a.mcodes + row * kMainCodeBytes + 8 * lane) = make_uint2(lo, hi);
-    if ((lane & 1) == 0) a.mscales[row * kMainScaleBytes + lane / 2] = uint8_t(X + 127);
-  }
 
-  // ---- indexer row: 128 elements, lane holds 4*lane .. 4*lane+3 ----
-  float r[4];
+  // ---- phase 2: indexer rows r = W_idx^T c (fp64 chain over i = 0..511) ----
   if (a.w_idx) {
+    __syncthreads();
+    const int col = threadIdx.x % kDi, grp = threadIdx.x / kDi;
+    double acc[kCompPerThread];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) cbuf[warp][16 * lane + i] = c[i];
-    __syncwarp();
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int q = 0; q < kCompPerThread; ++q) acc[q] = 0.0;
+#pragma unroll 4
     for (int i = 0; i < kD; ++i) {
-      const double ci = cbuf[warp][i];
+      const double wi = double(__ldg(a.w_idx + i * kDi + col));
 #pragma unroll
-      for (int m = 0; m < 4; ++m) acc[m] = __fma_rn(ci, double(__ldg(a.w_idx + i * kDi + lane + 32 * m)), acc[m]);
+      for (int q = 0; q < kCompPerThread; ++q)
+        acc[q] = __fma_rn(double(cbuf[grp * kCompPerThread + q][i]), wi, acc[q]);
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) rbuf[warp][lane + 32 * m] = __double2float_rn(acc[m]);
-    __syncwarp();
-#pragma unroll
-    for (int i = 0; i < 4; ++i) r[i] = rbuf[warp][4 * lane + i];
-  } else {
-    const uint2 u = __ldg(reinterpret_cast<const uint2*>(a.idx_raw + t0 * kDi + 4 * lane));
-    const uint32_t x0w[2] = {u.x, u.y};
-    if (a.ratio == 2) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.idx_raw + (t0 + 1) * kDi + 4 * lane));
-      const uint32_t x1w[2] = {v.x, v.y};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
-        const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
-        r[i] = __double2float_rn(__fma_rn(w0, x0, __dmul_rn(w1, x1)));
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) r[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
-    }
+    for (int q = 0; q < kCompPerThread; ++q) rbuf[grp * kCompPerThread + q][col] = __double2float_rn(acc[q]);
+    __syncthreads();
   }
-  {
-    float amax = fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3])));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-    const int X = mx_block_exp(amax);
-    const float inv = pow2f_neg(X);
-    uint32_t v = 0;
+
+  // ---- phase 3: encode the indexer rows (lane holds 4*lane .. 4*lane+3) ----
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v |= e2m1_code(r[i], inv) << (4 * i);
-    *reinterpret_cast<uint16_t*>(a.icodes + row * kIdxCodeBytes + 2 * lane) = uint16_t(v);
-    if ((lane & 7) == 0) a.iscales[row * kIdxScaleBytes + lane / 8] = uint8_t(X + 127);
+  for (int u = 0; u < 2; ++u) {
+    if (!ok[u]) continue;
+    const int e = warp + kCompWarps * u;
+    const int64_t t0 = toks[u], row = rows[u];
+    float r[4];
+    if (a.w_idx) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r[i] = rbuf[e][4 * lane + i];
+    } else {
+      double w0 = 1.0, w1 = 0.0;
+      if (a.ratio == 2) {
+        const double z0 = a.logits[t0], z1 = a.logits[t0 + 1];
+        const double m = fmax(z0, z1);
+        const double e0 = own_exp(__dsub_rn(z0, m)), e1 = own_exp(__dsub_rn(z1, m));
+        const double sum = __dadd_rn(e0, e1);
+        w0 = __ddiv_rn(e0, sum);
+        w1 = __ddiv_rn(e1, sum);
+      }
+      const uint2 uu = __ldg(reinterpret_cast<const uint2*>(a.idx_raw + t0 * kDi + 4 * lane));
+      const uint32_t x0w[2] = {uu.x, uu.y};
+      if (a.ratio == 2) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.idx_raw + (t0 + 1) * kDi + 4 * lane));
+        const uint32_t x1w[2] = {v.x, v.y};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+          const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
+          r[i] = __double2float_rn(__fma_rn(w0, x0, __dmul_rn(w1, x1)));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+      }
+    }
+    encode_row<4>(r, a.icodes + row * kIdxCodeBytes, a.iscales + row * kIdxScaleBytes, lane);
   }
 }
 
 void launch_compress(const CompressArgs& a, cudaStream_t st) {
   if (a.B == 0) return;
-  const int64_t gx = a.max_new > 0 ? (a.max_new + kCompWarps - 1) / kCompWarps : 1;
+  const int64_t gx = a.max_new > 0 ? (a.max_new + kCompEntries - 1) / kCompEntries : 1;
   k_compress<<<dim3(static_cast<unsigned>(gx), a.B), kCompWarps * 32, 0, st>>>(a);
 }
 

@@ -105,6 +105,8 @@ struct SelShared {
   uint32_t warp_sums[32];
   uint32_t total;
   uint32_t digit, rem;
+  int sel_warp;         // find_bin: the warp whose bin range holds the threshold
+  uint32_t sel_before;  // and the count above that range
 };
 
 // Block-wide exclusive scan of one uint32 per thread; returns the exclusive
@@ -138,28 +140,71 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
 
 // Finds, among `nbins` bins of `hist` scanned from the top, the bin where the
 // running count reaches `need`; returns it in sh.digit with the count still
-// needed from it in sh.rem.  (Whole block; `hist` in shared memory.)
+// needed from it in sh.rem.  (Whole block; `hist` in shared memory.)  Large
+// histograms are read with consecutive lanes on consecutive bins (no bank
+// conflicts): every warp sums a contiguous range of bins, a scan of the warp
+// totals picks the range that holds the threshold, and that warp walks its
+// range 32 bins at a time.
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32_t need, SelShared& sh) {
   if (threadIdx.x == 0) {  // defined result even for an inconsistent histogram
     sh.digit = 0;
     sh.rem = need;
   }
-  const int per = (nbins + kSelThreads - 1) / kSelThreads;
-  // thread j owns bins [nbins - per*(j+1), nbins - per*j) (top bins first)
-  const int hi = nbins - per * int(threadIdx.x);
-  const int lo = max(0, hi - per);
-  uint32_t mine = 0;
-  for (int b = lo; b < hi; ++b) mine += hist[b];
-  const uint32_t before = block_exclusive_scan(mine, sh.warp_sums, &sh.total);
-  if (before < need && before + mine >= need) {
-    uint32_t cum = before;
-    for (int b = hi - 1; b >= lo; --b) {
-      if (cum + hist[b] >= need) {
-        sh.digit = uint32_t(b);
-        sh.rem = need - cum;
+  if (nbins <= kSelThreads) {
+    // thread j owns bin nbins - 1 - j (top bins first)
+    const int b = nbins - 1 - int(threadIdx.x);
+    const uint32_t mine = b >= 0 ? hist[b] : 0u;
+    const uint32_t before = block_exclusive_scan(mine, sh.warp_sums, &sh.total);
+    if (before < need && before + mine >= need) {
+      sh.digit = uint32_t(b);
+      sh.rem = need - before;
+    }
+    __syncthreads();
+    return;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per_warp = nbins / (kSelThreads / 32);  // a multiple of 32
+  const int whi = nbins - per_warp * warp;          // warp w: bins [whi - per_warp, whi)
+  uint32_t t = 0;
+  for (int b = whi - per_warp + lane; b < whi; b += 32) t += hist[b];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  __syncthreads();  // sh.warp_sums may still be read by the caller's previous step
+  if (lane == 0) sh.warp_sums[warp] = t;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t v = sh.warp_sums[lane];  // lane = warp index, top range first
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, x - v < need && x >= need);
+    if (lane == 0) sh.sel_warp = hit ? __ffs(hit) - 1 : -1;
+    if (hit && lane == __ffs(hit) - 1) sh.sel_before = x - v;
+  }
+  __syncthreads();
+  if (warp == sh.sel_warp) {
+    uint32_t cum = sh.sel_before;
+    for (int top = whi; top > whi - per_warp; top -= 32) {
+      const int b = top - 1 - lane;  // lane 0 holds the highest bin of the group
+      const uint32_t v = hist[b];
+      uint32_t x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      const uint32_t hit = __ballot_sync(0xffffffffu, cum + x >= need);
+      if (hit) {
+        if (lane == __ffs(hit) - 1) {
+          sh.digit = uint32_t(b);
+          sh.rem = need - (cum + x - v);
+        }
         break;
       }
-      cum += hist[b];
+      cum += __shfl_sync(0xffffffffu, x, 31);
     }
   }
   __syncthreads();

@@ -55,6 +55,8 @@ def _run_full(kc, ks, off, lengths, qc, qs, w, P, k, want_scores=False):
     ([5000, 777, 3, 0, 4096, 12345], 64, 64),
     ([20000, 1, 9, 600], 2048, 512),        # nb <= P for short sequences
     ([100000, 65536], 2048, 512),
+    # more than 16384 blocks: the pool is collected by several CTAs per sequence first
+    ([300001, 150000, 70, 140000], 2048, 512),
 ])
 def test_index_full_matches_oracle(lengths, P, k):
     rng = np.random.default_rng(sum(lengths) + P)

@@ -230,7 +230,7 @@ csa2_status csa2_sparse_attn_prefill(const uint16_t* q, const int32_t* q_pos, in
  * allocations, or a serving loop held to a fixed memory budget).  The pages
  * have no counterpart of this call; it is a deployment convenience.
  * Same arguments, results and accuracy as csa2_sparse_attn_decode, except:
- *   - no workspace: the scratch is a fixed 10,527,488-byte array of device
+ *   - no workspace: the scratch is a fixed 16,843,520-byte array of device
  *     memory inside this library, which every GPU that loads the library keeps
  *     until the process exits; the call allocates nothing;
  *   - limits: B <= 64 and k <= 512; larger problems return

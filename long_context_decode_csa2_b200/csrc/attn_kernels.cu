@@ -3,10 +3,10 @@
 // KV Cache Compression", section "三个方向一起压小缓存": 512 entries per layer,
 // MXFP4 main KV, FP8 window; section "后 20 层干脆共用一份 KV": 128-token window).
 //
-// Work split: a segment's keys are chunks of 64 rows (ceil(k/64) chunks of
-// selected rows, then two window chunks), and R CTAs share a segment, each
-// walking a contiguous run of its chunks (R = SMs / segments, at most 4, so
-// that small batches still fill the GPU in one wave).  A CTA loads Q once,
+// Work split: a segment's keys are chunks (ceil(k/64) chunks of 64 selected
+// rows, then four window chunks of 32 rows), and R CTAs share a segment, each
+// walking a contiguous run of its chunks (R = 2 x SMs / segments, at most 4:
+// two CTAs fit on an SM, and small batches still fill the GPU in one wave).  A CTA loads Q once,
 // keeps an online softmax (running max, sum and output per head) across its
 // chunks, and while it computes one chunk, cp.async brings the next chunk's
 // raw rows (272-byte MXFP4 rows or 512-byte E4M3 rows) into a staging
@@ -35,7 +35,8 @@ constexpr int kAttnThreads = 256;                  // 8 warps
 constexpr int kPartFloats = kHq * kD + 2 * kHq;    // O, then m, then l
 constexpr int kQS = kD + 8;                        // smem row stride (halves) of Q and K
 constexpr int kPS = kChunk + 8;                    // smem row stride (halves) of P
-constexpr int kWinChunks = kWin / kChunk;          // 2
+constexpr int kWinRows = 32;                       // window rows per chunk (small staging buffer)
+constexpr int kWinChunks = kWin / kWinRows;        // 4
 constexpr int kMaxSplits = 4;                      // CTAs per segment at most
 constexpr int kMaxSlots = 2 * kMaxSplits;          // partials per segment (main + window per CTA)
 constexpr int kRawMain = kMainCodeBytes + kMainScaleBytes;  // 272: codes then scales (row stride 68
@@ -47,8 +48,8 @@ __host__ __device__ inline int attn_main_chunks(int k) { return (k + kChunk - 1)
 int attn_num_chunks(int k) { return attn_main_chunks(k) + kWinChunks; }
 
 int attn_splits(int S, int k) {
-  const int sms = num_sms();
-  int r = S > 0 ? sms / S : 1;
+  const int slots = 2 * num_sms();  // two CTAs per SM
+  int r = S > 0 ? slots / S : 1;
   r = std::min(r, std::min(kMaxSplits, attn_num_chunks(k)));
   return std::max(r, 1);
 }
@@ -63,7 +64,7 @@ struct AttnSmem {
   __half p[kHq][kPS];
   union {
     uint8_t main[kChunk][kRawMain];
-    uint8_t win[kChunk][kRawWin];
+    uint8_t win[kWinRows][kRawWin];
   } raw;                                 // staged raw rows of the next chunk
   float red_max[8][kHq];
   float red_sum[8][kHq];
@@ -73,6 +74,8 @@ struct AttnSmem {
   float fac[kMaxSlots][kHq];
   int last;
 };
+
+static_assert(sizeof(AttnSmem) <= 112 * 1024, "two attention CTAs must fit on one SM");
 
 // Rows of chunk c of segment s: how many, where from, and the window scale.
 struct ChunkSrc {
@@ -92,7 +95,7 @@ __device__ __forceinline__ ChunkSrc chunk_src(const AttnArgs& a, int s, int c) {
     r.nkeys = min(kChunk, a.k - c * kChunk);
     return r;
   }
-  const int wc = c - nmain;  // window chunk 0 or 1
+  const int wc = c - nmain;  // window chunk 0 .. kWinChunks-1
   int nwin;
   const uint8_t* base;
   if (a.q_pos == nullptr) {
@@ -110,8 +113,8 @@ __device__ __forceinline__ ChunkSrc chunk_src(const AttnArgs& a, int s, int c) {
     r.kscale = a.raw_scale;
     base = a.raw_win + lo * kD;
   }
-  r.nkeys = max(0, min(kChunk, nwin - wc * kChunk));
-  r.win_base = base + int64_t(wc) * kChunk * kD;
+  r.nkeys = max(0, min(kWinRows, nwin - wc * kWinRows));
+  r.win_base = base + int64_t(wc) * kWinRows * kD;
   return r;
 }
 
@@ -147,7 +150,7 @@ __device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, in
 #pragma unroll
       for (int i = 0; i < kMainCodeBytes / 4 / 16; ++i) sm100::cp_async16(dst + 16 * i, cs + 16 * i);
       if (qt == 0) sm100::cp_async16(sm.raw.main[r] + kMainCodeBytes, a.mscales + row * kMainScaleBytes);
-    } else {
+    } else {  // r < nkeys <= kWinRows
       const uint8_t* ws = src.win_base + int64_t(r) * kD + qt * (kD / 4);
       uint8_t* dst = sm.raw.win[r] + qt * (kD / 4);
 #pragma unroll
@@ -491,7 +494,7 @@ __device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm,
 }
 
 // grid = (R, S): CTA (r, s) takes chunks [r n / R, (r + 1) n / R) of segment s.
-__global__ void __launch_bounds__(kAttnThreads, 1) k_attn(AttnArgs a, int R) {
+__global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
   const int s = blockIdx.y, r = blockIdx.x, tid = threadIdx.x, row = tid & (kChunk - 1);
@@ -555,6 +558,7 @@ void launch_attention(const AttnArgs& a, cudaStream_t st) {
   const int R = attn_splits(a.S, a.k);
   const size_t smem = sizeof(AttnSmem);
   cudaFuncSetAttribute(k_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaFuncSetAttribute(k_attn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   k_attn<<<dim3(R, a.S), kAttnThreads, smem, st>>>(a, R);
 }
 

@@ -111,8 +111,10 @@ __device__ __forceinline__ void encode_row(const float (&x)[V], uint8_t* codes, 
 // (thread t: column t % 128 for eight entries, so every W_idx element read
 // feeds eight fma chains), and each warp then encodes its two indexer rows.
 __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
-  __shared__ float cbuf[kCompEntries][kD];
-  __shared__ float rbuf[kCompEntries][kDi];
+  // merged rows, widened once for the projection; projected rows
+  extern __shared__ __align__(16) unsigned char csm[];
+  double (*cbuf)[kD] = reinterpret_cast<double (*)[kD]>(csm);
+  float (*rbuf)[kDi] = reinterpret_cast<float (*)[kDi]>(csm + sizeof(double) * kCompEntries * kD);
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t tok0 = a.tok_off[b];
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
     }
     if (a.w_idx) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) cbuf[e][16 * lane + i] = c[i];
+      for (int i = 0; i < 16; ++i) cbuf[e][16 * lane + i] = double(c[i]);
     }
   }
 
@@ -189,7 +191,7 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
       const double wi = double(__ldg(a.w_idx + i * kDi + col));
 #pragma unroll
       for (int q = 0; q < kCompPerThread; ++q)
-        acc[q] = __fma_rn(double(cbuf[grp * kCompPerThread + q][i]), wi, acc[q]);
+        acc[q] = __fma_rn(cbuf[grp * kCompPerThread + q][i], wi, acc[q]);
     }
 #pragma unroll
     for (int q = 0; q < kCompPerThread; ++q) rbuf[grp * kCompPerThread + q][col] = __double2float_rn(acc[q]);
@@ -239,7 +241,9 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
 void launch_compress(const CompressArgs& a, cudaStream_t st) {
   if (a.B == 0) return;
   const int64_t gx = a.max_new > 0 ? (a.max_new + kCompEntries - 1) / kCompEntries : 1;
-  k_compress<<<dim3(static_cast<unsigned>(gx), a.B), kCompWarps * 32, 0, st>>>(a);
+  const size_t smem = sizeof(double) * kCompEntries * kD + sizeof(float) * kCompEntries * kDi;
+  cudaFuncSetAttribute(k_compress, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  k_compress<<<dim3(static_cast<unsigned>(gx), a.B), kCompWarps * 32, smem, st>>>(a);
 }
 
 }  // namespace csa2

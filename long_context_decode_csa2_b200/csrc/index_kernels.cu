@@ -39,15 +39,21 @@ void launch_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entrie
 // (key 0 = absent) by (key desc, index asc) and writes their ids ascending.
 // Keys are read in chunks of 16384 (16 consecutive keys per thread, four
 // 16-byte loads), so every thread keeps 64 bytes in flight per chunk.
-//   * small n (<= 16384): one chunk; the keys stay in registers through 8-bit
-//     radix passes (shared-memory histograms) and the ordered output;
-//   * large n: pass A builds a 15-bit histogram and finds the threshold
-//     bucket; pass B collects, in index order, the ids of the keys above the
-//     bucket and the (low bits, id) of the keys inside it (<= 12288); the
-//     exact threshold comes from radix passes over those candidates in shared
-//     memory, and the two ordered lists are merged into the output without a
-//     third pass over the keys.  A bucket with more than 12288 keys falls
-//     back to global radix passes and an ordered output pass.
+//   * the kernel that wrote the keys may also have histogrammed them (a row
+//     per segment in the workspace: 15 bits for block keys, 12 bits for pool
+//     candidates); the selection then starts from that row and zeroes it;
+//   * small n (<= 16384): one chunk; the keys stay in registers through radix
+//     digits of up to 8 bits (shared-memory histograms) and the ordered
+//     output;
+//   * large n: pass A builds a 15-bit histogram (unless the producer's row is
+//     given) and finds the threshold bucket; pass B collects, in index order,
+//     the ids of the keys above the bucket and the (low bits, id) of the keys
+//     inside it (<= 12288) -- or takes those lists from k_pool_collect, which
+//     splits the pass over four CTAs per segment; the exact threshold comes
+//     from radix passes over the candidates in shared memory, and the two
+//     ordered lists are merged into the output without another pass over the
+//     keys.  A bucket with more than 12288 keys falls back to global radix
+//     passes and an ordered output pass.
 // Output rule: key > T, or key == T among the first `rem` equal keys in
 // index order; ids leave in ascending order.
 // ---------------------------------------------------------------------------
@@ -215,63 +221,6 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32
   __syncthreads();
 }
 
-// find_bin over a histogram row in global memory (read through L2), for any
-// block size; also leaves the row's total count in sh.total.
-__device__ __forceinline__ void find_bin_global(const uint32_t* __restrict__ gh, int nbins, uint32_t need,
-                                                SelShared& sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = int(blockDim.x >> 5);
-  if (threadIdx.x == 0) {
-    sh.digit = 0;
-    sh.rem = need;
-  }
-  const int per_warp = nbins / nwarps;  // a multiple of 32
-  const int whi = nbins - per_warp * warp;
-  uint32_t t = 0;
-  for (int b = whi - per_warp + lane; b < whi; b += 32) t += __ldcg(gh + b);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-  __syncthreads();
-  if (lane == 0) sh.warp_sums[warp] = t;
-  __syncthreads();
-  if (warp == 0) {
-    const uint32_t v = lane < nwarps ? sh.warp_sums[lane] : 0u;
-    uint32_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    const uint32_t hit = __ballot_sync(0xffffffffu, x - v < need && x >= need);
-    if (lane == 0) sh.sel_warp = hit ? __ffs(hit) - 1 : -1;
-    if (hit && lane == __ffs(hit) - 1) sh.sel_before = x - v;
-    if (lane == 31) sh.total = x;
-  }
-  __syncthreads();
-  if (warp == sh.sel_warp) {
-    uint32_t cum = sh.sel_before;
-    for (int top = whi; top > whi - per_warp; top -= 32) {
-      const int b = top - 1 - lane;
-      const uint32_t v = __ldcg(gh + b);
-      uint32_t x = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      const uint32_t hit = __ballot_sync(0xffffffffu, cum + x >= need);
-      if (hit) {
-        if (lane == __ffs(hit) - 1) {
-          sh.digit = uint32_t(b);
-          sh.rem = need - (cum + x - v);
-        }
-        break;
-      }
-      cum += __shfl_sync(0xffffffffu, x, 31);
-    }
-  }
-  __syncthreads();
-}
-
 // Adds one to hist[bin] for an active lane.  (Aggregating equal bins across
 // the warp with match.any first was measured slower than the plain atomics.)
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
@@ -381,7 +330,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
                                                         const int32_t* __restrict__ seg_eff, int P,
                                                         const int32_t* __restrict__ pool, int k,
                                                         int32_t* __restrict__ out, uint32_t* __restrict__ ghist,
-                                                        const uint32_t* __restrict__ splits) {
+                                                        const uint32_t* __restrict__ splits,
+                                                        const uint32_t* __restrict__ thr) {
   extern __shared__ __align__(16) uint32_t dsm[];
   __shared__ SelShared sh;
   const int s = blockIdx.x;
@@ -487,7 +437,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   // ---- large n, pass A: 15-bit histogram of the present keys ----
   uint32_t* hist = dsm;
   uint32_t present = 0;
-  if (ghist) {
+  if (thr) {
+    // k_pool_threshold already read (and zeroed) the producer's row
+    if (tid == 0) present = __ldcg(thr + 4 * int64_t(s));
+  } else if (ghist) {
     present = take_hist<kHist1Bins>(ghist + int64_t(s) * kHist1Bins, hist);
   } else {
     for (int i = tid; i < kHist1Bins; i += kSelThreads) hist[i] = 0;
@@ -510,7 +463,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   const uint32_t total = sh.total;
   const bool all = total <= uint32_t(k);
   uint32_t b1 = 0, need = 0, cnt = 0;
-  if (!all) {
+  if (thr) {
+    b1 = __ldcg(thr + 4 * int64_t(s) + 1);
+    need = __ldcg(thr + 4 * int64_t(s) + 2);
+    cnt = __ldcg(thr + 4 * int64_t(s) + 3);
+  } else if (!all) {
     find_bin(hist, kHist1Bins, uint32_t(k), sh);
     b1 = sh.digit;
     need = sh.rem;
@@ -699,14 +656,41 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   }
 }
 
-// Pool select, first half: kPoolSplits CTAs per segment each collect, for
-// their contiguous range of block keys, the ids above the threshold bucket
-// and the bucket's (low bits, id) pairs in index order (the bucket comes
-// from the producer's histogram, read through L2).  k_select then merges the
-// short lists instead of streaming every key once more.
+// Pool select over block keys in three short kernels:
+//   k_pool_threshold (one CTA per segment): the producer's histogram row into
+//     shared memory (zeroing it), the threshold bucket -> thr[s] = (total,
+//     bucket, count still needed from it, bucket size);
+//   k_pool_collect (kPoolSplits CTAs per segment): for a contiguous range of
+//     block keys, the ids above the bucket and the bucket's (low bits, id)
+//     pairs, in index order;
+//   k_select: the exact threshold inside the bucket and the ordered merge of
+//     the short lists (no further pass over the keys).
+__global__ void __launch_bounds__(kSelThreads, 1) k_pool_threshold(uint32_t* __restrict__ ghist, int k,
+                                                                    uint32_t* __restrict__ thr) {
+  extern __shared__ __align__(16) uint32_t dsm[];
+  __shared__ SelShared sh;
+  const int s = blockIdx.x;
+  const uint32_t present = take_hist<kHist1Bins>(ghist + int64_t(s) * kHist1Bins, dsm);
+  block_exclusive_scan(present, sh.warp_sums, &sh.total);
+  const uint32_t total = sh.total;
+  uint32_t b1 = 0, need = 0, cnt = 0;
+  if (total > uint32_t(k)) {
+    find_bin(dsm, kHist1Bins, uint32_t(k), sh);
+    b1 = sh.digit;
+    need = sh.rem;
+    cnt = dsm[b1];
+  }
+  if (threadIdx.x == 0) {
+    thr[4 * int64_t(s)] = total;
+    thr[4 * int64_t(s) + 1] = b1;
+    thr[4 * int64_t(s) + 2] = need;
+    thr[4 * int64_t(s) + 3] = cnt;
+  }
+}
+
 __global__ void __launch_bounds__(kColThreads, 2) k_pool_collect(const uint32_t* __restrict__ bkeys, int64_t stride,
                                                                   const int32_t* __restrict__ seg_eff, int k,
-                                                                  const uint32_t* __restrict__ ghist,
+                                                                  const uint32_t* __restrict__ thr,
                                                                   uint32_t* __restrict__ splits) {
   __shared__ SelShared sh;
   const int s = blockIdx.y, r = blockIdx.x, tid = threadIdx.x;
@@ -717,9 +701,8 @@ __global__ void __launch_bounds__(kColThreads, 2) k_pool_collect(const uint32_t*
   uint32_t* A = rs + 4;
   uint32_t* Clow = A + kSelMaxK;
   uint32_t* Cidx = Clow + kSplitCandCap;
-  find_bin_global(ghist + int64_t(s) * kHist1Bins, kHist1Bins, uint32_t(k), sh);
-  const bool all = sh.total <= uint32_t(k);
-  const uint32_t b1 = sh.digit;
+  const bool all = __ldcg(thr + 4 * int64_t(s)) <= uint32_t(k);
+  const uint32_t b1 = __ldcg(thr + 4 * int64_t(s) + 1);
   const int64_t base = int64_t(s) * stride;
   uint32_t run_a = 0, run_c = 0;
   if (cl < ch) {
@@ -776,22 +759,24 @@ __global__ void __launch_bounds__(kColThreads, 2) k_pool_collect(const uint32_t*
   }
 }
 
-size_t pool_split_bytes(int S) { return size_t(S) * kPoolSplits * kSplitWords * sizeof(uint32_t); }
+size_t pool_split_bytes(int S) { return size_t(S) * (kPoolSplits * kSplitWords + 4) * sizeof(uint32_t); }
 
 template <int KIND>
 void launch_select_kind(const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P, const int32_t* pool,
-                        int k, int32_t* out, uint32_t* hist, const uint32_t* splits, int64_t n_bound,
-                        cudaStream_t st) {
+                        int k, int32_t* out, uint32_t* hist, const uint32_t* splits, const uint32_t* thr,
+                        int64_t n_bound, cudaStream_t st) {
   if (n_bound <= kSelSmallMax) {
     constexpr int NB = (KIND == kSelPoolCand) ? kCandHistBins : kHist1Bins;
     const size_t smem = (hist ? NB + 256 : 256) * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int((NB + 256) * sizeof(uint32_t)));
-    k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, nullptr);
+    k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, nullptr,
+                                                      nullptr);
   } else {
     const size_t smem = kSelLargeWords * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    k_select<KIND, false><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, splits);
+    k_select<KIND, false><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, splits,
+                                                       thr);
   }
 }
 
@@ -802,18 +787,24 @@ void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int
   switch (kind) {
     case kSelBlockKeys:
       if (splits && hist && in_stride > kSelSmallMax) {
+        uint32_t* thr = splits + size_t(S) * kPoolSplits * kSplitWords;
+        const size_t smem = kHist1Bins * sizeof(uint32_t);
+        cudaFuncSetAttribute(k_pool_threshold, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        k_pool_threshold<<<S, kSelThreads, smem, st>>>(hist, k, thr);
         k_pool_collect<<<dim3(kPoolSplits, S), kColThreads, 0, st>>>(static_cast<const uint32_t*>(in), in_stride,
-                                                                     seg_eff, k, hist, splits);
+                                                                     seg_eff, k, thr, splits);
+        launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, nullptr, splits, thr,
+                                          in_stride, st);
       } else {
-        splits = nullptr;
+        launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, hist, nullptr, nullptr,
+                                          in_stride, st);
       }
-      launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, hist, splits, in_stride, st);
       break;
     case kSelScores:
-      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, hist, nullptr, in_stride, st);
+      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, hist, nullptr, nullptr, in_stride, st);
       break;
     case kSelPoolCand:
-      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, nullptr, in_stride, st);
+      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, nullptr, nullptr, in_stride, st);
       break;
   }
 }

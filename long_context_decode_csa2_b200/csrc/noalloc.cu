@@ -23,12 +23,14 @@ constexpr int kNoAllocMaxTopk = 512;
 constexpr size_t kNoAllocStatusBytes = 256;                       // device status word
 constexpr size_t kNoAllocSeqBytes = 256;                          // reserved (layout unchanged)
 constexpr size_t kNoAllocCounterBytes = 256;                      // 64 arrival counters (self-resetting)
+constexpr size_t kNoAllocSlots = 8;                               // partials per sequence: up to 4 CTAs x
+                                                                  // (selected rows, window)
 constexpr size_t kNoAllocPartialBytes =                           // split-KV partials
-    size_t(kNoAllocMaxSeqs) * (kNoAllocMaxTopk / 128 + 1) * (kHq * kD + 2 * kHq) * sizeof(float);
+    size_t(kNoAllocMaxSeqs) * kNoAllocSlots * (kHq * kD + 2 * kHq) * sizeof(float);
 constexpr size_t kNoAllocScratchBytes =
     kNoAllocStatusBytes + kNoAllocSeqBytes + kNoAllocCounterBytes + kNoAllocPartialBytes;
 
-// The scratch: 10,527,488 bytes of device memory that every GPU which loads
+// The scratch: 16,843,520 bytes of device memory that every GPU which loads
 // this library keeps until the process exits.  All calls on a device share it
 // and it keeps whatever the last call left in it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];

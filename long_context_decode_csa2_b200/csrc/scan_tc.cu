@@ -10,12 +10,15 @@
 // One persistent CTA per SM walks a contiguous range of work items; an item
 // is 512 positions of one segment: 512 consecutive rows (scan) or the rows of
 // 64 pool blocks (pool scoring).  Per item:
-//   * warp 0 (producer) loads the 64-byte code rows with TMA tile copies
-//     (64-byte swizzle; two 256-row boxes for the scan, sixty-four 8-row boxes
-//     gathered by the 32 lanes for the pool), the 4-byte E8M0 scale words
-//     with bulk copies, and writes the item's B operand: the segment's
-//     indexer query laid out "one 32-element block per output column" (column
-//     4h+b holds head h's block b, zeros elsewhere);
+//   * the producer loads the 64-byte code rows and the 4-byte E8M0 scale
+//     words.  Scan: warp 0 issues two TMA tile copies of 256 rows (64-byte
+//     swizzle) and one bulk copy of the scale words.  Pool: four producer
+//     warps each gather 16 of the item's 64 blocks with cp.async (one warp
+//     instruction per 512-byte block, the swizzle applied to the
+//     destination) from the segment's pool ids held in shared memory.
+//     Warp 0 also writes the item's B operand: the segment's indexer query
+//     laid out "one 32-element block per output column" (column 4h+b holds
+//     head h's block b, zeros elsewhere);
 //   * warp 1 issues eight tcgen05.mma kind::mxf4 (M=128 positions, N=16,
 //     K=64) with every block scale = 1: each accumulator is D/4 for an exact
 //     integer |D| <= 4608, i.e. exact in fp32;
@@ -24,7 +27,8 @@
 //     (fp32 when the block exponents are close, else the same fp64 sum as the
 //     definition), combine the heads with the fp32 fma chain and emit rank
 //     keys: the maximum of every 8 positions (scan) or one key per candidate
-//     (pool; 0 for absent candidates).
+//     (pool; 0 for absent candidates), and add each key to its sequence's
+//     histogram row for the selection that follows.
 // Stages are recycled through mbarriers (smem ring of 4 for the scan, 6 for
 // the pool gather; TMEM ring of 3).
 // Every wait is time-bounded; on a timeout the kernel sets CSA2_DEV_TIMEOUT,

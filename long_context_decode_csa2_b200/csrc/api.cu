@@ -49,7 +49,6 @@ struct IndexFullWs {
   uint32_t* ckeys;
   float* scores;
   uint32_t* hist;  // [B][kSelHistBins] (block keys, then candidates), zero between calls
-  uint32_t* splits;  // pool candidates collected per (sequence, collect CTA)
   size_t bytes;
 };
 
@@ -64,7 +63,6 @@ IndexFullWs index_full_ws(void* ws, int B, int max_len, int P, int k, bool need_
   w.ckeys = (P >= k) ? c.take<uint32_t>(size_t(B) * P * kBlk) : nullptr;
   w.scores = need_scores ? c.take<float>(size_t(B) * max_len) : nullptr;
   w.hist = c.take<uint32_t>(size_t(B) * kSelHistBins);
-  w.splits = c.take<uint32_t>(pool_split_bytes(B) / sizeof(uint32_t));
   w.bytes = c.used;
   return w;
 }
@@ -132,8 +130,7 @@ csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, cons
   const csa2_status rc = launch_scan_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, ws.tile_start, B, q_codes, q_scales,
                                         w, ws.bkeys, nb, scores, max_len, ws.hist, ws.status, st);
   if (rc != CSA2_OK) return rc;
-  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, ws.hist, st,
-                ws.splits);
+  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, ws.hist, st);
   if (pool_blocks >= k) {
     // Every Top-k position's block ranks within the first k blocks, so the
     // Top-k over the pool equals the Top-k over all positions.

@@ -48,12 +48,11 @@ void launch_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entrie
 //   * large n: pass A builds a 15-bit histogram (unless the producer's row is
 //     given) and finds the threshold bucket; pass B collects, in index order,
 //     the ids of the keys above the bucket and the (low bits, id) of the keys
-//     inside it (<= 12288) -- or takes those lists from k_pool_collect, which
-//     splits the pass over four CTAs per segment; the exact threshold comes
-//     from radix passes over the candidates in shared memory, and the two
-//     ordered lists are merged into the output without another pass over the
-//     keys.  A bucket with more than 12288 keys falls back to global radix
-//     passes and an ordered output pass.
+//     inside it (<= 12288); the exact threshold comes from radix passes over
+//     those candidates in shared memory, and the two ordered lists are merged
+//     into the output without another pass over the keys.  A bucket with more
+//     than 12288 keys falls back to global radix passes and an ordered output
+//     pass.
 // Output rule: key > T, or key == T among the first `rem` equal keys in
 // index order; ids leave in ascending order.
 // ---------------------------------------------------------------------------
@@ -66,11 +65,6 @@ constexpr int kHist1Bins = kSelHistBins;
 constexpr int kLowBits = 32 - kHist1Bits;  // 17
 constexpr uint32_t kLowMask = (1u << kLowBits) - 1u;
 constexpr int kCandCap = 12288;
-constexpr int kPoolSplits = 4;                       // k_pool_collect CTAs per segment
-constexpr int kColThreads = 512;
-constexpr int kColChunk = kColThreads * 16;          // keys per collect chunk
-constexpr int kSplitCandCap = 4096;                  // bucket entries per collect CTA
-constexpr int kSplitWords = 4 + CSA2_MAX_TOPK + 2 * kSplitCandCap;  // counts, ids above, bucket (low, id)
 constexpr int kSelMaxK = CSA2_MAX_TOPK;
 // large-path shared memory: the histogram, later reused for the lists
 constexpr int kSelLargeWords = kHist1Bins;
@@ -133,7 +127,7 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   if (lane == 31) warp_sums[wid] = x;
   __syncthreads();
   if (wid == 0) {
-    const uint32_t ws = (lane < int(blockDim.x >> 5)) ? warp_sums[lane] : 0u;
+    const uint32_t ws = (lane < (kSelThreads / 32)) ? warp_sums[lane] : 0u;
     uint32_t z = ws;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -329,9 +323,7 @@ template <int KIND, bool SMALL>
 __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restrict__ in, int64_t in_stride,
                                                         const int32_t* __restrict__ seg_eff, int P,
                                                         const int32_t* __restrict__ pool, int k,
-                                                        int32_t* __restrict__ out, uint32_t* __restrict__ ghist,
-                                                        const uint32_t* __restrict__ splits,
-                                                        const uint32_t* __restrict__ thr) {
+                                                        int32_t* __restrict__ out, uint32_t* __restrict__ ghist) {
   extern __shared__ __align__(16) uint32_t dsm[];
   __shared__ SelShared sh;
   const int s = blockIdx.x;
@@ -437,10 +429,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   // ---- large n, pass A: 15-bit histogram of the present keys ----
   uint32_t* hist = dsm;
   uint32_t present = 0;
-  if (thr) {
-    // k_pool_threshold already read (and zeroed) the producer's row
-    if (tid == 0) present = __ldcg(thr + 4 * int64_t(s));
-  } else if (ghist) {
+  if (ghist) {
     present = take_hist<kHist1Bins>(ghist + int64_t(s) * kHist1Bins, hist);
   } else {
     for (int i = tid; i < kHist1Bins; i += kSelThreads) hist[i] = 0;
@@ -463,11 +452,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   const uint32_t total = sh.total;
   const bool all = total <= uint32_t(k);
   uint32_t b1 = 0, need = 0, cnt = 0;
-  if (thr) {
-    b1 = __ldcg(thr + 4 * int64_t(s) + 1);
-    need = __ldcg(thr + 4 * int64_t(s) + 2);
-    cnt = __ldcg(thr + 4 * int64_t(s) + 3);
-  } else if (!all) {
+  if (!all) {
     find_bin(hist, kHist1Bins, uint32_t(k), sh);
     b1 = sh.digit;
     need = sh.rem;
@@ -511,37 +496,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   uint32_t* h2 = Cidx + kCandCap;        // [512]
   uint32_t* Csel = h2 + 512;             // [kSelMaxK] selected bucket ids
   uint32_t run_a = 0, run_c = 0;
-  // the lists may already be collected by k_pool_collect (several CTAs per
-  // segment); they are used unless one of them overflowed
-  bool collected = false;
-  if (splits) {
-    const uint32_t* sp = splits + int64_t(s) * kPoolSplits * kSplitWords;
-    uint32_t ta = 0, tc = 0, bad = 0;
-#pragma unroll
-    for (int r = 0; r < kPoolSplits; ++r) {
-      ta += __ldcg(sp + r * kSplitWords);
-      tc += __ldcg(sp + r * kSplitWords + 1);
-      bad |= __ldcg(sp + r * kSplitWords + 2);
-    }
-    collected = bad == 0u && ta <= uint32_t(kSelMaxK) && tc <= uint32_t(kCandCap);
-    if (collected) {
-      uint32_t oa = 0, oc = 0;
-      for (int r = 0; r < kPoolSplits; ++r) {
-        const uint32_t* rs = sp + r * kSplitWords;
-        const uint32_t na = __ldcg(rs), nc = __ldcg(rs + 1);
-        for (uint32_t i = tid; i < na; i += kSelThreads) A[oa + i] = __ldcg(rs + 4 + i);
-        for (uint32_t i = tid; i < nc; i += kSelThreads) {
-          Clow[oc + i] = __ldcg(rs + 4 + kSelMaxK + i);
-          Cidx[oc + i] = __ldcg(rs + 4 + kSelMaxK + kSplitCandCap + i);
-        }
-        oa += na;
-        oc += nc;
-      }
-      run_a = oa;
-      run_c = oc;
-    }
-  }
-  if (!collected) {
+  {
     uint32_t kk[kSelPer], nx[kSelPer];
     load_keys<KIND>(in, base, int64_t(tid) * kSelPer, n, kk);
     for (int64_t c0 = 0; c0 < n; c0 += kSelChunk) {
@@ -656,155 +611,35 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   }
 }
 
-// Pool select over block keys in three short kernels:
-//   k_pool_threshold (one CTA per segment): the producer's histogram row into
-//     shared memory (zeroing it), the threshold bucket -> thr[s] = (total,
-//     bucket, count still needed from it, bucket size);
-//   k_pool_collect (kPoolSplits CTAs per segment): for a contiguous range of
-//     block keys, the ids above the bucket and the bucket's (low bits, id)
-//     pairs, in index order;
-//   k_select: the exact threshold inside the bucket and the ordered merge of
-//     the short lists (no further pass over the keys).
-__global__ void __launch_bounds__(kSelThreads, 1) k_pool_threshold(uint32_t* __restrict__ ghist, int k,
-                                                                    uint32_t* __restrict__ thr) {
-  extern __shared__ __align__(16) uint32_t dsm[];
-  __shared__ SelShared sh;
-  const int s = blockIdx.x;
-  const uint32_t present = take_hist<kHist1Bins>(ghist + int64_t(s) * kHist1Bins, dsm);
-  block_exclusive_scan(present, sh.warp_sums, &sh.total);
-  const uint32_t total = sh.total;
-  uint32_t b1 = 0, need = 0, cnt = 0;
-  if (total > uint32_t(k)) {
-    find_bin(dsm, kHist1Bins, uint32_t(k), sh);
-    b1 = sh.digit;
-    need = sh.rem;
-    cnt = dsm[b1];
-  }
-  if (threadIdx.x == 0) {
-    thr[4 * int64_t(s)] = total;
-    thr[4 * int64_t(s) + 1] = b1;
-    thr[4 * int64_t(s) + 2] = need;
-    thr[4 * int64_t(s) + 3] = cnt;
-  }
-}
-
-__global__ void __launch_bounds__(kColThreads, 2) k_pool_collect(const uint32_t* __restrict__ bkeys, int64_t stride,
-                                                                  const int32_t* __restrict__ seg_eff, int k,
-                                                                  const uint32_t* __restrict__ thr,
-                                                                  uint32_t* __restrict__ splits) {
-  __shared__ SelShared sh;
-  const int s = blockIdx.y, r = blockIdx.x, tid = threadIdx.x;
-  const int64_t n = (int64_t(seg_eff[s]) + kBlk - 1) / kBlk;
-  const int64_t nchunks = (n + kColChunk - 1) / kColChunk;
-  const int64_t cl = nchunks * r / kPoolSplits, ch = nchunks * (r + 1) / kPoolSplits;
-  uint32_t* rs = splits + (int64_t(s) * kPoolSplits + r) * kSplitWords;
-  uint32_t* A = rs + 4;
-  uint32_t* Clow = A + kSelMaxK;
-  uint32_t* Cidx = Clow + kSplitCandCap;
-  const bool all = __ldcg(thr + 4 * int64_t(s)) <= uint32_t(k);
-  const uint32_t b1 = __ldcg(thr + 4 * int64_t(s) + 1);
-  const int64_t base = int64_t(s) * stride;
-  uint32_t run_a = 0, run_c = 0;
-  if (cl < ch) {
-    uint32_t kk[kSelPer], nx[kSelPer];
-    load_keys<kSelBlockKeys>(bkeys, base, cl * kColChunk + int64_t(tid) * kSelPer, n, kk);
-    for (int64_t c = cl; c < ch; ++c) {
-      const int64_t c0 = c * kColChunk;
-      if (c + 1 < ch) load_keys<kSelBlockKeys>(bkeys, base, c0 + kColChunk + int64_t(tid) * kSelPer, n, nx);
-      uint32_t mx = 0;
-#pragma unroll
-      for (int e = 0; e < kSelPer; ++e) mx = max(mx, kk[e]);
-      const bool hot = mx != 0u && (all || (mx >> kLowBits) >= b1);
-      uint32_t na = 0, nc = 0;
-      if (hot) {
-#pragma unroll
-        for (int e = 0; e < kSelPer; ++e) {
-          const uint32_t key = kk[e], hi = key >> kLowBits;
-          if (key != 0u) {
-            if (all || hi > b1) ++na;
-            else if (hi == b1) ++nc;
-          }
-        }
-      }
-      const uint32_t ex = block_exclusive_scan((na << 16) | nc, sh.warp_sums, &sh.total);
-      const uint32_t tot = sh.total;
-      uint32_t a = run_a + (ex >> 16), cc = run_c + (ex & 0xFFFFu);
-      const uint32_t i0 = uint32_t(c0) + uint32_t(tid) * kSelPer;
-#pragma unroll
-      for (int e = 0; e < kSelPer && hot; ++e) {
-        const uint32_t key = kk[e], hi = key >> kLowBits;
-        if (key != 0u) {
-          if (all || hi > b1) {
-            if (a < uint32_t(kSelMaxK)) A[a] = i0 + e;
-            ++a;
-          } else if (hi == b1) {
-            if (cc < uint32_t(kSplitCandCap)) {
-              Clow[cc] = key & kLowMask;
-              Cidx[cc] = i0 + e;
-            }
-            ++cc;
-          }
-        }
-      }
-      run_a += tot >> 16;
-      run_c += tot & 0xFFFFu;
-#pragma unroll
-      for (int e = 0; e < kSelPer; ++e) kk[e] = nx[e];
-    }
-  }
-  if (tid == 0) {
-    rs[0] = min(run_a, uint32_t(kSelMaxK));
-    rs[1] = min(run_c, uint32_t(kSplitCandCap));
-    rs[2] = (run_a > uint32_t(kSelMaxK) || run_c > uint32_t(kSplitCandCap)) ? 1u : 0u;
-  }
-}
-
-size_t pool_split_bytes(int S) { return size_t(S) * (kPoolSplits * kSplitWords + 4) * sizeof(uint32_t); }
-
 template <int KIND>
 void launch_select_kind(const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P, const int32_t* pool,
-                        int k, int32_t* out, uint32_t* hist, const uint32_t* splits, const uint32_t* thr,
-                        int64_t n_bound, cudaStream_t st) {
+                        int k, int32_t* out, uint32_t* hist, int64_t n_bound, cudaStream_t st) {
   if (n_bound <= kSelSmallMax) {
     constexpr int NB = (KIND == kSelPoolCand) ? kCandHistBins : kHist1Bins;
     const size_t smem = (hist ? NB + 256 : 256) * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int((NB + 256) * sizeof(uint32_t)));
-    k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, nullptr,
-                                                      nullptr);
+    k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist);
   } else {
     const size_t smem = kSelLargeWords * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    k_select<KIND, false><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, splits,
-                                                       thr);
+    k_select<KIND, false><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist);
   }
 }
 
 void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P,
-                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st, uint32_t* splits) {
+                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st) {
   if (S == 0) return;
   // n per segment is at most the row stride of the input
   switch (kind) {
     case kSelBlockKeys:
-      if (splits && hist && in_stride > kSelSmallMax) {
-        uint32_t* thr = splits + size_t(S) * kPoolSplits * kSplitWords;
-        const size_t smem = kHist1Bins * sizeof(uint32_t);
-        cudaFuncSetAttribute(k_pool_threshold, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        k_pool_threshold<<<S, kSelThreads, smem, st>>>(hist, k, thr);
-        k_pool_collect<<<dim3(kPoolSplits, S), kColThreads, 0, st>>>(static_cast<const uint32_t*>(in), in_stride,
-                                                                     seg_eff, k, thr, splits);
-        launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, nullptr, splits, thr,
-                                          in_stride, st);
-      } else {
-        launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, hist, nullptr, nullptr,
-                                          in_stride, st);
-      }
+      launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
       break;
     case kSelScores:
-      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, hist, nullptr, nullptr, in_stride, st);
+      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
       break;
     case kSelPoolCand:
-      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, nullptr, nullptr, in_stride, st);
+      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
       break;
   }
 }

@@ -96,12 +96,8 @@ enum SelectKind : int {
 };
 // `hist` (or null): the keys' histogram rows, zeroed on return: [S][kSelHistBins]
 // for block keys, [S][kCandHistBins] for pool candidates.
-// `splits` (block keys only, or null): scratch of pool_split_bytes(S) for
-// collecting the pool candidates with several CTAs per segment first.
 void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P,
-                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st,
-                   uint32_t* splits = nullptr);
-size_t pool_split_bytes(int S);
+                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st);
 
 // Attention partials + combine.
 struct AttnArgs {

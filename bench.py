@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling captures)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager steps instead of replays of one captured CUDA graph")
     ap.add_argument("--sequential", action="store_true",
                     help="issue every call on one stream (isolated per-call times) instead of the concurrent tail")
     ap.add_argument("--context", type=int, default=0,
@@ -170,12 +172,13 @@ def time_oracle(wl, samples, nthreads, jobs=None):
 
 # ----------------------------------------------------------------------------
 
-def decode_config(wl, l2_bytes, sequential):
+def decode_config(wl, l2_bytes, sequential, graph=True):
     """The `config` object of a decode line (both arms)."""
     return {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len, "layers": wl.pattern,
             "pool_blocks": wl.P, "topk": wl.k, "window": 128,
             "l2": "no flush: inputs larger than L2 (%.2f GB read per step)" % (l2_bytes / 1e9),
-            "schedule": "sequential" if sequential else "concurrent tail (side streams)"}
+            "schedule": ("sequential" if sequential else "concurrent tail (side streams)")
+                        + (", one CUDA graph per step" if graph else "")}
 
 
 def rank_workload(wl, rank):
@@ -293,6 +296,14 @@ def run_ours(args):
     if step.device_flags():
         raise RuntimeError("device status flags set during warm-up")
 
+    # the timed steps replay one captured CUDA graph of the whole step (the
+    # default); the per-call times come from a separate eager pass
+    graph = None
+    if not args.no_graph:
+        graph = step.capture(caches, off_d, len_d, layers_dev)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -301,12 +312,19 @@ def run_ours(args):
         time.sleep(0.5)  # let the sampler start before the timed region
         t0.record(stream)
         for _ in range(args.steps):
-            run_step(record=True)
+            if graph is not None:
+                graph.replay()
+            else:
+                run_step(record=True)
         t1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1) / args.steps
+    if graph is not None:
+        for _ in range(min(args.steps, 50)):
+            run_step(record=True)
+        torch.cuda.synchronize()
     per_call = {name: sum(a.elapsed_time(b) for a, b in lst) / len(lst) for name, lst in ev_calls.items()}
     full_ms = [a.elapsed_time(b) for a, b in ev_calls["csa2_index_full"]]
     ms = max_over_ranks(ms, device, world)
@@ -396,7 +414,7 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "int32+f64 indexer, f16 tensor-core attention (f32 accumulate)",
             "data": "synthetic",
-            "config": decode_config(wl, ab["total"], args.sequential),
+            "config": decode_config(wl, ab["total"], args.sequential, graph is not None),
             "tokens_per_s": job_throughput(world, wl.B, ms),
             "hbm_algorithmic_gbs": ab["total"] / (ms * 1e-3) / 1e9,
             "hbm_frac_of_8tbs": ab["total"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
@@ -572,7 +590,8 @@ def run_reference(args):
     res = {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int32+f64 (CPU oracle)",
-           "data": "synthetic", "config": decode_config(wl, algorithmic_bytes(wl)["total"], args.sequential),
+           "data": "synthetic", "config": decode_config(wl, algorithmic_bytes(wl)["total"], args.sequential,
+                                                        not args.no_graph),
            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": nthreads, "kind": "oracle",
                             "sample": f"{args.steps} queries (one per step) over {len(samples)} sequences of the "
                                       f"workload, {nthreads} host threads at a time; {secs:.1f} s"},

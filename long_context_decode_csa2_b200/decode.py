@@ -179,6 +179,23 @@ class DecodeStep:
                 main.wait_event(ev)
         return self.out
 
+    def capture(self, caches, seq_row_off, seq_len, layers):
+        """Records one step into a CUDA graph; ``graph.replay()`` then runs the
+        whole step (every call, both schedules, with the same buffers) as one
+        launch.  Call ``run`` once before capturing (warm-up), and do not
+        change the tensors' addresses afterwards."""
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(device=self.out.device)
+        cap.wait_stream(torch.cuda.current_stream())
+        hook, self.hook = self.hook, None
+        try:
+            with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
+                self.run(caches, seq_row_off, seq_len, layers)
+        finally:
+            self.hook = hook
+        torch.cuda.current_stream().wait_stream(cap)
+        return graph
+
     def device_flags(self) -> int:
         flags = C.device_status(self.ws_full)
         for ws in {id(w): w for w in self.ws_re + self.ws_attn if w is not None}.values():

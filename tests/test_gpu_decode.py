@@ -136,3 +136,27 @@ def test_decode_with_input_events_and_layer_callbacks():
     for layer in range(len(layers)):
         assert np.array_equal(host(step.topk[layer]), host(plain.topk[layer]))
         assert np.array_equal(outs[layer].numpy(), host(plain.out[layer]))
+
+
+def test_decode_step_replayed_from_a_cuda_graph():
+    """A captured step replays to the same bits as the eager step."""
+    wl = W.DecodeWorkload("graph_small", np.array([70000, 4096, 777]), "FRRU", needles=8)
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    caches_h = [W.full_cache_host(wl, f, layers[f]["q_codes"], layers[f]["q_scales"]) for f in wl.full_layers()]
+    caches_d = [FullCache(C.cache(dev(c["idx_codes"]), dev(c["idx_scales"])),
+                          C.cache(dev(c["main_codes"]), dev(c["main_scales"]))) for c in caches_h]
+    off_d, len_d = dev(caches_h[0]["seq_row_off"]), dev(wl.lengths.astype(np.int32))
+    dl = _device_layers(layers)
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
+    step.run(caches_d, off_d, len_d, dl)
+    torch.cuda.synchronize()
+    eager = [host(t).copy() for t in step.topk], host(step.out).copy()
+    graph = step.capture(caches_d, off_d, len_d, dl)
+    step.out.zero_()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert step.device_flags() == 0
+    for layer in range(len(wl.pattern)):
+        assert np.array_equal(host(step.topk[layer]), eager[0][layer])
+    assert np.array_equal(host(step.out), eager[1])

@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="long_decode_b64_l1m")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling captures)")
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager steps instead of replays of one captured CUDA graph")
@@ -349,11 +349,9 @@ def run_ours(args):
             out_host[layer].copy_(step.out[layer], non_blocking=True)
             top_host[layer].copy_(step.topk[layer], non_blocking=True)
 
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        h2d_stream.wait_stream(stream)  # the previous step no longer reads the inputs
+    def e2e_step():
+        cur = torch.cuda.current_stream()
+        h2d_stream.wait_stream(cur)  # the previous step no longer reads the inputs
         with torch.cuda.stream(h2d_stream):
             for l in range(n_layers):
                 for k in keys_in:
@@ -362,7 +360,28 @@ def run_ours(args):
                     (dst.view(torch.int16) if dst.dtype == torch.bfloat16 else dst).copy_(src, non_blocking=True)
                 ev_in[l].record(h2d_stream)
         step.run(caches, off_d, len_d, layers_dev, ready=ev_in, on_layer_done=copy_out)
-        stream.wait_stream(d2h_stream)  # the step ends when its results are on the host
+        cur.wait_stream(d2h_stream)  # the step ends when its results are on the host
+        cur.wait_stream(h2d_stream)
+
+    e2e_graph = None
+    if graph is not None:  # the whole end-to-end step (copies included) as one graph as well
+        e2e_step()
+        torch.cuda.synchronize()
+        e2e_graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(device=device)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(e2e_graph, stream=cap, capture_error_mode="thread_local"):
+            e2e_step()
+        stream.wait_stream(cap)
+        torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        if e2e_graph is not None:
+            e2e_graph.replay()
+        else:
+            e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps

@@ -152,6 +152,9 @@ csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
  *   out        [B][16][512] fp32;  lse [B][16] fp32 or NULL
  * Accuracy: max-abs error <= 2e-3 and relative-L2 error <= 1e-3 against exact
  * arithmetic for inputs whose dequantised values are exact in fp16.
+ * The workspace size depends on B, k and the current device (how many CTAs
+ * share a sequence follows its SM count): query it with the device current on
+ * which the call will run.
  * ------------------------------------------------------------------------- */
 size_t csa2_sparse_attn_decode_workspace_bytes(int B, int k);
 csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv, const int64_t* seq_row_off,

@@ -480,17 +480,7 @@ __global__ void __launch_bounds__(1024) k_seg_prep(SegDesc sd, int S, int32_t* s
     const int s = base + threadIdx.x;
     int32_t ntile = 0;
     if (s < S) {
-      int64_t L = sd.len[s];
-      const int64_t off = sd.row_off ? sd.row_off[s] : sd.row0;
-      if (L < 0) L = 0;
-      if (L > sd.max_len) {
-        set_status(status, CSA2_DEV_LENGTH);
-        L = sd.max_len;
-      }
-      if ((off & 7) != 0 || off < 0 || off + L > sd.cache_rows) {
-        set_status(status, CSA2_DEV_ROW_LAYOUT);
-        L = 0;
-      }
+      const int64_t L = seg_len_checked(sd, s, status);
       seg_eff[s] = int32_t(L);
       ntile = int32_t((L + kTile - 1) / kTile);
     }

@@ -352,19 +352,20 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
     uint32_t T = 0, rem = 0;
     if (ghist) {
       // the top HB bits from the producer's histogram; the low bits by radix
-      // digits of up to 8 bits over the keys of the threshold bucket only
+      // digits of up to 10 bits over the keys of the threshold bucket only
+      // (two digits for both histogram widths)
       uint32_t* hist = dsm;       // NB
-      uint32_t* h2 = dsm + NB;    // 256
+      uint32_t* h2 = dsm + NB;    // 1024
       store_hist<NB>(ghist + int64_t(s) * NB, hist, hp);
       __syncthreads();
       if (total > uint32_t(k)) {
         find_bin(hist, NB, uint32_t(k), sh);
         uint32_t prefix = sh.digit << (32 - HB), pmask = ~((1u << (32 - HB)) - 1u);
         rem = sh.rem;
-        for (int hi = 31 - HB; hi >= 0; hi -= 8) {
-          const int width = min(8, hi + 1), shift = hi - width + 1;
+        for (int hi = 31 - HB; hi >= 0; hi -= 10) {
+          const int width = min(10, hi + 1), shift = hi - width + 1;
           const uint32_t dm = (1u << width) - 1u;
-          if (tid < 256) h2[tid] = 0;
+          h2[tid] = 0;  // 1024 threads, 1024 bins
           __syncthreads();
 #pragma unroll
           for (int e = 0; e < kSelPer; ++e) {
@@ -616,9 +617,9 @@ void launch_select_kind(const void* in, int64_t in_stride, const int32_t* seg_ef
                         int k, int32_t* out, uint32_t* hist, int64_t n_bound, cudaStream_t st) {
   if (n_bound <= kSelSmallMax) {
     constexpr int NB = (KIND == kSelPoolCand) ? kCandHistBins : kHist1Bins;
-    const size_t smem = (hist ? NB + 256 : 256) * sizeof(uint32_t);
+    const size_t smem = (hist ? NB + 1024 : 256) * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         int((NB + 256) * sizeof(uint32_t)));
+                         int((NB + 1024) * sizeof(uint32_t)));
     k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist);
   } else {
     const size_t smem = kSelLargeWords * sizeof(uint32_t);

@@ -14,6 +14,7 @@ no data-path collective); rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -71,7 +72,10 @@ def algorithmic_bytes(wl):
     scan = int((L * 68).sum()) * 1  # only the first Full layer scans (default plan)
     pool = int((pooled * 68).sum()) * n_pool
     attn = wl.B * (wl.k * 272 + 128 * 512) * len(wl.pattern)
-    return dict(scan=scan, pool=pool, attn=attn, total=scan + pool + attn, n_full=n_scan)
+    # ratio 2: per Full layer one raw token + logit per sequence, W_idx, and
+    # one 340-byte entry per sequence every second step
+    append = n_scan * (wl.B * (512 * 2 + 4) + 512 * 128 * 4 + wl.B * 340 // 2) if wl.ratio == 2 else 0
+    return dict(scan=scan, pool=pool, attn=attn, append=append, total=scan + pool + attn + append, n_full=n_scan)
 
 
 class ClockSampler:
@@ -158,8 +162,21 @@ def time_oracle(wl, samples, nthreads, jobs=None):
 
     import oracle
 
+    toks = None
+    if wl.ratio == 2:
+        import synth
+
+        toks = [dict(raw=synth.normal_bf16(wl.seed, synth.T_RAW, 0, f, 512).reshape(1, 512),
+                     logit=synth.normal_f32(wl.seed, synth.T_LOGITS, 0, f, 1),
+                     w_idx=synth.normal_f32(wl.seed, synth.T_WIDX, 0, f, 512 * 128, log2_div=13).reshape(512, 128))
+                for f in wl.full_layers()]
+
     def one(j):
         ch, L, lb = samples[j % len(samples)]
+        if toks:  # ratio 2: the step's append (a pending token completes an entry)
+            for t in toks:
+                pend = [dict(raw=t["raw"][0], logit=float(t["logit"][0]), idx=None)]
+                oracle.compress_stream(pend, t["raw"], t["logit"], np.array([0, 1]), w_idx=t["w_idx"], nthreads=1)
         oracle.decode_step(wl.pattern, ch, np.array([0]), np.array([L], np.int32), lb, wl.P, wl.k,
                            1 / math.sqrt(512), nthreads=1)
 
@@ -174,7 +191,9 @@ def time_oracle(wl, samples, nthreads, jobs=None):
 
 def decode_config(wl, l2_bytes, sequential, graph=True):
     """The `config` object of a decode line (both arms)."""
-    return {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len, "layers": wl.pattern,
+    extra = ({"ratio": 2, "append": "one raw token per sequence per Full layer per step (csa2_compress_stream, "
+                                    "W_idx projection)"} if wl.ratio == 2 else {})
+    return {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len, "layers": wl.pattern, **extra,
             "pool_blocks": wl.P, "topk": wl.k, "window": 128,
             "l2": "no flush: inputs larger than L2 (%.2f GB read per step)" % (l2_bytes / 1e9),
             "schedule": ("sequential" if sequential else "concurrent tail (side streams)")
@@ -188,8 +207,7 @@ def rank_workload(wl, rank):
 
     if rank == 0:
         return wl
-    return W.DecodeWorkload(wl.name, wl.lengths, wl.pattern, wl.P, wl.k, wl.needles, wl.lognormal,
-                            seed=wl.seed + 1000 * rank)
+    return dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
 
 
 def max_over_ranks(x, device, world):
@@ -235,6 +253,28 @@ def build_workload(wl, rank, device):
     return wl, layers, caches_dev, caches, layers_dev, to_dev(off), to_dev(wl.lengths.astype(np.int32))
 
 
+def new_token_inputs(wl, device):
+    """Ratio 2: per Full layer the step's new raw token of every sequence
+    (bf16), its logit and the layer's W_idx (host arrays and device copies)."""
+    import synth
+
+    host, devs = [], []
+    for i, f in enumerate(wl.full_layers()):
+        h = dict(raw=synth.normal_bf16(wl.seed, synth.T_RAW, 0, f, wl.B * 512).reshape(wl.B, 512),
+                 logit=synth.normal_f32(wl.seed, synth.T_LOGITS, 0, f, wl.B) * 2,
+                 w_idx=synth.normal_f32(wl.seed, synth.T_WIDX, 0, f, 512 * 128, log2_div=13).reshape(512, 128))
+        host.append(h)
+        d = {}
+        import torch
+
+        for k, v in h.items():
+            v = np.ascontiguousarray(v)
+            d[k] = (torch.from_numpy(v.view(np.int16)).to(device).view(torch.bfloat16) if v.dtype == np.uint16
+                    else torch.from_numpy(v).to(device))
+        devs.append(d)
+    return host, devs
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -255,15 +295,27 @@ def run_ours(args):
 
     wl = W.decode_workloads()[args.workload]
     if args.batch:
-        wl = W.DecodeWorkload(wl.name + f"_b{args.batch}", wl.lengths[:args.batch], wl.pattern, wl.P, wl.k,
-                              wl.needles, wl.lognormal, wl.seed)
+        wl = dataclasses.replace(wl, name=wl.name + f"_b{args.batch}", lengths=wl.lengths[:args.batch])
     if args.context:
-        wl = W.DecodeWorkload(wl.name + f"_l{args.context}", np.full(wl.B, args.context), wl.pattern, wl.P, wl.k,
-                              min(wl.needles, max(1, args.context // 1024)), wl.lognormal, wl.seed)
+        wl = dataclasses.replace(wl, name=wl.name + f"_l{args.context}", lengths=np.full(wl.B, args.context),
+                                 needles=min(wl.needles, max(1, args.context // 1024)))
     wl, layers, caches_dev, caches, layers_dev, off_d, len_d = build_workload(wl, rank, device)
     C.lib()
-    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, concurrent=not args.sequential)
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=not args.sequential,
+                      ratio=wl.ratio)
     stream = torch.cuda.current_stream()
+    toks_host, toks_dev = new_token_inputs(wl, device) if wl.ratio == 2 else (None, None)
+    len0 = len_d.clone()
+    if wl.ratio == 2 and max(args.steps, args.e2e_steps + 1, args.warmup + 3) > 2 * wl.room:
+        raise SystemExit(f"at most {2 * wl.room} steps per timed phase fit the caches' spare rows")
+
+    def reset_lengths():
+        """Ratio 2: every phase starts from the initial lengths (the steps
+        append into the spare rows again)."""
+        if wl.ratio == 2:
+            len_d.copy_(len0)
+            for pair in step.pairs:
+                pair.pend_n.zero_()
 
     # events around every C-ABI call of the timed region, on the stream the
     # call runs on; csa2_index_full (full-context scan, block max, pool,
@@ -287,7 +339,7 @@ def run_ours(args):
 
     def run_step(record=False):
         recording[0] = record
-        step.run(caches, off_d, len_d, layers_dev)
+        step.run(caches, off_d, len_d, layers_dev, new_tokens=toks_dev)
         recording[0] = False
 
     for _ in range(args.warmup):
@@ -300,10 +352,11 @@ def run_ours(args):
     # default); the per-call times come from a separate eager pass
     graph = None
     if not args.no_graph:
-        graph = step.capture(caches, off_d, len_d, layers_dev)
+        graph = step.capture(caches, off_d, len_d, layers_dev, new_tokens=toks_dev)
         for _ in range(3):
             graph.replay()
         torch.cuda.synchronize()
+    reset_lengths()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -321,6 +374,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1) / args.steps
+    reset_lengths()
     if graph is not None:
         for _ in range(min(args.steps, 50)):
             run_step(record=True)
@@ -334,6 +388,11 @@ def run_ours(args):
     host_in = [{k: torch.from_numpy(np.ascontiguousarray(
         L[k].view(np.int16) if L[k].dtype == np.uint16 else L[k])).pin_memory() for k in keys_in} for L in layers]
     h2d = sum(t.numel() * t.element_size() for L in host_in for t in L.values())
+    # ratio 2: the new raw tokens and logits come from the host every step
+    tok_in = ([{k: torch.from_numpy(np.ascontiguousarray(h[k].view(np.int16) if h[k].dtype == np.uint16 else h[k]))
+                .pin_memory() for k in ("raw", "logit")} for h in toks_host] if toks_host else [])
+    h2d += sum(t.numel() * t.element_size() for T in tok_in for t in T.values())
+    full_of_layer = {l: i for i, l in enumerate(wl.full_layers())}
     out_host = torch.empty(step.out.shape, dtype=torch.float32).pin_memory()
     top_host = torch.empty((n_layers, wl.B, wl.k), dtype=torch.int32).pin_memory()
     d2h = out_host.numel() * 4 + top_host.numel() * 4
@@ -358,8 +417,12 @@ def run_ours(args):
                     dst = layers_dev[l][k]
                     src = host_in[l][k]
                     (dst.view(torch.int16) if dst.dtype == torch.bfloat16 else dst).copy_(src, non_blocking=True)
+                if tok_in and l in full_of_layer:
+                    for k, src in tok_in[full_of_layer[l]].items():
+                        dst = toks_dev[full_of_layer[l]][k]
+                        (dst.view(torch.int16) if dst.dtype == torch.bfloat16 else dst).copy_(src, non_blocking=True)
                 ev_in[l].record(h2d_stream)
-        step.run(caches, off_d, len_d, layers_dev, ready=ev_in, on_layer_done=copy_out)
+        step.run(caches, off_d, len_d, layers_dev, ready=ev_in, on_layer_done=copy_out, new_tokens=toks_dev)
         cur.wait_stream(d2h_stream)  # the step ends when its results are on the host
         cur.wait_stream(h2d_stream)
 
@@ -376,6 +439,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    reset_lengths()
     e0.record(stream)
     for _ in range(args.e2e_steps):
         if e2e_graph is not None:
@@ -420,6 +484,7 @@ def run_ours(args):
             # index_full: prep, scan, pool select, pool score, Top-k select;
             # reindex: pool score, select; attention: one kernel
             launches_per_step += {"scan": 5, "reindex": 2, "reuse": 0}[act] + 1
+        launches_per_step += len(step.pairs)  # ratio 2: one append per Full layer
         res = {
             "metric": METRIC,
             "value": job_throughput(world, wl.B, ms),
@@ -588,8 +653,7 @@ def run_reference(args):
         del caches_dev
     else:
         # no GPU to generate the full-size caches: shorter contexts (named in the config)
-        small = W.DecodeWorkload(wl.name + "_l65536_host", np.full(nthreads, min(wl.max_len, 65536)), wl.pattern,
-                                 wl.P, wl.k, wl.needles, wl.lognormal)
+        small = dataclasses.replace(wl, name=wl.name + "_l65536_host", lengths=np.full(nthreads, min(wl.max_len, 65536)))
         wl = small
         layers = [W.layer_inputs_host(small, l) for l in range(len(small.pattern))]
         caches = [W.full_cache_host(small, f, layers[f]["q_codes"], layers[f]["q_scales"])

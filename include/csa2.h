@@ -193,6 +193,41 @@ csa2_status csa2_compress_append(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * csa2_compress_stream -- ratio-2 append that keeps an odd trailing token on
+ * the device (decode: one raw token per sequence per step, and every second
+ * token completes an entry).
+ * Source: as csa2_compress_append; [V41] architecture figure caption (the
+ * compressor merges disjoint pairs of consecutive tokens) applied while
+ * generating.
+ * Sequence b's token stream is its pending token (if pend_n[b] == 1)
+ * followed by raw tokens tok_off[b] .. tok_off[b+1]-1 of this call.  Entries
+ * are the stream's pairs (0,1), (2,3), ..., merged, projected and encoded
+ * exactly as csa2_compress_append with ratio 2, and written at cache rows
+ * seq_row_off[b] + seq_len_in[b] + j.  If the stream has odd length, its last
+ * token (bf16 row, logit, idx_raw row) is kept in pend_raw[b], pend_logit[b],
+ * pend_idx[b] and pend_n[b] = 1; otherwise pend_n[b] = 0.  Appending a
+ * sequence's tokens over any number of calls gives the same cache bytes as
+ * one csa2_compress_append of all of them.
+ *   pend_n     [B] int32 (0 or 1), read and written in place
+ *   pend_raw   [B][512] bf16 (16-byte aligned), pend_logit [B] fp32
+ *   pend_idx   [B][128] bf16 (8-byte aligned) when idx_raw is used; NULL with w_idx
+ *   seq_len_out [B] receives seq_len_in + entries; it may be seq_len_in
+ *              itself (updated in place) or NULL (not written)
+ *   logits     required; raw / idx_raw may be NULL when n_tok == 0
+ *   max_new    host: upper bound of (pend_n[b] + tokens of b) / 2 (grid sizing)
+ *   workspace  csa2_compress_stream_workspace_bytes(B), zero-filled before the
+ *              first call (its counters return to zero after each call)
+ * Everything else as csa2_compress_append.
+ * ------------------------------------------------------------------------- */
+size_t csa2_compress_stream_workspace_bytes(int B);
+csa2_status csa2_compress_stream(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k, const uint16_t* raw,
+                                 const float* logits, const float* w_idx, const uint16_t* idx_raw,
+                                 const int64_t* tok_off, const int64_t* seq_row_off, const int32_t* seq_len_in,
+                                 int32_t* seq_len_out, int32_t* pend_n, uint16_t* pend_raw, float* pend_logit,
+                                 uint16_t* pend_idx, int B, int64_t n_tok, int64_t max_new, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * csa2_index_prefill -- causal Full-mode indexer for a prefill chunk.
  * Source: [V41] hierarchical indexer (as csa2_index_full), applied to every
  * query of a causal prefill chunk.

@@ -52,6 +52,8 @@ def lib():
             "csa2_sparse_attn_decode": (I, [P, Cache, P, P, P, I, P, P, P, F, P, P, I, P, Z, P]),
             "csa2_compress_append_workspace_bytes": (Z, [I]),
             "csa2_compress_append": (I, [Cache, Cache, P, P, P, P, P, P, P, P, I, I, I64, I64, P, Z, P]),
+            "csa2_compress_stream_workspace_bytes": (Z, [I]),
+            "csa2_compress_stream": (I, [Cache, Cache, P, P, P, P, P, P, P, P, P, P, P, P, I, I64, I64, P, Z, P]),
             "csa2_index_prefill_workspace_bytes": (Z, [I, I64, I, I]),
             "csa2_index_prefill": (I, [Cache, P, P, P, P, I, I64, I64, I, I, I, P, P, P, Z, P]),
             "csa2_sparse_attn_prefill_workspace_bytes": (Z, [I, I]),
@@ -177,6 +179,23 @@ def csa2_compress_append(main_kv, idx_k, raw, logits, tok_off, seq_row_off, seq_
                                     _ptr(tok_off), _ptr(seq_row_off), _ptr(seq_len_in), _ptr(seq_len_out), B, ratio,
                                     raw.shape[0], int(max_new), wp, wn, _stream(stream))
     _check(rc, "csa2_compress_append")
+
+
+def csa2_compress_stream_workspace_bytes(B):
+    return lib().csa2_compress_stream_workspace_bytes(B)
+
+
+def csa2_compress_stream(main_kv, idx_k, raw, logits, tok_off, seq_row_off, seq_len_in, seq_len_out, pend_n, pend_raw,
+                         pend_logit, max_new, ws, w_idx=None, idx_raw=None, pend_idx=None, stream=None):
+    """seq_len_out may be seq_len_in (in place) or None; raw may be None when no token is appended."""
+    B = seq_len_in.shape[0]
+    wp, wn = _ws(ws)
+    n_tok = raw.shape[0] if raw is not None else 0
+    rc = lib().csa2_compress_stream(main_kv, idx_k, _ptr(raw), _ptr(logits), _ptr(w_idx), _ptr(idx_raw),
+                                    _ptr(tok_off), _ptr(seq_row_off), _ptr(seq_len_in), _ptr(seq_len_out),
+                                    _ptr(pend_n), _ptr(pend_raw), _ptr(pend_logit), _ptr(pend_idx), B, n_tok,
+                                    int(max_new), wp, wn, _stream(stream))
+    _check(rc, "csa2_compress_stream")
 
 
 def csa2_index_prefill_workspace_bytes(T, n_entries, pool_blocks, k):

@@ -285,6 +285,63 @@ csa2_status csa2_compress_append(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_
   return check_launch(fn);
 }
 
+size_t csa2_compress_stream_workspace_bytes(int B) {
+  return kStatusBytes + round_up(size_t(B > 0 ? B : 0) * sizeof(uint32_t), 256);
+}
+
+csa2_status csa2_compress_stream(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k, const uint16_t* raw,
+                                 const float* logits, const float* w_idx, const uint16_t* idx_raw,
+                                 const int64_t* tok_off, const int64_t* seq_row_off, const int32_t* seq_len_in,
+                                 int32_t* seq_len_out, int32_t* pend_n, uint16_t* pend_raw, float* pend_logit,
+                                 uint16_t* pend_idx, int B, int64_t n_tok, int64_t max_new, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_compress_stream";
+  if (B < 0 || n_tok < 0 || max_new < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
+  if (B == 0) return CSA2_OK;
+  if (!cache_ok(main_kv) || !cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad cache");
+  if (!tok_off || !seq_row_off || !seq_len_in || !pend_n || !pend_raw || !pend_logit || !logits || !workspace)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (n_tok > 0 && !raw) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null raw");
+  if ((w_idx == nullptr) == (idx_raw == nullptr && pend_idx == nullptr))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": give w_idx, or idx_raw with pend_idx");
+  if (w_idx && (idx_raw || pend_idx))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": w_idx excludes idx_raw and pend_idx");
+  if (!w_idx && (!pend_idx || (n_tok > 0 && !idx_raw)))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": idx_raw needs pend_idx");
+  if ((raw && !aligned16(raw)) || !aligned16(pend_raw) || (idx_raw && (reinterpret_cast<uintptr_t>(idx_raw) & 7)) ||
+      (pend_idx && (reinterpret_cast<uintptr_t>(pend_idx) & 7)))
+    return fail(CSA2_ERR_INVALID_ARG,
+                std::string(fn) + ": raw and pend_raw must be 16-byte, idx_raw and pend_idx 8-byte aligned");
+  if (workspace_bytes < csa2_compress_stream_workspace_bytes(B))
+    return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  CompressArgs a{};
+  a.mcodes = main_kv.codes;
+  a.mscales = main_kv.scales;
+  a.mrows = main_kv.rows;
+  a.icodes = idx_k.codes;
+  a.iscales = idx_k.scales;
+  a.irows = idx_k.rows;
+  a.raw = raw;
+  a.logits = logits;
+  a.w_idx = w_idx;
+  a.idx_raw = idx_raw;
+  a.tok_off = tok_off;
+  a.seq_row_off = seq_row_off;
+  a.seq_len_in = seq_len_in;
+  a.seq_len_out = seq_len_out;
+  a.B = B;
+  a.ratio = 2;
+  a.max_new = max_new;
+  a.status = static_cast<uint32_t*>(workspace);
+  a.pend_n = pend_n;
+  a.pend_raw = pend_raw;
+  a.pend_logit = pend_logit;
+  a.pend_idx = pend_idx;
+  a.arrive = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + kStatusBytes);
+  launch_compress(a, static_cast<cudaStream_t>(stream));
+  return check_launch(fn);
+}
+
 // ---------------------------------------------------------------------------
 namespace {
 struct PrefillWs {

@@ -106,135 +106,197 @@ __device__ __forceinline__ void encode_row(const float (&x)[V], uint8_t* codes, 
   if ((lane % (32 / V)) == 0) scales[lane / (32 / V)] = uint8_t(X + 127);
 }
 
+// Token s of sequence b's stream: the pending token (s < pn) or raw token
+// tok0 + s - pn of this call.
+struct TokenSrc {
+  const CompressArgs& a;
+  int b, pn;
+  int64_t tok0;
+  __device__ const uint16_t* row(int64_t s) const {
+    return s < pn ? a.pend_raw + int64_t(b) * kD : a.raw + (tok0 + s - pn) * kD;
+  }
+  __device__ const uint16_t* idx_row(int64_t s) const {
+    return s < pn ? a.pend_idx + int64_t(b) * kDi : a.idx_raw + (tok0 + s - pn) * kDi;
+  }
+  __device__ double logit(int64_t s) const { return s < pn ? a.pend_logit[b] : a.logits[tok0 + s - pn]; }
+};
+
+// Pair weights w = softmax(z0, z1) in double with the own exp.
+__device__ __forceinline__ void pair_weights(double z0, double z1, double& w0, double& w1) {
+  const double m = fmax(z0, z1);
+  const double e0 = own_exp(__dsub_rn(z0, m)), e1 = own_exp(__dsub_rn(z1, m));
+  const double sum = __dadd_rn(e0, e1);
+  w0 = __ddiv_rn(e0, sum);
+  w1 = __ddiv_rn(e1, sum);
+}
+
 // grid = (ceil(max_new / 16), B), block = 256.  Each warp merges and encodes
 // two entries' main rows; the optional W_idx projection is shared by the CTA
-// (thread t: column t % 128 for eight entries, so every W_idx element read
-// feeds eight fma chains), and each warp then encodes its two indexer rows.
+// (thread t: column t % 128 of the entries e = 2q + t / 128, so every W_idx
+// element read feeds up to eight fma chains), and each warp then encodes its
+// two indexer rows.  Streaming mode (a.pend_n != null): the sequence's token
+// stream starts with its pending token, the last CTA of the sequence to
+// finish keeps an odd trailing token as the new pending one and writes the
+// new lengths (all CTAs have read the old ones by then).
 __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
   // merged rows, widened once for the projection; projected rows
   extern __shared__ __align__(16) unsigned char csm[];
   double (*cbuf)[kD] = reinterpret_cast<double (*)[kD]>(csm);
   float (*rbuf)[kDi] = reinterpret_cast<float (*)[kDi]>(csm + sizeof(double) * kCompEntries * kD);
+  __shared__ int last_cta;
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool streaming = a.pend_n != nullptr;
   const int64_t tok0 = a.tok_off[b];
-  const int64_t ntok = a.tok_off[b + 1] - tok0;
-  const int64_t nnew = ntok > 0 ? ntok / a.ratio : 0;
-  if (blockIdx.x == 0 && threadIdx.x == 0) a.seq_len_out[b] = a.seq_len_in[b] + int32_t(nnew);
+  const int64_t ntok = max(int64_t(0), a.tok_off[b + 1] - tok0);
+  const int pn = streaming ? (a.pend_n[b] != 0 ? 1 : 0) : 0;
+  const int64_t nstream = ntok + pn;
+  const int64_t nnew = nstream / a.ratio;
+  const int32_t len_in = a.seq_len_in[b];
+  if (!streaming && blockIdx.x == 0 && threadIdx.x == 0) a.seq_len_out[b] = len_in + int32_t(nnew);
+  const TokenSrc src{a, b, pn, tok0};
   const int64_t j0 = int64_t(blockIdx.x) * kCompEntries;
-  if (j0 >= nnew) return;  // uniform for the whole CTA
 
-  // ---- phase 1: merge + encode the main rows (entries warp, warp + 8) ----
-  bool ok[2];
-  int64_t rows[2], toks[2];
+  if (j0 < nnew) {  // uniform for the whole CTA
+    const int nvalid = int(min(int64_t(kCompEntries), nnew - j0));
+    // ---- phase 1: merge + encode the main rows (entries warp, warp + 8) ----
+    bool ok[2];
+    int64_t rows[2];
+    double w0s[2], w1s[2];
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int e = warp + kCompWarps * u;
-    const int64_t j = j0 + e;
-    const int64_t row = a.seq_row_off[b] + a.seq_len_in[b] + j;
-    ok[u] = j < nnew;
-    if (ok[u] && (row < 0 || row >= a.mrows || row >= a.irows)) {
-      if (lane == 0) set_status(a.status, CSA2_DEV_ROW_LAYOUT);
-      ok[u] = false;
-    }
-    rows[u] = row;
-    toks[u] = tok0 + a.ratio * j;  // first raw token of the entry
-    float c[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) c[i] = 0.0f;
-    if (ok[u]) {
-      const int64_t t0 = toks[u];
-      double w0 = 1.0, w1 = 0.0;
-      if (a.ratio == 2) {
-        const double z0 = a.logits[t0], z1 = a.logits[t0 + 1];
-        const double m = fmax(z0, z1);
-        const double e0 = own_exp(__dsub_rn(z0, m)), e1 = own_exp(__dsub_rn(z1, m));
-        const double sum = __dadd_rn(e0, e1);
-        w0 = __ddiv_rn(e0, sum);
-        w1 = __ddiv_rn(e1, sum);
+    for (int u = 0; u < 2; ++u) {
+      const int e = warp + kCompWarps * u;
+      const int64_t j = j0 + e;
+      const int64_t row = a.seq_row_off[b] + len_in + j;
+      ok[u] = j < nnew;
+      if (ok[u] && (row < 0 || row >= a.mrows || row >= a.irows)) {
+        if (lane == 0) set_status(a.status, CSA2_DEV_ROW_LAYOUT);
+        ok[u] = false;
       }
-      // lane holds elements 16*lane .. 16*lane+15
-      const uint4* p0 = reinterpret_cast<const uint4*>(a.raw + t0 * kD + 16 * lane);
-      const uint4 u0 = __ldg(p0), u1 = __ldg(p0 + 1);
-      const uint32_t x0w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-      if (a.ratio == 2) {
-        const uint4* p1 = reinterpret_cast<const uint4*>(a.raw + (t0 + 1) * kD + 16 * lane);
-        const uint4 v0 = __ldg(p1), v1 = __ldg(p1 + 1);
-        const uint32_t x1w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      rows[u] = row;
+      w0s[u] = 1.0;
+      w1s[u] = 0.0;
+      float c[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
-          const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
-          c[i] = __double2float_rn(__fma_rn(w0, x0, __dmul_rn(w1, x1)));
+      for (int i = 0; i < 16; ++i) c[i] = 0.0f;
+      if (ok[u]) {
+        const int64_t s0 = a.ratio * j;  // first stream token of the entry
+        if (a.ratio == 2) pair_weights(src.logit(s0), src.logit(s0 + 1), w0s[u], w1s[u]);
+        // lane holds elements 16*lane .. 16*lane+15
+        const uint4* p0 = reinterpret_cast<const uint4*>(src.row(s0) + 16 * lane);
+        const uint4 u0 = __ldg(p0), u1 = __ldg(p0 + 1);
+        const uint32_t x0w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        if (a.ratio == 2) {
+          const uint4* p1 = reinterpret_cast<const uint4*>(src.row(s0 + 1) + 16 * lane);
+          const uint4 v0 = __ldg(p1), v1 = __ldg(p1 + 1);
+          const uint32_t x1w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+            const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
+            c[i] = __double2float_rn(__fma_rn(w0s[u], x0, __dmul_rn(w1s[u], x1)));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) c[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+        }
+        encode_row<16>(c, a.mcodes + row * kMainCodeBytes, a.mscales + row * kMainScaleBytes, lane);
+      }
+      if (a.w_idx) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) cbuf[e][16 * lane + i] = double(c[i]);
+      }
+    }
+
+    // ---- phase 2: indexer rows r = W_idx^T c (fp64 chain over i = 0..511) ----
+    if (a.w_idx) {
+      __syncthreads();
+      const int col = threadIdx.x % kDi, grp = threadIdx.x / kDi;
+      if (nvalid <= kCompGroups) {
+        // one entry per group (a decode append): a single chain per thread
+        if (grp < nvalid) {
+          double acc = 0.0;
+#pragma unroll 8
+          for (int i = 0; i < kD; ++i) acc = __fma_rn(cbuf[grp][i], double(__ldg(a.w_idx + i * kDi + col)), acc);
+          rbuf[grp][col] = __double2float_rn(acc);
         }
       } else {
+        double acc[kCompPerThread];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) c[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
-      }
-      encode_row<16>(c, a.mcodes + row * kMainCodeBytes, a.mscales + row * kMainScaleBytes, lane);
-    }
-    if (a.w_idx) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) cbuf[e][16 * lane + i] = double(c[i]);
-    }
-  }
-
-  // ---- phase 2: indexer rows r = W_idx^T c (fp64 chain over i = 0..511) ----
-  if (a.w_idx) {
-    __syncthreads();
-    const int col = threadIdx.x % kDi, grp = threadIdx.x / kDi;
-    double acc[kCompPerThread];
-#pragma unroll
-    for (int q = 0; q < kCompPerThread; ++q) acc[q] = 0.0;
+        for (int q = 0; q < kCompPerThread; ++q) acc[q] = 0.0;
 #pragma unroll 4
-    for (int i = 0; i < kD; ++i) {
-      const double wi = double(__ldg(a.w_idx + i * kDi + col));
+        for (int i = 0; i < kD; ++i) {
+          const double wi = double(__ldg(a.w_idx + i * kDi + col));
 #pragma unroll
-      for (int q = 0; q < kCompPerThread; ++q)
-        acc[q] = __fma_rn(cbuf[grp * kCompPerThread + q][i], wi, acc[q]);
-    }
-#pragma unroll
-    for (int q = 0; q < kCompPerThread; ++q) rbuf[grp * kCompPerThread + q][col] = __double2float_rn(acc[q]);
-    __syncthreads();
-  }
-
-  // ---- phase 3: encode the indexer rows (lane holds 4*lane .. 4*lane+3) ----
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    if (!ok[u]) continue;
-    const int e = warp + kCompWarps * u;
-    const int64_t t0 = toks[u], row = rows[u];
-    float r[4];
-    if (a.w_idx) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) r[i] = rbuf[e][4 * lane + i];
-    } else {
-      double w0 = 1.0, w1 = 0.0;
-      if (a.ratio == 2) {
-        const double z0 = a.logits[t0], z1 = a.logits[t0 + 1];
-        const double m = fmax(z0, z1);
-        const double e0 = own_exp(__dsub_rn(z0, m)), e1 = own_exp(__dsub_rn(z1, m));
-        const double sum = __dadd_rn(e0, e1);
-        w0 = __ddiv_rn(e0, sum);
-        w1 = __ddiv_rn(e1, sum);
-      }
-      const uint2 uu = __ldg(reinterpret_cast<const uint2*>(a.idx_raw + t0 * kDi + 4 * lane));
-      const uint32_t x0w[2] = {uu.x, uu.y};
-      if (a.ratio == 2) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.idx_raw + (t0 + 1) * kDi + 4 * lane));
-        const uint32_t x1w[2] = {v.x, v.y};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
-          const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
-          r[i] = __double2float_rn(__fma_rn(w0, x0, __dmul_rn(w1, x1)));
+          for (int q = 0; q < kCompPerThread; ++q)
+            acc[q] = __fma_rn(cbuf[q * kCompGroups + grp][i], wi, acc[q]);
         }
-      } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) r[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+        for (int q = 0; q < kCompPerThread; ++q) rbuf[q * kCompGroups + grp][col] = __double2float_rn(acc[q]);
       }
+      __syncthreads();
     }
-    encode_row<4>(r, a.icodes + row * kIdxCodeBytes, a.iscales + row * kIdxScaleBytes, lane);
+
+    // ---- phase 3: encode the indexer rows (lane holds 4*lane .. 4*lane+3) ----
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!ok[u]) continue;
+      const int e = warp + kCompWarps * u;
+      const int64_t s0 = a.ratio * (j0 + e), row = rows[u];
+      float r[4];
+      if (a.w_idx) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] = rbuf[e][4 * lane + i];
+      } else {
+        const uint2 uu = __ldg(reinterpret_cast<const uint2*>(src.idx_row(s0) + 4 * lane));
+        const uint32_t x0w[2] = {uu.x, uu.y};
+        if (a.ratio == 2) {
+          const uint2 v = __ldg(reinterpret_cast<const uint2*>(src.idx_row(s0 + 1) + 4 * lane));
+          const uint32_t x1w[2] = {v.x, v.y};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const double x0 = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+            const double x1 = bf16f(uint16_t(x1w[i / 2] >> (16 * (i & 1))));
+            r[i] = __double2float_rn(__fma_rn(w0s[u], x0, __dmul_rn(w1s[u], x1)));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) r[i] = bf16f(uint16_t(x0w[i / 2] >> (16 * (i & 1))));
+        }
+      }
+      encode_row<4>(r, a.icodes + row * kIdxCodeBytes, a.iscales + row * kIdxScaleBytes, lane);
+    }
+  }
+  if (!streaming) return;
+
+  // ---- streaming: the last CTA of the sequence updates the pending token ----
+  // The barrier orders this CTA's reads of the pending token and of the
+  // lengths before thread 0's release-acquire arrival (gpu scope).
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.arrive + b) : "memory");
+    last_cta = old == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!last_cta) return;
+  const int64_t keep = nstream - nnew * a.ratio;  // 0 or 1 trailing tokens
+  const int64_t s_last = nstream - 1;
+  if (keep == 1 && s_last >= pn) {  // a raw token of this call becomes the pending one
+    const uint32_t* from = reinterpret_cast<const uint32_t*>(src.row(s_last));
+    uint32_t* to = reinterpret_cast<uint32_t*>(a.pend_raw + int64_t(b) * kD);
+    for (int i = threadIdx.x; i < kD / 2; i += blockDim.x) to[i] = __ldcg(from + i);
+    if (a.pend_idx) {
+      const uint32_t* fi = reinterpret_cast<const uint32_t*>(src.idx_row(s_last));
+      uint32_t* ti = reinterpret_cast<uint32_t*>(a.pend_idx + int64_t(b) * kDi);
+      for (int i = threadIdx.x; i < kDi / 2; i += blockDim.x) ti[i] = __ldcg(fi + i);
+    }
+    if (threadIdx.x == 0) a.pend_logit[b] = a.logits[tok0 + s_last - pn];
+  }
+  if (threadIdx.x == 0) {
+    a.pend_n[b] = int32_t(keep);
+    if (a.seq_len_out) a.seq_len_out[b] = len_in + int32_t(nnew);
+    a.arrive[b] = 0u;  // ready for the next call
   }
 }
 

@@ -149,6 +149,12 @@ struct CompressArgs {
   int ratio;
   int64_t max_new;
   uint32_t* status;
+  // streaming mode (pend_n != null): the pending half-pair of every sequence
+  int32_t* pend_n;       // [B] 0 or 1, read and written
+  uint16_t* pend_raw;    // [B][512] bf16
+  float* pend_logit;     // [B]
+  uint16_t* pend_idx;    // [B][128] bf16, or null (W_idx projection)
+  uint32_t* arrive;      // [B] arrival counters, zero between calls
 };
 void launch_compress(const CompressArgs& a, cudaStream_t st);
 

@@ -16,6 +16,12 @@ notes):
 
 Every layer attends its selection plus its own FP8 window.  This module only
 sequences C-ABI calls; all arithmetic runs in ``libcsa2.so``.
+
+With ``ratio=2`` (compressed entries during generation) each step first
+appends the new raw token of every Full layer's caches with
+``csa2_compress_stream``: the odd token of a pair waits on the device, every
+second step completes an entry, and the sequence lengths advance in place
+before the indexer sees them.
 """
 from __future__ import annotations
 
@@ -55,6 +61,28 @@ def layer_plan(pattern: str, full_rescan: bool = False):
     return plan
 
 
+class PairStream:
+    """Pending half-pairs of one Full layer's caches for ratio-2 appends
+    during decode (one raw token per sequence per step)."""
+
+    def __init__(self, B: int, device, projection: bool = True):
+        dev = torch.device(device)
+        self.pend_n = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.pend_raw = torch.zeros((B, C.MAIN_DIM), dtype=torch.bfloat16, device=dev)
+        self.pend_logit = torch.zeros(B, dtype=torch.float32, device=dev)
+        self.pend_idx = None if projection else torch.zeros((B, C.IDX_DIM), dtype=torch.bfloat16, device=dev)
+        self.tok_off = torch.arange(B + 1, dtype=torch.int64, device=dev)
+        self.ws = C.workspace(C.csa2_compress_stream_workspace_bytes(B), dev)
+
+    def append(self, cache: FullCache, tok: dict, seq_row_off, seq_len, update_len: bool, stream=None):
+        """tok: raw [B,512] bf16, logit [B] fp32, and w_idx [512,128] fp32 or
+        idx_raw [B,128] bf16.  update_len: write the new lengths into seq_len."""
+        C.csa2_compress_stream(cache.main, cache.idx, tok["raw"], tok["logit"], self.tok_off, seq_row_off, seq_len,
+                               seq_len if update_len else None, self.pend_n, self.pend_raw, self.pend_logit, 1,
+                               self.ws, w_idx=tok.get("w_idx"), idx_raw=tok.get("idx_raw"), pend_idx=self.pend_idx,
+                               stream=stream)
+
+
 class DecodeStep:
     """Owns the workspaces and outputs of one decode step; ``run`` enqueues it.
 
@@ -67,8 +95,12 @@ class DecodeStep:
     caller's stream in layer order."""
 
     def __init__(self, pattern: str, B: int, max_len: int, P: int = 2048, k: int = 512, full_rescan: bool = False,
-                 device="cuda", sm_scale: float | None = None, concurrent: bool = True, side_streams: int = 3):
+                 device="cuda", sm_scale: float | None = None, concurrent: bool = True, side_streams: int = 3,
+                 ratio: int = 1, projection: bool = True):
+        if ratio not in (1, 2):
+            raise ValueError("ratio must be 1 or 2")
         self.pattern, self.B, self.max_len, self.P, self.k = pattern, B, max_len, P, k
+        self.ratio = ratio
         self.plan = layer_plan(pattern, full_rescan)
         self.sm_scale = sm_scale if sm_scale is not None else 1.0 / math.sqrt(C.MAIN_DIM)
         self.concurrent = concurrent
@@ -95,6 +127,9 @@ class DecodeStep:
         self.out = torch.zeros((nL, B, C.Q_HEADS, C.MAIN_DIM), dtype=torch.float32, device=dev)
         self.lse = torch.zeros((nL, B, C.Q_HEADS), dtype=torch.float32, device=dev)
         self.scores = None
+        # ratio 2: one pending-token state per Full layer's caches
+        n_full = sum(1 for m in pattern if m == "F")
+        self.pairs = [PairStream(B, dev, projection) for _ in range(n_full)] if ratio == 2 else []
         # optional callable(call_name, "begin" | "end", stream), e.g. to record events
         self.hook = None
 
@@ -107,7 +142,8 @@ class DecodeStep:
         if self.hook is not None:
             self.hook(name, phase, stream)
 
-    def run(self, caches, seq_row_off, seq_len, layers, stream=None, ready=None, on_layer_done=None):
+    def run(self, caches, seq_row_off, seq_len, layers, stream=None, ready=None, on_layer_done=None,
+            new_tokens=None):
         """caches: [FullCache] per Full layer; layers: per layer dict of device
         tensors q, q_codes, q_scales, w, win, win_scale, win_len.
 
@@ -115,8 +151,24 @@ class DecodeStep:
         event (e.g. its inputs arriving on a copy stream).  on_layer_done:
         optional callable(layer, event), called once the layer's attention is
         enqueued, with an event that completes after it (e.g. to copy the
-        layer's output out while later layers run)."""
+        layer's output out while later layers run).
+
+        new_tokens (ratio 2 only): per Full layer a dict for
+        ``PairStream.append``; the appends run first, on the caller's stream,
+        and advance ``seq_len`` in place."""
         main = stream if stream is not None else torch.cuda.current_stream()
+        if self.ratio == 2:
+            if new_tokens is None or len(new_tokens) != len(self.pairs):
+                raise ValueError("a ratio-2 step needs one new token dict per Full layer")
+            full_layers = [layer for layer, m, _, _ in self.plan if m == "F"]
+            for f, (pair, tok) in enumerate(zip(self.pairs, new_tokens)):
+                if ready is not None:
+                    main.wait_event(ready[full_layers[f]])
+                self._hook("csa2_compress_stream", "begin", main)
+                pair.append(caches[f], tok, seq_row_off, seq_len, update_len=f == len(self.pairs) - 1, stream=main)
+                self._hook("csa2_compress_stream", "end", main)
+        elif new_tokens is not None:
+            raise ValueError("new_tokens is for ratio-2 steps")
         pool, pool_ev = None, None
         last, last_ev = None, None
         side = 0
@@ -179,7 +231,7 @@ class DecodeStep:
                 main.wait_event(ev)
         return self.out
 
-    def capture(self, caches, seq_row_off, seq_len, layers):
+    def capture(self, caches, seq_row_off, seq_len, layers, new_tokens=None):
         """Records one step into a CUDA graph; ``graph.replay()`` then runs the
         whole step (every call, both schedules, with the same buffers) as one
         launch.  Call ``run`` once before capturing (warm-up), and do not
@@ -190,7 +242,7 @@ class DecodeStep:
         hook, self.hook = self.hook, None
         try:
             with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
-                self.run(caches, seq_row_off, seq_len, layers)
+                self.run(caches, seq_row_off, seq_len, layers, new_tokens=new_tokens)
         finally:
             self.hook = hook
         torch.cuda.current_stream().wait_stream(cap)
@@ -198,6 +250,7 @@ class DecodeStep:
 
     def device_flags(self) -> int:
         flags = C.device_status(self.ws_full)
-        for ws in {id(w): w for w in self.ws_re + self.ws_attn if w is not None}.values():
+        extra = [p.ws for p in self.pairs]
+        for ws in {id(w): w for w in self.ws_re + self.ws_attn + extra if w is not None}.values():
             flags |= C.device_status(ws)
         return flags

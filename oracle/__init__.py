@@ -223,6 +223,47 @@ def compress(raw_bf16, logits, ratio, w_idx=None, idx_raw_bf16=None, nthreads=0,
     return mc, ms, ic, isc
 
 
+def compress_stream(pend, raw_bf16, logits, tok_off, w_idx=None, idx_raw_bf16=None, nthreads=0):
+    """Ratio-2 append with a pending half-pair per sequence.
+
+    Entries are the disjoint pairs (2j, 2j+1) of each sequence's raw token
+    stream ("DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache
+    Compression", architecture figure caption and section
+    "三个方向一起压小缓存": no overlap between entries), however the stream is
+    cut into calls.  Sequence b's stream for this call is its pending token
+    (pend[b], or None) followed by raw tokens tok_off[b] .. tok_off[b+1]-1;
+    its complete pairs are compressed with ``compress`` and an odd trailing
+    token becomes the new pending one.
+
+    pend[b]: None or dict(raw=[512] uint16, logit=float, idx=[128] uint16 or None).
+    Returns (entries, new_pend): entries[b] = (mc, ms, ic, isc) of the new
+    entries (possibly empty), new_pend[b] as pend[b].
+    """
+    raw_bf16 = np.ascontiguousarray(raw_bf16, np.uint16).reshape(-1, 512)
+    logits = np.ascontiguousarray(logits, np.float32).reshape(-1)
+    use_idx = w_idx is None
+    if use_idx:
+        idx_raw_bf16 = np.ascontiguousarray(idx_raw_bf16, np.uint16).reshape(-1, 128)
+    entries, new_pend = [], []
+    for b in range(len(tok_off) - 1):
+        t0, t1 = int(tok_off[b]), int(tok_off[b + 1])
+        rows, zs, idx = [raw_bf16[t0:t1]], [logits[t0:t1]], [idx_raw_bf16[t0:t1]] if use_idx else None
+        if pend[b] is not None:
+            rows.insert(0, np.asarray(pend[b]["raw"], np.uint16).reshape(1, 512))
+            zs.insert(0, np.array([pend[b]["logit"]], np.float32))
+            if use_idx:
+                idx.insert(0, np.asarray(pend[b]["idx"], np.uint16).reshape(1, 128))
+        x, z = np.concatenate(rows), np.concatenate(zs)
+        xi = np.concatenate(idx) if use_idx else None
+        n = x.shape[0]
+        m = n // 2 * 2
+        entries.append(compress(x[:m], z[:m], 2, w_idx=w_idx, idx_raw_bf16=xi[:m] if use_idx else None,
+                                nthreads=nthreads))
+        new_pend.append(None if n == m else dict(raw=x[m].copy(), logit=float(z[m]),
+                                                 idx=xi[m].copy() if use_idx else None))
+    return entries, new_pend
+
+
 def index_prefill(kcodes, kscales, row0, n_entries, qc, qs, w, q_pos, ratio, P, k, q_ids=None, nthreads=0):
     """Causal prefill indexer; q_ids selects a subset of queries (rows of the outputs)."""
     h = _Hold()

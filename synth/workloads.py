@@ -11,6 +11,10 @@ attention.  The five workloads:
                                4096-query causal prefill chunk
 * ``ragged_decode_b48_20l``  - batch 48, lengths log-uniform on [4096, 2^20],
                                20 layers (F R U R U) x 4
+* ``ratio2_decode_b64_l1m``  - as ``long_decode_b64_l1m`` over ratio-2 entries
+                               (2^20 entries = 2^21 raw tokens); each step also
+                               appends one raw token per sequence, so the
+                               caches carry spare rows
 """
 from __future__ import annotations
 
@@ -31,6 +35,8 @@ class DecodeWorkload:
     needles: int = 0
     lognormal: bool = False
     seed: int = 2026
+    ratio: int = 1      # 2: entries are compressed pairs, appended during decode
+    room: int = 0       # spare cache rows per sequence beyond its length
 
     @property
     def B(self):
@@ -42,7 +48,7 @@ class DecodeWorkload:
 
     def row_offsets(self):
         """Sequence b starts at a multiple of 8; total capacity is a multiple of 8."""
-        pad = (self.lengths + 7) // 8 * 8
+        pad = (self.lengths + self.room + 7) // 8 * 8
         off = np.concatenate([[0], np.cumsum(pad)[:-1]]).astype(np.int64)
         return off, int(pad.sum())
 
@@ -80,6 +86,8 @@ def decode_workloads():
                                               lognormal=True),
         "ragged_decode_b48_20l": DecodeWorkload("ragged_decode_b48_20l", synth.log_uniform_lengths(2026, 48),
                                                 "FRURU" * 4, needles=32),
+        "ratio2_decode_b64_l1m": DecodeWorkload("ratio2_decode_b64_l1m", np.full(64, 1 << 20), "FRRU", needles=256,
+                                                lognormal=True, ratio=2, room=1024),
     }
 
 
@@ -118,7 +126,7 @@ def full_cache_host(wl: DecodeWorkload, layer: int, q_codes, q_scales) -> dict:
     mc = np.zeros((rows, 256), np.uint8)
     msc = np.zeros((rows, 16), np.uint8)
     for b in range(wl.B):
-        n = int((wl.lengths[b] + 7) // 8 * 8)
+        n = int((wl.lengths[b] + wl.room + 7) // 8 * 8)
         nk = synth.stream_key(wl.seed, synth.T_ROWNORM, b, 0) if wl.lognormal else None
         c, s = synth.mxfp4_rows(wl.seed, synth.T_IDXK_CODES, synth.T_IDXK_SCALES, b, layer, 0, n, 128, nk)
         ic[off[b]:off[b] + n], isc[off[b]:off[b] + n] = c, s
@@ -142,7 +150,7 @@ def full_cache_device(wl: DecodeWorkload, layer: int, q_codes, q_scales, device=
     mc = torch.empty((rows, 256), dtype=torch.uint8, device=device)
     msc = torch.empty((rows, 16), dtype=torch.uint8, device=device)
     for b in range(wl.B):
-        n = int((wl.lengths[b] + 7) // 8 * 8)
+        n = int((wl.lengths[b] + wl.room + 7) // 8 * 8)
         o = int(off[b])
         sg.mxfp4_rows_into(ic[o:o + n], isc[o:o + n], wl.seed, synth.T_IDXK_CODES, synth.T_IDXK_SCALES, b, layer, 0,
                            n, 128, wl.lognormal)

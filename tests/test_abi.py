@@ -93,3 +93,26 @@ def test_workspace_sizes_grow_with_the_problem():
     # (O [16 x 512] + max + sum per head, fp32)
     assert L.csa2_sparse_attn_decode_workspace_bytes(64, 512) >= 64 * 2 * (16 * 512 + 32) * 4
     assert L.csa2_sparse_attn_decode_workspace_bytes(128, 512) > L.csa2_sparse_attn_decode_workspace_bytes(16, 512)
+
+
+def test_compress_stream_validation():
+    """csa2_compress_stream: arguments checked on the host, nothing launched."""
+    L = C.lib()
+    ws = L.csa2_compress_stream_workspace_bytes(4)
+    assert ws >= 256 + 4 * 4 and ws % 256 == 0
+    assert L.csa2_compress_stream_workspace_bytes(1000) > ws
+
+    def call(raw=FAKE, logits=FAKE, w_idx=FAKE, idx_raw=None, pend_n=FAKE, pend_raw=FAKE, pend_idx=None, B=4,
+             n_tok=4, ws_bytes=1 << 20):
+        return L.csa2_compress_stream(_cache(), _cache(), raw, logits, w_idx, idx_raw, FAKE, FAKE, FAKE, FAKE, pend_n,
+                                      pend_raw, FAKE, pend_idx, B, n_tok, 1, FAKE, ws_bytes, None)
+
+    assert call(B=0) == 0                                   # nothing to do
+    assert call(logits=None) == -1                          # logits are required
+    assert call(pend_n=None) == -1                          # pending state is required
+    assert call(w_idx=None) == -1                           # no indexer source
+    assert call(w_idx=None, idx_raw=FAKE) == -1             # idx_raw without a pending idx buffer
+    assert call(idx_raw=FAKE, pend_idx=FAKE) == -1          # both sources
+    assert call(pend_raw=FAKE + 8) == -1                    # misaligned pending row
+    assert call(raw=None) == -1                             # tokens but no raw rows
+    assert call(ws_bytes=256) == -3                         # no room for the counters

@@ -160,3 +160,73 @@ def test_decode_step_replayed_from_a_cuda_graph():
     for layer in range(len(wl.pattern)):
         assert np.array_equal(host(step.topk[layer]), eager[0][layer])
     assert np.array_equal(host(step.out), eager[1])
+
+
+def _new_tokens(seed, B, n_full, step, proj):
+    """Per Full layer: one raw bf16 token per sequence, its logit, and the
+    layer's W_idx (or a raw indexer row)."""
+    import synth
+
+    out = []
+    for f in range(n_full):
+        t = dict(raw=synth.normal_bf16(seed, synth.T_RAW, step, f, B * 512).reshape(B, 512),
+                 logit=synth.normal_f32(seed, synth.T_LOGITS, step, f, B) * 2)
+        if proj:
+            t["w_idx"] = synth.normal_f32(seed, synth.T_WIDX, 0, f, 512 * 128, log2_div=13).reshape(512, 128)
+        else:
+            t["idx_raw"] = synth.normal_bf16(seed, synth.T_IDXRAW, step, f, B * 128).reshape(B, 128)
+        out.append(t)
+    return out
+
+
+@pytest.mark.parametrize("proj", [True, False])
+def test_ratio2_decode_steps(proj):
+    """Ratio-2 decode: every step appends one raw token per sequence to each
+    Full layer's caches (an entry every second step, the odd token pending
+    on the device) and then runs the layer pattern over the grown caches.
+    Cache bytes, lengths and the last step's Top-k are bit-exact with the
+    oracle (streaming appends, then its decode step); attention within
+    tolerance."""
+    lens0 = np.array([9001, 4096, 20000, 333], np.int64)
+    room, steps, pattern = 16, 5, "FRUFR"
+    wl = W.DecodeWorkload("r2_small", lens0, pattern, needles=16, ratio=2, room=room)
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(pattern))]
+    fulls = wl.full_layers()
+    caches_h = [W.full_cache_host(wl, f, layers[f]["q_codes"], layers[f]["q_scales"]) for f in fulls]
+    caches_d = [FullCache(C.cache(dev(c["idx_codes"]), dev(c["idx_scales"])),
+                          C.cache(dev(c["main_codes"]), dev(c["main_scales"]))) for c in caches_h]
+    off = caches_h[0]["seq_row_off"]
+    off_d, len_d = dev(off), dev(lens0.astype(np.int32))
+    step = DecodeStep(pattern, wl.B, wl.max_len + room, wl.P, wl.k, ratio=2, projection=proj)
+    dl = _device_layers(layers)
+    pend = [[None] * wl.B for _ in fulls]
+    lens = lens0.copy()
+    for t in range(steps):
+        toks = _new_tokens(77, wl.B, len(fulls), t, proj)
+        step.run(caches_d, off_d, len_d, dl, new_tokens=[{k: dev(v) for k, v in tk.items()} for tk in toks])
+        # the oracle's appends into its own copies of the caches
+        tok_off = np.arange(wl.B + 1, dtype=np.int64)
+        new_lens = lens.copy()
+        for f, (c, tk) in enumerate(zip(caches_h, toks)):
+            ent, pend[f] = oracle.compress_stream(pend[f], tk["raw"], tk["logit"], tok_off, w_idx=tk.get("w_idx"),
+                                                  idx_raw_bf16=tk.get("idx_raw"))
+            for b in range(wl.B):
+                ne = ent[b][0].shape[0]
+                r0 = int(off[b] + lens[b])
+                for key, arr in zip(("main_codes", "main_scales", "idx_codes", "idx_scales"), ent[b]):
+                    c[key][r0:r0 + ne] = arr
+                new_lens[b] = lens[b] + ne
+        lens = new_lens
+    torch.cuda.synchronize()
+    assert step.device_flags() == 0
+    assert host(len_d).tolist() == lens.tolist()
+    assert lens.tolist() == (lens0 + steps // 2).tolist()
+    for c_h, c_d in zip(caches_h, caches_d):
+        for key, t in (("main_codes", c_d.main._keep[0]), ("main_scales", c_d.main._keep[1]),
+                       ("idx_codes", c_d.idx._keep[0]), ("idx_scales", c_d.idx._keep[1])):
+            assert np.array_equal(host(t), c_h[key]), key
+    ref = oracle.decode_step(pattern, caches_h, off, lens.astype(np.int32), layers, wl.P, wl.k, 1 / math.sqrt(512))
+    for layer in range(len(pattern)):
+        assert np.array_equal(host(step.topk[layer]), ref["topk"][layer]), f"layer {layer} Top-k"
+        check_attention(host(step.out[layer]), ref["out"][layer], host(step.lse[layer]), ref["lse"][layer],
+                        what=f"layer {layer}")

@@ -108,3 +108,83 @@ def test_prefill_visibility_rule(orc):
         bkey = [max(key[8 * b:min(vis, 8 * b + 8)]) for b in range(nb)]
         wp = sorted(sorted(range(nb), key=lambda b: (-bkey[b], b))[:P])
         assert pool[i].tolist() == wp + [-1] * (P - len(wp))
+
+
+# --- streaming (ratio-2 decode) appends -------------------------------------
+
+def _stream_inputs(n, seed=31):
+    bits = synth.normal_bf16(seed, synth.T_RAW, 0, 0, n * 512).reshape(n, 512)
+    ibits = synth.normal_bf16(seed, synth.T_IDXRAW, 0, 0, n * 128).reshape(n, 128)
+    z = synth.normal_f32(seed, synth.T_LOGITS, 0, 0, n) * 2
+    return bits, ibits, z
+
+
+def test_stream_chunks_equal_one_shot_append(orc):
+    """Entries are the disjoint pairs (2j, 2j+1) of the token stream, so any
+    cut of the stream into calls gives the one-shot append's bytes."""
+    n = 45
+    bits, ibits, z = _stream_inputs(n)
+    one = orc.compress(bits[:n - 1], z[:n - 1], 2, idx_raw_bf16=ibits[:n - 1])
+    rng = np.random.default_rng(5)
+    cuts = [0]
+    while cuts[-1] < n:
+        cuts.append(min(n, cuts[-1] + int(rng.integers(0, 6))))
+    pend, got = [None], [[], [], [], []]
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        ent, pend = orc.compress_stream(pend, bits[a:b], z[a:b], [0, b - a], idx_raw_bf16=ibits[a:b])
+        for part, arr in zip(got, ent[0]):
+            part.append(arr)
+    for want, part in zip(one, got):
+        assert np.array_equal(np.concatenate(part), want)
+    # n is odd: the last token is pending, bit for bit
+    assert pend[0] is not None
+    assert np.array_equal(pend[0]["raw"], bits[n - 1]) and np.array_equal(pend[0]["idx"], ibits[n - 1])
+    assert np.float32(pend[0]["logit"]) == z[n - 1]
+
+
+def test_stream_one_token_per_call_pairs_consecutive_tokens(orc):
+    """With equal logits, entry j is the average of tokens 2j and 2j+1 (the
+    pending token is the first of the pair, the new token the second)."""
+    n = 12
+    bits, ibits, _ = _stream_inputs(n, seed=32)
+    x = synth.bf16_bits_to_f32(bits).astype(np.float64)
+    z = np.zeros(n, np.float32)
+    pend, entries = [None], []
+    for t in range(n):
+        ent, pend = orc.compress_stream(pend, bits[t:t + 1], z[t:t + 1], [0, 1], idx_raw_bf16=ibits[t:t + 1])
+        assert ent[0][0].shape[0] == (t % 2)          # an entry every second token
+        assert (pend[0] is None) == (t % 2 == 1)
+        if t % 2:
+            entries.append(ent[0])
+    for j, (mc, ms, _, _) in enumerate(entries):
+        avg = np.array([[rn32(Fraction(x[2 * j, i]) / 2 + Fraction(x[2 * j + 1, i]) / 2) for i in range(512)]],
+                       np.float32)
+        wc, ws = orc.mxfp4_encode(avg)
+        assert np.array_equal(mc, wc) and np.array_equal(ms, ws)
+
+
+def test_stream_projection_and_ragged_batch(orc):
+    """Several sequences in one call, some with a pending token, some empty,
+    with the W_idx projection: per sequence equal to the one-shot append of
+    the pending token followed by the new tokens."""
+    bits, _, z = _stream_inputs(40, seed=33)
+    w_idx = synth.normal_f32(33, synth.T_WIDX, 0, 0, 512 * 128, log2_div=13).reshape(512, 128)
+    tok_off = np.array([0, 0, 1, 6, 6, 15], np.int64)
+    pend = [None, dict(raw=bits[30], logit=float(z[30]), idx=None), None,
+            dict(raw=bits[31], logit=float(z[31]), idx=None), dict(raw=bits[32], logit=float(z[32]), idx=None)]
+    ent, new = orc.compress_stream(pend, bits[:15], z[:15], tok_off, w_idx=w_idx)
+    for b in range(5):
+        t0, t1 = tok_off[b], tok_off[b + 1]
+        rows = list(range(t0, t1))
+        xs = ([bits[30 + [None, 0, None, 1, 2][b]]] if pend[b] is not None else []) + [bits[t] for t in rows]
+        zs = ([z[30 + [None, 0, None, 1, 2][b]]] if pend[b] is not None else []) + [z[t] for t in rows]
+        m = len(xs) // 2 * 2
+        if m:
+            want = orc.compress(np.stack(xs[:m]), np.array(zs[:m], np.float32), 2, w_idx=w_idx)
+            for w_, g_ in zip(want, ent[b]):
+                assert np.array_equal(w_, g_)
+        else:
+            assert ent[b][0].shape[0] == 0
+        assert (new[b] is None) == (len(xs) % 2 == 0)
+        if new[b] is not None:
+            assert np.array_equal(new[b]["raw"], xs[-1])

@@ -66,12 +66,15 @@ def algorithmic_bytes(wl):
     (the Full layer re-scores its pool for its own Top-512, each Reindex layer
     scores the pool); each attention 512*272 + 128*512 B."""
     L = wl.lengths.astype(np.int64)
-    pooled = np.minimum(wl.P * 8, (L + 7) // 8 * 8)
     n_scan = sum(1 for _, m in enumerate(wl.pattern) if m == "F")
     n_pool = sum(1 for m in wl.pattern if m in "FR")
     scan = int((L * 68).sum()) * 1  # only the first Full layer scans (default plan)
+    # a verification step scores and attends per query, but reads each
+    # sequence's indexer K once
+    Lq = wl.verify_queries()[1].astype(np.int64) if wl.queries_per_seq else L
+    pooled = np.minimum(wl.P * 8, (Lq + 7) // 8 * 8)
     pool = int((pooled * 68).sum()) * n_pool
-    attn = wl.B * (wl.k * 272 + 128 * 512) * len(wl.pattern)
+    attn = len(Lq) * (wl.k * 272 + 128 * 512) * len(wl.pattern)
     # ratio 2: per Full layer one raw token + logit per sequence, W_idx, and
     # one 340-byte entry per sequence every second step
     append = n_scan * (wl.B * (512 * 2 + 4) + 512 * 128 * 4 + wl.B * 340 // 2) if wl.ratio == 2 else 0
@@ -142,14 +145,17 @@ def oracle_sample_inputs(wl, layers, caches_dev, seqs):
     import torch
 
     off = wl.row_offsets()[0]
+    m = wl.queries_per_seq
     out = []
     for b in seqs:
         o, L = int(off[b]), int(wl.lengths[b])
         ch = [dict(idx_codes=c["idx_codes"][o:o + L].cpu().numpy(), idx_scales=c["idx_scales"][o:o + L].cpu().numpy(),
                    main_codes=c["main_codes"][o:o + L].cpu().numpy(),
                    main_scales=c["main_scales"][o:o + L].cpu().numpy()) for c in caches_dev]
-        lb = [{k: v[b:b + 1] for k, v in Ld.items()} for Ld in layers]
-        out.append((ch, L, lb))
+        rows = slice(b * m, (b + 1) * m) if m else slice(b, b + 1)
+        lb = [{k: v[rows] for k, v in Ld.items()} for Ld in layers]
+        vis = wl.verify_queries()[1][rows] if m else np.array([L], np.int32)
+        out.append((ch, vis, lb))
     torch.cuda.synchronize()
     return out
 
@@ -172,19 +178,19 @@ def time_oracle(wl, samples, nthreads, jobs=None):
                 for f in wl.full_layers()]
 
     def one(j):
-        ch, L, lb = samples[j % len(samples)]
+        ch, vis, lb = samples[j % len(samples)]
         if toks:  # ratio 2: the step's append (a pending token completes an entry)
             for t in toks:
                 pend = [dict(raw=t["raw"][0], logit=float(t["logit"][0]), idx=None)]
                 oracle.compress_stream(pend, t["raw"], t["logit"], np.array([0, 1]), w_idx=t["w_idx"], nthreads=1)
-        oracle.decode_step(wl.pattern, ch, np.array([0]), np.array([L], np.int32), lb, wl.P, wl.k,
+        oracle.decode_step(wl.pattern, ch, np.zeros(len(vis), np.int64), np.asarray(vis, np.int32), lb, wl.P, wl.k,
                            1 / math.sqrt(512), nthreads=1)
 
     n = len(samples) if jobs is None else jobs
     t0 = time.perf_counter()
     with ThreadPoolExecutor(max_workers=nthreads) as ex:
         list(ex.map(one, range(n)))
-    return time.perf_counter() - t0, n
+    return time.perf_counter() - t0, n * max(1, wl.queries_per_seq)
 
 
 # ----------------------------------------------------------------------------
@@ -193,6 +199,10 @@ def decode_config(wl, l2_bytes, sequential, graph=True):
     """The `config` object of a decode line (both arms)."""
     extra = ({"ratio": 2, "append": "one raw token per sequence per Full layer per step (csa2_compress_stream, "
                                     "W_idx projection)"} if wl.ratio == 2 else {})
+    if wl.queries_per_seq:
+        extra["queries_per_seq"] = wl.queries_per_seq
+        extra["verify"] = ("candidate i sees all entries but the last %d - i; value counts candidate queries"
+                           % (wl.queries_per_seq - 1))
     return {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len, "layers": wl.pattern, **extra,
             "pool_blocks": wl.P, "topk": wl.k, "window": 128,
             "l2": "no flush: inputs larger than L2 (%.2f GB read per step)" % (l2_bytes / 1e9),
@@ -235,8 +245,15 @@ def build_workload(wl, rank, device):
     from long_context_decode_csa2_b200.decode import FullCache
 
     wl = rank_workload(wl, rank)
-    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
-    caches_dev = [W.full_cache_device(wl, f, layers[f]["q_codes"], layers[f]["q_scales"], device)
+    m = wl.queries_per_seq
+    if m:  # one set of layer inputs per candidate query; needles aimed at each sequence's first one
+        wq = dataclasses.replace(wl, lengths=wl.verify_queries()[1].astype(np.int64), queries_per_seq=0,
+                                 seed=wl.seed + 7)
+        layers = [W.layer_inputs_host(wq, l) for l in range(len(wl.pattern))]
+    else:
+        layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    first = slice(None, None, m) if m else slice(None)
+    caches_dev = [W.full_cache_device(wl, f, layers[f]["q_codes"][first], layers[f]["q_scales"][first], device)
                   for f in wl.full_layers()]
     caches = [FullCache(C.cache(c["idx_codes"], c["idx_scales"]), C.cache(c["main_codes"], c["main_scales"]))
               for c in caches_dev]
@@ -301,8 +318,14 @@ def run_ours(args):
                                  needles=min(wl.needles, max(1, args.context // 1024)))
     wl, layers, caches_dev, caches, layers_dev, off_d, len_d = build_workload(wl, rank, device)
     C.lib()
+    m = wl.queries_per_seq
+    n_q = wl.B * m if m else wl.B  # queries per step on this rank
     step = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=not args.sequential,
-                      ratio=wl.ratio)
+                      ratio=wl.ratio, queries=n_q if m else None)
+    vq = {}
+    if m:
+        q_off_h, q_vis_h = wl.verify_queries()
+        vq = dict(q_off=torch.from_numpy(q_off_h).to(device), q_vis=torch.from_numpy(q_vis_h).to(device))
     stream = torch.cuda.current_stream()
     toks_host, toks_dev = new_token_inputs(wl, device) if wl.ratio == 2 else (None, None)
     len0 = len_d.clone()
@@ -339,7 +362,7 @@ def run_ours(args):
 
     def run_step(record=False):
         recording[0] = record
-        step.run(caches, off_d, len_d, layers_dev, new_tokens=toks_dev)
+        step.run(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
         recording[0] = False
 
     for _ in range(args.warmup):
@@ -352,7 +375,7 @@ def run_ours(args):
     # default); the per-call times come from a separate eager pass
     graph = None
     if not args.no_graph:
-        graph = step.capture(caches, off_d, len_d, layers_dev, new_tokens=toks_dev)
+        graph = step.capture(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
         for _ in range(3):
             graph.replay()
         torch.cuda.synchronize()
@@ -380,7 +403,8 @@ def run_ours(args):
             run_step(record=True)
         torch.cuda.synchronize()
     per_call = {name: sum(a.elapsed_time(b) for a, b in lst) / len(lst) for name, lst in ev_calls.items()}
-    full_ms = [a.elapsed_time(b) for a, b in ev_calls["csa2_index_full"]]
+    scan_call = "csa2_index_multi" if m else "csa2_index_full"
+    full_ms = [a.elapsed_time(b) for a, b in ev_calls[scan_call]]
     ms = max_over_ranks(ms, device, world)
 
     # end to end: host (pinned) query inputs -> device, step, outputs -> host
@@ -394,7 +418,7 @@ def run_ours(args):
     h2d += sum(t.numel() * t.element_size() for T in tok_in for t in T.values())
     full_of_layer = {l: i for i, l in enumerate(wl.full_layers())}
     out_host = torch.empty(step.out.shape, dtype=torch.float32).pin_memory()
-    top_host = torch.empty((n_layers, wl.B, wl.k), dtype=torch.int32).pin_memory()
+    top_host = torch.empty((n_layers, n_q, wl.k), dtype=torch.int32).pin_memory()
     d2h = out_host.numel() * 4 + top_host.numel() * 4
     # Inputs go in on a copy stream, one event per layer, so that later
     # layers' copies overlap the scan; each layer's output and Top-k go out on
@@ -422,7 +446,7 @@ def run_ours(args):
                         dst = toks_dev[full_of_layer[l]][k]
                         (dst.view(torch.int16) if dst.dtype == torch.bfloat16 else dst).copy_(src, non_blocking=True)
                 ev_in[l].record(h2d_stream)
-        step.run(caches, off_d, len_d, layers_dev, ready=ev_in, on_layer_done=copy_out, new_tokens=toks_dev)
+        step.run(caches, off_d, len_d, layers_dev, ready=ev_in, on_layer_done=copy_out, new_tokens=toks_dev, **vq)
         cur.wait_stream(d2h_stream)  # the step ends when its results are on the host
         cur.wait_stream(h2d_stream)
 
@@ -487,7 +511,7 @@ def run_ours(args):
         launches_per_step += len(step.pairs)  # ratio 2: one append per Full layer
         res = {
             "metric": METRIC,
-            "value": job_throughput(world, wl.B, ms),
+            "value": job_throughput(world, n_q, ms),
             "unit": "queries/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -499,15 +523,15 @@ def run_ours(args):
             "dtype": "int32+f64 indexer, f16 tensor-core attention (f32 accumulate)",
             "data": "synthetic",
             "config": decode_config(wl, ab["total"], args.sequential, graph is not None),
-            "tokens_per_s": job_throughput(world, wl.B, ms),
+            "tokens_per_s": job_throughput(world, n_q, ms),
             "hbm_algorithmic_gbs": ab["total"] / (ms * 1e-3) / 1e9,
             "hbm_frac_of_8tbs": ab["total"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
-            "roofline": {"kernel": "csa2_index_full (scan + block max + pool + Top-512)", "bound": "hbm",
+            "roofline": {"kernel": scan_call + " (scan + block max + pool + Top-512)", "bound": "hbm",
                          "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": peak_kind, "traffic": traffic, "algorithmic_bytes": full_bytes,
                          "avg_ms": full_avg},
             "cpu_baseline": cpu,
-            "e2e": {"value": job_throughput(world, wl.B, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": job_throughput(world, n_q, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "per_call_ms": per_call,
@@ -655,15 +679,24 @@ def run_reference(args):
         # no GPU to generate the full-size caches: shorter contexts (named in the config)
         small = dataclasses.replace(wl, name=wl.name + "_l65536_host", lengths=np.full(nthreads, min(wl.max_len, 65536)))
         wl = small
-        layers = [W.layer_inputs_host(small, l) for l in range(len(small.pattern))]
-        caches = [W.full_cache_host(small, f, layers[f]["q_codes"], layers[f]["q_scales"])
+        m = small.queries_per_seq
+        if m:
+            wq = dataclasses.replace(small, lengths=small.verify_queries()[1].astype(np.int64), queries_per_seq=0,
+                                     seed=small.seed + 7)
+            layers = [W.layer_inputs_host(wq, l) for l in range(len(small.pattern))]
+        else:
+            layers = [W.layer_inputs_host(small, l) for l in range(len(small.pattern))]
+        first = slice(None, None, m) if m else slice(None)
+        caches = [W.full_cache_host(small, f, layers[f]["q_codes"][first], layers[f]["q_scales"][first])
                   for f in small.full_layers()]
         samples = []
         off = small.row_offsets()[0]
         for b in range(nthreads):
             o, L = int(off[b]), int(small.lengths[b])
             ch = [{k: c[k][o:o + L] for k in ("idx_codes", "idx_scales", "main_codes", "main_scales")} for c in caches]
-            samples.append((ch, L, [{k: v[b:b + 1] for k, v in Ld.items()} for Ld in layers]))
+            rows = slice(b * m, (b + 1) * m) if m else slice(b, b + 1)
+            vis = small.verify_queries()[1][rows] if m else np.array([L], np.int32)
+            samples.append((ch, vis, [{k: v[rows] for k, v in Ld.items()} for Ld in layers]))
     # one timed step = one query (a full decode step of one sequence); the K
     # steps run nthreads at a time, so K steps take about K/nthreads queries'
     # time (about a minute for K = 400 on 8 cores)
@@ -676,8 +709,9 @@ def run_reference(args):
            "data": "synthetic", "config": decode_config(wl, algorithmic_bytes(wl)["total"], args.sequential,
                                                         not args.no_graph),
            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": nthreads, "kind": "oracle",
-                            "sample": f"{args.steps} queries (one per step) over {len(samples)} sequences of the "
-                                      f"workload, {nthreads} host threads at a time; {secs:.1f} s"},
+                            "sample": f"{nseq} queries ({max(1, wl.queries_per_seq)} per step) over "
+                                      f"{len(samples)} sequences of the workload, {nthreads} host threads at a "
+                                      f"time; {secs:.1f} s"},
            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res))
 

@@ -246,6 +246,35 @@ csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * csa2_index_multi -- Full-mode indexer for a batch of sequences with several
+ * queries each (the candidate tokens of a speculative-decoding verification
+ * step), reading every sequence's indexer K once for all of its queries.
+ * Source: [V41] hierarchical indexer (as csa2_index_full) and section
+ * "DSpark" (several draft positions per request verified in one forward,
+ * the verification length chosen per request).
+ * Sequence b owns queries q_off[b] .. q_off[b+1]-1 (ascending offsets within
+ * [0, Q]); query i sees the first q_vis[i] entries of its sequence (cache
+ * rows seq_row_off[b] ..).  Per query: the same score, block pool and Top-k
+ * as csa2_index_full over its visible entries (the pool fast path, so
+ * pool_blocks >= k).
+ *   q_codes [Q][4][64] (16-byte aligned), q_scales [Q][4][4], w [Q][4]
+ *   seq_row_off [B] int64 (multiples of 8); q_off [B+1] int32; q_vis [Q] int32
+ *   max_vis    host: upper bound of q_vis (larger values are clamped and
+ *              flagged CSA2_DEV_LENGTH)
+ *   pool_out [Q][P], topk_out [Q][k] (queries of no sequence get -1 rows)
+ *   q_row_off_out [Q] int64 or NULL: receives each query's seq_row_off, so
+ *              that csa2_index_reindex and csa2_sparse_attn_decode can take
+ *              the queries as Q segments (row offsets q_row_off_out, lengths
+ *              q_vis)
+ * ------------------------------------------------------------------------- */
+size_t csa2_index_multi_workspace_bytes(int B, int Q, int64_t max_vis, int pool_blocks, int k);
+csa2_status csa2_index_multi(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                             const float* w, const int64_t* seq_row_off, const int32_t* q_off, const int32_t* q_vis,
+                             int B, int Q, int64_t max_vis, int pool_blocks, int k, int32_t* pool_out,
+                             int32_t* topk_out, int64_t* q_row_off_out, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* ---------------------------------------------------------------------------
  * csa2_sparse_attn_prefill -- causal sparse attention of a prefill chunk.
  * Query i attends its selected entries (topk[i][j] >= 0, each < the visible
  * count of csa2_index_prefill) and the raw FP8 window rows

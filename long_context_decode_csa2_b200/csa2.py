@@ -54,6 +54,8 @@ def lib():
             "csa2_compress_append": (I, [Cache, Cache, P, P, P, P, P, P, P, P, I, I, I64, I64, P, Z, P]),
             "csa2_compress_stream_workspace_bytes": (Z, [I]),
             "csa2_compress_stream": (I, [Cache, Cache, P, P, P, P, P, P, P, P, P, P, P, P, I, I64, I64, P, Z, P]),
+            "csa2_index_multi_workspace_bytes": (Z, [I, I, I64, I, I]),
+            "csa2_index_multi": (I, [Cache, P, P, P, P, P, P, I, I, I64, I, I, P, P, P, P, Z, P]),
             "csa2_index_prefill_workspace_bytes": (Z, [I, I64, I, I]),
             "csa2_index_prefill": (I, [Cache, P, P, P, P, I, I64, I64, I, I, I, P, P, P, Z, P]),
             "csa2_sparse_attn_prefill_workspace_bytes": (Z, [I, I]),
@@ -196,6 +198,20 @@ def csa2_compress_stream(main_kv, idx_k, raw, logits, tok_off, seq_row_off, seq_
                                     _ptr(pend_n), _ptr(pend_raw), _ptr(pend_logit), _ptr(pend_idx), B, n_tok,
                                     int(max_new), wp, wn, _stream(stream))
     _check(rc, "csa2_compress_stream")
+
+
+def csa2_index_multi_workspace_bytes(B, Q, max_vis, pool_blocks, k):
+    return lib().csa2_index_multi_workspace_bytes(B, Q, max_vis, pool_blocks, k)
+
+
+def csa2_index_multi(idx_k, q_codes, q_scales, w, seq_row_off, q_off, q_vis, max_vis, pool_blocks, k, pool_out,
+                     topk_out, ws, q_row_off_out=None, stream=None):
+    B, Q = seq_row_off.shape[0], q_vis.shape[0]
+    wp, wn = _ws(ws)
+    rc = lib().csa2_index_multi(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(q_off),
+                                _ptr(q_vis), B, Q, int(max_vis), pool_blocks, k, _ptr(pool_out), _ptr(topk_out),
+                                _ptr(q_row_off_out), wp, wn, _stream(stream))
+    _check(rc, "csa2_index_multi")
 
 
 def csa2_index_prefill_workspace_bytes(T, n_entries, pool_blocks, k):

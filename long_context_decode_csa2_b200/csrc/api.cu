@@ -408,6 +408,77 @@ csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
 }
 
 // ---------------------------------------------------------------------------
+namespace {
+struct MultiWs {
+  uint32_t* status;
+  int32_t* vis;
+  int64_t* q_row_off;
+  int4* groups;
+  uint32_t* bkeys;
+  uint32_t* ckeys;
+  size_t bytes;
+};
+MultiWs multi_ws(void* ws, int B, int Q, int64_t max_vis, int P) {
+  Carve c(ws);
+  MultiWs w;
+  w.status = c.take<uint32_t>(kStatusBytes / 4);
+  w.vis = c.take<int32_t>(size_t(Q));
+  w.q_row_off = c.take<int64_t>(size_t(Q));
+  w.groups = c.take<int4>(size_t(multi_group_bound(B, Q)));
+  w.bkeys = c.take<uint32_t>(size_t(Q) * size_t(block_key_stride(max_vis)));
+  w.ckeys = c.take<uint32_t>(size_t(Q) * P * kBlk);
+  w.bytes = c.used;
+  return w;
+}
+}  // namespace
+
+size_t csa2_index_multi_workspace_bytes(int B, int Q, int64_t max_vis, int pool_blocks, int k) {
+  (void)k;
+  if (B < 0 || Q < 0 || max_vis < 0 || pool_blocks < 0) return 0;
+  return multi_ws(nullptr, B, Q, max_vis, pool_blocks).bytes;
+}
+
+csa2_status csa2_index_multi(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                             const int64_t* seq_row_off, const int32_t* q_off, const int32_t* q_vis, int B, int Q,
+                             int64_t max_vis, int pool_blocks, int k, int32_t* pool_out, int32_t* topk_out,
+                             int64_t* q_row_off_out, void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_multi";
+  if (B < 0 || Q < 0 || max_vis < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
+  if (pool_blocks < 1 || pool_blocks > CSA2_MAX_POOL_BLOCKS || k < 1 || k > CSA2_MAX_TOPK)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": pool_blocks and k must be in 1..2048");
+  if (pool_blocks < k)
+    return fail(CSA2_ERR_UNSUPPORTED, std::string(fn) + ": the multi-query indexer needs pool_blocks >= k");
+  if (Q == 0) return CSA2_OK;
+  if (B == 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": queries without sequences");
+  if (!cache_ok(idx_k) || max_vis > idx_k.rows || max_vis > INT32_MAX)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad cache or max_vis");
+  if (!q_codes || !q_scales || !w || !seq_row_off || !q_off || !q_vis || !pool_out || !topk_out || !workspace)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (!aligned16(q_codes) || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      (q_row_off_out && (reinterpret_cast<uintptr_t>(q_row_off_out) & 7)))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": q_codes must be 16-byte and workspace 256-byte aligned");
+  MultiWs ws = multi_ws(workspace, B, Q, max_vis, pool_blocks);
+  if (workspace_bytes < ws.bytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int64_t* row_off = q_row_off_out ? q_row_off_out : ws.q_row_off;
+  const int G = multi_group_bound(B, Q);
+  const int64_t nb = block_key_stride(max_vis);
+  launch_multi_prep(seq_row_off, q_off, q_vis, B, Q, G, max_vis, idx_k.rows, ws.groups, row_off, ws.vis, ws.status,
+                    st);
+  const csa2_status rc0 = launch_multi_tc(idx_k.codes, idx_k.scales, idx_k.rows, seq_row_off, ws.groups, G, ws.vis,
+                                          Q, max_vis, q_codes, q_scales, w, ws.bkeys, nb, ws.status, st);
+  if (rc0 != CSA2_OK) return rc0;
+  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, Q, 0, nullptr, pool_blocks, pool_out, nullptr, st);
+  SegDesc sd{row_off, 0, ws.vis, max_vis, idx_k.rows};
+  const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.vis, Q, q_codes, q_scales, w, pool_out,
+                                        pool_blocks, ws.ckeys, nullptr, ws.status, st);
+  if (rc != CSA2_OK) return rc;
+  launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.vis, Q, pool_blocks, pool_out, k, topk_out,
+                nullptr, st);
+  return check_launch(fn);
+}
+
+// ---------------------------------------------------------------------------
 size_t csa2_sparse_attn_prefill_workspace_bytes(int T, int k) {
   Carve c(nullptr);
   c.take<uint32_t>(kStatusBytes / 4);

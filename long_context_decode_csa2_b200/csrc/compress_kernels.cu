@@ -213,11 +213,18 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
       __syncthreads();
       const int col = threadIdx.x % kDi, grp = threadIdx.x / kDi;
       if (nvalid <= kCompGroups) {
-        // one entry per group (a decode append): a single chain per thread
+        // one entry per group (a decode append): a single chain per thread;
+        // W_idx is read 64 rows at a time, so the chain waits for one L2
+        // round trip per 64 terms rather than per few
         if (grp < nvalid) {
           double acc = 0.0;
-#pragma unroll 8
-          for (int i = 0; i < kD; ++i) acc = __fma_rn(cbuf[grp][i], double(__ldg(a.w_idx + i * kDi + col)), acc);
+          for (int i0 = 0; i0 < kD; i0 += 64) {
+            float wv[64];
+#pragma unroll
+            for (int u = 0; u < 64; ++u) wv[u] = __ldg(a.w_idx + (i0 + u) * kDi + col);
+#pragma unroll
+            for (int u = 0; u < 64; ++u) acc = __fma_rn(cbuf[grp][i0 + u], double(wv[u]), acc);
+          }
           rbuf[grp][col] = __double2float_rn(acc);
         }
       } else {

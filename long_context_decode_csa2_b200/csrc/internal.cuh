@@ -83,6 +83,19 @@ csa2_status launch_prefill_tc(const uint8_t* kcodes, const uint8_t* kscales, int
                               const uint8_t* q_scales, const float* w, uint32_t* bkeys, int64_t nb_stride,
                               uint32_t* status, cudaStream_t st);
 
+// Multi-query scan (a batch of sequences with a few queries each): the group
+// table (at most multi_group_bound(B, Q) groups of <= 8 queries of one
+// sequence), each query's first cache row and checked visible count, then
+// the block keys [Q][nb_stride] of every query on the tensor cores.
+int multi_group_bound(int B, int Q);
+void launch_multi_prep(const int64_t* seq_row_off, const int32_t* q_off, const int32_t* q_vis, int B, int Q, int G,
+                       int64_t max_vis, int64_t cache_rows, int4* groups, int64_t* q_row_off, int32_t* vis,
+                       uint32_t* status, cudaStream_t st);
+csa2_status launch_multi_tc(const uint8_t* kcodes, const uint8_t* kscales, int64_t cache_rows,
+                            const int64_t* seq_row_off, const int4* groups, int G, const int32_t* vis, int Q,
+                            int64_t max_vis, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                            uint32_t* bkeys, int64_t nb_stride, uint32_t* status, cudaStream_t st);
+
 // Visible entry counts of prefill queries.
 void launch_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entries, int32_t* vis, uint32_t* status,
                         cudaStream_t st);

@@ -26,6 +26,13 @@
 //     and write the maximum of every 8 positions as one rank key.
 // Items past the visibility of every query of a group are skipped by all
 // roles alike.  Every wait is time-bounded (CSA2_DEV_TIMEOUT on expiry).
+//
+// The same kernel serves a batch of sequences with a few queries each (the
+// candidate tokens of a speculative-decoding verification step, section
+// "DSpark" of the same page: several positions per request scored in one
+// forward): a group is then up to 8 consecutive queries of one sequence,
+// read from a group table that k_multi_prep builds, and every item loads its
+// group's own sequence rows.
 #include <algorithm>
 
 #include "device_common.cuh"
@@ -82,6 +89,8 @@ struct __align__(1024) PfSmem {
 };
 
 struct PfParams {
+  const int4* groups;       // [n_groups] {sequence, first query, queries, 0}, or null: group g = queries 8g..
+  const int64_t* seq_row_off;  // [B] first cache row of each sequence (with groups)
   const uint8_t* kscales;
   const uint8_t* q_codes;   // [T][4][64]
   const uint8_t* q_scales;  // [T][4][4]
@@ -105,18 +114,29 @@ __device__ __forceinline__ bool pf_aborted(PfSmem& sm) {
   return *reinterpret_cast<volatile int*>(&sm.abort_flag) != 0;
 }
 
-// Largest visibility among the group's queries.
-__device__ __forceinline__ int group_vis(const PfParams& p, int g) {
-  int m = 0;
-  for (int j = 0; j < kQG; ++j) {
-    const int qi = g * kQG + j;
-    if (qi < p.T) m = max(m, __ldg(p.vis + qi));
+// Queries and cache rows of group g.
+struct GroupRef {
+  int q0, nq;
+  int64_t row0;
+};
+__device__ __forceinline__ GroupRef group_ref(const PfParams& p, int g) {
+  if (p.groups) {
+    const int4 e = __ldg(p.groups + g);
+    return GroupRef{e.y, e.z, e.z > 0 ? __ldg(p.seq_row_off + e.x) : 0};
   }
+  const int q0 = g * kQG;
+  return GroupRef{q0, min(kQG, p.T - q0), p.row0};
+}
+
+// Largest visibility among the group's queries.
+__device__ __forceinline__ int group_vis(const PfParams& p, const GroupRef& gr) {
+  int m = 0;
+  for (int j = 0; j < gr.nq; ++j) m = max(m, __ldg(p.vis + gr.q0 + j));
   return m;
 }
 
 // Writes group g's B operand and scale contexts into stage s (whole warp).
-__device__ __forceinline__ void build_group(PfSmem& sm, int s, const PfParams& p, int g, int lane) {
+__device__ __forceinline__ void build_group(PfSmem& sm, int s, const PfParams& p, const GroupRef& gr, int lane) {
   uint8_t* bo = sm.bop[s];
 #pragma unroll
   for (int m = 0; m < kN * kIdxCodeBytes / 16 / 32; ++m)
@@ -127,17 +147,17 @@ __device__ __forceinline__ void build_group(PfSmem& sm, int s, const PfParams& p
   for (int m = 0; m < kN / 32; ++m) {
     const int c = lane + 32 * m;
     const int j = c >> 4, h = (c >> 2) & 3, b = c & 3;
-    const int qi = g * kQG + j;
-    if (qi < p.T) {
+    const int qi = gr.q0 + j;
+    if (j < gr.nq) {
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.q_codes + int64_t(qi) * kHi * 64 + h * 64 + b * 16));
       const int n = 16 * j + 4 * h + b;
       *reinterpret_cast<uint4*>(bo + n * 64 + ((b ^ ((n >> 1) & 3)) << 4)) = v;
     }
   }
   if (lane < kQG) {
-    const int qi = g * kQG + lane;
+    const int qi = gr.q0 + lane;
     QCtxS& q = sm.qctx[s][lane];
-    if (qi < p.T) {
+    if (lane < gr.nq) {
       make_qctx(q.c, p.q_scales + int64_t(qi) * 16, p.w + int64_t(qi) * kHi);
       q.vis = __ldg(p.vis + qi);
     } else {
@@ -196,11 +216,13 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
     if (lane < kSt) sm.built[lane] = -1;
     __syncwarp();
     int issued = 0, cg = -1, gmax = 0;
+    GroupRef gr{0, 0, 0};
     for (int it = i0; it < i1; ++it) {
       const int g = it / p.n_tiles, tile = it - g * p.n_tiles;
       if (g != cg) {
         cg = g;
-        gmax = group_vis(p, g);
+        gr = group_ref(p, g);
+        gmax = group_vis(p, gr);
       }
       if (int64_t(tile) * kPT >= gmax) continue;
       const int t = issued, s = t % kSt, round = t / kSt;
@@ -211,13 +233,13 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       }
       if (__any_sync(0xffffffffu, pf_aborted(sm))) break;
       if (sm.built[s] != g) {
-        build_group(sm, s, p, g, lane);
+        build_group(sm, s, p, gr, lane);
         if (lane == 0) sm.built[s] = g;
       }
       __syncwarp();
       if (lane == 0) {
         sm.info[s] = make_int2(g, tile);
-        const int64_t row = p.row0 + int64_t(tile) * kPT;
+        const int64_t row = gr.row0 + int64_t(tile) * kPT;
         const int64_t left = p.cache_rows - row;  // > 0 and a multiple of 8
         const uint32_t sbytes = uint32_t(left < kPT ? left : kPT) * 4u;
         sm100::mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sbytes);
@@ -242,7 +264,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
         const int g = it / p.n_tiles, tile = it - g * p.n_tiles;
         if (g != cg) {
           cg = g;
-          gmax = group_vis(p, g);
+          gmax = group_vis(p, group_ref(p, g));
         }
         if (int64_t(tile) * kPT >= gmax) continue;
         const int s = t % kSt, a = t % kAc;
@@ -277,11 +299,13 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
     const int j0 = team * kQPT;  // this team's queries of the group
     const uint32_t lane_base = uint32_t(32 * q4) << 16;
     int t = -1, cg = -1, gmax = 0;
+    GroupRef gr{0, 0, 0};
     for (int it = i0; it < i1; ++it) {
       const int g = it / p.n_tiles, tile = it - g * p.n_tiles;
       if (g != cg) {
         cg = g;
-        gmax = group_vis(p, g);
+        gr = group_ref(p, g);
+        gmax = group_vis(p, gr);
       }
       if (int64_t(tile) * kPT >= gmax) continue;
       ++t;
@@ -310,7 +334,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
         if (pos < q.vis) key = rank_key(exact_score(v[jj], ks, q.c));
         key = group8_max(key);
         if ((lane & 7) == 0 && pos < q.vis)
-          p.bkeys[int64_t(g * kQG + j) * p.nb_stride + pos / kBlk] = key;
+          p.bkeys[int64_t(gr.q0 + j) * p.nb_stride + pos / kBlk] = key;
       }
       sm100::tc_fence_before();
       __syncwarp();
@@ -329,7 +353,146 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
   }
 }
 
+// Group table and per-query rows of a batch of sequences with a few queries
+// each (one CTA of 1024 threads).  Sequence b owns queries q_off[b] ..
+// q_off[b+1]-1, cut into groups of at most 8; every query gets its
+// sequence's first row and its checked visible count (negative -> 0, above
+// max_vis -> clamped with CSA2_DEV_LENGTH, outside the cache ->
+// 0 with CSA2_DEV_ROW_LAYOUT); queries of no sequence see nothing.
+__global__ void __launch_bounds__(1024) k_multi_prep(const int64_t* seq_row_off, const int32_t* q_off,
+                                                     const int32_t* q_vis, int B, int Q, int G, int64_t max_vis,
+                                                     int64_t cache_rows, int4* groups, int64_t* q_row_off,
+                                                     int32_t* vis, uint32_t* status) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int q = threadIdx.x; q < Q; q += blockDim.x) {
+    vis[q] = 0;
+    q_row_off[q] = 0;
+  }
+  for (int g = threadIdx.x; g < G; g += blockDim.x) groups[g] = make_int4(0, 0, 0, 0);
+  if (threadIdx.x == 0) carry = 0;
+  // the offsets must be ascending within [0, Q], so that the sequences'
+  // query ranges are disjoint; otherwise no query sees anything
+  bool ok = true;
+  for (int b = threadIdx.x; b <= B; b += blockDim.x) {
+    const int32_t v = q_off[b];
+    if (v < 0 || v > Q || (b > 0 && q_off[b - 1] > v)) ok = false;
+  }
+  if (!__syncthreads_and(ok)) {
+    if (threadIdx.x == 0) set_status(status, CSA2_DEV_LENGTH);
+    return;
+  }
+  for (int base = 0; base < B; base += 1024) {
+    const int b = base + threadIdx.x;
+    int32_t q0 = 0, nq = 0;
+    if (b < B) {
+      q0 = q_off[b];
+      nq = q_off[b + 1] - q0;
+    }
+    const int32_t ng = (nq + kQG - 1) / kQG;
+    int32_t x = ng;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      const int32_t ws = warp_sums[lane];
+      int32_t z = ws;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, z, o);
+        if (lane >= o) z += y;
+      }
+      warp_sums[lane] = z - ws;
+    }
+    __syncthreads();
+    const int32_t first = carry + warp_sums[wid] + x - ng;
+    if (nq > 0) {
+      const int64_t off = seq_row_off[b];
+      for (int c = 0; c < ng; ++c) {
+        if (first + c < G) {
+          groups[first + c] = make_int4(b, q0 + kQG * c, min(kQG, nq - kQG * c), 0);
+        } else {
+          set_status(status, CSA2_DEV_LENGTH);
+        }
+      }
+      for (int i = 0; i < nq; ++i) {
+        int64_t v = q_vis[q0 + i];
+        if (v < 0) v = 0;
+        if (v > max_vis) {
+          set_status(status, CSA2_DEV_LENGTH);
+          v = max_vis;
+        }
+        if ((off & 7) != 0 || off < 0 || off + v > cache_rows) {
+          set_status(status, CSA2_DEV_ROW_LAYOUT);
+          v = 0;
+        }
+        vis[q0 + i] = int32_t(v);
+        q_row_off[q0 + i] = off;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 1023) carry = first + ng;
+    __syncthreads();
+  }
+}
+
+csa2_status launch_groups_tc(const CUtensorMap& map, PfParams& p, int64_t max_vis, cudaStream_t st) {
+  p.n_tiles = int((max_vis + kPT - 1) / kPT);
+  const int64_t n_items = int64_t(p.n_groups) * p.n_tiles;
+  if (n_items > INT32_MAX) return fail(CSA2_ERR_UNSUPPORTED, "csa2 multi-query scan: too many query tiles");
+  // more than half of the SM's shared memory, so that one CTA (and one
+  // 512-column TMEM allocation) runs per SM
+  const size_t smem = std::max<size_t>(sizeof(PfSmem) + 1024, 120 * 1024);
+  cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  const int grid = int(std::min<int64_t>(num_sms(), n_items));
+  k_prefill_tc<<<grid, kThr, smem, st>>>(map, p);
+  return CSA2_OK;
+}
+
 }  // namespace
+
+int multi_group_bound(int B, int Q) {
+  const int64_t g = (int64_t(Q) + 7 * int64_t(B)) / kQG + 1;
+  return int(std::min<int64_t>(std::max<int64_t>(g, 1), std::max(Q, 1)));
+}
+
+void launch_multi_prep(const int64_t* seq_row_off, const int32_t* q_off, const int32_t* q_vis, int B, int Q, int G,
+                       int64_t max_vis, int64_t cache_rows, int4* groups, int64_t* q_row_off, int32_t* vis,
+                       uint32_t* status, cudaStream_t st) {
+  k_multi_prep<<<1, 1024, 0, st>>>(seq_row_off, q_off, q_vis, B, Q, G, max_vis, cache_rows, groups, q_row_off, vis,
+                                   status);
+}
+
+csa2_status launch_multi_tc(const uint8_t* kcodes, const uint8_t* kscales, int64_t cache_rows,
+                            const int64_t* seq_row_off, const int4* groups, int G, const int32_t* vis, int Q,
+                            int64_t max_vis, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                            uint32_t* bkeys, int64_t nb_stride, uint32_t* status, cudaStream_t st) {
+  if (Q == 0 || max_vis == 0) return CSA2_OK;
+  CUtensorMap map;
+  const csa2_status rc = code_map(&map, kcodes, cache_rows, kPT);
+  if (rc != CSA2_OK) return rc;
+  PfParams p{};
+  p.groups = groups;
+  p.seq_row_off = seq_row_off;
+  p.kscales = kscales;
+  p.q_codes = q_codes;
+  p.q_scales = q_scales;
+  p.w = w;
+  p.vis = vis;
+  p.T = Q;
+  p.row0 = 0;
+  p.cache_rows = cache_rows;
+  p.n_groups = G;
+  p.bkeys = bkeys;
+  p.nb_stride = nb_stride;
+  p.status = status;
+  return launch_groups_tc(map, p, max_vis, st);
+}
 
 csa2_status launch_prefill_tc(const uint8_t* kcodes, const uint8_t* kscales, int64_t row0, int64_t cache_rows,
                               const int32_t* vis, int T, int64_t max_vis, const uint8_t* q_codes,
@@ -349,19 +512,10 @@ csa2_status launch_prefill_tc(const uint8_t* kcodes, const uint8_t* kscales, int
   p.row0 = row0;
   p.cache_rows = cache_rows;
   p.n_groups = (T + kQG - 1) / kQG;
-  p.n_tiles = int((max_vis + kPT - 1) / kPT);
   p.bkeys = bkeys;
   p.nb_stride = nb_stride;
   p.status = status;
-  const int64_t n_items = int64_t(p.n_groups) * p.n_tiles;
-  if (n_items > INT32_MAX) return fail(CSA2_ERR_UNSUPPORTED, "csa2_index_prefill: too many query tiles");
-  // more than half of the SM's shared memory, so that one CTA (and one
-  // 512-column TMEM allocation) runs per SM
-  const size_t smem = std::max<size_t>(sizeof(PfSmem) + 1024, 120 * 1024);
-  cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  const int grid = int(std::min<int64_t>(num_sms(), n_items));
-  k_prefill_tc<<<grid, kThr, smem, st>>>(map, p);
-  return CSA2_OK;
+  return launch_groups_tc(map, p, max_vis, st);
 }
 
 }  // namespace csa2

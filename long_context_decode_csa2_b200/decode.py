@@ -22,6 +22,13 @@ appends the new raw token of every Full layer's caches with
 ``csa2_compress_stream``: the odd token of a pair waits on the device, every
 second step completes an entry, and the sequence lengths advance in place
 before the indexer sees them.
+
+With ``queries=Q`` (speculative verification, the page's section "DSpark":
+several candidate positions per request checked in one forward) a step
+carries up to Q queries in total, a ragged number per sequence (``q_off``),
+each with its own visible entry count (``q_vis``).  The scanning Full layer
+reads every sequence's indexer K once for all of its queries
+(``csa2_index_multi``); the later calls take the queries as Q segments.
 """
 from __future__ import annotations
 
@@ -96,19 +103,28 @@ class DecodeStep:
 
     def __init__(self, pattern: str, B: int, max_len: int, P: int = 2048, k: int = 512, full_rescan: bool = False,
                  device="cuda", sm_scale: float | None = None, concurrent: bool = True, side_streams: int = 3,
-                 ratio: int = 1, projection: bool = True):
+                 ratio: int = 1, projection: bool = True, queries: int | None = None):
         if ratio not in (1, 2):
             raise ValueError("ratio must be 1 or 2")
+        if queries is not None and ratio != 1:
+            raise ValueError("verification steps take their entries as given (ratio 1 appends are the caller's)")
         self.pattern, self.B, self.max_len, self.P, self.k = pattern, B, max_len, P, k
         self.ratio = ratio
+        self.queries = queries
+        nq = B if queries is None else queries  # segments of the calls after the scan
         self.plan = layer_plan(pattern, full_rescan)
         self.sm_scale = sm_scale if sm_scale is not None else 1.0 / math.sqrt(C.MAIN_DIM)
         self.concurrent = concurrent
         dev = torch.device(device)
         nL = len(pattern)
-        self.ws_full = C.workspace(C.csa2_index_full_workspace_bytes(B, max_len, P, k), dev)
-        re_bytes = C.csa2_index_reindex_workspace_bytes(B, P, k)
-        attn_bytes = C.csa2_sparse_attn_decode_workspace_bytes(B, k)
+        if queries is None:
+            self.ws_full = C.workspace(C.csa2_index_full_workspace_bytes(B, max_len, P, k), dev)
+            self.q_row_off = None
+        else:
+            self.ws_full = C.workspace(C.csa2_index_multi_workspace_bytes(B, queries, max_len, P, k), dev)
+            self.q_row_off = torch.zeros(queries, dtype=torch.int64, device=dev)
+        re_bytes = C.csa2_index_reindex_workspace_bytes(nq, P, k)
+        attn_bytes = C.csa2_sparse_attn_decode_workspace_bytes(nq, k)
         if concurrent:
             self.ws_re = [C.workspace(re_bytes, dev) if act == "reindex" else None for _, _, _, act in self.plan]
             self.ws_attn = [C.workspace(attn_bytes, dev) for _ in range(nL)]
@@ -121,11 +137,11 @@ class DecodeStep:
             self.ws_attn = [ws_attn] * nL
         # one pool per scanning layer (a rescan must not overwrite a pool that
         # an earlier Reindex layer may still be reading)
-        self.pools = {layer: torch.full((B, P), -1, dtype=torch.int32, device=dev)
+        self.pools = {layer: torch.full((nq, P), -1, dtype=torch.int32, device=dev)
                       for layer, _, _, act in self.plan if act == "scan"}
-        self.topk = [torch.full((B, k), -1, dtype=torch.int32, device=dev) for _ in range(nL)]
-        self.out = torch.zeros((nL, B, C.Q_HEADS, C.MAIN_DIM), dtype=torch.float32, device=dev)
-        self.lse = torch.zeros((nL, B, C.Q_HEADS), dtype=torch.float32, device=dev)
+        self.topk = [torch.full((nq, k), -1, dtype=torch.int32, device=dev) for _ in range(nL)]
+        self.out = torch.zeros((nL, nq, C.Q_HEADS, C.MAIN_DIM), dtype=torch.float32, device=dev)
+        self.lse = torch.zeros((nL, nq, C.Q_HEADS), dtype=torch.float32, device=dev)
         self.scores = None
         # ratio 2: one pending-token state per Full layer's caches
         n_full = sum(1 for m in pattern if m == "F")
@@ -143,7 +159,7 @@ class DecodeStep:
             self.hook(name, phase, stream)
 
     def run(self, caches, seq_row_off, seq_len, layers, stream=None, ready=None, on_layer_done=None,
-            new_tokens=None):
+            new_tokens=None, q_off=None, q_vis=None):
         """caches: [FullCache] per Full layer; layers: per layer dict of device
         tensors q, q_codes, q_scales, w, win, win_scale, win_len.
 
@@ -155,7 +171,14 @@ class DecodeStep:
 
         new_tokens (ratio 2 only): per Full layer a dict for
         ``PairStream.append``; the appends run first, on the caller's stream,
-        and advance ``seq_len`` in place."""
+        and advance ``seq_len`` in place.
+
+        q_off [B+1], q_vis [Q] (verification steps only, device int32): the
+        queries of sequence b are q_off[b] .. q_off[b+1]-1, query i sees the
+        first q_vis[i] entries; layer inputs are then per query and seq_len
+        is not used."""
+        if (self.queries is None) != (q_off is None and q_vis is None):
+            raise ValueError("q_off / q_vis go with (and only with) a verification step")
         main = stream if stream is not None else torch.cuda.current_stream()
         if self.ratio == 2:
             if new_tokens is None or len(new_tokens) != len(self.pairs):
@@ -171,6 +194,9 @@ class DecodeStep:
             raise ValueError("new_tokens is for ratio-2 steps")
         pool, pool_ev = None, None
         last, last_ev = None, None
+        # segments of the calls after the scan: sequences, or the queries of a
+        # verification step (rows written by csa2_index_multi)
+        seg_row_off, seg_len = (seq_row_off, seq_len) if self.queries is None else (self.q_row_off, q_vis)
         side = 0
         for layer, mode, f, act in self.plan:
             L = layers[layer]
@@ -180,10 +206,17 @@ class DecodeStep:
                 if ev_ready is not None:
                     main.wait_event(ev_ready)
                 pool = self.pools[layer]
-                self._hook("csa2_index_full", "begin", main)
-                C.csa2_index_full(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len, self.max_len,
-                                  self.P, self.k, pool, self.topk[layer], self.ws_full, stream=main)
-                self._hook("csa2_index_full", "end", main)
+                if self.queries is None:
+                    self._hook("csa2_index_full", "begin", main)
+                    C.csa2_index_full(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len,
+                                      self.max_len, self.P, self.k, pool, self.topk[layer], self.ws_full, stream=main)
+                    self._hook("csa2_index_full", "end", main)
+                else:
+                    self._hook("csa2_index_multi", "begin", main)
+                    C.csa2_index_multi(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, q_off, q_vis,
+                                       self.max_len, self.P, self.k, pool, self.topk[layer], self.ws_full,
+                                       q_row_off_out=self.q_row_off, stream=main)
+                    self._hook("csa2_index_multi", "end", main)
                 last = self.topk[layer]
                 if self.concurrent:
                     self.ev_idx[layer].record(main)
@@ -199,7 +232,7 @@ class DecodeStep:
                 if self.concurrent:
                     s.wait_event(pool_ev)
                 self._hook("csa2_index_reindex", "begin", s)
-                C.csa2_index_reindex(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len, pool,
+                C.csa2_index_reindex(cache.idx, L["q_codes"], L["q_scales"], L["w"], seg_row_off, seg_len, pool,
                                      self.k, self.topk[layer], self.ws_re[layer], stream=s)
                 self._hook("csa2_index_reindex", "end", s)
                 last = self.topk[layer]
@@ -213,7 +246,7 @@ class DecodeStep:
             elif self.concurrent:  # scan: the attention runs beside the next layers
                 s.wait_event(last_ev)
             self._hook("csa2_sparse_attn_decode", "begin", s)
-            C.csa2_sparse_attn_decode(L["q"], cache.main, seq_row_off, seq_len, last, L["win"], L["win_scale"],
+            C.csa2_sparse_attn_decode(L["q"], cache.main, seg_row_off, seg_len, last, L["win"], L["win_scale"],
                                       L["win_len"], self.sm_scale, self.out[layer], self.ws_attn[layer],
                                       lse=self.lse[layer], stream=s)
             self._hook("csa2_sparse_attn_decode", "end", s)
@@ -231,7 +264,7 @@ class DecodeStep:
                 main.wait_event(ev)
         return self.out
 
-    def capture(self, caches, seq_row_off, seq_len, layers, new_tokens=None):
+    def capture(self, caches, seq_row_off, seq_len, layers, new_tokens=None, q_off=None, q_vis=None):
         """Records one step into a CUDA graph; ``graph.replay()`` then runs the
         whole step (every call, both schedules, with the same buffers) as one
         launch.  Call ``run`` once before capturing (warm-up), and do not
@@ -242,7 +275,7 @@ class DecodeStep:
         hook, self.hook = self.hook, None
         try:
             with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
-                self.run(caches, seq_row_off, seq_len, layers, new_tokens=new_tokens)
+                self.run(caches, seq_row_off, seq_len, layers, new_tokens=new_tokens, q_off=q_off, q_vis=q_vis)
         finally:
             self.hook = hook
         torch.cuda.current_stream().wait_stream(cap)

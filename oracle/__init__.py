@@ -169,6 +169,31 @@ def index_full(kcodes, kscales, qc, qs, w, seq_row_off, seq_len, P, k, want_scor
     return pool, top, sc
 
 
+def multi_query_rows(seq_row_off, q_off, q_vis):
+    """Per query of a batch with several queries per sequence: its sequence's
+    first cache row and its visible entry count (queries of no sequence: row
+    0, nothing visible)."""
+    q_vis = np.asarray(q_vis, np.int64)
+    rows = np.zeros(q_vis.shape[0], np.int64)
+    vis = np.zeros(q_vis.shape[0], np.int32)
+    for b in range(len(q_off) - 1):
+        for i in range(int(q_off[b]), int(q_off[b + 1])):
+            rows[i] = seq_row_off[b]
+            vis[i] = max(0, int(q_vis[i]))
+    return rows, vis
+
+
+def index_multi(kcodes, kscales, qc, qs, w, seq_row_off, q_off, q_vis, P, k, nthreads=0):
+    """Full-mode indexer for several queries per sequence (speculative
+    verification, "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache
+    Compression", section "DSpark"): every query is its own Full-mode query
+    over the first q_vis[i] entries of its sequence.  Returns (pool [Q,P],
+    topk [Q,k])."""
+    rows, vis = multi_query_rows(seq_row_off, q_off, q_vis)
+    pool, top, _ = index_full(kcodes, kscales, qc, qs, w, rows, vis, P, k, nthreads=nthreads)
+    return pool, top
+
+
 def index_reindex(kcodes, kscales, qc, qs, w, seq_row_off, seq_len, pool, k, nthreads=0):
     h = _Hold()
     pool = np.ascontiguousarray(pool, np.int32)

@@ -11,6 +11,9 @@ attention.  The five workloads:
                                4096-query causal prefill chunk
 * ``ragged_decode_b48_20l``  - batch 48, lengths log-uniform on [4096, 2^20],
                                20 layers (F R U R U) x 4
+* ``verify_decode_b64_l1m_m6`` - as ``long_decode_b64_l1m`` with six candidate
+                               queries per sequence (speculative verification):
+                               query i sees all entries but the last 5 - i
 * ``ratio2_decode_b64_l1m``  - as ``long_decode_b64_l1m`` over ratio-2 entries
                                (2^20 entries = 2^21 raw tokens); each step also
                                appends one raw token per sequence, so the
@@ -37,6 +40,7 @@ class DecodeWorkload:
     seed: int = 2026
     ratio: int = 1      # 2: entries are compressed pairs, appended during decode
     room: int = 0       # spare cache rows per sequence beyond its length
+    queries_per_seq: int = 0  # > 0: a verification step with this many candidate queries per sequence
 
     @property
     def B(self):
@@ -51,6 +55,14 @@ class DecodeWorkload:
         pad = (self.lengths + self.room + 7) // 8 * 8
         off = np.concatenate([[0], np.cumsum(pad)[:-1]]).astype(np.int64)
         return off, int(pad.sum())
+
+    def verify_queries(self):
+        """q_off [B+1], q_vis [Q]: candidate i of sequence b sees all of its
+        entries but the last m - 1 - i (the later candidates' own)."""
+        m = self.queries_per_seq
+        q_off = (np.arange(self.B + 1) * m).astype(np.int32)
+        q_vis = (np.repeat(self.lengths, m) - (m - 1 - np.tile(np.arange(m), self.B))).astype(np.int32)
+        return q_off, q_vis
 
     def full_layers(self):
         return [i for i, m in enumerate(self.pattern) if m == "F"]
@@ -86,6 +98,8 @@ def decode_workloads():
                                               lognormal=True),
         "ragged_decode_b48_20l": DecodeWorkload("ragged_decode_b48_20l", synth.log_uniform_lengths(2026, 48),
                                                 "FRURU" * 4, needles=32),
+        "verify_decode_b64_l1m_m6": DecodeWorkload("verify_decode_b64_l1m_m6", np.full(64, 1 << 20), "FRRU",
+                                                   needles=256, lognormal=True, queries_per_seq=6),
         "ratio2_decode_b64_l1m": DecodeWorkload("ratio2_decode_b64_l1m", np.full(64, 1 << 20), "FRRU", needles=256,
                                                 lognormal=True, ratio=2, room=1024),
     }

@@ -230,3 +230,100 @@ def test_ratio2_decode_steps(proj):
         assert np.array_equal(host(step.topk[layer]), ref["topk"][layer]), f"layer {layer} Top-k"
         check_attention(host(step.out[layer]), ref["out"][layer], host(step.lse[layer]), ref["lse"][layer],
                         what=f"layer {layer}")
+
+
+def _verify_case(lens, m_per_seq, pattern, needles=16, lognormal=False, seqs_checked=None):
+    """A verification step: sequence b carries m_per_seq[b] candidate queries
+    whose entries are already in its cache; candidate i sees all but the
+    last m_b - 1 - i entries."""
+    wl = W.DecodeWorkload("verify_small", np.asarray(lens), pattern, needles=needles, lognormal=lognormal)
+    m = np.asarray(m_per_seq)
+    q_off = np.concatenate([[0], np.cumsum(m)]).astype(np.int32)
+    q_vis = np.concatenate([wl.lengths[b] - (m[b] - 1 - np.arange(m[b])) for b in range(wl.B)]).astype(np.int32)
+    Q = int(q_off[-1])
+    wq = W.DecodeWorkload("verify_small_q", q_vis.astype(np.int64), pattern, seed=wl.seed + 7)
+    layers = [W.layer_inputs_host(wq, l) for l in range(len(pattern))]
+    return wl, q_off, q_vis, Q, layers
+
+
+def test_verify_step_ragged_queries():
+    """Speculative verification: 6, 0, 3 and 9 candidate queries on four
+    sequences (9 spans two query groups of the scan); Top-k bit-exact and
+    attention within tolerance against the oracle's step over the queries
+    as their own segments."""
+    wl, q_off, q_vis, Q, layers = _verify_case([9001, 4096, 20000, 333], [6, 0, 3, 9], "FRUFR")
+    fulls = wl.full_layers()
+    first = np.minimum(q_off[:-1], Q - 1)  # needles aimed at each sequence's first query
+    caches_h = [W.full_cache_host(wl, f, layers[f]["q_codes"][first], layers[f]["q_scales"][first]) for f in fulls]
+    caches_d = [FullCache(C.cache(dev(c["idx_codes"]), dev(c["idx_scales"])),
+                          C.cache(dev(c["main_codes"]), dev(c["main_scales"]))) for c in caches_h]
+    off = caches_h[0]["seq_row_off"]
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, queries=Q)
+    step.run(caches_d, dev(off), None, _device_layers(layers), q_off=dev(q_off), q_vis=dev(q_vis))
+    torch.cuda.synchronize()
+    assert step.device_flags() == 0
+    rows, vis = oracle.multi_query_rows(off, q_off, q_vis)
+    assert np.array_equal(host(step.q_row_off), rows)
+    ref = oracle.decode_step(wl.pattern, caches_h, rows, vis, layers, wl.P, wl.k, 1 / math.sqrt(512))
+    for layer in range(len(wl.pattern)):
+        assert np.array_equal(host(step.topk[layer]), ref["topk"][layer]), f"layer {layer} Top-k"
+        check_attention(host(step.out[layer]), ref["out"][layer], host(step.lse[layer]), ref["lse"][layer],
+                        what=f"layer {layer}")
+    assert np.array_equal(host(step.pool), ref["pools"][max(ref["pools"])])
+
+
+def test_verify_index_multi_matches_oracle_and_single_queries():
+    """csa2_index_multi alone: equal to the oracle, and to csa2_index_full
+    run once per query (the same sequence repeated as a segment)."""
+    wl, q_off, q_vis, Q, layers = _verify_case([70000, 8, 131072], [5, 2, 8], "F", needles=8)
+    first = np.minimum(q_off[:-1], Q - 1)
+    c = W.full_cache_host(wl, 0, layers[0]["q_codes"][first], layers[0]["q_scales"][first])
+    idx = C.cache(dev(c["idx_codes"]), dev(c["idx_scales"]))
+    L = layers[0]
+    pool = torch.full((Q, wl.P), -1, dtype=torch.int32, device="cuda")
+    top = torch.full((Q, wl.k), -1, dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_index_multi_workspace_bytes(wl.B, Q, wl.max_len, wl.P, wl.k))
+    C.csa2_index_multi(idx, dev(L["q_codes"]), dev(L["q_scales"]), dev(L["w"]), dev(c["seq_row_off"]), dev(q_off),
+                       dev(q_vis), wl.max_len, wl.P, wl.k, pool, top, ws)
+    torch.cuda.synchronize()
+    assert C.device_status(ws) == 0
+    want_p, want_t = oracle.index_multi(c["idx_codes"], c["idx_scales"], L["q_codes"], L["q_scales"], L["w"],
+                                        c["seq_row_off"], q_off, q_vis, wl.P, wl.k)
+    assert np.array_equal(host(pool), want_p) and np.array_equal(host(top), want_t)
+    rows, vis = oracle.multi_query_rows(c["seq_row_off"], q_off, q_vis)
+    pool1 = torch.full((Q, wl.P), -1, dtype=torch.int32, device="cuda")
+    top1 = torch.full((Q, wl.k), -1, dtype=torch.int32, device="cuda")
+    ws1 = C.workspace(C.csa2_index_full_workspace_bytes(Q, wl.max_len, wl.P, wl.k))
+    C.csa2_index_full(idx, dev(L["q_codes"]), dev(L["q_scales"]), dev(L["w"]), dev(rows), dev(vis), wl.max_len, wl.P,
+                      wl.k, pool1, top1, ws1)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(pool1), host(pool)) and np.array_equal(host(top1), host(top))
+
+
+def test_verify_step_full_size_sampled():
+    """B = 64, L = 2^20, six candidate queries per sequence, F R R U: the
+    whole batch runs on the GPU; the queries of two sequences are recomputed
+    by the oracle."""
+    base = W.decode_workloads()["long_decode_b64_l1m"]
+    m = 6
+    wl, q_off, q_vis, Q, layers = _verify_case(base.lengths, [m] * base.B, base.pattern, needles=base.needles,
+                                               lognormal=True)
+    c = W.full_cache_device(wl, 0, layers[0]["q_codes"][::m], layers[0]["q_scales"][::m])
+    cache = FullCache(C.cache(c["idx_codes"], c["idx_scales"]), C.cache(c["main_codes"], c["main_scales"]))
+    off = c["seq_row_off"]
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, queries=Q)
+    step.run([cache], dev(off), None, _device_layers(layers), q_off=dev(q_off), q_vis=dev(q_vis))
+    torch.cuda.synchronize()
+    assert step.device_flags() == 0
+    for b in (0, 41):
+        o = int(off[b])
+        Lb = int(wl.lengths[b])
+        ch = dict(idx_codes=host(c["idx_codes"][o:o + Lb]), idx_scales=host(c["idx_scales"][o:o + Lb]),
+                  main_codes=host(c["main_codes"][o:o + Lb]), main_scales=host(c["main_scales"][o:o + Lb]))
+        qs = slice(int(q_off[b]), int(q_off[b + 1]))
+        lb = [{k: v[qs] for k, v in L_.items()} for L_ in layers]
+        ref = oracle.decode_step(wl.pattern, [ch], np.zeros(m, np.int64), q_vis[qs], lb, wl.P, wl.k,
+                                 1 / math.sqrt(512))
+        for layer in range(len(wl.pattern)):
+            assert np.array_equal(host(step.topk[layer][qs]), ref["topk"][layer]), (b, layer)
+            check_attention(host(step.out[layer][qs]), ref["out"][layer], what=f"seq {b} layer {layer}")

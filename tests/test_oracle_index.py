@@ -155,3 +155,44 @@ def test_needles_always_selected(orc):
     pool, top, _ = orc.index_full(kc, ks, qc[0][None], qc[1][None], w[None], np.array([0]), np.array([L]), 256, 512)
     assert set(pos.tolist()) <= set(top[0].tolist())
     assert set((pos // 8).tolist()) <= set(pool[0].tolist())
+
+
+def test_index_multi_each_query_sees_its_own_prefix(orc):
+    """Several queries per sequence (speculative verification): query i of
+    sequence b ranks exactly the first q_vis[i] entries of b, checked by
+    brute force (scores of those entries, full sort); queries of no sequence
+    select nothing."""
+    rng = np.random.default_rng(15)
+    L, P, k = 300, 16, 8
+    kc, ks = _rand_rows(rng, 3 * 304, 128, 125, 127)
+    seq_row_off = np.array([0, 304, 608], np.int64)
+    q_off = np.array([0, 3, 3, 7], np.int32)            # 3 queries, none, 4 queries; query 7 belongs to none
+    q_vis = np.array([L, L - 1, 5, 299, 300, 64, 1, 200], np.int32)
+    Q = len(q_vis)
+    qs_ = [_rand_query(rng, 125, 127) for _ in range(Q)]
+    qc = np.stack([q[0] for q in qs_])
+    qsc = np.stack([q[1] for q in qs_])
+    w = np.stack([q[2] for q in qs_])
+    pool, top = orc.index_multi(kc, ks, qc, qsc, w, seq_row_off, q_off, q_vis, P, k)
+    owner = [0, 0, 0, 2, 2, 2, 2, None]
+    for i in range(Q):
+        if owner[i] is None:
+            assert (top[i] == -1).all() and (pool[i] == -1).all()
+            continue
+        r0, v = int(seq_row_off[owner[i]]), int(q_vis[i])
+        bp, bt, _ = _brute_full(orc, kc[r0:], ks[r0:], qc[i], qsc[i], w[i], v, P, k)
+        assert pool[i].tolist() == bp and top[i].tolist() == bt, i
+
+
+def test_index_multi_one_query_per_sequence_is_index_full(orc):
+    rng = np.random.default_rng(16)
+    B, L = 4, 512
+    kc, ks = _rand_rows(rng, B * L, 128, 124, 128)
+    qc = rng.integers(0, 256, (B, 4, 64), dtype=np.uint8)
+    qsc = rng.integers(124, 129, (B, 4, 4), dtype=np.uint8)
+    w = (0.5 + rng.random((B, 4))).astype(np.float32)
+    off = np.arange(B, dtype=np.int64) * L
+    lens = np.array([512, 17, 400, 256], np.int32)
+    pool_f, top_f, _ = orc.index_full(kc, ks, qc, qsc, w, off, lens, 64, 32)
+    pool_m, top_m = orc.index_multi(kc, ks, qc, qsc, w, off, np.arange(B + 1, dtype=np.int32), lens, 64, 32)
+    assert np.array_equal(pool_f, pool_m) and np.array_equal(top_f, top_m)

@@ -398,6 +398,30 @@ def run_ours(args):
         dist.barrier()
     ms = t0.elapsed_time(t1) / args.steps
     reset_lengths()
+    # the same step with every call in layer order on one stream (the order a
+    # model whose layer inputs depend on the previous layer would impose),
+    # also replayed from a graph
+    seq_ms = None
+    if graph is not None and not args.sequential:
+        step_seq = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=False, ratio=wl.ratio,
+                              queries=n_q if m else None)
+        step_seq.run(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
+        g_seq = step_seq.capture(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
+        for _ in range(3):
+            g_seq.replay()
+        reset_lengths()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            g_seq.replay()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        seq_ms = max_over_ranks(s0.elapsed_time(s1) / args.steps, device, world)
+        if step_seq.device_flags():
+            raise RuntimeError("device status flags set in the layer-order step")
+        del g_seq, step_seq
+        reset_lengths()
     if graph is not None:
         for _ in range(min(args.steps, 50)):
             run_step(record=True)
@@ -535,6 +559,8 @@ def run_ours(args):
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "per_call_ms": per_call,
+            "layer_order_graph": (None if seq_ms is None else
+                                  {"ms_per_step": seq_ms, "queries_per_s": job_throughput(world, n_q, seq_ms)}),
             "clocks": clk.summary(),
             "device_flags": flags,
         }

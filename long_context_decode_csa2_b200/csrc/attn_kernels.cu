@@ -61,7 +61,8 @@ size_t attn_partial_bytes(int S, int k) {
 struct AttnSmem {
   __half q[kHq][kQS];
   __half kv[kChunk][kQS];
-  __half p[kHq][kPS];
+  __half p[kHq][kPS];                    // softmax weights, fp16 head ...
+  __half plo[kHq][kPS];                  // ... and the fp16 rest (p - head)
   union {
     uint8_t main[kChunk][kRawMain];
     uint8_t win[kWinRows][kRawWin];
@@ -338,10 +339,16 @@ __device__ __forceinline__ void chunk_update(const AttnArgs& a, AttnSmem& sm, fl
     const int hh = j >> 1;
     const float p0 = (mnew[hh] == -INFINITY) ? 0.0f : __expf(sv[j] - mnew[hh]);
     const float p1 = (mnew[hh] == -INFINITY) ? 0.0f : __expf(sv[j + 1] - mnew[hh]);
+    // p = head + rest, both fp16 (the rest is exact in fp32); P V runs on
+    // both, so the weights carry about 22 bits and the sum uses exactly the
+    // weights the MMAs see
     const __half2 ph = __floats2half2_rn(p0, p1);
-    const float2 pr = __half22float2(ph);  // the sum uses the rounded fp16 weights
-    sum[hh] += pr.x + pr.y;
+    const float2 pr = __half22float2(ph);
+    const __half2 pl = __floats2half2_rn(p0 - pr.x, p1 - pr.y);
+    const float2 plr = __half22float2(pl);
+    sum[hh] += (pr.x + plr.x) + (pr.y + plr.y);
     *reinterpret_cast<__half2*>(&sm.p[g + 8 * hh][8 * warp + 2 * t]) = ph;
+    *reinterpret_cast<__half2*>(&sm.plo[g + 8 * hh][8 * warp + 2 * t]) = pl;
   }
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
@@ -381,14 +388,17 @@ __device__ __forceinline__ void chunk_update(const AttnArgs& a, AttnSmem& sm, fl
     const int vc = 8 * (lane >> 4);                     // dim offset within the n-tile pair
     const int kend = (nkeys + 15) & ~15;
     for (int k0 = 0; k0 < kend; k0 += 16) {
-      uint32_t af[4];
+      uint32_t af[4], al[4];
       ldsm_x4(af, &sm.p[pr_][k0 + pc]);
+      ldsm_x4(al, &sm.plo[pr_][k0 + pc]);
 #pragma unroll
       for (int np = 0; np < 4; ++np) {
         uint32_t bf[4];
         ldsm_x4_t(bf, &sm.kv[k0 + vr][64 * warp + 16 * np + vc]);
         mma16816(oacc[2 * np], af, bf[0], bf[1]);
         mma16816(oacc[2 * np + 1], af, bf[2], bf[3]);
+        mma16816(oacc[2 * np], al, bf[0], bf[1]);
+        mma16816(oacc[2 * np + 1], al, bf[2], bf[3]);
       }
     }
   }

@@ -47,11 +47,23 @@ __host__ __device__ inline int attn_main_chunks(int k) { return (k + kChunk - 1)
 
 int attn_num_chunks(int k) { return attn_main_chunks(k) + kWinChunks; }
 
+// CTAs per segment: the R that minimises (waves of S*R CTAs, two per SM) x
+// (chunks per CTA), the fewest CTAs among equals (fewer partials to merge).
 int attn_splits(int S, int k) {
-  const int slots = 2 * num_sms();  // two CTAs per SM
-  int r = S > 0 ? slots / S : 1;
-  r = std::min(r, std::min(kMaxSplits, attn_num_chunks(k)));
-  return std::max(r, 1);
+  if (S <= 0) return 1;
+  const int64_t slots = 2 * int64_t(num_sms());  // two CTAs per SM
+  const int nch = attn_num_chunks(k);
+  int best = 1;
+  int64_t best_cost = INT64_MAX;
+  for (int r = 1; r <= std::min(kMaxSplits, nch); ++r) {
+    const int64_t waves = (int64_t(S) * r + slots - 1) / slots;
+    const int64_t cost = waves * ((nch + r - 1) / r);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = r;
+    }
+  }
+  return best;
 }
 
 size_t attn_partial_bytes(int S, int k) {

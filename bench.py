@@ -569,6 +569,42 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def prefill_cpu_baseline(pw, seed, nthreads, nq=64, n_comp=8192):
+    """The oracle's prefill step estimated from a bounded sample: the
+    indexer and attention of `nq` queries spread over the chunk (each sees
+    about 131072 entries) and the compression of `n_comp` raw tokens (W_idx
+    projection), scaled to T queries and n_raw tokens.  The oracle's cache
+    rows are drawn by the input generator, not taken from the GPU."""
+    import oracle
+    import synth
+
+    n_raw, T, ratio, P, k = pw.n_raw, pw.T, pw.ratio, pw.P, pw.k
+    n_ent = n_raw // ratio
+    ic, isc = synth.mxfp4_rows(seed, synth.T_IDXK_CODES, synth.T_IDXK_SCALES, 0, 0, 0, n_ent, 128)
+    mc, msc = synth.mxfp4_rows(seed, synth.T_MAIN_CODES, synth.T_MAIN_SCALES, 0, 0, 0, n_ent, 512)
+    raw_win = synth.e4m3_rows(seed, synth.T_RAWWIN, 0, 0, 0, n_raw)
+    q_pos = np.linspace(n_raw - T, n_raw - 1, nq).astype(np.int32)
+    qc, qs = synth.mxfp4_rows(seed, synth.T_QIDX_CODES, synth.T_QIDX_SCALES, 0, 0, 0, nq * 4, 128)
+    qc, qs = qc.reshape(nq, 4, 64), qs.reshape(nq, 4, 4)
+    w = synth.head_weights(seed, 0, 0, nq * 4).reshape(nq, 4)
+    q = synth.normal_bf16(seed, synth.T_Q, 0, 0, nq * 16 * 512).reshape(nq, 16, 512)
+    raw = synth.normal_bf16(seed, synth.T_RAW, 0, 0, n_comp * 512).reshape(n_comp, 512)
+    z = synth.normal_f32(seed, synth.T_LOGITS, 0, 0, n_comp)
+    w_idx = synth.normal_f32(seed, synth.T_WIDX, 0, 0, 512 * 128, log2_div=13).reshape(512, 128)
+    t0 = time.perf_counter()
+    _, top = oracle.index_prefill(ic, isc, 0, n_ent, qc, qs, w, q_pos, ratio, P, k, nthreads=nthreads)
+    oracle.attn_prefill(q, q_pos, mc, msc, 0, n_ent, ratio, top, raw_win, float(synth.window_scale(seed, 0, 0)),
+                        1 / math.sqrt(512), nthreads=nthreads)
+    t1 = time.perf_counter()
+    oracle.compress(raw, z, ratio, w_idx=w_idx, nthreads=nthreads)
+    t2 = time.perf_counter()
+    est = (t1 - t0) * T / nq + (t2 - t1) * n_raw / n_comp
+    return {"value": T / est, "unit": "queries/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"indexer + attention of {nq} of the {T} queries ({t1 - t0:.1f} s) and compression of "
+                      f"{n_comp} of the {n_raw} raw tokens ({t2 - t1:.1f} s), scaled to one whole prefill step "
+                      f"({est:.0f} s)"}
+
+
 def run_prefill(args):
     """Prefill workload: ratio-2 compression of n_raw tokens into a fresh
     cache (with the W_idx projection), the causal indexer for T queries, and
@@ -667,6 +703,44 @@ def run_prefill(args):
         torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, device, world)
     per_call = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) for n, v in times.items()}
+
+    # end to end: every input of the step from pinned host memory (raw tokens,
+    # logits, queries and their indexer inputs, the raw FP8 window rows), the
+    # outputs (attention output, Top-k) back to the host
+    host_in = {name: t.cpu().pin_memory() for name, t in (("raw", raw), ("logits", logits), ("q", q),
+                                                          ("q_codes", q_codes), ("q_scales", q_scales), ("w", w),
+                                                          ("raw_win", raw_win))}
+    dev_in = {"raw": raw, "logits": logits, "q": q, "q_codes": q_codes, "q_scales": q_scales, "w": w,
+              "raw_win": raw_win}
+    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    top_h = torch.empty(top.shape, dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = out_h.numel() * 4 + top_h.numel() * 4
+    e_steps = max(1, min(args.e2e_steps, 10))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        for name, src in host_in.items():
+            dev_in[name].copy_(src, non_blocking=True)
+        step(False)
+        out_h.copy_(out, non_blocking=True)
+        top_h.copy_(top, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, device, world)
+
+    # roofline of the indexer (the dominant call): the causal FP4 score GEMM's
+    # useful FLOPs against the FP4 tensor peak (measured bf16 x the nominal
+    # fp4 / bf16 ratio of 4); its time is the exact epilogue's, not the MMAs'
+    n_vis = np.minimum(np.arange(n_raw - T, n_raw, dtype=np.int64) + 1, n_raw) // ratio
+    flops = float(n_vis.sum()) * 4 * 128 * 2
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    bf16 = float(json.load(open(pk))["bf16_tflops"]) if os.path.exists(pk) else 1590.0
+    achieved = flops / (per_call["csa2_index_prefill"] * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = prefill_cpu_baseline(pw, seed, min(os.cpu_count() or 1, 8))
     if rank == 0:
         print(json.dumps({
             "metric": "prefill queries/sec (ratio-2 compression of 262144 tokens, 4096-query causal chunk)",
@@ -677,6 +751,17 @@ def run_prefill(args):
             "config": {"workload": pw.name, "raw_tokens": n_raw, "entries": n_ent, "queries": T, "pool_blocks": P,
                        "topk": k, "window": 128},
             "compress_tokens_per_s": n_raw / (per_call["csa2_compress_append"] * 1e-3),
+            "roofline": {"kernel": "csa2_index_prefill (causal FP4 score GEMM + block max + pool + Top-512)",
+                         "bound": "tensor", "achieved": achieved, "peak": 4 * bf16, "unit": "TFLOP/s",
+                         "frac": achieved / (4 * bf16),
+                         "peak_kind": "measured bf16 x 4 (nominal fp4 / bf16)" if os.path.exists(pk) else "fallback",
+                         "traffic": None, "note": "bound in fact by the exact CUDA-core epilogue"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": job_throughput(world, T, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            # compress 1; indexer: visibility, scan, pool select, pool scoring, Top-k select; attention:
+            # visibility, attention
+            "gpu_launches": 8 * args.steps,
             "per_call_ms": per_call, "clocks": clk.summary(), "device_flags": flags}))
     if world > 1:
         dist.destroy_process_group()

@@ -146,12 +146,19 @@ def oracle_sample_inputs(wl, layers, caches_dev, seqs):
 
     off = wl.row_offsets()[0]
     m = wl.queries_per_seq
+    table = wl.page_table() if wl.page_rows else None
     out = []
     for b in seqs:
         o, L = int(off[b]), int(wl.lengths[b])
-        ch = [dict(idx_codes=c["idx_codes"][o:o + L].cpu().numpy(), idx_scales=c["idx_scales"][o:o + L].cpu().numpy(),
-                   main_codes=c["main_codes"][o:o + L].cpu().numpy(),
-                   main_scales=c["main_scales"][o:o + L].cpu().numpy()) for c in caches_dev]
+        if table is None:
+            rows = slice(o, o + L)
+        else:  # the sequence's rows through its page table
+            t = np.arange(L, dtype=np.int64)
+            rows = torch.from_numpy(table[b][t // wl.page_rows].astype(np.int64) * wl.page_rows
+                                    + t % wl.page_rows).to(caches_dev[0]["idx_codes"].device)
+        ch = [dict(idx_codes=c["idx_codes"][rows].cpu().numpy(), idx_scales=c["idx_scales"][rows].cpu().numpy(),
+                   main_codes=c["main_codes"][rows].cpu().numpy(),
+                   main_scales=c["main_scales"][rows].cpu().numpy()) for c in caches_dev]
         rows = slice(b * m, (b + 1) * m) if m else slice(b, b + 1)
         lb = [{k: v[rows] for k, v in Ld.items()} for Ld in layers]
         vis = wl.verify_queries()[1][rows] if m else np.array([L], np.int32)
@@ -199,6 +206,8 @@ def decode_config(wl, l2_bytes, sequential, graph=True):
     """The `config` object of a decode line (both arms)."""
     extra = ({"ratio": 2, "append": "one raw token per sequence per Full layer per step (csa2_compress_stream, "
                                     "W_idx projection)"} if wl.ratio == 2 else {})
+    if wl.page_rows:
+        extra["paged"] = "%d-row pages, page table shuffled over the whole cache pool" % wl.page_rows
     if wl.queries_per_seq:
         extra["queries_per_seq"] = wl.queries_per_seq
         extra["verify"] = ("candidate i sees all entries but the last %d - i; value counts candidate queries"
@@ -267,7 +276,13 @@ def build_workload(wl, rank, device):
     keys = ("q", "q_codes", "q_scales", "w", "win", "win_scale", "win_len")
     layers_dev = [{k: to_dev(L[k]) for k in keys} for L in layers]
     off = caches_dev[0]["seq_row_off"]
-    return wl, layers, caches_dev, caches, layers_dev, to_dev(off), to_dev(wl.lengths.astype(np.int32))
+    if wl.page_rows:  # the same cache pool read through a shuffled page table
+        from long_context_decode_csa2_b200 import csa2 as C2
+
+        off_d = C2.PageTable(to_dev(wl.page_table()), wl.page_rows)
+    else:
+        off_d = to_dev(off)
+    return wl, layers, caches_dev, caches, layers_dev, off_d, to_dev(wl.lengths.astype(np.int32))
 
 
 def new_token_inputs(wl, device):

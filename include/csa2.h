@@ -246,6 +246,48 @@ csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Paged caches: csa2_index_full_paged, csa2_index_reindex_paged,
+ * csa2_sparse_attn_decode_paged, csa2_compress_stream_paged.
+ * The same operations, results and errors as the calls without the suffix,
+ * for caches kept as fixed-size pages (a serving engine's block tables)
+ * instead of one contiguous row range per sequence.  Position t of sequence
+ * b lives at cache row
+ *     pages[b * max_pages + t / page_rows] * page_rows + t % page_rows
+ * (in every cache the call touches, all sharing the page table).
+ *   pages      [B][max_pages] int32 physical page ids (4-byte aligned); the
+ *              entries for positions >= the sequence's length are not read
+ *   page_rows  host: rows per page, a power of two in [512, 2^24] (one scan
+ *              work item of 512 rows never crosses a page)
+ *   max_pages  host: row stride of `pages` (>= 1); a length above
+ *              max_pages * page_rows empties the sequence and sets
+ *              CSA2_DEV_ROW_LAYOUT
+ * Every cache's `rows` must be a multiple of page_rows.  A page id outside
+ * the cache sets CSA2_DEV_ROW_LAYOUT and reads (or writes) page 0 instead,
+ * so no access leaves the cache.
+ * ------------------------------------------------------------------------- */
+csa2_status csa2_index_full_paged(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                  const float* w, const int32_t* pages, int page_rows, int max_pages,
+                                  const int32_t* seq_len, int B, int max_len, int pool_blocks, int k,
+                                  int32_t* pool_out, int32_t* topk_out, float* scores_out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+csa2_status csa2_index_reindex_paged(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                     const float* w, const int32_t* pages, int page_rows, int max_pages,
+                                     const int32_t* seq_len, const int32_t* pool, int B, int pool_blocks, int k,
+                                     int32_t* topk_out, void* workspace, size_t workspace_bytes, void* stream);
+csa2_status csa2_sparse_attn_decode_paged(const uint16_t* q, csa2_mxfp4_cache main_kv, const int32_t* pages,
+                                          int page_rows, int max_pages, const int32_t* seq_len, const int32_t* topk,
+                                          int k, const uint8_t* win, const float* win_scale, const int32_t* win_len,
+                                          float sm_scale, float* out, float* lse, int B, void* workspace,
+                                          size_t workspace_bytes, void* stream);
+csa2_status csa2_compress_stream_paged(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k, const uint16_t* raw,
+                                       const float* logits, const float* w_idx, const uint16_t* idx_raw,
+                                       const int64_t* tok_off, const int32_t* pages, int page_rows, int max_pages,
+                                       const int32_t* seq_len_in, int32_t* seq_len_out, int32_t* pend_n,
+                                       uint16_t* pend_raw, float* pend_logit, uint16_t* pend_idx, int B,
+                                       int64_t n_tok, int64_t max_new, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
+/* ---------------------------------------------------------------------------
  * csa2_index_multi -- Full-mode indexer for a batch of sequences with several
  * queries each (the candidate tokens of a speculative-decoding verification
  * step), reading every sequence's indexer K once for all of its queries.

@@ -31,6 +31,20 @@ class MXFP4Cache(C.Structure):
     _fields_ = [("codes", C.c_void_p), ("scales", C.c_void_p), ("rows", C.c_int64)]
 
 
+class PageTable:
+    """Paged cache layout: ``pages`` [B, max_pages] int32 CUDA tensor of page
+    ids, ``page_rows`` rows per page (a power of two, >= 512).  Pass it where a
+    call takes ``seq_row_off``; the ``*_paged`` entry point is used then."""
+
+    def __init__(self, pages: torch.Tensor, page_rows: int):
+        assert pages.dtype == torch.int32 and pages.dim() == 2
+        self.pages, self.page_rows = pages, int(page_rows)
+
+    @property
+    def max_pages(self):
+        return self.pages.shape[1]
+
+
 def lib():
     """Load (building first if the sources are newer) the CUDA library."""
     global _lib
@@ -56,6 +70,11 @@ def lib():
             "csa2_compress_stream": (I, [Cache, Cache, P, P, P, P, P, P, P, P, P, P, P, P, I, I64, I64, P, Z, P]),
             "csa2_index_multi_workspace_bytes": (Z, [I, I, I64, I, I]),
             "csa2_index_multi": (I, [Cache, P, P, P, P, P, P, I, I, I64, I, I, P, P, P, P, Z, P]),
+            "csa2_index_full_paged": (I, [Cache, P, P, P, P, I, I, P, I, I, I, I, P, P, P, P, Z, P]),
+            "csa2_index_reindex_paged": (I, [Cache, P, P, P, P, I, I, P, P, I, I, I, P, P, Z, P]),
+            "csa2_sparse_attn_decode_paged": (I, [P, Cache, P, I, I, P, P, I, P, P, P, F, P, P, I, P, Z, P]),
+            "csa2_compress_stream_paged": (I, [Cache, Cache, P, P, P, P, P, P, I, I, P, P, P, P, P, P, I, I64, I64, P,
+                                               Z, P]),
             "csa2_index_prefill_workspace_bytes": (Z, [I, I64, I, I]),
             "csa2_index_prefill": (I, [Cache, P, P, P, P, I, I64, I64, I, I, I, P, P, P, Z, P]),
             "csa2_sparse_attn_prefill_workspace_bytes": (Z, [I, I]),
@@ -137,6 +156,13 @@ def csa2_index_full(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, max_len, 
                     ws, scores_out=None, stream=None):
     B = seq_len.shape[0]
     wp, wn = _ws(ws)
+    if isinstance(seq_row_off, PageTable):
+        pt = seq_row_off
+        rc = lib().csa2_index_full_paged(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(pt.pages), pt.page_rows,
+                                         pt.max_pages, _ptr(seq_len), B, max_len, pool_blocks, k, _ptr(pool_out),
+                                         _ptr(topk_out), _ptr(scores_out), wp, wn, _stream(stream))
+        _check(rc, "csa2_index_full_paged")
+        return
     rc = lib().csa2_index_full(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len), B,
                                max_len, pool_blocks, k, _ptr(pool_out), _ptr(topk_out), _ptr(scores_out), wp, wn,
                                _stream(stream))
@@ -150,6 +176,13 @@ def csa2_index_reindex_workspace_bytes(B, pool_blocks, k):
 def csa2_index_reindex(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, pool, k, topk_out, ws, stream=None):
     B, P = pool.shape
     wp, wn = _ws(ws)
+    if isinstance(seq_row_off, PageTable):
+        pt = seq_row_off
+        rc = lib().csa2_index_reindex_paged(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(pt.pages),
+                                            pt.page_rows, pt.max_pages, _ptr(seq_len), _ptr(pool), B, P, k,
+                                            _ptr(topk_out), wp, wn, _stream(stream))
+        _check(rc, "csa2_index_reindex_paged")
+        return
     rc = lib().csa2_index_reindex(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len),
                                   _ptr(pool), B, P, k, _ptr(topk_out), wp, wn, _stream(stream))
     _check(rc, "csa2_index_reindex")
@@ -163,6 +196,14 @@ def csa2_sparse_attn_decode(q, main_kv, seq_row_off, seq_len, topk, win, win_sca
                             lse=None, stream=None):
     B, k = topk.shape
     wp, wn = _ws(ws)
+    if isinstance(seq_row_off, PageTable):
+        pt = seq_row_off
+        rc = lib().csa2_sparse_attn_decode_paged(_ptr(q), main_kv, _ptr(pt.pages), pt.page_rows, pt.max_pages,
+                                                 _ptr(seq_len), _ptr(topk), k, _ptr(win), _ptr(win_scale),
+                                                 _ptr(win_len), float(sm_scale), _ptr(out), _ptr(lse), B, wp, wn,
+                                                 _stream(stream))
+        _check(rc, "csa2_sparse_attn_decode_paged")
+        return
     rc = lib().csa2_sparse_attn_decode(_ptr(q), main_kv, _ptr(seq_row_off), _ptr(seq_len), _ptr(topk), k, _ptr(win),
                                        _ptr(win_scale), _ptr(win_len), float(sm_scale), _ptr(out), _ptr(lse), B, wp,
                                        wn, _stream(stream))
@@ -193,6 +234,15 @@ def csa2_compress_stream(main_kv, idx_k, raw, logits, tok_off, seq_row_off, seq_
     B = seq_len_in.shape[0]
     wp, wn = _ws(ws)
     n_tok = raw.shape[0] if raw is not None else 0
+    if isinstance(seq_row_off, PageTable):
+        pt = seq_row_off
+        rc = lib().csa2_compress_stream_paged(main_kv, idx_k, _ptr(raw), _ptr(logits), _ptr(w_idx), _ptr(idx_raw),
+                                              _ptr(tok_off), _ptr(pt.pages), pt.page_rows, pt.max_pages,
+                                              _ptr(seq_len_in), _ptr(seq_len_out), _ptr(pend_n), _ptr(pend_raw),
+                                              _ptr(pend_logit), _ptr(pend_idx), B, n_tok, int(max_new), wp, wn,
+                                              _stream(stream))
+        _check(rc, "csa2_compress_stream_paged")
+        return
     rc = lib().csa2_compress_stream(main_kv, idx_k, _ptr(raw), _ptr(logits), _ptr(w_idx), _ptr(idx_raw),
                                     _ptr(tok_off), _ptr(seq_row_off), _ptr(seq_len_in), _ptr(seq_len_out),
                                     _ptr(pend_n), _ptr(pend_raw), _ptr(pend_logit), _ptr(pend_idx), B, n_tok,

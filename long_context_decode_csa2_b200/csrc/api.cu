@@ -41,6 +41,28 @@ bool cache_ok(const csa2_mxfp4_cache& c) {
   return c.codes && c.scales && aligned16(c.codes) && aligned16(c.scales) && c.rows >= 0 && (c.rows % 8) == 0;
 }
 
+// Paged layout arguments: page_rows a power of two in [512, 2^24] (a scan
+// item of 512 rows never crosses a page), every cache a whole number of
+// pages.  Sets *shift = log2(page_rows).
+bool pages_ok(const int32_t* pages, int page_rows, int max_pages, int64_t rows_a, int64_t rows_b, int* shift) {
+  if (!pages || (reinterpret_cast<uintptr_t>(pages) & 3) || max_pages < 1) return false;
+  if (page_rows < 512 || page_rows > (1 << 24) || (page_rows & (page_rows - 1))) return false;
+  if (rows_a % page_rows != 0 || rows_b % page_rows != 0) return false;
+  int sh = 0;
+  while ((1 << sh) < page_rows) ++sh;
+  *shift = sh;
+  return true;
+}
+
+SegDesc paged_desc(const int32_t* pages, int shift, int max_pages, const int32_t* len, int64_t max_len,
+                   int64_t cache_rows) {
+  SegDesc sd{nullptr, 0, len, max_len, cache_rows};
+  sd.pages = pages;
+  sd.page_shift = shift;
+  sd.max_pages = max_pages;
+  return sd;
+}
+
 struct IndexFullWs {
   uint32_t* status;
   int32_t* seg_eff;
@@ -106,17 +128,12 @@ size_t csa2_index_full_workspace_bytes(int B, int max_len, int pool_blocks, int 
   return index_full_ws(nullptr, B, max_len, pool_blocks, k, pool_blocks < k).bytes;
 }
 
-csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
-                            const int64_t* seq_row_off, const int32_t* seq_len, int B, int max_len,
-                            int pool_blocks, int k, int32_t* pool_out, int32_t* topk_out, float* scores_out,
-                            void* workspace, size_t workspace_bytes, void* stream) {
-  const char* fn = "csa2_index_full";
-  if (B < 0 || max_len < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
-  if (pool_blocks < 1 || pool_blocks > CSA2_MAX_POOL_BLOCKS || k < 1 || k > CSA2_MAX_TOPK)
-    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": pool_blocks and k must be in 1..2048");
-  if (B == 0) return CSA2_OK;
-  if (!cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad indexer-K cache");
-  if (!q_codes || !q_scales || !w || !seq_row_off || !seq_len || !pool_out || !topk_out || !workspace)
+namespace {
+csa2_status index_full_impl(const char* fn, csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                            const float* w, SegDesc sd, int B, int max_len, int pool_blocks, int k, int32_t* pool_out,
+                            int32_t* topk_out, float* scores_out, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!q_codes || !q_scales || !w || !sd.len || !pool_out || !topk_out || !workspace)
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
   if (!aligned16(q_codes) || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": q_codes must be 16-byte and workspace 256-byte aligned");
@@ -124,7 +141,6 @@ csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, cons
   IndexFullWs ws = index_full_ws(workspace, B, max_len, pool_blocks, k, need_scores);
   if (workspace_bytes < ws.bytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SegDesc sd{seq_row_off, 0, seq_len, max_len, idx_k.rows};
   const int64_t nb = block_key_stride(max_len);
   float* scores = scores_out ? scores_out : ws.scores;
   const csa2_status rc = launch_scan_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, ws.tile_start, B, q_codes, q_scales,
@@ -145,6 +161,44 @@ csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, cons
   return check_launch(fn);
 }
 
+csa2_status index_full_args(const char* fn, const csa2_mxfp4_cache& idx_k, int B, int max_len, int pool_blocks,
+                            int k) {
+  if (B < 0 || max_len < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
+  if (pool_blocks < 1 || pool_blocks > CSA2_MAX_POOL_BLOCKS || k < 1 || k > CSA2_MAX_TOPK)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": pool_blocks and k must be in 1..2048");
+  if (B > 0 && !cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad indexer-K cache");
+  return CSA2_OK;
+}
+}  // namespace
+
+csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                            const int64_t* seq_row_off, const int32_t* seq_len, int B, int max_len,
+                            int pool_blocks, int k, int32_t* pool_out, int32_t* topk_out, float* scores_out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_full";
+  const csa2_status rc = index_full_args(fn, idx_k, B, max_len, pool_blocks, k);
+  if (rc != CSA2_OK || B == 0) return rc;
+  if (!seq_row_off) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  return index_full_impl(fn, idx_k, q_codes, q_scales, w, SegDesc{seq_row_off, 0, seq_len, max_len, idx_k.rows}, B,
+                         max_len, pool_blocks, k, pool_out, topk_out, scores_out, workspace, workspace_bytes, stream);
+}
+
+csa2_status csa2_index_full_paged(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                  const float* w, const int32_t* pages, int page_rows, int max_pages,
+                                  const int32_t* seq_len, int B, int max_len, int pool_blocks, int k,
+                                  int32_t* pool_out, int32_t* topk_out, float* scores_out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_full_paged";
+  const csa2_status rc = index_full_args(fn, idx_k, B, max_len, pool_blocks, k);
+  if (rc != CSA2_OK || B == 0) return rc;
+  int shift = 0;
+  if (!pages_ok(pages, page_rows, max_pages, idx_k.rows, idx_k.rows, &shift))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad page table or page size");
+  return index_full_impl(fn, idx_k, q_codes, q_scales, w,
+                         paged_desc(pages, shift, max_pages, seq_len, max_len, idx_k.rows), B, max_len, pool_blocks,
+                         k, pool_out, topk_out, scores_out, workspace, workspace_bytes, stream);
+}
+
 // ---------------------------------------------------------------------------
 size_t csa2_index_reindex_workspace_bytes(int B, int pool_blocks, int k) {
   (void)k;
@@ -156,17 +210,19 @@ size_t csa2_index_reindex_workspace_bytes(int B, int pool_blocks, int k) {
   return c.used;
 }
 
-csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
-                               const float* w, const int64_t* seq_row_off, const int32_t* seq_len,
-                               const int32_t* pool, int B, int pool_blocks, int k, int32_t* topk_out,
-                               void* workspace, size_t workspace_bytes, void* stream) {
-  const char* fn = "csa2_index_reindex";
+namespace {
+csa2_status reindex_args(const char* fn, const csa2_mxfp4_cache& idx_k, int B, int pool_blocks, int k) {
   if (B < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
   if (pool_blocks < 1 || pool_blocks > CSA2_MAX_POOL_BLOCKS || k < 1 || k > CSA2_MAX_TOPK)
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": pool_blocks and k must be in 1..2048");
-  if (B == 0) return CSA2_OK;
-  if (!cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad indexer-K cache");
-  if (!q_codes || !q_scales || !w || !seq_row_off || !seq_len || !pool || !topk_out || !workspace)
+  if (B > 0 && !cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad indexer-K cache");
+  return CSA2_OK;
+}
+
+csa2_status reindex_impl(const char* fn, csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                         const float* w, SegDesc sd, const int32_t* pool, int B, int pool_blocks, int k,
+                         int32_t* topk_out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q_codes || !q_scales || !w || !sd.len || !pool || !topk_out || !workspace)
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
   if (reinterpret_cast<uintptr_t>(workspace) & 255)
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": workspace must be 256-byte aligned");
@@ -178,7 +234,6 @@ csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
   uint32_t* ckeys = c.take<uint32_t>(size_t(B) * pool_blocks * kBlk);
   uint32_t* hist = c.take<uint32_t>(size_t(B) * kCandHistBins);  // zero between calls
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SegDesc sd{seq_row_off, 0, seq_len, INT32_MAX, idx_k.rows};
   (void)seg_eff;  // lengths are checked inside the kernels
   const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, nullptr, B, q_codes, q_scales, w, pool,
                                         pool_blocks, ckeys, hist, status, st);
@@ -186,6 +241,33 @@ csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
   launch_select(kSelPoolCand, ckeys, int64_t(pool_blocks) * kBlk, nullptr, B, pool_blocks, pool, k, topk_out, hist,
                 st);
   return check_launch(fn);
+}
+}  // namespace
+
+csa2_status csa2_index_reindex(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                               const float* w, const int64_t* seq_row_off, const int32_t* seq_len,
+                               const int32_t* pool, int B, int pool_blocks, int k, int32_t* topk_out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_reindex";
+  const csa2_status rc = reindex_args(fn, idx_k, B, pool_blocks, k);
+  if (rc != CSA2_OK || B == 0) return rc;
+  if (!seq_row_off) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  return reindex_impl(fn, idx_k, q_codes, q_scales, w, SegDesc{seq_row_off, 0, seq_len, INT32_MAX, idx_k.rows}, pool,
+                      B, pool_blocks, k, topk_out, workspace, workspace_bytes, stream);
+}
+
+csa2_status csa2_index_reindex_paged(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                     const float* w, const int32_t* pages, int page_rows, int max_pages,
+                                     const int32_t* seq_len, const int32_t* pool, int B, int pool_blocks, int k,
+                                     int32_t* topk_out, void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_reindex_paged";
+  const csa2_status rc = reindex_args(fn, idx_k, B, pool_blocks, k);
+  if (rc != CSA2_OK || B == 0) return rc;
+  int shift = 0;
+  if (!pages_ok(pages, page_rows, max_pages, idx_k.rows, idx_k.rows, &shift))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad page table or page size");
+  return reindex_impl(fn, idx_k, q_codes, q_scales, w, paged_desc(pages, shift, max_pages, seq_len, INT32_MAX, idx_k.rows),
+                      pool, B, pool_blocks, k, topk_out, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -198,15 +280,18 @@ size_t csa2_sparse_attn_decode_workspace_bytes(int B, int k) {
   return c.used;
 }
 
-csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv, const int64_t* seq_row_off,
-                                    const int32_t* seq_len, const int32_t* topk, int k, const uint8_t* win,
-                                    const float* win_scale, const int32_t* win_len, float sm_scale, float* out,
-                                    float* lse, int B, void* workspace, size_t workspace_bytes, void* stream) {
-  const char* fn = "csa2_sparse_attn_decode";
+namespace {
+csa2_status attn_decode_args(const char* fn, const csa2_mxfp4_cache& main_kv, int B, int k) {
   if (B < 0 || k < 1 || k > CSA2_MAX_TOPK) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad B or k");
-  if (B == 0) return CSA2_OK;
-  if (!cache_ok(main_kv)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad main-KV cache");
-  if (!q || !seq_row_off || !seq_len || !topk || !win || !win_scale || !win_len || !out || !workspace)
+  if (B > 0 && !cache_ok(main_kv)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad main-KV cache");
+  return CSA2_OK;
+}
+
+csa2_status attn_decode_impl(const char* fn, const uint16_t* q, csa2_mxfp4_cache main_kv, SegDesc sd,
+                             const int32_t* topk, int k, const uint8_t* win, const float* win_scale,
+                             const int32_t* win_len, float sm_scale, float* out, float* lse, int B, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (!q || !sd.len || !topk || !win || !win_scale || !win_len || !out || !workspace)
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
   if (!aligned16(win) || !aligned16(q) || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": q/win must be 16-byte, workspace 256-byte aligned");
@@ -221,7 +306,7 @@ csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv,
   a.q = q;
   a.mcodes = main_kv.codes;
   a.mscales = main_kv.scales;
-  a.sd = SegDesc{seq_row_off, 0, seq_len, INT32_MAX, main_kv.rows};
+  a.sd = sd;
   a.seg_eff = nullptr;  // checked per segment inside the kernel
   (void)seg_eff;
   a.topk = topk;
@@ -236,6 +321,34 @@ csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   launch_attention(a, st);
   return check_launch(fn);
+}
+}  // namespace
+
+csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv, const int64_t* seq_row_off,
+                                    const int32_t* seq_len, const int32_t* topk, int k, const uint8_t* win,
+                                    const float* win_scale, const int32_t* win_len, float sm_scale, float* out,
+                                    float* lse, int B, void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_sparse_attn_decode";
+  const csa2_status rc = attn_decode_args(fn, main_kv, B, k);
+  if (rc != CSA2_OK || B == 0) return rc;
+  if (!seq_row_off) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  return attn_decode_impl(fn, q, main_kv, SegDesc{seq_row_off, 0, seq_len, INT32_MAX, main_kv.rows}, topk, k, win,
+                          win_scale, win_len, sm_scale, out, lse, B, workspace, workspace_bytes, stream);
+}
+
+csa2_status csa2_sparse_attn_decode_paged(const uint16_t* q, csa2_mxfp4_cache main_kv, const int32_t* pages,
+                                          int page_rows, int max_pages, const int32_t* seq_len, const int32_t* topk,
+                                          int k, const uint8_t* win, const float* win_scale, const int32_t* win_len,
+                                          float sm_scale, float* out, float* lse, int B, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_sparse_attn_decode_paged";
+  const csa2_status rc = attn_decode_args(fn, main_kv, B, k);
+  if (rc != CSA2_OK || B == 0) return rc;
+  int shift = 0;
+  if (!pages_ok(pages, page_rows, max_pages, main_kv.rows, main_kv.rows, &shift))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad page table or page size");
+  return attn_decode_impl(fn, q, main_kv, paged_desc(pages, shift, max_pages, seq_len, INT32_MAX, main_kv.rows), topk,
+                          k, win, win_scale, win_len, sm_scale, out, lse, B, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -289,17 +402,17 @@ size_t csa2_compress_stream_workspace_bytes(int B) {
   return kStatusBytes + round_up(size_t(B > 0 ? B : 0) * sizeof(uint32_t), 256);
 }
 
-csa2_status csa2_compress_stream(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k, const uint16_t* raw,
-                                 const float* logits, const float* w_idx, const uint16_t* idx_raw,
-                                 const int64_t* tok_off, const int64_t* seq_row_off, const int32_t* seq_len_in,
+namespace {
+// seq_row_off (contiguous layout) or pages / shift / max_pages (paged)
+csa2_status compress_stream_impl(const char* fn, csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k,
+                                 const uint16_t* raw, const float* logits, const float* w_idx,
+                                 const uint16_t* idx_raw, const int64_t* tok_off, const int64_t* seq_row_off,
+                                 const int32_t* pages, int shift, int max_pages, const int32_t* seq_len_in,
                                  int32_t* seq_len_out, int32_t* pend_n, uint16_t* pend_raw, float* pend_logit,
                                  uint16_t* pend_idx, int B, int64_t n_tok, int64_t max_new, void* workspace,
                                  size_t workspace_bytes, void* stream) {
-  const char* fn = "csa2_compress_stream";
-  if (B < 0 || n_tok < 0 || max_new < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
-  if (B == 0) return CSA2_OK;
-  if (!cache_ok(main_kv) || !cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad cache");
-  if (!tok_off || !seq_row_off || !seq_len_in || !pend_n || !pend_raw || !pend_logit || !logits || !workspace)
+  if (!tok_off || !(seq_row_off || pages) || !seq_len_in || !pend_n || !pend_raw || !pend_logit || !logits ||
+      !workspace)
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
   if (n_tok > 0 && !raw) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null raw");
   if ((w_idx == nullptr) == (idx_raw == nullptr && pend_idx == nullptr))
@@ -338,8 +451,52 @@ csa2_status csa2_compress_stream(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_
   a.pend_logit = pend_logit;
   a.pend_idx = pend_idx;
   a.arrive = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + kStatusBytes);
+  a.pages = pages;
+  a.page_shift = shift;
+  a.max_pages = max_pages;
   launch_compress(a, static_cast<cudaStream_t>(stream));
   return check_launch(fn);
+}
+
+csa2_status compress_stream_args(const char* fn, const csa2_mxfp4_cache& main_kv, const csa2_mxfp4_cache& idx_k,
+                                 int B, int64_t n_tok, int64_t max_new) {
+  if (B < 0 || n_tok < 0 || max_new < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
+  if (B > 0 && (!cache_ok(main_kv) || !cache_ok(idx_k)))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad cache");
+  return CSA2_OK;
+}
+}  // namespace
+
+csa2_status csa2_compress_stream(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k, const uint16_t* raw,
+                                 const float* logits, const float* w_idx, const uint16_t* idx_raw,
+                                 const int64_t* tok_off, const int64_t* seq_row_off, const int32_t* seq_len_in,
+                                 int32_t* seq_len_out, int32_t* pend_n, uint16_t* pend_raw, float* pend_logit,
+                                 uint16_t* pend_idx, int B, int64_t n_tok, int64_t max_new, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_compress_stream";
+  const csa2_status rc = compress_stream_args(fn, main_kv, idx_k, B, n_tok, max_new);
+  if (rc != CSA2_OK || B == 0) return rc;
+  if (!seq_row_off) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  return compress_stream_impl(fn, main_kv, idx_k, raw, logits, w_idx, idx_raw, tok_off, seq_row_off, nullptr, 0, 0,
+                              seq_len_in, seq_len_out, pend_n, pend_raw, pend_logit, pend_idx, B, n_tok, max_new,
+                              workspace, workspace_bytes, stream);
+}
+
+csa2_status csa2_compress_stream_paged(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k, const uint16_t* raw,
+                                       const float* logits, const float* w_idx, const uint16_t* idx_raw,
+                                       const int64_t* tok_off, const int32_t* pages, int page_rows, int max_pages,
+                                       const int32_t* seq_len_in, int32_t* seq_len_out, int32_t* pend_n,
+                                       uint16_t* pend_raw, float* pend_logit, uint16_t* pend_idx, int B, int64_t n_tok,
+                                       int64_t max_new, void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_compress_stream_paged";
+  const csa2_status rc = compress_stream_args(fn, main_kv, idx_k, B, n_tok, max_new);
+  if (rc != CSA2_OK || B == 0) return rc;
+  int shift = 0;
+  if (!pages_ok(pages, page_rows, max_pages, main_kv.rows, idx_k.rows, &shift))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad page table or page size");
+  return compress_stream_impl(fn, main_kv, idx_k, raw, logits, w_idx, idx_raw, tok_off, nullptr, pages, shift,
+                              max_pages, seq_len_in, seq_len_out, pend_n, pend_raw, pend_logit, pend_idx, B, n_tok,
+                              max_new, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

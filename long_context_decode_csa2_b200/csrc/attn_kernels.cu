@@ -156,8 +156,7 @@ __device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, in
   }
   if (ok) {
     if (!src.is_win) {
-      const int64_t off = a.sd.row_off ? a.sd.row_off[s] : a.sd.row0;
-      const int64_t row = off + tpos;
+      const int64_t row = seg_row(a.sd, s, tpos, a.status);
       const uint8_t* cs = a.mcodes + row * kMainCodeBytes + qt * (kMainCodeBytes / 4);
       uint8_t* dst = sm.raw.main[r] + qt * (kMainCodeBytes / 4);
 #pragma unroll

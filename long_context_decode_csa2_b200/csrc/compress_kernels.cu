@@ -167,8 +167,21 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
     for (int u = 0; u < 2; ++u) {
       const int e = warp + kCompWarps * u;
       const int64_t j = j0 + e;
-      const int64_t row = a.seq_row_off[b] + len_in + j;
       ok[u] = j < nnew;
+      int64_t row = -1;
+      if (ok[u]) {
+        if (a.pages) {
+          const int64_t t = int64_t(len_in) + j;
+          if (len_in < 0 || t >= (int64_t(a.max_pages) << a.page_shift)) {
+            if (lane == 0) set_status(a.status, CSA2_DEV_ROW_LAYOUT);
+            ok[u] = false;
+          } else {
+            row = paged_row(a.pages + int64_t(b) * a.max_pages, a.page_shift, min(a.mrows, a.irows), t, a.status);
+          }
+        } else {
+          row = a.seq_row_off[b] + len_in + j;
+        }
+      }
       if (ok[u] && (row < 0 || row >= a.mrows || row >= a.irows)) {
         if (lane == 0) set_status(a.status, CSA2_DEV_ROW_LAYOUT);
         ok[u] = false;

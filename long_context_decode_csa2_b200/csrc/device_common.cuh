@@ -16,19 +16,49 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t flag) {
 // Checked visible length of segment s: negative lengths count as 0, lengths
 // above the host bound are clamped (CSA2_DEV_LENGTH), and a misaligned or
 // out-of-capacity row range makes the segment empty (CSA2_DEV_ROW_LAYOUT).
+// In the paged layout a length beyond the segment's page-table row makes
+// the segment empty (CSA2_DEV_ROW_LAYOUT); page ids are checked where they
+// are used (paged_row).
 __device__ __forceinline__ int64_t seg_len_checked(const SegDesc& sd, int s, uint32_t* status) {
   int64_t L = sd.len[s];
-  const int64_t off = sd.row_off ? sd.row_off[s] : sd.row0;
   if (L < 0) L = 0;
   if (L > sd.max_len) {
     set_status(status, CSA2_DEV_LENGTH);
     L = sd.max_len;
   }
+  if (sd.pages) {
+    if (L > (int64_t(sd.max_pages) << sd.page_shift)) {
+      set_status(status, CSA2_DEV_ROW_LAYOUT);
+      L = 0;
+    }
+    return L;
+  }
+  const int64_t off = sd.row_off ? sd.row_off[s] : sd.row0;
   if ((off & 7) != 0 || off < 0 || off + L > sd.cache_rows) {
     set_status(status, CSA2_DEV_ROW_LAYOUT);
     L = 0;
   }
   return L;
+}
+
+// Cache row of position t (< the checked length) of a sequence whose
+// page-table row is `row`: a page id outside the cache is reported
+// (CSA2_DEV_ROW_LAYOUT) and read as page 0, so no access leaves the cache.
+__device__ __forceinline__ int64_t paged_row(const int32_t* row, int shift, int64_t cache_rows, int64_t t,
+                                             uint32_t* status) {
+  int64_t pg = __ldg(row + (t >> shift));
+  if (pg < 0 || ((pg + 1) << shift) > cache_rows) {
+    set_status(status, CSA2_DEV_ROW_LAYOUT);
+    pg = 0;
+  }
+  return (pg << shift) + (t & ((int64_t(1) << shift) - 1));
+}
+
+// Cache row of position t of segment s (either layout).
+__device__ __forceinline__ int64_t seg_row(const SegDesc& sd, int s, int64_t t, uint32_t* status) {
+  if (sd.pages)
+    return paged_row(sd.pages + int64_t(s) * sd.max_pages, sd.page_shift, sd.cache_rows, t, status);
+  return (sd.row_off ? sd.row_off[s] : sd.row0) + t;
 }
 
 // Order-preserving map of an fp32 score to a uint32 key; -0 ranks as +0.

@@ -44,6 +44,11 @@ struct SegDesc {
   const int32_t* len;      // [S]
   int64_t max_len;         // host bound
   int64_t cache_rows;      // capacity of the cache
+  // paged layout (pages != null): position t of segment s lives in row
+  // pages[s * max_pages + (t >> page_shift)] * 2^page_shift + t % 2^page_shift
+  const int32_t* pages;
+  int page_shift;
+  int max_pages;
 };
 
 // Selection histograms: one row per segment in the workspace over the top
@@ -168,6 +173,10 @@ struct CompressArgs {
   float* pend_logit;     // [B]
   uint16_t* pend_idx;    // [B][128] bf16, or null (W_idx projection)
   uint32_t* arrive;      // [B] arrival counters, zero between calls
+  // paged layout (pages != null; then seq_row_off is unused)
+  const int32_t* pages;  // [B][max_pages]
+  int page_shift;
+  int max_pages;
 };
 void launch_compress(const CompressArgs& a, cudaStream_t st);
 

@@ -284,12 +284,15 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
             pool_seg = b;
           }
           // lane i < kSlotsPerWarp owns slot pw * kSlotsPerWarp + i of the item
+          // (block id and first cache row; -1 = absent)
           int32_t my = -1;
+          int64_t myrow = -1;
           if (lane < kSlotsPerWarp) {
             const int32_t bk = sm.segpool[pw][j * kSlotsPerWarp + lane];
             const bool in_range = bk >= 0 && int64_t(bk) * kBlk < seq_len;
             if (bk >= 0 && !in_range) set_status(p.status, CSA2_DEV_INDEX_RANGE);
             my = in_range ? bk : -1;
+            if (in_range) myrow = p.sd.pages ? seg_row(p.sd, b, int64_t(bk) * kBlk, p.status) : seq_off + int64_t(bk) * kBlk;
             sm.blk[s][pw * kSlotsPerWarp + lane] = my;
           }
           if (pw == 0 && lane == 0) sm.info[s] = make_int2(b, j);
@@ -297,21 +300,21 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
           // destination in the 64-byte swizzle the MMA descriptor expects
           const int r8 = lane >> 2, ch = lane & 3;
           const int phys = r8 * 64 + ((ch ^ ((r8 >> 1) & 3)) << 4);
-          const uint8_t* kbase = p.kcodes + seq_off * kIdxCodeBytes + lane * 16;
+          const uint8_t* kbase = p.kcodes + lane * 16;
           uint8_t* abase = sm.a[s] + pw * kSlotsPerWarp * kBlk * kIdxCodeBytes + phys;
 #pragma unroll
           for (int i = 0; i < kSlotsPerWarp; ++i) {
-            const int32_t bk = __shfl_sync(0xffffffffu, my, i);
-            if (bk >= 0) sm100::cp_async16(abase + i * kBlk * kIdxCodeBytes, kbase + int64_t(bk) * kBlk * kIdxCodeBytes);
+            const int64_t row = __shfl_sync(0xffffffffu, myrow, i);
+            if (row >= 0) sm100::cp_async16(abase + i * kBlk * kIdxCodeBytes, kbase + row * kIdxCodeBytes);
           }
           // scales: 32 bytes per block, two 16-byte chunks
 #pragma unroll
           for (int c0 = 0; c0 < 2 * kSlotsPerWarp; c0 += 32) {
             const int c = c0 + lane, i = (c >> 1) & 31;
-            const int32_t bk = __shfl_sync(0xffffffffu, my, i);
-            if (c < 2 * kSlotsPerWarp && bk >= 0)
+            const int64_t row = __shfl_sync(0xffffffffu, myrow, i);
+            if (c < 2 * kSlotsPerWarp && row >= 0)
               sm100::cp_async16(&sm.sc[s][(pw * kSlotsPerWarp + i) * kBlk + 4 * (c & 1)],
-                                p.kscales + (seq_off + int64_t(bk) * kBlk) * 4 + 16 * (c & 1));
+                                p.kscales + row * 4 + 16 * (c & 1));
           }
           sm100::cp_async_commit();
           // signal the item issued kGatherDepth items ago once its copies landed
@@ -326,7 +329,9 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
           const int64_t rem_rows = seq_len - int64_t(j) * kTile;
           const int rows_valid = rem_rows < kTile ? int(rem_rows) : kTile;
           const uint32_t sbytes = uint32_t((rows_valid + 7) & ~7) * 4u;
-          const int64_t row0 = seq_off + int64_t(j) * kTile;
+          // an item never crosses a page (pages hold a multiple of kTile rows)
+          const int64_t row0 =
+              p.sd.pages ? seg_row(p.sd, b, int64_t(j) * kTile, p.status) : seq_off + int64_t(j) * kTile;
           sm100::mbar_arrive_expect_tx(&sm.full[s], kCodeBytes + sbytes);
 #pragma unroll
           for (int bx = 0; bx < kTile / kBoxRows; ++bx)

@@ -14,6 +14,9 @@ attention.  The five workloads:
 * ``verify_decode_b64_l1m_m6`` - as ``long_decode_b64_l1m`` with six candidate
                                queries per sequence (speculative verification):
                                query i sees all entries but the last 5 - i
+* ``paged_decode_b64_l1m``   - as ``long_decode_b64_l1m`` with the caches read
+                               through a page table (4096-row pages, the
+                               whole pool's pages shuffled across sequences)
 * ``ratio2_decode_b64_l1m``  - as ``long_decode_b64_l1m`` over ratio-2 entries
                                (2^20 entries = 2^21 raw tokens); each step also
                                appends one raw token per sequence, so the
@@ -41,6 +44,24 @@ class DecodeWorkload:
     ratio: int = 1      # 2: entries are compressed pairs, appended during decode
     room: int = 0       # spare cache rows per sequence beyond its length
     queries_per_seq: int = 0  # > 0: a verification step with this many candidate queries per sequence
+    page_rows: int = 0  # > 0: the caches are read through a page table of pages this size
+
+    def page_table(self):
+        """[B, max_pages] int32: the contiguous layout's pages (sequence b
+        owns pages off[b] / page_rows ..) dealt out in a seeded random order,
+        so sequence b's logical page i is some other physical page."""
+        off, rows = self.row_offsets()
+        pr = self.page_rows
+        assert rows % pr == 0 and (off % pr == 0).all(), "sequences must start on page boundaries"
+        n_pages = rows // pr
+        need = (self.lengths + self.room + pr - 1) // pr
+        perm = np.random.default_rng(self.seed + 17).permutation(n_pages).astype(np.int32)
+        table = np.zeros((self.B, int(need.max())), np.int32)
+        o = 0
+        for b, n in enumerate(need):
+            table[b, :n] = perm[o:o + n]
+            o += n
+        return table
 
     @property
     def B(self):
@@ -100,6 +121,8 @@ def decode_workloads():
                                                 "FRURU" * 4, needles=32),
         "verify_decode_b64_l1m_m6": DecodeWorkload("verify_decode_b64_l1m_m6", np.full(64, 1 << 20), "FRRU",
                                                    needles=256, lognormal=True, queries_per_seq=6),
+        "paged_decode_b64_l1m": DecodeWorkload("paged_decode_b64_l1m", np.full(64, 1 << 20), "FRRU", needles=256,
+                                               lognormal=True, page_rows=4096),
         "ratio2_decode_b64_l1m": DecodeWorkload("ratio2_decode_b64_l1m", np.full(64, 1 << 20), "FRRU", needles=256,
                                                 lognormal=True, ratio=2, room=1024),
     }

@@ -288,6 +288,56 @@ csa2_status csa2_compress_stream_paged(csa2_mxfp4_cache main_kv, csa2_mxfp4_cach
                                        void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Context parallelism: one long sequence split over G shards (GPUs), shard g
+ * holding entries [lo_g, hi_g) (lo_g a multiple of 8) in its own caches.
+ * Source: [V41] hierarchical indexer: the block pool and every Top-k are
+ * best-first selections by (score desc, position asc), so the global winners
+ * lie in the union of every shard's own winners, ranked by the same keys;
+ * attention over disjoint key sets combines through their log-sum-exps.
+ * A step: each shard runs csa2_index_full on its range, ranks its pool and
+ * Top-k with csa2_score_positions, the shards exchange (key, id) lists (an
+ * all-gather), csa2_topk_merge picks the global pool / Top-k and hands each
+ * shard its own part; Reindex layers score their shard's part of the pool
+ * (csa2_index_reindex + csa2_score_positions + csa2_topk_merge); attention
+ * runs per shard on its selected entries (the window on the shard holding
+ * the newest tokens), and csa2_attn_combine mixes the partial outputs.
+ *
+ * csa2_score_positions: the rank key (order-preserving uint32 of the exact
+ * score, 0 = absent) of listed positions (block 1) or of listed 8-position
+ * blocks (block 8: the maximum over the block's visible positions), for the
+ * same query inputs as csa2_index_full.  The keys are bit-identical to the
+ * ones the indexer ranks by.
+ *   ids [B][n] int32 positions or block ids (< 0: key 0; beyond the visible
+ *   length: key 0 and CSA2_DEV_INDEX_RANGE); keys_out [B][n] uint32
+ *   workspace: csa2_score_positions_workspace_bytes(B)
+ * csa2_topk_merge: per sequence b the k best of the G*n candidates
+ * (keys[g][b][i], ids[g][b][i] + src_off[g][b]) by (key desc, id asc), key 0
+ * never chosen, written ascending to out [B][k] (-1 padded).  Within a
+ * sequence the global ids must ascend with (g, i) (each shard's list
+ * ascending, shards in position order), which the lists from
+ * csa2_index_full / csa2_index_reindex with src_off = lo_g (or lo_g / 8 for
+ * block ids) satisfy.  src_off [G][B] int64 or NULL (ids already global).
+ * out_local [B][k] or NULL: out[b][j] - lo[b] where lo[b] <= out[b][j] <
+ * hi[b], else -1 (this shard's part, in its own coordinates).
+ *   workspace: csa2_topk_merge_workspace_bytes(G, B, n); G*n <= 2^24
+ * csa2_attn_combine: out_parts [G][B][16][512] and lse_parts [G][B][16] (from
+ * csa2_sparse_attn_decode per shard; a shard with nothing selected has lse
+ * -inf) -> out [B][16][512] = sum_g e^(lse_g - M) out_g / sum_g e^(lse_g - M)
+ * and lse [B][16] = M + log(sum) (lse may be NULL), M = max_g lse_g.
+ * ------------------------------------------------------------------------- */
+size_t csa2_score_positions_workspace_bytes(int B);
+csa2_status csa2_score_positions(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                 const float* w, const int64_t* seq_row_off, const int32_t* seq_len,
+                                 const int32_t* ids, int B, int n, int block, uint32_t* keys_out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+size_t csa2_topk_merge_workspace_bytes(int G, int B, int n);
+csa2_status csa2_topk_merge(const uint32_t* keys, const int32_t* ids, const int64_t* src_off, int G, int B, int n,
+                            int k, const int64_t* lo, const int64_t* hi, int32_t* out, int32_t* out_local,
+                            void* workspace, size_t workspace_bytes, void* stream);
+csa2_status csa2_attn_combine(const float* out_parts, const float* lse_parts, int G, int B, float* out, float* lse,
+                              void* stream);
+
+/* ---------------------------------------------------------------------------
  * csa2_index_multi -- Full-mode indexer for a batch of sequences with several
  * queries each (the candidate tokens of a speculative-decoding verification
  * step), reading every sequence's indexer K once for all of its queries.

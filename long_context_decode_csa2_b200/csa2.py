@@ -75,6 +75,11 @@ def lib():
             "csa2_sparse_attn_decode_paged": (I, [P, Cache, P, I, I, P, P, I, P, P, P, F, P, P, I, P, Z, P]),
             "csa2_compress_stream_paged": (I, [Cache, Cache, P, P, P, P, P, P, I, I, P, P, P, P, P, P, I, I64, I64, P,
                                                Z, P]),
+            "csa2_score_positions_workspace_bytes": (Z, [I]),
+            "csa2_score_positions": (I, [Cache, P, P, P, P, P, P, I, I, I, P, P, Z, P]),
+            "csa2_topk_merge_workspace_bytes": (Z, [I, I, I]),
+            "csa2_topk_merge": (I, [P, P, P, I, I, I, I, P, P, P, P, P, Z, P]),
+            "csa2_attn_combine": (I, [P, P, I, I, P, P, P]),
             "csa2_index_prefill_workspace_bytes": (Z, [I, I64, I, I]),
             "csa2_index_prefill": (I, [Cache, P, P, P, P, I, I64, I64, I, I, I, P, P, P, Z, P]),
             "csa2_sparse_attn_prefill_workspace_bytes": (Z, [I, I]),
@@ -262,6 +267,39 @@ def csa2_index_multi(idx_k, q_codes, q_scales, w, seq_row_off, q_off, q_vis, max
                                 _ptr(q_vis), B, Q, int(max_vis), pool_blocks, k, _ptr(pool_out), _ptr(topk_out),
                                 _ptr(q_row_off_out), wp, wn, _stream(stream))
     _check(rc, "csa2_index_multi")
+
+
+def csa2_score_positions_workspace_bytes(B):
+    return lib().csa2_score_positions_workspace_bytes(B)
+
+
+def csa2_score_positions(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, ids, block, keys_out, ws, stream=None):
+    """keys_out [B, n] uint32 (int32 tensors carry the bits) <- rank keys of ids [B, n] (block 1 or 8)."""
+    B, n = ids.shape
+    wp, wn = _ws(ws)
+    rc = lib().csa2_score_positions(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len),
+                                    _ptr(ids), B, n, int(block), _ptr(keys_out), wp, wn, _stream(stream))
+    _check(rc, "csa2_score_positions")
+
+
+def csa2_topk_merge_workspace_bytes(G, B, n):
+    return lib().csa2_topk_merge_workspace_bytes(G, B, n)
+
+
+def csa2_topk_merge(keys, ids, src_off, k, out, ws, lo=None, hi=None, out_local=None, stream=None):
+    """keys / ids [G, B, n] from the shards -> out [B, k] (and out_local [B, k] for [lo, hi))."""
+    G, B, n = ids.shape
+    wp, wn = _ws(ws)
+    rc = lib().csa2_topk_merge(_ptr(keys), _ptr(ids), _ptr(src_off), G, B, n, k, _ptr(lo), _ptr(hi), _ptr(out),
+                               _ptr(out_local), wp, wn, _stream(stream))
+    _check(rc, "csa2_topk_merge")
+
+
+def csa2_attn_combine(out_parts, lse_parts, out, lse=None, stream=None):
+    """out_parts [G, B, 16, 512], lse_parts [G, B, 16] -> out [B, 16, 512], lse [B, 16]."""
+    G, B = lse_parts.shape[0], lse_parts.shape[1]
+    rc = lib().csa2_attn_combine(_ptr(out_parts), _ptr(lse_parts), G, B, _ptr(out), _ptr(lse), _stream(stream))
+    _check(rc, "csa2_attn_combine")
 
 
 def csa2_index_prefill_workspace_bytes(T, n_entries, pool_blocks, k):

@@ -636,6 +636,76 @@ csa2_status csa2_index_multi(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, con
 }
 
 // ---------------------------------------------------------------------------
+size_t csa2_score_positions_workspace_bytes(int B) {
+  (void)B;
+  return kStatusBytes;
+}
+
+csa2_status csa2_score_positions(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                 const float* w, const int64_t* seq_row_off, const int32_t* seq_len,
+                                 const int32_t* ids, int B, int n, int block, uint32_t* keys_out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_score_positions";
+  if (B < 0 || n < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative size");
+  if (block != 1 && block != kBlk) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": block must be 1 or 8");
+  if (B == 0 || n == 0) return CSA2_OK;
+  if (!cache_ok(idx_k)) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad indexer-K cache");
+  if (!q_codes || !q_scales || !w || !seq_row_off || !seq_len || !ids || !keys_out || !workspace)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (workspace_bytes < kStatusBytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  SegDesc sd{seq_row_off, 0, seq_len, INT32_MAX, idx_k.rows};
+  launch_score_positions(idx_k.codes, idx_k.scales, sd, q_codes, q_scales, w, ids, B, n, block, keys_out,
+                         static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream));
+  return check_launch(fn);
+}
+
+size_t csa2_topk_merge_workspace_bytes(int G, int B, int n) {
+  if (G < 0 || B < 0 || n < 0) return 0;
+  Carve c(nullptr);
+  c.take<uint32_t>(kStatusBytes / 4);
+  c.take<uint32_t>(size_t(B) * G * n);
+  c.take<int32_t>(size_t(B) * G * n);
+  return c.used;
+}
+
+csa2_status csa2_topk_merge(const uint32_t* keys, const int32_t* ids, const int64_t* src_off, int G, int B, int n,
+                            int k, const int64_t* lo, const int64_t* hi, int32_t* out, int32_t* out_local,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_topk_merge";
+  if (G < 1 || B < 0 || n < 0 || k < 1 || k > CSA2_MAX_TOPK)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad G, B, n or k");
+  if (int64_t(G) * n > (int64_t(1) << 24)) return fail(CSA2_ERR_UNSUPPORTED, std::string(fn) + ": too many candidates");
+  if (B == 0) return CSA2_OK;
+  if (!keys || !ids || !out || !workspace || (out_local && (!lo || !hi)))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": workspace must be 256-byte aligned");
+  if (workspace_bytes < csa2_topk_merge_workspace_bytes(G, B, n))
+    return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  Carve c(workspace);
+  uint32_t* status = c.take<uint32_t>(kStatusBytes / 4);
+  uint32_t* keys_t = c.take<uint32_t>(size_t(B) * G * n);
+  int32_t* ids_t = c.take<int32_t>(size_t(B) * G * n);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  launch_merge_gather(keys, ids, src_off, G, B, n, keys_t, ids_t, status, st);
+  launch_select(kSelExplicit, keys_t, int64_t(G) * n, nullptr, B, G * n, ids_t, k, out, nullptr, st);
+  if (out_local) launch_localize(out, B, k, lo, hi, out_local, st);
+  return check_launch(fn);
+}
+
+csa2_status csa2_attn_combine(const float* out_parts, const float* lse_parts, int G, int B, float* out, float* lse,
+                              void* stream) {
+  const char* fn = "csa2_attn_combine";
+  if (G < 1 || B < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad G or B");
+  if (B == 0) return CSA2_OK;
+  if (!out_parts || !lse_parts || !out) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (!aligned16(out_parts) || !aligned16(out))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": out_parts and out must be 16-byte aligned");
+  launch_attn_combine(out_parts, lse_parts, G, B, out, lse, static_cast<cudaStream_t>(stream));
+  return check_launch(fn);
+}
+
+// ---------------------------------------------------------------------------
 size_t csa2_sparse_attn_prefill_workspace_bytes(int T, int k) {
   Carve c(nullptr);
   c.take<uint32_t>(kStatusBytes / 4);

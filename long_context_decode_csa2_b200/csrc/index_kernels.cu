@@ -103,6 +103,7 @@ __device__ __forceinline__ void load_keys(const void* in, int64_t base, int64_t 
 template <int KIND>
 __device__ __forceinline__ int32_t sel_id(const int32_t* pool, int s, int P, int64_t i) {
   if (KIND == kSelPoolCand) return pool[int64_t(s) * P + i / kBlk] * kBlk + int32_t(i % kBlk);
+  if (KIND == kSelExplicit) return pool[int64_t(s) * P + i];
   return static_cast<int32_t>(i);
 }
 
@@ -331,6 +332,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   int64_t n;
   if (KIND == kSelBlockKeys) n = (int64_t(seg_eff[s]) + kBlk - 1) / kBlk;
   else if (KIND == kSelScores) n = seg_eff[s];
+  else if (KIND == kSelExplicit) n = P;
   else n = int64_t(P) * kBlk;
   const int64_t base = int64_t(s) * in_stride;
   int32_t* o = out + int64_t(s) * k;
@@ -641,6 +643,9 @@ void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int
       break;
     case kSelPoolCand:
       launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
+      break;
+    case kSelExplicit:
+      launch_select_kind<kSelExplicit>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
       break;
   }
 }

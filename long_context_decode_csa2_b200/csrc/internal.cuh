@@ -101,6 +101,20 @@ csa2_status launch_multi_tc(const uint8_t* kcodes, const uint8_t* kscales, int64
                             int64_t max_vis, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
                             uint32_t* bkeys, int64_t nb_stride, uint32_t* status, cudaStream_t st);
 
+// Context-parallel pieces (cp_kernels.cu): exact keys of listed positions
+// (blk 1) or blocks (blk 8); shards' candidate lists [G][B][n] -> [B][G*n]
+// with global ids; ids inside [lo, hi) made local; lse-weighted merge of
+// attention partials [G][B].
+void launch_score_positions(const uint8_t* kcodes, const uint8_t* kscales, const SegDesc& sd, const uint8_t* q_codes,
+                            const uint8_t* q_scales, const float* w, const int32_t* ids, int B, int n, int blk,
+                            uint32_t* keys_out, uint32_t* status, cudaStream_t st);
+void launch_merge_gather(const uint32_t* keys, const int32_t* ids, const int64_t* src_off, int G, int B, int n,
+                         uint32_t* keys_t, int32_t* ids_t, uint32_t* status, cudaStream_t st);
+void launch_localize(const int32_t* out, int B, int k, const int64_t* lo, const int64_t* hi, int32_t* out_local,
+                     cudaStream_t st);
+void launch_attn_combine(const float* out_parts, const float* lse_parts, int G, int B, float* out, float* lse,
+                         cudaStream_t st);
+
 // Visible entry counts of prefill queries.
 void launch_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entries, int32_t* vis, uint32_t* status,
                         cudaStream_t st);
@@ -111,6 +125,7 @@ enum SelectKind : int {
   kSelBlockKeys = 0,  // u32 keys, n = ceil(seg_eff/8), id = index
   kSelScores = 1,     // fp32 scores, n = seg_eff, id = index
   kSelPoolCand = 2,   // u32 keys, n = P*8, id = 8*pool[i/8] + i%8
+  kSelExplicit = 3,   // u32 keys, n = P, id = pool[i] (ids ascending with i)
 };
 // `hist` (or null): the keys' histogram rows, zeroed on return: [S][kSelHistBins]
 // for block keys, [S][kCandHistBins] for pool candidates.

@@ -89,3 +89,66 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
 
     assert bench.run_reference(Args()) is None
     assert capsys.readouterr().out == ""
+
+
+# --- context-parallel exchange: one sequence split over two gloo ranks ---
+
+def _cp_worker(rank, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(WORLD))
+    import datetime
+
+    from long_context_decode_csa2_b200.cp import dist_gather, shard_bounds
+
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD, timeout=datetime.timedelta(seconds=120))
+    try:
+        wl = W.DecodeWorkload("cp_gloo", np.array([6001]), "F", P=64, k=64, needles=4)
+        L0 = W.layer_inputs_host(wl, 0)
+        c = W.full_cache_host(wl, 0, L0["q_codes"], L0["q_scales"])
+        bounds = shard_bounds(wl.lengths, WORLD)
+        lo, hi = int(bounds[rank, 0]), int(bounds[rank + 1, 0])
+        # this rank's own winners over its range (the oracle stands in for the GPU calls here)
+        _, top, sc = oracle.index_full(c["idx_codes"][lo:hi], c["idx_scales"][lo:hi], L0["q_codes"], L0["q_scales"],
+                                       L0["w"], np.array([0]), np.array([hi - lo], np.int32), wl.P, wl.k,
+                                       want_scores=True)
+        keys = np.array([oracle.rank_key(sc[0, t]) if t >= 0 else 0 for t in top[0]], np.uint32)
+        ids = np.where(top[0] >= 0, top[0] + lo, -1).astype(np.int64)
+        g_keys = dist_gather()([torch.from_numpy(keys.view(np.int32).astype(np.int64))])
+        g_ids = dist_gather()([torch.from_numpy(ids)])
+        np.savez(os.path.join(out_dir, f"cp{rank}.npz"), keys=g_keys.numpy(), ids=g_ids.numpy(), bounds=bounds)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_exchange_two_gloo_ranks(tmp_path):
+    """Each rank's Top-k over its shard, all-gathered in rank order, holds
+    the whole sequence's Top-k: merging the union by (key desc, position
+    asc) equals the single-process selection."""
+    mp.start_processes(_cp_worker, args=(_free_port(), str(tmp_path)), nprocs=WORLD, start_method="spawn", join=True)
+    r = [np.load(tmp_path / f"cp{i}.npz") for i in range(WORLD)]
+    assert np.array_equal(r[0]["keys"], r[1]["keys"]) and np.array_equal(r[0]["ids"], r[1]["ids"])
+    b = r[0]["bounds"]
+    assert b[0, 0] == 0 and b[-1, 0] == 6001 and b[1, 0] % 8 == 0
+    keys = (r[0]["keys"].astype(np.int64) & 0xFFFFFFFF).ravel()
+    ids = r[0]["ids"].ravel()
+    assert (np.diff(ids[ids >= 0]) > 0).all()  # shard order = position order
+    ok = ids >= 0
+    merged = oracle.topk(keys[ok].astype(np.uint32), ids[ok], 64)
+    wl = W.DecodeWorkload("cp_gloo", np.array([6001]), "F", P=64, k=64, needles=4)
+    L0 = W.layer_inputs_host(wl, 0)
+    c = W.full_cache_host(wl, 0, L0["q_codes"], L0["q_scales"])
+    _, whole, _ = oracle.index_full(c["idx_codes"], c["idx_scales"], L0["q_codes"], L0["q_scales"], L0["w"],
+                                    np.array([0]), np.array([6001], np.int32), 64, 64)
+    assert merged.tolist() == whole[0].tolist()
+
+
+def test_shard_bounds_cover_each_sequence_in_whole_blocks():
+    from long_context_decode_csa2_b200.cp import shard_bounds
+
+    L = np.array([0, 7, 8, 1000, 1 << 20, 33001])
+    for G in (1, 2, 3, 8):
+        b = shard_bounds(L, G)
+        assert b.shape == (G + 1, len(L))
+        assert (b[0] == 0).all() and (b[-1] == L).all() and (np.diff(b, axis=0) >= 0).all()
+        assert (b[1:-1] % 8 == 0).all()
+        assert (np.diff(b, axis=0).max(axis=0) <= L // G + 8).all()

@@ -49,6 +49,9 @@ def parse():
                     help="issue every call on one stream (isolated per-call times) instead of the concurrent tail")
     ap.add_argument("--context", type=int, default=0,
                     help="override every sequence's length (small profiling captures of the attention)")
+    ap.add_argument("--cp", type=int, default=0,
+                    help="context-parallel step over this many shards of every sequence: one per rank under "
+                         "torchrun, all in this process on one GPU")
     return ap.parse_args()
 
 
@@ -842,12 +845,127 @@ def run_reference(args):
     print(json.dumps(res))
 
 
+def run_cp(args):
+    """Context-parallel decode step (cp.py): the workload's sequences split
+    into G shards.  Under torchrun G = the world size, one shard per rank,
+    exchanging through NCCL all-gathers (strong scaling: the sequences are
+    fixed, each rank holds 1/G of them); in one process all G shards run on
+    this GPU one after the other."""
+    import torch
+    import torch.distributed as dist
+
+    import synth.workloads as W
+    from long_context_decode_csa2_b200 import csa2 as C
+    from long_context_decode_csa2_b200.cp import Shard, ShardedStep, dist_gather, shard_bounds, stack_gather
+    from long_context_decode_csa2_b200.decode import FullCache
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
+    G = world if world > 1 else args.cp
+    mine = [rank] if world > 1 else list(range(G))
+    wl = W.decode_workloads()[args.workload]
+    if wl.queries_per_seq or wl.ratio != 1 or wl.page_rows:
+        raise SystemExit("--cp runs the plain decode workloads")
+    if args.batch:
+        wl = dataclasses.replace(wl, name=wl.name + f"_b{args.batch}", lengths=wl.lengths[:args.batch])
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    caches_dev = [W.full_cache_device(wl, f, layers[f]["q_codes"], layers[f]["q_scales"], device)
+                  for f in wl.full_layers()]
+    off = caches_dev[0]["seq_row_off"]
+    bounds = shard_bounds(wl.lengths, G)
+    keys = ("q", "q_codes", "q_scales", "w", "win", "win_scale", "win_len")
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+        return torch.from_numpy(a).to(device)
+
+    shards = []
+    for g in mine:
+        lens = (bounds[g + 1] - bounds[g]).astype(np.int64)
+        pad = (lens + 7) // 8 * 8
+        soff = np.concatenate([[0], np.cumsum(pad)[:-1]]).astype(np.int64)
+        rows = int(max(8, pad.sum()))
+        shard_caches = []
+        for c in caches_dev:  # this shard's rows of every sequence, gathered on the device
+            idx = torch.cat([torch.arange(int(off[b] + bounds[g, b]), int(off[b] + bounds[g + 1, b]), device=device)
+                             for b in range(wl.B)] or [torch.zeros(0, dtype=torch.int64, device=device)])
+            planes = {}
+            for key in ("idx_codes", "idx_scales", "main_codes", "main_scales"):
+                t = torch.zeros((rows, c[key].shape[1]), dtype=torch.uint8, device=device)
+                dst = torch.cat([torch.arange(int(soff[b]), int(soff[b] + lens[b]), device=device)
+                                 for b in range(wl.B)])
+                t[dst] = c[key][idx]
+                planes[key] = t
+            shard_caches.append(FullCache(C.cache(planes["idx_codes"], planes["idx_scales"]),
+                                          C.cache(planes["main_codes"], planes["main_scales"])))
+        lg = []
+        for L in layers:
+            Lg = {k: to_dev(L[k]) for k in keys}
+            if g != G - 1:  # the window lives on the shard with the newest entries
+                Lg["win_len"] = torch.zeros_like(Lg["win_len"])
+            lg.append(Lg)
+        shards.append(Shard(caches=shard_caches, seq_row_off=to_dev(soff), seq_len=to_dev(lens.astype(np.int32)),
+                            lo=to_dev(bounds[g]), hi=to_dev(bounds[g + 1]), layers=lg))
+    del caches_dev
+    torch.cuda.empty_cache()
+    src_pos = to_dev(bounds[:-1])
+    src_blk = to_dev(bounds[:-1] // 8)
+    max_shard = int((bounds[1:] - bounds[:-1]).max())
+    step = ShardedStep(wl.pattern, wl.B, max_shard, len(mine), G, wl.P, wl.k,
+                       gather=dist_gather() if world > 1 else stack_gather)
+    for _ in range(args.warmup):
+        step.run(shards, src_pos, src_blk)
+    torch.cuda.synchronize()
+    if step.device_flags():
+        raise RuntimeError("device status flags set during warm-up")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.5)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step.run(shards, src_pos, src_blk)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, device, world)
+    if rank == 0:
+        ab = algorithmic_bytes(wl)
+        print(json.dumps({
+            "metric": METRIC, "value": wl.B / (ms * 1e-3), "unit": "queries/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None,
+            "dtype": "int32+f64 indexer, f16 tensor-core attention (f32 accumulate)", "data": "synthetic",
+            "config": dict(decode_config(wl, ab["total"], True, False), cp_shards=G,
+                           cp_mode="one shard per rank (NCCL all-gather)" if world > 1 else
+                           "all shards on this GPU, one after the other"),
+            "hbm_algorithmic_gbs": ab["total"] / (ms * 1e-3) / 1e9,
+            "clocks": clk.summary(), "device_flags": step.device_flags()}))
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
     elif args.workload.startswith("prefill"):
         run_prefill(args)
+    elif args.cp:
+        run_cp(args)
     else:
         run_ours(args)
 

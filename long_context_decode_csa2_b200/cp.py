@@ -179,6 +179,17 @@ class ShardedStep:
             C.csa2_attn_combine(outs, lses, self.out[layer], self.lse[layer])
         return self.out
 
+    def capture(self, shards, src_pos, src_blk):
+        """Records one step into a CUDA graph (call ``run`` once first);
+        ``graph.replay()`` then runs it as one launch with the same buffers."""
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(device=self.out.device)
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
+            self.run(shards, src_pos, src_blk)
+        torch.cuda.current_stream().wait_stream(cap)
+        return graph
+
     def device_flags(self) -> int:
         flags = 0
         for st in self.local:

@@ -24,17 +24,26 @@ __device__ __forceinline__ int dbl_e2m1(uint32_t nib) {
 
 // grid (ceil(n * blk / 256), B), block 256.  Thread = (listed id i, offset o
 // < blk): the exact score of position id*blk + o from the 68-byte key row,
-// reduced to the key of the id (block maximum for blk = 8).
+// reduced to the key of the id (block maximum for blk = 8).  The block dots
+// are integer dp4a over doubled E2M1 values (|value| <= 12 fits int8).
 __global__ void __launch_bounds__(256) k_score_positions(const uint8_t* kcodes, const uint8_t* kscales, SegDesc sd,
                                                          const uint8_t* q_codes, const uint8_t* q_scales,
                                                          const float* w, const int32_t* ids, int n, int blk,
                                                          uint32_t* keys_out, uint32_t* status) {
-  __shared__ int8_t qv[kHi][kDi];
+  __shared__ uint32_t qw[kHi][kDi / 4];  // query: int8x4 of elements 4i .. 4i+3 per head
+  __shared__ uint16_t lut[256];          // code byte -> two int8 doubled values (low nibble first)
   __shared__ IdxQCtx qc;
   const int b = blockIdx.y;
-  for (int e = threadIdx.x; e < kHi * kDi; e += blockDim.x) {
-    const uint32_t byte = q_codes[int64_t(b) * kHi * 64 + e / 2];
-    qv[e / kDi][e % kDi] = int8_t(dbl_e2m1((e & 1) ? (byte >> 4) : (byte & 15u)));
+  {
+    const int t = threadIdx.x;  // 256 threads: one LUT entry each
+    const uint32_t lo = uint32_t(dbl_e2m1(t & 15u)) & 255u, hi = uint32_t(dbl_e2m1(uint32_t(t) >> 4)) & 255u;
+    lut[t] = uint16_t(lo | (hi << 8));
+  }
+  __syncthreads();
+  if (threadIdx.x < kHi * kDi / 4) {  // 128 words: two query code bytes each
+    const int h = threadIdx.x / (kDi / 4), i = threadIdx.x % (kDi / 4);
+    const uint8_t* qc8 = q_codes + int64_t(b) * kHi * 64 + h * 64 + 2 * i;
+    qw[h][i] = uint32_t(lut[qc8[0]]) | (uint32_t(lut[qc8[1]]) << 16);
   }
   if (threadIdx.x == 0) make_qctx(qc, q_scales + int64_t(b) * kHi * 4, w + int64_t(b) * kHi);
   __syncthreads();
@@ -60,13 +69,15 @@ __global__ void __launch_bounds__(256) k_score_positions(const uint8_t* kcodes, 
         const uint4 c = __ldg(kr + bb);
         const uint32_t words[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
+        for (int wd = 0; wd < 4; ++wd) {  // bytes 4wd .. 4wd+3 = elements 8wd .. 8wd+7 of the block
+          const uint32_t x = words[wd];
+          const int k0 = int(uint32_t(lut[x & 255u]) | (uint32_t(lut[(x >> 8) & 255u]) << 16));
+          const int k1 = int(uint32_t(lut[(x >> 16) & 255u]) | (uint32_t(lut[x >> 24]) << 16));
+          const int qi = 8 * bb + 2 * wd;  // word index of element 32bb + 8wd
 #pragma unroll
-          for (int nb = 0; nb < 8; ++nb) {
-            const int e = 32 * bb + 8 * wd + nb;
-            const int kv = dbl_e2m1((words[wd] >> (4 * nb)) & 15u);
-#pragma unroll
-            for (int h = 0; h < kHi; ++h) D[h][bb] += kv * int(qv[h][e]);
+          for (int h = 0; h < kHi; ++h) {
+            D[h][bb] = __dp4a(k0, int(qw[h][qi]), D[h][bb]);
+            D[h][bb] = __dp4a(k1, int(qw[h][qi + 1]), D[h][bb]);
           }
         }
       }

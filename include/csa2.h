@@ -246,6 +246,24 @@ csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * csa2_index_full_pool + csa2_index_full_topk -- csa2_index_full in two
+ * calls, so that work which needs only the pool (the Reindex layers) can
+ * start while the Full layer's own Top-k is still being selected.
+ * csa2_index_full_pool runs the scan and writes pool_out; a later
+ * csa2_index_full_topk on the same stream, with the same arguments, the
+ * same workspace (untouched in between) and that pool, writes topk_out.
+ * Together they give exactly csa2_index_full's results.
+ * ------------------------------------------------------------------------- */
+csa2_status csa2_index_full_pool(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                 const float* w, const int64_t* seq_row_off, const int32_t* seq_len, int B,
+                                 int max_len, int pool_blocks, int k, int32_t* pool_out, float* scores_out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+csa2_status csa2_index_full_topk(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                 const float* w, const int64_t* seq_row_off, const int32_t* seq_len, int B,
+                                 int max_len, int pool_blocks, int k, const int32_t* pool, int32_t* topk_out,
+                                 float* scores_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Paged caches: csa2_index_full_paged, csa2_index_reindex_paged,
  * csa2_sparse_attn_decode_paged, csa2_compress_stream_paged.
  * The same operations, results and errors as the calls without the suffix,

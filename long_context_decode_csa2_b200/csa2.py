@@ -70,6 +70,8 @@ def lib():
             "csa2_compress_stream": (I, [Cache, Cache, P, P, P, P, P, P, P, P, P, P, P, P, I, I64, I64, P, Z, P]),
             "csa2_index_multi_workspace_bytes": (Z, [I, I, I64, I, I]),
             "csa2_index_multi": (I, [Cache, P, P, P, P, P, P, I, I, I64, I, I, P, P, P, P, Z, P]),
+            "csa2_index_full_pool": (I, [Cache, P, P, P, P, P, I, I, I, I, P, P, P, Z, P]),
+            "csa2_index_full_topk": (I, [Cache, P, P, P, P, P, I, I, I, I, P, P, P, P, Z, P]),
             "csa2_index_full_paged": (I, [Cache, P, P, P, P, I, I, P, I, I, I, I, P, P, P, P, Z, P]),
             "csa2_index_reindex_paged": (I, [Cache, P, P, P, P, I, I, P, P, I, I, I, P, P, Z, P]),
             "csa2_sparse_attn_decode_paged": (I, [P, Cache, P, I, I, P, P, I, P, P, P, F, P, P, I, P, Z, P]),
@@ -172,6 +174,26 @@ def csa2_index_full(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, max_len, 
                                max_len, pool_blocks, k, _ptr(pool_out), _ptr(topk_out), _ptr(scores_out), wp, wn,
                                _stream(stream))
     _check(rc, "csa2_index_full")
+
+
+def csa2_index_full_pool(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, max_len, pool_blocks, k, pool_out, ws,
+                         scores_out=None, stream=None):
+    B = seq_len.shape[0]
+    wp, wn = _ws(ws)
+    rc = lib().csa2_index_full_pool(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len),
+                                    B, max_len, pool_blocks, k, _ptr(pool_out), _ptr(scores_out), wp, wn,
+                                    _stream(stream))
+    _check(rc, "csa2_index_full_pool")
+
+
+def csa2_index_full_topk(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, max_len, pool_blocks, k, pool, topk_out,
+                         ws, scores_out=None, stream=None):
+    B = seq_len.shape[0]
+    wp, wn = _ws(ws)
+    rc = lib().csa2_index_full_topk(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len),
+                                    B, max_len, pool_blocks, k, _ptr(pool), _ptr(topk_out), _ptr(scores_out), wp, wn,
+                                    _stream(stream))
+    _check(rc, "csa2_index_full_topk")
 
 
 def csa2_index_reindex_workspace_bytes(B, pool_blocks, k):

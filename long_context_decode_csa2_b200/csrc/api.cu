@@ -129,11 +129,13 @@ size_t csa2_index_full_workspace_bytes(int B, int max_len, int pool_blocks, int 
 }
 
 namespace {
+// phases: 1 = scan + block pool, 2 = Top-k (from the workspace state phase 1
+// left), 3 = both
 csa2_status index_full_impl(const char* fn, csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
                             const float* w, SegDesc sd, int B, int max_len, int pool_blocks, int k, int32_t* pool_out,
                             int32_t* topk_out, float* scores_out, void* workspace, size_t workspace_bytes,
-                            void* stream) {
-  if (!q_codes || !q_scales || !w || !sd.len || !pool_out || !topk_out || !workspace)
+                            void* stream, int phases = 3) {
+  if (!q_codes || !q_scales || !w || !sd.len || !pool_out || (!topk_out && (phases & 2)) || !workspace)
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
   if (!aligned16(q_codes) || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": q_codes must be 16-byte and workspace 256-byte aligned");
@@ -143,10 +145,13 @@ csa2_status index_full_impl(const char* fn, csa2_mxfp4_cache idx_k, const uint8_
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t nb = block_key_stride(max_len);
   float* scores = scores_out ? scores_out : ws.scores;
-  const csa2_status rc = launch_scan_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, ws.tile_start, B, q_codes, q_scales,
-                                        w, ws.bkeys, nb, scores, max_len, ws.hist, ws.status, st);
-  if (rc != CSA2_OK) return rc;
-  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, ws.hist, st);
+  if (phases & 1) {
+    const csa2_status rc = launch_scan_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, ws.tile_start, B, q_codes,
+                                          q_scales, w, ws.bkeys, nb, scores, max_len, ws.hist, ws.status, st);
+    if (rc != CSA2_OK) return rc;
+    launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, ws.hist, st);
+  }
+  if (!(phases & 2)) return check_launch(fn);
   if (pool_blocks >= k) {
     // Every Top-k position's block ranks within the first k blocks, so the
     // Top-k over the pool equals the Top-k over all positions.
@@ -181,6 +186,32 @@ csa2_status csa2_index_full(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, cons
   if (!seq_row_off) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
   return index_full_impl(fn, idx_k, q_codes, q_scales, w, SegDesc{seq_row_off, 0, seq_len, max_len, idx_k.rows}, B,
                          max_len, pool_blocks, k, pool_out, topk_out, scores_out, workspace, workspace_bytes, stream);
+}
+
+csa2_status csa2_index_full_pool(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                 const float* w, const int64_t* seq_row_off, const int32_t* seq_len, int B,
+                                 int max_len, int pool_blocks, int k, int32_t* pool_out, float* scores_out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_full_pool";
+  const csa2_status rc = index_full_args(fn, idx_k, B, max_len, pool_blocks, k);
+  if (rc != CSA2_OK || B == 0) return rc;
+  if (!seq_row_off) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  return index_full_impl(fn, idx_k, q_codes, q_scales, w, SegDesc{seq_row_off, 0, seq_len, max_len, idx_k.rows}, B,
+                         max_len, pool_blocks, k, pool_out, nullptr, scores_out, workspace, workspace_bytes, stream,
+                         1);
+}
+
+csa2_status csa2_index_full_topk(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,
+                                 const float* w, const int64_t* seq_row_off, const int32_t* seq_len, int B,
+                                 int max_len, int pool_blocks, int k, const int32_t* pool, int32_t* topk_out,
+                                 float* scores_out, void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "csa2_index_full_topk";
+  const csa2_status rc = index_full_args(fn, idx_k, B, max_len, pool_blocks, k);
+  if (rc != CSA2_OK || B == 0) return rc;
+  if (!seq_row_off) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  return index_full_impl(fn, idx_k, q_codes, q_scales, w, SegDesc{seq_row_off, 0, seq_len, max_len, idx_k.rows}, B,
+                         max_len, pool_blocks, k, const_cast<int32_t*>(pool), topk_out, scores_out, workspace,
+                         workspace_bytes, stream, 2);
 }
 
 csa2_status csa2_index_full_paged(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales,

@@ -130,6 +130,7 @@ class DecodeStep:
             self.ws_attn = [C.workspace(attn_bytes, dev) for _ in range(nL)]
             self.streams = [torch.cuda.Stream(device=dev) for _ in range(max(1, side_streams))]
             self.ev_idx = [torch.cuda.Event() for _ in range(nL)]
+            self.ev_pool = [torch.cuda.Event() for _ in range(nL)]
             self.ev_done = [torch.cuda.Event() for _ in range(nL)]
         else:
             ws_re, ws_attn = C.workspace(re_bytes, dev), C.workspace(attn_bytes, dev)
@@ -206,7 +207,18 @@ class DecodeStep:
                 if ev_ready is not None:
                     main.wait_event(ev_ready)
                 pool = self.pools[layer]
-                if self.queries is None:
+                if self.queries is None and self.concurrent and isinstance(seq_row_off, torch.Tensor):
+                    # the pool is ready before the Full layer's own Top-k: the
+                    # Reindex layers start from it while the Top-k is selected
+                    self._hook("csa2_index_full", "begin", main)
+                    C.csa2_index_full_pool(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len,
+                                           self.max_len, self.P, self.k, pool, self.ws_full, stream=main)
+                    self.ev_pool[layer].record(main)
+                    C.csa2_index_full_topk(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len,
+                                           self.max_len, self.P, self.k, pool, self.topk[layer], self.ws_full,
+                                           stream=main)
+                    self._hook("csa2_index_full", "end", main)
+                elif self.queries is None:
                     self._hook("csa2_index_full", "begin", main)
                     C.csa2_index_full(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len,
                                       self.max_len, self.P, self.k, pool, self.topk[layer], self.ws_full, stream=main)
@@ -220,7 +232,9 @@ class DecodeStep:
                 last = self.topk[layer]
                 if self.concurrent:
                     self.ev_idx[layer].record(main)
-                    pool_ev = last_ev = self.ev_idx[layer]
+                    last_ev = self.ev_idx[layer]
+                    pool_ev = self.ev_pool[layer] if self.queries is None and isinstance(seq_row_off, torch.Tensor) \
+                        else self.ev_idx[layer]
             if self.concurrent:
                 s = self.streams[side % len(self.streams)]
                 side += 1

@@ -103,7 +103,7 @@ class DecodeStep:
 
     def __init__(self, pattern: str, B: int, max_len: int, P: int = 2048, k: int = 512, full_rescan: bool = False,
                  device="cuda", sm_scale: float | None = None, concurrent: bool = True, side_streams: int = 3,
-                 ratio: int = 1, projection: bool = True, queries: int | None = None):
+                 ratio: int = 1, projection: bool = True, queries: int | None = None, split_full: bool = False):
         if ratio not in (1, 2):
             raise ValueError("ratio must be 1 or 2")
         if queries is not None and ratio != 1:
@@ -111,6 +111,10 @@ class DecodeStep:
         self.pattern, self.B, self.max_len, self.P, self.k = pattern, B, max_len, P, k
         self.ratio = ratio
         self.queries = queries
+        # concurrent steps only: issue the scanning Full layer as pool + Top-k,
+        # so that the Reindex layers start from the pool (they then compete
+        # with the Full layer's own pool scoring; measured no faster at B = 64)
+        self.split_full = split_full and concurrent
         nq = B if queries is None else queries  # segments of the calls after the scan
         self.plan = layer_plan(pattern, full_rescan)
         self.sm_scale = sm_scale if sm_scale is not None else 1.0 / math.sqrt(C.MAIN_DIM)
@@ -207,7 +211,8 @@ class DecodeStep:
                 if ev_ready is not None:
                     main.wait_event(ev_ready)
                 pool = self.pools[layer]
-                if self.queries is None and self.concurrent and isinstance(seq_row_off, torch.Tensor):
+                split = self.split_full and self.queries is None and isinstance(seq_row_off, torch.Tensor)
+                if split:
                     # the pool is ready before the Full layer's own Top-k: the
                     # Reindex layers start from it while the Top-k is selected
                     self._hook("csa2_index_full", "begin", main)
@@ -233,8 +238,7 @@ class DecodeStep:
                 if self.concurrent:
                     self.ev_idx[layer].record(main)
                     last_ev = self.ev_idx[layer]
-                    pool_ev = self.ev_pool[layer] if self.queries is None and isinstance(seq_row_off, torch.Tensor) \
-                        else self.ev_idx[layer]
+                    pool_ev = self.ev_pool[layer] if split else self.ev_idx[layer]
             if self.concurrent:
                 s = self.streams[side % len(self.streams)]
                 side += 1

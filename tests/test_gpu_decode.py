@@ -327,3 +327,25 @@ def test_verify_step_full_size_sampled():
         for layer in range(len(wl.pattern)):
             assert np.array_equal(host(step.topk[layer][qs]), ref["topk"][layer]), (b, layer)
             check_attention(host(step.out[layer][qs]), ref["out"][layer], what=f"seq {b} layer {layer}")
+
+
+def test_decode_with_the_full_layer_split_in_two_calls():
+    """csa2_index_full_pool + csa2_index_full_topk (split_full) give the same
+    bits as the single call, with the Reindex layers started from the pool."""
+    wl = W.DecodeWorkload("split_small", np.array([70000, 4096, 777]), "FRRU", needles=8)
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    caches_h = [W.full_cache_host(wl, f, layers[f]["q_codes"], layers[f]["q_scales"]) for f in wl.full_layers()]
+    caches_d = [FullCache(C.cache(dev(c["idx_codes"]), dev(c["idx_scales"])),
+                          C.cache(dev(c["main_codes"]), dev(c["main_scales"]))) for c in caches_h]
+    off_d, len_d = dev(caches_h[0]["seq_row_off"]), dev(wl.lengths.astype(np.int32))
+    dl = _device_layers(layers)
+    plain = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
+    split = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, split_full=True)
+    plain.run(caches_d, off_d, len_d, dl)
+    split.run(caches_d, off_d, len_d, dl)
+    torch.cuda.synchronize()
+    assert plain.device_flags() == 0 and split.device_flags() == 0
+    assert np.array_equal(host(split.pool), host(plain.pool))
+    for layer in range(len(wl.pattern)):
+        assert np.array_equal(host(split.topk[layer]), host(plain.topk[layer]))
+    assert np.array_equal(host(split.out), host(plain.out))

@@ -132,3 +132,29 @@ def test_reindex_flags_out_of_range_pool_block():
     assert C.device_status(ws) == 1       # CSA2_DEV_INDEX_RANGE
     got = host(top)[0]
     assert set(got[got >= 0].tolist()) == set(range(8, 16)) | set(range(40, 48))
+
+
+@pytest.mark.parametrize("qmin,qmax", [(100, 150), (2, 253)])
+def test_index_multi_extreme_scales(qmin, qmax):
+    """The multi-query scan applies the query block scales inside the MMA
+    when they lie in [8, 240] and in the epilogue otherwise; with wide key
+    and query exponent spreads (fp64 epilogue path) and out-of-range query
+    scales (epilogue scaling) the results stay bit-exact."""
+    rng = np.random.default_rng(qmin + qmax)
+    lengths = [3000, 2048, 777]
+    kc, ks, off, _ = _random_cache(rng, lengths, smin=90, smax=160)
+    m = np.array([3, 9, 2])
+    q_off = np.concatenate([[0], np.cumsum(m)]).astype(np.int32)
+    Q = int(q_off[-1])
+    qc, qs, w = _queries(rng, Q, smin=qmin, smax=qmax)
+    q_vis = np.concatenate([lengths[b] - np.arange(m[b])[::-1] * 5 for b in range(3)]).astype(np.int32)
+    P, k = 128, 100
+    pool = torch.full((Q, P), -7, dtype=torch.int32, device="cuda")
+    top = torch.full((Q, k), -7, dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_index_multi_workspace_bytes(3, Q, max(lengths), P, k))
+    C.csa2_index_multi(C.cache(dev(kc), dev(ks)), dev(qc), dev(qs), dev(w), dev(off), dev(q_off), dev(q_vis),
+                       max(lengths), P, k, pool, top, ws)
+    torch.cuda.synchronize()
+    assert C.device_status(ws) == 0
+    wp, wt = oracle.index_multi(kc, ks, qc, qs, w, off, q_off, q_vis, P, k)
+    assert np.array_equal(host(pool), wp) and np.array_equal(host(top), wt)

@@ -40,6 +40,7 @@
 // read from a group table that k_multi_prep builds, and every item loads its
 // group's own sequence rows.
 #include <algorithm>
+#include <cstddef>
 
 #include "device_common.cuh"
 #include "sm100.cuh"
@@ -87,7 +88,6 @@ struct __align__(1024) PfSmem {
   uint8_t a[kSt][kTileBytes];           // code rows, 64-byte swizzled
   uint8_t bop[kSt][kN * kIdxCodeBytes]; // B operand of the stage's group
   uint32_t sfb[kSt][2][32][4];          // query scale words per MMA: row r, word c = column 32c + r
-  int sfb_on[kSt];                      // the stage's group carries its query scales in the MMA
   uint32_t sc[kSt][kPT];                // E8M0 scale words of the rows
   int2 info[kSt];                       // (group, tile)
   QCtxS qctx[kSt][kQG];
@@ -99,7 +99,15 @@ struct __align__(1024) PfSmem {
   uint32_t tmem_base;
   int abort_flag;
   int built[kSt];                       // group whose B operand each stage holds
+  int sfb_on[kSt];                      // the stage's group carries its query scales in the MMA
 };
+// alignment the copies need: TMA tiles and MMA operands (1024 bytes, 64-byte
+// swizzle), tcgen05.cp sources and bulk-copy destinations (16 bytes)
+static_assert(offsetof(PfSmem, a) % 1024 == 0 && kTileBytes % 1024 == 0, "code tiles misaligned");
+static_assert(offsetof(PfSmem, bop) % 1024 == 0 && (kN * kIdxCodeBytes) % 1024 == 0, "B operand misaligned");
+static_assert(offsetof(PfSmem, sfb) % 16 == 0, "scale-factor copy source misaligned");
+static_assert(offsetof(PfSmem, sc) % 16 == 0 && (kPT * 4) % 16 == 0, "bulk-copy destination misaligned");
+static_assert(offsetof(PfSmem, full) % 8 == 0, "mbarriers misaligned");
 
 struct PfParams {
   const int4* groups;       // [n_groups] {sequence, first query, queries, 0}, or null: group g = queries 8g..

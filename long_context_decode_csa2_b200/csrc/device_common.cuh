@@ -162,43 +162,6 @@ __device__ __forceinline__ float exact_score(const uint32_t (&v)[16], const KeyS
   return sc;
 }
 
-// The same score from accumulators that already carry the query's block
-// scales: v[4h+b] = D_{h,b}/4 * 2^(eq-127) exactly (the MMA applied them).
-// Only the key's block scales remain; every product and partial sum equals
-// the one exact_score forms, so the result is bit-identical.
-__device__ __forceinline__ float exact_score_qscaled(const uint32_t (&v)[16], const KeyScale& ks, const IdxQCtx& q) {
-  const bool fast = (ks.kmax - ks.kmin + q.qspread <= 9) && (q.qlo + ks.kmin - 254 >= -100) &&
-                    (q.qhi + ks.kmax - 254 <= 100);
-  float d[kHi];
-  if (fast) {
-    float kf[4];
-#pragma unroll
-    for (int bb = 0; bb < 4; ++bb)  // 2^(ek-127), exact (byte 0: the subnormal 2^-127)
-      kf[bb] = __uint_as_float(ks.kb[bb] ? uint32_t(ks.kb[bb]) << 23 : 0x00200000u);
-#pragma unroll
-    for (int h = 0; h < kHi; ++h) {
-      float acc = __fmul_rn(__uint_as_float(v[4 * h]), kf[0]);
-#pragma unroll
-      for (int bb = 1; bb < 4; ++bb) acc = __fmaf_rn(__uint_as_float(v[4 * h + bb]), kf[bb], acc);
-      d[h] = acc;
-    }
-  } else {
-#pragma unroll
-    for (int h = 0; h < kHi; ++h) {
-      double acc = 0.0;
-#pragma unroll
-      for (int bb = 0; bb < 4; ++bb)
-        acc = __dadd_rn(acc, __dmul_rn(double(__uint_as_float(v[4 * h + bb])), pow2d(ks.kb[bb] - 127)));
-      d[h] = __double2float_rn(acc);
-    }
-  }
-  float sc = __fmul_rn(q.w[0], d[0]);
-#pragma unroll
-  for (int h = 1; h < kHi; ++h) sc = __fmaf_rn(q.w[h], d[h], sc);
-  if (sc == 0.0f) sc = 0.0f;
-  return sc;
-}
-
 __device__ __forceinline__ float exact_score(const uint32_t (&v)[16], uint32_t sw, const IdxQCtx& q) {
   return exact_score(v, key_scale(sw), q);
 }

@@ -17,19 +17,13 @@
 //     changes it also writes the group's B operand, 128 rows of which row
 //     16j + 4h + b holds block b of head h of query j (zeros elsewhere), and
 //     the queries' scale contexts;
-//   * warp 1 copies the group's query block scales into tensor memory
-//     (tcgen05.cp) and issues two tcgen05.mma kind::mxf4 (M = 128 positions,
-//     N = 128, K = 64) with key scales 1 and the query scales: column n holds
-//     a single query block, so its accumulator is that block's exact dot
-//     D/4 times 2^(eq-127), a single exact product;
+//   * warp 1 issues two tcgen05.mma kind::mxf4 (M = 128 positions, N = 128,
+//     K = 64) with every block scale = 1, so each accumulator is an exact
+//     block dot D/4;
 //   * four teams of four epilogue warps (two of the eight queries each) read
-//     each position's 16 accumulators per query, apply the key's block
-//     scales and form the exact score (the same rounding as the decode scan),
-//     mask positions the query cannot see, and write the maximum of every 8
-//     positions as one rank key.
-// A group with query scale bytes outside [8, 240] (where D/4 * 2^(eq-127)
-// could leave the fp32 normal range) runs with unit query scales and applies
-// them in the epilogue instead.
+//     each position's 16 accumulators per query, form the exact score (the
+//     same rounding as the decode scan), mask positions the query cannot see,
+//     and write the maximum of every 8 positions as one rank key.
 // Items past the visibility of every query of a group are skipped by all
 // roles alike.  Every wait is time-bounded (CSA2_DEV_TIMEOUT on expiry).
 //
@@ -55,18 +49,13 @@ constexpr int kPT = 128;                 // positions per item (MMA M)
 constexpr int kSt = 6;                   // smem ring
 constexpr int kAc = 3;                   // TMEM accumulator ring, kN columns each
 constexpr int kTmemCols = 512;
-// Scale factors in tensor memory (layout of kind::mxf4 with M = N = 128: the
-// factor of A row m / B column n for the MMA's K-block j sits in lane m /
-// (every lane quarter) n % 32, column base + m / 32 / n / 32, byte j).
-constexpr uint32_t kSfa = 384;           // key scales: 4 columns, all 2^0
-constexpr uint32_t kSfb = 392;           // query scales: 8 columns per stage (2 MMAs x 4)
+constexpr uint32_t kSf = 448;            // scale-factor columns (all 2^0)
 constexpr int kTeams = 4;                // epilogue teams of 4 warps, all on every item
 constexpr int kQPT = kQG / kTeams;       // queries per team and item
 constexpr int kEpiWarps = 4 * kTeams;
 constexpr int kThr = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
 constexpr uint32_t kTileBytes = kPT * kIdxCodeBytes;
-static_assert(kAc * kN <= int(kSfa), "TMEM accumulators overlap the scale factors");
-static_assert(kSfb + 8 * kSt <= uint32_t(kTmemCols), "scale factors exceed the allocation");
+static_assert(kAc * kN <= int(kSf), "TMEM accumulators overlap the scale factors");
 
 struct __align__(16) QCtxS {
   IdxQCtx c;
@@ -87,7 +76,6 @@ __device__ __forceinline__ QCtxS load_qctx(const QCtxS& src) {
 struct __align__(1024) PfSmem {
   uint8_t a[kSt][kTileBytes];           // code rows, 64-byte swizzled
   uint8_t bop[kSt][kN * kIdxCodeBytes]; // B operand of the stage's group
-  uint32_t sfb[kSt][2][32][4];          // query scale words per MMA: row r, word c = column 32c + r
   uint32_t sc[kSt][kPT];                // E8M0 scale words of the rows
   int2 info[kSt];                       // (group, tile)
   QCtxS qctx[kSt][kQG];
@@ -99,13 +87,11 @@ struct __align__(1024) PfSmem {
   uint32_t tmem_base;
   int abort_flag;
   int built[kSt];                       // group whose B operand each stage holds
-  int sfb_on[kSt];                      // the stage's group carries its query scales in the MMA
 };
 // alignment the copies need: TMA tiles and MMA operands (1024 bytes, 64-byte
-// swizzle), tcgen05.cp sources and bulk-copy destinations (16 bytes)
+// swizzle), bulk-copy destinations (16 bytes)
 static_assert(offsetof(PfSmem, a) % 1024 == 0 && kTileBytes % 1024 == 0, "code tiles misaligned");
 static_assert(offsetof(PfSmem, bop) % 1024 == 0 && (kN * kIdxCodeBytes) % 1024 == 0, "B operand misaligned");
-static_assert(offsetof(PfSmem, sfb) % 16 == 0, "scale-factor copy source misaligned");
 static_assert(offsetof(PfSmem, sc) % 16 == 0 && (kPT * 4) % 16 == 0, "bulk-copy destination misaligned");
 static_assert(offsetof(PfSmem, full) % 8 == 0, "mbarriers misaligned");
 
@@ -175,23 +161,6 @@ __device__ __forceinline__ void build_group(PfSmem& sm, int s, const PfParams& p
       *reinterpret_cast<uint4*>(bo + n * 64 + ((b ^ ((n >> 1) & 3)) << 4)) = v;
     }
   }
-  // query scales into the MMA when every one of the group's lies in [8, 240]
-  bool in_range = true;
-  for (int e = lane; e < gr.nq * kHi * 4; e += 32) {
-    const int v = __ldg(p.q_scales + int64_t(gr.q0) * kHi * 4 + e);
-    in_range = in_range && v >= 8 && v <= 240;
-  }
-  const bool scaled = __all_sync(0xffffffffu, in_range);
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {  // 256 words: (MMA kk, row r, word c) for column n = 32c + r
-    const int wi = lane + 32 * m, kk = wi >> 7, r = (wi >> 2) & 31, c = wi & 3;
-    const int n = 32 * c + r, j = n >> 4, h = (n >> 2) & 3, b = n & 3;
-    uint32_t eq = 127;
-    if (scaled && j < gr.nq) eq = __ldg(p.q_scales + int64_t(gr.q0 + j) * kHi * 4 + h * 4 + b);
-    const uint32_t b0 = (b == 2 * kk) ? eq : 127u, b1 = (b == 2 * kk + 1) ? eq : 127u;
-    sm.sfb[s][kk][r][c] = b0 | (b1 << 8) | 0x7F7F0000u;
-  }
-  if (lane == 0) sm.sfb_on[s] = scaled ? 1 : 0;
   if (lane < kQG) {
     const int qi = gr.q0 + lane;
     QCtxS& q = sm.qctx[s][lane];
@@ -239,9 +208,10 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp >= 2 && warp < 6) {  // unit key scales (columns kSfa .. kSfa+7)
+  if (warp >= 2 && warp < 6) {  // unit block scales in columns kSf .. kSf+63
     const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
-    sm100::tmem_st8_same(tmem + lane_base + kSfa, 0x7F7F7F7Fu);
+#pragma unroll
+    for (int c = 0; c < 64; c += 8) sm100::tmem_st8_same(tmem + lane_base + kSf + c, 0x7F7F7F7Fu);
     sm100::tmem_st_wait();
   }
   sm100::tc_fence_before();
@@ -295,7 +265,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = sm100::idesc_mxf4(kPT, kN);
-      const uint32_t sfa = tmem + kSfa;
+      const uint32_t sfa = tmem + kSf, sfb = tmem + kSf + 32;
       int t = 0, cg = -1, gmax = 0;
       for (int it = i0; it < i1; ++it) {
         const int g = it / p.n_tiles, tile = it - g * p.n_tiles;
@@ -317,13 +287,10 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
         sm100::tc_fence_after();
         const uint32_t abase = sm100::smem_u32(sm.a[s]);
         const uint32_t bbase = sm100::smem_u32(sm.bop[s]);
-        const uint32_t sfb = tmem + kSfb + 8u * uint32_t(s);
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) sm100::tmem_cp_32x128b_x4(sfb + 4u * kk, sm100::smem_u32(&sm.sfb[s][kk][0][0]));
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
           sm100::mma_mxf4(tmem + a * kN, sm100::smem_desc_k64b(abase + kk * 32), sm100::smem_desc_k64b(bbase + kk * 32),
-                          idesc, uint32_t(kk), sfa, sfb + 4u * kk);
+                          idesc, uint32_t(kk), sfa, sfb);
         sm100::mma_commit(&sm.empty[s]);
         sm100::mma_commit(&sm.tfull[a]);
         ++t;
@@ -360,7 +327,6 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       const int pl = 32 * q4 + lane;
       const int64_t pos = int64_t(tile) * kPT + pl;
       const KeyScale ks = key_scale(sm.sc[s][pl]);
-      const bool scaled = sm.sfb_on[s] != 0;
       const uint32_t tcol = tmem + lane_base + uint32_t(a * kN);
       uint32_t v[kQPT][16];
 #pragma unroll
@@ -372,7 +338,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
         const int j = j0 + jj;
         const QCtxS q = load_qctx(sm.qctx[s][j]);
         uint32_t key = 0;
-        if (pos < q.vis) key = rank_key(scaled ? exact_score_qscaled(v[jj], ks, q.c) : exact_score(v[jj], ks, q.c));
+        if (pos < q.vis) key = rank_key(exact_score(v[jj], ks, q.c));
         key = group8_max(key);
         if ((lane & 7) == 0 && pos < q.vis)
           p.bkeys[int64_t(gr.q0 + j) * p.nb_stride + pos / kBlk] = key;

@@ -188,19 +188,6 @@ __device__ __forceinline__ uint64_t smem_desc_k64b(uint32_t saddr) {
   return d;
 }
 
-// Copy of a 32-row x 16-byte shared-memory matrix (rows 16 bytes apart, no
-// swizzle) into tensor memory: row r lands in lane r of every lane quarter,
-// the 16 bytes in 4 consecutive columns from taddr.  Ordered before later
-// tcgen05.mma issued by the same thread.
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint32_t saddr) {
-  uint64_t d = 0;
-  d |= uint64_t((saddr >> 4) & 0x3FFFu);      // start address
-  d |= uint64_t((128 >> 4) & 0x3FFFu) << 16;  // leading byte offset
-  d |= uint64_t((128 >> 4) & 0x3FFFu) << 32;  // stride byte offset: 8-row groups 128 bytes apart
-  d |= uint64_t(1) << 46;                     // version; no swizzle
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
-}
-
 // Instruction descriptor of kind::mxf4 (E2M1 x E2M1, E8M0 scales, fp32
 // accumulate), both operands K-major, M x N tile.
 __host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {

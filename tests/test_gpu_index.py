@@ -136,12 +136,10 @@ def test_reindex_flags_out_of_range_pool_block():
 
 @pytest.mark.parametrize("qmin,qmax", [(100, 150), (2, 200)])
 def test_index_multi_extreme_scales(qmin, qmax):
-    """The multi-query scan applies the query block scales inside the MMA
-    when they lie in [8, 240] and in the epilogue otherwise; with wide key
-    and query exponent spreads (fp64 epilogue path) and out-of-range query
-    scales (epilogue scaling) the results stay bit-exact.  Scales stay low
-    enough that no score overflows: an infinite head sum can turn into NaN,
-    whose bits differ between the CPU and the GPU."""
+    """The multi-query scan with wide key and query exponent spreads (its
+    fp64 epilogue path) and query scale bytes far from 127 stays bit-exact.
+    Scales stay low enough that no score overflows: an infinite head sum can
+    turn into NaN, whose bits differ between the CPU and the GPU."""
     rng = np.random.default_rng(qmin + qmax)
     lengths = [3000, 2048, 777]
     kc, ks, off, _ = _random_cache(rng, lengths, smin=90, smax=160)

@@ -149,3 +149,36 @@ def test_paged_bad_page_id_is_flagged():
     step.run([_device_caches(c)], C.PageTable(dev(table), 512), dev(wl.lengths.astype(np.int32)), _layers_dev([L0]))
     torch.cuda.synchronize()
     assert step.device_flags() & 2  # CSA2_DEV_ROW_LAYOUT
+
+
+def test_paged_ratio2_decode_steps_equal_contiguous():
+    """Ratio-2 decode through a page table: appends land in the pages and
+    every step's results equal the contiguous layout's."""
+    lens0 = np.array([4000, 1030, 2048], np.int64)
+    room, steps, page_rows = 24, 5, 512
+    wl = W.DecodeWorkload("paged_r2", lens0, "FRRU", needles=8, ratio=2, room=room)
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    c = W.full_cache_host(wl, 0, layers[0]["q_codes"], layers[0]["q_scales"])
+    off = c["seq_row_off"]
+    caps = [int(x) for x in (lens0 + room + 7) // 8 * 8]
+    table, n_pages = _page_table(caps, page_rows, 2, seed=9)
+    paged_c = _to_pages(c, off, caps, table, page_rows, n_pages, seed=10)
+    dl = _layers_dev(layers)
+    plain = DecodeStep(wl.pattern, wl.B, wl.max_len + room, wl.P, wl.k, ratio=2, projection=False)
+    paged = DecodeStep(wl.pattern, wl.B, wl.max_len + room, wl.P, wl.k, ratio=2, projection=False)
+    cp, cg = _device_caches(c), _device_caches(paged_c)
+    len_p, len_g = dev(lens0.astype(np.int32)), dev(lens0.astype(np.int32))
+    pt = C.PageTable(dev(table), page_rows)
+    import synth
+    for t in range(steps):
+        tok = dict(raw=dev(synth.normal_bf16(90, synth.T_RAW, t, 0, wl.B * 512).reshape(wl.B, 512)),
+                   logit=dev(synth.normal_f32(90, synth.T_LOGITS, t, 0, wl.B)),
+                   idx_raw=dev(synth.normal_bf16(90, synth.T_IDXRAW, t, 0, wl.B * 128).reshape(wl.B, 128)))
+        plain.run([cp], dev(off), len_p, dl, new_tokens=[tok])
+        paged.run([cg], pt, len_g, dl, new_tokens=[tok])
+        torch.cuda.synchronize()
+        for layer in range(len(wl.pattern)):
+            assert np.array_equal(host(paged.topk[layer]), host(plain.topk[layer])), (t, layer)
+        assert np.array_equal(host(paged.out), host(plain.out)), t
+    assert plain.device_flags() == 0 and paged.device_flags() == 0
+    assert host(len_g).tolist() == host(len_p).tolist() == (lens0 + steps // 2).tolist()

@@ -147,7 +147,6 @@ class DecodeStep:
         self.topk = [torch.full((nq, k), -1, dtype=torch.int32, device=dev) for _ in range(nL)]
         self.out = torch.zeros((nL, nq, C.Q_HEADS, C.MAIN_DIM), dtype=torch.float32, device=dev)
         self.lse = torch.zeros((nL, nq, C.Q_HEADS), dtype=torch.float32, device=dev)
-        self.scores = None
         # ratio 2: one pending-token state per Full layer's caches
         n_full = sum(1 for m in pattern if m == "F")
         self.pairs = [PairStream(B, dev, projection) for _ in range(n_full)] if ratio == 2 else []

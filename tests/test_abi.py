@@ -116,3 +116,40 @@ def test_compress_stream_validation():
     assert call(pend_raw=FAKE + 8) == -1                    # misaligned pending row
     assert call(raw=None) == -1                             # tokens but no raw rows
     assert call(ws_bytes=256) == -3                         # no room for the counters
+
+
+def test_widened_calls_validation():
+    """The verification, paged, context-parallel and split calls check their
+    arguments on the host and launch nothing when they fail."""
+    L = C.lib()
+    c = _cache()
+    # csa2_index_multi: pool smaller than k, queries without sequences, max_vis past the cache
+    args = [c, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE]
+    assert L.csa2_index_multi(*args, 2, 6, 100, 64, 512, FAKE, FAKE, None, FAKE, 1 << 30, None) == -2
+    assert L.csa2_index_multi(*args, 0, 6, 100, 512, 512, FAKE, FAKE, None, FAKE, 1 << 30, None) == -1
+    assert L.csa2_index_multi(*args, 2, 6, 4096, 512, 512, FAKE, FAKE, None, FAKE, 1 << 30, None) == -1
+    assert L.csa2_index_multi(*args, 2, 6, 100, 512, 512, FAKE, FAKE, None, FAKE, 16, None) == -3
+    assert L.csa2_index_multi(*args, 2, 0, 100, 512, 512, FAKE, FAKE, None, FAKE, 16, None) == 0
+    # paged calls: page size not a power of two / below 512, cache not a whole number of pages
+    assert L.csa2_index_full_paged(_cache(rows=2048), FAKE, FAKE, FAKE, FAKE, 768, 4, FAKE, 2, 1000, 64, 64, FAKE,
+                                   FAKE, None, FAKE, 1 << 30, None) == -1
+    assert L.csa2_index_full_paged(_cache(rows=2048), FAKE, FAKE, FAKE, FAKE, 256, 4, FAKE, 2, 1000, 64, 64, FAKE,
+                                   FAKE, None, FAKE, 1 << 30, None) == -1
+    assert L.csa2_index_full_paged(_cache(rows=1000), FAKE, FAKE, FAKE, FAKE, 512, 4, FAKE, 2, 1000, 64, 64, FAKE,
+                                   FAKE, None, FAKE, 1 << 30, None) == -1
+    assert L.csa2_sparse_attn_decode_paged(FAKE, _cache(rows=1024), None, 512, 4, FAKE, FAKE, 512, FAKE, FAKE, FAKE,
+                                           0.1, FAKE, None, 2, FAKE, 1 << 30, None) == -1
+    assert L.csa2_index_reindex_paged(_cache(rows=1024), FAKE, FAKE, FAKE, FAKE, 512, 0, FAKE, FAKE, 2, 64, 64, FAKE,
+                                      FAKE, 1 << 30, None) == -1
+    # context parallelism: block must be 1 or 8; merge k out of range; too small a workspace; combine needs G >= 1
+    assert L.csa2_score_positions(c, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 4, FAKE, FAKE, 256, None) == -1
+    assert L.csa2_topk_merge(FAKE, FAKE, None, 2, 3, 100, 0, None, None, FAKE, None, FAKE, 1 << 20, None) == -1
+    assert L.csa2_topk_merge(FAKE, FAKE, None, 2, 3, 100, 64, None, None, FAKE, None, FAKE, 256, None) == -3
+    assert L.csa2_topk_merge(FAKE, FAKE, None, 2, 3, 100, 64, None, None, FAKE, FAKE, FAKE, 1 << 20, None) == -1
+    assert L.csa2_attn_combine(FAKE, FAKE, 0, 2, FAKE, None, None) == -1
+    assert L.csa2_topk_merge_workspace_bytes(3, 4, 100) > L.csa2_topk_merge_workspace_bytes(2, 4, 100)
+    # split Full layer: the same checks as csa2_index_full
+    assert L.csa2_index_full_pool(c, FAKE, FAKE, FAKE, None, FAKE, 2, 1000, 0, 64, FAKE, None, FAKE, 1 << 30,
+                                  None) == -1
+    assert L.csa2_index_full_topk(c, FAKE, FAKE, FAKE, None, FAKE, 2, 1000, 64, 64, FAKE, FAKE, None, FAKE, 1 << 30,
+                                  None) == -1

@@ -806,8 +806,25 @@ def run_reference(args):
 
     import synth.workloads as W
 
-    wl = W.decode_workloads()[args.workload]
     nthreads = min(os.cpu_count() or 1, 8)
+    if args.workload.startswith("prefill"):
+        # the oracle's prefill step, estimated from a bounded sample per timed step
+        pw = W.prefill_workload()
+        runs = [prefill_cpu_baseline(pw, pw.seed, nthreads) for _ in range(max(1, min(args.steps, 3)))]
+        value = statistics.median(r["value"] for r in runs)
+        ms = 1e3 * pw.T / value
+        print(json.dumps({"impl": "reference", "metric": "prefill queries/sec (ratio-2 compression of 262144 tokens, "
+                          "4096-query causal chunk)", "value": value, "unit": "queries/s", "n_gpus": world,
+                          "steps": len(runs), "warmup": 0, "ms_per_step": ms, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "int32+f64 (CPU oracle)",
+                          "data": "synthetic",
+                          "config": {"workload": pw.name, "raw_tokens": pw.n_raw, "entries": pw.n_entries,
+                                     "queries": pw.T, "pool_blocks": pw.P, "topk": pw.k, "window": 128},
+                          "cpu_baseline": dict(runs[0], value=value),
+                          "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return
+    wl = W.decode_workloads()[args.workload]
     if torch.cuda.is_available():
         # inputs from the device generator (same bytes as the NumPy generator)
         wl2, layers, caches_dev, _, _, _, _ = build_workload(wl, 0, torch.device("cuda", 0))

@@ -49,6 +49,8 @@ def parse():
                     help="issue every call on one stream (isolated per-call times) instead of the concurrent tail")
     ap.add_argument("--context", type=int, default=0,
                     help="override every sequence's length (small profiling captures of the attention)")
+    ap.add_argument("--full-rescan", action="store_true",
+                    help="every Full layer scans its whole context and rebuilds the pool (default: only the first)")
     ap.add_argument("--cp", type=int, default=0,
                     help="context-parallel step over this many shards of every sequence: one per rank under "
                          "torchrun, all in this process on one GPU")
@@ -63,7 +65,7 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def algorithmic_bytes(wl):
+def algorithmic_bytes(wl, full_rescan=False):
     """Per step, from the method's own reads (no scratch traffic):
     Full scan L*68 B; each pool-scored layer min(16384, 8*ceil(L/8))*68 B
     (the Full layer re-scores its pool for its own Top-512, each Reindex layer
@@ -71,7 +73,8 @@ def algorithmic_bytes(wl):
     L = wl.lengths.astype(np.int64)
     n_scan = sum(1 for _, m in enumerate(wl.pattern) if m == "F")
     n_pool = sum(1 for m in wl.pattern if m in "FR")
-    scan = int((L * 68).sum()) * 1  # only the first Full layer scans (default plan)
+    # only the first Full layer scans (default plan); with full_rescan every one does
+    scan = int((L * 68).sum()) * (n_scan if full_rescan else 1)
     # a verification step scores and attends per query, but reads each
     # sequence's indexer K once
     Lq = wl.verify_queries()[1].astype(np.int64) if wl.queries_per_seq else L
@@ -205,12 +208,14 @@ def time_oracle(wl, samples, nthreads, jobs=None):
 
 # ----------------------------------------------------------------------------
 
-def decode_config(wl, l2_bytes, sequential, graph=True):
+def decode_config(wl, l2_bytes, sequential, graph=True, full_rescan=False):
     """The `config` object of a decode line (both arms)."""
     extra = ({"ratio": 2, "append": "one raw token per sequence per Full layer per step (csa2_compress_stream, "
                                     "W_idx projection)"} if wl.ratio == 2 else {})
     if wl.page_rows:
         extra["paged"] = "%d-row pages, page table shuffled over the whole cache pool" % wl.page_rows
+    if wl.pattern.count("F") > 1:
+        extra["full_layers"] = "every Full layer scans" if full_rescan else "the first Full layer scans, the others select in its pool"
     if wl.queries_per_seq:
         extra["queries_per_seq"] = wl.queries_per_seq
         extra["verify"] = ("candidate i sees all entries but the last %d - i; value counts candidate queries"
@@ -339,7 +344,7 @@ def run_ours(args):
     m = wl.queries_per_seq
     n_q = wl.B * m if m else wl.B  # queries per step on this rank
     step = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=not args.sequential,
-                      ratio=wl.ratio, queries=n_q if m else None)
+                      ratio=wl.ratio, queries=n_q if m else None, full_rescan=args.full_rescan)
     vq = {}
     if m:
         q_off_h, q_vis_h = wl.verify_queries()
@@ -422,7 +427,7 @@ def run_ours(args):
     seq_ms = None
     if graph is not None and not args.sequential:
         step_seq = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=False, ratio=wl.ratio,
-                              queries=n_q if m else None)
+                              queries=n_q if m else None, full_rescan=args.full_rescan)
         step_seq.run(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
         g_seq = step_seq.capture(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
         for _ in range(3):
@@ -528,10 +533,11 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e2e_ms, device, world)
     flags = step.device_flags()
 
-    ab = algorithmic_bytes(wl)
+    ab = algorithmic_bytes(wl, args.full_rescan)
     peak, peak_kind = measured_peaks()
     full_avg = sum(full_ms) / len(full_ms)
-    full_bytes = ab["scan"] + ab["pool"] // max(1, sum(1 for m in wl.pattern if m in "FR"))
+    full_bytes = (ab["scan"] // (ab["n_full"] if args.full_rescan else 1)
+                  + ab["pool"] // max(1, sum(1 for m in wl.pattern if m in "FR")))
     achieved = full_bytes / (full_avg * 1e-3) / 1e9
     traffic = None
     prof = os.path.join(ROOT, "profiles", "index_full_traffic.json")
@@ -574,7 +580,7 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "int32+f64 indexer, f16 tensor-core attention (f32 accumulate)",
             "data": "synthetic",
-            "config": decode_config(wl, ab["total"], args.sequential, graph is not None),
+            "config": decode_config(wl, ab["total"], args.sequential, graph is not None, args.full_rescan),
             "tokens_per_s": job_throughput(world, n_q, ms),
             "hbm_algorithmic_gbs": ab["total"] / (ms * 1e-3) / 1e9,
             "hbm_frac_of_8tbs": ab["total"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,

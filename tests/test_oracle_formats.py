@@ -93,7 +93,9 @@ def test_mxfp4_roundtrip_all_codes_and_scales(orc):
         for c in range(16):
             v = float(e2m1_from_bits(c) * pow2(s - 127))
             anchor = float(6 * pow2(s - 127))
-            if not (np.isfinite(np.float32(anchor)) and np.float32(anchor) == anchor and np.float32(v) == v):
+            with np.errstate(over="ignore"):                # scales past fp32's range are skipped
+                a32, v32 = np.float32(anchor), np.float32(v)
+            if not (np.isfinite(a32) and a32 == anchor and v32 == v):
                 continue
             blk = np.full(32, 0.0, np.float32)
             blk[0], blk[1] = v, anchor

@@ -831,7 +831,8 @@ def run_reference(args):
                                   "d2h_bytes_per_step": 0}}))
         return
     wl = W.decode_workloads()[args.workload]
-    if torch.cuda.is_available():
+    on_gpu = torch.cuda.is_available()
+    if on_gpu:
         # inputs from the device generator (same bytes as the NumPy generator)
         wl2, layers, caches_dev, _, _, _, _ = build_workload(wl, 0, torch.device("cuda", 0))
         seqs = list(range(nthreads))
@@ -875,6 +876,9 @@ def run_reference(args):
                                       f"{len(samples)} sequences of the workload, {nthreads} host threads at a "
                                       f"time; {secs:.1f} s"},
            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if not on_gpu:  # the GPU arm's cache and launch notes do not describe a host-only run
+        res["config"]["l2"] = "host-only run (no GPU): contexts shortened to %d" % wl.max_len
+        res["config"].pop("schedule")
     print(json.dumps(res))
 
 

@@ -111,6 +111,48 @@ def _ptr(t):
     return t.data_ptr()
 
 
+# Element types of the C ABI's pointer arguments and the torch dtypes that
+# may carry them (same width, same kind of number).
+_KINDS = {
+    "u8": (torch.uint8, torch.int8, torch.float8_e4m3fn),   # E2M1 codes, E8M0 scales, E4M3 bytes
+    "bf16": (torch.bfloat16, torch.int16, torch.uint16),    # bf16 bit patterns
+    "i32": (torch.int32, torch.uint32),                     # int32 ids / lengths, uint32 keys and flags
+    "f32": (torch.float32,),
+    "i64": (torch.int64, torch.uint64),
+}
+
+
+def _arg(fn, name, t, kind, numel=0):
+    """Device pointer of an optional tensor argument, after checking that its
+    elements have the C type's width and kind and that it holds at least
+    `numel` of them (the library cannot see buffer sizes)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise Csa2Error(-1, fn, f"{name}: expected a torch tensor, got {type(t).__name__}")
+    if t.dtype not in _KINDS[kind]:
+        raise Csa2Error(-1, fn, f"{name}: {kind} elements expected, got {t.dtype}")
+    if t.numel() < numel:
+        raise Csa2Error(-1, fn, f"{name}: at least {numel} elements expected, got {t.numel()}")
+    return _ptr(t)
+
+
+def _queries(fn, n, q_codes, q_scales, w):
+    """Pointers of n indexer queries: codes [n][4][64], scales [n][4][4], weights [n][4]."""
+    return (_arg(fn, "q_codes", q_codes, "u8", n * IDX_HEADS * IDX_DIM // 2),
+            _arg(fn, "q_scales", q_scales, "u8", n * IDX_HEADS * IDX_DIM // 32),
+            _arg(fn, "w", w, "f32", n * IDX_HEADS))
+
+
+def _window(fn, n, win, win_scale, win_len):
+    return (_arg(fn, "win", win, "u8", n * WINDOW * MAIN_DIM), _arg(fn, "win_scale", win_scale, "f32", n),
+            _arg(fn, "win_len", win_len, "i32", n))
+
+
+def _attn_out(fn, n, out, lse):
+    return _arg(fn, "out", out, "f32", n * Q_HEADS * MAIN_DIM), _arg(fn, "lse", lse, "f32", n * Q_HEADS)
+
+
 def _stream(stream):
     s = stream if stream is not None else torch.cuda.current_stream()
     return C.c_void_p(s.cuda_stream)
@@ -159,41 +201,60 @@ def csa2_index_full_workspace_bytes(B, max_len, pool_blocks, k):
     return lib().csa2_index_full_workspace_bytes(B, max_len, pool_blocks, k)
 
 
+def _full_args(fn, q_codes, q_scales, w, seq_len, max_len, pool_blocks, k, pool_out, topk_out, scores_out):
+    B = seq_len.shape[0]
+    return (B, *_queries(fn, B, q_codes, q_scales, w), _arg(fn, "seq_len", seq_len, "i32", B),
+            _arg(fn, "pool_out", pool_out, "i32", B * pool_blocks), _arg(fn, "topk_out", topk_out, "i32", B * k),
+            _arg(fn, "scores_out", scores_out, "f32", B * max_len))
+
+
+def _row_off(fn, seq_row_off, B):
+    return _arg(fn, "seq_row_off", seq_row_off, "i64", B)
+
+
+def _pages(fn, pt, B):
+    return _arg(fn, "pages", pt.pages, "i32", B * pt.max_pages)
+
+
 def csa2_index_full(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, max_len, pool_blocks, k, pool_out, topk_out,
                     ws, scores_out=None, stream=None):
-    B = seq_len.shape[0]
     wp, wn = _ws(ws)
     if isinstance(seq_row_off, PageTable):
-        pt = seq_row_off
-        rc = lib().csa2_index_full_paged(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(pt.pages), pt.page_rows,
-                                         pt.max_pages, _ptr(seq_len), B, max_len, pool_blocks, k, _ptr(pool_out),
-                                         _ptr(topk_out), _ptr(scores_out), wp, wn, _stream(stream))
-        _check(rc, "csa2_index_full_paged")
+        fn, pt = "csa2_index_full_paged", seq_row_off
+        B, qc, qs, wv, sl, po, to, so = _full_args(fn, q_codes, q_scales, w, seq_len, max_len, pool_blocks, k,
+                                                   pool_out, topk_out, scores_out)
+        rc = lib().csa2_index_full_paged(idx_k, qc, qs, wv, _pages(fn, pt, B), pt.page_rows, pt.max_pages, sl, B,
+                                         max_len, pool_blocks, k, po, to, so, wp, wn, _stream(stream))
+        _check(rc, fn)
         return
-    rc = lib().csa2_index_full(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len), B,
-                               max_len, pool_blocks, k, _ptr(pool_out), _ptr(topk_out), _ptr(scores_out), wp, wn,
-                               _stream(stream))
-    _check(rc, "csa2_index_full")
+    fn = "csa2_index_full"
+    B, qc, qs, wv, sl, po, to, so = _full_args(fn, q_codes, q_scales, w, seq_len, max_len, pool_blocks, k, pool_out,
+                                               topk_out, scores_out)
+    rc = lib().csa2_index_full(idx_k, qc, qs, wv, _row_off(fn, seq_row_off, B), sl, B, max_len, pool_blocks, k, po,
+                               to, so, wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_index_full_pool(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, max_len, pool_blocks, k, pool_out, ws,
                          scores_out=None, stream=None):
-    B = seq_len.shape[0]
+    fn = "csa2_index_full_pool"
     wp, wn = _ws(ws)
-    rc = lib().csa2_index_full_pool(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len),
-                                    B, max_len, pool_blocks, k, _ptr(pool_out), _ptr(scores_out), wp, wn,
-                                    _stream(stream))
-    _check(rc, "csa2_index_full_pool")
+    B, qc, qs, wv, sl, po, _, so = _full_args(fn, q_codes, q_scales, w, seq_len, max_len, pool_blocks, k, pool_out,
+                                              None, scores_out)
+    rc = lib().csa2_index_full_pool(idx_k, qc, qs, wv, _row_off(fn, seq_row_off, B), sl, B, max_len, pool_blocks, k,
+                                    po, so, wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_index_full_topk(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, max_len, pool_blocks, k, pool, topk_out,
                          ws, scores_out=None, stream=None):
-    B = seq_len.shape[0]
+    fn = "csa2_index_full_topk"
     wp, wn = _ws(ws)
-    rc = lib().csa2_index_full_topk(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len),
-                                    B, max_len, pool_blocks, k, _ptr(pool), _ptr(topk_out), _ptr(scores_out), wp, wn,
-                                    _stream(stream))
-    _check(rc, "csa2_index_full_topk")
+    B, qc, qs, wv, sl, po, to, so = _full_args(fn, q_codes, q_scales, w, seq_len, max_len, pool_blocks, k, pool,
+                                               topk_out, scores_out)
+    rc = lib().csa2_index_full_topk(idx_k, qc, qs, wv, _row_off(fn, seq_row_off, B), sl, B, max_len, pool_blocks, k,
+                                    po, to, so, wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_index_reindex_workspace_bytes(B, pool_blocks, k):
@@ -203,52 +264,70 @@ def csa2_index_reindex_workspace_bytes(B, pool_blocks, k):
 def csa2_index_reindex(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, pool, k, topk_out, ws, stream=None):
     B, P = pool.shape
     wp, wn = _ws(ws)
-    if isinstance(seq_row_off, PageTable):
+    paged = isinstance(seq_row_off, PageTable)
+    fn = "csa2_index_reindex_paged" if paged else "csa2_index_reindex"
+    qc, qs, wv = _queries(fn, B, q_codes, q_scales, w)
+    sl, pp = _arg(fn, "seq_len", seq_len, "i32", B), _arg(fn, "pool", pool, "i32", B * P)
+    to = _arg(fn, "topk_out", topk_out, "i32", B * k)
+    if paged:
         pt = seq_row_off
-        rc = lib().csa2_index_reindex_paged(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(pt.pages),
-                                            pt.page_rows, pt.max_pages, _ptr(seq_len), _ptr(pool), B, P, k,
-                                            _ptr(topk_out), wp, wn, _stream(stream))
-        _check(rc, "csa2_index_reindex_paged")
-        return
-    rc = lib().csa2_index_reindex(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len),
-                                  _ptr(pool), B, P, k, _ptr(topk_out), wp, wn, _stream(stream))
-    _check(rc, "csa2_index_reindex")
+        rc = lib().csa2_index_reindex_paged(idx_k, qc, qs, wv, _pages(fn, pt, B), pt.page_rows, pt.max_pages, sl, pp,
+                                            B, P, k, to, wp, wn, _stream(stream))
+    else:
+        rc = lib().csa2_index_reindex(idx_k, qc, qs, wv, _row_off(fn, seq_row_off, B), sl, pp, B, P, k, to, wp, wn,
+                                      _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_sparse_attn_decode_workspace_bytes(B, k):
     return lib().csa2_sparse_attn_decode_workspace_bytes(B, k)
 
 
+def _decode_args(fn, q, seq_len, topk, win, win_scale, win_len, out, lse):
+    B, k = topk.shape
+    return (B, k, _arg(fn, "q", q, "bf16", B * Q_HEADS * MAIN_DIM), _arg(fn, "seq_len", seq_len, "i32", B),
+            _arg(fn, "topk", topk, "i32", B * k), *_window(fn, B, win, win_scale, win_len), *_attn_out(fn, B, out, lse))
+
+
 def csa2_sparse_attn_decode(q, main_kv, seq_row_off, seq_len, topk, win, win_scale, win_len, sm_scale, out, ws,
                             lse=None, stream=None):
-    B, k = topk.shape
     wp, wn = _ws(ws)
-    if isinstance(seq_row_off, PageTable):
+    paged = isinstance(seq_row_off, PageTable)
+    fn = "csa2_sparse_attn_decode_paged" if paged else "csa2_sparse_attn_decode"
+    B, k, qp, sl, tp, wi, wsc, wl, op, lp = _decode_args(fn, q, seq_len, topk, win, win_scale, win_len, out, lse)
+    if paged:
         pt = seq_row_off
-        rc = lib().csa2_sparse_attn_decode_paged(_ptr(q), main_kv, _ptr(pt.pages), pt.page_rows, pt.max_pages,
-                                                 _ptr(seq_len), _ptr(topk), k, _ptr(win), _ptr(win_scale),
-                                                 _ptr(win_len), float(sm_scale), _ptr(out), _ptr(lse), B, wp, wn,
-                                                 _stream(stream))
-        _check(rc, "csa2_sparse_attn_decode_paged")
-        return
-    rc = lib().csa2_sparse_attn_decode(_ptr(q), main_kv, _ptr(seq_row_off), _ptr(seq_len), _ptr(topk), k, _ptr(win),
-                                       _ptr(win_scale), _ptr(win_len), float(sm_scale), _ptr(out), _ptr(lse), B, wp,
-                                       wn, _stream(stream))
-    _check(rc, "csa2_sparse_attn_decode")
+        rc = lib().csa2_sparse_attn_decode_paged(qp, main_kv, _pages(fn, pt, B), pt.page_rows, pt.max_pages, sl, tp,
+                                                 k, wi, wsc, wl, float(sm_scale), op, lp, B, wp, wn, _stream(stream))
+    else:
+        rc = lib().csa2_sparse_attn_decode(qp, main_kv, _row_off(fn, seq_row_off, B), sl, tp, k, wi, wsc, wl,
+                                           float(sm_scale), op, lp, B, wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_compress_append_workspace_bytes(B):
     return lib().csa2_compress_append_workspace_bytes(B)
 
 
+def _append_args(fn, raw, logits, w_idx, idx_raw, tok_off, seq_len_in, seq_len_out):
+    """Pointers of the token inputs and lengths shared by the append calls."""
+    B = seq_len_in.shape[0]
+    n_tok = raw.shape[0] if raw is not None else 0
+    return (B, n_tok, _arg(fn, "raw", raw, "bf16", n_tok * MAIN_DIM), _arg(fn, "logits", logits, "f32", n_tok),
+            _arg(fn, "w_idx", w_idx, "f32", MAIN_DIM * IDX_DIM), _arg(fn, "idx_raw", idx_raw, "bf16", n_tok * IDX_DIM),
+            _arg(fn, "tok_off", tok_off, "i64", B + 1), _arg(fn, "seq_len_in", seq_len_in, "i32", B),
+            _arg(fn, "seq_len_out", seq_len_out, "i32", B))
+
+
 def csa2_compress_append(main_kv, idx_k, raw, logits, tok_off, seq_row_off, seq_len_in, seq_len_out, ratio, max_new,
                          ws, w_idx=None, idx_raw=None, stream=None):
-    B = seq_len_in.shape[0]
+    fn = "csa2_compress_append"
     wp, wn = _ws(ws)
-    rc = lib().csa2_compress_append(main_kv, idx_k, _ptr(raw), _ptr(logits), _ptr(w_idx), _ptr(idx_raw),
-                                    _ptr(tok_off), _ptr(seq_row_off), _ptr(seq_len_in), _ptr(seq_len_out), B, ratio,
-                                    raw.shape[0], int(max_new), wp, wn, _stream(stream))
-    _check(rc, "csa2_compress_append")
+    B, n_tok, rp, lg, wi, ir, to, li, lo = _append_args(fn, raw, logits, w_idx, idx_raw, tok_off, seq_len_in,
+                                                        seq_len_out)
+    rc = lib().csa2_compress_append(main_kv, idx_k, rp, lg, wi, ir, to, _row_off(fn, seq_row_off, B), li, lo, B,
+                                    ratio, n_tok, int(max_new), wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_compress_stream_workspace_bytes(B):
@@ -258,23 +337,22 @@ def csa2_compress_stream_workspace_bytes(B):
 def csa2_compress_stream(main_kv, idx_k, raw, logits, tok_off, seq_row_off, seq_len_in, seq_len_out, pend_n, pend_raw,
                          pend_logit, max_new, ws, w_idx=None, idx_raw=None, pend_idx=None, stream=None):
     """seq_len_out may be seq_len_in (in place) or None; raw may be None when no token is appended."""
-    B = seq_len_in.shape[0]
     wp, wn = _ws(ws)
-    n_tok = raw.shape[0] if raw is not None else 0
-    if isinstance(seq_row_off, PageTable):
+    paged = isinstance(seq_row_off, PageTable)
+    fn = "csa2_compress_stream_paged" if paged else "csa2_compress_stream"
+    B, n_tok, rp, lg, wi, ir, to, li, lo = _append_args(fn, raw, logits, w_idx, idx_raw, tok_off, seq_len_in,
+                                                        seq_len_out)
+    pend = (_arg(fn, "pend_n", pend_n, "i32", B), _arg(fn, "pend_raw", pend_raw, "bf16", B * MAIN_DIM),
+            _arg(fn, "pend_logit", pend_logit, "f32", B), _arg(fn, "pend_idx", pend_idx, "bf16", B * IDX_DIM))
+    if paged:
         pt = seq_row_off
-        rc = lib().csa2_compress_stream_paged(main_kv, idx_k, _ptr(raw), _ptr(logits), _ptr(w_idx), _ptr(idx_raw),
-                                              _ptr(tok_off), _ptr(pt.pages), pt.page_rows, pt.max_pages,
-                                              _ptr(seq_len_in), _ptr(seq_len_out), _ptr(pend_n), _ptr(pend_raw),
-                                              _ptr(pend_logit), _ptr(pend_idx), B, n_tok, int(max_new), wp, wn,
+        rc = lib().csa2_compress_stream_paged(main_kv, idx_k, rp, lg, wi, ir, to, _pages(fn, pt, B), pt.page_rows,
+                                              pt.max_pages, li, lo, *pend, B, n_tok, int(max_new), wp, wn,
                                               _stream(stream))
-        _check(rc, "csa2_compress_stream_paged")
-        return
-    rc = lib().csa2_compress_stream(main_kv, idx_k, _ptr(raw), _ptr(logits), _ptr(w_idx), _ptr(idx_raw),
-                                    _ptr(tok_off), _ptr(seq_row_off), _ptr(seq_len_in), _ptr(seq_len_out),
-                                    _ptr(pend_n), _ptr(pend_raw), _ptr(pend_logit), _ptr(pend_idx), B, n_tok,
-                                    int(max_new), wp, wn, _stream(stream))
-    _check(rc, "csa2_compress_stream")
+    else:
+        rc = lib().csa2_compress_stream(main_kv, idx_k, rp, lg, wi, ir, to, _row_off(fn, seq_row_off, B), li, lo,
+                                        *pend, B, n_tok, int(max_new), wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_index_multi_workspace_bytes(B, Q, max_vis, pool_blocks, k):
@@ -283,12 +361,15 @@ def csa2_index_multi_workspace_bytes(B, Q, max_vis, pool_blocks, k):
 
 def csa2_index_multi(idx_k, q_codes, q_scales, w, seq_row_off, q_off, q_vis, max_vis, pool_blocks, k, pool_out,
                      topk_out, ws, q_row_off_out=None, stream=None):
+    fn = "csa2_index_multi"
     B, Q = seq_row_off.shape[0], q_vis.shape[0]
     wp, wn = _ws(ws)
-    rc = lib().csa2_index_multi(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(q_off),
-                                _ptr(q_vis), B, Q, int(max_vis), pool_blocks, k, _ptr(pool_out), _ptr(topk_out),
-                                _ptr(q_row_off_out), wp, wn, _stream(stream))
-    _check(rc, "csa2_index_multi")
+    rc = lib().csa2_index_multi(idx_k, *_queries(fn, Q, q_codes, q_scales, w), _row_off(fn, seq_row_off, B),
+                                _arg(fn, "q_off", q_off, "i32", B + 1), _arg(fn, "q_vis", q_vis, "i32", Q), B, Q,
+                                int(max_vis), pool_blocks, k, _arg(fn, "pool_out", pool_out, "i32", Q * pool_blocks),
+                                _arg(fn, "topk_out", topk_out, "i32", Q * k),
+                                _arg(fn, "q_row_off_out", q_row_off_out, "i64", Q), wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_score_positions_workspace_bytes(B):
@@ -297,11 +378,13 @@ def csa2_score_positions_workspace_bytes(B):
 
 def csa2_score_positions(idx_k, q_codes, q_scales, w, seq_row_off, seq_len, ids, block, keys_out, ws, stream=None):
     """keys_out [B, n] uint32 (int32 tensors carry the bits) <- rank keys of ids [B, n] (block 1 or 8)."""
+    fn = "csa2_score_positions"
     B, n = ids.shape
     wp, wn = _ws(ws)
-    rc = lib().csa2_score_positions(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(seq_row_off), _ptr(seq_len),
-                                    _ptr(ids), B, n, int(block), _ptr(keys_out), wp, wn, _stream(stream))
-    _check(rc, "csa2_score_positions")
+    rc = lib().csa2_score_positions(idx_k, *_queries(fn, B, q_codes, q_scales, w), _row_off(fn, seq_row_off, B),
+                                    _arg(fn, "seq_len", seq_len, "i32", B), _arg(fn, "ids", ids, "i32", B * n), B, n,
+                                    int(block), _arg(fn, "keys_out", keys_out, "i32", B * n), wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_topk_merge_workspace_bytes(G, B, n):
@@ -310,18 +393,24 @@ def csa2_topk_merge_workspace_bytes(G, B, n):
 
 def csa2_topk_merge(keys, ids, src_off, k, out, ws, lo=None, hi=None, out_local=None, stream=None):
     """keys / ids [G, B, n] from the shards -> out [B, k] (and out_local [B, k] for [lo, hi))."""
+    fn = "csa2_topk_merge"
     G, B, n = ids.shape
     wp, wn = _ws(ws)
-    rc = lib().csa2_topk_merge(_ptr(keys), _ptr(ids), _ptr(src_off), G, B, n, k, _ptr(lo), _ptr(hi), _ptr(out),
-                               _ptr(out_local), wp, wn, _stream(stream))
-    _check(rc, "csa2_topk_merge")
+    rc = lib().csa2_topk_merge(_arg(fn, "keys", keys, "i32", G * B * n), _arg(fn, "ids", ids, "i32", G * B * n),
+                               _arg(fn, "src_off", src_off, "i64", G * B), G, B, n, k, _arg(fn, "lo", lo, "i64", B),
+                               _arg(fn, "hi", hi, "i64", B), _arg(fn, "out", out, "i32", B * k),
+                               _arg(fn, "out_local", out_local, "i32", B * k), wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_attn_combine(out_parts, lse_parts, out, lse=None, stream=None):
     """out_parts [G, B, 16, 512], lse_parts [G, B, 16] -> out [B, 16, 512], lse [B, 16]."""
+    fn = "csa2_attn_combine"
     G, B = lse_parts.shape[0], lse_parts.shape[1]
-    rc = lib().csa2_attn_combine(_ptr(out_parts), _ptr(lse_parts), G, B, _ptr(out), _ptr(lse), _stream(stream))
-    _check(rc, "csa2_attn_combine")
+    rc = lib().csa2_attn_combine(_arg(fn, "out_parts", out_parts, "f32", G * B * Q_HEADS * MAIN_DIM),
+                                 _arg(fn, "lse_parts", lse_parts, "f32", G * B * Q_HEADS), G, B,
+                                 *_attn_out(fn, B, out, lse), _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_index_prefill_workspace_bytes(T, n_entries, pool_blocks, k):
@@ -330,11 +419,14 @@ def csa2_index_prefill_workspace_bytes(T, n_entries, pool_blocks, k):
 
 def csa2_index_prefill(idx_k, q_codes, q_scales, w, q_pos, row0, n_entries, ratio, pool_blocks, k, pool_out,
                        topk_out, ws, stream=None):
+    fn = "csa2_index_prefill"
     T = q_pos.shape[0]
     wp, wn = _ws(ws)
-    rc = lib().csa2_index_prefill(idx_k, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(q_pos), T, row0, n_entries,
-                                  ratio, pool_blocks, k, _ptr(pool_out), _ptr(topk_out), wp, wn, _stream(stream))
-    _check(rc, "csa2_index_prefill")
+    rc = lib().csa2_index_prefill(idx_k, *_queries(fn, T, q_codes, q_scales, w), _arg(fn, "q_pos", q_pos, "i32", T), T,
+                                  row0, n_entries, ratio, pool_blocks, k,
+                                  _arg(fn, "pool_out", pool_out, "i32", T * pool_blocks),
+                                  _arg(fn, "topk_out", topk_out, "i32", T * k), wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_sparse_attn_prefill_workspace_bytes(T, k):
@@ -343,12 +435,16 @@ def csa2_sparse_attn_prefill_workspace_bytes(T, k):
 
 def csa2_sparse_attn_prefill(q, q_pos, main_kv, row0, n_entries, ratio, topk, raw_win, win_scale, sm_scale, out, ws,
                              lse=None, stream=None):
+    fn = "csa2_sparse_attn_prefill"
     T, k = topk.shape
     wp, wn = _ws(ws)
-    rc = lib().csa2_sparse_attn_prefill(_ptr(q), _ptr(q_pos), T, main_kv, row0, n_entries, ratio, _ptr(topk), k,
-                                        _ptr(raw_win), raw_win.shape[0], float(win_scale), float(sm_scale), _ptr(out),
-                                        _ptr(lse), wp, wn, _stream(stream))
-    _check(rc, "csa2_sparse_attn_prefill")
+    rc = lib().csa2_sparse_attn_prefill(_arg(fn, "q", q, "bf16", T * Q_HEADS * MAIN_DIM),
+                                        _arg(fn, "q_pos", q_pos, "i32", T), T, main_kv, row0, n_entries, ratio,
+                                        _arg(fn, "topk", topk, "i32", T * k), k,
+                                        _arg(fn, "raw_win", raw_win, "u8", raw_win.shape[0] * MAIN_DIM),
+                                        raw_win.shape[0], float(win_scale), float(sm_scale), *_attn_out(fn, T, out, lse),
+                                        wp, wn, _stream(stream))
+    _check(rc, fn)
 
 
 def csa2_sparse_attn_decode_noalloc(q, main_kv, seq_row_off, seq_len, topk, win, win_scale, win_len, sm_scale, out,
@@ -357,8 +453,9 @@ def csa2_sparse_attn_decode_noalloc(q, main_kv, seq_row_off, seq_len, topk, win,
 
     For callers that may not allocate device memory while they run.  All calls
     on one device share the scratch, so calls that overlap on the GPU race."""
-    B, k = topk.shape
-    rc = lib().csa2_sparse_attn_decode_noalloc(_ptr(q), main_kv, _ptr(seq_row_off), _ptr(seq_len), _ptr(topk), k,
-                                               _ptr(win), _ptr(win_scale), _ptr(win_len), float(sm_scale), _ptr(out),
-                                               _ptr(lse), _ptr(flags_out), B, _stream(stream))
-    _check(rc, "csa2_sparse_attn_decode_noalloc")
+    fn = "csa2_sparse_attn_decode_noalloc"
+    B, k, qp, sl, tp, wi, wsc, wl, op, lp = _decode_args(fn, q, seq_len, topk, win, win_scale, win_len, out, lse)
+    rc = lib().csa2_sparse_attn_decode_noalloc(qp, main_kv, _row_off(fn, seq_row_off, B), sl, tp, k, wi, wsc, wl,
+                                               float(sm_scale), op, lp, _arg(fn, "flags_out", flags_out, "i32", 1), B,
+                                               _stream(stream))
+    _check(rc, fn)

@@ -206,6 +206,14 @@ def time_oracle(wl, samples, nthreads, jobs=None):
     return time.perf_counter() - t0, n * max(1, wl.queries_per_seq)
 
 
+def single_thread_oracle(wl, samples):
+    """The oracle on one host thread (one query of the first sample), and the
+    host's core count, for the cpu_baseline object."""
+    secs, nq = time_oracle(wl, samples[:1], 1, jobs=1)
+    return {"single_thread": {"value": nq / secs, "unit": "queries/s", "sample": f"{nq} query, one thread, "
+                              f"{secs:.2f} s"}, "host_cores": os.cpu_count()}
+
+
 # ----------------------------------------------------------------------------
 
 def decode_config(wl, l2_bytes, sequential, graph=True, full_rescan=False):
@@ -557,7 +565,8 @@ def run_ours(args):
         cpu = {"value": nq / secs, "unit": "queries/s", "cores": min(nthreads, len(samples)), "kind": "oracle",
                "sample": f"{nq} queries (each sequence {seqs} of the batch decoded 3 times; L={wl.max_len}, "
                          f"one full {wl.pattern} step per query, one host thread per query); {secs:.1f} s wall, "
-                         f"{secs * min(nthreads, len(samples)):.0f} core-seconds"}
+                         f"{secs * min(nthreads, len(samples)):.0f} core-seconds",
+               **single_thread_oracle(wl, samples)}
 
     if rank == 0:
         launches_per_step = 0
@@ -874,7 +883,7 @@ def run_reference(args):
            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": nthreads, "kind": "oracle",
                             "sample": f"{nseq} queries ({max(1, wl.queries_per_seq)} per step) over "
                                       f"{len(samples)} sequences of the workload, {nthreads} host threads at a "
-                                      f"time; {secs:.1f} s"},
+                                      f"time; {secs:.1f} s", **single_thread_oracle(wl, samples)},
            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     if not on_gpu:  # the GPU arm's cache and launch notes do not describe a host-only run
         res["config"]["l2"] = "host-only run (no GPU): contexts shortened to %d" % wl.max_len

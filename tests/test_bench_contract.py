@@ -30,6 +30,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["vs_baseline"] is None
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert cb["single_thread"]["value"] > 0 and cb["host_cores"] >= cb["cores"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"].endswith("_host") and "host-only" in d["config"]["l2"]
     assert abs(d["ms_per_step"] * d["value"] / 1e3 - 1) < 1e-9  # one query per timed step, same clock

@@ -249,6 +249,9 @@ csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
  * csa2_index_full_pool + csa2_index_full_topk -- csa2_index_full in two
  * calls, so that work which needs only the pool (the Reindex layers) can
  * start while the Full layer's own Top-k is still being selected.
+ * Source: as csa2_index_full (the pool and the Full layer's own Top-k are
+ * two outputs of the one indexer step there); the split into two calls is
+ * this library's scheduling choice.
  * csa2_index_full_pool runs the scan and writes pool_out; a later
  * csa2_index_full_topk on the same stream, with the same arguments, the
  * same workspace (untouched in between) and that pool, writes topk_out.
@@ -266,6 +269,9 @@ csa2_status csa2_index_full_topk(csa2_mxfp4_cache idx_k, const uint8_t* q_codes,
 /* ---------------------------------------------------------------------------
  * Paged caches: csa2_index_full_paged, csa2_index_reindex_paged,
  * csa2_sparse_attn_decode_paged, csa2_compress_stream_paged.
+ * Source: the operations are those of the calls without the suffix and cite
+ * the same sections; the pages have no counterpart of the paged layout,
+ * which is how serving engines keep KV caches.
  * The same operations, results and errors as the calls without the suffix,
  * for caches kept as fixed-size pages (a serving engine's block tables)
  * instead of one contiguous row range per sequence.  Position t of sequence
@@ -386,6 +392,9 @@ csa2_status csa2_index_multi(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, con
 
 /* ---------------------------------------------------------------------------
  * csa2_sparse_attn_prefill -- causal sparse attention of a prefill chunk.
+ * Source: as csa2_sparse_attn_decode ([V41] sections "三个方向一起压小缓存"
+ * and "后 20 层干脆共用一份 KV"), applied to every query of a causal chunk
+ * with the visibility rule of csa2_index_prefill.
  * Query i attends its selected entries (topk[i][j] >= 0, each < the visible
  * count of csa2_index_prefill) and the raw FP8 window rows
  * max(0, q_pos[i]-127) .. q_pos[i] of raw_win (one fp32 scale), in one

@@ -153,3 +153,17 @@ def test_widened_calls_validation():
                                   None) == -1
     assert L.csa2_index_full_topk(c, FAKE, FAKE, FAKE, None, FAKE, 2, 1000, 64, 64, FAKE, FAKE, None, FAKE, 1 << 30,
                                   None) == -1
+
+
+def test_every_entry_point_cites_its_source():
+    """Each operation declared in include/csa2.h sits under a comment block
+    that names the passage defining it (or says the pages have none)."""
+    src = open(HEADER).read()
+    decls = [(m.start(), m.group(1)) for m in re.finditer(r"^csa2_status (csa2_\w+)\(", src, re.M)]
+    assert len(decls) >= 15
+    helpers = {"csa2_device_status"}  # reads the status word back; no operation of the method
+    for pos, name in decls:
+        if name in helpers:
+            continue
+        block = src[src.rfind("/*", 0, pos):pos]
+        assert "Source:" in block or "no counterpart" in block, name

@@ -1,9 +1,10 @@
 """Thin Python binding of the CSA2 C ABI (``include/csa2.h``).
 
-Argument marshalling only: every function below forwards torch CUDA tensors
-as raw device pointers to the function of the same name in ``libcsa2.so`` and
-raises on a non-zero status.  All computation happens in the library's CUDA
-kernels; there is no fallback of any kind.  Workspaces come from
+Argument marshalling only: every function below checks each tensor's element
+type and size against the C declaration (the library sees only pointers),
+forwards the torch CUDA tensors as raw device pointers to the function of the
+same name in ``libcsa2.so`` and raises on a non-zero status.  All computation
+happens in the library's CUDA kernels; there is no fallback of any kind.  Workspaces come from
 ``workspace(nbytes)`` (zero-filled, 256-byte aligned torch allocations).
 """
 from __future__ import annotations

@@ -34,6 +34,7 @@ MUTANTS = [
     ("e8m0 bias", "std::ldexp(1.0, byte - 127)", "std::ldexp(1.0, byte - 128)"),
     ("e4m3 subnormal exponent", "std::ldexp(m / 8.0, -6)", "std::ldexp(m / 8.0, -7)"),
     ("e4m3 bias", "std::ldexp(1.0 + m / 8.0, e - 7)", "std::ldexp(1.0 + m / 8.0, e - 8)"),
+    ("e4m3 has no NaN", '  if (e == 15 && m == 7) return std::nan("");\n', ""),
     ("nibble order", "return (e & 1) ? (b >> 4) : (b & 15);", "return (e & 1) ? (b & 15) : (b >> 4);"),
     ("ties round down", "return (i % 2 == 0) ? i : i + 1;", "return i;"),
     ("ties round up", "return (i % 2 == 0) ? i : i + 1;", "return i + 1;"),
@@ -59,6 +60,11 @@ MUTANTS = [
     ("top-k left unsorted", "std::sort(sel.begin(), sel.end());", ""),
     ("block key is the last position", "bkey[b] = std::max(bkey[b], rank_key(s[t]));", "bkey[b] = rank_key(s[t]);"),
     ("block drops its last position", "std::min(L, (b + 1) * kBlk)", "std::min(L, b * kBlk + kBlk - 1)"),
+    ("pool one block short", "topk_select(bkey, bid, P, pool_out)", "topk_select(bkey, bid, P - 1, pool_out)"),
+    ("reindex drops each block's last position", "for (int j = 0; j < kBlk; ++j) {",
+     "for (int j = 0; j < kBlk - 1; ++j) {"),
+    ("rank key keeps the sign of zero", "uint32_t rank_key(float s) {\n  if (s == 0.0f) s = 0.0f;",
+     "uint32_t rank_key(float s) {"),
     ("reindex block is not scaled by 8", "int64_t t = int64_t(blk) * kBlk + j;", "int64_t t = int64_t(blk) + j;"),
     # attention
     ("attention drops sm_scale", "lg[j] = sm_scale * acc;", "lg[j] = acc;"),
@@ -66,6 +72,7 @@ MUTANTS = [
     ("attention not normalised", "for (int d = 0; d < kD; ++d) o[d] /= l;", ""),
     ("window scale dropped", "int64_t(kD), double(win_scale[b]))", "int64_t(kD), 1.0)"),
     ("window skips its first row", "for (int r = 0; r < win_len[b]; ++r)", "for (int r = 1; r < win_len[b]; ++r)"),
+    ("window ignores its length", "for (int r = 0; r < win_len[b]; ++r)", "for (int r = 0; r < 128; ++r)"),
     ("prefill window one row wider", "std::max<int64_t>(0, p - 127)", "std::max<int64_t>(0, p - 128)"),
     # compression
     ("pair weights swapped", "w0 = a / s;", "w0 = b / s;"),

@@ -233,3 +233,16 @@ def test_paged_step_reads_through_the_page_table(fake):
         pages_arg = a[2] if name == "csa2_sparse_attn_decode_paged" else a[4]
         assert pages_arg == pt.pages.data_ptr()
         assert 512 in a and pt.max_pages in a
+
+
+def test_every_wrapper_checks_its_tensors():
+    """Outside the checked helper, raw pointers are taken only for the cache
+    planes (checked in cache()), workspaces and the status read-back."""
+    import ast
+    import inspect
+
+    tree = ast.parse(inspect.getsource(C))
+    allowed = {"_arg", "cache", "_ws", "device_status", "_ptr"}
+    for fn in [n for n in tree.body if isinstance(n, ast.FunctionDef)]:
+        uses = [c for c in ast.walk(fn) if isinstance(c, ast.Call) and getattr(c.func, "id", None) == "_ptr"]
+        assert not uses or fn.name in allowed, fn.name

@@ -154,8 +154,11 @@ double own_exp(double x) {
 //   s_t = sum_h w_h * (q_h . k_t)   (no ReLU), one 128-d key per position
 // shared by the 4 indexer heads.  Exactness: per head h and 32-block b the
 // doubled-E2M1 integer dot D (|D| <= 4608) times 2^(eq+ek-2) is exact; the
-// four block terms are summed in fp64 in order b = 0..3 (exact whenever the
-// exponent spread is <= 38) and rounded once to fp32 (d_h).  The head
+// four block terms are summed in fp64 in order b = 0..3 and rounded once to
+// fp32 (d_h).  That sum is the exact block sum whenever the block exponents
+// of a head lie within 38 of each other (four 13-bit integers fit fp64's
+// 53-bit significand); beyond that the ordered fp64 sum itself is the
+// definition (both sides add in this order).  The head
 // combination is s = w0*d0, then fmaf(w_h, d_h, s) for h = 1..3, in fp32.
 // -0 becomes +0.
 // ---------------------------------------------------------------------------
@@ -183,7 +186,13 @@ float index_score(const uint8_t* kc, const uint8_t* ks, const uint8_t* qc, const
 }
 
 // Order-preserving map of a score to uint32 (larger score -> larger key).
+// The pages rank by score alone; a NaN score (a head sum of +inf and -inf,
+// or 0 * inf) has no place in that order.  Reading: every NaN ranks below
+// every number, -inf included, and NaNs tie among themselves (so the lower
+// position wins): all NaNs map to key 1 (-inf maps to 0x007FFFFF; 0 stays
+// free to mean "absent" elsewhere).
 uint32_t rank_key(float s) {
+  if (std::isnan(s)) return 1u;
   if (s == 0.0f) s = 0.0f;
   uint32_t u;
   std::memcpy(&u, &s, 4);

@@ -196,3 +196,95 @@ def test_index_multi_one_query_per_sequence_is_index_full(orc):
     pool_f, top_f, _ = orc.index_full(kc, ks, qc, qsc, w, off, lens, 64, 32)
     pool_m, top_m = orc.index_multi(kc, ks, qc, qsc, w, off, np.arange(B + 1, dtype=np.int32), lens, 64, 32)
     assert np.array_equal(pool_f, pool_m) and np.array_equal(top_f, top_m)
+
+
+def _overflow_case(L=1000):
+    """Rows whose exact head dots overflow fp32: query head 0 is +6 on blocks
+    0-1 and head 1 is -6 on blocks 2-3 (zeros elsewhere), at scale byte 200
+    (2^73); planted key rows of +6 at scale byte 250 (2^123) give block dots
+    of +-(32*12*12)*2^(73+123-2), far above fp32's range; heads 2, 3 (random
+    codes) sit at scale bytes 10 and 12, finite against every row.  Rows 100..119 (+6 on blocks 0-1): d0 = +inf, d1 = 0,
+    score +inf.  Rows 120..859 (+6 everywhere): d0 = +inf, d1 = -inf, score
+    NaN.  Rows 860..899 (+6 on blocks 2-3): d0 = 0, d1 = -inf, score -inf.
+    Other rows are random at normal scales (finite scores)."""
+    rng = np.random.default_rng(91)
+    kc, ks = _rand_rows(rng, L, 128, 124, 128)
+    qc = rng.integers(0, 256, (4, 64), dtype=np.uint8)
+    qs = rng.integers(124, 129, (4, 4), dtype=np.uint8)
+    qc[0, :32], qc[0, 32:] = 0x77, 0x00      # head 0: +6 on blocks 0, 1
+    qc[1, :32], qc[1, 32:] = 0x00, 0xFF      # head 1: -6 on blocks 2, 3
+    qs[0], qs[1] = 200, 200
+    qs[2], qs[3] = 10, 12                    # heads 2, 3 stay finite against the planted rows
+    w = np.array([1.0, 0.75, 1.25, 0.5], np.float32)
+    kinds = np.zeros(L, np.int8)
+    for lo, hi, code, kind in ((100, 120, (0x77, 0x00), 1), (120, 860, (0x77, 0x77), 2), (860, 900, (0x00, 0x77), 3)):
+        kc[lo:hi, :32], kc[lo:hi, 32:] = code
+        ks[lo:hi] = 250
+        kinds[lo:hi] = kind
+    return kc, ks, qc, qs, w, kinds
+
+
+def test_rank_key_nan_ranks_below_every_number(orc):
+    """Every NaN (any sign or payload) ranks below every number, -inf
+    included, and NaNs tie among themselves; key 0 stays "absent"."""
+    nans = np.array([0x7FC00000, 0xFFC00000, 0x7F800001, 0xFFFFFFFF, 0x7FFFFFFF], np.uint32).view(np.float32)
+    assert all(orc.rank_key(v) == 1 for v in nans)
+    assert orc.rank_key(-np.inf) == 0x007FFFFF
+    assert orc.rank_key(np.inf) == 0xFF800000
+    # scores [NaN, -inf, 1, NaN, -3], best 4 by (score desc, position asc):
+    # 1 (pos 2), -3 (pos 4), -inf (pos 1), the first NaN (pos 0)
+    s = np.array([np.nan, -np.inf, 1.0, np.nan, -3.0], np.float32)
+    key = [orc.rank_key(v) for v in s]
+    assert orc.topk(key, np.arange(5), 4).tolist() == [0, 1, 2, 4]
+
+
+def test_overflowing_scores_are_inf_and_nan(orc):
+    kc, ks, qc, qs, w, kinds = _overflow_case()
+    s = orc.index_scores(kc, ks, np.arange(len(kinds)), qc, qs, w)
+    assert np.all(s[kinds == 1] == np.inf)
+    assert np.all(np.isnan(s[kinds == 2]))
+    assert np.all(s[kinds == 3] == -np.inf)
+    assert np.all(np.isfinite(s[kinds == 0]))
+    # the Top-512: the 20 +inf rows, the 200 finite rows, the 40 -inf rows and
+    # then the first 252 NaN rows by position (brute force over the sort rule)
+    _, top, _ = orc.index_full(kc, ks, qc, qs, w, np.array([0]), np.array([len(kinds)], np.int32), 64, 512)
+    want = sorted(list(range(100, 120)) + list(range(100)) + list(range(900, 1000)) + list(range(860, 900))
+                  + list(range(120, 120 + 252)))
+    assert top[0].tolist() == want
+
+
+def test_score_with_wide_exponent_spread_is_the_ordered_fp64_sum(orc):
+    """Beyond a block-exponent spread of 38 the four block terms of a head no
+    longer add exactly in fp64 (13-bit integers 2^39 apart and more).  The
+    definition is then the fp64 sum in block order 0..3, rounded once to fp32;
+    this pins the oracle to that order on rows where it differs from the exact
+    sum."""
+    from fractions import Fraction
+
+    from tests._exact import frac32, rn32, row_values
+
+    rng = np.random.default_rng(93)
+    differs = 0
+    for trial in range(40):
+        kc, ks = _rand_rows(rng, 1, 128)
+        qc, qs, w = _rand_query(rng, 125, 129)
+        # block 0 huge, blocks 1..3 tiny: spreads of 60..90 exponents
+        ks[0] = [127 + 40, 127 - rng.integers(20, 50), 127 - rng.integers(20, 50), 127 - 20]
+        got = orc.index_scores(kc, ks, np.arange(1), qc, qs, w)[0]
+        k = row_values(kc[0], ks[0])
+        d = []
+        for h in range(4):
+            q = row_values(qc[h], qs[h])
+            acc = 0.0
+            exact = Fraction(0)
+            for b in range(4):
+                term = sum(q[i] * k[i] for i in range(32 * b, 32 * b + 32))   # exact block dot
+                acc = acc + float(term)           # fp64 add in block order (each term exact in fp64)
+                exact += term
+            d.append(np.float32(acc))
+            differs += int(Fraction(acc) != exact)
+        s = rn32(frac32(w[0]) * frac32(d[0]))
+        for h in range(1, 4):
+            s = rn32(frac32(w[h]) * frac32(d[h]) + frac32(s))
+        assert got.tobytes() == np.float32(0.0 if s == 0 else s).tobytes(), trial
+    assert differs > 0     # the ordered sum really differs from the exact one somewhere

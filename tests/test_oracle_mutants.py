@@ -63,8 +63,9 @@ MUTANTS = [
     ("pool one block short", "topk_select(bkey, bid, P, pool_out)", "topk_select(bkey, bid, P - 1, pool_out)"),
     ("reindex drops each block's last position", "for (int j = 0; j < kBlk; ++j) {",
      "for (int j = 0; j < kBlk - 1; ++j) {"),
-    ("rank key keeps the sign of zero", "uint32_t rank_key(float s) {\n  if (s == 0.0f) s = 0.0f;",
-     "uint32_t rank_key(float s) {"),
+    ("rank key keeps the sign of zero", "  if (s == 0.0f) s = 0.0f;\n  uint32_t u;", "  uint32_t u;"),
+    ("NaN ranked by its bits", "  if (std::isnan(s)) return 1u;\n", ""),
+    ("NaN ranked first", "  if (std::isnan(s)) return 1u;", "  if (std::isnan(s)) return 0xFFFFFFFFu;"),
     ("reindex block is not scaled by 8", "int64_t t = int64_t(blk) * kBlk + j;", "int64_t t = int64_t(blk) + j;"),
     # attention
     ("attention drops sm_scale", "lg[j] = sm_scale * acc;", "lg[j] = acc;"),

@@ -206,12 +206,20 @@ def time_oracle(wl, samples, nthreads, jobs=None):
     return time.perf_counter() - t0, n * max(1, wl.queries_per_seq)
 
 
+def host_cores():
+    """Host cores this process may run on (the oracle baselines use them all)."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
 def single_thread_oracle(wl, samples):
     """The oracle on one host thread (one query of the first sample), and the
     host's core count, for the cpu_baseline object."""
     secs, nq = time_oracle(wl, samples[:1], 1, jobs=1)
     return {"single_thread": {"value": nq / secs, "unit": "queries/s", "sample": f"{nq} query, one thread, "
-                              f"{secs:.2f} s"}, "host_cores": os.cpu_count()}
+                              f"{secs:.2f} s"}, "host_cores": host_cores()}
 
 
 # ----------------------------------------------------------------------------
@@ -557,7 +565,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        nthreads = min(os.cpu_count() or 1, 8)
+        nthreads = host_cores()
         seqs = list(range(0, wl.B, max(1, wl.B // nthreads)))[:nthreads]
         samples = oracle_sample_inputs(wl, layers, caches_dev, seqs)
         jobs = 3 * len(samples)
@@ -783,7 +791,7 @@ def run_prefill(args):
     achieved = flops / (per_call["csa2_index_prefill"] * 1e-3) / 1e12
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = prefill_cpu_baseline(pw, seed, min(os.cpu_count() or 1, 8))
+        cpu = prefill_cpu_baseline(pw, seed, host_cores())
     if rank == 0:
         print(json.dumps({
             "metric": "prefill queries/sec (ratio-2 compression of 262144 tokens, 4096-query causal chunk)",
@@ -821,7 +829,7 @@ def run_reference(args):
 
     import synth.workloads as W
 
-    nthreads = min(os.cpu_count() or 1, 8)
+    nthreads = host_cores()
     if args.workload.startswith("prefill"):
         # the oracle's prefill step, estimated from a bounded sample per timed step
         pw = W.prefill_workload()
@@ -844,7 +852,7 @@ def run_reference(args):
     if on_gpu:
         # inputs from the device generator (same bytes as the NumPy generator)
         wl2, layers, caches_dev, _, _, _, _ = build_workload(wl, 0, torch.device("cuda", 0))
-        seqs = list(range(nthreads))
+        seqs = list(range(min(nthreads, wl.B)))
         samples = oracle_sample_inputs(wl2, layers, caches_dev, seqs)
         del caches_dev
     else:

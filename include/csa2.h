@@ -41,6 +41,14 @@
  *     may run concurrently.  Calls keep internal counters and histograms in
  *     the workspace and leave them zero when they finish; after a call that
  *     set a device flag, zero-fill the workspace again before reusing it.
+ *     Words 2 and 3 (int32) of the status block are test controls, zero (off)
+ *     in a zero-filled workspace: word 2, if nonzero, replaces the pipeline
+ *     wait limit of the tensor-core scans (microseconds; built in: 2 s);
+ *     word 3, if nonzero, makes each scan CTA's producer withhold the copies
+ *     of its first work item so that a wait runs out (CSA2_DEV_TIMEOUT).
+ *     They exist to test the timeout path; leave them zero otherwise.
+ *     Word 4 is a diagnostic count of selections whose threshold bucket held
+ *     more than 12288 keys (they then fall back to global radix passes).
  *   - Return value: CSA2_OK, or a negative error; on an error nothing was
  *     launched, except CSA2_ERR_CUDA (a launch failed; see csa2_last_error()).
  *     Arguments are validated on the host before the first launch.
@@ -416,16 +424,23 @@ csa2_status csa2_sparse_attn_prefill(const uint16_t* q, const int32_t* q_pos, in
  * allocations, or a serving loop held to a fixed memory budget).  The pages
  * have no counterpart of this call; it is a deployment convenience.
  * Same arguments, results and accuracy as csa2_sparse_attn_decode, except:
- *   - no workspace: the scratch is a fixed 16,843,520-byte array of device
- *     memory inside this library, which every GPU that loads the library keeps
- *     until the process exits; the call allocates nothing;
+ *   - no workspace: the scratch is a fixed 16,843,264-byte array of device
+ *     memory inside this library, which every GPU where the library's device
+ *     code is loaded keeps until the process exits;
+ *   - when that memory is committed: under CUDA's lazy module loading (the
+ *     default) the array and the attention kernel are loaded on a device the
+ *     first time a call touches them there, so the first call per device may
+ *     allocate (once).  A call with B = 0 does exactly that set-up on the
+ *     current device and launches nothing (the other pointers are not read):
+ *     make it outside the region where allocation is forbidden and before any
+ *     stream capture.  Every later call on that device allocates nothing;
  *   - limits: B <= 64 and k <= 512; larger problems return
  *     CSA2_ERR_UNSUPPORTED with a message, and nothing is launched;
  *   - flags_out: device uint32 that receives this call's CSA2_DEV_* flags, or
  *     NULL;
- *   - the first call on a device looks up the scratch's device address (once
- *     per device, with that device current); make that first call before any
- *     stream capture;
+ *   - the scratch's device address is looked up once per device and kept for
+ *     the life of the process: do not use the library across a
+ *     cudaDeviceReset;
  *   - all calls on a device share the one scratch array: calls that may run
  *     at the same time on the GPU (different streams, or different host
  *     threads) race and corrupt each other's results.  Serialise them.

@@ -448,6 +448,16 @@ def csa2_sparse_attn_prefill(q, q_pos, main_kv, row0, n_entries, ratio, topk, ra
     _check(rc, fn)
 
 
+def noalloc_setup(stream=None):
+    """The B = 0 call of csa2_sparse_attn_decode_noalloc: loads the library's
+    scratch array and the attention kernel on the current device (the one
+    time that call may allocate device memory) and launches nothing."""
+    fn = "csa2_sparse_attn_decode_noalloc"
+    rc = lib().csa2_sparse_attn_decode_noalloc(None, MXFP4Cache(None, None, 0), None, None, None, 1, None, None, None,
+                                               0.0, None, None, None, 0, _stream(stream))
+    _check(rc, fn)
+
+
 def csa2_sparse_attn_decode_noalloc(q, main_kv, seq_row_off, seq_len, topk, win, win_scale, win_len, sm_scale, out,
                                     lse=None, flags_out=None, stream=None):
     """csa2_sparse_attn_decode without a workspace (fixed library scratch; B <= 64, k <= 512).
@@ -456,6 +466,8 @@ def csa2_sparse_attn_decode_noalloc(q, main_kv, seq_row_off, seq_len, topk, win,
     on one device share the scratch, so calls that overlap on the GPU race."""
     fn = "csa2_sparse_attn_decode_noalloc"
     B, k, qp, sl, tp, wi, wsc, wl, op, lp = _decode_args(fn, q, seq_len, topk, win, win_scale, win_len, out, lse)
+    if B == 0:
+        return noalloc_setup(stream)
     rc = lib().csa2_sparse_attn_decode_noalloc(qp, main_kv, _row_off(fn, seq_row_off, B), sl, tp, k, wi, wsc, wl,
                                                float(sm_scale), op, lp, _arg(fn, "flags_out", flags_out, "i32", 1), B,
                                                _stream(stream))

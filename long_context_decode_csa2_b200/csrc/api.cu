@@ -149,7 +149,8 @@ csa2_status index_full_impl(const char* fn, csa2_mxfp4_cache idx_k, const uint8_
     const csa2_status rc = launch_scan_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, ws.tile_start, B, q_codes,
                                           q_scales, w, ws.bkeys, nb, scores, max_len, ws.hist, ws.status, st);
     if (rc != CSA2_OK) return rc;
-    launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, ws.hist, st);
+    launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, ws.hist, st,
+                  ws.status);
   }
   if (!(phases & 2)) return check_launch(fn);
   if (pool_blocks >= k) {
@@ -161,7 +162,7 @@ csa2_status index_full_impl(const char* fn, csa2_mxfp4_cache idx_k, const uint8_
     launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.seg_eff, B, pool_blocks, pool_out, k,
                   topk_out, ws.hist, st);
   } else {
-    launch_select(kSelScores, scores, max_len, ws.seg_eff, B, 0, nullptr, k, topk_out, nullptr, st);
+    launch_select(kSelScores, scores, max_len, ws.seg_eff, B, 0, nullptr, k, topk_out, nullptr, st, ws.status);
   }
   return check_launch(fn);
 }
@@ -602,6 +603,7 @@ struct MultiWs {
   int32_t* vis;
   int64_t* q_row_off;
   int4* groups;
+  int32_t* n_groups;
   uint32_t* bkeys;
   uint32_t* ckeys;
   size_t bytes;
@@ -613,6 +615,7 @@ MultiWs multi_ws(void* ws, int B, int Q, int64_t max_vis, int P) {
   w.vis = c.take<int32_t>(size_t(Q));
   w.q_row_off = c.take<int64_t>(size_t(Q));
   w.groups = c.take<int4>(size_t(multi_group_bound(B, Q)));
+  w.n_groups = c.take<int32_t>(1);
   w.bkeys = c.take<uint32_t>(size_t(Q) * size_t(block_key_stride(max_vis)));
   w.ckeys = c.take<uint32_t>(size_t(Q) * P * kBlk);
   w.bytes = c.used;
@@ -651,10 +654,10 @@ csa2_status csa2_index_multi(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, con
   int64_t* row_off = q_row_off_out ? q_row_off_out : ws.q_row_off;
   const int G = multi_group_bound(B, Q);
   const int64_t nb = block_key_stride(max_vis);
-  launch_multi_prep(seq_row_off, q_off, q_vis, B, Q, G, max_vis, idx_k.rows, ws.groups, row_off, ws.vis, ws.status,
-                    st);
-  const csa2_status rc0 = launch_multi_tc(idx_k.codes, idx_k.scales, idx_k.rows, seq_row_off, ws.groups, G, ws.vis,
-                                          Q, max_vis, q_codes, q_scales, w, ws.bkeys, nb, ws.status, st);
+  launch_multi_prep(seq_row_off, q_off, q_vis, B, Q, G, max_vis, idx_k.rows, ws.groups, row_off, ws.vis,
+                    ws.n_groups, ws.status, st);
+  const csa2_status rc0 = launch_multi_tc(idx_k.codes, idx_k.scales, idx_k.rows, seq_row_off, ws.groups, G,
+                                          ws.n_groups, ws.vis, Q, max_vis, q_codes, q_scales, w, ws.bkeys, nb, ws.status, st);
   if (rc0 != CSA2_OK) return rc0;
   launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, Q, 0, nullptr, pool_blocks, pool_out, nullptr, st);
   SegDesc sd{row_off, 0, ws.vis, max_vis, idx_k.rows};

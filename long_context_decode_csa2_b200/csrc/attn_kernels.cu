@@ -574,13 +574,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
   combine_if_last(a, sm, s, R, nslots);
 }
 
+void prepare_attention() {
+  // setting the attributes loads the kernel's module on the current device
+  cudaFuncSetAttribute(k_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sizeof(AttnSmem)));
+  cudaFuncSetAttribute(k_attn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+}
+
 void launch_attention(const AttnArgs& a, cudaStream_t st) {
   if (a.S == 0) return;
   const int R = attn_splits(a.S, a.k);
-  const size_t smem = sizeof(AttnSmem);
-  cudaFuncSetAttribute(k_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  cudaFuncSetAttribute(k_attn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  k_attn<<<dim3(R, a.S), kAttnThreads, smem, st>>>(a, R);
+  prepare_attention();
+  k_attn<<<dim3(R, a.S), kAttnThreads, sizeof(AttnSmem), st>>>(a, R);
 }
 
 }  // namespace csa2

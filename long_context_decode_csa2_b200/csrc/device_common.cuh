@@ -61,9 +61,29 @@ __device__ __forceinline__ int64_t seg_row(const SegDesc& sd, int s, int64_t t, 
   return (sd.row_off ? sd.row_off[s] : sd.row0) + t;
 }
 
+// Test controls of the tensor-core kernels (see kCtlWaitUs): the pipeline
+// wait limit in ns (the built-in `dflt` unless word 2 is set) and whether the
+// producer withholds its first work item (word 3).
+struct PipeCtl {
+  uint64_t wait_ns;
+  bool withhold;
+};
+__device__ __forceinline__ PipeCtl pipe_ctl(const uint32_t* status, uint64_t dflt) {
+  PipeCtl c{dflt, false};
+  if (status) {
+    const uint32_t us = __ldcg(status + kCtlWaitUs);
+    if (us) c.wait_ns = uint64_t(us) * 1000ull;
+    c.withhold = __ldcg(status + kCtlWithhold) != 0u;
+  }
+  return c;
+}
+
 // Order-preserving map of an fp32 score to a uint32 key; -0 ranks as +0.
-// Key 0 is reserved for "absent" (only a negative NaN would map there).
+// Every NaN (whatever its sign and payload) maps to key 1, below every
+// number including -inf (key 0x007FFFFF), so NaN positions rank last and
+// among themselves by position.  Key 0 is reserved for "absent".
 __device__ __forceinline__ uint32_t rank_key(float s) {
+  if (s != s) return 1u;
   if (s == 0.0f) s = 0.0f;
   uint32_t u = __float_as_uint(s);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);

@@ -324,7 +324,8 @@ template <int KIND, bool SMALL>
 __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restrict__ in, int64_t in_stride,
                                                         const int32_t* __restrict__ seg_eff, int P,
                                                         const int32_t* __restrict__ pool, int k,
-                                                        int32_t* __restrict__ out, uint32_t* __restrict__ ghist) {
+                                                        int32_t* __restrict__ out, uint32_t* __restrict__ ghist,
+                                                        uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) uint32_t dsm[];
   __shared__ SelShared sh;
   const int s = blockIdx.x;
@@ -466,6 +467,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   if (!all && cnt > uint32_t(kCandCap)) {
     // more than kCandCap keys share the threshold bucket: global radix passes
     // over the low 17 bits (9 + 8), then an ordered pass over the keys
+    if (status && tid == 0) atomicAdd(status + kDiagOverfull, 1u);
     uint32_t prefix = b1 << kLowBits, pmask = ~kLowMask, r = need;
     uint32_t* h2 = dsm;
     const int shifts[2] = {8, 0};
@@ -616,36 +618,36 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
 
 template <int KIND>
 void launch_select_kind(const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P, const int32_t* pool,
-                        int k, int32_t* out, uint32_t* hist, int64_t n_bound, cudaStream_t st) {
+                        int k, int32_t* out, uint32_t* hist, int64_t n_bound, cudaStream_t st, uint32_t* status) {
   if (n_bound <= kSelSmallMax) {
     constexpr int NB = (KIND == kSelPoolCand) ? kCandHistBins : kHist1Bins;
     const size_t smem = (hist ? NB + 1024 : 256) * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int((NB + 1024) * sizeof(uint32_t)));
-    k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist);
+    k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, status);
   } else {
     const size_t smem = kSelLargeWords * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    k_select<KIND, false><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist);
+    k_select<KIND, false><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, status);
   }
 }
 
 void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P,
-                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st) {
+                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st, uint32_t* status) {
   if (S == 0) return;
   // n per segment is at most the row stride of the input
   switch (kind) {
     case kSelBlockKeys:
-      launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
+      launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status);
       break;
     case kSelScores:
-      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
+      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status);
       break;
     case kSelPoolCand:
-      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
+      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status);
       break;
     case kSelExplicit:
-      launch_select_kind<kSelExplicit>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st);
+      launch_select_kind<kSelExplicit>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status);
       break;
   }
 }

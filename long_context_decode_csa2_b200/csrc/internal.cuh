@@ -21,6 +21,17 @@ constexpr int kIdxScaleBytes = kDi / 32;      // 4
 constexpr int kMainCodeBytes = kD / 2;        // 256
 constexpr int kMainScaleBytes = kD / 32;      // 16
 constexpr size_t kStatusBytes = 256;          // head of every workspace
+// Words of that head: 0 = the device status flags (CSA2_DEV_*); 2 and 3 are
+// test controls of the tensor-core kernels, zero (= off) in a zero-filled
+// workspace: word 2, if nonzero, replaces their pipeline wait limit (in
+// microseconds); word 3, if nonzero, makes each CTA's producer withhold the
+// copies of its first work item, so that a wait must run out (tests of the
+// timeout path use them).
+constexpr int kCtlWaitUs = 2;
+constexpr int kCtlWithhold = 3;
+// Word 4 is a diagnostic counter: selections that found more than 12288 keys
+// in their threshold bucket and fell back to global radix passes add one.
+constexpr int kDiagOverfull = 4;
 
 // ---------------------------------------------------------------------------
 // Host-side error plumbing (thread-local message, no other global state).
@@ -90,14 +101,16 @@ csa2_status launch_prefill_tc(const uint8_t* kcodes, const uint8_t* kscales, int
 
 // Multi-query scan (a batch of sequences with a few queries each): the group
 // table (at most multi_group_bound(B, Q) groups of <= 8 queries of one
-// sequence), each query's first cache row and checked visible count, then
-// the block keys [Q][nb_stride] of every query on the tensor cores.
+// sequence) with its real group count, each query's first cache row and
+// checked visible count, then the block keys [Q][nb_stride] of every query on
+// the tensor cores (work split over the real groups only).
 int multi_group_bound(int B, int Q);
 void launch_multi_prep(const int64_t* seq_row_off, const int32_t* q_off, const int32_t* q_vis, int B, int Q, int G,
                        int64_t max_vis, int64_t cache_rows, int4* groups, int64_t* q_row_off, int32_t* vis,
-                       uint32_t* status, cudaStream_t st);
+                       int32_t* n_groups, uint32_t* status, cudaStream_t st);
 csa2_status launch_multi_tc(const uint8_t* kcodes, const uint8_t* kscales, int64_t cache_rows,
-                            const int64_t* seq_row_off, const int4* groups, int G, const int32_t* vis, int Q,
+                            const int64_t* seq_row_off, const int4* groups, int G, const int32_t* n_groups,
+                            const int32_t* vis, int Q,
                             int64_t max_vis, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
                             uint32_t* bkeys, int64_t nb_stride, uint32_t* status, cudaStream_t st);
 
@@ -129,8 +142,10 @@ enum SelectKind : int {
 };
 // `hist` (or null): the keys' histogram rows, zeroed on return: [S][kSelHistBins]
 // for block keys, [S][kCandHistBins] for pool candidates.
+// `status` (or null): the workspace's status block (diagnostic counter).
 void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P,
-                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st);
+                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st,
+                   uint32_t* status = nullptr);
 
 // Attention partials + combine.
 struct AttnArgs {
@@ -161,6 +176,9 @@ struct AttnArgs {
 int attn_num_chunks(int k);
 size_t attn_partial_bytes(int S, int k);
 void launch_attention(const AttnArgs& a, cudaStream_t st);
+// Loads the attention kernel on the current device and sets its launch
+// attributes (launch_attention does this itself).
+void prepare_attention();
 
 // Compression + MXFP4 encode.
 struct CompressArgs {

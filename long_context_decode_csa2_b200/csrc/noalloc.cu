@@ -1,5 +1,5 @@
 // csa2_sparse_attn_decode_noalloc: the sparse-attention decode call with no
-// workspace argument and no device allocation anywhere.
+// workspace argument and no device allocation of its own.
 //
 // Who needs it: callers that are not allowed to allocate device memory when
 // they run.  Examples are plugins executed inside another inference runtime
@@ -9,6 +9,15 @@
 // that cudaMalloc / cudaFree can cause.  Such a caller passes only its inputs
 // and outputs; the scratch this call needs lives in a fixed array of the
 // library's own device memory, declared below.
+//
+// When that memory is committed: the array belongs to this file's device
+// module.  Under CUDA's lazy module loading (the default) a module is loaded,
+// and its device memory committed, the first time the process touches it on a
+// device, here the address lookup of the array.  The attention kernel's own
+// module loads at its first launch in the same way.  So the first call on a
+// device may allocate (once); a call with B = 0 does only that set-up and
+// launches nothing, so a caller can make it before entering the region where
+// it may not allocate.
 #include <mutex>
 #include <string>
 
@@ -21,23 +30,26 @@ namespace {
 constexpr int kNoAllocMaxSeqs = 64;
 constexpr int kNoAllocMaxTopk = 512;
 constexpr size_t kNoAllocStatusBytes = 256;                       // device status word
-constexpr size_t kNoAllocSeqBytes = 256;                          // reserved (layout unchanged)
 constexpr size_t kNoAllocCounterBytes = 256;                      // 64 arrival counters (self-resetting)
 constexpr size_t kNoAllocSlots = 8;                               // partials per sequence: up to 4 CTAs x
                                                                   // (selected rows, window)
 constexpr size_t kNoAllocPartialBytes =                           // split-KV partials
     size_t(kNoAllocMaxSeqs) * kNoAllocSlots * (kHq * kD + 2 * kHq) * sizeof(float);
 constexpr size_t kNoAllocScratchBytes =
-    kNoAllocStatusBytes + kNoAllocSeqBytes + kNoAllocCounterBytes + kNoAllocPartialBytes;
+    kNoAllocStatusBytes + kNoAllocCounterBytes + kNoAllocPartialBytes;
+static_assert(kNoAllocScratchBytes == 16843264, "the documented scratch size");
 
-// The scratch: 16,843,520 bytes of device memory that every GPU which loads
-// this library keeps until the process exits.  All calls on a device share it
-// and it keeps whatever the last call left in it.
+// The scratch: 16,843,264 bytes of device memory that every GPU on which this
+// library's device code is loaded keeps until the process exits.  All calls
+// on a device share it and it keeps whatever the last call left in it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Host code cannot use g_noalloc_scratch as a pointer (on the host the name
 // is only a stand-in for the device symbol), so its device address is looked
-// up once per device, with that device current, and cached here.
+// up once per device, with that device current, and cached here.  The cache
+// assumes the device's context lives as long as the process: after a
+// cudaDeviceReset the module may reload elsewhere, so the library must not be
+// used across a reset.
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
@@ -71,11 +83,20 @@ extern "C" csa2_status csa2_sparse_attn_decode_noalloc(const uint16_t* q, csa2_m
                                                        float* out, float* lse, uint32_t* flags_out, int B,
                                                        void* stream) {
   const char* fn = "csa2_sparse_attn_decode_noalloc";
-  if (B < 0 || k < 1) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad B or k");
+  if (B < 0) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": negative B");
+  if (B == 0) {
+    // set-up only: load this file's module (the scratch) and the attention
+    // kernel's module on the current device, launch nothing
+    void* base = nullptr;
+    const csa2_status rc = scratch_address(&base);
+    if (rc != CSA2_OK) return rc;
+    prepare_attention();
+    return check_launch(fn);
+  }
+  if (k < 1) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad k");
   if (B > kNoAllocMaxSeqs || k > kNoAllocMaxTopk)
     return fail(CSA2_ERR_UNSUPPORTED, std::string(fn) + ": at most 64 sequences and k <= 512 (fixed scratch of " +
                                           std::to_string(kNoAllocScratchBytes) + " bytes); use csa2_sparse_attn_decode");
-  if (B == 0) return CSA2_OK;
   if (!(main_kv.codes && main_kv.scales && aligned16(main_kv.codes) && aligned16(main_kv.scales) && main_kv.rows >= 0 &&
         main_kv.rows % 8 == 0))
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": bad main-KV cache");
@@ -92,11 +113,11 @@ extern "C" csa2_status csa2_sparse_attn_decode_noalloc(const uint16_t* q, csa2_m
   char* p = static_cast<char*>(base);
   AttnArgs a{};
   a.status = reinterpret_cast<uint32_t*>(p);
-  a.counters = reinterpret_cast<int32_t*>(p + kNoAllocStatusBytes + kNoAllocSeqBytes);
-  a.partial = reinterpret_cast<float*>(p + kNoAllocStatusBytes + kNoAllocSeqBytes + kNoAllocCounterBytes);
+  a.counters = reinterpret_cast<int32_t*>(p + kNoAllocStatusBytes);
+  a.partial = reinterpret_cast<float*>(p + kNoAllocStatusBytes + kNoAllocCounterBytes);
   // The status word must start at zero for this call.  The arrival counters
-  // are zero when the library loads and every call leaves them at zero; the
-  // visible counts and partials are fully written before they are read.
+  // are zero when the module loads and every call leaves them at zero; the
+  // partials are fully written before they are read.
   cudaError_t e = cudaMemsetAsync(a.status, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return fail(CSA2_ERR_CUDA, std::string(fn) + ": " + cudaGetErrorString(e));
   a.q = q;

@@ -106,7 +106,8 @@ struct PfParams {
   int T;
   int64_t row0;
   int64_t cache_rows;
-  int n_groups;
+  int n_groups;             // groups (with a group table: its capacity)
+  const int32_t* n_groups_dev;  // with a group table: the groups k_multi_prep wrote, or null
   int n_tiles;
   uint32_t* bkeys;          // [T][nb_stride]
   int64_t nb_stride;
@@ -182,7 +183,13 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   PfSmem& sm = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_items = p.n_groups * p.n_tiles;
+  // items are split over the groups that exist (the table's capacity is a
+  // host bound; empty entries past the real count would idle their CTAs)
+  const int n_groups = p.n_groups_dev ? min(p.n_groups, max(0, __ldg(p.n_groups_dev))) : p.n_groups;
+  const int n_items = n_groups * p.n_tiles;
+  // wait limit of the pipeline (2 s unless a test sets it); a test may also
+  // have the producer withhold its first item's copies
+  const PipeCtl ctl = pipe_ctl(p.status, 2000000000ull);
   const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
   const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
 
@@ -233,7 +240,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       }
       if (int64_t(tile) * kPT >= gmax) continue;
       const int t = issued, s = t % kSt, round = t / kSt;
-      const bool ok = round == 0 || sm100::mbar_wait(&sm.empty[s], (round - 1) & 1);
+      const bool ok = round == 0 || sm100::mbar_wait(&sm.empty[s], (round - 1) & 1, ctl.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) pf_abort(sm, p.status);
         break;
@@ -249,15 +256,19 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
         const int64_t row = gr.row0 + int64_t(tile) * kPT;
         const int64_t left = p.cache_rows - row;  // > 0 and a multiple of 8
         const uint32_t sbytes = uint32_t(left < kPT ? left : kPT) * 4u;
-        sm100::mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sbytes);
-        sm100::tma_load_2d(sm.a[s], &tmap, 0, int32_t(row), &sm.full[s]);
-        sm100::bulk_load(sm.sc[s], p.kscales + row * 4, sbytes, &sm.full[s]);
+        if (!(ctl.withhold && t == 0)) {  // (a test withholds item 0: stage 0 never fills)
+          sm100::mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sbytes);
+          sm100::tma_load_2d(sm.a[s], &tmap, 0, int32_t(row), &sm.full[s]);
+          sm100::bulk_load(sm.sc[s], p.kscales + row * 4, sbytes, &sm.full[s]);
+        }
       }
       ++issued;
     }
-    // every copy this warp issued has landed before the CTA exits
+    // every copy this warp issued has landed before the CTA exits (a withheld
+    // item 0 leaves stage 0 without copies; it is never refilled)
     if (lane == 0)
       for (int s = 0; s < kSt && s < issued; ++s) {
+        if (ctl.withhold && s == 0) continue;
         const int last_round = (issued - 1 - s) / kSt;
         if (!sm100::mbar_wait(&sm.full[s], last_round & 1, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
       }
@@ -275,11 +286,11 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
         }
         if (int64_t(tile) * kPT >= gmax) continue;
         const int s = t % kSt, a = t % kAc;
-        if (!sm100::mbar_wait(&sm.full[s], (t / kSt) & 1)) {
+        if (!sm100::mbar_wait(&sm.full[s], (t / kSt) & 1, ctl.wait_ns)) {
           pf_abort(sm, p.status);
           break;
         }
-        if (t >= kAc && !sm100::mbar_wait(&sm.tempty[a], ((t / kAc) - 1) & 1)) {
+        if (t >= kAc && !sm100::mbar_wait(&sm.tempty[a], ((t / kAc) - 1) & 1, ctl.wait_ns)) {
           pf_abort(sm, p.status);
           break;
         }
@@ -317,7 +328,8 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       if (int64_t(tile) * kPT >= gmax) continue;
       ++t;
       const int s = t % kSt, a = t % kAc;
-      const bool ok = sm100::mbar_wait(&sm.full[s], (t / kSt) & 1) && sm100::mbar_wait(&sm.tfull[a], (t / kAc) & 1);
+      const bool ok = sm100::mbar_wait(&sm.full[s], (t / kSt) & 1, ctl.wait_ns) &&
+                      sm100::mbar_wait(&sm.tfull[a], (t / kAc) & 1, ctl.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) pf_abort(sm, p.status);
         break;
@@ -369,7 +381,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
 __global__ void __launch_bounds__(1024) k_multi_prep(const int64_t* seq_row_off, const int32_t* q_off,
                                                      const int32_t* q_vis, int B, int Q, int G, int64_t max_vis,
                                                      int64_t cache_rows, int4* groups, int64_t* q_row_off,
-                                                     int32_t* vis, uint32_t* status) {
+                                                     int32_t* vis, int32_t* n_groups, uint32_t* status) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -387,7 +399,10 @@ __global__ void __launch_bounds__(1024) k_multi_prep(const int64_t* seq_row_off,
     if (v < 0 || v > Q || (b > 0 && q_off[b - 1] > v)) ok = false;
   }
   if (!__syncthreads_and(ok)) {
-    if (threadIdx.x == 0) set_status(status, CSA2_DEV_LENGTH);
+    if (threadIdx.x == 0) {
+      set_status(status, CSA2_DEV_LENGTH);
+      *n_groups = 0;
+    }
     return;
   }
   for (int base = 0; base < B; base += 1024) {
@@ -446,6 +461,7 @@ __global__ void __launch_bounds__(1024) k_multi_prep(const int64_t* seq_row_off,
     if (threadIdx.x == 1023) carry = first + ng;
     __syncthreads();
   }
+  if (threadIdx.x == 0) *n_groups = min(carry, G);
 }
 
 csa2_status launch_groups_tc(const CUtensorMap& map, PfParams& p, int64_t max_vis, cudaStream_t st) {
@@ -470,13 +486,14 @@ int multi_group_bound(int B, int Q) {
 
 void launch_multi_prep(const int64_t* seq_row_off, const int32_t* q_off, const int32_t* q_vis, int B, int Q, int G,
                        int64_t max_vis, int64_t cache_rows, int4* groups, int64_t* q_row_off, int32_t* vis,
-                       uint32_t* status, cudaStream_t st) {
+                       int32_t* n_groups, uint32_t* status, cudaStream_t st) {
   k_multi_prep<<<1, 1024, 0, st>>>(seq_row_off, q_off, q_vis, B, Q, G, max_vis, cache_rows, groups, q_row_off, vis,
-                                   status);
+                                   n_groups, status);
 }
 
 csa2_status launch_multi_tc(const uint8_t* kcodes, const uint8_t* kscales, int64_t cache_rows,
-                            const int64_t* seq_row_off, const int4* groups, int G, const int32_t* vis, int Q,
+                            const int64_t* seq_row_off, const int4* groups, int G, const int32_t* n_groups,
+                            const int32_t* vis, int Q,
                             int64_t max_vis, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
                             uint32_t* bkeys, int64_t nb_stride, uint32_t* status, cudaStream_t st) {
   if (Q == 0 || max_vis == 0) return CSA2_OK;
@@ -495,6 +512,7 @@ csa2_status launch_multi_tc(const uint8_t* kcodes, const uint8_t* kscales, int64
   p.row0 = 0;
   p.cache_rows = cache_rows;
   p.n_groups = G;
+  p.n_groups_dev = n_groups;
   p.bkeys = bkeys;
   p.nb_stride = nb_stride;
   p.status = status;

@@ -169,6 +169,10 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int n_items = kPool ? p.S * p.items_per_seg : __ldg(p.tile_start + p.S);
+  // wait limit of the pipeline (2 s unless a test sets it) and, in the scan
+  // only, a test's request to withhold the first item's copies
+  const PipeCtl ctl = pipe_ctl(p.status, 2000000000ull);
+  const bool withhold = ctl.withhold && !kPool;
   const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
   const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
 
@@ -249,7 +253,7 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
           }
           j = it - seq_start;
         }
-        const bool ok = round == 0 || sm100::mbar_wait(&sm.empty[s], (round - 1) & 1);
+        const bool ok = round == 0 || sm100::mbar_wait(&sm.empty[s], (round - 1) & 1, ctl.wait_ns);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) abort_kernel(sm, p.status);
           break;
@@ -332,12 +336,14 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
           // an item never crosses a page (pages hold a multiple of kTile rows)
           const int64_t row0 =
               p.sd.pages ? seg_row(p.sd, b, int64_t(j) * kTile, p.status) : seq_off + int64_t(j) * kTile;
-          sm100::mbar_arrive_expect_tx(&sm.full[s], kCodeBytes + sbytes);
+          if (!(withhold && t == 0)) {  // (a test withholds item 0: stage 0 never fills)
+            sm100::mbar_arrive_expect_tx(&sm.full[s], kCodeBytes + sbytes);
 #pragma unroll
-          for (int bx = 0; bx < kTile / kBoxRows; ++bx)
-            sm100::tma_load_2d(sm.a[s] + bx * kBoxRows * kIdxCodeBytes, &tmap, 0, int32_t(row0 + bx * kBoxRows),
-                               &sm.full[s]);
-          sm100::bulk_load(sm.sc[s], p.kscales + row0 * 4, sbytes, &sm.full[s]);
+            for (int bx = 0; bx < kTile / kBoxRows; ++bx)
+              sm100::tma_load_2d(sm.a[s] + bx * kBoxRows * kIdxCodeBytes, &tmap, 0, int32_t(row0 + bx * kBoxRows),
+                                 &sm.full[s]);
+            sm100::bulk_load(sm.sc[s], p.kscales + row0 * 4, sbytes, &sm.full[s]);
+          }
         }
         ++issued;
       }
@@ -349,9 +355,12 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
           for (int t = max(0, issued - kGatherDepth); t < issued; ++t) sm100::mbar_arrive(&sm.full[t % kStages]);
       }
     }
-    // drain: every copy this warp issued has landed before the CTA exits
+    // drain: every copy this warp issued has landed before the CTA exits (a
+    // withheld item 0 leaves stage 0 without copies: it is never refilled,
+    // since that needs item 0 consumed first)
     if (!kPool && lane == 0)
       for (int s = 0; s < kStages && s < issued; ++s) {
+        if (withhold && s == 0) continue;
         const int last_round = (issued - 1 - s) / kStages;
         if (!sm100::mbar_wait(&sm.full[s], last_round & 1, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
       }
@@ -362,11 +371,11 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
       const uint32_t sfa = tmem + kSfCol, sfb = tmem + kSfCol + 32;
       for (int it = i0; it < i1; ++it) {
         const int t = it - i0, s = t % kStages, a = t % kAcc;
-        if (!sm100::mbar_wait(&sm.full[s], (t / kStages) & 1)) {
+        if (!sm100::mbar_wait(&sm.full[s], (t / kStages) & 1, ctl.wait_ns)) {
           abort_kernel(sm, p.status);
           break;
         }
-        if (t >= kAcc && !sm100::mbar_wait(&sm.tempty[a], ((t / kAcc) - 1) & 1)) {
+        if (t >= kAcc && !sm100::mbar_wait(&sm.tempty[a], ((t / kAcc) - 1) & 1, ctl.wait_ns)) {
           abort_kernel(sm, p.status);
           break;
         }
@@ -398,8 +407,8 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
     IdxQCtx qc;
     for (int it = i0 + team; it < i1; it += kEpiTeams) {
       const int t = it - i0, s = t % kStages, a = t % kAcc;
-      const bool ok =
-          sm100::mbar_wait(&sm.full[s], (t / kStages) & 1) && sm100::mbar_wait(&sm.tfull[a], (t / kAcc) & 1);
+      const bool ok = sm100::mbar_wait(&sm.full[s], (t / kStages) & 1, ctl.wait_ns) &&
+                      sm100::mbar_wait(&sm.tfull[a], (t / kAcc) & 1, ctl.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) abort_kernel(sm, p.status);
         break;

@@ -2,6 +2,7 @@
 against the oracle's own step: pools and Top-k bit-exact, attention within
 tolerance.  Includes the full-size configurations (sampled for the 1M one)."""
 import math
+import os
 
 import numpy as np
 import pytest
@@ -68,32 +69,93 @@ def test_decode_stack_full_size():
     _run_and_compare(W.decode_workloads()["stack_decode_b32_l128k"])
 
 
-def test_decode_long_full_size_sampled():
-    """B=64, L=2^20, F R R U: the whole batch runs on the GPU; three sequences
-    are recomputed by the oracle (their cache rows copied back from the device
-    generator, which equals the NumPy generator byte for byte)."""
-    wl = W.decode_workloads()["long_decode_b64_l1m"]
+def _host_cores():
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def _compare_streamed(wl, step, caches_dev, layers, full_rescan=False, group_bytes=4 << 30):
+    """Every sequence of a step that ran on device-resident caches, against
+    the oracle's decode step.  The sequences' cache rows are copied to the
+    host a group at a time (at most `group_bytes` of cache rows, at most one
+    sequence per host core), so host memory stays bounded; the oracle runs
+    each group on all host cores.  Top-k of every layer and the pool of every
+    scanning layer bit-exact; attention within tolerance per sequence and
+    layer."""
+    off = caches_dev[0]["seq_row_off"]
+    lens = wl.lengths.astype(np.int64)
+    per_pos = 340 * len(caches_dev)  # 68 B indexer K + 272 B main KV per Full layer
+    sm = 1 / math.sqrt(512)
+    topk = [host(t) for t in step.topk]
+    pools = {layer: host(t) for layer, t in step.pools.items()}
+    out, lse = host(step.out), host(step.lse)
+    b = 0
+    while b < wl.B:
+        group, size = [], 0
+        while b < wl.B and len(group) < _host_cores() and (not group or size + lens[b] * per_pos <= group_bytes):
+            group.append(b)
+            size += int(lens[b]) * per_pos
+            b += 1
+        pad = (lens[group] + 7) // 8 * 8
+        off_h = np.concatenate([[0], np.cumsum(pad)[:-1]]).astype(np.int64)
+        rows = int(pad.sum())
+        caches_h = []
+        for c in caches_dev:
+            h = dict(idx_codes=np.zeros((rows, 64), np.uint8), idx_scales=np.zeros((rows, 4), np.uint8),
+                     main_codes=np.zeros((rows, 256), np.uint8), main_scales=np.zeros((rows, 16), np.uint8))
+            for j, bb in enumerate(group):
+                o, L, oh = int(off[bb]), int(lens[bb]), int(off_h[j])
+                for key in h:
+                    h[key][oh:oh + L] = host(c[key][o:o + L])
+            caches_h.append(h)
+        lg = [{k: (v[group] if isinstance(v, np.ndarray) and v.ndim >= 1 and v.shape[0] == wl.B else v)
+               for k, v in L_.items()} for L_ in layers]
+        ref = oracle.decode_step(wl.pattern, caches_h, off_h, lens[group].astype(np.int32), lg, wl.P, wl.k, sm,
+                                 full_rescan=full_rescan)
+        for layer in range(len(wl.pattern)):
+            assert np.array_equal(topk[layer][group], ref["topk"][layer]), (group, layer)
+            for j, bb in enumerate(group):
+                check_attention(out[layer][bb], ref["out"][layer][j], lse[layer][bb], ref["lse"][layer][j],
+                                what=f"seq {bb} layer {layer}")
+        assert sorted(ref["pools"]) == sorted(pools)
+        for layer, pool in ref["pools"].items():
+            assert np.array_equal(pools[layer][group], pool), (group, layer)
+
+
+def _full_size_step(wl, full_rescan=False):
     layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
-    c = W.full_cache_device(wl, 0, layers[0]["q_codes"], layers[0]["q_scales"])
-    cache = FullCache(C.cache(c["idx_codes"], c["idx_scales"]), C.cache(c["main_codes"], c["main_scales"]))
-    off = c["seq_row_off"]
-    lens = wl.lengths.astype(np.int32)
-    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k)
-    step.run([cache], dev(off), dev(lens), _device_layers(layers))
+    caches = [W.full_cache_device(wl, f, layers[f]["q_codes"], layers[f]["q_scales"]) for f in wl.full_layers()]
+    fc = [FullCache(C.cache(c["idx_codes"], c["idx_scales"]), C.cache(c["main_codes"], c["main_scales"]))
+          for c in caches]
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, full_rescan=full_rescan)
+    step.run(fc, dev(caches[0]["seq_row_off"]), dev(wl.lengths.astype(np.int32)), _device_layers(layers))
     torch.cuda.synchronize()
     assert step.device_flags() == 0
-    for b in (0, 37, 63):
-        o, L = int(off[b]), int(lens[b])
-        ch = dict(idx_codes=host(c["idx_codes"][o:o + L]), idx_scales=host(c["idx_scales"][o:o + L]),
-                  main_codes=host(c["main_codes"][o:o + L]), main_scales=host(c["main_scales"][o:o + L]))
-        lb = [{k: (v[b:b + 1] if isinstance(v, np.ndarray) and v.ndim >= 1 and v.shape[0] == wl.B else v)
-               for k, v in L_.items()} for L_ in layers]
-        ref = oracle.decode_step(wl.pattern, [ch], np.array([0]), np.array([L], np.int32), lb, wl.P, wl.k,
-                                 1 / math.sqrt(512))
-        for layer in range(4):
-            assert np.array_equal(host(step.topk[layer][b:b + 1]), ref["topk"][layer]), (b, layer)
-            check_attention(host(step.out[layer][b:b + 1]), ref["out"][layer], what=f"seq {b} layer {layer}")
-        assert np.array_equal(host(step.pool[b:b + 1]), ref["pools"][0])
+    return step, caches, layers
+
+
+def test_decode_long_full_size_all_sequences():
+    """B = 64, L = 2^20, F R R U, the bench's launch configuration: every one
+    of the 64 sequences checked against the oracle (cache rows streamed to
+    the host from the device generator, which equals the NumPy generator
+    byte for byte)."""
+    wl = W.decode_workloads()["long_decode_b64_l1m"]
+    step, caches, layers = _full_size_step(wl)
+    _compare_streamed(wl, step, caches, layers)
+
+
+@pytest.mark.parametrize("rescan", [False, True])
+def test_decode_ragged_20_layers_full_size(rescan):
+    """B = 48, lengths log-uniform on [4096, 2^20], 20 layers (F R U R U) x 4
+    with four Full layers' own caches, at full size, under the pages' plan
+    (only the first Full layer scans; later Full layers select inside its
+    pool with their own caches) and with every Full layer rescanning: every
+    sequence, every layer, against the oracle."""
+    wl = W.decode_workloads()["ragged_decode_b48_20l"]
+    step, caches, layers = _full_size_step(wl, full_rescan=rescan)
+    _compare_streamed(wl, step, caches, layers, full_rescan=rescan)
 
 
 def test_decode_with_input_events_and_layer_callbacks():

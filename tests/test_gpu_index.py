@@ -134,12 +134,13 @@ def test_reindex_flags_out_of_range_pool_block():
     assert set(got[got >= 0].tolist()) == set(range(8, 16)) | set(range(40, 48))
 
 
-@pytest.mark.parametrize("qmin,qmax", [(100, 150), (2, 200)])
+@pytest.mark.parametrize("qmin,qmax", [(100, 150), (2, 200), (2, 253), (180, 253)])
 def test_index_multi_extreme_scales(qmin, qmax):
     """The multi-query scan with wide key and query exponent spreads (its
-    fp64 epilogue path) and query scale bytes far from 127 stays bit-exact.
-    Scales stay low enough that no score overflows: an infinite head sum can
-    turn into NaN, whose bits differ between the CPU and the GPU."""
+    fp64 epilogue path) and query scale bytes over the whole E8M0 range stays
+    bit-exact.  Near the top of the range head dots overflow to +-inf and
+    head sums of +inf and -inf give NaN; every NaN ranks below every number
+    on both sides."""
     rng = np.random.default_rng(qmin + qmax)
     lengths = [3000, 2048, 777]
     kc, ks, off, _ = _random_cache(rng, lengths, smin=90, smax=160)
@@ -158,3 +159,88 @@ def test_index_multi_extreme_scales(qmin, qmax):
     assert C.device_status(ws) == 0
     wp, wt = oracle.index_multi(kc, ks, qc, qs, w, off, q_off, q_vis, P, k)
     assert np.array_equal(host(pool), wp) and np.array_equal(host(top), wt)
+
+
+def test_index_infinite_and_nan_scores():
+    """Scores that overflow fp32 to +-inf, and head sums of +inf and -inf
+    (NaN), on both Full-layer paths (stored scores when P < k, the pool
+    re-score when P >= k), Reindex and the multi-query scan: pools and Top-k
+    bit-exact with the oracle (every NaN ranks below every number, NaNs by
+    position); stored scores equal bit for bit, NaN where the oracle's is."""
+    from tests.test_oracle_index import _overflow_case
+
+    kc0, ks0, qc0, qs0, w0, kinds = _overflow_case(1000)
+    rng = np.random.default_rng(92)
+    kc1, ks1, _, _ = _random_cache(rng, [3001])
+    kc = np.concatenate([kc0, kc1])      # sequence 0: rows 0..999, sequence 1: rows 1000..4000
+    ks = np.concatenate([ks0, ks1])
+    off = np.array([0, 1000], np.int64)
+    lengths = [1000, 3001]
+    qc, qs, w = np.stack([qc0, qc0]), np.stack([qs0, qs0]), np.stack([w0, w0])
+    # P < k: Top-k over the stored scores
+    gp, gt, gs = _run_full(kc, ks, off, lengths, qc, qs, w, 64, 512, want_scores=True)
+    op, ot, osc = oracle.index_full(kc, ks, qc, qs, w, off, np.asarray(lengths), 64, 512, want_scores=True)
+    assert np.array_equal(gp, op) and np.array_equal(gt, ot)
+    for b, L in enumerate(lengths):
+        nan = np.isnan(osc[b, :L])
+        assert np.array_equal(np.isnan(gs[b, :L]), nan)
+        assert np.array_equal(gs[b, :L][~nan].view(np.uint32), osc[b, :L][~nan].view(np.uint32))
+    assert np.isnan(osc[0, 120:860]).all() and (osc[0, 100:120] == np.inf).all()
+    # P >= k: the pool re-score path, with NaN positions inside the Top-k
+    gp, gt, _ = _run_full(kc, ks, off, lengths, qc, qs, w, 128, 400)
+    op, ot, _ = oracle.index_full(kc, ks, qc, qs, w, off, np.asarray(lengths), 128, 400)
+    assert np.array_equal(gp, op) and np.array_equal(gt, ot)
+    assert set(range(120, 260)) <= set(gt[0].tolist())   # the first 140 NaN positions
+    # Reindex inside that pool
+    want = oracle.index_reindex(kc, ks, qc, qs, w, off, np.asarray(lengths), op, 400)
+    top = torch.full((2, 400), -7, dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_index_reindex_workspace_bytes(2, 128, 400))
+    keep = [dev(qc), dev(qs), dev(w), dev(off), dev(np.asarray(lengths, np.int32)), dev(op)]
+    C.csa2_index_reindex(C.cache(dev(kc), dev(ks)), *keep[:5], keep[5], 400, top, ws)
+    torch.cuda.synchronize()
+    assert C.device_status(ws) == 0
+    assert np.array_equal(host(top), want)
+    # the multi-query scan: two queries on sequence 0, one on sequence 1
+    q_off = np.array([0, 2, 3], np.int32)
+    q_vis = np.array([1000, 950, 3001], np.int32)
+    qm, qsm, wm = qc[[0, 0, 1]], qs[[0, 0, 1]], w[[0, 0, 1]]
+    pool = torch.full((3, 128), -7, dtype=torch.int32, device="cuda")
+    top = torch.full((3, 400), -7, dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_index_multi_workspace_bytes(2, 3, 3001, 128, 400))
+    C.csa2_index_multi(C.cache(dev(kc), dev(ks)), dev(qm), dev(qsm), dev(wm), dev(off), dev(q_off), dev(q_vis), 3001,
+                       128, 400, pool, top, ws)
+    torch.cuda.synchronize()
+    assert C.device_status(ws) == 0
+    wp, wt = oracle.index_multi(kc, ks, qm, qsm, wm, off, q_off, q_vis, 128, 400)
+    assert np.array_equal(host(pool), wp) and np.array_equal(host(top), wt)
+
+
+@pytest.mark.parametrize("P,k", [(2048, 512), (256, 512)])
+def test_select_overfull_threshold_bucket(P, k):
+    """Every indexer-K row identical: all keys tie, so the threshold bucket
+    holds every key (far more than the 12288 the in-block lists take) and the
+    selections fall back to global radix passes, which a diagnostic counter
+    in the status block (word 4) records.  The pool must be blocks 0..P-1 and
+    the Top-k positions 0..k-1, as the oracle says."""
+    rng = np.random.default_rng(17)
+    lengths = [300001, 140000]
+    kc, ks, off, _ = _random_cache(rng, lengths)
+    kc[:] = kc[0]
+    ks[:] = ks[0]
+    qc, qs, w = _queries(rng, 2)
+    B, max_len = 2, max(lengths)
+    cache = C.cache(dev(kc), dev(ks))
+    args = [dev(qc), dev(qs), dev(w), dev(off), dev(np.asarray(lengths, np.int32))]
+    pool = torch.full((B, P), -7, dtype=torch.int32, device="cuda")
+    top = torch.full((B, k), -7, dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_index_full_workspace_bytes(B, max_len, P, k))
+    C.csa2_index_full(cache, *args, max_len, P, k, pool, top, ws)
+    torch.cuda.synchronize()
+    overfull = int(ws[:32].view(torch.int32)[4].item())
+    assert C.device_status(ws) == 0
+    # the pool select of both sequences (and with P < k the Top-k over the
+    # stored scores as well) took the global radix path
+    assert overfull == (2 if P >= k else 4), overfull
+    op, ot, _ = oracle.index_full(kc, ks, qc, qs, w, off, np.asarray(lengths), P, k)
+    assert np.array_equal(host(pool), op) and np.array_equal(host(top), ot)
+    assert host(pool)[0].tolist() == list(range(P)) and host(top)[1].tolist() == list(range(k))

@@ -64,7 +64,11 @@ def test_prefill_reduced(P, k, use_proj, T):
     check_attention(g["out"], ro, g["lse"], rl)
 
 
-def test_prefill_full_size_sampled():
+def test_prefill_full_size_512_queries():
+    """The full prefill workload (262144 raw tokens, 4096 queries): every
+    compressed and quantised byte, and a seeded subset of 512 query rows (the
+    first 8, the last 8 and 496 drawn at random) for pools, Top-k and
+    attention."""
     pw = W.prefill_workload()
     inp = W.prefill_inputs_host(pw)
     g = _gpu_prefill(inp, pw.n_raw, pw.T, pw.ratio, pw.P, pw.k, pw.use_projection)
@@ -72,7 +76,10 @@ def test_prefill_full_size_sampled():
     n = g["n_ent"]
     for a, b in ((g["mc"], mc), (g["ms"], ms), (g["ic"], ic), (g["isc"], isc)):
         assert np.array_equal(a[:n], b)
-    ids = np.array([0, 1, 2, 1000, 2047, 3000, 4094, 4095], np.int32)
+    rng = np.random.default_rng(4096)
+    middle = rng.choice(np.arange(8, pw.T - 8), 496, replace=False)
+    ids = np.sort(np.concatenate([np.arange(8), middle, np.arange(pw.T - 8, pw.T)])).astype(np.int32)
+    assert len(np.unique(ids)) == 512
     pool, top = oracle.index_prefill(ic, isc, 0, n, inp["q_codes"], inp["q_scales"], inp["w"], inp["q_pos"], 2, pw.P,
                                      pw.k, q_ids=ids)
     assert np.array_equal(g["pool"][ids], pool) and np.array_equal(g["top"][ids], top)

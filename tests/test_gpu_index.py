@@ -187,14 +187,14 @@ def test_index_infinite_and_nan_scores():
         assert np.array_equal(gs[b, :L][~nan].view(np.uint32), osc[b, :L][~nan].view(np.uint32))
     assert np.isnan(osc[0, 120:860]).all() and (osc[0, 100:120] == np.inf).all()
     # P >= k: the pool re-score path, with NaN positions inside the Top-k
-    gp, gt, _ = _run_full(kc, ks, off, lengths, qc, qs, w, 128, 400)
-    op, ot, _ = oracle.index_full(kc, ks, qc, qs, w, off, np.asarray(lengths), 128, 400)
+    gp, gt, _ = _run_full(kc, ks, off, lengths, qc, qs, w, 512, 400)
+    op, ot, _ = oracle.index_full(kc, ks, qc, qs, w, off, np.asarray(lengths), 512, 400)
     assert np.array_equal(gp, op) and np.array_equal(gt, ot)
     assert set(range(120, 260)) <= set(gt[0].tolist())   # the first 140 NaN positions
     # Reindex inside that pool
     want = oracle.index_reindex(kc, ks, qc, qs, w, off, np.asarray(lengths), op, 400)
     top = torch.full((2, 400), -7, dtype=torch.int32, device="cuda")
-    ws = C.workspace(C.csa2_index_reindex_workspace_bytes(2, 128, 400))
+    ws = C.workspace(C.csa2_index_reindex_workspace_bytes(2, 512, 400))
     keep = [dev(qc), dev(qs), dev(w), dev(off), dev(np.asarray(lengths, np.int32)), dev(op)]
     C.csa2_index_reindex(C.cache(dev(kc), dev(ks)), *keep[:5], keep[5], 400, top, ws)
     torch.cuda.synchronize()
@@ -204,14 +204,14 @@ def test_index_infinite_and_nan_scores():
     q_off = np.array([0, 2, 3], np.int32)
     q_vis = np.array([1000, 950, 3001], np.int32)
     qm, qsm, wm = qc[[0, 0, 1]], qs[[0, 0, 1]], w[[0, 0, 1]]
-    pool = torch.full((3, 128), -7, dtype=torch.int32, device="cuda")
+    pool = torch.full((3, 512), -7, dtype=torch.int32, device="cuda")
     top = torch.full((3, 400), -7, dtype=torch.int32, device="cuda")
-    ws = C.workspace(C.csa2_index_multi_workspace_bytes(2, 3, 3001, 128, 400))
+    ws = C.workspace(C.csa2_index_multi_workspace_bytes(2, 3, 3001, 512, 400))
     C.csa2_index_multi(C.cache(dev(kc), dev(ks)), dev(qm), dev(qsm), dev(wm), dev(off), dev(q_off), dev(q_vis), 3001,
-                       128, 400, pool, top, ws)
+                       512, 400, pool, top, ws)
     torch.cuda.synchronize()
     assert C.device_status(ws) == 0
-    wp, wt = oracle.index_multi(kc, ks, qm, qsm, wm, off, q_off, q_vis, 128, 400)
+    wp, wt = oracle.index_multi(kc, ks, qm, qsm, wm, off, q_off, q_vis, 512, 400)
     assert np.array_equal(host(pool), wp) and np.array_equal(host(top), wt)
 
 

@@ -522,6 +522,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
   const int n = attn_main_chunks(a.k) + kWinChunks;
   const int c0 = int(int64_t(n) * r / R), c1 = int(int64_t(n) * (r + 1) / R);
   const int nslots = 2 * R;
+  launch_dependents();
   float oacc[8][4];
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt)
@@ -531,6 +532,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
     sm.m_run[tid] = -INFINITY;
     sm.l_run[tid] = 0.0f;
   }
+  grid_wait();  // the Top-k ids, queries and rows may come from the previous kernel
   bool ok = false;
   int32_t tnext = -1;
   if (c0 < c1) {
@@ -584,7 +586,7 @@ void launch_attention(const AttnArgs& a, cudaStream_t st) {
   if (a.S == 0) return;
   const int R = attn_splits(a.S, a.k);
   prepare_attention();
-  k_attn<<<dim3(R, a.S), kAttnThreads, sizeof(AttnSmem), st>>>(a, R);
+  launch_k(k_attn, dim3(R, a.S), dim3(kAttnThreads), sizeof(AttnSmem), st, a, R);
 }
 
 }  // namespace csa2

@@ -144,6 +144,8 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
   double (*cbuf)[kD] = reinterpret_cast<double (*)[kD]>(csm);
   float (*rbuf)[kDi] = reinterpret_cast<float (*)[kDi]>(csm + sizeof(double) * kCompEntries * kD);
   __shared__ int last_cta;
+  launch_dependents();
+  grid_wait();
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool streaming = a.pend_n != nullptr;
@@ -325,7 +327,7 @@ void launch_compress(const CompressArgs& a, cudaStream_t st) {
   const int64_t gx = a.max_new > 0 ? (a.max_new + kCompEntries - 1) / kCompEntries : 1;
   const size_t smem = sizeof(double) * kCompEntries * kD + sizeof(float) * kCompEntries * kDi;
   cudaFuncSetAttribute(k_compress, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  k_compress<<<dim3(static_cast<unsigned>(gx), a.B), kCompWarps * 32, smem, st>>>(a);
+  launch_k(k_compress, dim3(static_cast<unsigned>(gx), a.B), dim3(kCompWarps * 32), smem, st, a);
 }
 
 }  // namespace csa2

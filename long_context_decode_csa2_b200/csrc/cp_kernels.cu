@@ -33,6 +33,8 @@ __global__ void __launch_bounds__(256) k_score_positions(const uint8_t* kcodes, 
   __shared__ uint32_t qw[kHi][kDi / 4];  // query: int8x4 of elements 4i .. 4i+3 per head
   __shared__ uint16_t lut[256];          // code byte -> two int8 doubled values (low nibble first)
   __shared__ IdxQCtx qc;
+  launch_dependents();
+  grid_wait();
   const int b = blockIdx.y;
   {
     const int t = threadIdx.x;  // 256 threads: one LUT entry each
@@ -99,6 +101,8 @@ __global__ void __launch_bounds__(256) k_score_positions(const uint8_t* kcodes, 
 // with ids made global by the shard's offset src_off[g][b] (or as given).
 __global__ void k_merge_gather(const uint32_t* keys, const int32_t* ids, const int64_t* src_off, int G, int B, int n,
                                uint32_t* keys_t, int32_t* ids_t, uint32_t* status) {
+  launch_dependents();
+  grid_wait();
   const int b = blockIdx.y;
   const int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;  // candidate g * n + i of segment b
   if (c >= int64_t(G) * n) return;
@@ -120,6 +124,8 @@ __global__ void k_merge_gather(const uint32_t* keys, const int32_t* ids, const i
 // out_local[b][j] = out[b][j] - lo[b] where lo[b] <= out[b][j] < hi[b], else -1.
 __global__ void k_localize(const int32_t* out, int B, int k, const int64_t* lo, const int64_t* hi,
                            int32_t* out_local) {
+  launch_dependents();
+  grid_wait();
   const int b = blockIdx.y;
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= k) return;
@@ -131,6 +137,8 @@ __global__ void k_localize(const int32_t* out, int B, int k, const int64_t* lo, 
 // out = sum_g exp(lse_g - M) out_g / sum_g exp(lse_g - M), lse = M + log(sum).
 __global__ void __launch_bounds__(512) k_attn_combine(const float* out_parts, const float* lse_parts, int G, int B,
                                                       float* out, float* lse) {
+  launch_dependents();
+  grid_wait();
   const int b = blockIdx.x, h = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float M = -INFINITY;
   for (int g = 0; g < G; ++g) M = fmaxf(M, lse_parts[(int64_t(g) * B + b) * kHq + h]);
@@ -167,28 +175,28 @@ void launch_score_positions(const uint8_t* kcodes, const uint8_t* kscales, const
                             uint32_t* keys_out, uint32_t* status, cudaStream_t st) {
   if (B == 0 || n == 0) return;
   const int64_t threads = int64_t(n) * blk;
-  k_score_positions<<<dim3(unsigned((threads + 255) / 256), B), 256, 0, st>>>(kcodes, kscales, sd, q_codes, q_scales,
-                                                                              w, ids, n, blk, keys_out, status);
+  launch_k(k_score_positions, dim3(unsigned((threads + 255) / 256), B), dim3(256), 0, st, kcodes, kscales, sd, q_codes,
+           q_scales, w, ids, n, blk, keys_out, status);
 }
 
 void launch_merge_gather(const uint32_t* keys, const int32_t* ids, const int64_t* src_off, int G, int B, int n,
                          uint32_t* keys_t, int32_t* ids_t, uint32_t* status, cudaStream_t st) {
   const int64_t c = int64_t(G) * n;
   if (B == 0 || c == 0) return;
-  k_merge_gather<<<dim3(unsigned((c + 255) / 256), B), 256, 0, st>>>(keys, ids, src_off, G, B, n, keys_t, ids_t,
-                                                                     status);
+  launch_k(k_merge_gather, dim3(unsigned((c + 255) / 256), B), dim3(256), 0, st, keys, ids, src_off, G, B, n, keys_t,
+           ids_t, status);
 }
 
 void launch_localize(const int32_t* out, int B, int k, const int64_t* lo, const int64_t* hi, int32_t* out_local,
                      cudaStream_t st) {
   if (B == 0 || k == 0) return;
-  k_localize<<<dim3(unsigned((k + 255) / 256), B), 256, 0, st>>>(out, B, k, lo, hi, out_local);
+  launch_k(k_localize, dim3(unsigned((k + 255) / 256), B), dim3(256), 0, st, out, B, k, lo, hi, out_local);
 }
 
 void launch_attn_combine(const float* out_parts, const float* lse_parts, int G, int B, float* out, float* lse,
                          cudaStream_t st) {
   if (B == 0) return;
-  k_attn_combine<<<B, 512, 0, st>>>(out_parts, lse_parts, G, B, out, lse);
+  launch_k(k_attn_combine, dim3(B), dim3(512), 0, st, out_parts, lse_parts, G, B, out, lse);
 }
 
 }  // namespace csa2

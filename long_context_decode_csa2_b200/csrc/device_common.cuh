@@ -9,6 +9,15 @@
 
 namespace csa2 {
 
+// Programmatic dependent launch (every kernel here is launched with it, see
+// launch_k): launch_dependents lets the stream's next kernel be scheduled and
+// run its prologue while this one still works; grid_wait blocks until every
+// prerequisite grid has completed and its memory writes are visible.  Each
+// kernel calls grid_wait in every CTA before its first global access, so the
+// usual stream order holds for all data (and completes transitively).
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t flag) {
   if (status) atomicOr(status, flag);
 }

@@ -16,6 +16,8 @@ namespace csa2 {
 // ---------------------------------------------------------------------------
 __global__ void k_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entries, int32_t* vis,
                               uint32_t* status) {
+  launch_dependents();
+  grid_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= T) return;
   int64_t p = q_pos[i];
@@ -31,7 +33,7 @@ __global__ void k_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_
 void launch_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entries, int32_t* vis, uint32_t* status,
                         cudaStream_t st) {
   if (T == 0) return;
-  k_prefill_vis<<<(T + 255) / 256, 256, 0, st>>>(q_pos, T, ratio, n_entries, vis, status);
+  launch_k(k_prefill_vis, dim3((T + 255) / 256), dim3(256), 0, st, q_pos, T, ratio, n_entries, vis, status);
 }
 
 // ---------------------------------------------------------------------------
@@ -328,6 +330,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
                                                         uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) uint32_t dsm[];
   __shared__ SelShared sh;
+  launch_dependents();
+  grid_wait();
   const int s = blockIdx.x;
   const int tid = threadIdx.x;
   int64_t n;
@@ -624,11 +628,13 @@ void launch_select_kind(const void* in, int64_t in_stride, const int32_t* seg_ef
     const size_t smem = (hist ? NB + 1024 : 256) * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int((NB + 1024) * sizeof(uint32_t)));
-    k_select<KIND, true><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, status);
+    launch_k(k_select<KIND, true>, dim3(S), dim3(kSelThreads), smem, st, in, in_stride, seg_eff, P, pool, k, out, hist,
+             status);
   } else {
     const size_t smem = kSelLargeWords * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    k_select<KIND, false><<<S, kSelThreads, smem, st>>>(in, in_stride, seg_eff, P, pool, k, out, hist, status);
+    launch_k(k_select<KIND, false>, dim3(S), dim3(kSelThreads), smem, st, in, in_stride, seg_eff, P, pool, k, out,
+             hist, status);
   }
 }
 

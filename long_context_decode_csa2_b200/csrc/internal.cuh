@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 
 #include "csa2.h"
 
@@ -40,6 +41,24 @@ void set_error(const std::string& msg);
 csa2_status fail(csa2_status code, const std::string& msg);
 csa2_status check_launch(const char* what);
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Launches `kernel` on `st` with programmatic stream serialisation: it may
+// start (and run its prologue up to grid_wait) while the previous kernel of
+// the stream finishes.  Errors surface through cudaGetLastError.
+template <typename... KArgs, typename... Args>
+inline void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Row stride (in keys) of the per-block key arrays: whole 16-byte groups, so
 // every row starts 16-byte aligned for vector loads.

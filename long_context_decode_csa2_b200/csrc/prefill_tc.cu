@@ -183,16 +183,9 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   PfSmem& sm = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // items are split over the groups that exist (the table's capacity is a
-  // host bound; empty entries past the real count would idle their CTAs)
-  const int n_groups = p.n_groups_dev ? min(p.n_groups, max(0, __ldg(p.n_groups_dev))) : p.n_groups;
-  const int n_items = n_groups * p.n_tiles;
-  // wait limit of the pipeline (2 s unless a test sets it); a test may also
-  // have the producer withhold its first item's copies
-  const PipeCtl ctl = pipe_ctl(p.status, 2000000000ull);
-  const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
-  const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
+  launch_dependents();
 
+  // prologue (touches no global memory): barriers, tensor memory, unit scales
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSt; ++s) {
       sm100::mbar_init(&sm.full[s], 1);
@@ -224,6 +217,17 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
+  grid_wait();  // the group table, visible counts and queries come from earlier kernels
+
+  // items are split over the groups that exist (the table's capacity is a
+  // host bound; empty entries past the real count would idle their CTAs)
+  const int n_groups = p.n_groups_dev ? min(p.n_groups, max(0, __ldg(p.n_groups_dev))) : p.n_groups;
+  const int n_items = n_groups * p.n_tiles;
+  // wait limit of the pipeline (2 s unless a test sets it); a test may also
+  // have the producer withhold its first item's copies
+  const PipeCtl ctl = pipe_ctl(p.status, 2000000000ull);
+  const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
+  const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -384,6 +388,8 @@ __global__ void __launch_bounds__(1024) k_multi_prep(const int64_t* seq_row_off,
                                                      int32_t* vis, int32_t* n_groups, uint32_t* status) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
+  launch_dependents();
+  grid_wait();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int q = threadIdx.x; q < Q; q += blockDim.x) {
     vis[q] = 0;
@@ -473,7 +479,7 @@ csa2_status launch_groups_tc(const CUtensorMap& map, PfParams& p, int64_t max_vi
   const size_t smem = std::max<size_t>(sizeof(PfSmem) + 1024, 120 * 1024);
   cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   const int grid = int(std::min<int64_t>(num_sms(), n_items));
-  k_prefill_tc<<<grid, kThr, smem, st>>>(map, p);
+  launch_k(k_prefill_tc, dim3(grid), dim3(kThr), smem, st, map, p);
   return CSA2_OK;
 }
 
@@ -487,8 +493,8 @@ int multi_group_bound(int B, int Q) {
 void launch_multi_prep(const int64_t* seq_row_off, const int32_t* q_off, const int32_t* q_vis, int B, int Q, int G,
                        int64_t max_vis, int64_t cache_rows, int4* groups, int64_t* q_row_off, int32_t* vis,
                        int32_t* n_groups, uint32_t* status, cudaStream_t st) {
-  k_multi_prep<<<1, 1024, 0, st>>>(seq_row_off, q_off, q_vis, B, Q, G, max_vis, cache_rows, groups, q_row_off, vis,
-                                   n_groups, status);
+  launch_k(k_multi_prep, dim3(1), dim3(1024), 0, st, seq_row_off, q_off, q_vis, B, Q, G, max_vis, cache_rows, groups,
+           q_row_off, vis, n_groups, status);
 }
 
 csa2_status launch_multi_tc(const uint8_t* kcodes, const uint8_t* kscales, int64_t cache_rows,

@@ -167,15 +167,9 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  launch_dependents();
 
-  const int n_items = kPool ? p.S * p.items_per_seg : __ldg(p.tile_start + p.S);
-  // wait limit of the pipeline (2 s unless a test sets it) and, in the scan
-  // only, a test's request to withhold the first item's copies
-  const PipeCtl ctl = pipe_ctl(p.status, 2000000000ull);
-  const bool withhold = ctl.withhold && !kPool;
-  const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
-  const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
-
+  // prologue (touches no global memory): barriers, tensor memory, unit scales
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       sm100::mbar_init(&sm.full[s], kPool ? kPoolProducers : 1);
@@ -209,6 +203,15 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
+  grid_wait();  // the item prefix, lengths, pool and histograms come from earlier kernels
+
+  const int n_items = kPool ? p.S * p.items_per_seg : __ldg(p.tile_start + p.S);
+  // wait limit of the pipeline (2 s unless a test sets it) and, in the scan
+  // only, a test's request to withhold the first item's copies
+  const PipeCtl ctl = pipe_ctl(p.status, 2000000000ull);
+  const bool withhold = ctl.withhold && !kPool;
+  const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
+  const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
 
   if (warp == 0 || warp >= kFirstExtra) {
     // ------------------------------------------------------------ producer(s)
@@ -487,6 +490,8 @@ __global__ void __launch_bounds__(1024) k_seg_prep(SegDesc sd, int S, int32_t* s
                                                     uint32_t* status) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
+  launch_dependents();
+  grid_wait();
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -575,7 +580,7 @@ void launch_index_tc(const CUtensorMap& map, const ScanParams& p, int64_t max_it
   const size_t smem = sizeof(ScanSmem<Ring<kPool>::kStages>) + 1024;
   cudaFuncSetAttribute(k_index_tc<kPool>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   const int grid = int(std::min<int64_t>(num_sms(), std::max<int64_t>(max_items, 1)));
-  k_index_tc<kPool><<<grid, threads_of<kPool>(), smem, st>>>(map, p);
+  launch_k(k_index_tc<kPool>, dim3(grid), dim3(threads_of<kPool>()), smem, st, map, p);
 }
 
 }  // namespace
@@ -587,7 +592,7 @@ csa2_status launch_scan_tc(const uint8_t* kcodes, const uint8_t* kscales, const 
                            const float* w, uint32_t* bkeys, int64_t nb_stride, float* scores, int64_t score_stride,
                            uint32_t* hist, uint32_t* status, cudaStream_t st) {
   if (S == 0) return CSA2_OK;
-  k_seg_prep<<<1, 1024, 0, st>>>(sd, S, seg_eff, tile_start, status);
+  launch_k(k_seg_prep, dim3(1), dim3(1024), 0, st, sd, S, seg_eff, tile_start, status);
   if (sd.max_len == 0) return CSA2_OK;
   CUtensorMap map;
   const csa2_status rc = code_map(&map, kcodes, sd.cache_rows, kBoxRows);

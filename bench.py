@@ -51,6 +51,9 @@ def parse():
                     help="override every sequence's length (small profiling captures of the attention)")
     ap.add_argument("--full-rescan", action="store_true",
                     help="every Full layer scans its whole context and rebuilds the pool (default: only the first)")
+    ap.add_argument("--peaks", action="store_true",
+                    help="measure the roofline denominators a copy and a GEMM do not give: read-only HBM stream "
+                         "(128-bit loads, bulk copies), tcgen05 FP4 rate at N = 16 and 128, FP64 FMA rate")
     ap.add_argument("--cp", type=int, default=0,
                     help="context-parallel step over this many shards of every sequence: one per rank under "
                          "torchrun, all in this process on one GPU")
@@ -1023,8 +1026,83 @@ def run_cp(args):
         dist.destroy_process_group()
 
 
+PEAKS_SRC = os.path.join(ROOT, "bench_peaks.cu")
+PEAKS_LIB = os.path.join(ROOT, "_build", "libcsa2_peaks.so")
+
+
+def build_peaks(force=False):
+    """Compiles the peak probes (bench_peaks.cu) for sm_100a."""
+    if force or not os.path.exists(PEAKS_LIB) or os.path.getmtime(PEAKS_LIB) < os.path.getmtime(PEAKS_SRC):
+        os.makedirs(os.path.dirname(PEAKS_LIB), exist_ok=True)
+        tmp = PEAKS_LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
+                               "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"), "-I", ROOT,
+                               PEAKS_SRC, "-o", tmp])
+        os.replace(tmp, PEAKS_LIB)
+    return PEAKS_LIB
+
+
+def run_peaks(args):
+    """Roofline denominators measured on this GPU (one JSON line): the
+    read-only HBM stream with 128-bit loads and with bulk copies into shared
+    memory (4 GiB read once per repetition, more than L2), tcgen05.mma
+    kind::mxf4 (unit scales) at M = 128, K = 64 and N = 16 / 128, and FP64
+    FMA.  Median of 10 timed repetitions after 3 warm-ups, CUDA events."""
+    import ctypes
+
+    import torch
+
+    lib = ctypes.CDLL(build_peaks())
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    sms = lib.peaks_num_sms()
+    nbytes = 4 << 30
+    buf = torch.ones(nbytes, dtype=torch.uint8, device=dev)
+    sink = torch.zeros(sms * 8, dtype=torch.int64, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    P = ctypes.c_void_p
+
+    def timed(launch, reps=10, warm=3):
+        for _ in range(warm):
+            assert launch() == 0
+        ms = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            assert launch() == 0
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return statistics.median(ms)
+
+    out = {}
+    with ClockSampler(0) as clk:
+        ms = timed(lambda: lib.peaks_read_ldg(P(buf.data_ptr()), ctypes.c_longlong(nbytes // 16),
+                                              P(sink.data_ptr()), sp))
+        out["hbm_read_ldg128_gbs"] = nbytes / (ms * 1e-3) / 1e9
+        ms = timed(lambda: lib.peaks_read_bulk(P(buf.data_ptr()), ctypes.c_longlong(nbytes), P(err.data_ptr()), sp))
+        out["hbm_read_bulk_gbs"] = nbytes / (ms * 1e-3) / 1e9
+        for n, iters in ((16, 400000), (128, 60000)):
+            ms = timed(lambda: lib.peaks_mma_mxf4(n, iters, P(err.data_ptr()), sp))
+            out[f"fp4_mxf4_n{n}_tflops"] = sms * iters * 2.0 * 128 * n * 64 / (ms * 1e-3) / 1e12
+        iters = 20000
+        ms = timed(lambda: lib.peaks_fma64(iters, P(sink.data_ptr()), sp))
+        out["fp64_fma_tflops"] = sms * 8 * 256 * 8 * iters * 2.0 / (ms * 1e-3) / 1e12
+    torch.cuda.synchronize()
+    out["probe_errors"] = int(err.item())
+    out["sms"] = sms
+    print(json.dumps({"peaks": out, "clocks": clk.summary(),
+                      "method": "bench_peaks.cu kernels, CUDA events, median of 10 after 3 warm-ups; HBM probes read "
+                                "4 GiB once per repetition"}))
+
+
 def main():
     args = parse()
+    if args.peaks:
+        run_peaks(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     elif args.workload.startswith("prefill"):

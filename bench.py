@@ -785,12 +785,12 @@ def run_prefill(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, device, world)
 
     # roofline of the indexer (the dominant call): the causal FP4 score GEMM's
-    # useful FLOPs against the FP4 tensor peak (measured bf16 x the nominal
-    # fp4 / bf16 ratio of 4); its time is the exact epilogue's, not the MMAs'
+    # useful FLOPs against the FP4 tensor peak at the kernel's MMA shape
+    # (kind::mxf4, N = 128), measured here by the peak probe; its time is the
+    # exact epilogue's, not the MMAs'
     n_vis = np.minimum(np.arange(n_raw - T, n_raw, dtype=np.int64) + 1, n_raw) // ratio
     flops = float(n_vis.sum()) * 4 * 128 * 2
-    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    bf16 = float(json.load(open(pk))["bf16_tflops"]) if os.path.exists(pk) else 1590.0
+    fp4_peak, fp4_kind = fp4_peak_tflops()
     achieved = flops / (per_call["csa2_index_prefill"] * 1e-3) / 1e12
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -806,9 +806,8 @@ def run_prefill(args):
                        "topk": k, "window": 128},
             "compress_tokens_per_s": n_raw / (per_call["csa2_compress_append"] * 1e-3),
             "roofline": {"kernel": "csa2_index_prefill (causal FP4 score GEMM + block max + pool + Top-512)",
-                         "bound": "tensor", "achieved": achieved, "peak": 4 * bf16, "unit": "TFLOP/s",
-                         "frac": achieved / (4 * bf16),
-                         "peak_kind": "measured bf16 x 4 (nominal fp4 / bf16)" if os.path.exists(pk) else "fallback",
+                         "bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": achieved / fp4_peak, "peak_kind": fp4_kind,
                          "traffic": None, "note": "bound in fact by the exact CUDA-core epilogue"},
             "cpu_baseline": cpu,
             "e2e": {"value": job_throughput(world, T, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
@@ -1040,6 +1039,40 @@ def build_peaks(force=False):
                                PEAKS_SRC, "-o", tmp])
         os.replace(tmp, PEAKS_LIB)
     return PEAKS_LIB
+
+
+def fp4_peak_tflops():
+    """The FP4 tensor-core rate at the prefill indexer's MMA shape (kind::mxf4,
+    M = N = 128, K = 64), measured now with the peak probe; if the probe
+    cannot run, the measured bf16 rate x 4 (the nominal fp4 / bf16 ratio)."""
+    import ctypes
+
+    import torch
+
+    try:
+        lib = ctypes.CDLL(build_peaks())
+        sms = lib.peaks_num_sms()
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        stream = torch.cuda.current_stream()
+        iters, ms = 60000, []
+        for rep in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            assert lib.peaks_mma_mxf4(128, iters, ctypes.c_void_p(err.data_ptr()),
+                                      ctypes.c_void_p(stream.cuda_stream)) == 0
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                ms.append(e0.elapsed_time(e1))
+        if int(err.item()) == 0:
+            return sms * iters * 2.0 * 128 * 128 * 64 / (statistics.median(ms) * 1e-3) / 1e12, \
+                "measured now: tcgen05 kind::mxf4, N = 128 (bench_peaks.cu)"
+    except Exception:
+        pass
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk):
+        return 4 * float(json.load(open(pk))["bf16_tflops"]), "measured bf16 x 4 (nominal fp4 / bf16)"
+    return 4 * 1590.0, "fallback bf16 x 4"
 
 
 def run_peaks(args):

@@ -69,6 +69,7 @@ struct IndexFullWs {
   int32_t* tile_start;
   uint32_t* bkeys;
   uint32_t* ckeys;
+  int32_t* topblk;  // [B][k]: the best k blocks of every pool (when P >= k)
   float* scores;
   uint32_t* hist;  // [B][kSelHistBins] (block keys, then candidates), zero between calls
   size_t bytes;
@@ -82,7 +83,8 @@ IndexFullWs index_full_ws(void* ws, int B, int max_len, int P, int k, bool need_
   w.tile_start = c.take<int32_t>(scan_tc_prefix_ints(B));
   const size_t nb = size_t(block_key_stride(max_len));
   w.bkeys = c.take<uint32_t>(size_t(B) * nb);
-  w.ckeys = (P >= k) ? c.take<uint32_t>(size_t(B) * P * kBlk) : nullptr;
+  w.ckeys = (P >= k) ? c.take<uint32_t>(size_t(B) * k * kBlk) : nullptr;
+  w.topblk = (P >= k) ? c.take<int32_t>(size_t(B) * k) : nullptr;
   w.scores = need_scores ? c.take<float>(size_t(B) * max_len) : nullptr;
   w.hist = c.take<uint32_t>(size_t(B) * kSelHistBins);
   w.bytes = c.used;
@@ -149,18 +151,19 @@ csa2_status index_full_impl(const char* fn, csa2_mxfp4_cache idx_k, const uint8_
     const csa2_status rc = launch_scan_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, ws.tile_start, B, q_codes,
                                           q_scales, w, ws.bkeys, nb, scores, max_len, ws.hist, ws.status, st);
     if (rc != CSA2_OK) return rc;
+    // the pool, and (P >= k) the best k blocks among it
     launch_select(kSelBlockKeys, ws.bkeys, nb, ws.seg_eff, B, 0, nullptr, pool_blocks, pool_out, ws.hist, st,
-                  ws.status);
+                  ws.status, ws.topblk, k);
   }
   if (!(phases & 2)) return check_launch(fn);
   if (pool_blocks >= k) {
     // Every Top-k position's block ranks within the first k blocks, so the
-    // Top-k over the pool equals the Top-k over all positions.
+    // Top-k over the positions of those blocks equals the Top-k over all
+    // positions: re-score their 8k positions and select.
     const csa2_status rc2 = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.seg_eff, B, q_codes, q_scales, w,
-                                           pool_out, pool_blocks, ws.ckeys, ws.hist, ws.status, st);
+                                           ws.topblk, k, ws.ckeys, ws.hist, ws.status, st);
     if (rc2 != CSA2_OK) return rc2;
-    launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.seg_eff, B, pool_blocks, pool_out, k,
-                  topk_out, ws.hist, st);
+    launch_select(kSelPoolCand, ws.ckeys, int64_t(k) * kBlk, ws.seg_eff, B, k, ws.topblk, k, topk_out, ws.hist, st);
   } else {
     launch_select(kSelScores, scores, max_len, ws.seg_eff, B, 0, nullptr, k, topk_out, nullptr, st, ws.status);
   }
@@ -538,6 +541,7 @@ struct PrefillWs {
   int32_t* vis;
   uint32_t* bkeys;
   uint32_t* ckeys;
+  int32_t* topblk;  // [T][k]: the best k blocks of every pool
   float* scores;
   size_t bytes;
 };
@@ -548,7 +552,9 @@ PrefillWs prefill_ws(void* ws, int T, int64_t n_entries, int P, int k) {
   w.vis = c.take<int32_t>(size_t(T));
   const size_t nb = size_t(block_key_stride(n_entries));
   w.bkeys = c.take<uint32_t>(size_t(T) * nb);
-  w.ckeys = c.take<uint32_t>(size_t(T) * P * kBlk);
+  w.ckeys = c.take<uint32_t>(size_t(T) * k * kBlk);
+  w.topblk = c.take<int32_t>(size_t(T) * k);
+  (void)P;
   w.scores = nullptr;
   w.bytes = c.used;
   return w;
@@ -586,13 +592,14 @@ csa2_status csa2_index_prefill(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, c
   const csa2_status rc0 = launch_prefill_tc(idx_k.codes, idx_k.scales, row0, idx_k.rows, ws.vis, T, n_entries, q_codes,
                                             q_scales, w, ws.bkeys, nb, ws.status, st);
   if (rc0 != CSA2_OK) return rc0;
-  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, T, 0, nullptr, pool_blocks, pool_out, nullptr, st);
+  // the pool, the best k blocks among it, and the Top-k over their positions
+  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, T, 0, nullptr, pool_blocks, pool_out, nullptr, st, ws.status,
+                ws.topblk, k);
   SegDesc sd{nullptr, row0, ws.vis, n_entries, idx_k.rows};
-  const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.vis, T, q_codes, q_scales, w, pool_out,
-                                        pool_blocks, ws.ckeys, nullptr, ws.status, st);
+  const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.vis, T, q_codes, q_scales, w, ws.topblk, k,
+                                        ws.ckeys, nullptr, ws.status, st);
   if (rc != CSA2_OK) return rc;
-  launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.vis, T, pool_blocks, pool_out, k, topk_out,
-                nullptr, st);
+  launch_select(kSelPoolCand, ws.ckeys, int64_t(k) * kBlk, ws.vis, T, k, ws.topblk, k, topk_out, nullptr, st);
   return check_launch(fn);
 }
 
@@ -606,9 +613,10 @@ struct MultiWs {
   int32_t* n_groups;
   uint32_t* bkeys;
   uint32_t* ckeys;
+  int32_t* topblk;  // [Q][k]: the best k blocks of every pool
   size_t bytes;
 };
-MultiWs multi_ws(void* ws, int B, int Q, int64_t max_vis, int P) {
+MultiWs multi_ws(void* ws, int B, int Q, int64_t max_vis, int k) {
   Carve c(ws);
   MultiWs w;
   w.status = c.take<uint32_t>(kStatusBytes / 4);
@@ -617,7 +625,8 @@ MultiWs multi_ws(void* ws, int B, int Q, int64_t max_vis, int P) {
   w.groups = c.take<int4>(size_t(multi_group_bound(B, Q)));
   w.n_groups = c.take<int32_t>(1);
   w.bkeys = c.take<uint32_t>(size_t(Q) * size_t(block_key_stride(max_vis)));
-  w.ckeys = c.take<uint32_t>(size_t(Q) * P * kBlk);
+  w.ckeys = c.take<uint32_t>(size_t(Q) * k * kBlk);
+  w.topblk = c.take<int32_t>(size_t(Q) * k);
   w.bytes = c.used;
   return w;
 }
@@ -626,7 +635,7 @@ MultiWs multi_ws(void* ws, int B, int Q, int64_t max_vis, int P) {
 size_t csa2_index_multi_workspace_bytes(int B, int Q, int64_t max_vis, int pool_blocks, int k) {
   (void)k;
   if (B < 0 || Q < 0 || max_vis < 0 || pool_blocks < 0) return 0;
-  return multi_ws(nullptr, B, Q, max_vis, pool_blocks).bytes;
+  return multi_ws(nullptr, B, Q, max_vis, k).bytes;
 }
 
 csa2_status csa2_index_multi(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
@@ -648,7 +657,7 @@ csa2_status csa2_index_multi(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, con
   if (!aligned16(q_codes) || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
       (q_row_off_out && (reinterpret_cast<uintptr_t>(q_row_off_out) & 7)))
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": q_codes must be 16-byte and workspace 256-byte aligned");
-  MultiWs ws = multi_ws(workspace, B, Q, max_vis, pool_blocks);
+  MultiWs ws = multi_ws(workspace, B, Q, max_vis, k);
   if (workspace_bytes < ws.bytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int64_t* row_off = q_row_off_out ? q_row_off_out : ws.q_row_off;
@@ -657,15 +666,17 @@ csa2_status csa2_index_multi(csa2_mxfp4_cache idx_k, const uint8_t* q_codes, con
   launch_multi_prep(seq_row_off, q_off, q_vis, B, Q, G, max_vis, idx_k.rows, ws.groups, row_off, ws.vis,
                     ws.n_groups, ws.status, st);
   const csa2_status rc0 = launch_multi_tc(idx_k.codes, idx_k.scales, idx_k.rows, seq_row_off, ws.groups, G,
-                                          ws.n_groups, ws.vis, Q, max_vis, q_codes, q_scales, w, ws.bkeys, nb, ws.status, st);
+                                          ws.n_groups, ws.vis, Q, max_vis, q_codes, q_scales, w, ws.bkeys, nb,
+                                          ws.status, st);
   if (rc0 != CSA2_OK) return rc0;
-  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, Q, 0, nullptr, pool_blocks, pool_out, nullptr, st);
+  // the pool, the best k blocks among it, and the Top-k over their positions
+  launch_select(kSelBlockKeys, ws.bkeys, nb, ws.vis, Q, 0, nullptr, pool_blocks, pool_out, nullptr, st, ws.status,
+                ws.topblk, k);
   SegDesc sd{row_off, 0, ws.vis, max_vis, idx_k.rows};
-  const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.vis, Q, q_codes, q_scales, w, pool_out,
-                                        pool_blocks, ws.ckeys, nullptr, ws.status, st);
+  const csa2_status rc = launch_pool_tc(idx_k.codes, idx_k.scales, sd, ws.vis, Q, q_codes, q_scales, w, ws.topblk, k,
+                                        ws.ckeys, nullptr, ws.status, st);
   if (rc != CSA2_OK) return rc;
-  launch_select(kSelPoolCand, ws.ckeys, int64_t(pool_blocks) * kBlk, ws.vis, Q, pool_blocks, pool_out, k, topk_out,
-                nullptr, st);
+  launch_select(kSelPoolCand, ws.ckeys, int64_t(k) * kBlk, ws.vis, Q, k, ws.topblk, k, topk_out, nullptr, st);
   return check_launch(fn);
 }
 

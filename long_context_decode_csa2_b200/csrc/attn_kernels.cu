@@ -139,14 +139,29 @@ __device__ __forceinline__ int32_t chunk_tpos(const AttnArgs& a, int s, int c, i
   return idx < a.k ? __ldg(a.topk + int64_t(s) * a.k + idx) : -1;
 }
 
+// Segment facts every gather needs, read once per CTA: the checked visible
+// length and (contiguous layout) the first cache row.
+struct SegInfo {
+  int64_t eff;
+  int64_t row_base;  // -1 in the paged layout
+};
+
+__device__ __forceinline__ SegInfo seg_info(const AttnArgs& a, int s) {
+  SegInfo g;
+  g.eff = a.seg_eff ? int64_t(a.seg_eff[s]) : seg_len_checked(a.sd, s, a.status);
+  g.row_base = a.sd.pages ? int64_t(-1) : (a.sd.row_off ? a.sd.row_off[s] : a.sd.row0);
+  return g;
+}
+
 // Issues the cp.async copies of chunk c's rows into sm.raw (this thread: row
 // r = tid % 64, quarter tid / 64 of it) and returns whether row r is present.
-__device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, int s, int c, int32_t tpos) {
+__device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, int s, int c, int32_t tpos,
+                                             const SegInfo& g) {
   const int tid = threadIdx.x, r = tid & (kChunk - 1), qt = tid / kChunk;
   const ChunkSrc src = chunk_src(a, s, c);
   bool ok = r < src.nkeys;
   if (!src.is_win && ok) {
-    const int64_t eff = a.seg_eff ? int64_t(a.seg_eff[s]) : seg_len_checked(a.sd, s, a.status);
+    const int64_t eff = g.eff;
     if (tpos >= eff) {
       if (qt == 0) set_status(a.status, CSA2_DEV_INDEX_RANGE);
       ok = false;
@@ -156,7 +171,7 @@ __device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, in
   }
   if (ok) {
     if (!src.is_win) {
-      const int64_t row = seg_row(a.sd, s, tpos, a.status);
+      const int64_t row = g.row_base >= 0 ? g.row_base + tpos : seg_row(a.sd, s, tpos, a.status);
       const uint8_t* cs = a.mcodes + row * kMainCodeBytes + qt * (kMainCodeBytes / 4);
       uint8_t* dst = sm.raw.main[r] + qt * (kMainCodeBytes / 4);
 #pragma unroll
@@ -295,21 +310,23 @@ __device__ __forceinline__ void chunk_update(const AttnArgs& a, AttnSmem& sm, fl
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   // ---- S: warp w owns keys 8w .. 8w+7; two accumulators over alternate k-steps ----
-  float sa[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
+  // four independent accumulators over alternate k-steps (chains of 8 MMAs)
+  float sacc[4][4] = {};
   {
     const int kr = 8 * warp + (lane & 7);
     const int kc = 8 * ((lane >> 3) & 1);
     const int qr = (lane & 7) + 8 * ((lane >> 3) & 1);
     const int qc = 8 * (lane >> 4);
-#pragma unroll 4
-    for (int k0 = 0; k0 < kD; k0 += 32) {
-      uint32_t af[4], bf[2], af2[4], bf2[2];
-      ldsm_x4(af, &sm.q[qr][k0 + qc]);
-      ldsm_x2(bf, &sm.kv[kr][k0 + kc]);
-      ldsm_x4(af2, &sm.q[qr][k0 + 16 + qc]);
-      ldsm_x2(bf2, &sm.kv[kr][k0 + 16 + kc]);
-      mma16816(sa, af, bf[0], bf[1]);
-      mma16816(sb, af2, bf2[0], bf2[1]);
+#pragma unroll 2
+    for (int k0 = 0; k0 < kD; k0 += 64) {
+      uint32_t af[4][4], bf[4][2];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        ldsm_x4(af[u], &sm.q[qr][k0 + 16 * u + qc]);
+        ldsm_x2(bf[u], &sm.kv[kr][k0 + 16 * u + kc]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) mma16816(sacc[u], af[u], bf[u][0], bf[u][1]);
     }
   }
   // ---- logits, chunk maxima (per head) ----
@@ -319,7 +336,8 @@ __device__ __forceinline__ void chunk_update(const AttnArgs& a, AttnSmem& sm, fl
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int key = 8 * warp + 2 * t + (j & 1);
-    const float v = (key < nkeys && sm.valid[key]) ? (sa[j] + sb[j]) * lscale : -INFINITY;
+    const float v =
+        (key < nkeys && sm.valid[key]) ? ((sacc[0][j] + sacc[1][j]) + (sacc[2][j] + sacc[3][j])) * lscale : -INFINITY;
     sv[j] = v;
     mx[j >> 1] = fmaxf(mx[j >> 1], v);
   }
@@ -492,22 +510,29 @@ __device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm,
   float4 o[kOV];
 #pragma unroll
   for (int m = 0; m < kOV; ++m) o[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c = 0; c < nslots; ++c) {
-    float4 v[kOV];
-    float f[kOV];
+  // two slots per pass: both slots' loads are in flight together (slot
+  // order of the sums unchanged)
+  for (int c = 0; c < nslots; c += 2) {
+    float4 v[2][kOV];
+    float f[2][kOV];
 #pragma unroll
-    for (int m = 0; m < kOV; ++m) {
-      f[m] = sm.fac[c][(4 * (tid + m * kAttnThreads)) / kD];
-      v[m] = f[m] != 0.0f ? __ldcg(reinterpret_cast<const float4*>(base + c * kPartFloats) + tid + m * kAttnThreads)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-    for (int m = 0; m < kOV; ++m) {
-      o[m].x = fmaf(v[m].x, f[m], o[m].x);
-      o[m].y = fmaf(v[m].y, f[m], o[m].y);
-      o[m].z = fmaf(v[m].z, f[m], o[m].z);
-      o[m].w = fmaf(v[m].w, f[m], o[m].w);
-    }
+      for (int m = 0; m < kOV; ++m) {
+        f[u][m] = c + u < nslots ? sm.fac[c + u][(4 * (tid + m * kAttnThreads)) / kD] : 0.0f;
+        v[u][m] = f[u][m] != 0.0f
+                      ? __ldcg(reinterpret_cast<const float4*>(base + (c + u) * kPartFloats) + tid + m * kAttnThreads)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int m = 0; m < kOV; ++m) {
+        o[m].x = fmaf(v[u][m].x, f[u][m], o[m].x);
+        o[m].y = fmaf(v[u][m].y, f[u][m], o[m].y);
+        o[m].z = fmaf(v[u][m].z, f[u][m], o[m].z);
+        o[m].w = fmaf(v[u][m].w, f[u][m], o[m].w);
+      }
   }
 #pragma unroll
   for (int m = 0; m < kOV; ++m) reinterpret_cast<float4*>(a.out + int64_t(s) * kHq * kD)[tid + m * kAttnThreads] = o[m];
@@ -533,10 +558,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
     sm.l_run[tid] = 0.0f;
   }
   grid_wait();  // the Top-k ids, queries and rows may come from the previous kernel
+  const SegInfo sg = seg_info(a, s);
   bool ok = false;
   int32_t tnext = -1;
   if (c0 < c1) {
-    ok = issue_gather(a, sm, s, c0, chunk_tpos(a, s, c0, row));
+    ok = issue_gather(a, sm, s, c0, chunk_tpos(a, s, c0, row), sg);
     sm100::cp_async_commit();
     tnext = (c0 + 1 < c1) ? chunk_tpos(a, s, c0 + 1, row) : -1;
   }
@@ -558,7 +584,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
     dequant_chunk(a, sm, src.is_win, ok);
     __syncthreads();  // keys ready; the staging buffer is free
     if (c + 1 < c1) {
-      ok = issue_gather(a, sm, s, c + 1, tnext);
+      ok = issue_gather(a, sm, s, c + 1, tnext, sg);
       sm100::cp_async_commit();
       tnext = (c + 2 < c1) ? chunk_tpos(a, s, c + 2, row) : -1;
     }

@@ -322,16 +322,14 @@ __device__ void ordered_output_global(const void* in, int64_t base, int64_t n, u
   for (int j = int(nsel) + tid; j < k; j += kSelThreads) o[j] = -1;
 }
 
+// The selection of segment s = blockIdx.x (whole CTA); `dsm` is the dynamic
+// shared memory the launch gave.
 template <int KIND, bool SMALL>
-__global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restrict__ in, int64_t in_stride,
-                                                        const int32_t* __restrict__ seg_eff, int P,
-                                                        const int32_t* __restrict__ pool, int k,
-                                                        int32_t* __restrict__ out, uint32_t* __restrict__ ghist,
-                                                        uint32_t* __restrict__ status) {
-  extern __shared__ __align__(16) uint32_t dsm[];
-  __shared__ SelShared sh;
-  launch_dependents();
-  grid_wait();
+__device__ __forceinline__ void select_segment(const void* __restrict__ in, int64_t in_stride,
+                                               const int32_t* __restrict__ seg_eff, int P,
+                                               const int32_t* __restrict__ pool, int k, int32_t* __restrict__ out,
+                                               uint32_t* __restrict__ ghist, uint32_t* __restrict__ status,
+                                               uint32_t* dsm, SelShared& sh) {
   const int s = blockIdx.x;
   const int tid = threadIdx.x;
   int64_t n;
@@ -620,40 +618,176 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   }
 }
 
+// Adds one to hist[bin] for every active lane, one atomic per distinct bin of
+// the warp (the keys near the top of a pool share their high bits, so plain
+// shared atomics would serialise on a few bins).
+__device__ __forceinline__ void hist_add_warp(uint32_t* hist, uint32_t bin, bool active) {
+  const uint32_t am = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const uint32_t peers = __match_any_sync(am, bin);
+  if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
+}
+
+// After segment s's pool (`o`: n_pool <= 2048 block ids, ascending, then -1)
+// is written: its best `kb` blocks by (block key desc, id asc), ascending,
+// into tb (-1 padded).  Every one of the kb best positions lies in those
+// blocks: each block ranked before the block b of a selected position p
+// holds a position ranked before p (its own best; among equal keys the
+// lower block holds the lower position), which is then selected too, so
+// fewer than kb blocks rank before b.  The position Top-kb is therefore taken
+// from the 8 kb positions of these blocks instead of the whole pool's.
+// Radix digits of 8 bits start below the bits every pool key shares.
+__device__ __forceinline__ void top_blocks_of_pool(const uint32_t* __restrict__ keys, const int32_t* o, int n_pool,
+                                                   int kb, int32_t* __restrict__ tb, uint32_t* hist,
+                                                   SelShared& sh) {
+  __syncthreads();  // the pool written by every thread of the CTA is visible
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  uint32_t kk[2];
+  int32_t id[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {  // entries 2 tid, 2 tid + 1 (ids ascend with the entry)
+    const int i = 2 * tid + e;
+    id[e] = i < n_pool ? o[i] : -1;
+    kk[e] = id[e] >= 0 ? keys[id[e]] : 0u;
+  }
+  // present count, and the AND / OR of the present keys
+  uint32_t cnt = (kk[0] != 0u) + (kk[1] != 0u);
+  uint32_t kand = (kk[0] ? kk[0] : ~0u) & (kk[1] ? kk[1] : ~0u), kor = kk[0] | kk[1];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    kand &= __shfl_xor_sync(0xffffffffu, kand, off);
+    kor |= __shfl_xor_sync(0xffffffffu, kor, off);
+  }
+  uint32_t* wred = hist;  // 3 x 32 words, before the histogram uses them
+  if (lane == 0) {
+    wred[wid] = cnt;
+    wred[32 + wid] = kand;
+    wred[64 + wid] = kor;
+  }
+  __syncthreads();
+  uint32_t total = 0, all_and = ~0u, all_or = 0u;
+#pragma unroll 8
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    total += wred[w];
+    all_and &= wred[32 + w];
+    all_or |= wred[64 + w];
+  }
+  __syncthreads();  // wred is read by everyone before the histogram reuses it
+  uint32_t T = 0, rem = 0;
+  if (total > uint32_t(kb)) {
+    const uint32_t diff = all_and ^ all_or;  // bits on which the present keys differ
+    rem = uint32_t(kb);
+    if (diff == 0u) {
+      T = all_and;  // every present key equal: the lowest ids win
+    } else {
+      const int top = 31 - __clz(diff);
+      const uint32_t common = top == 31 ? 0u : ~((2u << top) - 1u);
+      uint32_t prefix = all_and & common, pmask = common;
+      for (int hi = top; hi >= 0; hi -= 8) {
+        const int width = min(8, hi + 1), shift = hi - width + 1;
+        const uint32_t dm = (1u << width) - 1u;
+        if (tid < 256) hist[tid] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          hist_add_warp(hist, (kk[e] >> shift) & dm, kk[e] != 0u && (kk[e] & pmask) == prefix);
+        __syncthreads();
+        find_bin(hist, 1 << width, rem, sh);
+        prefix |= sh.digit << shift;
+        pmask |= dm << shift;
+        rem = sh.rem;
+      }
+      T = prefix;
+    }
+  }
+  // ordered output: key > T, or key == T among the first rem (ids ascend with the entry)
+  uint32_t gt = 0, eq = 0;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    gt += (kk[e] > T);
+    eq += (kk[e] == T && kk[e] != 0u);
+  }
+  const uint32_t ex = block_exclusive_scan((gt << 16) | eq, sh.warp_sums, &sh.total);
+  const uint32_t tot = sh.total;
+  uint32_t g = ex >> 16, q = ex & 0xFFFFu;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    if (kk[e] > T) {
+      const uint32_t at = g + min(q, rem);
+      if (at < uint32_t(kb)) tb[at] = id[e];
+      ++g;
+    } else if (kk[e] == T && kk[e] != 0u) {
+      if (q < rem && g + q < uint32_t(kb)) tb[g + q] = id[e];
+      ++q;
+    }
+  }
+  const uint32_t nsel = (tot >> 16) + min(tot & 0xFFFFu, rem);
+  for (int j = int(nsel) + tid; j < kb; j += kSelThreads) tb[j] = -1;
+}
+
+// One CTA (1024 threads) per segment.  Block-key selections may also write
+// the best `kb` blocks of each pool into topblk [S][kb] (see
+// top_blocks_of_pool).
+template <int KIND, bool SMALL>
+__global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restrict__ in, int64_t in_stride,
+                                                        const int32_t* __restrict__ seg_eff, int P,
+                                                        const int32_t* __restrict__ pool, int k,
+                                                        int32_t* __restrict__ out, uint32_t* __restrict__ ghist,
+                                                        uint32_t* __restrict__ status, int32_t* __restrict__ topblk,
+                                                        int kb) {
+  extern __shared__ __align__(16) uint32_t dsm[];
+  __shared__ SelShared sh;
+  launch_dependents();
+  grid_wait();
+  select_segment<KIND, SMALL>(in, in_stride, seg_eff, P, pool, k, out, ghist, status, dsm, sh);
+  if (KIND == kSelBlockKeys && topblk != nullptr) {
+    const int s = blockIdx.x;
+    top_blocks_of_pool(static_cast<const uint32_t*>(in) + int64_t(s) * in_stride, out + int64_t(s) * k, k, kb,
+                       topblk + int64_t(s) * kb, dsm, sh);
+  }
+}
+
 template <int KIND>
 void launch_select_kind(const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P, const int32_t* pool,
-                        int k, int32_t* out, uint32_t* hist, int64_t n_bound, cudaStream_t st, uint32_t* status) {
+                        int k, int32_t* out, uint32_t* hist, int64_t n_bound, cudaStream_t st, uint32_t* status,
+                        int32_t* topblk, int kb) {
   if (n_bound <= kSelSmallMax) {
     constexpr int NB = (KIND == kSelPoolCand) ? kCandHistBins : kHist1Bins;
     const size_t smem = (hist ? NB + 1024 : 256) * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int((NB + 1024) * sizeof(uint32_t)));
     launch_k(k_select<KIND, true>, dim3(S), dim3(kSelThreads), smem, st, in, in_stride, seg_eff, P, pool, k, out, hist,
-             status);
+             status, topblk, kb);
   } else {
     const size_t smem = kSelLargeWords * sizeof(uint32_t);
     cudaFuncSetAttribute(k_select<KIND, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     launch_k(k_select<KIND, false>, dim3(S), dim3(kSelThreads), smem, st, in, in_stride, seg_eff, P, pool, k, out,
-             hist, status);
+             hist, status, topblk, kb);
   }
 }
 
 void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P,
-                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st, uint32_t* status) {
+                   const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st, uint32_t* status,
+                   int32_t* topblk, int kb) {
   if (S == 0) return;
   // n per segment is at most the row stride of the input
   switch (kind) {
     case kSelBlockKeys:
-      launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status);
+      launch_select_kind<kSelBlockKeys>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status, topblk,
+                                        kb);
       break;
     case kSelScores:
-      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status);
+      launch_select_kind<kSelScores>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status,
+                                     nullptr, 0);
       break;
     case kSelPoolCand:
-      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status);
+      launch_select_kind<kSelPoolCand>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status,
+                                       nullptr, 0);
       break;
     case kSelExplicit:
-      launch_select_kind<kSelExplicit>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status);
+      launch_select_kind<kSelExplicit>(in, in_stride, seg_eff, S, P, pool, k, out, hist, in_stride, st, status,
+                                       nullptr, 0);
       break;
   }
 }

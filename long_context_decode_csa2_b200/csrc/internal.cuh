@@ -162,9 +162,12 @@ enum SelectKind : int {
 // `hist` (or null): the keys' histogram rows, zeroed on return: [S][kSelHistBins]
 // for block keys, [S][kCandHistBins] for pool candidates.
 // `status` (or null): the workspace's status block (diagnostic counter).
+// Block-key selections (the pool, k = its size) may also write the best `kb`
+// blocks of every pool, ascending, into topblk [S][kb]: the blocks that hold
+// every one of the segment's kb best positions.
 void launch_select(SelectKind kind, const void* in, int64_t in_stride, const int32_t* seg_eff, int S, int P,
                    const int32_t* pool, int k, int32_t* out, uint32_t* hist, cudaStream_t st,
-                   uint32_t* status = nullptr);
+                   uint32_t* status = nullptr, int32_t* topblk = nullptr, int kb = 0);
 
 // Attention partials + combine.
 struct AttnArgs {

@@ -69,13 +69,17 @@ def measured_peaks():
 
 
 def algorithmic_bytes(wl, full_rescan=False):
-    """Per step, from the method's own reads (no scratch traffic):
-    Full scan L*68 B; each pool-scored layer min(16384, 8*ceil(L/8))*68 B
-    (the Full layer re-scores its pool for its own Top-512, each Reindex layer
-    scores the pool); each attention 512*272 + 128*512 B."""
+    """Per step, from the method's own reads (no scratch traffic): each
+    scanning Full layer L*68 B; each layer that selects inside the pool (a
+    Reindex layer, or a later Full layer under the pages' plan)
+    min(16384, 8*ceil(L/8))*68 B; each attention 512*272 + 128*512 B.  The
+    scanning Full layer's own Top-512, taken by re-scoring the positions of
+    its best 512 blocks (8*512*68 B per sequence), is an implementation step
+    and not counted."""
     L = wl.lengths.astype(np.int64)
     n_scan = sum(1 for _, m in enumerate(wl.pattern) if m == "F")
-    n_pool = sum(1 for m in wl.pattern if m in "FR")
+    # pool-scored layers: Reindex, and the Full layers after the first unless they rescan
+    n_pool = sum(1 for m in wl.pattern if m == "R") + (0 if full_rescan else max(0, n_scan - 1))
     # only the first Full layer scans (default plan); with full_rescan every one does
     scan = int((L * 68).sum()) * (n_scan if full_rescan else 1)
     # a verification step scores and attends per query, but reads each
@@ -555,8 +559,8 @@ def run_ours(args):
     ab = algorithmic_bytes(wl, args.full_rescan)
     peak, peak_kind = measured_peaks()
     full_avg = sum(full_ms) / len(full_ms)
-    full_bytes = (ab["scan"] // (ab["n_full"] if args.full_rescan else 1)
-                  + ab["pool"] // max(1, sum(1 for m in wl.pattern if m in "FR")))
+    # the dominant call's algorithmic bytes: its scan (one Full layer's)
+    full_bytes = ab["scan"] // (ab["n_full"] if args.full_rescan else 1)
     achieved = full_bytes / (full_avg * 1e-3) / 1e9
     traffic = None
     prof = os.path.join(ROOT, "profiles", "index_full_traffic.json")

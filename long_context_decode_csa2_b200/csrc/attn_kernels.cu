@@ -6,16 +6,25 @@
 // Work split: a segment's keys are chunks (ceil(k/64) chunks of 64 selected
 // rows, then four window chunks of 32 rows), and R CTAs share a segment, each
 // walking a contiguous run of its chunks (R = 2 x SMs / segments, at most 4:
-// two CTAs fit on an SM, and small batches still fill the GPU in one wave).  A CTA loads Q once,
-// keeps an online softmax (running max, sum and output per head) across its
-// chunks, and while it computes one chunk, cp.async brings the next chunk's
-// raw rows (272-byte MXFP4 rows or 512-byte E4M3 rows) into a staging
-// buffer; the Top-k ids are loaded one chunk earlier still.  Each chunk's
-// rows are dequantised exactly into fp16 in shared memory (E2M1 x 2^X and
-// raw E4M3 are exact in fp16 inside the range checked below), and both
-// products run on the tensor cores with warp-level mma (fp16 inputs, fp32
-// accumulation):
-//   S = Q K^T  (16 heads x 64 keys),  P = exp(S*scale - max),  O = P V.
+// two CTAs fit on an SM, and small batches still fill the GPU in one wave).
+// While a CTA computes one chunk, cp.async brings the next chunk's raw rows
+// (272-byte MXFP4 rows or 512-byte E4M3 rows) into the other half of a
+// double buffer; the Top-k ids are loaded one chunk earlier still.
+//
+// Both products run on the tensor cores with warp-level mma (fp16 inputs,
+// fp32 accumulation), and the rows are converted to fp16 once, in registers
+// (E2M1 x 2^X and E4M3 are exact in fp16 inside the range checked below):
+//   S = Q K^T  (16 heads x 64 keys): warp (h, q) takes the keys of half h
+//       and the 128 dims of quarter q, reads their raw bytes, converts them
+//       and keeps its Q fragments in registers for the whole kernel; the four
+//       quarters' partial scores meet in shared memory and are summed in a
+//       fixed order.  Inside each 32-dim scale block the reduction order of
+//       the dims is permuted so that a thread's 8 consecutive dims (one
+//       32-bit word of E2M1 codes) form its B fragments of two k-steps; Q
+//       uses the same permutation.  The converted rows go to shared memory.
+//   P = exp(S*scale - max), split into an fp16 head and an fp16 rest.
+//   O = P V: warp w owns dims 64w .. 64w+63 and reads V (the same rows)
+//       with transposing ldmatrix.
 // The window's fp32 scale multiplies its logits and its output in fp32, never
 // the fp16 values, so a CTA keeps the window chunks in a partial of their
 // own.  Each CTA writes its partials (O, max, sum per head); the last CTA of
@@ -33,7 +42,7 @@ namespace csa2 {
 constexpr int kChunk = 64;                         // keys per chunk
 constexpr int kAttnThreads = 256;                  // 8 warps
 constexpr int kPartFloats = kHq * kD + 2 * kHq;    // O, then m, then l
-constexpr int kQS = kD + 8;                        // smem row stride (halves) of Q and K
+constexpr int kQS = kD + 8;                        // smem row stride (halves) of the converted rows
 constexpr int kPS = kChunk + 8;                    // smem row stride (halves) of P
 constexpr int kWinRows = 32;                       // window rows per chunk (small staging buffer)
 constexpr int kWinChunks = kWin / kWinRows;        // 4
@@ -70,20 +79,24 @@ size_t attn_partial_bytes(int S, int k) {
   return size_t(S) * 2 * attn_splits(S, k) * kPartFloats * sizeof(float);
 }
 
+// Staged raw rows of one chunk.  Row strides of 68 and 132 words put the
+// rows a warp reads together on different banks.
+union RawRows {
+  uint8_t main[kChunk][kRawMain];
+  uint8_t win[kWinRows][kRawWin];
+};
+
 struct AttnSmem {
-  __half q[kHq][kQS];
-  __half kv[kChunk][kQS];
+  __half kv[kChunk][kQS];                // the chunk's rows in fp16
+  RawRows raw;                           // staged raw rows of the next chunk
+  float4 s_part[2][4][4][32];            // partial scores [key half][dim quarter][n-tile][lane]
   __half p[kHq][kPS];                    // softmax weights, fp16 head ...
   __half plo[kHq][kPS];                  // ... and the fp16 rest (p - head)
-  union {
-    uint8_t main[kChunk][kRawMain];
-    uint8_t win[kWinRows][kRawWin];
-  } raw;                                 // staged raw rows of the next chunk
   float red_max[8][kHq];
   float red_sum[8][kHq];
   float m_run[kHq];                      // online softmax state of the current part
   float l_run[kHq];
-  int valid[kChunk];
+  int valid[2][kChunk];                  // row present (this chunk's and the next one's)
   float fac[kMaxSlots][kHq];
   int last;
 };
@@ -154,8 +167,10 @@ __device__ __forceinline__ SegInfo seg_info(const AttnArgs& a, int s) {
 }
 
 // Issues the cp.async copies of chunk c's rows into sm.raw (this thread: row
-// r = tid % 64, quarter tid / 64 of it) and returns whether row r is present.
-__device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, int s, int c, int32_t tpos,
+// r = tid % 64, quarter tid / 64 of it) and records in sm.valid[vb] whether
+// row r is present.  An absent row is written as zeros (codes 0, unit scales), so
+// the products read exact zeros from it.
+__device__ __forceinline__ void issue_gather(const AttnArgs& a, AttnSmem& sm, int vb, int s, int c, int32_t tpos,
                                              const SegInfo& g) {
   const int tid = threadIdx.x, r = tid & (kChunk - 1), qt = tid / kChunk;
   const ChunkSrc src = chunk_src(a, s, c);
@@ -169,22 +184,35 @@ __device__ __forceinline__ bool issue_gather(const AttnArgs& a, AttnSmem& sm, in
       ok = false;
     }
   }
-  if (ok) {
-    if (!src.is_win) {
+  RawRows& rr = sm.raw;
+  if (!src.is_win) {
+    uint8_t* dst = rr.main[r] + qt * (kMainCodeBytes / 4);
+    if (ok) {
       const int64_t row = g.row_base >= 0 ? g.row_base + tpos : seg_row(a.sd, s, tpos, a.status);
       const uint8_t* cs = a.mcodes + row * kMainCodeBytes + qt * (kMainCodeBytes / 4);
-      uint8_t* dst = sm.raw.main[r] + qt * (kMainCodeBytes / 4);
 #pragma unroll
       for (int i = 0; i < kMainCodeBytes / 4 / 16; ++i) sm100::cp_async16(dst + 16 * i, cs + 16 * i);
-      if (qt == 0) sm100::cp_async16(sm.raw.main[r] + kMainCodeBytes, a.mscales + row * kMainScaleBytes);
-    } else {  // r < nkeys <= kWinRows
+      if (qt == 0) sm100::cp_async16(rr.main[r] + kMainCodeBytes, a.mscales + row * kMainScaleBytes);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kMainCodeBytes / 4 / 16; ++i) *reinterpret_cast<uint4*>(dst + 16 * i) = make_uint4(0, 0, 0, 0);
+      if (qt == 0)
+        *reinterpret_cast<uint4*>(rr.main[r] + kMainCodeBytes) =
+            make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+    }
+    if (qt == 0) sm.valid[vb][r] = ok;
+  } else if (r < kWinRows) {
+    uint8_t* dst = rr.win[r] + qt * (kD / 4);
+    if (ok) {
       const uint8_t* ws = src.win_base + int64_t(r) * kD + qt * (kD / 4);
-      uint8_t* dst = sm.raw.win[r] + qt * (kD / 4);
 #pragma unroll
       for (int i = 0; i < kD / 4 / 16; ++i) sm100::cp_async16(dst + 16 * i, ws + 16 * i);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kD / 4 / 16; ++i) *reinterpret_cast<uint4*>(dst + 16 * i) = make_uint4(0, 0, 0, 0);
     }
+    if (qt == 0) sm.valid[vb][r] = ok;
   }
-  return ok;
 }
 
 // Two E2M1 codes (low nibble = lower element) -> f16x2, exact.
@@ -212,11 +240,6 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
 }
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
-}
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
@@ -225,119 +248,163 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Q of segment s: bf16 -> fp16 into sm.q (exact for |q| in [2^-14, 65504];
-// smaller values keep 2^-24 resolution).
-__device__ __forceinline__ void load_q(const AttnArgs& a, AttnSmem& sm, int s) {
-  const int tid = threadIdx.x;
-  constexpr int kQV = kHq * kD / 8 / kAttnThreads;  // 16-byte vectors per thread (4)
-  uint4 qv[kQV];
-  const uint4* qsrc = reinterpret_cast<const uint4*>(a.q + int64_t(s) * kHq * kD);
-#pragma unroll
-  for (int m = 0; m < kQV; ++m) qv[m] = __ldg(qsrc + tid + m * kAttnThreads);
-#pragma unroll
-  for (int m = 0; m < kQV; ++m) {
-    const int e = 8 * (tid + m * kAttnThreads);
-    const int h = e / kD, d = e % kD;
-    const uint32_t w[4] = {qv[m].x, qv[m].y, qv[m].z, qv[m].w};
-    uint32_t o[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
-      if (fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f) set_status(a.status, CSA2_DEV_FP16_RANGE);
-      const __half2 h2 = __floats2half2_rn(lo, hi);
-      o[q] = *reinterpret_cast<const uint32_t*>(&h2);
-    }
-    *reinterpret_cast<uint4*>(&sm.q[h][d]) = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-}
-
-// Staged raw rows -> fp16 keys in sm.kv (absent rows as zeros) and the
-// row-valid flags.  Thread: row r = tid % 64, blocks tid/64 + 4i.
-__device__ __forceinline__ void dequant_chunk(const AttnArgs& a, AttnSmem& sm, bool is_win, bool row_ok) {
-  const int tid = threadIdx.x;
-  const int r = tid & (kChunk - 1);
-  constexpr int kBPT = 16 / (kAttnThreads / kChunk);  // blocks per thread (4)
-  const int b0 = tid / kChunk;
-  if (b0 == 0) sm.valid[r] = row_ok;
-#pragma unroll
-  for (int i = 0; i < kBPT; ++i) {
-    const int b = b0 + 4 * i;
-    uint4* dst = reinterpret_cast<uint4*>(&sm.kv[r][32 * b]);
-    if (!row_ok) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
-      continue;
-    }
-    if (!is_win) {
-      // fp16-exact iff the block exponent X = byte - 127 lies in [-23, 13]
-      const uint4 cw = *reinterpret_cast<const uint4*>(sm.raw.main[r] + 16 * b);
-      const uint32_t sb = sm.raw.main[r][kMainCodeBytes + b];
-      if (sb < 104u || sb > 140u) set_status(a.status, CSA2_DEV_FP16_RANGE);
-      const int X = int(sb) - 127;
-      const uint16_t xb = X >= -14 ? uint16_t((X + 15) << 10) : uint16_t(1u << (X + 24 > 0 ? X + 24 : 0));
-      const uint32_t sc2 = uint32_t(xb) | (uint32_t(xb) << 16);
-      const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t hv[4];
-#pragma unroll
-        for (int n = 0; n < 4; ++n) hv[n] = hmul2_u32(cvt_e2m1x2((w4[q] >> (8 * n)) & 255u), sc2);
-        dst[q] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-      }
-    } else {
-      const uint4 v0 = *reinterpret_cast<const uint4*>(sm.raw.win[r] + 32 * b);
-      const uint4 v1 = *reinterpret_cast<const uint4*>(sm.raw.win[r] + 32 * b + 16);
-      const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        dst[q] = make_uint4(cvt_e4m3x2(w8[2 * q] & 0xFFFFu), cvt_e4m3x2(w8[2 * q] >> 16),
-                            cvt_e4m3x2(w8[2 * q + 1] & 0xFFFFu), cvt_e4m3x2(w8[2 * q + 1] >> 16));
-    }
-  }
-}
-
-__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
 }
 
-// One chunk (keys in sm.kv) into the running softmax state: S = Q K^T for the
-// chunk's keys, the running max / sum per head (sm.m_run, sm.l_run) and the
-// output accumulator oacc (warp w: dims 64w .. 64w+63, rows g and g+8).
-__device__ __forceinline__ void chunk_update(const AttnArgs& a, AttnSmem& sm, float (&oacc)[8][4], int nkeys,
-                                             float kscale) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  // ---- S: warp w owns keys 8w .. 8w+7; two accumulators over alternate k-steps ----
-  // four independent accumulators over alternate k-steps (chains of 8 MMAs)
+// 2^X as an fp16 pair for an E8M0 scale byte (X = byte - 127); exact for X in
+// [-24, 15].
+__device__ __forceinline__ uint32_t e8m0_f16x2(uint32_t sb) {
+  const int X = int(sb) - 127;
+  const uint16_t xb = X >= -14 ? uint16_t((X + 15) << 10) : uint16_t(1u << (X + 24 > 0 ? X + 24 : 0));
+  return uint32_t(xb) | (uint32_t(xb) << 16);
+}
+
+// One 32-bit word of E2M1 codes (8 consecutive dims) times its block scale:
+// f[m] = dims 2m, 2m+1 of the word.
+__device__ __forceinline__ void conv_fp4_word(uint32_t w, uint32_t sc2, uint32_t (&f)[4]) {
+#pragma unroll
+  for (int m = 0; m < 4; ++m) f[m] = hmul2_u32(cvt_e2m1x2((w >> (8 * m)) & 255u), sc2);
+}
+// Eight consecutive E4M3 bytes: f[m] = dims 2m, 2m+1.
+__device__ __forceinline__ void conv_e4m3_pair(uint2 v, uint32_t (&f)[4]) {
+  f[0] = cvt_e4m3x2(v.x & 0xFFFFu);
+  f[1] = cvt_e4m3x2(v.x >> 16);
+  f[2] = cvt_e4m3x2(v.y & 0xFFFFu);
+  f[3] = cvt_e4m3x2(v.y >> 16);
+}
+
+// This thread's Q fragments (lane = 4g + t): for each of the warp's four
+// scale blocks (dims 32(4q + j) ..), dims 8t .. 8t+7 of heads g (qa) and g+8
+// (qb) as fp16 pairs.  bf16 -> fp16 is exact for |q| in [2^-14, 65504];
+// smaller values keep 2^-24 resolution.
+struct QFrag {
+  uint4 qa[4], qb[4];
+};
+
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v, uint32_t* status) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
+    if (fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f) set_status(status, CSA2_DEV_FP16_RANGE);
+    const __half2 h2 = __floats2half2_rn(lo, hi);
+    o[q] = *reinterpret_cast<const uint32_t*>(&h2);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void load_q_frag(const AttnArgs& a, int s, int quarter, QFrag& qf) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const uint16_t* qs = a.q + int64_t(s) * kHq * kD;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int d = 32 * (4 * quarter + j) + 8 * t;
+    qf.qa[j] = __ldg(reinterpret_cast<const uint4*>(qs + g * kD + d));
+    qf.qb[j] = __ldg(reinterpret_cast<const uint4*>(qs + (g + 8) * kD + d));
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    qf.qa[j] = bf16x8_to_f16x8(qf.qa[j], a.status);
+    qf.qb[j] = bf16x8_to_f16x8(qf.qb[j], a.status);
+  }
+}
+
+// Partial scores of one chunk: warp (h, q) = (warp / 4, warp % 4) computes
+// S over dims of quarter q for the 32 keys of half h (4 n-tiles) and leaves
+// them in sm.s_part; the converted rows go to sm.kv.  For k-step (j, e) of
+// block j, the thread's B fragment is (dims 4e, 4e+1 | 4e+2, 4e+3 of its
+// word) and its A fragment the same dims of Q, so the k order inside the
+// block is a permutation of the dims.
+__device__ __forceinline__ void qk_partial(const AttnArgs& a, AttnSmem& sm, bool is_win, int nkeys,
+                                           const QFrag& qf) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3, kh = warp >> 2, dq = warp & 3;
+  if (32 * kh >= nkeys) return;  // (window chunks) no keys in this half
+  const RawRows& rr = sm.raw;
   float sacc[4][4] = {};
-  {
-    const int kr = 8 * warp + (lane & 7);
-    const int kc = 8 * ((lane >> 3) & 1);
-    const int qr = (lane & 7) + 8 * ((lane >> 3) & 1);
-    const int qc = 8 * (lane >> 4);
-#pragma unroll 2
-    for (int k0 = 0; k0 < kD; k0 += 64) {
-      uint32_t af[4][4], bf[4][2];
+  if (!is_win) {
+    uint32_t wd[4][4], sw[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        ldsm_x4(af[u], &sm.q[qr][k0 + 16 * u + qc]);
-        ldsm_x2(bf[u], &sm.kv[kr][k0 + 16 * u + kc]);
+    for (int nt = 0; nt < 4; ++nt) {
+      const uint8_t* row = rr.main[32 * kh + 8 * nt + g];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wd[nt][j] = *reinterpret_cast<const uint32_t*>(row + 16 * (4 * dq + j) + 4 * t);
+      sw[nt] = *reinterpret_cast<const uint32_t*>(row + kMainCodeBytes + 4 * dq);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t sb = (sw[nt] >> (8 * j)) & 255u;
+        // fp16-exact iff the block exponent X = byte - 127 lies in [-23, 13]
+        if (t == 0 && (sb < 104u || sb > 140u)) set_status(a.status, CSA2_DEV_FP16_RANGE);
       }
+    }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) mma16816(sacc[u], af[u], bf[u][0], bf[u][1]);
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t qa0[4] = {qf.qa[j].x, qf.qb[j].x, qf.qa[j].y, qf.qb[j].y};
+      const uint32_t qa1[4] = {qf.qa[j].z, qf.qb[j].z, qf.qa[j].w, qf.qb[j].w};
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        uint32_t f[4];
+        conv_fp4_word(wd[nt][j], e8m0_f16x2((sw[nt] >> (8 * j)) & 255u), f);
+        mma16816(sacc[nt], qa0, f[0], f[1]);
+        mma16816(sacc[nt], qa1, f[2], f[3]);
+        *reinterpret_cast<uint4*>(&sm.kv[32 * kh + 8 * nt + g][32 * (4 * dq + j) + 8 * t]) =
+            make_uint4(f[0], f[1], f[2], f[3]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t qa0[4] = {qf.qa[j].x, qf.qb[j].x, qf.qa[j].y, qf.qb[j].y};
+      const uint32_t qa1[4] = {qf.qa[j].z, qf.qb[j].z, qf.qa[j].w, qf.qb[j].w};
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const uint8_t* row = rr.win[32 * kh + 8 * nt + g];
+        uint32_t f[4];
+        conv_e4m3_pair(*reinterpret_cast<const uint2*>(row + 32 * (4 * dq + j) + 8 * t), f);
+        mma16816(sacc[nt], qa0, f[0], f[1]);
+        mma16816(sacc[nt], qa1, f[2], f[3]);
+        *reinterpret_cast<uint4*>(&sm.kv[32 * kh + 8 * nt + g][32 * (4 * dq + j) + 8 * t]) =
+            make_uint4(f[0], f[1], f[2], f[3]);
+      }
     }
   }
-  // ---- logits, chunk maxima (per head) ----
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) sm.s_part[kh][dq][nt][lane] = make_float4(sacc[nt][0], sacc[nt][1], sacc[nt][2], sacc[nt][3]);
+}
+
+// The rest of one chunk (partial scores in sm.s_part, rows in sm.kv): the
+// running max / sum per head (sm.m_run, sm.l_run) and the output accumulator
+// oacc (warp w: dims 64w .. 64w+63, heads g and g+8 of lane 4g + t).
+__device__ __forceinline__ void softmax_pv(const AttnArgs& a, AttnSmem& sm, int vb, float (&oacc)[8][4], int nkeys,
+                                           float kscale) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  // ---- S of keys 8w .. 8w+7: the four quarters in order, then the chunk maxima ----
+  float sacc[4];
+  {
+    const int kh = warp >> 2, nt = warp & 3;
+    float4 v = sm.s_part[kh][0][nt][lane];
+#pragma unroll
+    for (int q = 1; q < 4; ++q) {
+      const float4 u = sm.s_part[kh][q][nt][lane];
+      v.x += u.x, v.y += u.y, v.z += u.z, v.w += u.w;
+    }
+    sacc[0] = v.x, sacc[1] = v.y, sacc[2] = v.z, sacc[3] = v.w;
+  }
   const float lscale = a.sm_scale * kscale;
   float sv[4];
   float mx[2] = {-INFINITY, -INFINITY};  // heads g, g+8
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int key = 8 * warp + 2 * t + (j & 1);
-    const float v =
-        (key < nkeys && sm.valid[key]) ? ((sacc[0][j] + sacc[1][j]) + (sacc[2][j] + sacc[3][j])) * lscale : -INFINITY;
+    const float v = (key < nkeys && sm.valid[vb][key]) ? sacc[j] * lscale : -INFINITY;
     sv[j] = v;
     mx[j >> 1] = fmaxf(mx[j >> 1], v);
   }
@@ -559,17 +626,18 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
   }
   grid_wait();  // the Top-k ids, queries and rows may come from the previous kernel
   const SegInfo sg = seg_info(a, s);
-  bool ok = false;
   int32_t tnext = -1;
   if (c0 < c1) {
-    ok = issue_gather(a, sm, s, c0, chunk_tpos(a, s, c0, row), sg);
+    issue_gather(a, sm, 0, s, c0, chunk_tpos(a, s, c0, row), sg);
     sm100::cp_async_commit();
     tnext = (c0 + 1 < c1) ? chunk_tpos(a, s, c0 + 1, row) : -1;
   }
-  load_q(a, sm, s);  // overlaps the first gather
+  QFrag qf;
+  load_q_frag(a, s, (tid >> 5) & 3, qf);  // overlaps the first gather
   bool in_win = false, wrote_main = false;
   float win_scale = 1.0f;
   for (int c = c0; c < c1; ++c) {
+    const int vb = (c - c0) & 1;
     const ChunkSrc src = chunk_src(a, s, c);
     if (src.is_win && !in_win) {
       if (c > c0) {  // this CTA's selected rows are done: their partial
@@ -580,15 +648,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
       win_scale = src.kscale;
     }
     sm100::cp_async_wait<0>();
-    __syncthreads();  // this chunk's rows (and Q) are in shared memory
-    dequant_chunk(a, sm, src.is_win, ok);
-    __syncthreads();  // keys ready; the staging buffer is free
+    __syncthreads();  // this chunk's rows are staged; the last chunk's P V is done
+    qk_partial(a, sm, src.is_win, src.nkeys, qf);
+    __syncthreads();  // converted rows and partial scores written; the staging buffer is free
     if (c + 1 < c1) {
-      ok = issue_gather(a, sm, s, c + 1, tnext, sg);
+      issue_gather(a, sm, vb ^ 1, s, c + 1, tnext, sg);
       sm100::cp_async_commit();
       tnext = (c + 2 < c1) ? chunk_tpos(a, s, c + 2, row) : -1;
     }
-    chunk_update(a, sm, oacc, src.nkeys, src.kscale);
+    softmax_pv(a, sm, vb, oacc, src.nkeys, src.kscale);
   }
   if (in_win) {
     flush_part(a, sm, oacc, s, nslots, 2 * r + 1, win_scale);

@@ -7,6 +7,7 @@
 // sparse indexer, 8-position blocks ranked by their maximum, pool of at most
 // 2048 blocks, Top-512 per layer, FP4 indexer q/k).
 #include "device_common.cuh"
+#include "sm100.cuh"
 
 namespace csa2 {
 
@@ -55,6 +56,11 @@ void launch_prefill_vis(const int32_t* q_pos, int T, int ratio, int64_t n_entrie
 //     into the output without another pass over the keys.  A bucket with more
 //     than 12288 keys falls back to global radix passes and an ordered output
 //     pass.
+//   * large n from a producer's histogram, few segments: a cluster of two
+//     CTAs per segment.  CTA 0 takes the histogram and finds the threshold
+//     bucket, and sends it to CTA 1; each CTA collects the lists of one half
+//     of the key chunks; CTA 1 writes its lists behind CTA 0's (their total
+//     lengths follow from the histogram) and CTA 0 finishes alone.
 // Output rule: key > T, or key == T among the first `rem` equal keys in
 // index order; ids leave in ascending order.
 // ---------------------------------------------------------------------------
@@ -115,6 +121,7 @@ struct SelShared {
   uint32_t digit, rem;
   int sel_warp;         // find_bin: the warp whose bin range holds the threshold
   uint32_t sel_before;  // and the count above that range
+  uint32_t xfer[6];     // cluster: (total, bucket, need, count) to CTA 1, (na, nc) to CTA 0
 };
 
 // Block-wide exclusive scan of one uint32 per thread; returns the exclusive
@@ -322,15 +329,18 @@ __device__ void ordered_output_global(const void* in, int64_t base, int64_t n, u
   for (int j = int(nsel) + tid; j < k; j += kSelThreads) o[j] = -1;
 }
 
-// The selection of segment s = blockIdx.x (whole CTA); `dsm` is the dynamic
-// shared memory the launch gave.
-template <int KIND, bool SMALL>
+// The selection of segment s = blockIdx.x / CL (whole CTA, or with CL = 2
+// the two CTAs of a cluster, large path with a producer histogram only);
+// `dsm` is the dynamic shared memory the launch gave.
+template <int KIND, bool SMALL, int CL>
 __device__ __forceinline__ void select_segment(const void* __restrict__ in, int64_t in_stride,
                                                const int32_t* __restrict__ seg_eff, int P,
                                                const int32_t* __restrict__ pool, int k, int32_t* __restrict__ out,
                                                uint32_t* __restrict__ ghist, uint32_t* __restrict__ status,
                                                uint32_t* dsm, SelShared& sh) {
-  const int s = blockIdx.x;
+  static_assert(CL == 1 || (CL == 2 && !SMALL), "clusters serve the large path only");
+  const int s = blockIdx.x / CL;
+  const uint32_t rank = CL == 1 ? 0u : sm100::cluster_ctarank();
   const int tid = threadIdx.x;
   int64_t n;
   if (KIND == kSelBlockKeys) n = (int64_t(seg_eff[s]) + kBlk - 1) / kBlk;
@@ -435,7 +445,34 @@ __device__ __forceinline__ void select_segment(const void* __restrict__ in, int6
   // ---- large n, pass A: 15-bit histogram of the present keys ----
   uint32_t* hist = dsm;
   uint32_t present = 0;
-  if (ghist) {
+  uint32_t total = 0, b1 = 0, need = 0, cnt = 0;
+  if (CL == 2) {
+    // CTA 0 finds the threshold bucket from the producer's histogram and
+    // sends it to CTA 1 (ghist is non-null whenever CL == 2)
+    if (rank == 0) {
+      present = take_hist<kHist1Bins>(ghist + int64_t(s) * kHist1Bins, hist);
+      __syncthreads();
+      block_exclusive_scan(present, sh.warp_sums, &sh.total);
+      total = sh.total;
+      if (total > uint32_t(k)) {
+        find_bin(hist, kHist1Bins, uint32_t(k), sh);
+        b1 = sh.digit;
+        need = sh.rem;
+        cnt = hist[b1];
+      }
+      if (tid < 4) {
+        const uint32_t v = tid == 0 ? total : tid == 1 ? b1 : tid == 2 ? need : cnt;
+        sm100::st_cluster_u32(sm100::mapa_shared(sm100::smem_u32(&sh.xfer[tid]), 1), v);
+      }
+    }
+    sm100::cluster_sync();
+    if (rank == 1) {
+      total = sh.xfer[0];
+      b1 = sh.xfer[1];
+      need = sh.xfer[2];
+      cnt = sh.xfer[3];
+    }
+  } else if (ghist) {
     present = take_hist<kHist1Bins>(ghist + int64_t(s) * kHist1Bins, hist);
   } else {
     for (int i = tid; i < kHist1Bins; i += kSelThreads) hist[i] = 0;
@@ -453,20 +490,22 @@ __device__ __forceinline__ void select_segment(const void* __restrict__ in, int6
       for (int e = 0; e < kSelPer; ++e) kk[e] = nx[e];
     }
   }
-  __syncthreads();
-  block_exclusive_scan(present, sh.warp_sums, &sh.total);
-  const uint32_t total = sh.total;
-  const bool all = total <= uint32_t(k);
-  uint32_t b1 = 0, need = 0, cnt = 0;
-  if (!all) {
-    find_bin(hist, kHist1Bins, uint32_t(k), sh);
-    b1 = sh.digit;
-    need = sh.rem;
-    cnt = hist[b1];
+  if (CL == 1) {
+    __syncthreads();
+    block_exclusive_scan(present, sh.warp_sums, &sh.total);
+    total = sh.total;
+    if (total > uint32_t(k)) {
+      find_bin(hist, kHist1Bins, uint32_t(k), sh);
+      b1 = sh.digit;
+      need = sh.rem;
+      cnt = hist[b1];
+    }
   }
+  const bool all = total <= uint32_t(k);
   __syncthreads();  // the histogram's memory is reused below
 
   if (!all && cnt > uint32_t(kCandCap)) {
+    if (rank != 0) return;  // (both CTAs of a cluster decide alike; no cluster barrier follows)
     // more than kCandCap keys share the threshold bucket: global radix passes
     // over the low 17 bits (9 + 8), then an ordered pass over the keys
     if (status && tid == 0) atomicAdd(status + kDiagOverfull, 1u);
@@ -504,10 +543,17 @@ __device__ __forceinline__ void select_segment(const void* __restrict__ in, int6
   uint32_t* Csel = h2 + 512;             // [kSelMaxK] selected bucket ids
   uint32_t run_a = 0, run_c = 0;
   {
+    // this CTA's keys: all, or (cluster) one half of the chunks
+    int64_t lo = 0, hi = n;
+    if (CL == 2) {
+      const int64_t half = (n + 2 * kSelChunk - 1) / (2 * kSelChunk) * kSelChunk;
+      lo = rank == 0 ? 0 : half;
+      hi = rank == 0 ? (half < n ? half : n) : n;
+    }
     uint32_t kk[kSelPer], nx[kSelPer];
-    load_keys<KIND>(in, base, int64_t(tid) * kSelPer, n, kk);
-    for (int64_t c0 = 0; c0 < n; c0 += kSelChunk) {
-      if (c0 + kSelChunk < n) load_keys<KIND>(in, base, c0 + kSelChunk + int64_t(tid) * kSelPer, n, nx);
+    load_keys<KIND>(in, base, lo + int64_t(tid) * kSelPer, hi, kk);
+    for (int64_t c0 = lo; c0 < hi; c0 += kSelChunk) {
+      if (c0 + kSelChunk < hi) load_keys<KIND>(in, base, c0 + kSelChunk + int64_t(tid) * kSelPer, hi, nx);
       // most threads hold no key at or above the bucket: one max decides
       uint32_t mx = 0;
 #pragma unroll
@@ -551,6 +597,31 @@ __device__ __forceinline__ void select_segment(const void* __restrict__ in, int6
     }
   }
   __syncthreads();
+  if (CL == 2) {
+    // CTA 1's lists go behind CTA 0's: the histogram fixes both totals
+    const uint32_t na_tot = all ? total : uint32_t(k) - need, nc_tot = all ? 0u : cnt;
+    if (rank == 1) {
+      const uint32_t a_off = na_tot - min(run_a, na_tot), c_off = nc_tot - min(run_c, nc_tot);
+      for (uint32_t i = tid; i < run_a && a_off + i < uint32_t(kSelMaxK); i += kSelThreads)
+        sm100::st_cluster_u32(sm100::mapa_shared(sm100::smem_u32(&A[a_off + i]), 0), A[i]);
+      for (uint32_t i = tid; i < run_c && c_off + i < uint32_t(kCandCap); i += kSelThreads) {
+        sm100::st_cluster_u32(sm100::mapa_shared(sm100::smem_u32(&Clow[c_off + i]), 0), Clow[i]);
+        sm100::st_cluster_u32(sm100::mapa_shared(sm100::smem_u32(&Cidx[c_off + i]), 0), Cidx[i]);
+      }
+      if (tid < 2) sm100::st_cluster_u32(sm100::mapa_shared(sm100::smem_u32(&sh.xfer[4 + tid]), 0),
+                                         tid == 0 ? run_a : run_c);
+    }
+    sm100::cluster_sync();
+    if (rank == 1) return;
+    // the halves' lengths disagree with the histogram only after a producer
+    // failure that already set a flag: no pool then
+    if (run_a + sh.xfer[4] != na_tot || run_c + sh.xfer[5] != nc_tot || na_tot > uint32_t(kSelMaxK)) {
+      for (int j = tid; j < k; j += kSelThreads) o[j] = -1;
+      return;
+    }
+    run_a = na_tot;
+    run_c = nc_tot;
+  }
   // (the list lengths only exceed their capacities if the histogram and the
   // keys disagree, i.e. after a producer failure that already set a flag)
   run_a = min(run_a, uint32_t(kSelMaxK));
@@ -726,10 +797,10 @@ __device__ __forceinline__ void top_blocks_of_pool(const uint32_t* __restrict__ 
   for (int j = int(nsel) + tid; j < kb; j += kSelThreads) tb[j] = -1;
 }
 
-// One CTA (1024 threads) per segment.  Block-key selections may also write
-// the best `kb` blocks of each pool into topblk [S][kb] (see
-// top_blocks_of_pool).
-template <int KIND, bool SMALL>
+// One CTA (1024 threads) per segment, or a cluster of CL = 2.  Block-key
+// selections may also write the best `kb` blocks of each pool into topblk
+// [S][kb] (see top_blocks_of_pool).
+template <int KIND, bool SMALL, int CL>
 __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restrict__ in, int64_t in_stride,
                                                         const int32_t* __restrict__ seg_eff, int P,
                                                         const int32_t* __restrict__ pool, int k,
@@ -740,9 +811,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_select(const void* __restric
   __shared__ SelShared sh;
   launch_dependents();
   grid_wait();
-  select_segment<KIND, SMALL>(in, in_stride, seg_eff, P, pool, k, out, ghist, status, dsm, sh);
-  if (KIND == kSelBlockKeys && topblk != nullptr) {
-    const int s = blockIdx.x;
+  select_segment<KIND, SMALL, CL>(in, in_stride, seg_eff, P, pool, k, out, ghist, status, dsm, sh);
+  if (KIND == kSelBlockKeys && topblk != nullptr && (CL == 1 || sm100::cluster_ctarank() == 0)) {
+    const int s = blockIdx.x / CL;
     top_blocks_of_pool(static_cast<const uint32_t*>(in) + int64_t(s) * in_stride, out + int64_t(s) * k, k, kb,
                        topblk + int64_t(s) * kb, dsm, sh);
   }
@@ -755,14 +826,20 @@ void launch_select_kind(const void* in, int64_t in_stride, const int32_t* seg_ef
   if (n_bound <= kSelSmallMax) {
     constexpr int NB = (KIND == kSelPoolCand) ? kCandHistBins : kHist1Bins;
     const size_t smem = (hist ? NB + 1024 : 256) * sizeof(uint32_t);
-    cudaFuncSetAttribute(k_select<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(k_select<KIND, true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int((NB + 1024) * sizeof(uint32_t)));
-    launch_k(k_select<KIND, true>, dim3(S), dim3(kSelThreads), smem, st, in, in_stride, seg_eff, P, pool, k, out, hist,
-             status, topblk, kb);
+    launch_k(k_select<KIND, true, 1>, dim3(S), dim3(kSelThreads), smem, st, in, in_stride, seg_eff, P, pool, k, out,
+             hist, status, topblk, kb);
+  } else if (hist != nullptr && 2 * int64_t(S) <= num_sms()) {
+    // few segments: two CTAs (SMs) each, still one wave
+    const size_t smem = kSelLargeWords * sizeof(uint32_t);
+    cudaFuncSetAttribute(k_select<KIND, false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    launch_k_cluster(k_select<KIND, false, 2>, dim3(2 * S), dim3(kSelThreads), smem, st, 2, in, in_stride, seg_eff, P,
+                     pool, k, out, hist, status, topblk, kb);
   } else {
     const size_t smem = kSelLargeWords * sizeof(uint32_t);
-    cudaFuncSetAttribute(k_select<KIND, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    launch_k(k_select<KIND, false>, dim3(S), dim3(kSelThreads), smem, st, in, in_stride, seg_eff, P, pool, k, out,
+    cudaFuncSetAttribute(k_select<KIND, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    launch_k(k_select<KIND, false, 1>, dim3(S), dim3(kSelThreads), smem, st, in, in_stride, seg_eff, P, pool, k, out,
              hist, status, topblk, kb);
   }
 }

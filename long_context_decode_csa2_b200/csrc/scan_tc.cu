@@ -55,17 +55,12 @@ constexpr int kAcc = 3;                // TMEM accumulator ring (16 columns per 
 constexpr int kAccCols = 16 * kMT;
 constexpr int kTmemCols = 256;
 constexpr uint32_t kSfCol = 192;       // scale factors (all 0x7F = 2^0) live here
-// epilogue teams of 4 warps, items round-robin: the scan's rate is set by its
-// epilogue, so it gets three; the pool gather's extra producer warps leave
-// registers for two
-template <bool kPool>
-__host__ __device__ constexpr int epi_teams() { return kPool ? 2 : 3; }
-template <bool kPool>
-__host__ __device__ constexpr int first_extra() { return 2 + 4 * epi_teams<kPool>(); }  // first extra producer warp (pool mode)
+constexpr int kEpiTeams = 2;           // epilogue teams of 4 warps, items round-robin
+constexpr int kFirstExtra = 2 + 4 * kEpiTeams;  // first extra producer warp (pool mode)
 constexpr int kPoolProducers = 4;      // pool mode: warps sharing the gather of an item
 template <bool kPool>
 constexpr int threads_of() {           // producer, MMA, epilogue (+ extra producer) warps
-  return 32 * (first_extra<kPool>() + (kPool ? kPoolProducers - 1 : 0));
+  return 32 * (kFirstExtra + (kPool ? kPoolProducers - 1 : 0));
 }
 constexpr uint32_t kCodeBytes = kTile * kIdxCodeBytes;
 constexpr int kBoxRows = 256;          // TMA box height (scan)
@@ -218,7 +213,6 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
   const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
   const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
 
-  constexpr int kEpiTeams = epi_teams<kPool>(), kFirstExtra = first_extra<kPool>();
   if (warp == 0 || warp >= kFirstExtra) {
     // ------------------------------------------------------------ producer(s)
     // pool mode: warp 0 and the extra warps each gather kSlotsPerWarp blocks of

@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="long_decode_b64_l1m")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--groups", type=lambda v: [int(x) for x in v.split(",") if x], default=[2, 4],
+                    help="group counts of the grouped layer-order step also timed (comma list; empty: none)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling captures)")
     ap.add_argument("--no-graph", action="store_true",
@@ -447,10 +449,9 @@ def run_ours(args):
     # the same step with every call in layer order on one stream (the order a
     # model whose layer inputs depend on the previous layer would impose),
     # also replayed from a graph
-    seq_ms = None
-    if graph is not None and not args.sequential:
+    def layer_order_ms(groups):
         step_seq = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=False, ratio=wl.ratio,
-                              queries=n_q if m else None, full_rescan=args.full_rescan)
+                              queries=n_q if m else None, full_rescan=args.full_rescan, groups=groups)
         step_seq.run(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
         g_seq = step_seq.capture(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
         for _ in range(3):
@@ -463,11 +464,22 @@ def run_ours(args):
             g_seq.replay()
         s1.record(stream)
         torch.cuda.synchronize()
-        seq_ms = max_over_ranks(s0.elapsed_time(s1) / args.steps, device, world)
+        t = max_over_ranks(s0.elapsed_time(s1) / args.steps, device, world)
         if step_seq.device_flags():
             raise RuntimeError("device status flags set in the layer-order step")
         del g_seq, step_seq
         reset_lengths()
+        return t
+
+    seq_ms = None
+    group_ms = {}
+    if graph is not None and not args.sequential:
+        seq_ms = layer_order_ms(1)
+        # layer order per group of sequences (groups overlap each other)
+        if not m and isinstance(off_d, torch.Tensor):
+            for G in args.groups:
+                if 1 < G <= wl.B:
+                    group_ms[G] = layer_order_ms(G)
     if graph is not None:
         for _ in range(min(args.steps, 50)):
             run_step(record=True)
@@ -619,6 +631,8 @@ def run_ours(args):
             "per_call_ms": per_call,
             "layer_order_graph": (None if seq_ms is None else
                                   {"ms_per_step": seq_ms, "queries_per_s": job_throughput(world, n_q, seq_ms)}),
+            "layer_order_groups_graph": {str(G): {"ms_per_step": t, "queries_per_s": job_throughput(world, n_q, t)}
+                                         for G, t in group_ms.items()},
             "clocks": clk.summary(),
             "device_flags": flags,
         }

@@ -99,13 +99,24 @@ class DecodeStep:
     the step (pool scoring, Top-k selection, attention) overlaps across
     layers.  Each such call then gets its own workspace.  The caller's stream
     waits for all of them before ``run`` returns, and the scans stay on the
-    caller's stream in layer order."""
+    caller's stream in layer order.  That overlap needs every layer's inputs
+    up front, which a model running layer after layer does not have.
+
+    With ``concurrent=False`` every call runs in layer order.  ``groups=G``
+    then splits the batch into G groups of consecutive sequences after each
+    scanning layer: a group's calls stay in layer order on a stream of their
+    own, and the groups overlap.  Sequences are independent, so this is an
+    order a model can run (its layer l+1 queries of a group come from that
+    group's layer l outputs)."""
 
     def __init__(self, pattern: str, B: int, max_len: int, P: int = 2048, k: int = 512, full_rescan: bool = False,
                  device="cuda", sm_scale: float | None = None, concurrent: bool = True, side_streams: int = 3,
-                 ratio: int = 1, projection: bool = True, queries: int | None = None, split_full: bool = False):
+                 ratio: int = 1, projection: bool = True, queries: int | None = None, split_full: bool = False,
+                 groups: int = 1):
         if ratio not in (1, 2):
             raise ValueError("ratio must be 1 or 2")
+        if groups < 1 or groups > B or (groups > 1 and (concurrent or queries is not None)):
+            raise ValueError("groups > 1 is for layer-order steps over sequences, at most one group per sequence")
         if queries is not None and ratio != 1:
             raise ValueError("verification steps take their entries as given (ratio 1 appends are the caller's)")
         self.pattern, self.B, self.max_len, self.P, self.k = pattern, B, max_len, P, k
@@ -136,10 +147,24 @@ class DecodeStep:
             self.ev_idx = [torch.cuda.Event() for _ in range(nL)]
             self.ev_pool = [torch.cuda.Event() for _ in range(nL)]
             self.ev_done = [torch.cuda.Event() for _ in range(nL)]
+        elif groups > 1:
+            # group g: sequences bounds[g] .. bounds[g+1]-1, its own stream and workspaces
+            self.bounds = [g * B // groups for g in range(groups + 1)]
+            sizes = [self.bounds[g + 1] - self.bounds[g] for g in range(groups)]
+            self.ws_re = [[C.workspace(C.csa2_index_reindex_workspace_bytes(n, P, k), dev) for n in sizes]
+                          if act == "reindex" else None for _, _, _, act in self.plan]
+            self.ws_attn = [[C.workspace(C.csa2_sparse_attn_decode_workspace_bytes(n, k), dev) for n in sizes]
+                            for _ in range(nL)]
+            self.gstreams = [torch.cuda.Stream(device=dev) for _ in range(groups)]
+            self.join = torch.cuda.Stream(device=dev)  # layer-done events, off the groups' paths
+            self.ev_scan = [torch.cuda.Event() for _ in range(nL)]
+            self.ev_group = [[torch.cuda.Event() for _ in range(groups)] for _ in range(nL)]
+            self.ev_layer = [torch.cuda.Event() for _ in range(nL)]
         else:
             ws_re, ws_attn = C.workspace(re_bytes, dev), C.workspace(attn_bytes, dev)
             self.ws_re = [ws_re] * nL
             self.ws_attn = [ws_attn] * nL
+        self.groups = groups
         # one pool per scanning layer (a rescan must not overwrite a pool that
         # an earlier Reindex layer may still be reading)
         self.pools = {layer: torch.full((nq, P), -1, dtype=torch.int32, device=dev)
@@ -196,6 +221,8 @@ class DecodeStep:
                 self._hook("csa2_compress_stream", "end", main)
         elif new_tokens is not None:
             raise ValueError("new_tokens is for ratio-2 steps")
+        if self.groups > 1:
+            return self._run_groups(caches, seq_row_off, seq_len, layers, main, ready, on_layer_done)
         pool, pool_ev = None, None
         last, last_ev = None, None
         # segments of the calls after the scan: sequences, or the queries of a
@@ -281,6 +308,68 @@ class DecodeStep:
                 main.wait_event(ev)
         return self.out
 
+    def _run_groups(self, caches, seq_row_off, seq_len, layers, main, ready, on_layer_done):
+        """Layer order per group of sequences (``groups`` > 1): scans on the
+        caller's stream over the whole batch, everything else per group on
+        the group's stream."""
+        if not isinstance(seq_row_off, torch.Tensor):
+            raise ValueError("groups > 1 takes the contiguous layout (seq_row_off tensor)")
+        G, bd = self.groups, self.bounds
+        pool, last = None, None
+        started = False
+        for layer, mode, f, act in self.plan:
+            L = layers[layer]
+            cache = caches[f]
+            ev_ready = ready[layer] if ready is not None else None
+            if act == "scan":
+                if started:  # the batch's next scan follows every group's earlier layers
+                    for g in range(G):
+                        main.wait_event(self.ev_group[layer - 1][g])
+                if ev_ready is not None:
+                    main.wait_event(ev_ready)
+                pool = self.pools[layer]
+                self._hook("csa2_index_full", "begin", main)
+                C.csa2_index_full(cache.idx, L["q_codes"], L["q_scales"], L["w"], seq_row_off, seq_len,
+                                  self.max_len, self.P, self.k, pool, self.topk[layer], self.ws_full, stream=main)
+                self._hook("csa2_index_full", "end", main)
+                last = self.topk[layer]
+                self.ev_scan[layer].record(main)
+            started = True
+            if act == "reuse":
+                self.topk[layer] = last
+            for g in range(G):
+                b0, b1 = bd[g], bd[g + 1]
+                s = self.gstreams[g]
+                if act == "scan":
+                    s.wait_event(self.ev_scan[layer])
+                if ev_ready is not None and act != "scan":
+                    s.wait_event(ev_ready)
+                if act == "reindex":
+                    self._hook("csa2_index_reindex", "begin", s)
+                    C.csa2_index_reindex(cache.idx, L["q_codes"][b0:b1], L["q_scales"][b0:b1], L["w"][b0:b1],
+                                         seq_row_off[b0:b1], seq_len[b0:b1], pool[b0:b1], self.k,
+                                         self.topk[layer][b0:b1], self.ws_re[layer][g], stream=s)
+                    self._hook("csa2_index_reindex", "end", s)
+                self._hook("csa2_sparse_attn_decode", "begin", s)
+                C.csa2_sparse_attn_decode(L["q"][b0:b1], cache.main, seq_row_off[b0:b1], seq_len[b0:b1],
+                                          self.topk[layer][b0:b1], L["win"][b0:b1], L["win_scale"][b0:b1],
+                                          L["win_len"][b0:b1], self.sm_scale, self.out[layer][b0:b1],
+                                          self.ws_attn[layer][g], lse=self.lse[layer][b0:b1], stream=s)
+                self._hook("csa2_sparse_attn_decode", "end", s)
+                self.ev_group[layer][g].record(s)
+            if act == "reindex":
+                last = self.topk[layer]
+            if on_layer_done is not None:
+                # an event after every group's attention of this layer, on a
+                # stream of its own (no group waits for another)
+                for g in range(G):
+                    self.join.wait_event(self.ev_group[layer][g])
+                self.ev_layer[layer].record(self.join)
+                on_layer_done(layer, self.ev_layer[layer])
+        for g in range(G):
+            main.wait_event(self.ev_group[self.plan[-1][0]][g])
+        return self.out
+
     def capture(self, caches, seq_row_off, seq_len, layers, new_tokens=None, q_off=None, q_vis=None):
         """Records one step into a CUDA graph; ``graph.replay()`` then runs the
         whole step (every call, both schedules, with the same buffers) as one
@@ -301,6 +390,9 @@ class DecodeStep:
     def device_flags(self) -> int:
         flags = C.device_status(self.ws_full)
         extra = [p.ws for p in self.pairs]
-        for ws in {id(w): w for w in self.ws_re + self.ws_attn + extra if w is not None}.values():
+        flat = []
+        for w in self.ws_re + self.ws_attn:
+            flat.extend(w if isinstance(w, list) else [w])
+        for ws in {id(w): w for w in flat + extra if w is not None}.values():
             flags |= C.device_status(ws)
         return flags

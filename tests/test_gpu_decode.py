@@ -411,3 +411,44 @@ def test_decode_with_the_full_layer_split_in_two_calls():
     for layer in range(len(wl.pattern)):
         assert np.array_equal(host(split.topk[layer]), host(plain.topk[layer]))
     assert np.array_equal(host(split.out), host(plain.out))
+
+
+@pytest.mark.parametrize("groups,rescan", [(2, False), (3, True)])
+def test_decode_grouped_layer_order_matches_layer_order(groups, rescan):
+    """groups > 1 (layer order per group of sequences, groups on their own
+    streams, graph-captured too) gives the bits of the plain layer-order
+    step: every call sees its sequences alike in both.  With a rescan the
+    second Full layer scans again, after every group's earlier layers."""
+    wl = W.DecodeWorkload("grouped_small", np.array([70000, 4096, 777, 20000, 9]), "FRRUFR", needles=8)
+    layers = [W.layer_inputs_host(wl, l) for l in range(len(wl.pattern))]
+    caches_h = [W.full_cache_host(wl, f, layers[f]["q_codes"], layers[f]["q_scales"]) for f in wl.full_layers()]
+    caches_d = [FullCache(C.cache(dev(c["idx_codes"]), dev(c["idx_scales"])),
+                          C.cache(dev(c["main_codes"]), dev(c["main_scales"]))) for c in caches_h]
+    off_d, len_d = dev(caches_h[0]["seq_row_off"]), dev(wl.lengths.astype(np.int32))
+    dl = _device_layers(layers)
+    plain = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, concurrent=False, full_rescan=rescan)
+    grouped = DecodeStep(wl.pattern, wl.B, wl.max_len, wl.P, wl.k, concurrent=False, groups=groups,
+                         full_rescan=rescan)
+    plain.run(caches_d, off_d, len_d, dl)
+    done = []
+    grouped.run(caches_d, off_d, len_d, dl, on_layer_done=lambda layer, ev: done.append(layer))
+    torch.cuda.synchronize()
+    assert done == list(range(len(wl.pattern)))
+    assert plain.device_flags() == 0 and grouped.device_flags() == 0
+
+    def same(a, b):
+        for p in a.pools:
+            assert np.array_equal(host(a.pools[p]), host(b.pools[p])), f"pool of layer {p}"
+        for layer in range(len(wl.pattern)):
+            assert np.array_equal(host(a.topk[layer]), host(b.topk[layer])), f"layer {layer} Top-k"
+        assert np.array_equal(host(a.out), host(b.out))
+        assert np.array_equal(host(a.lse), host(b.lse))
+
+    same(grouped, plain)
+    grouped.out.zero_()
+    g = grouped.capture(caches_d, off_d, len_d, dl)
+    g.replay()
+    torch.cuda.synchronize()
+    same(grouped, plain)
+    del g
+

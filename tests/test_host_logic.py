@@ -5,7 +5,7 @@ import pytest
 
 import bench
 import synth.workloads as W
-from long_context_decode_csa2_b200.decode import layer_plan
+from long_context_decode_csa2_b200.decode import DecodeStep, layer_plan
 
 
 def test_algorithmic_bytes_of_the_default_step():
@@ -80,3 +80,13 @@ def test_layer_plan_rejects_bad_patterns():
     for bad in ("RF", "UF", "FX"):
         with pytest.raises(ValueError):
             layer_plan(bad)
+
+
+def test_decode_grouped_rejects_other_schedules():
+    """Grouped layer order is for plain decode steps (checked before any device memory is taken)."""
+    with pytest.raises(ValueError):
+        DecodeStep("FR", 4, 8192, groups=2)                      # concurrent steps overlap layers instead
+    with pytest.raises(ValueError):
+        DecodeStep("FR", 4, 8192, concurrent=False, groups=5)    # more groups than sequences
+    with pytest.raises(ValueError):
+        DecodeStep("FR", 4, 8192, concurrent=False, groups=2, queries=8)

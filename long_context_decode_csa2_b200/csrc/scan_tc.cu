@@ -15,7 +15,9 @@
 //     swizzle) and one bulk copy of the scale words.  Pool: four producer
 //     warps each gather 16 of the item's 64 blocks with cp.async (one warp
 //     instruction per 512-byte block, the swizzle applied to the
-//     destination) from the segment's pool ids held in shared memory.
+//     destination) from the segment's pool ids held in shared memory; each
+//     lane's copies arrive on the stage's barrier as they land
+//     (cp.async.mbarrier.arrive), so the producers never wait for them.
 //     Warp 0 also writes the item's B operand: the segment's indexer query
 //     laid out "one 32-element block per output column" (column 4h+b holds
 //     head h's block b, zeros elsewhere);
@@ -44,12 +46,11 @@ namespace {
 
 constexpr int kTile = 512;             // positions per work item
 constexpr int kMT = kTile / 128;       // 128-row MMA tiles per item
-// smem ring: 4 stages stream the contiguous scan fastest; the pool gather
-// signals a stage only kGatherDepth items after issuing it, so it needs more
+// smem ring: 4 stages stream the contiguous scan fastest; the pool gather's
+// small copies take longer to land, so it keeps more items in flight
 template <bool kPool>
 struct Ring {
   static constexpr int kStages = kPool ? 6 : 4;
-  static constexpr int kGatherDepth = 3;  // gathered items in flight before signalling
 };
 constexpr int kAcc = 3;                // TMEM accumulator ring (16 columns per MMA tile)
 constexpr int kAccCols = 16 * kMT;
@@ -116,6 +117,41 @@ struct ScanParams {
   uint32_t* status;
 };
 
+// Whole warp: the same, with up to 128 prefix entries loaded at once (one
+// round trip instead of a chain of them), also returning the segment's first
+// item and the next segment's; longer prefixes fall back.
+__device__ __forceinline__ int find_seq(const int32_t* tile_start, int S, int item);
+__device__ __forceinline__ int find_seq_warp(const int32_t* tile_start, int S, int item, int& start, int& next) {
+  if (S + 1 > 128) {
+    const int b = find_seq(tile_start, S, item);
+    start = __ldg(tile_start + b);
+    next = __ldg(tile_start + b + 1);
+    return b;
+  }
+  const int lane = threadIdx.x & 31;
+  int32_t v[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int j = lane + 32 * r;
+    v[r] = j <= S ? __ldg(tile_start + j) : INT32_MAX;
+  }
+  // the last j < S with tile_start[j] <= item (tile_start ascends, [0] = 0)
+  int last = 0;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const uint32_t m = __ballot_sync(0xffffffffu, lane + 32 * r < S && v[r] <= item);
+    if (m) last = 32 * r + 31 - __clz(m);
+  }
+  auto entry = [&](int j) {  // tile_start[j] for j <= S (the same j in every lane)
+    const int r = j >> 5;
+    const int32_t x = r == 0 ? v[0] : r == 1 ? v[1] : r == 2 ? v[2] : v[3];
+    return __shfl_sync(0xffffffffu, x, j & 31);
+  };
+  start = entry(last);
+  next = entry(last + 1);
+  return last;
+}
+
 __device__ __forceinline__ int find_seq(const int32_t* tile_start, int S, int item) {
   int lo = 0, hi = S;  // tile_start[lo] <= item < tile_start[hi]
   while (hi - lo > 1) {
@@ -161,7 +197,6 @@ template <bool kPool>
 __global__ void __launch_bounds__(threads_of<kPool>(), 1)
     k_index_tc(const __grid_constant__ CUtensorMap tmap, ScanParams p) {
   constexpr int kStages = Ring<kPool>::kStages;
-  constexpr int kGatherDepth = Ring<kPool>::kGatherDepth;
   using Smem = ScanSmem<kStages>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(
@@ -172,7 +207,9 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
   // prologue (touches no global memory): barriers, tensor memory, unit scales
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      sm100::mbar_init(&sm.full[s], kPool ? kPoolProducers : 1);
+      // pool: every producer lane arrives when its copies have landed, and
+      // lane 0 of each producer warp once more after the warp's writes
+      sm100::mbar_init(&sm.full[s], kPool ? kPoolProducers * 33 : 1);
       sm100::mbar_init(&sm.empty[s], 1 + 4);
     }
     for (int a = 0; a < kAcc; ++a) {
@@ -226,9 +263,7 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
       if (kPool) {
         b = i0 / p.items_per_seg;
       } else {
-        b = find_seq(p.tile_start, p.S, i0);
-        seq_start = __ldg(p.tile_start + b);
-        next_start = __ldg(p.tile_start + b + 1);
+        b = find_seq_warp(p.tile_start, p.S, i0, seq_start, next_start);
       }
       int64_t seq_off = seg_row_off(p, b);
       int64_t seq_len = seg_len(p, b);
@@ -262,6 +297,21 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
           break;
         }
         if (__any_sync(0xffffffffu, aborted(sm))) break;
+        // pool mode, new segment: this warp's share of its pool ids (one
+        // round trip per segment, in flight with the query's codes below);
+        // copies already issued carry their own addresses
+        constexpr int kPer = CSA2_MAX_POOL_BLOCKS / kPoolProducers / 32;
+        int32_t v[kPer];
+        const bool new_pool = kPool && pool_seg != b;
+        if (new_pool) {
+          const int32_t* src = p.pool + int64_t(b) * p.P;
+#pragma unroll
+          for (int m = 0; m < kPer; ++m) {
+            const int e = lane + 32 * m;  // entry (item e / kSlotsPerWarp, slot e % kSlotsPerWarp)
+            const int slot = (e / kSlotsPerWarp) * kPoolSlots + pw * kSlotsPerWarp + e % kSlotsPerWarp;
+            v[m] = slot < p.P ? __ldg(src + slot) : -1;
+          }
+        }
         if (pw == 0 && sm.built[s] != b) {
           if (qb != b) {
             qreg = __ldg(reinterpret_cast<const uint2*>(p.q_codes + int64_t(b) * kHi * 64) + lane);
@@ -273,18 +323,7 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
         }
         __syncwarp();
         if (kPool) {
-          if (pool_seg != b) {
-            // this warp's share of the segment's pool ids (one round trip per
-            // segment); copies already issued carry their own addresses
-            const int32_t* src = p.pool + int64_t(b) * p.P;
-            constexpr int kPer = CSA2_MAX_POOL_BLOCKS / kPoolProducers / 32;
-            int32_t v[kPer];
-#pragma unroll
-            for (int m = 0; m < kPer; ++m) {
-              const int e = lane + 32 * m;  // entry (item e / kSlotsPerWarp, slot e % kSlotsPerWarp)
-              const int slot = (e / kSlotsPerWarp) * kPoolSlots + pw * kSlotsPerWarp + e % kSlotsPerWarp;
-              v[m] = slot < p.P ? __ldg(src + slot) : -1;
-            }
+          if (new_pool) {
 #pragma unroll
             for (int m = 0; m < kPer; ++m) sm.segpool[pw][lane + 32 * m] = v[m];
             __syncwarp();
@@ -323,14 +362,14 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
               sm100::cp_async16(&sm.sc[s][(pw * kSlotsPerWarp + i) * kBlk + 4 * (c & 1)],
                                 p.kscales + row * 4 + 16 * (c & 1));
           }
-          sm100::cp_async_commit();
-          // signal the item issued kGatherDepth items ago once its copies landed
-          if (t >= kGatherDepth) {
-            sm100::cp_async_wait<kGatherDepth>();
-            sm100::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(&sm.full[(t - kGatherDepth) % kStages]);
-          }
+          // the stage completes once every lane's copies have landed and
+          // lane 0 has arrived after the warp's generic writes (slot blocks,
+          // item info, B operand: fenced for the async proxy); the MMA thread
+          // fences the landed copies itself after its wait
+          sm100::cp_async_mbar_arrive_noinc(&sm.full[s]);
+          sm100::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&sm.full[s]);
         } else if (lane == 0) {
           sm.info[s] = make_int2(b, j);
           const int64_t rem_rows = seq_len - int64_t(j) * kTile;
@@ -350,18 +389,12 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
         }
         ++issued;
       }
-      if (kPool) {
-        sm100::cp_async_wait<0>();
-        sm100::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0)
-          for (int t = max(0, issued - kGatherDepth); t < issued; ++t) sm100::mbar_arrive(&sm.full[t % kStages]);
-      }
+      if (kPool) sm100::cp_async_wait<0>();  // (landed already once the MMA consumed every stage)
     }
     // drain: every copy this warp issued has landed before the CTA exits (a
     // withheld item 0 leaves stage 0 without copies: it is never refilled,
     // since that needs item 0 consumed first)
-    if (!kPool && lane == 0)
+    if (lane == 0)
       for (int s = 0; s < kStages && s < issued; ++s) {
         if (withhold && s == 0) continue;
         const int last_round = (issued - 1 - s) / kStages;
@@ -383,6 +416,10 @@ __global__ void __launch_bounds__(threads_of<kPool>(), 1)
           break;
         }
         if (aborted(sm)) break;
+        // pool: the gathered rows were written by cp.async (generic proxy);
+        // the barrier made them visible here, the fence orders them before
+        // this thread's tensor-core (async proxy) reads
+        if (kPool) sm100::fence_proxy_async_smem();
         sm100::tc_fence_after();
         const uint32_t abase = sm100::smem_u32(sm.a[s]);
         const uint32_t bbase = sm100::smem_u32(sm.bop[s]);

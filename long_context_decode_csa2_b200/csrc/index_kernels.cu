@@ -358,6 +358,21 @@ __device__ __forceinline__ void select_segment(const void* __restrict__ in, int6
     const int64_t i0 = int64_t(tid) * kSelPer;
     HistPart<NB> hp;
     if (ghist) load_hist<NB>(ghist + int64_t(s) * NB, hp);  // in flight with the keys
+    // pool candidates: the pool ids of this thread's two blocks, loaded with
+    // the keys (not one dependent load per selected id at the end)
+    constexpr int kIdBlocks = KIND == kSelPoolCand ? kSelPer / kBlk : 1;
+    int32_t pid[kIdBlocks];
+    if (KIND == kSelPoolCand) {
+#pragma unroll
+      for (int m = 0; m < kIdBlocks; ++m) {
+        const int64_t bi = i0 / kBlk + m;
+        pid[m] = bi < P ? __ldg(pool + int64_t(s) * P + bi) : -1;
+      }
+    }
+    auto id_of = [&](int e) -> int32_t {
+      if (KIND == kSelPoolCand) return pid[e / kBlk] * kBlk + (e % kBlk);
+      return sel_id<KIND>(pool, s, P, i0 + e);
+    };
     load_keys<KIND>(in, base, i0, n, kk);
     uint32_t present = 0;
 #pragma unroll
@@ -430,10 +445,10 @@ __device__ __forceinline__ void select_segment(const void* __restrict__ in, int6
       const uint32_t key = kk[e];
       if (key > T) {
         const uint32_t at = g + min(q, rem);
-        if (at < uint32_t(k)) o[at] = sel_id<KIND>(pool, s, P, i0 + e);
+        if (at < uint32_t(k)) o[at] = id_of(e);
         ++g;
       } else if (key == T && key != 0u) {
-        if (q < rem && g + q < uint32_t(k)) o[g + q] = sel_id<KIND>(pool, s, P, i0 + e);
+        if (q < rem && g + q < uint32_t(k)) o[g + q] = id_of(e);
         ++q;
       }
     }

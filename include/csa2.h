@@ -52,6 +52,14 @@
  *   - Return value: CSA2_OK, or a negative error; on an error nothing was
  *     launched, except CSA2_ERR_CUDA (a launch failed; see csa2_last_error()).
  *     Arguments are validated on the host before the first launch.
+ *   - Stream order: every call runs after the work enqueued before it on
+ *     `stream`, with one refinement.  The kernels here let the stream's next
+ *     kernel start early and wait for their results themselves, and the
+ *     attention calls read their queries (q) before that wait, so while the
+ *     preceding kernel may still run.  No kernel of this library writes a
+ *     query; a query written by other earlier work (a copy, or a kernel that
+ *     does not trigger the early launch of its dependents) is complete before
+ *     it is read.
  */
 #ifndef CSA2_H
 #define CSA2_H

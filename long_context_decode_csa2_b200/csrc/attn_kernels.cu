@@ -624,7 +624,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
     sm.m_run[tid] = -INFINITY;
     sm.l_run[tid] = 0.0f;
   }
-  grid_wait();  // the Top-k ids, queries and rows may come from the previous kernel
+  // The queries are the caller's inputs, which no kernel of this library
+  // writes: they are read while the previous kernel (typically the Top-k
+  // selection) still runs.  A kernel that does not trigger its dependents
+  // early has completed before this one starts.
+  QFrag qf;
+  load_q_frag(a, s, (tid >> 5) & 3, qf);
+  grid_wait();  // the Top-k ids, lengths and rows may come from the previous kernel
   const SegInfo sg = seg_info(a, s);
   int32_t tnext = -1;
   if (c0 < c1) {
@@ -632,8 +638,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
     sm100::cp_async_commit();
     tnext = (c0 + 1 < c1) ? chunk_tpos(a, s, c0 + 1, row) : -1;
   }
-  QFrag qf;
-  load_q_frag(a, s, (tid >> 5) & 3, qf);  // overlaps the first gather
   bool in_win = false, wrote_main = false;
   float win_scale = 1.0f;
   for (int c = c0; c < c1; ++c) {

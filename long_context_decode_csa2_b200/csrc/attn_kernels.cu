@@ -4,12 +4,15 @@
 // MXFP4 main KV, FP8 window; section "后 20 层干脆共用一份 KV": 128-token window).
 //
 // Work split: a segment's keys are chunks (ceil(k/64) chunks of 64 selected
-// rows, then four window chunks of 32 rows), and R CTAs share a segment, each
-// walking a contiguous run of its chunks (R = 2 x SMs / segments, at most 4:
-// two CTAs fit on an SM, and small batches still fill the GPU in one wave).
-// While a CTA computes one chunk, cp.async brings the next chunk's raw rows
-// (272-byte MXFP4 rows or 512-byte E4M3 rows) into the other half of a
-// double buffer; the Top-k ids are loaded one chunk earlier still.
+// rows, and four window chunks of 32 rows), and R CTAs share a segment
+// (R = 2 x SMs / segments, at most 4: two CTAs fit on an SM, and small
+// batches still fill the GPU in one wave).  Each CTA takes an even share of
+// the window chunks and one of the selected chunks, windows first: the window
+// rows are the caller's inputs, so the first of them are staged before the
+// wait on the previous kernel.  While a CTA computes one chunk, cp.async
+// brings the next chunk's raw rows (272-byte MXFP4 rows or 512-byte E4M3
+// rows) into the staging buffer; the Top-k ids are loaded one chunk earlier
+// still.
 //
 // Both products run on the tensor cores with warp-level mma (fp16 inputs,
 // fp32 accumulation), and the rows are converted to fp16 once, in registers
@@ -606,13 +609,19 @@ __device__ __forceinline__ void combine_if_last(const AttnArgs& a, AttnSmem& sm,
   if (tid == 0) a.counters[s] = 0;
 }
 
-// grid = (R, S): CTA (r, s) takes chunks [r n / R, (r + 1) n / R) of segment s.
+// grid = (R, S): CTA (r, s) takes window chunks [4r/R, 4(r+1)/R) and main
+// chunks [m r/R, m (r+1)/R) of segment s (m main chunks), windows first.  The
+// window rows, like the queries, are the caller's inputs: the first window
+// chunk is staged before the wait on the previous kernel.
 __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
   const int s = blockIdx.y, r = blockIdx.x, tid = threadIdx.x, row = tid & (kChunk - 1);
-  const int n = attn_main_chunks(a.k) + kWinChunks;
-  const int c0 = int(int64_t(n) * r / R), c1 = int(int64_t(n) * (r + 1) / R);
+  const int nmain = attn_main_chunks(a.k);
+  const int w0 = kWinChunks * r / R, w1 = kWinChunks * (r + 1) / R;
+  const int m0 = int(int64_t(nmain) * r / R), m1 = int(int64_t(nmain) * (r + 1) / R);
+  const int nw = w1 - w0, nc = nw + (m1 - m0);
+  auto chunk_at = [&](int i) { return i < nw ? nmain + w0 + i : m0 + (i - nw); };
   const int nslots = 2 * R;
   launch_dependents();
   float oacc[8][4];
@@ -624,52 +633,52 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
     sm.m_run[tid] = -INFINITY;
     sm.l_run[tid] = 0.0f;
   }
-  // The queries are the caller's inputs, which no kernel of this library
-  // writes: they are read while the previous kernel (typically the Top-k
-  // selection) still runs.  A kernel that does not trigger its dependents
-  // early has completed before this one starts.
+  // The queries and the window rows are the caller's inputs, which no kernel
+  // of this library writes: they are read while the previous kernel
+  // (typically the Top-k selection) still runs.  A kernel that does not
+  // trigger its dependents early has completed before this one starts.
   QFrag qf;
   load_q_frag(a, s, (tid >> 5) & 3, qf);
+  if (nw > 0) {
+    const SegInfo unused{0, -1};  // (window chunks read no cache rows)
+    issue_gather(a, sm, 0, s, chunk_at(0), -1, unused);
+    sm100::cp_async_commit();
+  }
   grid_wait();  // the Top-k ids, lengths and rows may come from the previous kernel
   const SegInfo sg = seg_info(a, s);
-  int32_t tnext = -1;
-  if (c0 < c1) {
-    issue_gather(a, sm, 0, s, c0, chunk_tpos(a, s, c0, row), sg);
+  if (nw == 0 && nc > 0) {
+    issue_gather(a, sm, 0, s, chunk_at(0), chunk_tpos(a, s, chunk_at(0), row), sg);
     sm100::cp_async_commit();
-    tnext = (c0 + 1 < c1) ? chunk_tpos(a, s, c0 + 1, row) : -1;
   }
-  bool in_win = false, wrote_main = false;
+  int32_t tnext = nc > 1 ? chunk_tpos(a, s, chunk_at(1), row) : -1;
+  bool in_win = nw > 0;
   float win_scale = 1.0f;
-  for (int c = c0; c < c1; ++c) {
-    const int vb = (c - c0) & 1;
+  for (int i = 0; i < nc; ++i) {
+    const int c = chunk_at(i), vb = i & 1;
     const ChunkSrc src = chunk_src(a, s, c);
-    if (src.is_win && !in_win) {
-      if (c > c0) {  // this CTA's selected rows are done: their partial
-        flush_part(a, sm, oacc, s, nslots, 2 * r, 1.0f);
-        wrote_main = true;
-      }
-      in_win = true;
+    if (src.is_win) {
       win_scale = src.kscale;
+    } else if (in_win) {  // this CTA's window rows are done: their partial
+      flush_part(a, sm, oacc, s, nslots, 2 * r + 1, win_scale);
+      in_win = false;
     }
     sm100::cp_async_wait<0>();
     __syncthreads();  // this chunk's rows are staged; the last chunk's P V is done
     qk_partial(a, sm, src.is_win, src.nkeys, qf);
     __syncthreads();  // converted rows and partial scores written; the staging buffer is free
-    if (c + 1 < c1) {
-      issue_gather(a, sm, vb ^ 1, s, c + 1, tnext, sg);
+    if (i + 1 < nc) {
+      issue_gather(a, sm, vb ^ 1, s, chunk_at(i + 1), tnext, sg);
       sm100::cp_async_commit();
-      tnext = (c + 2 < c1) ? chunk_tpos(a, s, c + 2, row) : -1;
+      tnext = (i + 2 < nc) ? chunk_tpos(a, s, chunk_at(i + 2), row) : -1;
     }
     softmax_pv(a, sm, vb, oacc, src.nkeys, src.kscale);
   }
-  if (in_win) {
-    flush_part(a, sm, oacc, s, nslots, 2 * r + 1, win_scale);
-  } else if (c0 < c1) {
-    flush_part(a, sm, oacc, s, nslots, 2 * r, 1.0f);
-    wrote_main = true;
+  if (nc > 0) {  // the part in progress
+    if (in_win) flush_part(a, sm, oacc, s, nslots, 2 * r + 1, win_scale);
+    else flush_part(a, sm, oacc, s, nslots, 2 * r, 1.0f);
   }
-  if (!wrote_main) empty_part(a, s, nslots, 2 * r);
-  if (!in_win) empty_part(a, s, nslots, 2 * r + 1);
+  if (m1 == m0) empty_part(a, s, nslots, 2 * r);
+  if (nw == 0) empty_part(a, s, nslots, 2 * r + 1);
   sm100::cp_async_wait<0>();
   combine_if_last(a, sm, s, R, nslots);
 }

@@ -47,8 +47,11 @@ def parse():
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (small profiling captures)")
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager steps instead of replays of one captured CUDA graph")
-    ap.add_argument("--sequential", action="store_true",
-                    help="issue every call on one stream (isolated per-call times) instead of the concurrent tail")
+    ap.add_argument("--schedule", choices=["layer", "concurrent"], default="layer",
+                    help="the timed step: every call in layer order on one stream (the order a model runs; "
+                         "default), or the tail of every layer overlapped on side streams (needs every layer's "
+                         "inputs up front); the other one is timed as well and reported beside it")
+    ap.add_argument("--sequential", action="store_true", help="the same as --schedule layer")
     ap.add_argument("--context", type=int, default=0,
                     help="override every sequence's length (small profiling captures of the attention)")
     ap.add_argument("--full-rescan", action="store_true",
@@ -233,7 +236,7 @@ def single_thread_oracle(wl, samples):
 
 # ----------------------------------------------------------------------------
 
-def decode_config(wl, l2_bytes, sequential, graph=True, full_rescan=False):
+def decode_config(wl, l2_bytes, concurrent, graph=True, full_rescan=False):
     """The `config` object of a decode line (both arms)."""
     extra = ({"ratio": 2, "append": "one raw token per sequence per Full layer per step (csa2_compress_stream, "
                                     "W_idx projection)"} if wl.ratio == 2 else {})
@@ -248,8 +251,8 @@ def decode_config(wl, l2_bytes, sequential, graph=True, full_rescan=False):
     return {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.max_len, "layers": wl.pattern, **extra,
             "pool_blocks": wl.P, "topk": wl.k, "window": 128,
             "l2": "no flush: inputs larger than L2 (%.2f GB read per step)" % (l2_bytes / 1e9),
-            "schedule": ("sequential" if sequential else "concurrent tail (side streams)")
-                        + (", one CUDA graph per step" if graph else "")}
+            "schedule": ("concurrent tail (side streams: every layer's inputs given up front)" if concurrent
+                         else "layer order (one stream)") + (", one CUDA graph per step" if graph else "")}
 
 
 def rank_workload(wl, rank):
@@ -368,7 +371,8 @@ def run_ours(args):
     C.lib()
     m = wl.queries_per_seq
     n_q = wl.B * m if m else wl.B  # queries per step on this rank
-    step = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=not args.sequential,
+    concurrent = args.schedule == "concurrent" and not args.sequential
+    step = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=concurrent,
                       ratio=wl.ratio, queries=n_q if m else None, full_rescan=args.full_rescan)
     vq = {}
     if m:
@@ -446,11 +450,13 @@ def run_ours(args):
         dist.barrier()
     ms = t0.elapsed_time(t1) / args.steps
     reset_lengths()
-    # the same step with every call in layer order on one stream (the order a
-    # model whose layer inputs depend on the previous layer would impose),
-    # also replayed from a graph
-    def layer_order_ms(groups):
-        step_seq = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=False, ratio=wl.ratio,
+    # the same step in the other schedule (layer order: the order a model whose
+    # layer inputs depend on the previous layer imposes; concurrent: the tails
+    # of all layers overlapped, possible only with every layer's inputs given
+    # up front), and layer order per group of sequences, each replayed from a
+    # graph
+    def schedule_ms(conc, groups=1):
+        step_seq = DecodeStep(wl.pattern, wl.B, wl.max_len + wl.room, wl.P, wl.k, concurrent=conc, ratio=wl.ratio,
                               queries=n_q if m else None, full_rescan=args.full_rescan, groups=groups)
         step_seq.run(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
         g_seq = step_seq.capture(caches, off_d, len_d, layers_dev, new_tokens=toks_dev, **vq)
@@ -471,15 +477,15 @@ def run_ours(args):
         reset_lengths()
         return t
 
-    seq_ms = None
+    other_ms = None
     group_ms = {}
-    if graph is not None and not args.sequential:
-        seq_ms = layer_order_ms(1)
+    if graph is not None:
+        other_ms = schedule_ms(not concurrent)
         # layer order per group of sequences (groups overlap each other)
         if not m and isinstance(off_d, torch.Tensor):
             for G in args.groups:
                 if 1 < G <= wl.B:
-                    group_ms[G] = layer_order_ms(G)
+                    group_ms[G] = schedule_ms(False, G)
     if graph is not None:
         for _ in range(min(args.steps, 50)):
             run_step(record=True)
@@ -616,7 +622,7 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "int32+f64 indexer, f16 tensor-core attention (f32 accumulate)",
             "data": "synthetic",
-            "config": decode_config(wl, ab["total"], args.sequential, graph is not None, args.full_rescan),
+            "config": decode_config(wl, ab["total"], concurrent, graph is not None, args.full_rescan),
             "tokens_per_s": job_throughput(world, n_q, ms),
             "hbm_algorithmic_gbs": ab["total"] / (ms * 1e-3) / 1e9,
             "hbm_frac_of_8tbs": ab["total"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
@@ -629,8 +635,9 @@ def run_ours(args):
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "per_call_ms": per_call,
-            "layer_order_graph": (None if seq_ms is None else
-                                  {"ms_per_step": seq_ms, "queries_per_s": job_throughput(world, n_q, seq_ms)}),
+            ("layer_order_graph" if concurrent else "concurrent_layers_graph"):
+                (None if other_ms is None else
+                 {"ms_per_step": other_ms, "queries_per_s": job_throughput(world, n_q, other_ms)}),
             "layer_order_groups_graph": {str(G): {"ms_per_step": t, "queries_per_s": job_throughput(world, n_q, t)}
                                          for G, t in group_ms.items()},
             "clocks": clk.summary(),
@@ -906,7 +913,8 @@ def run_reference(args):
     res = {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int32+f64 (CPU oracle)",
-           "data": "synthetic", "config": decode_config(wl, algorithmic_bytes(wl)["total"], args.sequential,
+           "data": "synthetic", "config": decode_config(wl, algorithmic_bytes(wl)["total"],
+                                                        args.schedule == "concurrent" and not args.sequential,
                                                         not args.no_graph),
            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": nthreads, "kind": "oracle",
                             "sample": f"{nseq} queries ({max(1, wl.queries_per_seq)} per step) over "
@@ -1034,7 +1042,7 @@ def run_cp(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None,
             "dtype": "int32+f64 indexer, f16 tensor-core attention (f32 accumulate)", "data": "synthetic",
-            "config": dict(decode_config(wl, ab["total"], True, graph is not None), cp_shards=G,
+            "config": dict(decode_config(wl, ab["total"], False, graph is not None), cp_shards=G,
                            cp_mode="one shard per rank (NCCL all-gather)" if world > 1 else
                            "all shards on this GPU, one after the other"),
             "hbm_algorithmic_gbs": ab["total"] / (ms * 1e-3) / 1e9,

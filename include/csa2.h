@@ -197,9 +197,13 @@ csa2_status csa2_sparse_attn_decode(const uint16_t* q, csa2_mxfp4_cache main_kv,
  *   Both rows are MXFP4-encoded per OCP MX v1.0: X = floor(log2 amax) - 2,
  *   nearest E2M1 with ties to even, saturating at 6, sign kept.
  *   raw        [n_tok][512] bf16;  logits [n_tok] fp32 (ratio 2; may be NULL for ratio 1)
- *   w_idx      [512][128] fp32 or NULL;  idx_raw [n_tok][128] bf16 or NULL (exactly one given)
+ *   w_idx      [512][128] fp32 (8-byte aligned) or NULL;  idx_raw [n_tok][128] bf16 or NULL
+ *              (exactly one given)
  *   tok_off    [B+1] int64;  seq_row_off [B] int64;  seq_len_in [B], seq_len_out [B] int32
- *   n_tok      host: tok_off[B];  max_new host: upper bound of n_b (grid sizing)
+ *   n_tok      host: tok_off[B];  max_new host: upper bound of n_b (grid sizing;
+ *              entries beyond it are not written and CSA2_DEV_LENGTH is flagged)
+ *   workspace  csa2_compress_append_workspace_bytes(B) bytes (the status word),
+ *              256-byte aligned
  * ------------------------------------------------------------------------- */
 size_t csa2_compress_append_workspace_bytes(int B);
 csa2_status csa2_compress_append(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_k, const uint16_t* raw,

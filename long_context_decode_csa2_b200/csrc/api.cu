@@ -407,9 +407,13 @@ csa2_status csa2_compress_append(csa2_mxfp4_cache main_kv, csa2_mxfp4_cache idx_
   if (ratio == 2 && !logits) return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": ratio 2 needs logits");
   if ((w_idx == nullptr) == (idx_raw == nullptr))
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": give exactly one of w_idx and idx_raw");
-  if (!aligned16(raw) || (idx_raw && (reinterpret_cast<uintptr_t>(idx_raw) & 7)))
-    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": raw must be 16-byte and idx_raw 8-byte aligned");
-  if (workspace_bytes < kStatusBytes) return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
+  if (!aligned16(raw) || (idx_raw && (reinterpret_cast<uintptr_t>(idx_raw) & 7)) ||
+      (w_idx && (reinterpret_cast<uintptr_t>(w_idx) & 7)))
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": raw must be 16-byte, idx_raw and w_idx 8-byte aligned");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": workspace must be 256-byte aligned");
+  if (workspace_bytes < csa2_compress_append_workspace_bytes(B))
+    return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
   CompressArgs a{};
   a.mcodes = main_kv.codes;
   a.mscales = main_kv.scales;
@@ -457,9 +461,11 @@ csa2_status compress_stream_impl(const char* fn, csa2_mxfp4_cache main_kv, csa2_
   if (!w_idx && (!pend_idx || (n_tok > 0 && !idx_raw)))
     return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": idx_raw needs pend_idx");
   if ((raw && !aligned16(raw)) || !aligned16(pend_raw) || (idx_raw && (reinterpret_cast<uintptr_t>(idx_raw) & 7)) ||
-      (pend_idx && (reinterpret_cast<uintptr_t>(pend_idx) & 7)))
+      (pend_idx && (reinterpret_cast<uintptr_t>(pend_idx) & 7)) || (w_idx && (reinterpret_cast<uintptr_t>(w_idx) & 7)))
     return fail(CSA2_ERR_INVALID_ARG,
-                std::string(fn) + ": raw and pend_raw must be 16-byte, idx_raw and pend_idx 8-byte aligned");
+                std::string(fn) + ": raw and pend_raw must be 16-byte, idx_raw, pend_idx and w_idx 8-byte aligned");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(CSA2_ERR_INVALID_ARG, std::string(fn) + ": workspace must be 256-byte aligned");
   if (workspace_bytes < csa2_compress_stream_workspace_bytes(B))
     return fail(CSA2_ERR_WORKSPACE, std::string(fn) + ": workspace too small");
   CompressArgs a{};

@@ -76,8 +76,20 @@ __device__ __forceinline__ uint32_t e2m1_code(float x, float inv_scale) {
 
 constexpr int kCompWarps = 8;
 constexpr int kCompEntries = 16;                       // entries per CTA (two per warp)
-constexpr int kCompGroups = kCompWarps * 32 / kDi;     // projection: entry groups of the CTA (2)
-constexpr int kCompPerThread = kCompEntries / kCompGroups;  // entries per projecting thread (8)
+constexpr int kCompGroups = kCompWarps * 32 / kDi;     // one-chain projection: entry groups of the CTA (2)
+// Projection of a full CTA: thread t owns columns 2(t % 64), 2(t % 64) + 1
+// of the entries e = 4q + t / 64 (q = 0..3), eight chains, and reads two
+// consecutive terms of an entry's merged row per 16-byte shared load, so a
+// shared load feeds four FMAs; W_idx rows are loaded one block ahead of their
+// use.  (For 262144 tokens at ratio 2: one shared load per FMA, with each
+// W_idx load just before its use, 1.36 ms; this, 1.11 ms; W_idx widened to
+// fp64 once per call and read as doubles, 1.21 ms: twice the L2 bytes cost
+// more than the conversions it saves.)
+constexpr int kProjCols = 2;                                   // columns per projecting thread
+constexpr int kProjGroups = kCompWarps * 32 * kProjCols / kDi; // entry groups (4)
+constexpr int kProjEntries = kCompEntries / kProjGroups;       // entries per projecting thread (4)
+constexpr int kProjRows = 4;                                   // W_idx rows per prefetched block
+static_assert(kD % kProjRows == 0 && kProjRows % 2 == 0, "whole blocks of row pairs");
 
 // Writes one MXFP4 row of 32*V elements held V per lane (lane: elements
 // V*lane .. V*lane+V-1), blocks of 32 = 32/V lanes.
@@ -132,13 +144,13 @@ __device__ __forceinline__ void pair_weights(double z0, double z1, double& w0, d
 
 // grid = (ceil(max_new / 16), B), block = 256.  Each warp merges and encodes
 // two entries' main rows; the optional W_idx projection is shared by the CTA
-// (thread t: column t % 128 of the entries e = 2q + t / 128, so every W_idx
-// element read feeds up to eight fma chains), and each warp then encodes its
+// (thread t: columns 2(t % 64) and 2(t % 64) + 1 of the entries
+// e = 4q + t / 64, eight fma chains), and each warp then encodes its
 // two indexer rows.  Streaming mode (a.pend_n != null): the sequence's token
 // stream starts with its pending token, the last CTA of the sequence to
 // finish keeps an odd trailing token as the new pending one and writes the
 // new lengths (all CTAs have read the old ones by then).
-__global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
+__global__ void __launch_bounds__(kCompWarps * 32, 3) k_compress(CompressArgs a) {
   // merged rows, widened once for the projection; projected rows
   extern __shared__ __align__(16) unsigned char csm[];
   double (*cbuf)[kD] = reinterpret_cast<double (*)[kD]>(csm);
@@ -153,9 +165,14 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
   const int64_t ntok = max(int64_t(0), a.tok_off[b + 1] - tok0);
   const int pn = streaming ? (a.pend_n[b] != 0 ? 1 : 0) : 0;
   const int64_t nstream = ntok + pn;
-  const int64_t nnew = nstream / a.ratio;
+  const int64_t nnew_all = nstream / a.ratio;
+  // entries beyond the host's bound max_new (the grid) are not written: flagged
+  const int64_t nnew = min(nnew_all, a.max_new);
   const int32_t len_in = a.seq_len_in[b];
-  if (!streaming && blockIdx.x == 0 && threadIdx.x == 0) a.seq_len_out[b] = len_in + int32_t(nnew);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (nnew_all > a.max_new) set_status(a.status, CSA2_DEV_LENGTH);
+    if (!streaming) a.seq_len_out[b] = len_in + int32_t(nnew_all);
+  }
   const TokenSrc src{a, b, pn, tok0};
   const int64_t j0 = int64_t(blockIdx.x) * kCompEntries;
 
@@ -243,18 +260,38 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
           rbuf[grp][col] = __double2float_rn(acc);
         }
       } else {
-        double acc[kCompPerThread];
+        const int c0 = kProjCols * (threadIdx.x % (kDi / kProjCols)), pg = threadIdx.x / (kDi / kProjCols);
+        double acc[kProjEntries][kProjCols];
 #pragma unroll
-        for (int q = 0; q < kCompPerThread; ++q) acc[q] = 0.0;
-#pragma unroll 4
-        for (int i = 0; i < kD; ++i) {
-          const double wi = double(__ldg(a.w_idx + i * kDi + col));
+        for (int q = 0; q < kProjEntries; ++q) acc[q][0] = acc[q][1] = 0.0;
+        // W_idx rows come from L2 one block of kProjRows ahead of their use
+        const float2* wp = reinterpret_cast<const float2*>(a.w_idx + c0);
+        float2 wc[kProjRows], wn[kProjRows];
 #pragma unroll
-          for (int q = 0; q < kCompPerThread; ++q)
-            acc[q] = __fma_rn(cbuf[q * kCompGroups + grp][i], wi, acc[q]);
+        for (int r = 0; r < kProjRows; ++r) wc[r] = __ldg(wp + r * (kDi / 2));
+        for (int i0 = 0; i0 < kD; i0 += kProjRows) {
+          const int nxt = min(i0 + kProjRows, kD - kProjRows);  // the last block reloads itself
+#pragma unroll
+          for (int r = 0; r < kProjRows; ++r) wn[r] = __ldg(wp + (nxt + r) * (kDi / 2));
+#pragma unroll
+          for (int r = 0; r < kProjRows; r += 2) {
+#pragma unroll
+            for (int q = 0; q < kProjEntries; ++q) {
+              const double2 x = *reinterpret_cast<const double2*>(&cbuf[q * kProjGroups + pg][i0 + r]);
+              acc[q][0] = __fma_rn(x.x, double(wc[r].x), acc[q][0]);
+              acc[q][1] = __fma_rn(x.x, double(wc[r].y), acc[q][1]);
+              acc[q][0] = __fma_rn(x.y, double(wc[r + 1].x), acc[q][0]);
+              acc[q][1] = __fma_rn(x.y, double(wc[r + 1].y), acc[q][1]);
+            }
+          }
+#pragma unroll
+          for (int r = 0; r < kProjRows; ++r) wc[r] = wn[r];
         }
 #pragma unroll
-        for (int q = 0; q < kCompPerThread; ++q) rbuf[q * kCompGroups + grp][col] = __double2float_rn(acc[q]);
+        for (int q = 0; q < kProjEntries; ++q) {
+          rbuf[q * kProjGroups + pg][c0] = __double2float_rn(acc[q][0]);
+          rbuf[q * kProjGroups + pg][c0 + 1] = __double2float_rn(acc[q][1]);
+        }
       }
       __syncthreads();
     }
@@ -302,7 +339,7 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
   }
   __syncthreads();
   if (!last_cta) return;
-  const int64_t keep = nstream - nnew * a.ratio;  // 0 or 1 trailing tokens
+  const int64_t keep = nstream - nnew_all * a.ratio;  // 0 or 1 trailing tokens
   const int64_t s_last = nstream - 1;
   if (keep == 1 && s_last >= pn) {  // a raw token of this call becomes the pending one
     const uint32_t* from = reinterpret_cast<const uint32_t*>(src.row(s_last));
@@ -317,7 +354,7 @@ __global__ void __launch_bounds__(kCompWarps * 32) k_compress(CompressArgs a) {
   }
   if (threadIdx.x == 0) {
     a.pend_n[b] = int32_t(keep);
-    if (a.seq_len_out) a.seq_len_out[b] = len_in + int32_t(nnew);
+    if (a.seq_len_out) a.seq_len_out[b] = len_in + int32_t(nnew_all);
     a.arrive[b] = 0u;  // ready for the next call
   }
 }

@@ -75,6 +75,15 @@ def test_other_calls_validation():
     b3 = list(base)
     b3[4] = FAKE
     assert L.csa2_compress_append(*b3, 2, 10, 5, FAKE, 256, None) == -1
+    b4 = list(base)
+    b4[4], b4[5] = FAKE + 4, None                              # W_idx not 8-byte aligned
+    assert L.csa2_compress_append(*b4, 1, 10, 5, FAKE, 256, None) == -1
+    assert b"w_idx" in L.csa2_last_error()
+    ws = L.csa2_compress_append_workspace_bytes(1)
+    b5 = list(base)
+    b5[4], b5[5] = FAKE, None
+    assert L.csa2_compress_append(*b5, 1, 10, 5, FAKE, ws - 1, None) == -3
+    assert L.csa2_compress_append(*b5, 1, 10, 5, FAKE + 64, ws, None) == -1   # workspace alignment
     assert L.csa2_index_prefill(_cache(), FAKE, FAKE, FAKE, FAKE, 4, 0, 100, 2, 64, 512, FAKE, FAKE, FAKE, 1 << 30,
                                 None) == -2                    # pool smaller than k
     assert L.csa2_index_prefill(_cache(rows=64), FAKE, FAKE, FAKE, FAKE, 4, 0, 100, 2, 64, 64, FAKE, FAKE, FAKE,
@@ -114,6 +123,7 @@ def test_compress_stream_validation():
     assert call(w_idx=None, idx_raw=FAKE) == -1             # idx_raw without a pending idx buffer
     assert call(idx_raw=FAKE, pend_idx=FAKE) == -1          # both sources
     assert call(pend_raw=FAKE + 8) == -1                    # misaligned pending row
+    assert call(w_idx=FAKE + 4) == -1                       # W_idx read as float2: 8-byte alignment
     assert call(raw=None) == -1                             # tokens but no raw rows
     assert call(ws_bytes=256) == -3                         # no room for the counters
 

@@ -12,7 +12,7 @@ from tests._gpu import dev, host
 pytestmark = pytest.mark.gpu
 
 
-def _append(raw, logits, tok_off, seq_row_off, seq_len_in, rows, ratio, w_idx=None, idx_raw=None):
+def _append(raw, logits, tok_off, seq_row_off, seq_len_in, rows, ratio, w_idx=None, idx_raw=None, max_new=None):
     B = len(seq_len_in)
     mc = torch.zeros((rows, 256), dtype=torch.uint8, device="cuda")
     ms = torch.zeros((rows, 16), dtype=torch.uint8, device="cuda")
@@ -21,7 +21,8 @@ def _append(raw, logits, tok_off, seq_row_off, seq_len_in, rows, ratio, w_idx=No
     out_len = torch.zeros(B, dtype=torch.int32, device="cuda")
     ws = C.workspace(C.csa2_compress_append_workspace_bytes(B))
     ntok = np.diff(tok_off)
-    max_new = int((ntok // ratio).max()) if B else 0
+    if max_new is None:
+        max_new = int((ntok // ratio).max()) if B else 0
     keep = [dev(raw), dev(logits) if logits is not None else None, dev(tok_off), dev(seq_row_off), dev(seq_len_in),
             dev(w_idx) if w_idx is not None else None, dev(idx_raw) if idx_raw is not None else None]
     C.csa2_compress_append(C.cache(mc, ms), C.cache(ic, isc), keep[0], keep[1], keep[2], keep[3], keep[4], out_len,
@@ -46,6 +47,24 @@ def test_compress_single_sequence_bit_exact(ratio, proj):
     for g, w_ in zip(got[:4], want):
         assert np.array_equal(g[:ne], w_)
     assert not got[0][ne:].any()
+
+
+@pytest.mark.parametrize("max_new", [2, 40])
+def test_compress_beyond_max_new_is_flagged(max_new):
+    """More entries than the host bound: the first max_new are written (bit-exact;
+    at most two per CTA take the one-chain projection, more the shared one), the
+    rest are not, and CSA2_DEV_LENGTH is raised."""
+    n = 100
+    raw = synth.normal_bf16(9, synth.T_RAW, 0, 0, n * 512).reshape(n, 512)
+    w_idx = synth.normal_f32(9, synth.T_WIDX, 0, 0, 512 * 128, log2_div=13).reshape(512, 128)
+    got = _append(raw, None, np.array([0, n]), np.array([0]), np.array([0], np.int32), 104, 1, w_idx,
+                  max_new=max_new)
+    want = oracle.compress(raw, None, 1, w_idx=w_idx)
+    assert got[5] == 8                             # CSA2_DEV_LENGTH
+    assert got[4][0] == n                          # the length the call was asked for
+    for g, w_ in zip(got[:4], want):
+        assert np.array_equal(g[:max_new], w_[:max_new])
+        assert not g[max_new:].any()
 
 
 def test_compress_ragged_batch_appends_at_offsets():

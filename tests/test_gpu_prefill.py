@@ -86,3 +86,30 @@ def test_prefill_full_size_512_queries():
     ro, rl = oracle.attn_prefill(inp["q"], inp["q_pos"], mc, ms, 0, n, 2, top, inp["raw_win"], inp["win_scale"],
                                  1 / math.sqrt(512), q_ids=ids)
     check_attention(g["out"][ids], ro, g["lse"][ids], rl)
+
+
+@pytest.mark.parametrize("distinct", [1, 3])
+def test_prefill_index_heavy_ties(distinct):
+    """Indexer rows drawn from `distinct` different rows, so block keys and
+    candidate keys tie massively (with one row, every present key of a query
+    is the same): the selections' shared-prefix and equal-key rules decide
+    almost everything.  Pools and Top-k bit-exact."""
+    pw = W.prefill_workload()
+    T, n_raw, ratio, P, k = 24, 8192, 2, 64, 64
+    inp = W.prefill_inputs_host(pw, n_raw=n_raw, T=T)
+    n = n_raw // ratio
+    rows = (n + 7) // 8 * 8
+    rng = np.random.default_rng(100 + distinct)
+    pick = rng.integers(0, distinct, rows)
+    ic = rng.integers(0, 256, (distinct, 64), dtype=np.uint8)[pick]
+    isc = rng.integers(124, 129, (distinct, 4)).astype(np.uint8)[pick]
+    pool = torch.full((T, P), -7, dtype=torch.int32, device="cuda")
+    top = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_index_prefill_workspace_bytes(T, n, P, k))
+    C.csa2_index_prefill(C.cache(dev(ic), dev(isc)), dev(inp["q_codes"]), dev(inp["q_scales"]), dev(inp["w"]),
+                         dev(inp["q_pos"]), 0, n, ratio, P, k, pool, top, ws)
+    torch.cuda.synchronize()
+    assert C.device_status(ws) == 0
+    want_pool, want_top = oracle.index_prefill(ic, isc, 0, n, inp["q_codes"], inp["q_scales"], inp["w"],
+                                               inp["q_pos"], ratio, P, k)
+    assert np.array_equal(host(pool), want_pool) and np.array_equal(host(top), want_top)

@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       }
       if (int64_t(tile) * kPT >= gmax) continue;
       const int t = issued, s = t % kSt, round = t / kSt;
-      const bool ok = round == 0 || sm100::mbar_wait(&sm.empty[s], (round - 1) & 1, ctl.wait_ns);
+      const bool ok = round == 0 || sm100::mbar_wait_sleep(&sm.empty[s], (round - 1) & 1, ctl.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) pf_abort(sm, p.status);
         break;
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       for (int s = 0; s < kSt && s < issued; ++s) {
         if (ctl.withhold && s == 0) continue;
         const int last_round = (issued - 1 - s) / kSt;
-        if (!sm100::mbar_wait(&sm.full[s], last_round & 1, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
+        if (!sm100::mbar_wait_sleep(&sm.full[s], last_round & 1, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
       }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -290,11 +290,11 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
         }
         if (int64_t(tile) * kPT >= gmax) continue;
         const int s = t % kSt, a = t % kAc;
-        if (!sm100::mbar_wait(&sm.full[s], (t / kSt) & 1, ctl.wait_ns)) {
+        if (!sm100::mbar_wait_sleep(&sm.full[s], (t / kSt) & 1, ctl.wait_ns)) {
           pf_abort(sm, p.status);
           break;
         }
-        if (t >= kAc && !sm100::mbar_wait(&sm.tempty[a], ((t / kAc) - 1) & 1, ctl.wait_ns)) {
+        if (t >= kAc && !sm100::mbar_wait_sleep(&sm.tempty[a], ((t / kAc) - 1) & 1, ctl.wait_ns)) {
           pf_abort(sm, p.status);
           break;
         }
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
         ++t;
       }
       sm100::mma_commit(&sm.done);  // all MMAs complete before TMEM is released
-      if (!sm100::mbar_wait(&sm.done, 0, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
+      if (!sm100::mbar_wait_sleep(&sm.done, 0, 200000000ull)) set_status(p.status, CSA2_DEV_TIMEOUT);
     }
     __syncwarp();
   } else {
@@ -332,8 +332,8 @@ __global__ void __launch_bounds__(kThr, 1) k_prefill_tc(const __grid_constant__ 
       if (int64_t(tile) * kPT >= gmax) continue;
       ++t;
       const int s = t % kSt, a = t % kAc;
-      const bool ok = sm100::mbar_wait(&sm.full[s], (t / kSt) & 1, ctl.wait_ns) &&
-                      sm100::mbar_wait(&sm.tfull[a], (t / kAc) & 1, ctl.wait_ns);
+      const bool ok = sm100::mbar_wait_sleep(&sm.full[s], (t / kSt) & 1, ctl.wait_ns) &&
+                      sm100::mbar_wait_sleep(&sm.tfull[a], (t / kAc) & 1, ctl.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) pf_abort(sm, p.status);
         break;

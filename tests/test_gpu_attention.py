@@ -58,6 +58,9 @@ def _gpu_decode(d, sm):
     ([5000, 700, 131072], 512, [128, 37, 128], True),
     ([300, 64], 100, [0, 128], False),
     ([2000], 700, [5], False),
+    ([30000, 5000, 2047], 2048, [128, 128, 1], True),   # the largest Top-k the call accepts
+    ([40], 4, [0], False),                               # one to three selected rows, no window
+    ([40], 1, [1], False),                               # a single window row (the one selected is -1)
 ])
 def test_attention_decode_matches_oracle(lengths, k, win_len, lognormal):
     d = _case(len(lengths) * 31 + k, lengths, k, win_len, lognormal)

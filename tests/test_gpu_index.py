@@ -57,6 +57,8 @@ def _run_full(kc, ks, off, lengths, qc, qs, w, P, k, want_scores=False):
     ([100000, 65536], 2048, 512),
     # more than 16384 blocks: the pool is collected by several CTAs per sequence first
     ([300001, 150000, 70, 140000], 2048, 512),
+    ([40000, 20001, 16384], 2048, 2048),    # the largest pool and Top-k the calls accept
+    ([9000, 8, 1], 1, 1),                   # the smallest
 ])
 def test_index_full_matches_oracle(lengths, P, k):
     rng = np.random.default_rng(sum(lengths) + P)
@@ -99,7 +101,8 @@ def test_index_extreme_scales_and_all_ties():
     assert gt[0].tolist() == list(range(64)) and gp[0].tolist() == list(range(16))
 
 
-@pytest.mark.parametrize("lengths,P,k", [([9000, 70000, 5], 2048, 512), ([4096, 333], 64, 100)])
+@pytest.mark.parametrize("lengths,P,k", [([9000, 70000, 5], 2048, 512), ([4096, 333], 64, 100),
+                                         ([70000, 20000], 2048, 2048), ([5000], 1, 1)])
 def test_index_reindex_matches_oracle(lengths, P, k):
     rng = np.random.default_rng(len(lengths) * 7 + k)
     kc, ks, off, _ = _random_cache(rng, lengths)

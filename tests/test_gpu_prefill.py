@@ -43,7 +43,7 @@ def _gpu_prefill(inp, n_raw, T, ratio, P, k, use_proj):
                 lse=host(lse), n_ent=n_ent)
 
 
-@pytest.mark.parametrize("P,k,use_proj,T", [(2048, 512, True, 48), (64, 64, False, 45)])
+@pytest.mark.parametrize("P,k,use_proj,T", [(2048, 512, True, 48), (64, 64, False, 45), (2048, 2048, True, 20)])
 def test_prefill_reduced(P, k, use_proj, T):
     """T = 45 leaves a partial group of queries on the tensor-core scan; the
     first 16 queries see only a few entries each (causal masking)."""

@@ -436,7 +436,7 @@ csa2_status csa2_sparse_attn_prefill(const uint16_t* q, const int32_t* q_pos, in
  * allocations, or a serving loop held to a fixed memory budget).  The pages
  * have no counterpart of this call; it is a deployment convenience.
  * Same arguments, results and accuracy as csa2_sparse_attn_decode, except:
- *   - no workspace: the scratch is a fixed 16,843,264-byte array of device
+ *   - no workspace: the scratch is a fixed 8,421,888-byte array of device
  *     memory inside this library, which every GPU where the library's device
  *     code is loaded keeps until the process exits;
  *   - when that memory is committed: under CUDA's lazy module loading (the

@@ -5,8 +5,9 @@
 //
 // Work split: a segment's keys are chunks (ceil(k/64) chunks of 64 selected
 // rows, and four window chunks of 32 rows), and R CTAs share a segment
-// (R = 2 x SMs / segments, at most 4: two CTAs fit on an SM, and small
-// batches still fill the GPU in one wave).  Each CTA takes an even share of
+// (R <= 4, the one that minimises waves of CTAs, two per SM, times chunks
+// per CTA: 4 at a decode batch of 64, 1 for a prefill chunk of 4096
+// queries).  Each CTA takes an even share of
 // the window chunks and one of the selected chunks, windows first: the window
 // rows are the caller's inputs, so the first of them are staged before the
 // wait on the previous kernel.  While a CTA computes one chunk, cp.async
@@ -29,10 +30,13 @@
 //   O = P V: warp w owns dims 64w .. 64w+63 and reads V (the same rows)
 //       with transposing ldmatrix.
 // The window's fp32 scale multiplies its logits and its output in fp32, never
-// the fp16 values, so a CTA keeps the window chunks in a partial of their
-// own.  Each CTA writes its partials (O, max, sum per head); the last CTA of
-// a segment to finish combines them in a fixed order (deterministic) and
-// resets the segment's arrival counter.
+// the fp16 values: a CTA multiplies its accumulated output by it once, when
+// its window chunks are done and before its selected chunks, so one running
+// softmax state covers all of its chunks.  With R > 1 each CTA writes that
+// part (O, max, sum per head) and the last CTA of a segment to finish
+// combines the R parts in a fixed order (deterministic) and resets the
+// segment's arrival counter; a segment's only CTA (R = 1) divides by the sum
+// in registers and writes the output directly.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -50,7 +54,7 @@ constexpr int kPS = kChunk + 8;                    // smem row stride (halves) o
 constexpr int kWinRows = 32;                       // window rows per chunk (small staging buffer)
 constexpr int kWinChunks = kWin / kWinRows;        // 4
 constexpr int kMaxSplits = 4;                      // CTAs per segment at most
-constexpr int kMaxSlots = 2 * kMaxSplits;          // partials per segment (main + window per CTA)
+constexpr int kMaxSlots = kMaxSplits;              // partials per segment (one per CTA)
 constexpr int kRawMain = kMainCodeBytes + kMainScaleBytes;  // 272: codes then scales (row stride 68
                                                             // words: conflict-free 16-byte reads)
 constexpr int kRawWin = kD + 16;                   // 528: one E4M3 row + pad
@@ -78,8 +82,11 @@ int attn_splits(int S, int k) {
   return best;
 }
 
+// One partial per CTA; a segment's only CTA (R = 1) normalises its output
+// in registers and writes none.
 size_t attn_partial_bytes(int S, int k) {
-  return size_t(S) * 2 * attn_splits(S, k) * kPartFloats * sizeof(float);
+  const int R = attn_splits(S, k);
+  return R == 1 ? 0 : size_t(S) * R * kPartFloats * sizeof(float);
 }
 
 // Staged raw rows of one chunk.  Row strides of 68 and 132 words put the
@@ -503,10 +510,17 @@ __device__ __forceinline__ void softmax_pv(const AttnArgs& a, AttnSmem& sm, int 
   }
 }
 
-// Writes the running part (O x kscale, max, sum) to partial slot `slot` and
-// resets the state.
+// O *= f (the window rows' fp32 scale, applied once to their output).
+__device__ __forceinline__ void scale_acc(float (&oacc)[8][4], float f) {
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) oacc[nt][j] *= f;
+}
+
+// Writes the running part (O, max, sum) to partial slot `slot`.
 __device__ __forceinline__ void flush_part(const AttnArgs& a, AttnSmem& sm, float (&oacc)[8][4], int s, int nslots,
-                                           int slot, float kscale) {
+                                           int slot) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   float* part = a.partial + (int64_t(s) * nslots + slot) * kPartFloats;
@@ -514,17 +528,37 @@ __device__ __forceinline__ void flush_part(const AttnArgs& a, AttnSmem& sm, floa
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) {
     const int d = 64 * warp + 8 * nt + 2 * t;
-    *reinterpret_cast<float2*>(&part[g * kD + d]) = make_float2(oacc[nt][0] * kscale, oacc[nt][1] * kscale);
-    *reinterpret_cast<float2*>(&part[(g + 8) * kD + d]) = make_float2(oacc[nt][2] * kscale, oacc[nt][3] * kscale);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) oacc[nt][j] = 0.0f;
+    *reinterpret_cast<float2*>(&part[g * kD + d]) = make_float2(oacc[nt][0], oacc[nt][1]);
+    *reinterpret_cast<float2*>(&part[(g + 8) * kD + d]) = make_float2(oacc[nt][2], oacc[nt][3]);
   }
-  __syncthreads();
   if (tid < kHq) {
     part[kHq * kD + tid] = sm.m_run[tid];
     part[kHq * kD + kHq + tid] = sm.l_run[tid];
-    sm.m_run[tid] = -INFINITY;
-    sm.l_run[tid] = 0.0f;
+  }
+}
+
+// The only CTA of its segment: out = O / l and lse = max + log l per head,
+// from registers (the same factor 1 / l as a one-slot combine).
+__device__ __forceinline__ void finish_single(const AttnArgs& a, AttnSmem& sm, float (&oacc)[8][4], int s) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  __syncthreads();  // the running max / sum of the last chunk are written
+  float f[2];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const float M = sm.m_run[g + 8 * hh], L = sm.l_run[g + 8 * hh];
+    f[hh] = (M == -INFINITY) ? 0.0f : 1.0f / L;
+  }
+  float* o = a.out + int64_t(s) * kHq * kD;
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) {
+    const int d = 64 * warp + 8 * nt + 2 * t;
+    *reinterpret_cast<float2*>(&o[g * kD + d]) = make_float2(oacc[nt][0] * f[0], oacc[nt][1] * f[0]);
+    *reinterpret_cast<float2*>(&o[(g + 8) * kD + d]) = make_float2(oacc[nt][2] * f[1], oacc[nt][3] * f[1]);
+  }
+  if (a.lse && tid < kHq) {
+    const float M = sm.m_run[tid], L = sm.l_run[tid];
+    a.lse[int64_t(s) * kHq + tid] = (M == -INFINITY) ? -INFINITY : M + logf(L);
   }
 }
 
@@ -622,7 +656,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
   const int m0 = int(int64_t(nmain) * r / R), m1 = int(int64_t(nmain) * (r + 1) / R);
   const int nw = w1 - w0, nc = nw + (m1 - m0);
   auto chunk_at = [&](int i) { return i < nw ? nmain + w0 + i : m0 + (i - nw); };
-  const int nslots = 2 * R;
+  const int nslots = R;  // one part per CTA: its window rows' output is scaled into the running state
   launch_dependents();
   float oacc[8][4];
 #pragma unroll
@@ -658,8 +692,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
     const ChunkSrc src = chunk_src(a, s, c);
     if (src.is_win) {
       win_scale = src.kscale;
-    } else if (in_win) {  // this CTA's window rows are done: their partial
-      flush_part(a, sm, oacc, s, nslots, 2 * r + 1, win_scale);
+    } else if (in_win) {  // this CTA's window rows are done: their output takes the window's scale
+      scale_acc(oacc, win_scale);
       in_win = false;
     }
     sm100::cp_async_wait<0>();
@@ -673,13 +707,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_attn(AttnArgs a, int R) {
     }
     softmax_pv(a, sm, vb, oacc, src.nkeys, src.kscale);
   }
-  if (nc > 0) {  // the part in progress
-    if (in_win) flush_part(a, sm, oacc, s, nslots, 2 * r + 1, win_scale);
-    else flush_part(a, sm, oacc, s, nslots, 2 * r, 1.0f);
-  }
-  if (m1 == m0) empty_part(a, s, nslots, 2 * r);
-  if (nw == 0) empty_part(a, s, nslots, 2 * r + 1);
+  if (in_win) scale_acc(oacc, win_scale);  // (a CTA of window rows only)
   sm100::cp_async_wait<0>();
+  if (R == 1) {  // the segment's only CTA: no partial, no combine
+    finish_single(a, sm, oacc, s);
+    return;
+  }
+  if (nc > 0) flush_part(a, sm, oacc, s, nslots, r);
+  else empty_part(a, s, nslots, r);
   combine_if_last(a, sm, s, R, nslots);
 }
 

@@ -31,15 +31,15 @@ constexpr int kNoAllocMaxSeqs = 64;
 constexpr int kNoAllocMaxTopk = 512;
 constexpr size_t kNoAllocStatusBytes = 256;                       // device status word
 constexpr size_t kNoAllocCounterBytes = 256;                      // 64 arrival counters (self-resetting)
-constexpr size_t kNoAllocSlots = 8;                               // partials per sequence: up to 4 CTAs x
-                                                                  // (selected rows, window)
+constexpr size_t kNoAllocSlots = 4;                               // partials per sequence: one per CTA,
+                                                                  // up to 4 CTAs
 constexpr size_t kNoAllocPartialBytes =                           // split-KV partials
     size_t(kNoAllocMaxSeqs) * kNoAllocSlots * (kHq * kD + 2 * kHq) * sizeof(float);
 constexpr size_t kNoAllocScratchBytes =
     kNoAllocStatusBytes + kNoAllocCounterBytes + kNoAllocPartialBytes;
-static_assert(kNoAllocScratchBytes == 16843264, "the documented scratch size");
+static_assert(kNoAllocScratchBytes == 8421888, "the documented scratch size");
 
-// The scratch: 16,843,264 bytes of device memory that every GPU on which this
+// The scratch: 8,421,888 bytes of device memory that every GPU on which this
 // library's device code is loaded keeps until the process exits.  All calls
 // on a device share it and it keeps whatever the last call left in it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];

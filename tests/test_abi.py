@@ -98,9 +98,10 @@ def test_workspace_sizes_grow_with_the_problem():
     b = L.csa2_index_full_workspace_bytes(8, 1 << 16, 2048, 512)
     assert 256 < a < b and a % 256 == 0
     assert L.csa2_index_full_workspace_bytes(1, 8192, 256, 512) > L.csa2_index_full_workspace_bytes(1, 8192, 512, 512)
-    # attention: at least one CTA per sequence, each with a selected-rows and a window partial
-    # (O [16 x 512] + max + sum per head, fp32)
-    assert L.csa2_sparse_attn_decode_workspace_bytes(64, 512) >= 64 * 2 * (16 * 512 + 32) * 4
+    # attention at B = 64: four CTAs per sequence, one partial each (O [16 x 512] + max + sum per
+    # head, fp32); a segment's only CTA (many segments) writes no partial
+    assert L.csa2_sparse_attn_decode_workspace_bytes(64, 512) >= 64 * 4 * (16 * 512 + 32) * 4
+    assert L.csa2_sparse_attn_decode_workspace_bytes(4096, 512) < 4096 * (16 * 512 + 32) * 4
     assert L.csa2_sparse_attn_decode_workspace_bytes(128, 512) > L.csa2_sparse_attn_decode_workspace_bytes(16, 512)
 
 

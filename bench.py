@@ -745,19 +745,26 @@ def run_prefill(args):
     names = ("csa2_compress_append", "csa2_index_prefill", "csa2_sparse_attn_prefill")
     times = {n: [] for n in names}
 
-    def step(record):
+    dev_in = {"raw": raw, "logits": logits, "q": q, "q_codes": q_codes, "q_scales": q_scales, "w": w,
+              "raw_win": raw_win}
+    dev_out = {"top": top, "out": out}
+
+    def step(record, x=None, y=None):
+        x = x or dev_in
+        y = y or dev_out
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
         if record:
             ev[0].record(stream)
-        C.csa2_compress_append(main, idx, raw, logits, tok_off, row_off, len_in, len_out, ratio, n_ent, ws1,
+        C.csa2_compress_append(main, idx, x["raw"], x["logits"], tok_off, row_off, len_in, len_out, ratio, n_ent, ws1,
                                w_idx=w_idx)
         if record:
             ev[1].record(stream)
-        C.csa2_index_prefill(idx, q_codes, q_scales, w, q_pos, 0, n_ent, ratio, P, k, pool, top, ws2)
+        C.csa2_index_prefill(idx, x["q_codes"], x["q_scales"], x["w"], q_pos, 0, n_ent, ratio, P, k, pool, y["top"],
+                             ws2)
         if record:
             ev[2].record(stream)
-        C.csa2_sparse_attn_prefill(q, q_pos, main, 0, n_ent, ratio, top, raw_win, win_scale, 1 / math.sqrt(512), out,
-                                   ws3, lse=lse)
+        C.csa2_sparse_attn_prefill(x["q"], q_pos, main, 0, n_ent, ratio, y["top"], x["raw_win"], win_scale,
+                                   1 / math.sqrt(512), y["out"], ws3, lse=lse)
         if record:
             ev[3].record(stream)
             for i, n in enumerate(names):
@@ -785,26 +792,48 @@ def run_prefill(args):
 
     # end to end: every input of the step from pinned host memory (raw tokens,
     # logits, queries and their indexer inputs, the raw FP8 window rows), the
-    # outputs (attention output, Top-k) back to the host
-    host_in = {name: t.cpu().pin_memory() for name, t in (("raw", raw), ("logits", logits), ("q", q),
-                                                          ("q_codes", q_codes), ("q_scales", q_scales), ("w", w),
-                                                          ("raw_win", raw_win))}
-    dev_in = {"raw": raw, "logits": logits, "q": q, "q_codes": q_codes, "q_scales": q_scales, "w": w,
-              "raw_win": raw_win}
+    # outputs (attention output, Top-k) back to the host.  Prefill chunks are
+    # independent requests, so, as a serving loop would, each step's inputs
+    # are copied in on one copy stream while the previous step computes
+    # (double-buffered), and each step's results leave on another while the
+    # next one computes; the timed region ends when the last results are on
+    # the host.
+    host_in = {name: t.cpu().pin_memory() for name, t in dev_in.items()}
+    ins = [dev_in, {name: t.clone() for name, t in dev_in.items()}]
+    outs = [dev_out, {name: t.clone() for name, t in dev_out.items()}]
     out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
     top_h = torch.empty(top.shape, dtype=torch.int32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = out_h.numel() * 4 + top_h.numel() * 4
     e_steps = max(1, min(args.e2e_steps, 10))
+    h2d_stream, d2h_stream = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
+
+    def copy_in(x):
+        with torch.cuda.stream(h2d_stream):
+            for name, src in host_in.items():
+                x[name].copy_(src, non_blocking=True)
+
+    out_done = [None, None]  # per output set: its last results are on the host
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e_steps):
-        for name, src in host_in.items():
-            dev_in[name].copy_(src, non_blocking=True)
-        step(False)
-        out_h.copy_(out, non_blocking=True)
-        top_h.copy_(top, non_blocking=True)
+    copy_in(ins[0])  # the first step's inputs (each step copies the next step's)
+    for i in range(e_steps):
+        p = i % 2
+        stream.wait_stream(h2d_stream)  # this step's inputs are on the device
+        if i + 1 < e_steps:
+            h2d_stream.wait_stream(stream)  # the step that last read the other input set has finished
+            copy_in(ins[1 - p])
+        if out_done[p] is not None:
+            stream.wait_event(out_done[p])  # the results last written to this output set have left
+        step(False, ins[p], outs[p])
+        d2h_stream.wait_stream(stream)
+        with torch.cuda.stream(d2h_stream):
+            out_h.copy_(outs[p]["out"], non_blocking=True)
+            top_h.copy_(outs[p]["top"], non_blocking=True)
+            out_done[p] = torch.cuda.Event()
+            out_done[p].record(d2h_stream)
+    stream.wait_stream(d2h_stream)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, device, world)

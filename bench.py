@@ -511,11 +511,30 @@ def run_ours(args):
     # inputs go in on one copy stream, results come out on another
     h2d_stream, d2h_stream = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
 
-    def copy_out(layer, ev):
-        d2h_stream.wait_event(ev)
+    def copy_now(layer):
         with torch.cuda.stream(d2h_stream):
             out_host[layer].copy_(step.out[layer], non_blocking=True)
             top_host[layer].copy_(step.topk[layer], non_blocking=True)
+
+    last_layer = n_layers - 1
+
+    def copy_out(layer, ev):
+        if layer == last_layer:  # leaves while the next step starts (see e2e_step)
+            return
+        d2h_stream.wait_event(ev)
+        copy_now(layer)
+
+    # The last layer's results are copied out at the start of the next step,
+    # beside its scan; of that step only the layers that overwrite those
+    # tensors wait for the copy: the last layer (its output) and, when the
+    # last layer reuses a Top-k, the layer that writes that Top-k.
+    topk_writer = last_layer
+    for layer, mode, f, act in step.plan:
+        if act != "reuse" and layer < last_layer:
+            topk_writer = layer
+    if step.plan[-1][3] != "reuse":
+        topk_writer = last_layer
+    gated = {last_layer, topk_writer}
 
     # Inputs are double-buffered: every step copies the NEXT step's inputs
     # from pinned host memory into the other buffer set while it computes, so
@@ -536,11 +555,19 @@ def run_ours(args):
 
     def e2e_step(p):
         cur = torch.cuda.current_stream()
+        start = torch.cuda.Event()
+        start.record(cur)
         h2d_stream.wait_stream(cur)  # the step that last read buffer 1 - p has finished
         with torch.cuda.stream(h2d_stream):
             copy_in(1 - p)
-        step.run(caches, off_d, len_d, bufs[p], on_layer_done=copy_out, new_tokens=tbufs[p], **vq)
-        cur.wait_stream(d2h_stream)  # the step ends when its results are on the host
+        # the previous step's last layer results (that step has completed)
+        d2h_stream.wait_stream(cur)
+        copy_now(last_layer)
+        out_gone = torch.cuda.Event()
+        out_gone.record(d2h_stream)
+        ready = [out_gone if layer in gated else start for layer in range(n_layers)]
+        step.run(caches, off_d, len_d, bufs[p], ready=ready, on_layer_done=copy_out, new_tokens=tbufs[p], **vq)
+        cur.wait_stream(d2h_stream)  # this step's copies of its other layers are on the host
         cur.wait_stream(h2d_stream)
 
     e2e_graphs = None
@@ -568,6 +595,9 @@ def run_ours(args):
             e2e_graphs[i % 2].replay()
         else:
             e2e_step(i % 2)
+    d2h_stream.wait_stream(stream)  # the last step's last layer
+    copy_now(last_layer)
+    stream.wait_stream(d2h_stream)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps

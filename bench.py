@@ -73,6 +73,19 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def deferred_copy_gates(plan) -> set:
+    """Layers of a decode step that overwrite what the previous step's last
+    layer copies out (its attention output and Top-k): the last layer itself
+    and, when it reuses a Top-k, the latest earlier layer that selected one
+    (a Reuse layer's Top-k is that layer's tensor).  plan: [(layer, mode,
+    full_index, action)] as decode.layer_plan returns."""
+    last = plan[-1][0]
+    writer = last
+    if plan[-1][3] == "reuse":
+        writer = max(layer for layer, _, _, act in plan if act != "reuse" and layer < last)
+    return {last, writer}
+
+
 def algorithmic_bytes(wl, full_rescan=False):
     """Per step, from the method's own reads (no scratch traffic): each
     scanning Full layer L*68 B; each layer that selects inside the pool (a
@@ -526,15 +539,8 @@ def run_ours(args):
 
     # The last layer's results are copied out at the start of the next step,
     # beside its scan; of that step only the layers that overwrite those
-    # tensors wait for the copy: the last layer (its output) and, when the
-    # last layer reuses a Top-k, the layer that writes that Top-k.
-    topk_writer = last_layer
-    for layer, mode, f, act in step.plan:
-        if act != "reuse" and layer < last_layer:
-            topk_writer = layer
-    if step.plan[-1][3] != "reuse":
-        topk_writer = last_layer
-    gated = {last_layer, topk_writer}
+    # tensors wait for the copy.
+    gated = deferred_copy_gates(step.plan)
 
     # Inputs are double-buffered: every step copies the NEXT step's inputs
     # from pinned host memory into the other buffer set while it computes, so

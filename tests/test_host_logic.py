@@ -90,3 +90,17 @@ def test_decode_grouped_rejects_other_schedules():
         DecodeStep("FR", 4, 8192, concurrent=False, groups=5)    # more groups than sequences
     with pytest.raises(ValueError):
         DecodeStep("FR", 4, 8192, concurrent=False, groups=2, queries=8)
+
+
+def test_deferred_copy_gates():
+    """The layers that must wait for the previous step's last-layer copy: the
+    last layer, and the layer whose Top-k tensor a final Reuse layer shares."""
+    from long_context_decode_csa2_b200.decode import layer_plan
+
+    assert bench.deferred_copy_gates(layer_plan("FRRU")) == {3, 2}
+    assert bench.deferred_copy_gates(layer_plan("FRUU")) == {3, 1}
+    assert bench.deferred_copy_gates(layer_plan("FRURU" * 4)) == {19, 18}
+    assert bench.deferred_copy_gates(layer_plan("FRRR")) == {3}
+    assert bench.deferred_copy_gates(layer_plan("F")) == {0}
+    assert bench.deferred_copy_gates(layer_plan("FU")) == {1, 0}
+    assert bench.deferred_copy_gates(layer_plan("FRFU", full_rescan=True)) == {3, 2}
